@@ -1,0 +1,227 @@
+"""fp64 CPU oracle for the chunked fast-weight update-and-read. TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this module. The CUDA library never calls it, and nothing here calls the CUDA library: the two
+share no code. Inputs are the exact values the GPU receives (bf16 tensors widened to float64,
+the same fp32 learning rates); every result is float64.
+
+Sources, cited by page title and the passage on it:
+
+  [TTT-read]  "RNN의 기억을 작은 모델로 바꾼다면: Test-Time Training 읽기" (ariser.io), a reading
+              of "Learning to (Learn at Test Time)". Section "읽는 동안 문제를 하나 더 푼다":
+              the per-token rule W_t = W_(t-1) - eta * grad l(W_(t-1); x_t), output read from the
+              *updated* model. Section "gradient를 효율적인 layer로 만드는 작업": mini-batch TTT and
+              its dual form, which equals the mini-batch update (not per-token SGD).
+              Section "원문의 긴 문맥 결과를 읽는 범위": state reset per sequence, batch items kept
+              apart.
+  [KVB]       "KV 바인딩 기반 테스트 시간 학습은 사실상 선형 어텐션이다" (aitrends.kr): one inner
+              step with a linear bias-free last layer gives o = q(S0 + k^T v); without weight
+              normalisation the state update is associative (parallel prefix scan); per-token
+              learning rates fold into the values; gradient ascent in the inner loop.
+  [IPT]       "In-Place 테스트 시점 학습: LLM을 위한 원활한 동적 적응 프레임워크" (aitrends.kr):
+              W_down of the gated MLP is the fast weight, refreshed once per chunk (C = 512..1024)
+              with one gradient step; the updated weight serves the *next* chunk; per-chunk deltas
+              combine by a prefix sum (associative scan), equal to the sequential update.
+
+Readings where the pages leave a step open (each also listed in the design notes):
+  * inner loss 1/2 ||k W - v||^2 with row vectors and W laid out [d_in][d_out], so the gradient
+    of token s at W is k_s^T (k_s W - v_s);
+  * the intra-chunk causal mask includes the diagonal (token t sees its own gradient, as the
+    per-token rule reads the updated model);
+  * a per-token learning rate scales the *source* token's gradient (or value);
+  * the associative mode adds eta_t k_t^T v_t (ascent on <k S, v>) and reads o_t = q_t S_t after
+    the update of token t;
+  * the In-Place chunk i reads W0 plus the deltas of chunks strictly before it, and the delta is
+    +eta Z_i^T Vhat_i.
+
+Pins (tests/test_oracle_pins.py): per-token SGD from autograd gradients at C=1; mini-batch
+gradient descent from autograd gradients at any C; the causal-linear-attention closed form at
+W0 = 0; o = q(S0 + k^T v) for one token; the sequential recurrence vs. the chunked and two-pass
+forms; eta folded into V; the In-Place block-causal linear-attention form and its one-chunk closed
+form; autograd ascent steps for the associative and In-Place deltas; hand-worked golden examples.
+Every function below has at least one pin.
+"""
+from __future__ import annotations
+
+from concurrent.futures import ThreadPoolExecutor
+from typing import Optional, Sequence
+
+import numpy as np
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def _eta_stream(eta, T: int) -> np.ndarray:
+    if np.ndim(eta) == 0:
+        return np.full(T, float(eta))
+    e = _f64(eta)
+    assert e.shape == (T,)
+    return e
+
+
+# --------------------------------------------------------------------------------------------
+# TTT-Linear, mini-batch dual form  [TTT-read, "gradient를 효율적인 layer로 만드는 작업"]
+# --------------------------------------------------------------------------------------------
+def dual_form_stream(Q, K, V, eta, W0, C: int):
+    """One (batch, head) stream. Q, K, V: [T, d]; eta: [T] or scalar; W0: [d, d] or None (zeros).
+
+    For each chunk of C tokens, with W the state at the chunk's start:
+        G   = K_c W - V_c                      (residuals; token s's gradient is k_s^T g_s)
+        O_c = Q_c W - (tril(Q_c K_c^T) * eta_s) G
+              i.e. token t reads W minus the eta-weighted gradients of tokens s <= t of its chunk
+        W   = W - K_c^T diag(eta_c) G          (one mini-batch step at the chunk-start W)
+    Returns (O [T, d], W_final [d, d]).
+    """
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    T, d = Q.shape
+    if C <= 0 or T % C:
+        raise ValueError("T must be a positive multiple of C")
+    e_all = _eta_stream(eta, T)
+    W = np.zeros((d, d)) if W0 is None else _f64(W0).copy()
+    O = np.empty((T, d))
+    for c0 in range(0, T, C):
+        q, k, v, e = Q[c0:c0 + C], K[c0:c0 + C], V[c0:c0 + C], e_all[c0:c0 + C]
+        G = k @ W - v
+        A = np.tril(q @ k.T) * e[None, :]
+        O[c0:c0 + C] = q @ W - A @ G
+        W = W - k.T @ (e[:, None] * G)
+    return O, W
+
+
+def _streams(fn, arrays, B: int, H: int, threads: int, streams: Optional[Sequence] = None):
+    idx = list(streams) if streams is not None else [(b, h) for b in range(B) for h in range(H)]
+    if threads <= 1:
+        return idx, [fn(b, h) for (b, h) in idx]
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        return idx, list(ex.map(lambda bh: fn(*bh), idx))
+
+
+def dual_form(Q, K, V, eta, W0, C: int, *, threads: int = 1, streams=None):
+    """All (b, h) streams of [B, H, T, d] inputs; eta [B, H, T] or scalar; W0 [B, H, d, d] or
+    None. Streams are independent [TTT-read, "원문의 긴 문맥 결과를 읽는 범위"].
+    ``streams`` selects a subset of (b, h) pairs; the result then holds only those, in order:
+    (O [n, T, d], W [n, d, d]). Without it the result is (O [B,H,T,d], W [B,H,d,d])."""
+    B, H, T, d = np.shape(Q)
+
+    def one(b, h):
+        e = eta if np.ndim(eta) == 0 else np.asarray(eta)[b, h]
+        w0 = None if W0 is None else np.asarray(W0)[b, h]
+        return dual_form_stream(np.asarray(Q)[b, h], np.asarray(K)[b, h], np.asarray(V)[b, h],
+                                e, w0, C)
+
+    idx, res = _streams(one, None, B, H, threads, streams)
+    O = np.stack([r[0] for r in res])
+    W = np.stack([r[1] for r in res])
+    if streams is None:
+        O = O.reshape(B, H, T, d)
+        W = W.reshape(B, H, d, d)
+    return O, W
+
+
+# --------------------------------------------------------------------------------------------
+# Associative (weight-norm-free, gradient-ascent) linear-attention mode  [KVB]
+# --------------------------------------------------------------------------------------------
+def assoc_recurrence_stream(Q, K, V, eta, S0):
+    """Sequential definition, one token at a time: S_t = S_(t-1) + eta_t k_t^T v_t, o_t = q_t S_t.
+    The chunk size does not enter. Returns (O [T, d], S_final [d, d])."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    T, d = Q.shape
+    e = _eta_stream(eta, T)
+    S = np.zeros((d, d)) if S0 is None else _f64(S0).copy()
+    O = np.empty((T, d))
+    for t in range(T):
+        S += e[t] * np.outer(K[t], V[t])
+        O[t] = Q[t] @ S
+    return O, S
+
+
+def assoc_chunked_stream(Q, K, V, eta, S0, C: int):
+    """Chunk form of the same recurrence: per chunk, O_c = Q_c S + (tril(Q_c K_c^T) * eta_s) V_c,
+    then S += K_c^T diag(eta_c) V_c. Equal to the sequential form by associativity [KVB]."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    T, d = Q.shape
+    if C <= 0 or T % C:
+        raise ValueError("T must be a positive multiple of C")
+    e_all = _eta_stream(eta, T)
+    S = np.zeros((d, d)) if S0 is None else _f64(S0).copy()
+    O = np.empty((T, d))
+    for c0 in range(0, T, C):
+        q, k, v, e = Q[c0:c0 + C], K[c0:c0 + C], V[c0:c0 + C], e_all[c0:c0 + C]
+        O[c0:c0 + C] = q @ S + (np.tril(q @ k.T) * e[None, :]) @ v
+        S = S + k.T @ (e[:, None] * v)
+    return O, S
+
+
+def assoc_two_pass_stream(Q, K, V, eta, S0, C: int, L: int):
+    """Two-pass prefix-scan form over superchunks of L tokens (L a multiple of C):
+    pass 1 sums each superchunk's state increment; an exclusive prefix sum (plus S0) gives each
+    superchunk's starting state; pass 2 runs the chunk form inside each superchunk from it
+    [KVB, associativity paragraph; IPT, associative-scan paragraph]."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    T, d = Q.shape
+    if L <= 0 or L % C or T % L:
+        raise ValueError("T must be a multiple of L, and L a multiple of C")
+    e_all = _eta_stream(eta, T)
+    starts = list(range(0, T, L))
+    deltas = [K[s:s + L].T @ (e_all[s:s + L, None] * V[s:s + L]) for s in starts]      # pass 1
+    S = np.zeros((d, d)) if S0 is None else _f64(S0).copy()
+    S_start = []
+    for dS in deltas:                                                                  # scan
+        S_start.append(S.copy())
+        S = S + dS
+    O = np.empty((T, d))
+    for s, Ss in zip(starts, S_start):                                                 # pass 2
+        O[s:s + L], _ = assoc_chunked_stream(Q[s:s + L], K[s:s + L], V[s:s + L],
+                                             e_all[s:s + L], Ss, C)
+    return O, S
+
+
+def assoc_scan(Q, K, V, eta, S0, *, threads: int = 1, streams=None, form: str = "sequential",
+               C: int = 64):
+    """All streams; ``form`` picks 'sequential' (the definition) or 'chunked' (pinned equal)."""
+    B, H, T, d = np.shape(Q)
+
+    def one(b, h):
+        e = eta if np.ndim(eta) == 0 else np.asarray(eta)[b, h]
+        s0 = None if S0 is None else np.asarray(S0)[b, h]
+        q, k, v = np.asarray(Q)[b, h], np.asarray(K)[b, h], np.asarray(V)[b, h]
+        if form == "sequential":
+            return assoc_recurrence_stream(q, k, v, e, s0)
+        return assoc_chunked_stream(q, k, v, e, s0, C)
+
+    idx, res = _streams(one, None, B, H, threads, streams)
+    O = np.stack([r[0] for r in res])
+    S = np.stack([r[1] for r in res])
+    if streams is None:
+        O = O.reshape(B, H, T, d)
+        S = S.reshape(B, H, d, d)
+    return O, S
+
+
+# --------------------------------------------------------------------------------------------
+# In-Place TTT W_down chunk update  [IPT]
+# --------------------------------------------------------------------------------------------
+def inplace_chunks(Z, Vhat, W0, eta: float, C: int, cols=None):
+    """Z [T, Dff]; Vhat [T, D]; W0 [Dff, D]. Sequentially over chunks i of C tokens:
+        O_i = Z_i W          (W = W0 plus the deltas of the chunks before i)
+        W   = W + eta Z_i^T Vhat_i
+    Returns (O [T, D'], W_final [Dff, D']) where D' = len(cols) when ``cols`` selects output
+    columns (each column of O and W depends only on the same column of Vhat and W0, so a column
+    subset is exact, not an approximation)."""
+    T, Dff = np.shape(Z)
+    if C <= 0 or T % C:
+        raise ValueError("T must be a positive multiple of C")
+    Vh = np.asarray(Vhat)
+    W = np.asarray(W0)
+    if cols is not None:
+        Vh = Vh[:, cols]
+        W = W[:, cols]
+    W = _f64(W).copy()
+    O = np.empty((T, W.shape[1]))
+    for c0 in range(0, T, C):
+        z = _f64(np.asarray(Z)[c0:c0 + C])
+        O[c0:c0 + C] = z @ W
+        W = W + eta * (z.T @ _f64(Vh[c0:c0 + C]))
+    return O, W

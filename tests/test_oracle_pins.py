@@ -1,0 +1,326 @@
+"""Pins of the fp64 oracle to facts fixed by the pages and by the mathematics (CPU only).
+
+Each test compares the oracle with something other than itself: gradients taken by autograd on
+the inner loss (not the hand-derived gradient the oracle uses), closed forms, hand-worked
+examples, or algebraically different forms of the same quantity. Sizes are tiny; fp64.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import ttt_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked.json")
+rng = np.random.default_rng(7)
+
+
+def _rand(*shape, scale=1.0):
+    return rng.standard_normal(shape) * scale
+
+
+# ----------------------------------------------------------------------------- autograd helpers
+def _grad_inner_loss(W: torch.Tensor, k: torch.Tensor, v: torch.Tensor) -> torch.Tensor:
+    """Gradient of the inner loss 1/2 ||k W - v||^2 at W, by autograd."""
+    Wr = W.detach().clone().requires_grad_(True)
+    loss = 0.5 * ((k @ Wr - v) ** 2).sum()
+    (g,) = torch.autograd.grad(loss, Wr)
+    return g
+
+
+def _per_token_sgd(Q, K, V, eta, W0):
+    """W_t = W_(t-1) - eta_t grad l(W_(t-1); x_t); o_t = q_t W_t (output from the updated model)."""
+    Q, K, V, eta = (torch.as_tensor(x, dtype=torch.float64) for x in (Q, K, V, eta))
+    W = torch.as_tensor(W0, dtype=torch.float64).clone()
+    O = torch.empty_like(Q)
+    for t in range(Q.shape[0]):
+        W = W - eta[t] * _grad_inner_loss(W, K[t], V[t])
+        O[t] = Q[t] @ W
+    return O.numpy(), W.numpy()
+
+
+def _minibatch_gd_by_definition(Q, K, V, eta, W0, C):
+    """Mini-batch TTT: all gradients of a chunk are taken at the chunk-start weight W_b; token t
+    reads W_b minus the eta-weighted gradients of tokens s <= t; the next chunk starts from W_b
+    minus all of the chunk's weighted gradients. Every W_t is formed explicitly."""
+    Q, K, V, eta = (torch.as_tensor(x, dtype=torch.float64) for x in (Q, K, V, eta))
+    W = torch.as_tensor(W0, dtype=torch.float64).clone()
+    O = torch.empty_like(Q)
+    for c0 in range(0, Q.shape[0], C):
+        grads = [eta[s] * _grad_inner_loss(W, K[s], V[s]) for s in range(c0, c0 + C)]
+        for t in range(c0, c0 + C):
+            Wt = W - sum(grads[: t - c0 + 1])
+            O[t] = Q[t] @ Wt
+        W = W - sum(grads)
+    return O.numpy(), W.numpy()
+
+
+# ----------------------------------------------------------------------------- dual form
+@pytest.mark.parametrize("d,T", [(1, 5), (3, 7), (8, 16)])
+def test_dual_C1_equals_per_token_sgd_autograd(d, T):
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.05, 0.4, T)
+    W0 = _rand(d, d, scale=0.3)
+    O, W = orc.dual_form_stream(Q, K, V, eta, W0, 1)
+    O_ref, W_ref = _per_token_sgd(Q, K, V, eta, W0)
+    np.testing.assert_allclose(O, O_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(W, W_ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("d,T,C", [(2, 8, 2), (4, 12, 4), (8, 32, 8), (8, 32, 32), (5, 18, 3)])
+def test_dual_equals_minibatch_gd_autograd(d, T, C):
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.05, 0.4, T)
+    W0 = _rand(d, d, scale=0.3)
+    O, W = orc.dual_form_stream(Q, K, V, eta, W0, C)
+    O_ref, W_ref = _minibatch_gd_by_definition(Q, K, V, eta, W0, C)
+    np.testing.assert_allclose(O, O_ref, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(W, W_ref, rtol=1e-11, atol=1e-12)
+
+
+def test_dual_scalar_eta_equals_constant_array():
+    d, T, C = 4, 16, 4
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    W0 = _rand(d, d)
+    a = orc.dual_form_stream(Q, K, V, 0.1, W0, C)
+    b = orc.dual_form_stream(Q, K, V, np.full(T, 0.1), W0, C)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_dual_W0_zero_first_chunk_is_causal_linear_attention():
+    """With W0 = 0 the first chunk's residuals are -V, so O = tril(Q K^T) diag(eta) V and
+    W = K^T diag(eta) V: causal linear attention ("TTT with KV binding is in fact linear
+    attention")."""
+    d, C = 6, 8
+    Q, K, V = _rand(C, d), _rand(C, d), _rand(C, d)
+    eta = rng.uniform(0.1, 0.5, C)
+    O, W = orc.dual_form_stream(Q, K, V, eta, None, C)
+    O_la = np.array([sum(eta[s] * (Q[t] @ K[s]) * V[s] for s in range(t + 1)) for t in range(C)])
+    W_la = sum(eta[s] * np.outer(K[s], V[s]) for s in range(C))
+    np.testing.assert_allclose(O, O_la, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(W, W_la, rtol=1e-12, atol=1e-13)
+
+
+def test_dual_chunked_differs_from_per_token():
+    """The dual form equals the mini-batch update, not per-token SGD."""
+    d, T = 4, 16
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    O1, W1 = orc.dual_form_stream(Q, K, V, 0.3, None, 1)
+    O4, W4 = orc.dual_form_stream(Q, K, V, 0.3, None, 4)
+    assert np.abs(O1 - O4).max() > 1e-3
+    assert np.abs(W1 - W4).max() > 1e-3
+
+
+def test_dual_state_carry_split_at_chunk_boundary():
+    """Running T tokens equals running the first half, then the second from its final W."""
+    d, T, C = 5, 24, 4
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.05, 0.3, T)
+    W0 = _rand(d, d)
+    O, W = orc.dual_form_stream(Q, K, V, eta, W0, C)
+    h = 12
+    Oa, Wa = orc.dual_form_stream(Q[:h], K[:h], V[:h], eta[:h], W0, C)
+    Ob, Wb = orc.dual_form_stream(Q[h:], K[h:], V[h:], eta[h:], Wa, C)
+    np.testing.assert_allclose(np.concatenate([Oa, Ob]), O, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(Wb, W, rtol=1e-13, atol=1e-14)
+
+
+def test_dual_batch_streams_independent_and_permutable():
+    B, H, T, d, C = 2, 3, 8, 3, 4
+    Q, K, V = _rand(B, H, T, d), _rand(B, H, T, d), _rand(B, H, T, d)
+    eta = rng.uniform(0.05, 0.3, (B, H, T))
+    W0 = _rand(B, H, d, d)
+    O, W = orc.dual_form(Q, K, V, eta, W0, C)
+    for b in range(B):
+        for h in range(H):
+            o, w = orc.dual_form_stream(Q[b, h], K[b, h], V[b, h], eta[b, h], W0[b, h], C)
+            np.testing.assert_array_equal(O[b, h], o)
+            np.testing.assert_array_equal(W[b, h], w)
+    # subset selection returns exactly those streams, and threads do not change results
+    Os, Ws = orc.dual_form(Q, K, V, eta, W0, C, streams=[(1, 2), (0, 1)], threads=2)
+    np.testing.assert_array_equal(Os[0], O[1, 2])
+    np.testing.assert_array_equal(Ws[1], W[0, 1])
+
+
+def test_dual_rejects_ragged_T():
+    with pytest.raises(ValueError):
+        orc.dual_form_stream(_rand(10, 2), _rand(10, 2), _rand(10, 2), 0.1, None, 4)
+
+
+# ----------------------------------------------------------------------------- associative mode
+def test_assoc_one_token_closed_form_and_autograd_ascent():
+    """o = q (S0 + k^T v) after one inner step ("TTT with KV binding is in fact linear
+    attention"); the step is gradient ascent on <k S, v> with learning rate 1 (autograd)."""
+    d = 5
+    q, k, v = _rand(d), _rand(d), _rand(d)
+    S0 = _rand(d, d)
+    O, S = orc.assoc_recurrence_stream(q[None], k[None], v[None], 1.0, S0)
+    np.testing.assert_allclose(O[0], q @ (S0 + np.outer(k, v)), rtol=1e-13)
+    St = torch.tensor(S0, requires_grad=True)
+    obj = (torch.tensor(k) @ St) @ torch.tensor(v)
+    (g,) = torch.autograd.grad(obj, St)
+    S1 = (St + 1.0 * g).detach().numpy()
+    np.testing.assert_allclose(S, S1, rtol=1e-13)
+    np.testing.assert_allclose(O[0], q @ S1, rtol=1e-13)
+
+
+def test_assoc_each_step_is_ascent_with_token_eta():
+    d, T = 3, 6
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.2, 1.0, T)
+    S_prev = _rand(d, d)
+    O, _ = orc.assoc_recurrence_stream(Q, K, V, eta, S_prev)
+    for t in range(T):
+        St = torch.tensor(S_prev, requires_grad=True)
+        (g,) = torch.autograd.grad((torch.tensor(K[t]) @ St) @ torch.tensor(V[t]), St)
+        S_prev = (St + eta[t] * g).detach().numpy()
+        np.testing.assert_allclose(O[t], Q[t] @ S_prev, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("T,C,L", [(24, 1, 24), (24, 4, 8), (24, 8, 24), (32, 8, 16), (30, 5, 10)])
+def test_assoc_chunked_and_two_pass_equal_sequential(T, C, L):
+    d = 4
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.1, 1.0, T)
+    S0 = _rand(d, d)
+    O, S = orc.assoc_recurrence_stream(Q, K, V, eta, S0)
+    Oc, Sc = orc.assoc_chunked_stream(Q, K, V, eta, S0, C)
+    Op, Sp = orc.assoc_two_pass_stream(Q, K, V, eta, S0, C, L)
+    for a, b in ((Oc, O), (Sc, S), (Op, O), (Sp, S)):
+        np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-12)
+
+
+def test_assoc_eta_folds_into_values():
+    d, T = 4, 10
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.1, 1.0, T)
+    O, S = orc.assoc_recurrence_stream(Q, K, V, eta, None)
+    O2, S2 = orc.assoc_recurrence_stream(Q, K, eta[:, None] * V, 1.0, None)
+    np.testing.assert_allclose(O, O2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S, S2, rtol=1e-12, atol=1e-13)
+
+
+def test_assoc_is_causal_linear_attention():
+    d, T = 3, 9
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.1, 1.0, T)
+    O, _ = orc.assoc_recurrence_stream(Q, K, V, eta, None)
+    O_la = np.array([sum(eta[s] * (Q[t] @ K[s]) * V[s] for s in range(t + 1)) for t in range(T)])
+    np.testing.assert_allclose(O, O_la, rtol=1e-12, atol=1e-13)
+
+
+def test_assoc_all_streams_helper():
+    B, H, T, d = 2, 2, 8, 3
+    Q, K, V = _rand(B, H, T, d), _rand(B, H, T, d), _rand(B, H, T, d)
+    eta = rng.uniform(0.1, 1.0, (B, H, T))
+    O, S = orc.assoc_scan(Q, K, V, eta, None)
+    Oc, Sc = orc.assoc_scan(Q, K, V, eta, None, form="chunked", C=4, threads=2)
+    np.testing.assert_allclose(O, Oc, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S, Sc, rtol=1e-12, atol=1e-13)
+    o, s = orc.assoc_recurrence_stream(Q[1, 0], K[1, 0], V[1, 0], eta[1, 0], None)
+    np.testing.assert_array_equal(O[1, 0], o)
+
+
+# ----------------------------------------------------------------------------- In-Place TTT
+def test_inplace_prefix_equals_block_strictly_causal_linear_attention():
+    """O_i = Z_i W0 + eta sum_{j<i} (Z_i Z_j^T) Vhat_j: the prefix-sum form read as linear
+    attention over earlier chunks only ("In-Place Test-Time Training", associative memory and
+    associative-scan paragraphs)."""
+    T, Dff, D, C, eta = 24, 7, 5, 6, 0.05
+    Z, Vh, W0 = _rand(T, Dff), _rand(T, D), _rand(Dff, D)
+    O, W = orc.inplace_chunks(Z, Vh, W0, eta, C)
+    O_la = np.empty((T, D))
+    for i0 in range(0, T, C):
+        acc = Z[i0:i0 + C] @ W0
+        for j0 in range(0, i0, C):
+            acc = acc + eta * (Z[i0:i0 + C] @ Z[j0:j0 + C].T) @ Vh[j0:j0 + C]
+        O_la[i0:i0 + C] = acc
+    np.testing.assert_allclose(O, O_la, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(W, W0 + eta * Z.T @ Vh, rtol=1e-12, atol=1e-12)
+
+
+def test_inplace_one_chunk_closed_form():
+    T, Dff, D = 8, 6, 3
+    Z, Vh, W0 = _rand(T, Dff), _rand(T, D), _rand(Dff, D)
+    O, W = orc.inplace_chunks(Z, Vh, W0, 0.01, T)
+    np.testing.assert_allclose(O, Z @ W0, rtol=1e-13)
+    np.testing.assert_allclose(W, W0 + 0.01 * Z.T @ Vh, rtol=1e-13)
+
+
+def test_inplace_delta_is_one_gradient_step_autograd():
+    """The per-chunk delta is one step (learning rate eta) of descent on -<Z_i W, Vhat_i>."""
+    T, Dff, D, eta = 4, 5, 3, 0.1
+    Z, Vh, W0 = _rand(T, Dff), _rand(T, D), _rand(Dff, D)
+    _, W = orc.inplace_chunks(Z, Vh, W0, eta, T)
+    Wt = torch.tensor(W0, requires_grad=True)
+    loss = -((torch.tensor(Z) @ Wt) * torch.tensor(Vh)).sum()
+    (g,) = torch.autograd.grad(loss, Wt)
+    np.testing.assert_allclose(W, (Wt - eta * g).detach().numpy(), rtol=1e-13)
+
+
+def test_inplace_column_subset_is_exact():
+    T, Dff, D, C = 12, 5, 9, 4
+    Z, Vh, W0 = _rand(T, Dff), _rand(T, D), _rand(Dff, D)
+    O, W = orc.inplace_chunks(Z, Vh, W0, 0.2, C)
+    cols = [0, 4, 8]
+    Os, Ws = orc.inplace_chunks(Z, Vh, W0, 0.2, C, cols=cols)
+    np.testing.assert_array_equal(Os, O[:, cols])
+    np.testing.assert_array_equal(Ws, W[:, cols])
+
+
+# ----------------------------------------------------------------------------- hand-worked
+def _golden():
+    with open(GOLDEN) as f:
+        g = json.load(f)
+    g.pop("_about")
+    return g
+
+
+@pytest.mark.parametrize("name", sorted(_golden()))
+def test_hand_worked_examples(name):
+    ex = _golden()[name]
+    if name.startswith("dual"):
+        O, W = orc.dual_form_stream(ex["Q"], ex["K"], ex["V"], np.array(ex["eta"]), ex["W0"],
+                                    ex["C"])
+        np.testing.assert_allclose(W, ex["W"], rtol=0, atol=1e-15)
+    elif name.startswith("assoc"):
+        O, S = orc.assoc_recurrence_stream(ex["Q"], ex["K"], ex["V"], np.array(ex["eta"]),
+                                           ex["S0"])
+        np.testing.assert_allclose(S, ex["S"], rtol=0, atol=1e-15)
+        Oc, _ = orc.assoc_chunked_stream(ex["Q"], ex["K"], ex["V"], np.array(ex["eta"]),
+                                         ex["S0"], len(ex["Q"]))
+        np.testing.assert_allclose(Oc, ex["O"], rtol=0, atol=1e-15)
+    else:
+        O, W = orc.inplace_chunks(ex["Z"], ex["Vhat"], ex["W0"], ex["eta"], ex["C"])
+        np.testing.assert_allclose(W, ex["W"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(O, ex["O"], rtol=0, atol=1e-15)
+
+
+# ----------------------------------------------------------------------------- planted mistakes
+def test_pins_catch_planted_mistakes(monkeypatch):
+    """A plausible slip in the oracle (mask without the diagonal, eta on the target token, a
+    sign flip) must fail the autograd pin. The slip is planted in a copy of the oracle's chunk
+    step, on the CPU."""
+    d, T, C = 4, 12, 4
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.05, 0.4, T)
+    W0 = _rand(d, d, scale=0.3)
+    O_ref, _ = _minibatch_gd_by_definition(Q, K, V, eta, W0, C)
+
+    def variant(mask_k, eta_on_target, sign):
+        W = W0.copy()
+        O = np.empty((T, d))
+        for c0 in range(0, T, C):
+            q, k, v, e = Q[c0:c0 + C], K[c0:c0 + C], V[c0:c0 + C], eta[c0:c0 + C]
+            G = k @ W - v
+            A = np.tril(q @ k.T, mask_k) * (e[:, None] if eta_on_target else e[None, :])
+            O[c0:c0 + C] = q @ W + sign * A @ G
+            W = W - k.T @ (e[:, None] * G)
+        return O
+
+    assert np.allclose(variant(0, False, -1), O_ref, rtol=1e-11, atol=1e-12)
+    for bad in ((-1, False, -1), (0, True, -1), (0, False, +1)):
+        assert not np.allclose(variant(*bad), O_ref, rtol=1e-6, atol=1e-8)
