@@ -1,0 +1,421 @@
+"""Throughput of the chunked fast-weight update-and-read on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one call of the operation over one batch of synthetic input (default workload: the
+TTT-Linear dual form at the 125M-layer shape, B=8 H=12 T=2048 d=64 C=16, bf16). Inputs are
+resident in HBM when timing starts; L2 is flushed (a 256 MiB write) before every timed step.
+Each step is bracketed by CUDA events on the launching stream; the sum over K steps, max over
+ranks, is the timed region, itself bracketed by a barrier and a device synchronize.
+
+Multi-GPU (torchrun, one process per GPU): every (batch, head) stream is independent, so each rank
+runs its own batch with no data-path collective (weak scaling); NCCL is used only for the barrier
+and the max-over-ranks reduction of the timings.
+
+--impl reference times the fp64 CPU oracle (the deliberately slow reference arm) on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "TTT-layer fwd tokens/s on 1 B200; % of bf16 tensor-peak/HBM roofline"
+DEFAULT_WORKLOAD = "dual_bf16_B8H12T2048_d64C16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DOMINANT_KERNEL = {"dual": ("dual_mma_kernel", "dual_mma.cu"),
+                   "assoc": ("assoc_pass2_kernel", "assoc_scan.cu"),
+                   "inplace": ("inplace_gemm_kernel", "inplace_ttt.cu")}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha(fname: str) -> str:
+    path = os.path.join(ROOT, "weight_linear_attention_ttt_b200", "csrc", fname)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(workload: str, kernel: str, sha: str):
+    """DRAM bytes per launch from a committed ncu summary, valid only for the same kernel
+    source (profiles/dram_traffic.txt: `workload kernel source_sha256_16 bytes_per_launch`)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        f = line.split()
+        if len(f) >= 4 and not line.startswith("#") and f[0] == workload and f[1] == kernel \
+                and f[2] == sha:
+            return float(f[3])
+    return None
+
+
+# ----------------------------------------------------------------------------- clocks (NVML)
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            try:
+                uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: clocks are reported as unavailable
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = get_reasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._h is not None:
+            self._t.join()
+
+    def summary(self):
+        if self._h is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- workload calls
+def make_call(w, x, stream_outputs=None):
+    """Returns step() -> outputs, running the whole operation once on the current stream."""
+    import torch
+
+    import weight_linear_attention_ttt_b200 as ttt
+
+    if w.kind == "dual":
+        O = torch.empty_like(x["Q"])
+        W = torch.empty((w.B, w.H, w.d, w.d), device=x["Q"].device, dtype=torch.float32)
+        return lambda: ttt.ttt_linear_dual_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W0"], C=w.C,
+                                               eta_scalar=x["eta_scalar"], O=O, W_out=W)
+    if w.kind == "assoc":
+        O = torch.empty_like(x["Q"])
+        S = torch.empty((w.B, w.H, w.d, w.d), device=x["Q"].device, dtype=torch.float32)
+        lib = ttt.load_library()
+        nbytes = lib.ttt_assoc_scan_workspace_size(w.B, w.H, w.T, w.d, w.C, 1)
+        ws = torch.empty(max(nbytes, 16), device=x["Q"].device, dtype=torch.uint8)
+        return lambda: ttt.ttt_assoc_scan_fwd(x["Q"], x["K"], x["V"], x["eta"], None, C=w.C,
+                                              eta_scalar=x["eta_scalar"], O=O, S_out=S,
+                                              workspace=ws)
+    if w.kind == "inplace":
+        O = torch.empty((w.T, w.D), device=x["Z"].device, dtype=torch.bfloat16)
+        Wf = torch.empty((w.Dff, w.D), device=x["Z"].device, dtype=torch.float32)
+        lib = ttt.load_library()
+        nbytes = lib.inplace_ttt_workspace_size(w.T, w.Dff, w.D, w.C)
+        ws = torch.empty(max(nbytes, 16), device=x["Z"].device, dtype=torch.uint8)
+        return lambda: ttt.inplace_ttt_chunk_fwd(x["Z"], x["Vhat"], x["W0"], x["eta"], C=w.C,
+                                                 O=O, W_out=Wf, workspace=ws)
+    raise ValueError(w.kind)
+
+
+def e2e_measure(w, x, steps: int, warmup: int):
+    """Same metric through the public API from pinned HOST buffers: every step copies its inputs
+    host->device, runs the operation and copies the result (O and the final state) back."""
+    import torch
+
+    import weight_linear_attention_ttt_b200 as ttt
+
+    host = {k: v.cpu().pin_memory() for k, v in x.items() if torch.is_tensor(v)}
+    dev = {k: torch.empty_like(v) for k, v in x.items() if torch.is_tensor(v)}
+    scal = {k: v for k, v in x.items() if not torch.is_tensor(v)}
+    if w.kind == "inplace":
+        out_shapes = [((w.T, w.D), torch.bfloat16), ((w.Dff, w.D), torch.float32)]
+    else:
+        out_shapes = [((w.B, w.H, w.T, w.d), x["Q"].dtype), ((w.B, w.H, w.d, w.d), torch.float32)]
+    outs_h = [torch.empty(s, dtype=dt).pin_memory() for s, dt in out_shapes]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+    xd = dict(dev, **scal)
+    if w.kind != "inplace" and x.get("eta") is None:
+        xd["eta"] = None
+    call = make_call(w, xd)
+
+    def step():
+        for k in host:
+            dev[k].copy_(host[k], non_blocking=True)
+        outs = call()
+        for h, d in zip(outs_h, outs):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    return ms, h2d, d2h
+
+
+def oracle_sample(w, x, budget_s: float, cursor: list):
+    """Runs the fp64 oracle on a bounded sample of the workload; returns (tokens, seconds,
+    threads, description). The sample is whole (b,h) streams (a prefix of chunks when one
+    stream exceeds the budget) or output-column subsets of the In-Place workload."""
+    import numpy as np
+
+    from oracle import ttt_oracle as orc
+
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    if w.kind in ("dual", "assoc"):
+        streams = [(b, h) for b in range(w.B) for h in range(w.H)]
+        Q, K, V = (x[k].float().cpu().numpy() for k in ("Q", "K", "V"))
+        eta = None if x["eta"] is None else x["eta"].cpu().numpy()
+        W0 = x["W0"].cpu().numpy()
+        # probe the cost of one chunk-run of one stream to size the sample
+        tok = 0
+        n_streams = 0
+        ncol = w.T if w.kind == "dual" else min(w.T, 4096)
+        while True:
+            b, h = streams[cursor[0] % len(streams)]
+            cursor[0] += 1
+            e = w.eta_const if eta is None else eta[b, h, :ncol]
+            if w.kind == "dual":
+                orc.dual_form_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
+                                     W0[b, h], w.C)
+            else:
+                orc.assoc_recurrence_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
+                                            None)
+            tok += ncol
+            n_streams += 1
+            if time.perf_counter() - t0 >= budget_s or n_streams >= len(streams):
+                break
+        desc = (f"{n_streams} (b,h) stream(s) x {ncol} tokens of the workload, "
+                f"{'dual-form per-chunk loop' if w.kind == 'dual' else 'sequential recurrence'}"
+                f", numpy fp64, 1 thread")
+        return tok / w.H, time.perf_counter() - t0, 1, desc
+    # In-Place: every 80th output column over all chunks (columns are independent)
+    cols = np.arange(cursor[0] % 80, w.D, 80)
+    cursor[0] += 1
+    Z = x["Z"].float().cpu().numpy()
+    Vh = x["Vhat"].float().cpu().numpy()[:, cols]
+    W0 = x["W0"].float().cpu().numpy()[:, cols]
+    t0 = time.perf_counter()
+    orc.inplace_chunks(Z, Vh, W0, x["eta"], w.C)
+    dt = time.perf_counter() - t0
+    frac = len(cols) / w.D
+    return w.T * frac, dt, threads, (f"{len(cols)} of {w.D} output columns over all "
+                                     f"{w.T // w.C} chunks, numpy fp64 BLAS")
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, w, rank, world):
+    """The oracle as the reference arm, on rank 0's host cores."""
+    import torch
+
+    from weight_linear_attention_ttt_b200 import inputs as inp
+
+    if rank != 0:
+        return 0
+    x = inp.make_inputs(w, "cpu")
+    cursor = [0]
+    per_step_budget = max(0.05, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(w, x, per_step_budget, cursor)
+    tok_total, sec_total, threads, desc = 0.0, 0.0, 1, ""
+    for _ in range(args.steps):
+        tok, sec, threads, desc = oracle_sample(w, x, per_step_budget, cursor)
+        tok_total += tok
+        sec_total += sec
+    value = tok_total / sec_total
+    ms = 1e3 * sec_total / args.steps
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "sample_per_step": desc},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import weight_linear_attention_ttt_b200 as ttt
+    from weight_linear_attention_ttt_b200 import inputs as inp
+    from weight_linear_attention_ttt_b200 import metrics
+
+    dev = torch.device("cuda", local_rank)
+    ttt.load_library()
+    x = inp.make_inputs(w, dev, seed=w.seed + 7919 * rank)
+    step = make_call(w, x)
+    flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
+    algo = metrics.algorithmic(w)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = ttt.launch_count()
+    with ClockSampler(local_rank) as clk:
+        for a, b in ev:
+            flush.zero_()
+            a.record()
+            step()
+            b.record()
+        torch.cuda.synchronize()
+    launches = ttt.launch_count() - n0
+    if world > 1:
+        dist.barrier()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * algo["tokens"] * args.steps / (total_ms / 1e3)
+    assert ttt.read_device_error() == 0, "a bounded device wait gave up during the bench"
+
+    # end to end from host buffers, same metric
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_ms, h2d, d2h = e2e_measure(w, x, e2e_steps, 2)
+    et = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(et, op=dist.ReduceOp.MAX)
+    e2e_value = world * algo["tokens"] / (float(et.item()) / 1e3)
+
+    pk, pk_kind = peaks()
+    kname, ksrc = DOMINANT_KERNEL[w.kind]
+    launches_per_step = launches / args.steps
+    if w.kind == "inplace":
+        achieved = algo["flops"] / (ms_per_step / 1e3) / 1e12
+        peak = pk["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak}
+    else:
+        achieved = algo["bytes"] / (ms_per_step / 1e3) / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak}
+    sha = kernel_source_sha(ksrc)
+    roof.update({"traffic": measured_traffic(w.name, kname, sha), "kernel": kname,
+                 "peak_source": f"{pk_kind} (MEASURED_PEAKS.json)" if pk_kind == "measured"
+                 else "fallback", "launches_per_step": launches_per_step,
+                 "kernel_source_sha": sha,
+                 "duration_us": 1e3 * ms_per_step / max(1.0, launches_per_step)
+                 if w.kind == "dual" else None})
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "kind": w.kind, "B": w.B, "H": w.H, "T": w.T,
+                       "d": w.d, "C": w.C, "tokens_per_step_per_gpu": algo["tokens"],
+                       "l2": "flushed (256 MiB write) before every timed step",
+                       "parallelism": f"dp{world} (independent streams per rank)"},
+            "roofline": roof, "clocks": clk.summary(), "gpu_launches": launches,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": float(et.item())}}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cursor = [0]
+        budget = args.cpu_budget
+        tok, sec, threads, desc = oracle_sample(w, {k: (v.cpu() if torch.is_tensor(v) else v)
+                                                    for k, v in x.items()}, budget, cursor)
+        line["cpu_baseline"] = {"value": tok / sec, "unit": "tokens/s", "cores": threads,
+                                "kind": "oracle", "sample": desc, "seconds": sec}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    from weight_linear_attention_ttt_b200 import inputs as inp
+
+    w = inp.WORKLOADS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,144 @@
+/*
+ * ttt.h - C ABI of the B200 (sm_100a) fast-weight update-and-read library (libttt_b200.so).
+ *
+ * Three operations, each the chunked update-and-read of a fast-weight state whose inner model is
+ * linear and bias-free:
+ *
+ *   ttt_linear_dual_fwd    TTT-Linear, mini-batch dual form.
+ *                          Source: "RNN의 기억을 작은 모델로 바꾼다면: Test-Time Training 읽기"
+ *                          (a reading of "Learning to (Learn at Test Time)"), section
+ *                          "gradient를 효율적인 layer로 만드는 작업" (mini-batch TTT and its dual
+ *                          form) and section "읽는 동안 문제를 하나 더 푼다" (per-token rule, output
+ *                          read from the updated model).
+ *   ttt_assoc_scan_fwd     weight-norm-free, gradient-ascent linear-attention form, computed
+ *                          chunk-parallel with a prefix scan over chunk states.
+ *                          Source: "KV 바인딩 기반 테스트 시간 학습은 사실상 선형 어텐션이다"
+ *                          (one-step closed form o = q(S0 + k^T v); removing weight normalisation
+ *                          restores associativity and allows a parallel prefix scan; per-token
+ *                          learning rates fold into the values; gradient ascent).
+ *   inplace_ttt_chunk_fwd  In-Place TTT: W_down of a gated MLP as the fast weight, one step per
+ *                          chunk, deltas combined by a prefix sum.
+ *                          Source: "In-Place 테스트 시점 학습: LLM을 위한 원활한 동적 적응 프레임워크"
+ *                          (gated-MLP paragraph, chunk-update paragraph, associative-scan
+ *                          paragraph).
+ *
+ * Conventions shared by every entry point
+ *   - Row vectors: q_t, k_t, v_t are 1 x d; the state W (or S) is d x d laid out [d_in][d_out]
+ *     (row-major), and a token reads o_t = q_t W.
+ *   - Tensors [B,H,T,d] are contiguous row-major; stream (b,h) owns rows (b*H+h)*T .. +T-1.
+ *   - All pointers except host-side scalars are DEVICE pointers owned by the caller. The library
+ *     allocates no device memory of its own and never synchronises: all work is enqueued on
+ *     `stream` (0 = the legacy default stream) in order. Scratch memory is the caller's
+ *     `workspace` of at least the size the matching *_workspace_size() returns.
+ *   - Errors that the host can detect (null or misaligned pointers, bad sizes, unsupported
+ *     shapes, short workspace) return a status BEFORE anything is launched; outputs are then
+ *     untouched. A failed launch returns TTT_ERR_CUDA. Details of the last error of the calling
+ *     thread are in ttt_last_error_message().
+ *   - Every device pointer must be 16-byte aligned.
+ *   - Outputs must not overlap inputs, except the documented state aliasing (W_out == W0,
+ *     S_out == S0 is allowed: the state is read before it is written).
+ *   - Numerics: bf16 operands go through the tensor cores with fp32 accumulation; the state is
+ *     kept in fp32; outputs O are rounded (nearest-even) to the input dtype; final states are
+ *     fp32. fp32 inputs use an exact-fp32 CUDA-core path (no TF32).
+ */
+#ifndef TTT_B200_TTT_H
+#define TTT_B200_TTT_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTT_OK = 0,
+  TTT_ERR_INVALID_ARG = 1, /* null/misaligned pointer, non-positive size, T % C != 0, bad dtype */
+  TTT_ERR_UNSUPPORTED = 2, /* valid but not implemented: head dim, chunk size, dtype combination */
+  TTT_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than *_workspace_size() */
+  TTT_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed */
+  TTT_ERR_TIMEOUT = 5      /* reserved: a bounded device-side wait gave up (none wait today) */
+} ttt_status_t;
+
+typedef enum { TTT_DTYPE_F32 = 0, TTT_DTYPE_BF16 = 1 } ttt_dtype_t;
+
+/* Static, human-readable name of a status code. */
+const char* ttt_status_string(int status);
+
+/* Detail of the last non-OK status returned on the calling thread ("" if none). */
+const char* ttt_last_error_message(void);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int ttt_version(void);
+
+/* Number of kernels this library has launched in this process (all entry points, all devices). */
+uint64_t ttt_launch_count(void);
+
+/* Reads and clears the current device's error word. Bit 0 set means a bounded device-side wait
+ * gave up (a kernel stopped early; its outputs are incomplete). SYNCHRONOUS: waits for all work
+ * on the device to finish. Returns TTT_OK or TTT_ERR_CUDA. */
+int ttt_read_device_error(unsigned* value);
+
+/* --------------------------------------------------------------------------------------------
+ * TTT-Linear, mini-batch dual form (per stream (b,h), W = W0, for each chunk c of C tokens):
+ *     G   = K_c W - V_c                                  residual of 1/2||k W - v||^2
+ *     O_c = Q_c W - (tril(Q_c K_c^T) diag(eta_c)) G      tril includes the diagonal
+ *     W   = W - K_c^T diag(eta_c) G
+ *
+ *  Q, K, V   [B,H,T,d] of dtype `dt` (fp32 or bf16).
+ *  eta       [B,H,T] fp32 per-token learning rates, or NULL to use `eta_scalar` for every token.
+ *            A learning rate scales its own (source) token's gradient.
+ *  W0        [B,H,d,d] fp32 initial state, or NULL for zeros.
+ *  O         [B,H,T,d] of dtype `dt` (output).
+ *  W_out     [B,H,d,d] fp32 final state (output); may be the same pointer as W0.
+ *  Supported: d in {32, 64, 128}; 1 <= C <= 64; T % C == 0. bf16 with C == 16 and d in
+ *  {32, 64, 128} runs the tensor-core path; other supported shapes run the CUDA-core path.
+ *  Workspace: none (ttt_linear_dual_workspace_size returns 0; `workspace` may be NULL).
+ * ------------------------------------------------------------------------------------------ */
+size_t ttt_linear_dual_workspace_size(int B, int H, int T, int d, int C, int dt);
+int ttt_linear_dual_fwd(const void* Q, const void* K, const void* V, const float* eta,
+                        float eta_scalar, const float* W0, void* O, float* W_out, int B, int H,
+                        int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+/* --------------------------------------------------------------------------------------------
+ * Associative (gradient-ascent, weight-norm-free) linear-attention mode, per stream:
+ *     S_t = S_(t-1) + eta_t k_t^T v_t,   o_t = q_t S_t      (S_0 = S0)
+ *  computed per chunk of C tokens as O_c = Q_c S + (tril(Q_c K_c^T) diag(eta_c)) V_c,
+ *  S += K_c^T diag(eta_c) V_c, with a two-pass prefix scan over superchunk states.
+ *
+ *  Q, K, V, O [B,H,T,d]; eta [B,H,T] fp32 or NULL (eta_scalar); S0 [B,H,d,d] fp32 or NULL
+ *  (zeros); S_out [B,H,d,d] fp32, may equal S0.
+ *  Supported: bf16, d == 128, C == 64, T % C == 0 (tensor-core path).
+ *  Workspace: ttt_assoc_scan_workspace_size() bytes (superchunk states, fp32).
+ * ------------------------------------------------------------------------------------------ */
+size_t ttt_assoc_scan_workspace_size(int B, int H, int T, int d, int C, int dt);
+int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float* eta,
+                       float eta_scalar, const float* S0, void* O, float* S_out, int B, int H,
+                       int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
+
+/* --------------------------------------------------------------------------------------------
+ * In-Place TTT, W_down chunk update (W = W0; for each chunk i of C tokens, in order):
+ *     O_i = Z_i W                  (W holds W0 plus the deltas of the chunks before i)
+ *     W   = W + eta Z_i^T Vhat_i
+ *
+ *  Z     [T,Dff] bf16 activations (the gated-MLP hidden state).
+ *  Vhat  [T,D]  bf16 targets.
+ *  W0    [Dff,D] bf16 initial W_down.
+ *  O     [T,D]  bf16 output.
+ *  W_out [Dff,D] fp32 final W_down (the running fp32 master).
+ *  Supported: T % C == 0; C % 128 == 0; Dff % 128 == 0; D % 256 == 0.
+ *  Workspace: inplace_ttt_workspace_size() bytes (bf16 copy of the running W).
+ * ------------------------------------------------------------------------------------------ */
+size_t inplace_ttt_workspace_size(int T, int Dff, int D, int C);
+int inplace_ttt_chunk_fwd(const void* Z, const void* Vhat, const void* W0, float eta, void* O,
+                          float* W_out, int T, int Dff, int D, int C, void* workspace,
+                          size_t workspace_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_B200_TTT_H */

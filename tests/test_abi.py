@@ -1,0 +1,105 @@
+"""The C-ABI library builds, loads and exports every declared symbol; host-side validation
+returns its status before anything is launched (CPU only: no compute call is made)."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+import weight_linear_attention_ttt_b200 as ttt
+from weight_linear_attention_ttt_b200 import build as ttt_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ttt_build.build()
+    return ttt.load_library()
+
+
+def _declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", src, flags=re.M):
+            if m.group(1) not in ("if", "defined"):
+                names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_header_declares_the_binding_symbols():
+    assert set(_declared_functions()) == set(ttt.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", ttt.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in _declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.ttt_status_string(0) == b"TTT_OK"
+    assert lib.ttt_status_string(3) == b"TTT_ERR_WORKSPACE"
+    assert lib.ttt_status_string(99) == b"TTT_ERR_UNKNOWN"
+    assert lib.ttt_version() >= 10000
+    assert lib.ttt_launch_count() == 0  # nothing launched on a CPU-only host
+
+
+# Fake, never-dereferenced device addresses: validation fails before any CUDA call.
+A = 1 << 20
+
+
+def _dual(lib, **kw):
+    args = dict(Q=A, K=2 * A, V=3 * A, eta=4 * A, eta_scalar=0.0, W0=5 * A, O=6 * A, W_out=7 * A,
+                B=1, H=1, T=64, d=64, C=16, dt=1, ws=0, ws_bytes=0, stream=0)
+    args.update(kw)
+    v = ctypes.c_void_p
+    return lib.ttt_linear_dual_fwd(v(args["Q"]), v(args["K"]), v(args["V"]), v(args["eta"]),
+                                   ctypes.c_float(args["eta_scalar"]), v(args["W0"]),
+                                   v(args["O"]), v(args["W_out"]), args["B"], args["H"],
+                                   args["T"], args["d"], args["C"], args["dt"], v(args["ws"]),
+                                   args["ws_bytes"], v(args["stream"]))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Q=0), 1), (dict(O=0), 1), (dict(W_out=0), 1),
+    (dict(K=2 * A + 8), 1),                  # misaligned
+    (dict(T=60), 1),                         # T % C != 0
+    (dict(B=0), 1), (dict(C=-16), 1), (dict(dt=7), 1),
+    (dict(d=48), 2), (dict(C=128, T=128), 2),
+    (dict(O=A + 64), 1),                     # O overlaps Q
+    (dict(W_out=5 * A + 64), 1),             # partial overlap with W0
+])
+def test_dual_validation(lib, kw, status):
+    assert _dual(lib, **kw) == status
+    assert lib.ttt_last_error_message() != b""
+    assert lib.ttt_launch_count() == 0
+
+
+def test_assoc_and_inplace_validation(lib):
+    v = ctypes.c_void_p
+    st = lib.ttt_assoc_scan_fwd(v(A), v(2 * A), v(3 * A), None, ctypes.c_float(1.0), None,
+                                v(6 * A), v(7 * A), 1, 1, 100, 128, 64, 1, None, 0, None)
+    assert st == 1  # T % C
+    st = lib.inplace_ttt_chunk_fwd(v(A), v(2 * A), v(3 * A), ctypes.c_float(1e-3), v(4 * A),
+                                   None, 2048, 256, 256, 1024, None, 0, None)
+    assert st == 1  # W_out null
+    st = lib.inplace_ttt_chunk_fwd(v(A), v(2 * A), v(3 * A), ctypes.c_float(1e-3), v(4 * A),
+                                   v(5 * A), 2000, 256, 256, 1024, None, 0, None)
+    assert st == 1  # T % C
+    assert lib.ttt_launch_count() == 0
+
+
+def test_python_binding_rejects_non_cuda_tensors(lib):
+    import torch
+
+    x = torch.zeros(1, 1, 16, 32)
+    with pytest.raises(ValueError):
+        ttt.ttt_linear_dual_fwd(x, x, x, C=16)

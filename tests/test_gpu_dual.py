@@ -1,0 +1,191 @@
+"""GPU parity of ttt_linear_dual_fwd against the fp64 oracle, through the C ABI.
+
+Tolerances (max over (b,h) slices of the relative L2 error, for O and for the final W):
+1e-4 for fp32 inputs, 1e-2 for bf16 inputs.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import weight_linear_attention_ttt_b200 as ttt
+from _helpers import f64, max_rel_l2
+from oracle import ttt_oracle as orc
+from weight_linear_attention_ttt_b200 import inputs as inp
+
+pytestmark = pytest.mark.gpu
+TOL = {"f32": 1e-4, "bf16": 1e-2}
+
+
+def run(x, C, **kw):
+    return ttt.ttt_linear_dual_fwd(x["Q"], x["K"], x["V"], x["eta"], x.get("W0"), C=C,
+                                   eta_scalar=x["eta_scalar"], **kw)
+
+
+def oracle(x, C, streams=None):
+    eta = x["eta_scalar"] if x["eta"] is None else x["eta"].cpu().numpy()
+    W0 = None if x.get("W0") is None else x["W0"].cpu().numpy()
+    Q, K, V = (x[k].float().cpu().numpy() for k in ("Q", "K", "V"))
+    return orc.dual_form(Q, K, V, eta, W0, C, threads=os.cpu_count() or 4, streams=streams)
+
+
+def check(x, C, O, W, tol, streams=None):
+    Or, Wr = oracle(x, C, streams)
+    if streams is not None:
+        O = torch.stack([O[b, h] for b, h in streams])
+        W = torch.stack([W[b, h] for b, h in streams])
+        lead = 1
+    else:
+        lead = 2
+    eo, ew = max_rel_l2(O, Or, lead), max_rel_l2(W, Wr, lead)
+    assert eo <= tol and ew <= tol, (eo, ew)
+    return eo, ew
+
+
+def workload(name, **over):
+    w = inp.WORKLOADS[name]
+    return w, inp.make_inputs(w, "cuda", **over)
+
+
+def test_fp32_tiny_workload(cuda_lib):
+    w, x = workload("dual_f32_B1H2T256_d32C16")
+    O, W = run(x, w.C)
+    check(x, w.C, O, W, TOL["f32"])
+    # W0 given as NULL (zeros) gives the same bits as an explicit zero tensor
+    x0 = dict(x, W0=None)
+    O0, W0_ = run(x0, w.C)
+    assert torch.equal(O, O0) and torch.equal(W, W0_)
+    assert ttt.read_device_error() == 0
+
+
+def test_bf16_125m_layer_workload(cuda_lib):
+    w, x = workload("dual_bf16_B8H12T2048_d64C16")
+    O, W = run(x, w.C)
+    eo, ew = check(x, w.C, O, W, TOL["bf16"])
+    print(f"dual 125M-layer workload: max rel L2 O {eo:.2e} W {ew:.2e}")
+    assert ttt.read_device_error() == 0
+
+
+def test_bf16_long_context_workload(cuda_lib):
+    w, x = workload("dual_bf16_B2H32T32768_d64C16")
+    O, W = run(x, w.C)
+    streams = [(0, 0), (0, 17), (1, 5), (1, 31)]
+    eo, ew = check(x, w.C, O, W, TOL["bf16"], streams)
+    print(f"dual long-context workload (4 sampled streams): max rel L2 O {eo:.2e} W {ew:.2e}")
+    # every stream is finite and was written
+    assert torch.isfinite(O.float()).all() and torch.isfinite(W).all()
+    assert ttt.read_device_error() == 0
+
+
+SWEEP = [(d, C, m, B, H) for d in (32, 64, 128) for C in (1, 16, 64) for m in (1, 2, 7)
+         for (B, H) in ((1, 1), (1, 3), (3, 1)) if (d + C + m + B) % 3 == 0 or C == 16]
+
+
+@pytest.mark.parametrize("d,C,m,B,H", SWEEP)
+def test_sweep_bf16(cuda_lib, d, C, m, B, H):
+    x = inp.dual_or_assoc_inputs(B, H, m * C, d, seed=d * 1000 + C * 10 + m, device="cuda",
+                                 normalise=("K", "V"))
+    O, W = run(x, C)
+    check(x, C, O, W, TOL["bf16"])
+
+
+@pytest.mark.parametrize("d,C,m", [(32, 16, 3), (64, 1, 5), (64, 64, 2), (128, 16, 2)])
+def test_sweep_fp32(cuda_lib, d, C, m):
+    x = inp.dual_or_assoc_inputs(2, 2, m * C, d, seed=7 + d + C, device="cuda", dtype="f32",
+                                 qkv="normal_1_over_d", eta="sigmoid_over_d")
+    O, W = run(x, C)
+    check(x, C, O, W, TOL["f32"])
+
+
+@pytest.mark.parametrize("T", [16, 48, 64, 80, 112, 1040])
+def test_ragged_stage_tails(cuda_lib, T):
+    """T that is not a multiple of the kernel's 64-token pipeline stage (partial last stage)."""
+    x = inp.dual_or_assoc_inputs(2, 3, T, 64, seed=T, device="cuda", normalise=("K", "V"))
+    O, W = run(x, 16)
+    check(x, 16, O, W, TOL["bf16"])
+
+
+def test_state_aliasing_W_out_equals_W0(cuda_lib):
+    x = inp.dual_or_assoc_inputs(2, 2, 256, 64, seed=3, device="cuda", normalise=("K", "V"))
+    O_ref, W_ref = run(x, 16)
+    W_io = x["W0"].clone()
+    O, W = ttt.ttt_linear_dual_fwd(x["Q"], x["K"], x["V"], x["eta"], W_io, C=16, W_out=W_io)
+    assert W.data_ptr() == W_io.data_ptr()
+    assert torch.equal(O, O_ref) and torch.equal(W_io, W_ref)
+
+
+def test_determinism_permutation_and_state_carry(cuda_lib):
+    x = inp.dual_or_assoc_inputs(2, 3, 512, 64, seed=11, device="cuda", normalise=("K", "V"))
+    O1, W1 = run(x, 16)
+    O2, W2 = run(x, 16)
+    assert torch.equal(O1, O2) and torch.equal(W1, W2)  # bitwise run-to-run
+    # batch items are independent: permuting streams permutes outputs, bit for bit
+    perm = torch.tensor([4, 0, 5, 2, 1, 3], device="cuda")
+    xp = {k: (v.reshape(6, *v.shape[2:])[perm].reshape(v.shape) if torch.is_tensor(v) else v)
+          for k, v in x.items()}
+    Op, Wp = run(xp, 16)
+    assert torch.equal(Op.reshape(6, 512, 64), O1.reshape(6, 512, 64)[perm])
+    assert torch.equal(Wp.reshape(6, 64, 64), W1.reshape(6, 64, 64)[perm])
+    # state carry: two calls over the halves, chained through W_out -> W0, equal one call
+    h = 208  # a chunk boundary that is not a pipeline-stage boundary
+    xa = {k: (v[:, :, :h] if torch.is_tensor(v) and v.dim() >= 3 and k != "W0" else v)
+          for k, v in x.items()}
+    xb = {k: (v[:, :, h:].contiguous() if torch.is_tensor(v) and v.dim() >= 3 and k != "W0"
+              else v) for k, v in x.items()}
+    xa = {k: (v.contiguous() if torch.is_tensor(v) else v) for k, v in xa.items()}
+    Oa, Wa = run(xa, 16)
+    xb["W0"] = Wa
+    Ob, Wb = run(xb, 16)
+    assert torch.equal(torch.cat([Oa, Ob], dim=2), O1) and torch.equal(Wb, W1)
+
+
+def test_column_split_variants_agree_bitwise(cuda_lib, monkeypatch):
+    x = inp.dual_or_assoc_inputs(1, 4, 256, 64, seed=5, device="cuda", normalise=("K", "V"))
+    outs = []
+    for split in ("1", "2"):
+        monkeypatch.setenv("TTT_DUAL_COLUMN_SPLIT", split)
+        outs.append(run(x, 16))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    x = inp.dual_or_assoc_inputs(1, 2, 128, 128, seed=6, device="cuda", normalise=("K", "V"))
+    outs = []
+    for split in ("1", "2"):
+        monkeypatch.setenv("TTT_DUAL_COLUMN_SPLIT", split)
+        outs.append(run(x, 16))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_degenerate_cases(cuda_lib):
+    # eta = 0: no update; O = Q W0
+    x = inp.dual_or_assoc_inputs(1, 2, 128, 64, seed=9, device="cuda", normalise=("K", "V"),
+                                 eta="const", eta_const=0.0)
+    O, W = run(x, 16)
+    assert torch.equal(W, x["W0"])
+    check(x, 16, O, W, TOL["bf16"])
+    # keys all zero: residual is -V but the update K^T G vanishes; O = Q W0
+    x["K"] = torch.zeros_like(x["K"])
+    x["eta"], x["eta_scalar"] = None, 0.5
+    O, W = run(x, 16)
+    assert torch.equal(W, x["W0"])
+    check(x, 16, O, W, TOL["bf16"])
+
+
+def test_one_launch_per_call(cuda_lib):
+    x = inp.dual_or_assoc_inputs(1, 1, 64, 64, seed=1, device="cuda")
+    n0 = ttt.launch_count()
+    run(x, 16)
+    run(x, 4)
+    assert ttt.launch_count() - n0 == 2
+
+
+def test_invalid_calls_raise_before_launch(cuda_lib):
+    x = inp.dual_or_assoc_inputs(1, 1, 64, 64, seed=1, device="cuda")
+    n0 = ttt.launch_count()
+    with pytest.raises(ttt.TTTError) as e:
+        run(x, 24)  # T % C != 0
+    assert e.value.status == 1
+    x48 = inp.dual_or_assoc_inputs(1, 1, 64, 48, seed=1, device="cuda")
+    with pytest.raises(ttt.TTTError) as e:
+        run(x48, 16)
+    assert e.value.status == 2
+    assert ttt.launch_count() == n0

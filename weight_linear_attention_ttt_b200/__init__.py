@@ -1,0 +1,195 @@
+"""Python binding of libttt_b200 (the C ABI declared in include/ttt.h).
+
+Argument marshalling only: each function checks torch tensors, allocates missing outputs and
+workspace with torch (device memory plumbing), and calls the C entry point of the same name on
+the current CUDA stream. Every step of the computation runs in the library's CUDA kernels; there
+is no CPU or PyTorch fallback, and a missing library raises at load time.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libttt_b200.so")
+
+TTT_DTYPE_F32 = 0
+TTT_DTYPE_BF16 = 1
+STATUS = {0: "TTT_OK", 1: "TTT_ERR_INVALID_ARG", 2: "TTT_ERR_UNSUPPORTED",
+          3: "TTT_ERR_WORKSPACE", 4: "TTT_ERR_CUDA", 5: "TTT_ERR_TIMEOUT"}
+
+# Every symbol include/ttt.h declares.
+EXPORTED_SYMBOLS = (
+    "ttt_status_string", "ttt_last_error_message", "ttt_version", "ttt_launch_count",
+    "ttt_read_device_error",
+    "ttt_linear_dual_workspace_size", "ttt_linear_dual_fwd",
+    "ttt_assoc_scan_workspace_size", "ttt_assoc_scan_fwd",
+    "inplace_ttt_workspace_size", "inplace_ttt_chunk_fwd",
+)
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+class TTTError(RuntimeError):
+    """A non-OK status from the library; ``status`` holds the code."""
+
+    def __init__(self, fn: str, status: int, detail: str):
+        super().__init__(f"{fn}: {STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Loads the CUDA library (once). Raises if it has not been built."""
+    global _LIB
+    if _LIB is not None and path is None:
+        return _LIB
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(
+            f"CUDA extension not built: {p} is missing "
+            "(run `python -m weight_linear_attention_ttt_b200.build`)")
+    lib = ctypes.CDLL(p)
+    c_int, c_float, c_size, vp, fp = (ctypes.c_int, ctypes.c_float, ctypes.c_size_t,
+                                      ctypes.c_void_p, ctypes.c_void_p)
+    lib.ttt_status_string.restype = ctypes.c_char_p
+    lib.ttt_status_string.argtypes = [c_int]
+    lib.ttt_last_error_message.restype = ctypes.c_char_p
+    lib.ttt_last_error_message.argtypes = []
+    lib.ttt_version.restype = c_int
+    lib.ttt_launch_count.restype = ctypes.c_uint64
+    lib.ttt_read_device_error.restype = c_int
+    lib.ttt_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    state_args = [vp, vp, vp, fp, c_float, fp, vp, fp, c_int, c_int, c_int, c_int, c_int, c_int,
+                  vp, c_size, vp]
+    for name in ("ttt_linear_dual_fwd", "ttt_assoc_scan_fwd"):
+        getattr(lib, name).restype = c_int
+        getattr(lib, name).argtypes = state_args
+    for name in ("ttt_linear_dual_workspace_size", "ttt_assoc_scan_workspace_size"):
+        getattr(lib, name).restype = c_size
+        getattr(lib, name).argtypes = [c_int] * 6
+    lib.inplace_ttt_workspace_size.restype = c_size
+    lib.inplace_ttt_workspace_size.argtypes = [c_int] * 4
+    lib.inplace_ttt_chunk_fwd.restype = c_int
+    lib.inplace_ttt_chunk_fwd.argtypes = [vp, vp, vp, c_float, vp, fp, c_int, c_int, c_int,
+                                          c_int, vp, c_size, vp]
+    if path is None:
+        _LIB = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise TTTError(fn, status, load_library().ttt_last_error_message().decode())
+
+
+def _stream_ptr(stream):
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    if t.dtype == torch.float32:
+        return TTT_DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return TTT_DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; expected float32 or bfloat16")
+
+
+def _require(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _state_call(fn_name: str, ws_name: str, Q, K, V, eta, eta_scalar, S0, C, O, S_out,
+                workspace, stream):
+    import torch
+
+    lib = load_library()
+    _require(Q.dim() == 4, "Q, K, V must be [B, H, T, d]")
+    B, H, T, d = Q.shape
+    for t in (Q, K, V):
+        _require(t.is_cuda and t.is_contiguous() and t.shape == Q.shape and t.dtype == Q.dtype,
+                 "Q, K, V must be contiguous CUDA tensors of one shape and dtype")
+    dt = _dtype_code(Q)
+    if eta is not None:
+        _require(eta.is_cuda and eta.dtype == torch.float32 and eta.is_contiguous() and
+                 tuple(eta.shape) == (B, H, T), "eta must be a contiguous fp32 [B, H, T] tensor")
+    if S0 is not None:
+        _require(S0.is_cuda and S0.dtype == torch.float32 and S0.is_contiguous() and
+                 tuple(S0.shape) == (B, H, d, d), "initial state must be fp32 [B, H, d, d]")
+    if O is None:
+        O = torch.empty_like(Q)
+    if S_out is None:
+        S_out = torch.empty((B, H, d, d), device=Q.device, dtype=torch.float32)
+    ws_bytes = getattr(lib, ws_name)(B, H, T, d, C, dt)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, device=Q.device, dtype=torch.uint8)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = getattr(lib, fn_name)(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), ctypes.c_float(eta_scalar),
+                               _ptr(S0), _ptr(O), _ptr(S_out), B, H, T, d, C, dt,
+                               _ptr(workspace), wsz, _stream_ptr(stream))
+    _check(fn_name, st)
+    return O, S_out
+
+
+def ttt_linear_dual_fwd(Q, K, V, eta=None, W0=None, *, C: int, eta_scalar: float = 0.0,
+                        O=None, W_out=None, workspace=None, stream=None) -> Tuple:
+    """TTT-Linear mini-batch dual form. Returns (O, W_out); see include/ttt.h."""
+    return _state_call("ttt_linear_dual_fwd", "ttt_linear_dual_workspace_size", Q, K, V, eta,
+                       eta_scalar, W0, C, O, W_out, workspace, stream)
+
+
+def ttt_assoc_scan_fwd(Q, K, V, eta=None, S0=None, *, C: int, eta_scalar: float = 0.0,
+                       O=None, S_out=None, workspace=None, stream=None) -> Tuple:
+    """Associative (gradient-ascent) linear-attention mode. Returns (O, S_out)."""
+    return _state_call("ttt_assoc_scan_fwd", "ttt_assoc_scan_workspace_size", Q, K, V, eta,
+                       eta_scalar, S0, C, O, S_out, workspace, stream)
+
+
+def inplace_ttt_chunk_fwd(Z, Vhat, W0, eta: float, *, C: int, O=None, W_out=None,
+                          workspace=None, stream=None) -> Tuple:
+    """In-Place TTT W_down chunk update. Returns (O, W_out)."""
+    import torch
+
+    lib = load_library()
+    _require(Z.dim() == 2 and Vhat.dim() == 2 and W0.dim() == 2, "Z, Vhat, W0 must be 2-D")
+    T, Dff = Z.shape
+    D = Vhat.shape[1]
+    for t in (Z, Vhat, W0):
+        _require(t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16,
+                 "Z, Vhat, W0 must be contiguous bf16 CUDA tensors")
+    _require(Vhat.shape[0] == T and tuple(W0.shape) == (Dff, D), "shape mismatch")
+    if O is None:
+        O = torch.empty((T, D), device=Z.device, dtype=torch.bfloat16)
+    if W_out is None:
+        W_out = torch.empty((Dff, D), device=Z.device, dtype=torch.float32)
+    ws_bytes = lib.inplace_ttt_workspace_size(T, Dff, D, C)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, device=Z.device, dtype=torch.uint8)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.inplace_ttt_chunk_fwd(_ptr(Z), _ptr(Vhat), _ptr(W0), ctypes.c_float(eta), _ptr(O),
+                                   _ptr(W_out), T, Dff, D, C, _ptr(workspace), wsz,
+                                   _stream_ptr(stream))
+    _check("inplace_ttt_chunk_fwd", st)
+    return O, W_out
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(load_library().ttt_launch_count())
+
+
+def read_device_error() -> int:
+    """Reads and clears the device error word (synchronous)."""
+    v = ctypes.c_uint(0)
+    _check("ttt_read_device_error", load_library().ttt_read_device_error(ctypes.byref(v)))
+    return int(v.value)

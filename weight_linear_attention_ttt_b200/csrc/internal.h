@@ -1,0 +1,74 @@
+// Internal launcher interface between the C ABI (ttt_api.cu) and the kernel translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+#include <cstddef>
+#include <cstdint>
+#include <string>
+
+namespace ttt {
+
+enum Status : int { kOk = 0, kInvalid = 1, kUnsupported = 2, kWorkspace = 3, kCuda = 4 };
+
+// Arguments of one dual-form or associative call, already validated by the ABI layer.
+struct StateArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const float* eta;  // [B,H,T] or nullptr
+  float eta_scalar;
+  const float* S0;   // [B,H,d,d] fp32 or nullptr (zeros)
+  void* O;
+  float* S_out;
+  int B, H, T, d, C;
+  int dt;            // 0 = fp32, 1 = bf16
+  void* ws;
+  size_t ws_bytes;
+};
+
+struct InplaceArgs {
+  const void* Z;
+  const void* Vhat;
+  const void* W0;
+  float eta;
+  void* O;
+  float* W_out;
+  int T, Dff, D, C;
+  void* ws;
+  size_t ws_bytes;
+};
+
+// Per-launch context handed to the launchers.
+struct LaunchCtx {
+  cudaStream_t stream;
+  unsigned* err;        // device error word (bounded waits report here)
+  std::string* msg;     // detail for a non-OK status
+};
+
+void count_launch(uint64_t n = 1);
+
+// 3-D tiled tensor map (dims innermost first; strides in bytes for dims 1 and 2).
+bool make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                  const uint64_t dims[3], const uint64_t strides[2], const uint32_t box[3],
+                  CUtensorMapSwizzle swizzle, std::string* msg);
+// 2-D tiled tensor map (dims innermost first; stride of dim 1 in bytes).
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                  const uint64_t dims[2], uint64_t stride1, const uint32_t box[2],
+                  CUtensorMapSwizzle swizzle, std::string* msg);
+
+// Dual form.
+bool dual_mma_supported(int d, int C, int dt);
+int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx);
+int launch_dual_simt(const StateArgs& a, const LaunchCtx& ctx);
+
+// Associative mode.
+size_t assoc_workspace_bytes(int B, int H, int T, int d, int C);
+bool assoc_supported(int d, int C, int dt);
+int launch_assoc(const StateArgs& a, const LaunchCtx& ctx);
+
+// In-Place W_down.
+size_t inplace_workspace_bytes(int T, int Dff, int D, int C);
+bool inplace_supported(int T, int Dff, int D, int C, std::string* why);
+int launch_inplace(const InplaceArgs& a, const LaunchCtx& ctx);
+
+}  // namespace ttt

@@ -1,0 +1,269 @@
+// C ABI of libttt_b200: argument validation, dispatch, tensor-map encoding, status reporting.
+// Declarations and the contract of every entry point live in include/ttt.h.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "internal.h"
+#include "ttt.h"
+
+namespace ttt {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Device error word written by bounded waits in the kernels (one per device context).
+__device__ unsigned g_device_error;
+
+static thread_local std::string t_last_error;
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn(std::string* msg) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  if (!fn && msg) *msg = "cuTensorMapEncodeTiled entry point not available";
+  return fn;
+}
+
+bool make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                  const uint64_t dims[3], const uint64_t strides[2], const uint32_t box[3],
+                  CUtensorMapSwizzle swizzle, std::string* msg) {
+  auto fn = encode_fn(msg);
+  if (!fn) return false;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    if (msg) *msg = "cuTensorMapEncodeTiled (3-D) failed with CUresult " + std::to_string(r);
+    return false;
+  }
+  return true;
+}
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                  const uint64_t dims[2], uint64_t stride1, const uint32_t box[2],
+                  CUtensorMapSwizzle swizzle, std::string* msg) {
+  auto fn = encode_fn(msg);
+  if (!fn) return false;
+  const cuuint32_t estr[2] = {1, 1};
+  const cuuint64_t strides[1] = {stride1};
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    if (msg) *msg = "cuTensorMapEncodeTiled (2-D) failed with CUresult " + std::to_string(r);
+    return false;
+  }
+  return true;
+}
+
+static unsigned* device_error_word(std::string* msg) {
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_device_error);
+  if (e != cudaSuccess) {
+    *msg = std::string("cudaGetSymbolAddress(error word): ") + cudaGetErrorString(e);
+    return nullptr;
+  }
+  return static_cast<unsigned*>(p);
+}
+
+namespace {
+
+int fail(int status, const std::string& why) {
+  t_last_error = why;
+  return status;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || !na || !nb) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// Shared checks of the dual-form and associative entry points.
+int check_state_args(const char* fn, const StateArgs& a, size_t need_ws) {
+  const std::string f(fn);
+  if (!a.Q || !a.K || !a.V || !a.O || !a.S_out)
+    return fail(TTT_ERR_INVALID_ARG, f + ": Q, K, V, O and the output state must be non-null");
+  if (a.B <= 0 || a.H <= 0 || a.T <= 0 || a.d <= 0 || a.C <= 0)
+    return fail(TTT_ERR_INVALID_ARG, f + ": B, H, T, d and C must be positive");
+  if (a.T % a.C != 0) return fail(TTT_ERR_INVALID_ARG, f + ": T must be a multiple of C");
+  if (a.dt != TTT_DTYPE_F32 && a.dt != TTT_DTYPE_BF16)
+    return fail(TTT_ERR_INVALID_ARG, f + ": dtype must be TTT_DTYPE_F32 or TTT_DTYPE_BF16");
+  const void* ptrs[] = {a.Q, a.K, a.V, a.O, a.S_out, a.eta, a.S0};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p))
+      return fail(TTT_ERR_INVALID_ARG, f + ": every device pointer must be 16-byte aligned");
+  if ((uint64_t)a.B * a.H * a.T * a.d >= (1ull << 40))
+    return fail(TTT_ERR_UNSUPPORTED, f + ": tensor too large");
+  const size_t esz = a.dt == TTT_DTYPE_F32 ? 4 : 2;
+  const size_t nx = (size_t)a.B * a.H * a.T * a.d * esz;
+  const size_t ns = (size_t)a.B * a.H * a.d * a.d * 4;
+  const size_t ne = (size_t)a.B * a.H * a.T * 4;
+  const void* ins[] = {a.Q, a.K, a.V};
+  for (const void* p : ins)
+    if (overlap(a.O, nx, p, nx) || overlap(a.S_out, ns, p, nx))
+      return fail(TTT_ERR_INVALID_ARG, f + ": outputs must not overlap Q, K or V");
+  if (overlap(a.O, nx, a.S_out, ns) || overlap(a.O, nx, a.eta, ne) ||
+      overlap(a.S_out, ns, a.eta, ne) || overlap(a.O, nx, a.S0, ns))
+    return fail(TTT_ERR_INVALID_ARG, f + ": outputs must not overlap eta, the initial state or "
+                                         "each other");
+  if (a.S0 && a.S0 != a.S_out && overlap(a.S0, ns, a.S_out, ns))
+    return fail(TTT_ERR_INVALID_ARG,
+                f + ": the output state may equal the initial state but not partly overlap it");
+  if (need_ws && (!a.ws || a.ws_bytes < need_ws))
+    return fail(TTT_ERR_WORKSPACE,
+                f + ": workspace of at least " + std::to_string(need_ws) + " bytes required");
+  if (need_ws && !aligned16(a.ws))
+    return fail(TTT_ERR_INVALID_ARG, f + ": workspace must be 16-byte aligned");
+  return TTT_OK;
+}
+
+int finish(int st, const std::string& msg) {
+  if (st != TTT_OK) t_last_error = msg;
+  return st;
+}
+
+}  // namespace
+}  // namespace ttt
+
+using namespace ttt;
+
+extern "C" {
+
+const char* ttt_status_string(int s) {
+  switch (s) {
+    case TTT_OK: return "TTT_OK";
+    case TTT_ERR_INVALID_ARG: return "TTT_ERR_INVALID_ARG";
+    case TTT_ERR_UNSUPPORTED: return "TTT_ERR_UNSUPPORTED";
+    case TTT_ERR_WORKSPACE: return "TTT_ERR_WORKSPACE";
+    case TTT_ERR_CUDA: return "TTT_ERR_CUDA";
+    case TTT_ERR_TIMEOUT: return "TTT_ERR_TIMEOUT";
+  }
+  return "TTT_ERR_UNKNOWN";
+}
+
+const char* ttt_last_error_message(void) { return t_last_error.c_str(); }
+
+int ttt_version(void) { return 10000; }
+
+uint64_t ttt_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int ttt_read_device_error(unsigned* value) {
+  if (!value) return fail(TTT_ERR_INVALID_ARG, "ttt_read_device_error: null output");
+  unsigned v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  if (e != cudaSuccess)
+    return fail(TTT_ERR_CUDA, std::string("ttt_read_device_error: ") + cudaGetErrorString(e));
+  *value = v;
+  return TTT_OK;
+}
+
+size_t ttt_linear_dual_workspace_size(int, int, int, int, int, int) { return 0; }
+
+int ttt_linear_dual_fwd(const void* Q, const void* K, const void* V, const float* eta,
+                        float eta_scalar, const float* W0, void* O, float* W_out, int B, int H,
+                        int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+  StateArgs a{Q, K, V, eta, eta_scalar, W0, O, W_out, B, H, T, d, C, dt, workspace,
+              workspace_bytes};
+  int st = check_state_args("ttt_linear_dual_fwd", a, 0);
+  if (st != TTT_OK) return st;
+  if (!(d == 32 || d == 64 || d == 128) || C > 64)
+    return fail(TTT_ERR_UNSUPPORTED,
+                "ttt_linear_dual_fwd: supported d in {32, 64, 128} and 1 <= C <= 64");
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  st = dual_mma_supported(d, C, dt) ? launch_dual_mma(a, ctx) : launch_dual_simt(a, ctx);
+  return finish(st, msg);
+}
+
+size_t ttt_assoc_scan_workspace_size(int B, int H, int T, int d, int C, int dt) {
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || !assoc_supported(d, C, dt)) return 0;
+  return assoc_workspace_bytes(B, H, T, d, C);
+}
+
+int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float* eta,
+                       float eta_scalar, const float* S0, void* O, float* S_out, int B, int H,
+                       int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
+  StateArgs a{Q, K, V, eta, eta_scalar, S0, O, S_out, B, H, T, d, C, dt, workspace,
+              workspace_bytes};
+  int st = check_state_args("ttt_assoc_scan_fwd", a, 0);
+  if (st != TTT_OK) return st;
+  if (!assoc_supported(d, C, dt))
+    return fail(TTT_ERR_UNSUPPORTED, "ttt_assoc_scan_fwd: supported bf16, d == 128, C == 64");
+  st = check_state_args("ttt_assoc_scan_fwd", a, assoc_workspace_bytes(B, H, T, d, C));
+  if (st != TTT_OK) return st;
+  if (overlap(workspace, workspace_bytes, O, (size_t)B * H * T * d * 2) ||
+      overlap(workspace, workspace_bytes, S_out, (size_t)B * H * d * d * 4))
+    return fail(TTT_ERR_INVALID_ARG, "ttt_assoc_scan_fwd: workspace overlaps an output");
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  return finish(launch_assoc(a, ctx), msg);
+}
+
+size_t inplace_ttt_workspace_size(int T, int Dff, int D, int C) {
+  if (T <= 0 || Dff <= 0 || D <= 0 || C <= 0) return 0;
+  return inplace_workspace_bytes(T, Dff, D, C);
+}
+
+int inplace_ttt_chunk_fwd(const void* Z, const void* Vhat, const void* W0, float eta, void* O,
+                          float* W_out, int T, int Dff, int D, int C, void* workspace,
+                          size_t workspace_bytes, cudaStream_t stream) {
+  const char* f = "inplace_ttt_chunk_fwd";
+  if (!Z || !Vhat || !W0 || !O || !W_out)
+    return fail(TTT_ERR_INVALID_ARG, std::string(f) + ": Z, Vhat, W0, O, W_out must be non-null");
+  if (T <= 0 || Dff <= 0 || D <= 0 || C <= 0)
+    return fail(TTT_ERR_INVALID_ARG, std::string(f) + ": T, Dff, D and C must be positive");
+  if (T % C != 0) return fail(TTT_ERR_INVALID_ARG, std::string(f) + ": T must be a multiple of C");
+  const void* ptrs[] = {Z, Vhat, W0, O, W_out, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p))
+      return fail(TTT_ERR_INVALID_ARG, std::string(f) + ": pointers must be 16-byte aligned");
+  std::string why;
+  if (!inplace_supported(T, Dff, D, C, &why))
+    return fail(TTT_ERR_UNSUPPORTED, std::string(f) + ": " + why);
+  const size_t nz = (size_t)T * Dff * 2, nv = (size_t)T * D * 2, nw = (size_t)Dff * D * 2;
+  const size_t no = (size_t)T * D * 2, nwo = (size_t)Dff * D * 4;
+  const void* ins[] = {Z, Vhat, W0};
+  const size_t nin[] = {nz, nv, nw};
+  for (int i = 0; i < 3; ++i)
+    if (overlap(O, no, ins[i], nin[i]) || overlap(W_out, nwo, ins[i], nin[i]) ||
+        overlap(workspace, workspace_bytes, ins[i], nin[i]))
+      return fail(TTT_ERR_INVALID_ARG, std::string(f) + ": outputs/workspace overlap an input");
+  if (overlap(O, no, W_out, nwo) || overlap(workspace, workspace_bytes, O, no) ||
+      overlap(workspace, workspace_bytes, W_out, nwo))
+    return fail(TTT_ERR_INVALID_ARG, std::string(f) + ": outputs/workspace overlap");
+  const size_t need = inplace_workspace_bytes(T, Dff, D, C);
+  if (need && (!workspace || workspace_bytes < need))
+    return fail(TTT_ERR_WORKSPACE, std::string(f) + ": workspace of at least " +
+                                       std::to_string(need) + " bytes required");
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  InplaceArgs a{Z, Vhat, W0, eta, O, W_out, T, Dff, D, C, workspace, workspace_bytes};
+  return finish(launch_inplace(a, ctx), msg);
+}
+
+}  // extern "C"

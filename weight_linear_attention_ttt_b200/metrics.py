@@ -1,0 +1,44 @@
+"""Algorithmic work of each operation: the flops and bytes the method itself must compute and
+move, used for roofline fractions. Workspace, superchunk-state and re-read traffic is NOT
+counted: it is overhead a kernel has to beat.
+
+Dual form, per token and head: K_c W, Q_c W, K_c^T G (2 d^2 flops each) plus the intra-chunk
+scores Q_c K_c^T and their product with G (2 C d each): 6 d^2 + 4 C d flops. Bytes: Q, K, V in
+and O out (d elements each) plus one fp32 learning rate, and per stream the fp32 state in and out.
+
+Associative mode, per token and head: Q S and K^T V (2 d^2 each) plus the causal C x C terms
+(4 C d, counted dense): 4 d^2 + 4 C d flops; bytes as the dual form.
+
+In-Place, per token: the read Z_i W and the update Z_i^T Vhat_i, 2 Dff D flops each; bytes: Z,
+Vhat, W0 (bf16), O (bf16) and the final fp32 W once each.
+"""
+from __future__ import annotations
+
+from .inputs import Workload
+
+
+def algorithmic(w: Workload) -> dict:
+    """{'flops': F, 'bytes': B, 'tokens': N} for one call of the workload."""
+    if w.kind in ("dual", "assoc"):
+        e = 4 if w.dtype == "f32" else 2
+        th = w.B * w.H * w.T
+        per_tok = (6 if w.kind == "dual" else 4) * w.d * w.d + 4 * w.C * w.d
+        eta_bytes = 4 if w.eta != "const" else 0
+        state_bytes = 2 * w.d * w.d * 4
+        return {"flops": th * per_tok,
+                "bytes": th * (4 * w.d * e + eta_bytes) + w.B * w.H * state_bytes,
+                "tokens": w.B * w.T}
+    if w.kind == "inplace":
+        T, F, D = w.T, w.Dff, w.D
+        return {"flops": 4 * F * D * T,
+                "bytes": T * F * 2 + T * D * 2 + F * D * 2 + T * D * 2 + F * D * 4,
+                "tokens": T}
+    raise ValueError(w.kind)
+
+
+def roofline_seconds(w: Workload, hbm_gbs: float, tensor_tflops: float) -> tuple:
+    """(seconds, bound) = the slower of flops at the tensor peak and bytes at HBM bandwidth."""
+    a = algorithmic(w)
+    t_flops = a["flops"] / (tensor_tflops * 1e12)
+    t_bytes = a["bytes"] / (hbm_gbs * 1e9)
+    return (t_bytes, "hbm") if t_bytes >= t_flops else (t_flops, "tensor")
