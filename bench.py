@@ -394,10 +394,16 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--override", action="append", default=[],
+                    help="shape override of the workload for reduced profiling cases, e.g. T=8192")
     args = ap.parse_args(argv)
     from weight_linear_attention_ttt_b200 import inputs as inp
 
     w = inp.WORKLOADS[args.workload]
+    if args.override:
+        import dataclasses
+
+        w = dataclasses.replace(w, **{k: int(v) for k, v in (o.split("=") for o in args.override)})
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

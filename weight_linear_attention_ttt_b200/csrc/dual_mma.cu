@@ -7,25 +7,29 @@
 //     O_c = Q_c W - tril(Q_c K_c^T) diag(eta_c) G
 //     W   = W - K_c^T diag(eta_c) G
 //
-// Design. The chunk loop is a serial chain through W, and C = 16 tokens give a chunk too little
-// work to hide latency, so the kernel is built around the chain's latency:
-//   * the state stays in registers for the whole sequence as fp32 MMA accumulators. Columns of W
-//     are independent (W's update mixes rows only), so each compute warp owns 16 output columns
-//     and keeps W^T[cols, :] (16 x d fp32) in the accumulator layout of m16n8k16;
-//   * the accumulator layout of W^T is, packed to bf16, exactly the A-operand layout of the next
-//     chunk's products, so no shuffle or shared-memory round trip sits on the chain:
-//         P^T = W^T K_c^T          (A = W^T, from registers; B = K_c rows via ldmatrix)
-//         E^T = (P^T - V_c^T) diag(eta)
-//         W^T -= E^T K_c           (A = E^T, from registers; B = K_c via ldmatrix.trans)
-//   * the outputs (Q_c W and the causal correction tril(Q_c K_c^T) diag(eta) G) hang off the
-//     chain and overlap with it;
+// Design. The chunk loop is a serial chain through W, and a 16-token chunk is too little work to
+// hide latency, so the kernel is organised around that chain:
+//   * The state never leaves registers. Columns of W are independent (the update mixes rows
+//     only), so each compute warp owns 8 output columns and keeps W[:, cols] (d x 8, fp32) as
+//     m16n8 MMA accumulators for the whole sequence. Two compute warps share each SM sub-
+//     partition, so two chains interleave and hide each other's latency.
+//   * Per chunk and warp (E = diag(eta) G, all products on mma.sync m16n8k16, fp32 accumulate):
+//         P    = K_c W[:, cols]            A = K_c (ldmatrix), B = bf16(W) (movmatrix.trans of
+//                                          the accumulators: no shared-memory round trip)
+//         E    = diag(eta) (P - V_c[:, cols])
+//         W[:, cols] -= K_c^T E           A = K_c^T (ldmatrix.trans), B = E (movmatrix.trans)
+//         O_c[:, cols] = Q_c W[:, cols] - mask(Q_c K_c^T) E
+//     Only P -> E -> update sits on the chain; the output products hang off it.
+//   * The causal scores mask(Q_c K_c^T) do not depend on W: the warps compute them once per
+//     pipeline stage (one 16x8 piece each), negate, round to bf16 and share them through shared
+//     memory in MMA-fragment order.
 //   * Q/K/V tiles arrive by TMA (3-D tensor maps over [B*H, T, d], 128-byte swizzle) into a
 //     multi-stage mbarrier ring filled by one producer warp; outputs leave through a
-//     double-buffered shared tile and TMA stores.
-// Precision: W is fp32 throughout; its operand copy, the residual and the scores are rounded to
-// bf16 once per chunk for the tensor cores (relative error ~2^-9 per product, fp32 accumulate).
+//     double-buffered shared tile and TMA stores (rows past T are clipped by the tensor map).
+// Precision: W is fp32 throughout; its operand copy, E and the scores are rounded to bf16 once
+// per chunk for the tensor cores (relative error ~2^-9 per operand, fp32 accumulation).
 #include <algorithm>
-#include <cstdio>
+#include <cstdlib>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -33,35 +37,39 @@
 namespace ttt {
 namespace {
 
-template <int D, int NW>
+template <int D, int NW, int CPS_ = 4>
 struct DualCfg {
   static constexpr int C = 16;
-  static constexpr int CPS = 4;                    // chunks per pipeline stage
+  static constexpr int CPS = CPS_;                 // chunks per pipeline stage
   static constexpr int R = C * CPS;                // token rows per stage
   static constexpr int SUB = D >= 64 ? 64 : D;     // columns per swizzled sub-tile
   static constexpr int RB = SUB * 2;               // bytes per sub-tile row
   static constexpr int NSUB = D / SUB;
   static constexpr int SUB_BYTES = R * RB;
   static constexpr int TILE_BYTES = NSUB * SUB_BYTES;
-  static constexpr int COLS = 16 * NW;             // output columns per CTA
+  static constexpr int COLS = 8 * NW;              // output columns per CTA
   static constexpr int NG = D / COLS;              // CTAs per stream
   static constexpr int OSUB = COLS >= 64 ? 64 : COLS;
   static constexpr int ORB = OSUB * 2;
   static constexpr int NOSUB = COLS / OSUB;
   static constexpr int OSUB_BYTES = R * ORB;
   static constexpr int OTILE_BYTES = NOSUB * OSUB_BYTES;
-  static constexpr int ETA_BYTES = 1024;           // R floats, padded to keep tiles aligned
+  static constexpr int ETA_BYTES = R * 4 <= 1024 ? 1024 : 2048;  // R floats, padded
   static constexpr int STAGE_BYTES = 3 * TILE_BYTES + ETA_BYTES;
+  static constexpr int L_BYTES = CPS * 32 * 16;    // shared scores: [chunk][lane][4 x bf16x2]
   static constexpr int BUDGET = 200 * 1024;
-  static constexpr int NSTAGE_FIT = (BUDGET - 2 * OTILE_BYTES) / STAGE_BYTES;
+  static constexpr int NSTAGE_FIT = (BUDGET - 2 * OTILE_BYTES - L_BYTES) / STAGE_BYTES;
   static constexpr int NSTAGE = NSTAGE_FIT > 8 ? 8 : NSTAGE_FIT;
-  static constexpr int BAR_OFF = NSTAGE * STAGE_BYTES + 2 * OTILE_BYTES;
+  static constexpr int OUT_OFF = NSTAGE * STAGE_BYTES;
+  static constexpr int L_OFF = OUT_OFF + 2 * OTILE_BYTES;
+  static constexpr int BAR_OFF = L_OFF + L_BYTES;
   static constexpr int SMEM = 1024 + BAR_OFF + 16 * NSTAGE;
   static constexpr int THREADS = 32 * (NW + 1);
-  static constexpr int KS = D / 16;                // 16-wide k-steps over d
+  static constexpr int KS = D / 16;                // 16-wide k-steps (and m-tiles) over d
   static_assert(NSTAGE >= 2, "pipeline depth");
   static_assert(R * 4 <= ETA_BYTES, "eta slot");
   static_assert(D % COLS == 0, "column split");
+  static_assert(COLS >= 16, "TMA store box of at least 32 bytes");
 };
 
 struct DualParams {
@@ -88,15 +96,44 @@ __device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
       : "memory");
   return r != 0;
 }
+// Transpose of an 8x8 bf16 tile held as one register per lane in MMA-fragment order.
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float ld_shared_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void ld_shared_v4(uint32_t a, uint32_t (&v)[4]) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+               : "r"(a));
+}
+__device__ __forceinline__ void st_shared_v2(uint32_t a, uint32_t x, uint32_t y) {
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(a), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void stsm_x2(uint32_t addr, uint32_t r0, uint32_t r1) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x2.shared.b16 [%0], {%1, %2};" ::"r"(addr), "r"(r0),
+               "r"(r1)
+               : "memory");
+}
 
-template <int D, int NW>
-__global__ void __launch_bounds__(DualCfg<D, NW>::THREADS, 1)
+template <int D, int NW, int CPS>
+__global__ void __launch_bounds__(DualCfg<D, NW, CPS>::THREADS, 1)
     dual_mma_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmO, const DualParams p) {
-  using Cfg = DualCfg<D, NW>;
-  constexpr int R = Cfg::R, KS = Cfg::KS, NSTAGE = Cfg::NSTAGE;
+  using Cfg = DualCfg<D, NW, CPS>;
+  constexpr int R = Cfg::R, KS = Cfg::KS, NSTAGE = Cfg::NSTAGE, RB = Cfg::RB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -157,31 +194,47 @@ __global__ void __launch_bounds__(DualCfg<D, NW>::THREADS, 1)
   // ------------------------------------------------------------------ compute warps
   const int g = lane >> 2, tq = lane & 3;
   const int mi = lane >> 3, rr = lane & 7;   // ldmatrix: which 8x8 matrix / which row
-  const int colw = 16 * warp;                // column offset inside the CTA's columns
-  const int colg = col_cta + colw;           // global column of this warp's first column
+  const int colw = 8 * warp;                 // first column of this warp inside the CTA's
+  const int colg = col_cta + colw;           // ... and in the stream's W
 
-  // Per-stream state: W^T[colg .. colg+15][0 .. D-1] as m16n8 fp32 accumulators.
-  float wacc[D / 8][4];
+  // Lane-constant parts of the swizzled shared-memory addresses. A chunk starts at row 16c,
+  // a multiple of 8, so the XOR pattern of every access is the same for all chunks and the
+  // address of chunk c is this offset plus 16c rows.
+  auto off = [&](int row, int col) -> uint32_t {
+    return (col / Cfg::SUB) * Cfg::SUB_BYTES + swz<RB>(row * RB + (col % Cfg::SUB) * 2);
+  };
+  uint32_t o_arow[KS], o_atrn[KS];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    // rows of K/Q as the A operand (M = tokens, K = d): matrices (r0-7,lo) (r8-15,lo)
+    // (r0-7,hi) (r8-15,hi) give the four A registers in order.
+    o_arow[ks] = off(8 * (mi & 1) + rr, 16 * ks + 8 * (mi >> 1));
+    // K^T as the A operand (M = d, K = tokens) via ldmatrix.trans: matrices
+    // (t0-7, d lo) (t0-7, d hi) (t8-15, d lo) (t8-15, d hi).
+    o_atrn[ks] = off(8 * (mi >> 1) + rr, 16 * ks + 8 * (mi & 1));
+  }
+  const uint32_t o_v0 = off(g, colg + 2 * tq), o_v1 = off(g + 8, colg + 2 * tq);
+  const uint32_t o_st = (colw / Cfg::OSUB) * Cfg::OSUB_BYTES +
+                        swz<Cfg::ORB>((8 * (mi & 1) + rr) * Cfg::ORB + (colw % Cfg::OSUB) * 2);
+  constexpr uint32_t CHUNK_ROWS_BYTES = 16 * RB;  // 16 rows of a sub-tile
+  constexpr uint32_t CHUNK_ROWS_OBYTES = 16 * Cfg::ORB;
+  const uint32_t sL = sbase + Cfg::L_OFF;
+
+  // W[:, colg .. colg+7] as m16n8 fp32 accumulators: m-tile mt holds rows 16mt .. 16mt+15.
+  float wc[KS][4];
   {
     const float* w0 = p.W0 ? p.W0 + (size_t)stream * D * D : nullptr;
 #pragma unroll
-    for (int j = 0; j < D / 8; ++j)
+    for (int mt = 0; mt < KS; ++mt)
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int row = 8 * j + 2 * tq + e;
-        wacc[j][e] = w0 ? w0[row * D + colg + g] : 0.f;
-        wacc[j][2 + e] = w0 ? w0[row * D + colg + g + 8] : 0.f;
+      for (int h = 0; h < 2; ++h) {
+        float2 v = make_float2(0.f, 0.f);
+        if (w0) v = *reinterpret_cast<const float2*>(w0 + (16 * mt + 8 * h + g) * D + colg +
+                                                     2 * tq);
+        wc[mt][2 * h] = v.x;
+        wc[mt][2 * h + 1] = v.y;
       }
   }
-
-  auto tile = [&](uint32_t base, int row, int col) -> uint32_t {
-    return base + (col / Cfg::SUB) * Cfg::SUB_BYTES +
-           swz<Cfg::RB>(row * Cfg::RB + (col % Cfg::SUB) * 2);
-  };
-  auto otile = [&](uint32_t base, int row, int col) -> uint32_t {
-    return base + (col / Cfg::OSUB) * Cfg::OSUB_BYTES +
-           swz<Cfg::ORB>(row * Cfg::ORB + (col % Cfg::OSUB) * 2);
-  };
 
   bool ok = true;
   for (int j = 0; j < nstg; ++j) {
@@ -190,94 +243,130 @@ __global__ void __launch_bounds__(DualCfg<D, NW>::THREADS, 1)
     const uint32_t sQ = sbase + s * Cfg::STAGE_BYTES;
     const uint32_t sK = sQ + Cfg::TILE_BYTES;
     const uint32_t sV = sK + Cfg::TILE_BYTES;
-    const float* sEta = reinterpret_cast<const float*>(smem + s * Cfg::STAGE_BYTES +
-                                                       3 * Cfg::TILE_BYTES);
-    const uint32_t sO = sbase + NSTAGE * Cfg::STAGE_BYTES + (j & 1) * Cfg::OTILE_BYTES;
+    const uint32_t sEta = sQ + 3 * Cfg::TILE_BYTES;
+    const uint32_t sO = sbase + Cfg::OUT_OFF + (j & 1) * Cfg::OTILE_BYTES;
     const int chunks = got ? min(R, T - j * R) / 16 : 0;
 
-#pragma unroll 1
-    for (int c = 0; c < chunks; ++c) {
-      const int r0 = 16 * c;
-      // ---- W-independent operands of this chunk
-      uint32_t kr[KS][4], qr[KS][4];
+    // ---- causal scores of this stage: piece (chunk cc, score columns 8jj..8jj+7) per warp,
+    //      stored negated and masked as the A fragments of -mask(Q_c K_c^T).
+    for (int pc = warp; pc < 2 * chunks; pc += NW) {
+      const int cc = pc >> 1, jj = pc & 1;
+      float lc[4] = {};
+#pragma unroll
+      for (int kp = 0; kp < (KS + 1) / 2; ++kp) {
+        // B = K^T (K = d, N = score columns): rows 8jj.. of K, matrices (k lo) (k hi) of two
+        // consecutive k-steps.
+        uint32_t kb[4], qa[4];
+        ldsm_x4(sK + cc * CHUNK_ROWS_BYTES + off(8 * jj + rr, 32 * kp + 8 * mi), kb);
+        ldsm_x4(sQ + cc * CHUNK_ROWS_BYTES + o_arow[2 * kp], qa);
+        mma16816(lc, qa[0], qa[1], qa[2], qa[3], kb[0], kb[1]);
+        if (2 * kp + 1 < KS) {
+          ldsm_x4(sQ + cc * CHUNK_ROWS_BYTES + o_arow[2 * kp + 1], qa);
+          mma16816(lc, qa[0], qa[1], qa[2], qa[3], kb[2], kb[3]);
+        }
+      }
+      // keep s <= t: s = 8jj + 2tq + e, t = g (+8)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (8 * jj + 2 * tq + (i & 1) > g + 8 * (i >> 1)) lc[i] = 0.f;
+      st_shared_v2(sL + cc * 512 + lane * 16 + jj * 8, pack_bf16(-lc[0], -lc[1]),
+                   pack_bf16(-lc[2], -lc[3]));
+    }
+    named_bar_sync(1, 32 * NW);
+
+    // Per chunk: operand loads, the chain, then the outputs. A warp issues in order and shared
+    // stores may alias later shared loads, so in a full stage the loads of chunk c+1 are placed
+    // in program order between chunk c's chain and its outputs: they then overlap chunk c's
+    // output products. A partial last stage runs the plain rolled loop.
+    struct Ops {
+      uint32_t ka[KS][4], kt[KS][4], qa[KS][4], la[4], v0, v1;
+      float eg, eg8;
+    };
+    auto load = [&](Ops& o, const int c) {
+      const uint32_t cb = c * CHUNK_ROWS_BYTES;
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        const int row = r0 + 8 * (mi >> 1) + rr, col = 16 * ks + 8 * (mi & 1);
-        ldsm_x4(tile(sK, row, col), kr[ks]);
-        ldsm_x4(tile(sQ, row, col), qr[ks]);
+        ldsm_x4(sK + cb + o_arow[ks], o.ka[ks]);
+        ldsm_x4_t(sK + cb + o_atrn[ks], o.kt[ks]);
       }
-      uint32_t vt[4];
-      ldsm_x4_t(tile(sV, r0 + 8 * (mi >> 1) + rr, colg + 8 * (mi & 1)), vt);
-      float e0, e1, e8, e9;  // eta of tokens 2tq, 2tq+1, 8+2tq, 9+2tq of the chunk
+      o.v0 = ld_shared_u32(sV + cb + o_v0);
+      o.v1 = ld_shared_u32(sV + cb + o_v1);
       if (p.eta) {
-        const float2 a = *reinterpret_cast<const float2*>(sEta + r0 + 2 * tq);
-        const float2 b = *reinterpret_cast<const float2*>(sEta + r0 + 8 + 2 * tq);
-        e0 = a.x; e1 = a.y; e8 = b.x; e9 = b.y;
+        o.eg = ld_shared_f32(sEta + 4 * (16 * c + g));
+        o.eg8 = ld_shared_f32(sEta + 4 * (16 * c + g + 8));
       } else {
-        e0 = e1 = e8 = e9 = p.eta_scalar;
+        o.eg = o.eg8 = p.eta_scalar;
       }
-
-      // ---- chain: W^T (bf16) -> P^T = W^T K^T -> E^T -> W^T -= E^T K
-      uint32_t wa[KS][4];
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) ldsm_x4(sQ + cb + o_arow[ks], o.qa[ks]);
+      ld_shared_v4(sL + c * 512 + lane * 16, o.la);
+    };
+    // chain: bf16(W) -> P = K W -> E -> W -= K^T E; returns bf16(W) and E as B fragments.
+    auto chain = [&](const Ops& o, uint32_t (&wb)[KS][2], uint32_t& eb0, uint32_t& eb1) {
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        wa[ks][0] = pack_bf16(wacc[2 * ks][0], wacc[2 * ks][1]);
-        wa[ks][1] = pack_bf16(wacc[2 * ks][2], wacc[2 * ks][3]);
-        wa[ks][2] = pack_bf16(wacc[2 * ks + 1][0], wacc[2 * ks + 1][1]);
-        wa[ks][3] = pack_bf16(wacc[2 * ks + 1][2], wacc[2 * ks + 1][3]);
+        wb[ks][0] = movm_t(pack_bf16(wc[ks][0], wc[ks][1]));
+        wb[ks][1] = movm_t(pack_bf16(wc[ks][2], wc[ks][3]));
       }
-      float pt[2][4] = {};
+      float pa[4] = {}, pb[4] = {};
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        mma16816(pt[0], wa[ks][0], wa[ks][1], wa[ks][2], wa[ks][3], kr[ks][0], kr[ks][1]);
-        mma16816(pt[1], wa[ks][0], wa[ks][1], wa[ks][2], wa[ks][3], kr[ks][2], kr[ks][3]);
+        if (ks & 1)
+          mma16816(pb, o.ka[ks][0], o.ka[ks][1], o.ka[ks][2], o.ka[ks][3], wb[ks][0], wb[ks][1]);
+        else
+          mma16816(pa, o.ka[ks][0], o.ka[ks][1], o.ka[ks][2], o.ka[ks][3], wb[ks][0], wb[ks][1]);
       }
-      uint32_t ea[4];
-      ea[0] = pack_bf16((pt[0][0] - bf16_lo(vt[0])) * e0, (pt[0][1] - bf16_hi(vt[0])) * e1);
-      ea[1] = pack_bf16((pt[0][2] - bf16_lo(vt[1])) * e0, (pt[0][3] - bf16_hi(vt[1])) * e1);
-      ea[2] = pack_bf16((pt[1][0] - bf16_lo(vt[2])) * e8, (pt[1][1] - bf16_hi(vt[2])) * e9);
-      ea[3] = pack_bf16((pt[1][2] - bf16_lo(vt[3])) * e8, (pt[1][3] - bf16_hi(vt[3])) * e9);
-      const uint32_t na0 = ea[0] ^ 0x80008000u, na1 = ea[1] ^ 0x80008000u;
-      const uint32_t na2 = ea[2] ^ 0x80008000u, na3 = ea[3] ^ 0x80008000u;
+      const float e0 = (pa[0] + pb[0] - bf16_lo(o.v0)) * o.eg;
+      const float e1 = (pa[1] + pb[1] - bf16_hi(o.v0)) * o.eg;
+      const float e2 = (pa[2] + pb[2] - bf16_lo(o.v1)) * o.eg8;
+      const float e3 = (pa[3] + pb[3] - bf16_hi(o.v1)) * o.eg8;
+      eb0 = movm_t(pack_bf16(e0, e1));  // B fragment: E tokens 0-7
+      eb1 = movm_t(pack_bf16(e2, e3));  // B fragment: E tokens 8-15
 #pragma unroll
-      for (int jp = 0; jp < KS; ++jp) {
-        uint32_t kt[4];
-        ldsm_x4_t(tile(sK, r0 + 8 * (mi & 1) + rr, 16 * jp + 8 * (mi >> 1)), kt);
-        mma16816(wacc[2 * jp], na0, na1, na2, na3, kt[0], kt[1]);
-        mma16816(wacc[2 * jp + 1], na0, na1, na2, na3, kt[2], kt[3]);
-      }
-
-      // ---- outputs: O = Q W (chunk-start W) - mask(Q K^T) diag(eta) G
-      float lc[2][4] = {};
+      for (int mt = 0; mt < KS; ++mt)
+        mma16816(wc[mt], o.kt[mt][0], o.kt[mt][1], o.kt[mt][2], o.kt[mt][3], eb0 ^ 0x80008000u,
+                 eb1 ^ 0x80008000u);
+    };
+    // outputs: O = Q W - mask(Q K^T) E   (W is the chunk-start state)
+    auto output = [&](const Ops& o, const int c, const uint32_t (&wb)[KS][2], uint32_t eb0,
+                      uint32_t eb1) {
+      float oa[4] = {}, ob[4] = {};
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        mma16816(lc[0], qr[ks][0], qr[ks][2], qr[ks][1], qr[ks][3], kr[ks][0], kr[ks][1]);
-        mma16816(lc[1], qr[ks][0], qr[ks][2], qr[ks][1], qr[ks][3], kr[ks][2], kr[ks][3]);
+        if (ks & 1)
+          mma16816(ob, o.qa[ks][0], o.qa[ks][1], o.qa[ks][2], o.qa[ks][3], wb[ks][0], wb[ks][1]);
+        else
+          mma16816(oa, o.qa[ks][0], o.qa[ks][1], o.qa[ks][2], o.qa[ks][3], wb[ks][0], wb[ks][1]);
       }
+      mma16816(oa, o.la[0], o.la[1], o.la[2], o.la[3], eb0, eb1);
+      stsm_x2(sO + c * CHUNK_ROWS_OBYTES + o_st, pack_bf16(oa[0] + ob[0], oa[1] + ob[1]),
+              pack_bf16(oa[2] + ob[2], oa[3] + ob[3]));
+    };
+    if (chunks == Cfg::CPS) {
+      Ops ops[2];
+      load(ops[0], 0);
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (8 * jj + 2 * tq + (i & 1) > g + 8 * (i >> 1)) lc[jj][i] = 0.f;
-      const uint32_t la0 = pack_bf16(-lc[0][0], -lc[0][1]), la1 = pack_bf16(-lc[0][2], -lc[0][3]);
-      const uint32_t la2 = pack_bf16(-lc[1][0], -lc[1][1]), la3 = pack_bf16(-lc[1][2], -lc[1][3]);
-      float o[2][4] = {};
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        mma16816(o[0], qr[ks][0], qr[ks][2], qr[ks][1], qr[ks][3], wa[ks][0], wa[ks][2]);
-        mma16816(o[1], qr[ks][0], qr[ks][2], qr[ks][1], qr[ks][3], wa[ks][1], wa[ks][3]);
+      for (int c = 0; c < Cfg::CPS; ++c) {
+        uint32_t wb[KS][2], eb0, eb1;
+        chain(ops[c & 1], wb, eb0, eb1);
+        if (c + 1 < Cfg::CPS) load(ops[(c + 1) & 1], c + 1);
+        output(ops[c & 1], c, wb, eb0, eb1);
       }
-      mma16816(o[0], la0, la1, la2, la3, ea[0], ea[2]);
-      mma16816(o[1], la0, la1, la2, la3, ea[1], ea[3]);
-      stsm_x4(otile(sO, r0 + 8 * (mi & 1) + rr, colw + 8 * (mi >> 1)),
-              pack_bf16(o[0][0], o[0][1]), pack_bf16(o[0][2], o[0][3]),
-              pack_bf16(o[1][0], o[1][1]), pack_bf16(o[1][2], o[1][3]));
+    } else {
+#pragma unroll 1
+      for (int c = 0; c < chunks; ++c) {
+        Ops o;
+        uint32_t wb[KS][2], eb0, eb1;
+        load(o, c);
+        chain(o, wb, eb0, eb1);
+        output(o, c, wb, eb0, eb1);
+      }
     }
 
     // Inputs of this stage are consumed; hand the slot back to the producer.
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar + 8 * s);
-    // Output tile -> global (TMA store, rows past T are clipped by the tensor map).
+    // Output tile -> global (TMA store).
     fence_proxy_async_smem();
     const bool failed = named_bar_or(1, 32 * NW, !got);
     if (!failed && threadIdx.x == 0) {
@@ -296,21 +385,19 @@ __global__ void __launch_bounds__(DualCfg<D, NW>::THREADS, 1)
   if (threadIdx.x == 0) bulk_wait<0>();
   if (!ok) return;
 
-  // Final state W[:, colg..colg+15].
+  // Final state W[:, colg .. colg+7].
   float* wo = p.Wout + (size_t)stream * D * D;
 #pragma unroll
-  for (int j = 0; j < D / 8; ++j)
+  for (int mt = 0; mt < KS; ++mt)
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int row = 8 * j + 2 * tq + e;
-      wo[row * D + colg + g] = wacc[j][e];
-      wo[row * D + colg + g + 8] = wacc[j][2 + e];
-    }
+    for (int h = 0; h < 2; ++h)
+      *reinterpret_cast<float2*>(wo + (16 * mt + 8 * h + g) * D + colg + 2 * tq) =
+          make_float2(wc[mt][2 * h], wc[mt][2 * h + 1]);
 }
 
-template <int D, int NW>
+template <int D, int NW, int CPS = 4>
 int launch_cfg(const StateArgs& a, const LaunchCtx& ctx) {
-  using Cfg = DualCfg<D, NW>;
+  using Cfg = DualCfg<D, NW, CPS>;
   const int BH = a.B * a.H;
   CUtensorMap tq, tk, tv, to;
   const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.T, (uint64_t)BH};
@@ -327,7 +414,7 @@ int launch_cfg(const StateArgs& a, const LaunchCtx& ctx) {
       !make_tmap_3d(&tv, a.V, bf, dims, strides, box_in, sw(Cfg::RB), ctx.msg) ||
       !make_tmap_3d(&to, a.O, bf, dims, strides, box_out, sw(Cfg::ORB), ctx.msg))
     return kCuda;
-  auto kern = dual_mma_kernel<D, NW>;
+  auto kern = dual_mma_kernel<D, NW, CPS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::SMEM);
   if (e != cudaSuccess) {
@@ -345,17 +432,17 @@ int launch_cfg(const StateArgs& a, const LaunchCtx& ctx) {
   return kOk;
 }
 
-// Column groups per stream: fewer streams than SMs leave SMs idle, and splitting the
-// (independent) columns of W over two CTAs doubles the number of chains in flight.
-int column_split(int streams, int d) {
-  const char* env = getenv("TTT_DUAL_COLUMN_SPLIT");  // tuning override: 1, 2 or 4
+// CTAs per stream. Each CTA holds one stream's column slice for the whole sequence, and one CTA
+// fits per SM, so a stream is split over two SMs (halving each SM's share of the serial chain's
+// MMA work) only when all CTAs still fit in one wave.
+int column_split(int streams) {
+  const char* env = getenv("TTT_DUAL_COLUMN_SPLIT");  // tuning override: 1 or 2
   const int forced = env ? atoi(env) : 0;
-  if (forced == 1 || forced == 2 || forced == 4) return std::min(forced, d / 16);
+  if (forced == 1 || forced == 2) return forced;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (d >= 64 && streams < sms) return 2;
-  return 1;
+  return 2 * streams <= sms ? 2 : 1;
 }
 
 }  // namespace
@@ -365,14 +452,20 @@ bool dual_mma_supported(int d, int C, int dt) {
 }
 
 int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
-  const int split = column_split(a.B * a.H, a.d);
+  const int split = column_split(a.B * a.H);
   switch (a.d) {
     case 32:
-      return launch_cfg<32, 2>(a, ctx);
-    case 64:
-      return split >= 2 ? launch_cfg<64, 2>(a, ctx) : launch_cfg<64, 4>(a, ctx);
+      return split == 2 ? launch_cfg<32, 2>(a, ctx) : launch_cfg<32, 4>(a, ctx);
+    case 64: {
+      // 8 chunks per pipeline stage halve the per-stage costs (score pieces, barriers, first
+      // loads); measured faster on the 125M- and 1.3B-layer shapes. 4 is kept as an override.
+      const char* env = getenv("TTT_DUAL_STAGE_CHUNKS");  // tuning override: 4 or 8
+      if (env && atoi(env) == 4)
+        return split == 2 ? launch_cfg<64, 4>(a, ctx) : launch_cfg<64, 8>(a, ctx);
+      return split == 2 ? launch_cfg<64, 4, 8>(a, ctx) : launch_cfg<64, 8, 8>(a, ctx);
+    }
     case 128:
-      return split >= 2 ? launch_cfg<128, 4>(a, ctx) : launch_cfg<128, 8>(a, ctx);
+      return split == 2 ? launch_cfg<128, 8>(a, ctx) : launch_cfg<128, 16>(a, ctx);
   }
   *ctx.msg = "dual_mma: unsupported head dim";
   return kUnsupported;
