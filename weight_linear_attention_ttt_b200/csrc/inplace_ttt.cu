@@ -1,14 +1,382 @@
-// In-Place TTT W_down chunk update.
+// In-Place TTT W_down chunk update on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Source: "In-Place Test-Time Training" (aitrends.kr): W_down of the gated MLP is the fast
+// weight; the sequence is cut into chunks; each chunk takes one gradient step on W_down, and the
+// updated weight serves the next chunk; per-chunk deltas combine by a prefix sum.
+//     W = W0;  for chunk i:  O_i = Z_i W;  W = W + eta Z_i^T Vhat_i
+//
+// Design. Within chunk i the read O_i = Z_i W_(i-1) and the update W_i = W_(i-1) + eta Z_i^T
+// Vhat_i are independent, so one persistent kernel per chunk runs both as tiles of one tile
+// list: 128x256 read tiles (K = Dff) and 128x256 update tiles (K = C). Read tiles are long, so
+// they are scheduled first, and every CTA takes the next tile from a global atomic counter.
+// The fp32 master W lives in W_out; the tensor cores read a bf16 copy of W, kept in a
+// double-buffered workspace (the update of chunk i writes copy i % 2 while the read of chunk i
+// still reads copy (i-1) % 2; chunk 0 reads the bf16 W0 input directly).
+// Warp roles per CTA: warp 0 issues TMA loads into a 4-stage shared-memory ring and fetches
+// tiles from the counter; warp 1 owns TMEM and issues tcgen05.mma from one thread into one of
+// two TMEM accumulators; warps 2-5 drain the other accumulator: bf16 O for read tiles,
+// W_out = W + eta * acc (fp32) and its bf16 copy for update tiles.
+#include <algorithm>
+
 #include "internal.h"
+#include "ptx.cuh"
+#include "umma.cuh"
 
 namespace ttt {
-size_t inplace_workspace_bytes(int, int, int, int) { return 0; }
-bool inplace_supported(int, int, int, int, std::string* why) {
-  *why = "not built yet";
-  return false;
+namespace {
+
+constexpr int BM = 128;     // tile rows (tokens for read tiles, Dff rows for update tiles)
+constexpr int BK = 64;      // K per pipeline stage
+constexpr int STAGES = 4;
+constexpr int THREADS = 192;
+
+template <int BN>
+struct IpCfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BK * BN * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int SMEM = 1024 + BAR_OFF + 256;
+  static constexpr int TMEM_COLS = 2 * BN;
+};
+
+struct IpParams {
+  const __nv_bfloat16* W0;   // [Dff, D] bf16 (source of chunk 0's update)
+  float* Wout;               // [Dff, D] fp32 running master
+  __nv_bfloat16* Wbf_next;   // [Dff, D] bf16 copy written by this chunk's update (or null)
+  __nv_bfloat16* O;          // [T, D]
+  float eta;
+  int first;                 // chunk 0: the update reads W0
+  int tok0;                  // first token of the chunk
+  int C, Dff, D;
+  int n_read, n_total;       // read tiles come first in the tile list
+  int* counter;
+  unsigned* err;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(THREADS, 1)
+    inplace_chunk_kernel(const __grid_constant__ CUtensorMap tmZk,   // Z, box 64 x 128
+                         const __grid_constant__ CUtensorMap tmZm,   // Z, box 64 x 64
+                         const __grid_constant__ CUtensorMap tmW,    // bf16 W read source
+                         const __grid_constant__ CUtensorMap tmV,    // Vhat, box 64 x 64
+                         const IpParams p) {
+  using Cfg = IpCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar = sbase + Cfg::BAR_OFF;
+  const uint32_t full = bar, empty = bar + 8 * STAGES;
+  const uint32_t tfull = bar + 16 * STAGES, tempty = tfull + 16;
+  const uint32_t sfull = tempty + 16, sempty = sfull + 16;
+  const uint32_t tslot = sempty + 16;                  // TMEM base address
+  volatile int* sched = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + 16 * STAGES + 80);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntn = p.D / BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + 8 * s, 1);
+      mbar_init(empty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull + 8 * b, 1);
+      mbar_init(tempty + 8 * b, 4);
+      mbar_init(sfull + 8 * b, 1);
+      mbar_init(sempty + 8 * b, 5);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) umma::tmem_alloc(tslot, Cfg::TMEM_COLS);
+  umma::fence_before();
+  __syncthreads();
+  umma::fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Cfg::BAR_OFF + 16 * STAGES +
+                                                              64);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ scheduler + TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmZk);
+      prefetch_tmap(&tmZm);
+      prefetch_tmap(&tmW);
+      prefetch_tmap(&tmV);
+      uint32_t kbt = 0;
+      for (int j = 0;; ++j) {
+        const int slot = j & 1;
+        if (j >= 2 && !mbar_wait(sempty + 8 * slot, ((j >> 1) - 1) & 1, p.err)) break;
+        const int t = atomicAdd(p.counter, 1);
+        sched[slot] = t;
+        mbar_arrive(sfull + 8 * slot);
+        if (t >= p.n_total) break;
+        const bool rd = t < p.n_read;
+        const int u = rd ? t : t - p.n_read;
+        const int mt = u / ntn, nt = u % ntn;
+        const int nkb = rd ? p.Dff / BK : p.C / BK;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb, ++kbt) {
+          const int s = kbt % STAGES;
+          if (kbt >= STAGES && !mbar_wait(empty + 8 * s, ((kbt / STAGES) - 1) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full + 8 * s;
+          const uint32_t sA = sbase + s * Cfg::STAGE_BYTES, sB = sA + Cfg::A_BYTES;
+          mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
+          if (rd) {
+            tma_load_2d(sA, &tmZk, fb, kb * BK, p.tok0 + BM * mt);
+#pragma unroll
+            for (int nb = 0; nb < BN / 64; ++nb)
+              tma_load_2d(sB + nb * 8192, &tmW, fb, BN * nt + 64 * nb, kb * BK);
+          } else {
+#pragma unroll
+            for (int mb = 0; mb < 2; ++mb)
+              tma_load_2d(sA + mb * 8192, &tmZm, fb, BM * mt + 64 * mb, p.tok0 + kb * BK);
+#pragma unroll
+            for (int nb = 0; nb < BN / 64; ++nb)
+              tma_load_2d(sB + nb * 8192, &tmV, fb, BN * nt + 64 * nb, p.tok0 + kb * BK);
+          }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (one thread)
+    if (lane == 0) {
+      const uint32_t idesc_rd = umma::idesc_bf16(BM, BN, false, true);
+      const uint32_t idesc_up = umma::idesc_bf16(BM, BN, true, true);
+      uint32_t kbt = 0;
+      for (int j = 0;; ++j) {
+        const int slot = j & 1;
+        if (!mbar_wait(sfull + 8 * slot, (j >> 1) & 1, p.err)) break;
+        const int t = sched[slot];
+        mbar_arrive(sempty + 8 * slot);
+        if (t >= p.n_total) break;
+        const bool rd = t < p.n_read;
+        const int nkb = rd ? p.Dff / BK : p.C / BK;
+        const int b = j & 1;
+        if (j >= 2 && !mbar_wait(tempty + 8 * b, ((j >> 1) - 1) & 1, p.err)) break;
+        umma::fence_after();
+        const uint32_t dt = tmem + b * BN;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb, ++kbt) {
+          const int s = kbt % STAGES;
+          if (!mbar_wait(full + 8 * s, (kbt / STAGES) & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          umma::fence_after();
+          const uint32_t sA = sbase + s * Cfg::STAGE_BYTES, sB = sA + Cfg::A_BYTES;
+#pragma unroll
+          for (int ks = 0; ks < BK / 16; ++ks) {
+            const uint64_t ad = rd ? umma::desc_kmajor(sA + 32 * ks)
+                                   : umma::desc_mnmajor(sA + 2048 * ks, 8192);
+            const uint64_t bd = umma::desc_mnmajor(sB + 2048 * ks, 8192);
+            umma::mma_ss(dt, ad, bd, rd ? idesc_rd : idesc_up, kb > 0 || ks > 0);
+          }
+          umma::commit(empty + 8 * s);
+        }
+        if (!ok) break;
+        umma::commit(tfull + 8 * b);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue warps 2..5
+    const int q = warp & 3;  // TMEM subpartition this warp may read
+    const int row = 32 * q + lane;
+    for (int j = 0;; ++j) {
+      const int slot = j & 1;
+      if (!mbar_wait(sfull + 8 * slot, (j >> 1) & 1, p.err)) break;
+      const int t = sched[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sempty + 8 * slot);
+      if (t >= p.n_total) break;
+      const bool rd = t < p.n_read;
+      const int u = rd ? t : t - p.n_read;
+      const int mt = u / ntn, nt = u % ntn;
+      const int b = j & 1;
+      if (!mbar_wait(tfull + 8 * b, (j >> 1) & 1, p.err)) break;
+      umma::fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t r[32];
+        umma::ld32x32(tmem + ((uint32_t)(32 * q) << 16) + b * BN + 32 * cc, r);
+        umma::wait_ld();
+        const int col = BN * nt + 32 * cc;
+        if (rd) {
+          uint4* dst = reinterpret_cast<uint4*>(p.O + (size_t)(p.tok0 + BM * mt + row) * p.D +
+                                                col);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            dst[v] = make_uint4(pack_bf16(__uint_as_float(r[8 * v]), __uint_as_float(r[8 * v + 1])),
+                                pack_bf16(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+                                pack_bf16(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+                                pack_bf16(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+        } else {
+          const size_t off = (size_t)(BM * mt + row) * p.D + col;
+          float w[32];
+          if (p.first) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.W0 + off);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint4 x = src[v];
+              const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                w[8 * v + 2 * e] = bf16_lo(xs[e]);
+                w[8 * v + 2 * e + 1] = bf16_hi(xs[e]);
+              }
+            }
+          } else {
+            const float4* src = reinterpret_cast<const float4*>(p.Wout + off);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float4 x = src[v];
+              w[4 * v] = x.x;
+              w[4 * v + 1] = x.y;
+              w[4 * v + 2] = x.z;
+              w[4 * v + 3] = x.w;
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) w[e] = fmaf(p.eta, __uint_as_float(r[e]), w[e]);
+          float4* dst = reinterpret_cast<float4*>(p.Wout + off);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          if (p.Wbf_next) {
+            uint4* db = reinterpret_cast<uint4*>(p.Wbf_next + off);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              db[v] = make_uint4(pack_bf16(w[8 * v], w[8 * v + 1]), pack_bf16(w[8 * v + 2], w[8 * v + 3]),
+                                 pack_bf16(w[8 * v + 4], w[8 * v + 5]),
+                                 pack_bf16(w[8 * v + 6], w[8 * v + 7]));
+          }
+        }
+      }
+      umma::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + 8 * b);
+    }
+  }
+  umma::fence_before();
+  __syncthreads();
+  if (warp == 1) umma::tmem_dealloc(tmem, Cfg::TMEM_COLS);
 }
-int launch_inplace(const InplaceArgs&, const LaunchCtx& ctx) {
-  *ctx.msg = "inplace_ttt_chunk_fwd: not built yet";
-  return kUnsupported;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int pick_bn(int D) { return D % 256 == 0 ? 256 : (D % 128 == 0 ? 128 : 64); }
+
+template <int BN>
+int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
+  using Cfg = IpCfg<BN>;
+  const int n = a.T / a.C;
+  const size_t wbf_bytes = (size_t)a.Dff * a.D * 2;
+  __nv_bfloat16* wbf[2] = {nullptr, nullptr};
+  int* counters = nullptr;
+  if (n > 1) {
+    wbf[0] = reinterpret_cast<__nv_bfloat16*>(a.ws);
+    wbf[1] = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(a.ws) + align256(wbf_bytes));
+    counters = reinterpret_cast<int*>(static_cast<uint8_t*>(a.ws) + 2 * align256(wbf_bytes));
+  } else {
+    counters = reinterpret_cast<int*>(a.ws);
+  }
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  CUtensorMap tzk, tzm, tv, tw0, tw[2];
+  {
+    const uint64_t dz[2] = {(uint64_t)a.Dff, (uint64_t)a.T};
+    const uint32_t bk[2] = {64, 128}, bm[2] = {64, 64};
+    const uint64_t dv[2] = {(uint64_t)a.D, (uint64_t)a.T};
+    const uint64_t dw[2] = {(uint64_t)a.D, (uint64_t)a.Dff};
+    if (!make_tmap_2d(&tzk, a.Z, bf, dz, (uint64_t)a.Dff * 2, bk, sw, ctx.msg) ||
+        !make_tmap_2d(&tzm, a.Z, bf, dz, (uint64_t)a.Dff * 2, bm, sw, ctx.msg) ||
+        !make_tmap_2d(&tv, a.Vhat, bf, dv, (uint64_t)a.D * 2, bm, sw, ctx.msg) ||
+        !make_tmap_2d(&tw0, a.W0, bf, dw, (uint64_t)a.D * 2, bm, sw, ctx.msg))
+      return kCuda;
+    for (int b = 0; b < 2; ++b)
+      if (wbf[b] && !make_tmap_2d(&tw[b], wbf[b], bf, dw, (uint64_t)a.D * 2, bm, sw, ctx.msg))
+        return kCuda;
+  }
+  auto kern = inplace_chunk_kernel<BN>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+  if (e == cudaSuccess) e = cudaMemsetAsync(counters, 0, sizeof(int) * n, ctx.stream);
+  if (e != cudaSuccess) {
+    *ctx.msg = std::string("inplace setup: ") + cudaGetErrorString(e);
+    return kCuda;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int ntn = a.D / BN;
+  const int n_read = (a.C / BM) * ntn, n_up = (a.Dff / BM) * ntn;
+  const int grid = std::min(sms, n_read + n_up);
+  for (int i = 0; i < n; ++i) {
+    IpParams p;
+    p.W0 = static_cast<const __nv_bfloat16*>(a.W0);
+    p.Wout = a.W_out;
+    p.Wbf_next = (i + 1 < n) ? wbf[i & 1] : nullptr;
+    p.O = static_cast<__nv_bfloat16*>(a.O);
+    p.eta = a.eta;
+    p.first = i == 0;
+    p.tok0 = i * a.C;
+    p.C = a.C;
+    p.Dff = a.Dff;
+    p.D = a.D;
+    p.n_read = n_read;
+    p.n_total = n_read + n_up;
+    p.counter = counters + i;
+    p.err = ctx.err;
+    const CUtensorMap& wsrc = i == 0 ? tw0 : tw[(i - 1) & 1];
+    kern<<<grid, THREADS, Cfg::SMEM, ctx.stream>>>(tzk, tzm, wsrc, tv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      *ctx.msg = std::string("inplace launch: ") + cudaGetErrorString(e);
+      return kCuda;
+    }
+    count_launch();
+  }
+  return kOk;
 }
+
+}  // namespace
+
+size_t inplace_workspace_bytes(int T, int Dff, int D, int C) {
+  const int n = T / C;
+  const size_t counters = align256(sizeof(int) * (size_t)std::max(n, 1));
+  if (n <= 1) return counters;
+  return 2 * align256((size_t)Dff * D * 2) + counters;
+}
+
+bool inplace_supported(int T, int Dff, int D, int C, std::string* why) {
+  if (C % BM != 0) {
+    *why = "C must be a multiple of 128";
+    return false;
+  }
+  if (Dff % BM != 0) {
+    *why = "Dff must be a multiple of 128";
+    return false;
+  }
+  if (D % 64 != 0) {
+    *why = "D must be a multiple of 64";
+    return false;
+  }
+  if ((long long)T * Dff >= (1ll << 40) || T / C > (1 << 20)) {
+    *why = "too large";
+    return false;
+  }
+  return true;
+}
+
+int launch_inplace(const InplaceArgs& a, const LaunchCtx& ctx) {
+  switch (pick_bn(a.D)) {
+    case 256: return launch_bn<256>(a, ctx);
+    case 128: return launch_bn<128>(a, ctx);
+    default: return launch_bn<64>(a, ctx);
+  }
+}
+
 }  // namespace ttt
