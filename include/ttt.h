@@ -137,6 +137,33 @@ int inplace_ttt_chunk_fwd(const void* Z, const void* Vhat, const void* W0, float
                           float* W_out, int T, int Dff, int D, int C, void* workspace,
                           size_t workspace_bytes, cudaStream_t stream);
 
+/* --------------------------------------------------------------------------------------------
+ * Allocation-free In-Place W_down update. The pages have no counterpart: this is an interface
+ * for callers that cannot provide a workspace, such as host runtimes that plan all device
+ * memory up front and refuse allocations while serving, or plugin interfaces that pass only
+ * input and output pointers.
+ *
+ *  Same computation, arguments and validation as inplace_ttt_chunk_fwd, minus the workspace:
+ *  the scratch (two bf16 copies of W_down and one tile counter per chunk) is a static device
+ *  array of inplace_ttt_noalloc_max_scratch_bytes() bytes (32 MiB) inside the library. Every
+ *  GPU that loads the library holds that array until the process exits.
+ *  - Calls allocate nothing: no cudaMalloc, no cudaFree, no allocating library routine. The
+ *    caller still provides Z, Vhat, W0, O and W_out.
+ *  - Shapes whose scratch (inplace_ttt_workspace_size) exceeds the maximum return
+ *    TTT_ERR_UNSUPPORTED before anything is launched, with the reason in
+ *    ttt_last_error_message(). With T > C the need is about 4 * Dff * D bytes.
+ *  - All calls share the one array and it keeps the previous call's contents; the tile counters
+ *    are zeroed on `stream` at the start of every call, and the W copies are always written
+ *    before they are read. Calls whose work overlaps on the GPU (different streams, or threads
+ *    racing on one device) race on the array: serialise them.
+ *  - The first call on each device looks up the array's device address (a one-time runtime
+ *    query for the current device). Make that first call before any stream capture begins.
+ * ------------------------------------------------------------------------------------------ */
+size_t inplace_ttt_noalloc_max_scratch_bytes(void);
+int inplace_ttt_chunk_fwd_noalloc(const void* Z, const void* Vhat, const void* W0, float eta,
+                                  void* O, float* W_out, int T, int Dff, int D, int C,
+                                  cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

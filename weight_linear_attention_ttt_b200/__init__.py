@@ -26,6 +26,7 @@ EXPORTED_SYMBOLS = (
     "ttt_linear_dual_workspace_size", "ttt_linear_dual_fwd",
     "ttt_assoc_scan_workspace_size", "ttt_assoc_scan_fwd",
     "inplace_ttt_workspace_size", "inplace_ttt_chunk_fwd",
+    "inplace_ttt_noalloc_max_scratch_bytes", "inplace_ttt_chunk_fwd_noalloc",
 )
 
 _LIB: Optional[ctypes.CDLL] = None
@@ -73,6 +74,11 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.inplace_ttt_chunk_fwd.restype = c_int
     lib.inplace_ttt_chunk_fwd.argtypes = [vp, vp, vp, c_float, vp, fp, c_int, c_int, c_int,
                                           c_int, vp, c_size, vp]
+    lib.inplace_ttt_noalloc_max_scratch_bytes.restype = c_size
+    lib.inplace_ttt_noalloc_max_scratch_bytes.argtypes = []
+    lib.inplace_ttt_chunk_fwd_noalloc.restype = c_int
+    lib.inplace_ttt_chunk_fwd_noalloc.argtypes = [vp, vp, vp, c_float, vp, fp, c_int, c_int,
+                                                  c_int, c_int, vp]
     if path is None:
         _LIB = lib
     return lib
@@ -180,6 +186,33 @@ def inplace_ttt_chunk_fwd(Z, Vhat, W0, eta: float, *, C: int, O=None, W_out=None
                                    _ptr(W_out), T, Dff, D, C, _ptr(workspace), wsz,
                                    _stream_ptr(stream))
     _check("inplace_ttt_chunk_fwd", st)
+    return O, W_out
+
+
+def inplace_ttt_chunk_fwd_noalloc(Z, Vhat, W0, eta: float, *, C: int, O=None, W_out=None,
+                                  stream=None) -> Tuple:
+    """In-Place W_down update through the library's allocation-free entry point: the C call
+    takes no workspace (its scratch is a fixed static device array shared by all calls), for
+    callers that cannot allocate device memory. Missing outputs are allocated here by torch for
+    convenience; pass O and W_out to allocate nothing. Returns (O, W_out)."""
+    import torch
+
+    lib = load_library()
+    _require(Z.dim() == 2 and Vhat.dim() == 2 and W0.dim() == 2, "Z, Vhat, W0 must be 2-D")
+    T, Dff = Z.shape
+    D = Vhat.shape[1]
+    for t in (Z, Vhat, W0):
+        _require(t.is_cuda and t.is_contiguous() and t.dtype == torch.bfloat16,
+                 "Z, Vhat, W0 must be contiguous bf16 CUDA tensors")
+    _require(Vhat.shape[0] == T and tuple(W0.shape) == (Dff, D), "shape mismatch")
+    if O is None:
+        O = torch.empty((T, D), device=Z.device, dtype=torch.bfloat16)
+    if W_out is None:
+        W_out = torch.empty((Dff, D), device=Z.device, dtype=torch.float32)
+    st = lib.inplace_ttt_chunk_fwd_noalloc(_ptr(Z), _ptr(Vhat), _ptr(W0), ctypes.c_float(eta),
+                                           _ptr(O), _ptr(W_out), T, Dff, D, C,
+                                           _stream_ptr(stream))
+    _check("inplace_ttt_chunk_fwd_noalloc", st)
     return O, W_out
 
 

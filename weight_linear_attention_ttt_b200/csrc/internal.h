@@ -46,6 +46,8 @@ struct LaunchCtx {
 };
 
 void count_launch(uint64_t n = 1);
+// Records the detail returned by ttt_last_error_message() on this thread.
+void set_last_error(const std::string& msg);
 
 // 3-D tiled tensor map (dims innermost first; strides in bytes for dims 1 and 2).
 bool make_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,

@@ -20,6 +20,7 @@ void count_launch(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxe
 __device__ unsigned g_device_error;
 
 static thread_local std::string t_last_error;
+void set_last_error(const std::string& msg) { t_last_error = msg; }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn(std::string* msg) {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
