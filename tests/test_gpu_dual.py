@@ -189,3 +189,16 @@ def test_invalid_calls_raise_before_launch(cuda_lib):
         run(x48, 16)
     assert e.value.status == 2
     assert ttt.launch_count() == n0
+
+
+@pytest.mark.parametrize("warp_cols", ["8", "16"])
+@pytest.mark.parametrize("split", ["1", "2"])
+def test_kernel_variants_match_oracle(cuda_lib, monkeypatch, warp_cols, split):
+    """Every tensor-core variant (8 or 16 output columns per warp, one or two CTAs per stream)
+    meets the bf16 tolerance on full and partial pipeline stages."""
+    monkeypatch.setenv("TTT_DUAL_WARP_COLS", warp_cols)
+    monkeypatch.setenv("TTT_DUAL_COLUMN_SPLIT", split)
+    for T in (144, 512):
+        x = inp.dual_or_assoc_inputs(2, 3, T, 64, seed=T + 3, device="cuda", normalise=("K", "V"))
+        O, W = run(x, 16)
+        check(x, 16, O, W, TOL["bf16"])

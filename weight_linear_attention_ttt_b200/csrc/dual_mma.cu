@@ -37,8 +37,9 @@
 namespace ttt {
 namespace {
 
-template <int D, int NW, int CPS_ = 4>
+template <int D, int NW, int CPS_ = 4, int WC_ = 8>
 struct DualCfg {
+  static constexpr int WC = WC_;                   // output columns per compute warp (8 or 16)
   static constexpr int C = 16;
   static constexpr int CPS = CPS_;                 // chunks per pipeline stage
   static constexpr int R = C * CPS;                // token rows per stage
@@ -47,7 +48,7 @@ struct DualCfg {
   static constexpr int NSUB = D / SUB;
   static constexpr int SUB_BYTES = R * RB;
   static constexpr int TILE_BYTES = NSUB * SUB_BYTES;
-  static constexpr int COLS = 8 * NW;              // output columns per CTA
+  static constexpr int COLS = WC * NW;             // output columns per CTA
   static constexpr int NG = D / COLS;              // CTAs per stream
   static constexpr int OSUB = COLS >= 64 ? 64 : COLS;
   static constexpr int ORB = OSUB * 2;
@@ -126,13 +127,13 @@ __device__ __forceinline__ void stsm_x2(uint32_t addr, uint32_t r0, uint32_t r1)
                : "memory");
 }
 
-template <int D, int NW, int CPS>
-__global__ void __launch_bounds__(DualCfg<D, NW, CPS>::THREADS, 1)
+template <int D, int NW, int CPS, int WC>
+__global__ void __launch_bounds__(DualCfg<D, NW, CPS, WC>::THREADS, 1)
     dual_mma_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmO, const DualParams p) {
-  using Cfg = DualCfg<D, NW, CPS>;
+  using Cfg = DualCfg<D, NW, CPS, WC>;
   constexpr int R = Cfg::R, KS = Cfg::KS, NSTAGE = Cfg::NSTAGE, RB = Cfg::RB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS>::THREADS, 1)
   // ------------------------------------------------------------------ compute warps
   const int g = lane >> 2, tq = lane & 3;
   const int mi = lane >> 3, rr = lane & 7;   // ldmatrix: which 8x8 matrix / which row
-  const int colw = 8 * warp;                 // first column of this warp inside the CTA's
+  const int colw = WC * warp;                // first column of this warp inside the CTA's
   const int colg = col_cta + colw;           // ... and in the stream's W
 
   // Lane-constant parts of the swizzled shared-memory addresses. A chunk starts at row 16c,
@@ -220,21 +221,46 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS>::THREADS, 1)
   constexpr uint32_t CHUNK_ROWS_OBYTES = 16 * Cfg::ORB;
   const uint32_t sL = sbase + Cfg::L_OFF;
 
-  // W[:, colg .. colg+7] as m16n8 fp32 accumulators: m-tile mt holds rows 16mt .. 16mt+15.
-  float wc[KS][4];
+  // The state as m16n8 fp32 accumulators.
+  //   WC = 8:  W[:, colg .. colg+7];    tile mt holds rows 16mt .. 16mt+15 of W.
+  //   WC = 16: W^T[colg .. colg+15, :]; tile j holds columns 8j .. 8j+7 of W^T (rows of W).
+  float wc[WC == 8 ? KS : D / 8][4];
   {
     const float* w0 = p.W0 ? p.W0 + (size_t)stream * D * D : nullptr;
+    if constexpr (WC == 8) {
 #pragma unroll
-    for (int mt = 0; mt < KS; ++mt)
+      for (int mt = 0; mt < KS; ++mt)
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float2 v = make_float2(0.f, 0.f);
-        if (w0) v = *reinterpret_cast<const float2*>(w0 + (16 * mt + 8 * h + g) * D + colg +
-                                                     2 * tq);
-        wc[mt][2 * h] = v.x;
-        wc[mt][2 * h + 1] = v.y;
-      }
+        for (int h = 0; h < 2; ++h) {
+          float2 v = make_float2(0.f, 0.f);
+          if (w0) v = *reinterpret_cast<const float2*>(w0 + (16 * mt + 8 * h + g) * D + colg +
+                                                       2 * tq);
+          wc[mt][2 * h] = v.x;
+          wc[mt][2 * h + 1] = v.y;
+        }
+    } else {
+#pragma unroll
+      for (int jt = 0; jt < D / 8; ++jt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int row = 8 * jt + 2 * tq + e;
+          wc[jt][e] = w0 ? w0[row * D + colg + g] : 0.f;
+          wc[jt][2 + e] = w0 ? w0[row * D + colg + g + 8] : 0.f;
+        }
+    }
   }
+  // WC = 16 operand addresses: K rows as the B operand of W^T K^T, K via ldmatrix.trans as the
+  // B operand of the update, V^T in accumulator order, and the 16-column output tile.
+  uint32_t o_brow[KS], o_btrn[KS];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    o_brow[ks] = off(8 * (mi >> 1) + rr, 16 * ks + 8 * (mi & 1));
+    o_btrn[ks] = off(8 * (mi & 1) + rr, 16 * ks + 8 * (mi >> 1));
+  }
+  const uint32_t o_vt = off(8 * (mi >> 1) + rr, colg + 8 * (mi & 1));
+  const uint32_t o_st16 =
+      (colw / Cfg::OSUB) * Cfg::OSUB_BYTES +
+      swz<Cfg::ORB>((8 * (mi & 1) + rr) * Cfg::ORB + ((colw + 8 * (mi >> 1)) % Cfg::OSUB) * 2);
 
   bool ok = true;
   for (int j = 0; j < nstg; ++j) {
@@ -274,6 +300,7 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS>::THREADS, 1)
     }
     named_bar_sync(1, 32 * NW);
 
+    if constexpr (WC == 8) {
     // Per chunk: operand loads, the chain, then the outputs. A warp issues in order and shared
     // stores may alias later shared loads, so in a full stage the loads of chunk c+1 are placed
     // in program order between chunk c's chain and its outputs: they then overlap chunk c's
@@ -363,6 +390,111 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS>::THREADS, 1)
       }
     }
 
+    } else {
+    // WC = 16: the warp keeps W^T[16 cols, :]; its accumulator layout packed to bf16 is the A
+    // operand of the next chunk's W^T K_c^T, so the chain needs no register transposes.
+    struct Ops16 {
+      uint32_t kb[KS][4], kt[KS][4], qa[KS][4], vt[4], la[4];
+      float e0, e1, e8, e9;
+    };
+    auto load16 = [&](Ops16& o, const int c) {
+      const uint32_t cb = c * CHUNK_ROWS_BYTES;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        ldsm_x4(sK + cb + o_brow[ks], o.kb[ks]);
+        ldsm_x4_t(sK + cb + o_btrn[ks], o.kt[ks]);
+      }
+      ldsm_x4_t(sV + cb + o_vt, o.vt);
+      if (p.eta) {
+        o.e0 = ld_shared_f32(sEta + 4 * (16 * c + 2 * tq));
+        o.e1 = ld_shared_f32(sEta + 4 * (16 * c + 2 * tq + 1));
+        o.e8 = ld_shared_f32(sEta + 4 * (16 * c + 8 + 2 * tq));
+        o.e9 = ld_shared_f32(sEta + 4 * (16 * c + 9 + 2 * tq));
+      } else {
+        o.e0 = o.e1 = o.e8 = o.e9 = p.eta_scalar;
+      }
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) ldsm_x4(sQ + cb + o_arow[ks], o.qa[ks]);
+      ld_shared_v4(sL + c * 512 + lane * 16, o.la);
+    };
+    // chain: bf16(W^T) -> P^T = W^T K^T -> E^T -> W^T -= E^T K; returns the A fragments of
+    // bf16(W^T) and of E^T.
+    auto chain16 = [&](const Ops16& o, uint32_t (&wa)[KS][4], uint32_t (&ea)[4]) {
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        wa[ks][0] = pack_bf16(wc[2 * ks][0], wc[2 * ks][1]);
+        wa[ks][1] = pack_bf16(wc[2 * ks][2], wc[2 * ks][3]);
+        wa[ks][2] = pack_bf16(wc[2 * ks + 1][0], wc[2 * ks + 1][1]);
+        wa[ks][3] = pack_bf16(wc[2 * ks + 1][2], wc[2 * ks + 1][3]);
+      }
+      float pa[2][4] = {}, pb[2][4] = {};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        float (&acc)[2][4] = (ks & 1) ? pb : pa;
+        mma16816(acc[0], wa[ks][0], wa[ks][1], wa[ks][2], wa[ks][3], o.kb[ks][0], o.kb[ks][1]);
+        mma16816(acc[1], wa[ks][0], wa[ks][1], wa[ks][2], wa[ks][3], o.kb[ks][2], o.kb[ks][3]);
+      }
+      float E[2][4];
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        const float ea0 = n ? o.e8 : o.e0, ea1 = n ? o.e9 : o.e1;
+        E[n][0] = (pa[n][0] + pb[n][0] - bf16_lo(o.vt[2 * n])) * ea0;
+        E[n][1] = (pa[n][1] + pb[n][1] - bf16_hi(o.vt[2 * n])) * ea1;
+        E[n][2] = (pa[n][2] + pb[n][2] - bf16_lo(o.vt[2 * n + 1])) * ea0;
+        E[n][3] = (pa[n][3] + pb[n][3] - bf16_hi(o.vt[2 * n + 1])) * ea1;
+      }
+      ea[0] = pack_bf16(E[0][0], E[0][1]);
+      ea[1] = pack_bf16(E[0][2], E[0][3]);
+      ea[2] = pack_bf16(E[1][0], E[1][1]);
+      ea[3] = pack_bf16(E[1][2], E[1][3]);
+      const uint32_t n0 = ea[0] ^ 0x80008000u, n1 = ea[1] ^ 0x80008000u;
+      const uint32_t n2 = ea[2] ^ 0x80008000u, n3 = ea[3] ^ 0x80008000u;
+#pragma unroll
+      for (int jp = 0; jp < KS; ++jp) {
+        mma16816(wc[2 * jp], n0, n1, n2, n3, o.kt[jp][0], o.kt[jp][1]);
+        mma16816(wc[2 * jp + 1], n0, n1, n2, n3, o.kt[jp][2], o.kt[jp][3]);
+      }
+    };
+    // outputs: O[:, 16 cols] = Q W - mask(Q K^T) E
+    auto output16 = [&](const Ops16& o, const int c, const uint32_t (&wa)[KS][4],
+                        const uint32_t (&ea)[4]) {
+      float oa[2][4] = {}, ob[2][4] = {};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        float (&acc)[2][4] = (ks & 1) ? ob : oa;
+        mma16816(acc[0], o.qa[ks][0], o.qa[ks][1], o.qa[ks][2], o.qa[ks][3], wa[ks][0], wa[ks][2]);
+        mma16816(acc[1], o.qa[ks][0], o.qa[ks][1], o.qa[ks][2], o.qa[ks][3], wa[ks][1], wa[ks][3]);
+      }
+      mma16816(oa[0], o.la[0], o.la[1], o.la[2], o.la[3], ea[0], ea[2]);
+      mma16816(oa[1], o.la[0], o.la[1], o.la[2], o.la[3], ea[1], ea[3]);
+      stsm_x4(sO + c * CHUNK_ROWS_OBYTES + o_st16,
+              pack_bf16(oa[0][0] + ob[0][0], oa[0][1] + ob[0][1]),
+              pack_bf16(oa[0][2] + ob[0][2], oa[0][3] + ob[0][3]),
+              pack_bf16(oa[1][0] + ob[1][0], oa[1][1] + ob[1][1]),
+              pack_bf16(oa[1][2] + ob[1][2], oa[1][3] + ob[1][3]));
+    };
+    if (chunks == Cfg::CPS) {
+      Ops16 ops[2];
+      load16(ops[0], 0);
+#pragma unroll
+      for (int c = 0; c < Cfg::CPS; ++c) {
+        uint32_t wa[KS][4], ea[4];
+        chain16(ops[c & 1], wa, ea);
+        if (c + 1 < Cfg::CPS) load16(ops[(c + 1) & 1], c + 1);
+        output16(ops[c & 1], c, wa, ea);
+      }
+    } else {
+#pragma unroll 1
+      for (int c = 0; c < chunks; ++c) {
+        Ops16 o;
+        uint32_t wa[KS][4], ea[4];
+        load16(o, c);
+        chain16(o, wa, ea);
+        output16(o, c, wa, ea);
+      }
+    }
+    }
+
     // Inputs of this stage are consumed; hand the slot back to the producer.
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar + 8 * s);
@@ -385,19 +517,30 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS>::THREADS, 1)
   if (threadIdx.x == 0) bulk_wait<0>();
   if (!ok) return;
 
-  // Final state W[:, colg .. colg+7].
+  // Final state.
   float* wo = p.Wout + (size_t)stream * D * D;
+  if constexpr (WC == 8) {
 #pragma unroll
-  for (int mt = 0; mt < KS; ++mt)
+    for (int mt = 0; mt < KS; ++mt)
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
-      *reinterpret_cast<float2*>(wo + (16 * mt + 8 * h + g) * D + colg + 2 * tq) =
-          make_float2(wc[mt][2 * h], wc[mt][2 * h + 1]);
+      for (int h = 0; h < 2; ++h)
+        *reinterpret_cast<float2*>(wo + (16 * mt + 8 * h + g) * D + colg + 2 * tq) =
+            make_float2(wc[mt][2 * h], wc[mt][2 * h + 1]);
+  } else {
+#pragma unroll
+    for (int jt = 0; jt < D / 8; ++jt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int row = 8 * jt + 2 * tq + e;
+        wo[row * D + colg + g] = wc[jt][e];
+        wo[row * D + colg + g + 8] = wc[jt][2 + e];
+      }
+  }
 }
 
-template <int D, int NW, int CPS = 4>
+template <int D, int NW, int CPS = 4, int WC = 8>
 int launch_cfg(const StateArgs& a, const LaunchCtx& ctx) {
-  using Cfg = DualCfg<D, NW, CPS>;
+  using Cfg = DualCfg<D, NW, CPS, WC>;
   const int BH = a.B * a.H;
   CUtensorMap tq, tk, tv, to;
   const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.T, (uint64_t)BH};
@@ -414,7 +557,7 @@ int launch_cfg(const StateArgs& a, const LaunchCtx& ctx) {
       !make_tmap_3d(&tv, a.V, bf, dims, strides, box_in, sw(Cfg::RB), ctx.msg) ||
       !make_tmap_3d(&to, a.O, bf, dims, strides, box_out, sw(Cfg::ORB), ctx.msg))
     return kCuda;
-  auto kern = dual_mma_kernel<D, NW, CPS>;
+  auto kern = dual_mma_kernel<D, NW, CPS, WC>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg::SMEM);
   if (e != cudaSuccess) {
@@ -459,7 +602,14 @@ int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
     case 64: {
       // 8 chunks per pipeline stage halve the per-stage costs (score pieces, barriers, first
       // loads); measured faster on the 125M- and 1.3B-layer shapes. 4 is kept as an override.
+      // Two CTAs per stream (8 columns per warp) when the streams leave half the SMs idle;
+      // otherwise one CTA per stream with 16 columns per warp, which halves the per-stream
+      // shared-memory operand traffic (measured faster on the 125M-layer shape).
       const char* env = getenv("TTT_DUAL_STAGE_CHUNKS");  // tuning override: 4 or 8
+      const char* wenv = getenv("TTT_DUAL_WARP_COLS");    // tuning override: 8 or 16
+      const int wcols = wenv ? atoi(wenv) : (split == 2 ? 8 : 16);
+      if (wcols == 16)
+        return split == 2 ? launch_cfg<64, 2, 8, 16>(a, ctx) : launch_cfg<64, 4, 8, 16>(a, ctx);
       if (env && atoi(env) == 4)
         return split == 2 ? launch_cfg<64, 4>(a, ctx) : launch_cfg<64, 8>(a, ctx);
       return split == 2 ? launch_cfg<64, 4, 8>(a, ctx) : launch_cfg<64, 8, 8>(a, ctx);
