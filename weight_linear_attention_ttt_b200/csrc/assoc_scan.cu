@@ -23,8 +23,12 @@
 //   MMA-O  D_O = Q_c bf16(S) + P * EV             (B = bf16 copy of S^T, K-major)
 //   MMA-U  D_S += EV^T K_c                        (A = EV, MN-major; B = K, MN-major)
 //   warps  D_S -> bf16 copy of S^T for the next chunk; D_O -> bf16 O tile -> TMA store
-// Warp 0 issues TMA loads (3-stage ring), warp 1 owns TMEM and issues the MMAs from one
-// thread, warps 2-5 are the compute/epilogue warps (one per TMEM sub-partition).
+// Warp 0 issues TMA loads (3-stage ring); warp 1 owns TMEM and issues the MMAs from one thread;
+// warps 2-5 ("attention" group) turn scores into the masked P tile, scale V by eta and drain O;
+// warps 6-9 ("state" group) only refresh the bf16 copy of S after each update. The serial
+// chain per chunk is therefore MMA-U -> S readout -> MMA-U; the attention work of the next
+// chunk and the outputs of this one run beside it. Each group has one warp per TMEM
+// sub-partition.
 #include <algorithm>
 #include <cstdlib>
 
@@ -38,7 +42,7 @@ namespace {
 constexpr int D = 128;       // head dim
 constexpr int C = 64;        // chunk
 constexpr int HALF = 64;     // output columns per CTA
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;   // TMA warp, MMA warp, 4 attention warps, 4 state warps
 constexpr int STAGES = 3;
 
 // shared-memory map (bytes from the 1024-aligned base)
@@ -95,6 +99,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t sready = bar + 104;                            // bf16 S copy written (x2)
   const uint32_t ofull = bar + 120, oempty = bar + 136;         // output accumulators
   const uint32_t tslot = bar + 160;
+  const uint32_t evfree = bar + 168;                            // pass 1: EV tile reusable (x2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // pass 2: blockIdx = (stream * P + part) * 2 + half; pass 1 only covers parts 0 .. P-2
@@ -119,6 +124,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(oempty + 8 * b, 4);
     }
     mbar_init(sdone, 1);
+    mbar_init(evfree, 1);
+    mbar_init(evfree + 8, 1);
     fence_mbar_init();
   }
   if (warp == 1) umma::tmem_alloc(tslot, TM_COLS);
@@ -175,15 +182,30 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma::commit(pfull + 8 * b);
         return true;
       };
-      bool ok = STATE_ONLY ? true : mma_scores(0);
+      bool ok = true;
+      if (!STATE_ONLY) {
+        ok = mma_scores(0);
+        if (ok && nch > 1) ok = mma_scores(1);
+      }
       for (int c = 0; ok && c < nch; ++c) {
         const int s = c % STAGES, b = c & 1;
         const uint32_t sQ = sbase + s * STAGE_BYTES, sK = sQ + Q_BYTES;
         const uint32_t sEV = sbase + EV_OFF + 8192 * b;
+        if (STATE_ONLY && !mbar_wait(full + 8 * s, (c / STAGES) & 1, p.err)) break;
+        if (!mbar_wait(aready + 8 * b, (c >> 1) & 1, p.err)) break;
+        if (!STATE_ONLY && !mbar_wait(sready + 8 * b, (c >> 1) & 1, p.err)) break;
+        umma::fence_after();
+        // state update first: it heads the serial chain
+#pragma unroll
+        for (int ks = 0; ks < C / 16; ++ks)
+          umma::mma_ss(tmem + TM_S, umma::desc_mnmajor(sEV + 2048 * ks, 8192),
+                       umma::desc_mnmajor(sK + 2048 * ks, 8192), id_u,
+                       STATE_ONLY ? (c > 0 || ks > 0) : true);
+        // Pass 2 signals every update (the state warps refresh the bf16 copy); pass 1 only
+        // frees the EV tile per chunk and signals the final update.
+        if (!STATE_ONLY || c + 1 == nch) umma::commit(sdone);
+        if (STATE_ONLY) umma::commit(evfree + 8 * b);
         if (!STATE_ONLY) {
-          if (c + 1 < nch && !mma_scores(c + 1)) break;
-          if (!mbar_wait(aready + 8 * b, (c >> 1) & 1, p.err)) break;
-          if (!mbar_wait(sready + 8 * b, (c >> 1) & 1, p.err)) break;
           if (c >= 2 && !mbar_wait(oempty + 8 * b, ((c >> 1) - 1) & 1, p.err)) break;
           umma::fence_after();
           const uint32_t sS = sbase + SB_OFF + 16384 * b, sP = sbase + P_OFF + 8192 * b;
@@ -198,68 +220,25 @@ __global__ void __launch_bounds__(THREADS, 1)
             umma::mma_ss(dO, umma::desc_kmajor(sP + 32 * ks),
                          umma::desc_mnmajor(sEV + 2048 * ks, 8192), id_o2, true);
           umma::commit(ofull + 8 * b);
-        } else {
-          if (!mbar_wait(full + 8 * s, (c / STAGES) & 1, p.err)) break;
-          if (!mbar_wait(aready + 8 * b, (c >> 1) & 1, p.err)) break;
-          umma::fence_after();
         }
-#pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          umma::mma_ss(tmem + TM_S, umma::desc_mnmajor(sEV + 2048 * ks, 8192),
-                       umma::desc_mnmajor(sK + 2048 * ks, 8192), id_u,
-                       STATE_ONLY ? (c > 0 || ks > 0) : true);
-        umma::commit(sdone);
         umma::commit(empty + 8 * s);
+        if (!STATE_ONLY && c + 2 < nch && !mma_scores(c + 2)) break;
       }
     }
-  } else {
-    // ---------------------------------------------------------------- compute warps 2..5
+  } else if (warp < 6) {
+    // ---------------------------------------------------------------- attention warps 2..5
     const int q = warp & 3;
     const int ctid = threadIdx.x - 64;        // 0..127
     const bool rowthr = lane < 16;            // holds an M = 64 accumulator row
-    const int r = 16 * q + lane;              // that row (t for scores / O, d_out for S)
+    const int r = 16 * q + lane;              // that row (token t of the chunk)
     const uint32_t tl = (uint32_t)(32 * q) << 16;
-    const int dcol = HALF * half + r;         // global output column of S row r
 
-    // Initial state S^T[half] -> TMEM (fp32) and the bf16 copy for chunk 0.
-    if (!STATE_ONLY) {
-      const float* src = nullptr;
-      if (part == 0) src = p.S0 ? p.S0 + (size_t)stream * D * D : nullptr;
-      else src = p.S_start + ((size_t)stream * (p.P - 1) + (part - 1)) * D * D;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          v[j] = __float_as_uint((rowthr && src) ? src[(32 * cc + j) * D + dcol] : 0.f);
-        umma::st32x32(tmem + tl + TM_S + 32 * cc, v);
-        if (rowthr) {
-          uint8_t* row = smem + SB_OFF + (cc >> 1) * 8192;
-#pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            const int k = (32 * cc + j) & 63;
-            *reinterpret_cast<uint4*>(row + swz<128>(r * 128 + 2 * k)) = make_uint4(
-                pack_bf16(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
-                pack_bf16(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])),
-                pack_bf16(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5])),
-                pack_bf16(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7])));
-          }
-        }
-      }
-      umma::wait_st();
-      fence_proxy_async_smem();
-      umma::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sready);
-    }
-
-    bool ok = true;
-    for (int c = 0; c < nch; ++c) {
+    // Produce chunk c's operands: masked scores -> P tile, eta * V half -> EV tile.
+    auto produce = [&](int c) -> bool {
       const int s = c % STAGES, b = c & 1;
       const uint8_t* stg = smem + s * STAGE_BYTES;
-      // ---- scores -> masked bf16 P tile
       if (!STATE_ONLY) {
-        if (!mbar_wait(pfull + 8 * b, (c >> 1) & 1, p.err)) { ok = false; break; }
+        if (!mbar_wait(pfull + 8 * b, (c >> 1) & 1, p.err)) return false;
         umma::fence_after();
         uint32_t v0[32], v1[32];
         umma::ld32x32(tmem + tl + TM_P + 64 * b, v0);
@@ -285,13 +264,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      // ---- eta-scaled V half -> EV tile (same swizzled layout as the TMA tile)
-      if (!mbar_wait(full + 8 * s, (c / STAGES) & 1, p.err)) { ok = false; break; }
+      if (!mbar_wait(full + 8 * s, (c / STAGES) & 1, p.err)) return false;
       {
         const uint8_t* vt = stg + Q_BYTES + K_BYTES;
         const float* et = reinterpret_cast<const float*>(stg + Q_BYTES + K_BYTES + V_BYTES);
         uint8_t* ev = smem + EV_OFF + 8192 * b;
-        // 8192 bytes = 512 x 16-byte pieces; piece i covers row (i / 8), eight columns.
+        // 8192 bytes = 512 x 16-byte pieces; piece i covers row (i / 8), eight columns; the
+        // EV tile uses the same swizzled layout as the TMA tile.
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
           const int i = ctid + 128 * it;
@@ -309,70 +288,118 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_arrive(aready + 8 * b);
         mbar_arrive(empty + 8 * s);
       }
-      // ---- state update done -> bf16 copy of S^T for the next chunk (pass 2)
-      if (!mbar_wait(sdone, c & 1, p.err)) { ok = false; break; }
+      return true;
+    };
+    // Drain chunk c's outputs: D_O -> bf16 O tile -> TMA store.
+    auto consume = [&](int c) -> bool {
+      const int b = c & 1;
+      if (!mbar_wait(ofull + 8 * b, (c >> 1) & 1, p.err)) return false;
       umma::fence_after();
-      const bool last = c + 1 == nch;
-      if (!STATE_ONLY && !last) {
-        const int nb = (c + 1) & 1;
-        uint8_t* sb = smem + SB_OFF + 16384 * nb;
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t v[32];
-          umma::ld32x32(tmem + tl + TM_S + 32 * cc, v);
-          umma::wait_ld();
-          if (rowthr) {
-            uint8_t* row = sb + (cc >> 1) * 8192;
+      uint32_t v0[32], v1[32];
+      umma::ld32x32(tmem + tl + TM_O + 64 * b, v0);
+      umma::ld32x32(tmem + tl + TM_O + 64 * b + 32, v1);
+      umma::wait_ld();
+      umma::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(oempty + 8 * b);
+      if (rowthr) {
+        uint8_t* orow = smem + O_OFF + 8192 * b;
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-              const int k = (32 * cc + j) & 63;
-              *reinterpret_cast<uint4*>(row + swz<128>(r * 128 + 2 * k)) = make_uint4(
-                  pack_bf16(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
-                  pack_bf16(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])),
-                  pack_bf16(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5])),
-                  pack_bf16(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7])));
-            }
-          }
+        for (int j = 0; j < 64; j += 8) {
+          const uint32_t* vv = j < 32 ? v0 + j : v1 + (j - 32);
+          *reinterpret_cast<uint4*>(orow + swz<128>(r * 128 + 2 * j)) = make_uint4(
+              pack_bf16(__uint_as_float(vv[0]), __uint_as_float(vv[1])),
+              pack_bf16(__uint_as_float(vv[2]), __uint_as_float(vv[3])),
+              pack_bf16(__uint_as_float(vv[4]), __uint_as_float(vv[5])),
+              pack_bf16(__uint_as_float(vv[6]), __uint_as_float(vv[7])));
         }
-        fence_proxy_async_smem();
-        umma::fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sready + 8 * nb);
       }
-      // ---- outputs (pass 2): D_O -> bf16 O tile -> TMA store
-      if (!STATE_ONLY) {
-        if (!mbar_wait(ofull + 8 * b, (c >> 1) & 1, p.err)) { ok = false; break; }
-        umma::fence_after();
-        uint32_t v0[32], v1[32];
-        umma::ld32x32(tmem + tl + TM_O + 64 * b, v0);
-        umma::ld32x32(tmem + tl + TM_O + 64 * b + 32, v1);
-        umma::wait_ld();
-        umma::fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(oempty + 8 * b);
-        if (rowthr) {
-          uint8_t* orow = smem + O_OFF + 8192 * b;
-#pragma unroll
-          for (int j = 0; j < 64; j += 8) {
-            const uint32_t* vv = j < 32 ? v0 + j : v1 + (j - 32);
-            *reinterpret_cast<uint4*>(orow + swz<128>(r * 128 + 2 * j)) = make_uint4(
-                pack_bf16(__uint_as_float(vv[0]), __uint_as_float(vv[1])),
-                pack_bf16(__uint_as_float(vv[2]), __uint_as_float(vv[3])),
-                pack_bf16(__uint_as_float(vv[4]), __uint_as_float(vv[5])),
-                pack_bf16(__uint_as_float(vv[6]), __uint_as_float(vv[7])));
-          }
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (ctid == 0) {
-          tma_store_3d(&tmO, sbase + O_OFF + 8192 * b, HALF * half, tok0 + c * C, stream);
-          bulk_commit();
-          bulk_wait_read<1>();
-        }
-        named_bar_sync(1, 128);
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (ctid == 0) {
+        tma_store_3d(&tmO, sbase + O_OFF + 8192 * b, HALF * half, tok0 + c * C, stream);
+        bulk_commit();
+        bulk_wait_read<1>();
       }
+      named_bar_sync(1, 128);
+      return true;
+    };
+    // Chunk c+1's operands are produced before chunk c's outputs are drained, so the MMA
+    // thread always has the next chunk's P / EV when the state chain allows it to go on.
+    // Buffer (c+1) % 2 is free: chunk c-1's MMAs finished before its outputs were drained.
+    bool ok = produce(0);
+    for (int c = 0; ok && c < nch; ++c) {
+      // pass 1 has no outputs to wait for: wait until the update of chunk c-1 released its
+      // EV tile instead.
+      if (STATE_ONLY && c >= 1 && c + 1 < nch &&
+          !mbar_wait(evfree + 8 * ((c + 1) & 1), (((c + 1) >> 1) - 1) & 1, p.err))
+        break;
+      if (c + 1 < nch && !produce(c + 1)) break;
+      if (!STATE_ONLY && !consume(c)) break;
     }
     if (ctid == 0) bulk_wait<0>();
+  } else {
+    // ---------------------------------------------------------------- state warps 6..9
+    const int q = warp & 3;
+    const bool rowthr = lane < 16;
+    const int r = 16 * q + lane;              // row of S^T[half] = output column index
+    const uint32_t tl = (uint32_t)(32 * q) << 16;
+    const int dcol = HALF * half + r;         // global output column of S row r
+
+    // Writes the fp32 state rows in TMEM as the bf16 copy (K-major [64 dout][128 din]).
+    auto to_bf16 = [&](int nb) {
+      uint8_t* sb = smem + SB_OFF + 16384 * nb;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        umma::ld32x32(tmem + tl + TM_S + 32 * cc, v);
+        umma::wait_ld();
+        if (rowthr) {
+          uint8_t* row = sb + (cc >> 1) * 8192;
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            const int k = (32 * cc + j) & 63;
+            *reinterpret_cast<uint4*>(row + swz<128>(r * 128 + 2 * k)) = make_uint4(
+                pack_bf16(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
+                pack_bf16(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])),
+                pack_bf16(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5])),
+                pack_bf16(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7])));
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      umma::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sready + 8 * nb);
+    };
+
+    // Initial state S^T[half] -> TMEM (fp32) and its bf16 copy for chunk 0.
+    if (!STATE_ONLY) {
+      const float* src = nullptr;
+      if (part == 0) src = p.S0 ? p.S0 + (size_t)stream * D * D : nullptr;
+      else src = p.S_start + ((size_t)stream * (p.P - 1) + (part - 1)) * D * D;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          v[j] = __float_as_uint((rowthr && src) ? src[(32 * cc + j) * D + dcol] : 0.f);
+        umma::st32x32(tmem + tl + TM_S + 32 * cc, v);
+      }
+      umma::wait_st();
+      to_bf16(0);
+    }
+    bool ok = true;
+    if (STATE_ONLY) {
+      ok = mbar_wait(sdone, 0, p.err);
+      umma::fence_after();
+    } else {
+      for (int c = 0; c < nch; ++c) {
+        if (!mbar_wait(sdone, c & 1, p.err)) { ok = false; break; }
+        umma::fence_after();
+        if (c + 1 < nch) to_bf16((c + 1) & 1);
+      }
+    }
     // ---- final state of the part: increment (pass 1) or S_out (pass 2, last part)
     if (ok && (STATE_ONLY || part == p.P - 1)) {
       float* dst = STATE_ONLY ? p.S_dst + ((size_t)stream * (p.P - 1) + part) * D * D
