@@ -244,11 +244,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma::ld32x32(tmem + tl + TM_P + 64 * b, v0);
         umma::ld32x32(tmem + tl + TM_P + 64 * b + 32, v1);
         umma::wait_ld();
+        umma::reg_fence(v0);
+        umma::reg_fence(v1);
         umma::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(pempty + 8 * b);
         if (rowthr) {
-          uint8_t* prow = smem + P_OFF + 8192 * b;
+          const uint32_t prow = sbase + P_OFF + 8192 * b;
 #pragma unroll
           for (int j = 0; j < 64; j += 8) {
             float f[8];
@@ -258,28 +260,36 @@ __global__ void __launch_bounds__(THREADS, 1)
               const float x = __uint_as_float(sidx < 32 ? v0[sidx] : v1[sidx - 32]);
               f[e] = sidx <= r ? x : 0.f;
             }
-            *reinterpret_cast<uint4*>(prow + swz<128>(r * 128 + 2 * j)) =
-                make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                           pack_bf16(f[6], f[7]));
+            sts128(prow + swz<128>(r * 128 + 2 * j),
+                   make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                              pack_bf16(f[6], f[7])));
           }
         }
       }
       if (!mbar_wait(full + 8 * s, (c / STAGES) & 1, p.err)) return false;
       {
-        const uint8_t* vt = stg + Q_BYTES + K_BYTES;
-        const float* et = reinterpret_cast<const float*>(stg + Q_BYTES + K_BYTES + V_BYTES);
-        uint8_t* ev = smem + EV_OFF + 8192 * b;
+        const uint32_t vt = sbase + s * STAGE_BYTES + Q_BYTES + K_BYTES;
+        const uint32_t et = vt + V_BYTES;
+        const uint32_t ev = sbase + EV_OFF + 8192 * b;
         // 8192 bytes = 512 x 16-byte pieces; piece i covers row (i / 8), eight columns; the
         // EV tile uses the same swizzled layout as the TMA tile.
+        uint4 x[4];
+        float e[4];
 #pragma unroll
         for (int it = 0; it < 4; ++it) {
           const int i = ctid + 128 * it;
-          const uint32_t o = swz<128>((i >> 3) * 128 + (i & 7) * 16);
-          const float e = p.eta ? et[i >> 3] : p.eta_scalar;
-          const uint4 x = *reinterpret_cast<const uint4*>(vt + o);
-          *reinterpret_cast<uint4*>(ev + o) = make_uint4(
-              pack_bf16(bf16_lo(x.x) * e, bf16_hi(x.x) * e), pack_bf16(bf16_lo(x.y) * e, bf16_hi(x.y) * e),
-              pack_bf16(bf16_lo(x.z) * e, bf16_hi(x.z) * e), pack_bf16(bf16_lo(x.w) * e, bf16_hi(x.w) * e));
+          x[it] = lds128(vt + swz<128>((i >> 3) * 128 + (i & 7) * 16));
+          e[it] = p.eta ? ldsf(et + 4 * (i >> 3)) : p.eta_scalar;
+        }
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          const int i = ctid + 128 * it;
+          const float f = e[it];
+          sts128(ev + swz<128>((i >> 3) * 128 + (i & 7) * 16),
+                 make_uint4(pack_bf16(bf16_lo(x[it].x) * f, bf16_hi(x[it].x) * f),
+                            pack_bf16(bf16_lo(x[it].y) * f, bf16_hi(x[it].y) * f),
+                            pack_bf16(bf16_lo(x[it].z) * f, bf16_hi(x[it].z) * f),
+                            pack_bf16(bf16_lo(x[it].w) * f, bf16_hi(x[it].w) * f)));
         }
       }
       fence_proxy_async_smem();
@@ -299,19 +309,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       umma::ld32x32(tmem + tl + TM_O + 64 * b, v0);
       umma::ld32x32(tmem + tl + TM_O + 64 * b + 32, v1);
       umma::wait_ld();
+      umma::reg_fence(v0);
+      umma::reg_fence(v1);
       umma::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(oempty + 8 * b);
       if (rowthr) {
-        uint8_t* orow = smem + O_OFF + 8192 * b;
+        const uint32_t orow = sbase + O_OFF + 8192 * b;
 #pragma unroll
         for (int j = 0; j < 64; j += 8) {
           const uint32_t* vv = j < 32 ? v0 + j : v1 + (j - 32);
-          *reinterpret_cast<uint4*>(orow + swz<128>(r * 128 + 2 * j)) = make_uint4(
-              pack_bf16(__uint_as_float(vv[0]), __uint_as_float(vv[1])),
-              pack_bf16(__uint_as_float(vv[2]), __uint_as_float(vv[3])),
-              pack_bf16(__uint_as_float(vv[4]), __uint_as_float(vv[5])),
-              pack_bf16(__uint_as_float(vv[6]), __uint_as_float(vv[7])));
+          sts128(orow + swz<128>(r * 128 + 2 * j),
+                 make_uint4(pack_bf16(__uint_as_float(vv[0]), __uint_as_float(vv[1])),
+                            pack_bf16(__uint_as_float(vv[2]), __uint_as_float(vv[3])),
+                            pack_bf16(__uint_as_float(vv[4]), __uint_as_float(vv[5])),
+                            pack_bf16(__uint_as_float(vv[6]), __uint_as_float(vv[7]))));
         }
       }
       fence_proxy_async_smem();
@@ -348,22 +360,25 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     // Writes the fp32 state rows in TMEM as the bf16 copy (K-major [64 dout][128 din]).
     auto to_bf16 = [&](int nb) {
-      uint8_t* sb = smem + SB_OFF + 16384 * nb;
-#pragma unroll 1
+      const uint32_t sb = sbase + SB_OFF + 16384 * nb;
+      uint32_t v[2][32];
+      umma::ld32x32(tmem + tl + TM_S, v[0]);
+#pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        umma::ld32x32(tmem + tl + TM_S + 32 * cc, v);
         umma::wait_ld();
+        umma::reg_fence(v[cc & 1]);
+        if (cc + 1 < 4) umma::ld32x32(tmem + tl + TM_S + 32 * (cc + 1), v[(cc + 1) & 1]);
+        const uint32_t* vv = v[cc & 1];
         if (rowthr) {
-          uint8_t* row = sb + (cc >> 1) * 8192;
+          const uint32_t row = sb + (cc >> 1) * 8192;
 #pragma unroll
           for (int j = 0; j < 32; j += 8) {
             const int k = (32 * cc + j) & 63;
-            *reinterpret_cast<uint4*>(row + swz<128>(r * 128 + 2 * k)) = make_uint4(
-                pack_bf16(__uint_as_float(v[j]), __uint_as_float(v[j + 1])),
-                pack_bf16(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])),
-                pack_bf16(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5])),
-                pack_bf16(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7])));
+            sts128(row + swz<128>(r * 128 + 2 * k),
+                   make_uint4(pack_bf16(__uint_as_float(vv[j]), __uint_as_float(vv[j + 1])),
+                              pack_bf16(__uint_as_float(vv[j + 2]), __uint_as_float(vv[j + 3])),
+                              pack_bf16(__uint_as_float(vv[j + 4]), __uint_as_float(vv[j + 5])),
+                              pack_bf16(__uint_as_float(vv[j + 6]), __uint_as_float(vv[j + 7]))));
           }
         }
       }
@@ -409,6 +424,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint32_t v[32];
         umma::ld32x32(tmem + tl + TM_S + 32 * cc, v);
         umma::wait_ld();
+        umma::reg_fence(v);
         if (rowthr)
 #pragma unroll
           for (int j = 0; j < 32; ++j) dst[(32 * cc + j) * D + dcol] = __uint_as_float(v[j]);

@@ -198,60 +198,75 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int b = j & 1;
       if (!mbar_wait(tfull + 8 * b, (j >> 1) & 1, p.err)) break;
       umma::fence_after();
-#pragma unroll 1
-      for (int cc = 0; cc < BN / 32; ++cc) {
-        uint32_t r[32];
-        umma::ld32x32(tmem + ((uint32_t)(32 * q) << 16) + b * BN + 32 * cc, r);
+      // Column chunks of 32: the TMEM load and (for update tiles) the global W load of chunk
+      // cc+1 are issued before chunk cc is processed.
+      constexpr int NCC = BN / 32;
+      uint32_t r[2][32];
+      float w[2][32];
+      auto load_w = [&](float (&dst)[32], int cc) {
+        const size_t off = (size_t)(BM * mt + row) * p.D + BN * nt + 32 * cc;
+        if (p.first) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.W0 + off);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 x = src[v];
+            const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              dst[8 * v + 2 * e] = bf16_lo(xs[e]);
+              dst[8 * v + 2 * e + 1] = bf16_hi(xs[e]);
+            }
+          }
+        } else {
+          const float4* src = reinterpret_cast<const float4*>(p.Wout + off);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const float4 x = src[v];
+            dst[4 * v] = x.x;
+            dst[4 * v + 1] = x.y;
+            dst[4 * v + 2] = x.z;
+            dst[4 * v + 3] = x.w;
+          }
+        }
+      };
+      const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + b * BN;
+      umma::ld32x32(tbase, r[0]);
+      if (!rd) load_w(w[0], 0);
+#pragma unroll
+      for (int cc = 0; cc < NCC; ++cc) {
         umma::wait_ld();
+        umma::reg_fence(r[cc & 1]);
+        if (cc + 1 < NCC) {
+          umma::ld32x32(tbase + 32 * (cc + 1), r[(cc + 1) & 1]);
+          if (!rd) load_w(w[(cc + 1) & 1], cc + 1);
+        }
+        const uint32_t* rv = r[cc & 1];
         const int col = BN * nt + 32 * cc;
         if (rd) {
           uint4* dst = reinterpret_cast<uint4*>(p.O + (size_t)(p.tok0 + BM * mt + row) * p.D +
                                                 col);
 #pragma unroll
           for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pack_bf16(__uint_as_float(r[8 * v]), __uint_as_float(r[8 * v + 1])),
-                                pack_bf16(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-                                pack_bf16(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-                                pack_bf16(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+            dst[v] = make_uint4(pack_bf16(__uint_as_float(rv[8 * v]), __uint_as_float(rv[8 * v + 1])),
+                                pack_bf16(__uint_as_float(rv[8 * v + 2]), __uint_as_float(rv[8 * v + 3])),
+                                pack_bf16(__uint_as_float(rv[8 * v + 4]), __uint_as_float(rv[8 * v + 5])),
+                                pack_bf16(__uint_as_float(rv[8 * v + 6]), __uint_as_float(rv[8 * v + 7])));
         } else {
           const size_t off = (size_t)(BM * mt + row) * p.D + col;
-          float w[32];
-          if (p.first) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.W0 + off);
+          float* wv = w[cc & 1];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const uint4 x = src[v];
-              const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                w[8 * v + 2 * e] = bf16_lo(xs[e]);
-                w[8 * v + 2 * e + 1] = bf16_hi(xs[e]);
-              }
-            }
-          } else {
-            const float4* src = reinterpret_cast<const float4*>(p.Wout + off);
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const float4 x = src[v];
-              w[4 * v] = x.x;
-              w[4 * v + 1] = x.y;
-              w[4 * v + 2] = x.z;
-              w[4 * v + 3] = x.w;
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) w[e] = fmaf(p.eta, __uint_as_float(r[e]), w[e]);
+          for (int e = 0; e < 32; ++e) wv[e] = fmaf(p.eta, __uint_as_float(rv[e]), wv[e]);
           float4* dst = reinterpret_cast<float4*>(p.Wout + off);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+            dst[v] = make_float4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
           if (p.Wbf_next) {
             uint4* db = reinterpret_cast<uint4*>(p.Wbf_next + off);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
-              db[v] = make_uint4(pack_bf16(w[8 * v], w[8 * v + 1]), pack_bf16(w[8 * v + 2], w[8 * v + 3]),
-                                 pack_bf16(w[8 * v + 4], w[8 * v + 5]),
-                                 pack_bf16(w[8 * v + 6], w[8 * v + 7]));
+              db[v] = make_uint4(pack_bf16(wv[8 * v], wv[8 * v + 1]), pack_bf16(wv[8 * v + 2], wv[8 * v + 3]),
+                                 pack_bf16(wv[8 * v + 4], wv[8 * v + 5]),
+                                 pack_bf16(wv[8 * v + 6], wv[8 * v + 7]));
           }
         }
       }

@@ -112,6 +112,12 @@ __device__ __forceinline__ void st32x32(uint32_t taddr, const uint32_t (&r)[32])
 __device__ __forceinline__ void wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// Orders every later use of `r` after the preceding wait_ld(): the registers written by an
+// asynchronous TMEM load pass through an empty volatile asm that the compiler cannot hoist.
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
+}
 __device__ __forceinline__ void wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
