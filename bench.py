@@ -296,6 +296,7 @@ def run_ours(args, w, rank, world, local_rank):
     import weight_linear_attention_ttt_b200 as ttt
     from weight_linear_attention_ttt_b200 import inputs as inp
     from weight_linear_attention_ttt_b200 import metrics
+    from weight_linear_attention_ttt_b200.shard import max_over_ranks
 
     dev = torch.device("cuda", local_rank)
     ttt.load_library()
@@ -324,11 +325,7 @@ def run_ours(args, w, rank, world, local_rank):
     launches = ttt.launch_count() - n0
     if world > 1:
         dist.barrier()
-    total_ms = sum(a.elapsed_time(b) for a, b in ev)
-    t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
     ms_per_step = total_ms / args.steps
     value = world * algo["tokens"] * args.steps / (total_ms / 1e3)
     assert ttt.read_device_error() == 0, "a bounded device wait gave up during the bench"
@@ -336,10 +333,8 @@ def run_ours(args, w, rank, world, local_rank):
     # end to end from host buffers, same metric
     e2e_steps = max(3, min(args.steps, 20))
     e2e_ms, h2d, d2h = e2e_measure(w, x, e2e_steps, 2)
-    et = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(et, op=dist.ReduceOp.MAX)
-    e2e_value = world * algo["tokens"] / (float(et.item()) / 1e3)
+    e2e_ms = max_over_ranks(e2e_ms, dev)
+    e2e_value = world * algo["tokens"] / (e2e_ms / 1e3)
 
     pk, pk_kind = peaks()
     kname, ksrc = DOMINANT_KERNEL[w.kind]
@@ -372,7 +367,7 @@ def run_ours(args, w, rank, world, local_rank):
                        "parallelism": f"dp{world} (independent streams per rank)"},
             "roofline": roof, "clocks": clk.summary(), "gpu_launches": launches,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": float(et.item())}}
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         cursor = [0]
         budget = args.cpu_budget

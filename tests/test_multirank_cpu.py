@@ -1,0 +1,85 @@
+"""Multi-rank path on CPU: two gloo ranks each compute their own share of the streams (the fp64
+oracle stands in for the GPU kernel on a GPU-less host), with no collective on the data path;
+gathering the shares reproduces the single-process result, and the timing reduction takes the
+max over ranks."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, outdir):
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    from oracle import ttt_oracle as orc
+    from weight_linear_attention_ttt_b200 import inputs as inp
+    from weight_linear_attention_ttt_b200.shard import (max_over_ranks, shard_columns,
+                                                        shard_streams)
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        # dual form: shard (b,h) streams along the batch dimension
+        x = inp.dual_or_assoc_inputs(4, 2, 64, 16, seed=3, device="cpu", normalise=("K", "V"))
+        mine = shard_streams(x, rank, world)
+        O, W = orc.dual_form(mine["Q"].float().numpy(), mine["K"].float().numpy(),
+                             mine["V"].float().numpy(), mine["eta"].numpy(),
+                             mine["W0"].numpy(), 16)
+        np.save(os.path.join(outdir, f"dual_O_{rank}.npy"), O)
+        np.save(os.path.join(outdir, f"dual_W_{rank}.npy"), W)
+        # In-Place: shard output columns; Z is shared
+        z = inp.inplace_inputs(64, 32, 24, seed=4, device="cpu", eta=0.05)
+        zc = shard_columns(z, rank, world)
+        Oi, Wi = orc.inplace_chunks(zc["Z"].float().numpy(), zc["Vhat"].float().numpy(),
+                                    zc["W0"].float().numpy(), zc["eta"], 32)
+        np.save(os.path.join(outdir, f"inp_O_{rank}.npy"), Oi)
+        np.save(os.path.join(outdir, f"inp_W_{rank}.npy"), Wi)
+        # timing reduction: max over ranks
+        m = max_over_ranks(10.0 + rank)
+        np.save(os.path.join(outdir, f"max_{rank}.npy"), np.array([m]))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_shard_without_data_collectives(tmp_path):
+    world = 2
+    mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    from oracle import ttt_oracle as orc
+    from weight_linear_attention_ttt_b200 import inputs as inp
+
+    x = inp.dual_or_assoc_inputs(4, 2, 64, 16, seed=3, device="cpu", normalise=("K", "V"))
+    O, W = orc.dual_form(x["Q"].float().numpy(), x["K"].float().numpy(), x["V"].float().numpy(),
+                         x["eta"].numpy(), x["W0"].numpy(), 16)
+    Og = np.concatenate([np.load(tmp_path / f"dual_O_{r}.npy") for r in range(world)])
+    Wg = np.concatenate([np.load(tmp_path / f"dual_W_{r}.npy") for r in range(world)])
+    np.testing.assert_array_equal(Og, O)
+    np.testing.assert_array_equal(Wg, W)
+
+    z = inp.inplace_inputs(64, 32, 24, seed=4, device="cpu", eta=0.05)
+    Oi, Wi = orc.inplace_chunks(z["Z"].float().numpy(), z["Vhat"].float().numpy(),
+                                z["W0"].float().numpy(), z["eta"], 32)
+    Oig = np.concatenate([np.load(tmp_path / f"inp_O_{r}.npy") for r in range(world)], axis=1)
+    Wig = np.concatenate([np.load(tmp_path / f"inp_W_{r}.npy") for r in range(world)], axis=1)
+    np.testing.assert_allclose(Oig, Oi, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(Wig, Wi, rtol=1e-12, atol=1e-12)
+
+    for r in range(world):
+        assert float(np.load(tmp_path / f"max_{r}.npy")[0]) == 11.0
