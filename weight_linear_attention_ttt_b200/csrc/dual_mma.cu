@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS, WC>::THREADS, 1)
 
     // ---- causal scores of this stage: piece (chunk cc, score columns 8jj..8jj+7) per warp,
     //      stored negated and masked as the A fragments of -mask(Q_c K_c^T).
-    for (int pc = warp; pc < 2 * chunks; pc += NW) {
+    for (int pc = warp; pc < (WC == 8 ? 2 * chunks : 0); pc += NW) {
       const int cc = pc >> 1, jj = pc & 1;
       float lc[4] = {};
 #pragma unroll
@@ -298,9 +298,9 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS, WC>::THREADS, 1)
       st_shared_v2(sL + cc * 512 + lane * 16 + jj * 8, pack_bf16(-lc[0], -lc[1]),
                    pack_bf16(-lc[2], -lc[3]));
     }
+    if constexpr (WC == 8) {
     named_bar_sync(1, 32 * NW);
 
-    if constexpr (WC == 8) {
     // Per chunk: operand loads, the chain, then the outputs. A warp issues in order and shared
     // stores may alias later shared loads, so in a full stage the loads of chunk c+1 are placed
     // in program order between chunk c's chain and its outputs: they then overlap chunk c's
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS, WC>::THREADS, 1)
     // WC = 16: the warp keeps W^T[16 cols, :]; its accumulator layout packed to bf16 is the A
     // operand of the next chunk's W^T K_c^T, so the chain needs no register transposes.
     struct Ops16 {
-      uint32_t kb[KS][4], kt[KS][4], qa[KS][4], vt[4], la[4];
+      uint32_t kb[KS][4], kt[KS][4], qa[KS][4], vt[4];
       float e0, e1, e8, e9;
     };
     auto load16 = [&](Ops16& o, const int c) {
@@ -415,7 +415,6 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS, WC>::THREADS, 1)
       }
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) ldsm_x4(sQ + cb + o_arow[ks], o.qa[ks]);
-      ld_shared_v4(sL + c * 512 + lane * 16, o.la);
     };
     // chain: bf16(W^T) -> P^T = W^T K^T -> E^T -> W^T -= E^T K; returns the A fragments of
     // bf16(W^T) and of E^T.
@@ -455,9 +454,26 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS, WC>::THREADS, 1)
         mma16816(wc[2 * jp + 1], n0, n1, n2, n3, o.kt[jp][2], o.kt[jp][3]);
       }
     };
-    // outputs: O[:, 16 cols] = Q W - mask(Q K^T) E
+    // outputs: O[:, 16 cols] = Q W - mask(Q K^T) E. The warp forms the causal scores itself from
+    // the Q and K fragments it already holds (A = Q rows, B = K rows), so no scores cross warps.
     auto output16 = [&](const Ops16& o, const int c, const uint32_t (&wa)[KS][4],
                         const uint32_t (&ea)[4]) {
+      float lc[2][4] = {}, ld[2][4] = {};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        float (&acc)[2][4] = (ks & 1) ? ld : lc;
+        mma16816(acc[0], o.qa[ks][0], o.qa[ks][1], o.qa[ks][2], o.qa[ks][3], o.kb[ks][0], o.kb[ks][1]);
+        mma16816(acc[1], o.qa[ks][0], o.qa[ks][1], o.qa[ks][2], o.qa[ks][3], o.kb[ks][2], o.kb[ks][3]);
+      }
+      // keep s <= t: entry (jj, i) is t = g + 8 (i >> 1), s = 8 jj + 2 tq + (i & 1)
+      float m[2][4];
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          m[jj][i] = (8 * jj + 2 * tq + (i & 1) > g + 8 * (i >> 1)) ? 0.f : -(lc[jj][i] + ld[jj][i]);
+      const uint32_t la0 = pack_bf16(m[0][0], m[0][1]), la1 = pack_bf16(m[0][2], m[0][3]);
+      const uint32_t la2 = pack_bf16(m[1][0], m[1][1]), la3 = pack_bf16(m[1][2], m[1][3]);
       float oa[2][4] = {}, ob[2][4] = {};
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
@@ -465,8 +481,8 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS, WC>::THREADS, 1)
         mma16816(acc[0], o.qa[ks][0], o.qa[ks][1], o.qa[ks][2], o.qa[ks][3], wa[ks][0], wa[ks][2]);
         mma16816(acc[1], o.qa[ks][0], o.qa[ks][1], o.qa[ks][2], o.qa[ks][3], wa[ks][1], wa[ks][3]);
       }
-      mma16816(oa[0], o.la[0], o.la[1], o.la[2], o.la[3], ea[0], ea[2]);
-      mma16816(oa[1], o.la[0], o.la[1], o.la[2], o.la[3], ea[1], ea[3]);
+      mma16816(oa[0], la0, la1, la2, la3, ea[0], ea[2]);
+      mma16816(oa[1], la0, la1, la2, la3, ea[1], ea[3]);
       stsm_x4(sO + c * CHUNK_ROWS_OBYTES + o_st16,
               pack_bf16(oa[0][0] + ob[0][0], oa[0][1] + ob[0][1]),
               pack_bf16(oa[0][2] + ob[0][2], oa[0][3] + ob[0][3]),
@@ -602,12 +618,12 @@ int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
     case 64: {
       // 8 chunks per pipeline stage halve the per-stage costs (score pieces, barriers, first
       // loads); measured faster on the 125M- and 1.3B-layer shapes. 4 is kept as an override.
-      // Two CTAs per stream (8 columns per warp) when the streams leave half the SMs idle;
-      // otherwise one CTA per stream with 16 columns per warp, which halves the per-stream
-      // shared-memory operand traffic (measured faster on the 125M-layer shape).
+      // 16 columns per warp (W^T form, the warp computes its own causal scores) was measured
+      // faster than 8 columns per warp on the 125M- and 1.3B-layer shapes, with one CTA per
+      // stream and with two. 8 columns and 4-chunk stages remain as tuning overrides.
       const char* env = getenv("TTT_DUAL_STAGE_CHUNKS");  // tuning override: 4 or 8
       const char* wenv = getenv("TTT_DUAL_WARP_COLS");    // tuning override: 8 or 16
-      const int wcols = wenv ? atoi(wenv) : (split == 2 ? 8 : 16);
+      const int wcols = wenv ? atoi(wenv) : 16;
       if (wcols == 16)
         return split == 2 ? launch_cfg<64, 2, 8, 16>(a, ctx) : launch_cfg<64, 4, 8, 16>(a, ctx);
       if (env && atoi(env) == 4)
