@@ -35,7 +35,8 @@ struct IpCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BK * BN * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int WST_OFF = STAGES * STAGE_BYTES;     // 2 x [128 rows][32 fp32] W tiles
+  static constexpr int BAR_OFF = WST_OFF + 2 * 16384;
   static constexpr int SMEM = 1024 + BAR_OFF + 256;
   static constexpr int TMEM_COLS = 2 * BN;
 };
@@ -54,12 +55,17 @@ struct IpParams {
   unsigned* err;
 };
 
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 template <int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     inplace_chunk_kernel(const __grid_constant__ CUtensorMap tmZk,   // Z, box 64 x 128
                          const __grid_constant__ CUtensorMap tmZm,   // Z, box 64 x 64
                          const __grid_constant__ CUtensorMap tmW,    // bf16 W read source
                          const __grid_constant__ CUtensorMap tmV,    // Vhat, box 64 x 64
+                         const __grid_constant__ CUtensorMap tmWf,   // W_out fp32, box 32 x 128
                          const IpParams p) {
   using Cfg = IpCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -71,6 +77,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tfull = bar + 16 * STAGES, tempty = tfull + 16;
   const uint32_t sfull = tempty + 16, sempty = sfull + 16;
   const uint32_t tslot = sempty + 16;                  // TMEM base address
+  const uint32_t wfull = tslot + 32;                   // W staging buffers loaded (x2)
   volatile int* sched = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + 16 * STAGES + 80);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntn = p.D / BN;
@@ -85,6 +92,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(tempty + 8 * b, 4);
       mbar_init(sfull + 8 * b, 1);
       mbar_init(sempty + 8 * b, 5);
+      mbar_init(wfull + 8 * b, 1);
     }
     fence_mbar_init();
   }
@@ -185,6 +193,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ epilogue warps 2..5
     const int q = warp & 3;  // TMEM subpartition this warp may read
     const int row = 32 * q + lane;
+    uint32_t wld = 0;        // W staging loads issued so far (selects buffer and phase)
     for (int j = 0;; ++j) {
       const int slot = j & 1;
       if (!mbar_wait(sfull + 8 * slot, (j >> 1) & 1, p.err)) break;
@@ -198,48 +207,32 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int b = j & 1;
       if (!mbar_wait(tfull + 8 * b, (j >> 1) & 1, p.err)) break;
       umma::fence_after();
-      // Column chunks of 32: the TMEM load and (for update tiles) the global W load of chunk
-      // cc+1 are issued before chunk cc is processed.
+      // Column chunks of 32. The TMEM load of chunk cc+1 is issued before chunk cc is
+      // processed. Update tiles read the running fp32 W through two shared-memory buffers that
+      // one thread fills by TMA two chunks ahead (a 16 KB tile per load); the first chunk's
+      // update reads the bf16 W0 directly from global memory.
       constexpr int NCC = BN / 32;
-      uint32_t r[2][32];
-      float w[2][32];
-      auto load_w = [&](float (&dst)[32], int cc) {
-        const size_t off = (size_t)(BM * mt + row) * p.D + BN * nt + 32 * cc;
-        if (p.first) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.W0 + off);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 x = src[v];
-            const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              dst[8 * v + 2 * e] = bf16_lo(xs[e]);
-              dst[8 * v + 2 * e + 1] = bf16_hi(xs[e]);
-            }
-          }
-        } else {
-          const float4* src = reinterpret_cast<const float4*>(p.Wout + off);
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const float4 x = src[v];
-            dst[4 * v] = x.x;
-            dst[4 * v + 1] = x.y;
-            dst[4 * v + 2] = x.z;
-            dst[4 * v + 3] = x.w;
-          }
-        }
+      const bool staged = !rd && !p.first;
+      const int ctid = threadIdx.x - 64;
+      auto issue_w = [&](int cc) {
+        const int wb = (int)((wld + cc) & 1);
+        const uint32_t dst = sbase + Cfg::WST_OFF + 16384 * wb;
+        mbar_arrive_expect_tx(wfull + 8 * wb, 16384);
+        tma_load_2d(dst, &tmWf, wfull + 8 * wb, BN * nt + 32 * cc, BM * mt);
       };
+      if (staged && ctid == 0) {
+        issue_w(0);
+        if (NCC > 1) issue_w(1);
+      }
+      uint32_t r[2][32];
+      float w[32];
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + b * BN;
       umma::ld32x32(tbase, r[0]);
-      if (!rd) load_w(w[0], 0);
 #pragma unroll
       for (int cc = 0; cc < NCC; ++cc) {
         umma::wait_ld();
         umma::reg_fence(r[cc & 1]);
-        if (cc + 1 < NCC) {
-          umma::ld32x32(tbase + 32 * (cc + 1), r[(cc + 1) & 1]);
-          if (!rd) load_w(w[(cc + 1) & 1], cc + 1);
-        }
+        if (cc + 1 < NCC) umma::ld32x32(tbase + 32 * (cc + 1), r[(cc + 1) & 1]);
         const uint32_t* rv = r[cc & 1];
         const int col = BN * nt + 32 * cc;
         if (rd) {
@@ -253,23 +246,55 @@ __global__ void __launch_bounds__(THREADS, 1)
                                 pack_bf16(__uint_as_float(rv[8 * v + 6]), __uint_as_float(rv[8 * v + 7])));
         } else {
           const size_t off = (size_t)(BM * mt + row) * p.D + col;
-          float* wv = w[cc & 1];
+          if (staged) {
+            const int wb = (int)((wld + cc) & 1);
+            // a wait that gives up only raises the error word: every thread must still reach
+            // the named barrier below
+            mbar_wait(wfull + 8 * wb, (uint32_t)(((wld + cc) >> 1) & 1), p.err);
+            const uint32_t src = sbase + Cfg::WST_OFF + 16384 * wb;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) wv[e] = fmaf(p.eta, __uint_as_float(rv[e]), wv[e]);
+            for (int v = 0; v < 8; ++v) {
+              const uint4 x = lds128(src + swz<128>(row * 128 + 16 * v));
+              w[4 * v] = __uint_as_float(x.x);
+              w[4 * v + 1] = __uint_as_float(x.y);
+              w[4 * v + 2] = __uint_as_float(x.z);
+              w[4 * v + 3] = __uint_as_float(x.w);
+            }
+          } else {
+            const uint4* src = reinterpret_cast<const uint4*>(p.W0 + off);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint4 x = src[v];
+              const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                w[8 * v + 2 * e] = bf16_lo(xs[e]);
+                w[8 * v + 2 * e + 1] = bf16_hi(xs[e]);
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) w[e] = fmaf(p.eta, __uint_as_float(rv[e]), w[e]);
           float4* dst = reinterpret_cast<float4*>(p.Wout + off);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+            dst[v] = make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
           if (p.Wbf_next) {
             uint4* db = reinterpret_cast<uint4*>(p.Wbf_next + off);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
-              db[v] = make_uint4(pack_bf16(wv[8 * v], wv[8 * v + 1]), pack_bf16(wv[8 * v + 2], wv[8 * v + 3]),
-                                 pack_bf16(wv[8 * v + 4], wv[8 * v + 5]),
-                                 pack_bf16(wv[8 * v + 6], wv[8 * v + 7]));
+              db[v] = make_uint4(pack_bf16(w[8 * v], w[8 * v + 1]), pack_bf16(w[8 * v + 2], w[8 * v + 3]),
+                                 pack_bf16(w[8 * v + 4], w[8 * v + 5]),
+                                 pack_bf16(w[8 * v + 6], w[8 * v + 7]));
+          }
+          if (staged) {
+            // every epilogue thread is done with this buffer: refill it two chunks ahead
+            named_bar_sync(1, 128);
+            if (ctid == 0 && cc + 2 < NCC) issue_w(cc + 2);
           }
         }
       }
+      if (staged) wld += NCC;
       umma::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + 8 * b);
@@ -300,7 +325,7 @@ int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
   }
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-  CUtensorMap tzk, tzm, tv, tw0, tw[2];
+  CUtensorMap tzk, tzm, tv, tw0, tw[2], twf;
   {
     const uint64_t dz[2] = {(uint64_t)a.Dff, (uint64_t)a.T};
     const uint32_t bk[2] = {64, 128}, bm[2] = {64, 64};
@@ -310,6 +335,10 @@ int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
         !make_tmap_2d(&tzm, a.Z, bf, dz, (uint64_t)a.Dff * 2, bm, sw, ctx.msg) ||
         !make_tmap_2d(&tv, a.Vhat, bf, dv, (uint64_t)a.D * 2, bm, sw, ctx.msg) ||
         !make_tmap_2d(&tw0, a.W0, bf, dw, (uint64_t)a.D * 2, bm, sw, ctx.msg))
+      return kCuda;
+    const uint32_t bwf[2] = {32, 128};
+    if (!make_tmap_2d(&twf, a.W_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dw, (uint64_t)a.D * 4, bwf,
+                      sw, ctx.msg))
       return kCuda;
     for (int b = 0; b < 2; ++b)
       if (wbf[b] && !make_tmap_2d(&tw[b], wbf[b], bf, dw, (uint64_t)a.D * 2, bm, sw, ctx.msg))
@@ -346,7 +375,7 @@ int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
     p.counter = counters + i;
     p.err = ctx.err;
     const CUtensorMap& wsrc = i == 0 ? tw0 : tw[(i - 1) & 1];
-    kern<<<grid, THREADS, Cfg::SMEM, ctx.stream>>>(tzk, tzm, wsrc, tv, p);
+    kern<<<grid, THREADS, Cfg::SMEM, ctx.stream>>>(tzk, tzm, wsrc, tv, twf, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
       *ctx.msg = std::string("inplace launch: ") + cudaGetErrorString(e);
