@@ -33,8 +33,8 @@ METRIC = "TTT-layer fwd tokens/s on 1 B200; % of bf16 tensor-peak/HBM roofline"
 DEFAULT_WORKLOAD = "dual_bf16_B8H12T2048_d64C16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DOMINANT_KERNEL = {"dual": ("dual_mma_kernel", "dual_mma.cu"),
-                   "assoc": ("assoc_pass2_kernel", "assoc_scan.cu"),
-                   "inplace": ("inplace_gemm_kernel", "inplace_ttt.cu")}
+                   "assoc": ("assoc_chunk_kernel", "assoc_scan.cu"),
+                   "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu")}
 
 
 def peaks():
