@@ -120,6 +120,29 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
                        cudaStream_t stream);
 
 /* --------------------------------------------------------------------------------------------
+ * State increment of a sequence slice in the associative mode (the first pass of the prefix
+ * scan over states, "KV 바인딩 기반 테스트 시간 학습은 사실상 선형 어텐션이다", associativity
+ * paragraph; per-chunk deltas combined by a prefix sum for context parallelism, "In-Place
+ * 테스트 시점 학습", associative-scan paragraph):
+ *     dS = sum_t eta_t k_t^T v_t  over the T tokens given
+ *  K, V [B,H,T,d]; eta [B,H,T] fp32 or NULL (eta_scalar); dS [B,H,d,d] fp32 output.
+ *  A context-parallel caller gives each device a slice of the sequence, exchanges the slices'
+ *  increments, and starts ttt_assoc_scan_fwd on its slice from S0 plus the earlier slices'
+ *  increments. Supported: bf16, d == 128, C == 64, T % C == 0. No workspace.
+ * ------------------------------------------------------------------------------------------ */
+int ttt_assoc_state_fwd(const void* K, const void* V, const float* eta, float eta_scalar,
+                        float* dS, int B, int H, int T, int d, int C, int dt,
+                        cudaStream_t stream);
+
+/* Prefix combination of per-slice state increments: out = S0 + sum_{r < upto} increments[r].
+ *  S0 [B,H,d,d] fp32 or NULL (zeros); increments [n_increments][B,H,d,d] fp32 (e.g. gathered
+ *  from all devices); out [B,H,d,d] fp32, may equal S0, must not overlap the increments.
+ *  With upto = this device's slice index it gives the slice's starting state; with
+ *  upto = n_increments, the state after the whole sequence. */
+int ttt_state_prefix_sum(const float* S0, const float* increments, int n_increments, int upto,
+                         int B, int H, int d, float* out, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------------------------
  * In-Place TTT, W_down chunk update (W = W0; for each chunk i of C tokens, in order):
  *     O_i = Z_i W                  (W holds W0 plus the deltas of the chunks before i)
  *     W   = W + eta Z_i^T Vhat_i

@@ -83,3 +83,79 @@ def test_two_gloo_ranks_shard_without_data_collectives(tmp_path):
 
     for r in range(world):
         assert float(np.load(tmp_path / f"max_{r}.npy")[0]) == 11.0
+
+
+def _cp_worker(rank, world, port, outdir):
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    from oracle import ttt_oracle as orc
+    from weight_linear_attention_ttt_b200 import inputs as inp
+    from weight_linear_attention_ttt_b200.context_parallel import assoc_scan_fwd_cp
+    from weight_linear_attention_ttt_b200.shard import split_range
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        B, H, T, d, C = 2, 2, 256, 8, 16
+        x = inp.dual_or_assoc_inputs(B, H, T, d, seed=12, device="cpu", normalise=("Q", "K"),
+                                     eta="sigmoid", w0="normal_0.02")
+        t0, t1 = split_range(T // C, rank, world)
+        sl = slice(t0 * C, t1 * C)
+        Q, K, V = (x[k][:, :, sl].double() for k in ("Q", "K", "V"))
+        eta = x["eta"][:, :, sl].double()
+        S0 = x["W0"].double()
+
+        def per_stream(fn, *args):
+            outs = [[fn(*(a[b, h] for a in args)) for h in range(H)] for b in range(B)]
+            return outs
+
+        def state_fn(K_, V_, e_):
+            res = per_stream(lambda k, v, e: orc.assoc_chunked_stream(k, k, v, e, None, C)[1],
+                             K_.numpy(), V_.numpy(), e_.numpy())
+            return torch.tensor(np.array(res))
+
+        def scan_fn(Q_, K_, V_, e_, s_):
+            res = per_stream(lambda q, k, v, e, s: orc.assoc_chunked_stream(q, k, v, e, s, C),
+                             Q_.numpy(), K_.numpy(), V_.numpy(), e_.numpy(), s_.numpy())
+            O = torch.tensor(np.array([[r[0] for r in row] for row in res]))
+            S = torch.tensor(np.array([[r[1] for r in row] for row in res]))
+            return O, S
+
+        def prefix_fn(s0, inc, upto):
+            return s0 + inc[:upto].sum(0)
+
+        O, S_final = assoc_scan_fwd_cp(Q, K, V, eta, S0, C=C, state_fn=state_fn,
+                                       scan_fn=scan_fn, prefix_fn=prefix_fn)
+        np.save(os.path.join(outdir, f"cp_O_{rank}.npy"), O.numpy())
+        np.save(os.path.join(outdir, f"cp_S_{rank}.npy"), S_final.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_parallel_assoc_scan_over_gloo_ranks(tmp_path, world):
+    """Each rank owns a slice of the sequence; one all-gather of the slices' state increments
+    and a prefix sum give every rank its starting state; the gathered outputs and the final
+    state equal the sequential recurrence."""
+    mp.start_processes(_cp_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    from oracle import ttt_oracle as orc
+    from weight_linear_attention_ttt_b200 import inputs as inp
+
+    x = inp.dual_or_assoc_inputs(2, 2, 256, 8, seed=12, device="cpu", normalise=("Q", "K"),
+                                 eta="sigmoid", w0="normal_0.02")
+    O, S = orc.assoc_scan(x["Q"].double().numpy(), x["K"].double().numpy(),
+                          x["V"].double().numpy(), x["eta"].double().numpy(),
+                          x["W0"].double().numpy())
+    Og = np.concatenate([np.load(tmp_path / f"cp_O_{r}.npy") for r in range(world)], axis=2)
+    np.testing.assert_allclose(Og, O, rtol=1e-10, atol=1e-12)
+    for r in range(world):
+        np.testing.assert_allclose(np.load(tmp_path / f"cp_S_{r}.npy"), S, rtol=1e-10,
+                                   atol=1e-12)

@@ -24,7 +24,8 @@ EXPORTED_SYMBOLS = (
     "ttt_status_string", "ttt_last_error_message", "ttt_version", "ttt_launch_count",
     "ttt_read_device_error",
     "ttt_linear_dual_workspace_size", "ttt_linear_dual_fwd",
-    "ttt_assoc_scan_workspace_size", "ttt_assoc_scan_fwd",
+    "ttt_assoc_scan_workspace_size", "ttt_assoc_scan_fwd", "ttt_assoc_state_fwd",
+    "ttt_state_prefix_sum",
     "inplace_ttt_workspace_size", "inplace_ttt_chunk_fwd",
     "inplace_ttt_noalloc_max_scratch_bytes", "inplace_ttt_chunk_fwd_noalloc",
 )
@@ -69,6 +70,11 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     for name in ("ttt_linear_dual_workspace_size", "ttt_assoc_scan_workspace_size"):
         getattr(lib, name).restype = c_size
         getattr(lib, name).argtypes = [c_int] * 6
+    lib.ttt_assoc_state_fwd.restype = c_int
+    lib.ttt_assoc_state_fwd.argtypes = [vp, vp, fp, c_float, fp, c_int, c_int, c_int, c_int,
+                                        c_int, c_int, vp]
+    lib.ttt_state_prefix_sum.restype = c_int
+    lib.ttt_state_prefix_sum.argtypes = [fp, fp, c_int, c_int, c_int, c_int, c_int, fp, vp]
     lib.inplace_ttt_workspace_size.restype = c_size
     lib.inplace_ttt_workspace_size.argtypes = [c_int] * 4
     lib.inplace_ttt_chunk_fwd.restype = c_int
@@ -159,6 +165,48 @@ def ttt_assoc_scan_fwd(Q, K, V, eta=None, S0=None, *, C: int, eta_scalar: float 
     """Associative (gradient-ascent) linear-attention mode. Returns (O, S_out)."""
     return _state_call("ttt_assoc_scan_fwd", "ttt_assoc_scan_workspace_size", Q, K, V, eta,
                        eta_scalar, S0, C, O, S_out, workspace, stream)
+
+
+def ttt_assoc_state_fwd(K, V, eta=None, *, C: int, eta_scalar: float = 0.0, dS=None,
+                        stream=None):
+    """State increment of a sequence slice: dS = sum_t eta_t k_t^T v_t. Returns dS."""
+    import torch
+
+    lib = load_library()
+    _require(K.dim() == 4 and K.shape == V.shape, "K, V must be [B, H, T, d] of one shape")
+    for t in (K, V):
+        _require(t.is_cuda and t.is_contiguous() and t.dtype == K.dtype,
+                 "K, V must be contiguous CUDA tensors of one dtype")
+    B, H, T, d = K.shape
+    if eta is not None:
+        _require(eta.is_cuda and eta.dtype == torch.float32 and eta.is_contiguous() and
+                 tuple(eta.shape) == (B, H, T), "eta must be a contiguous fp32 [B, H, T] tensor")
+    if dS is None:
+        dS = torch.empty((B, H, d, d), device=K.device, dtype=torch.float32)
+    st = lib.ttt_assoc_state_fwd(_ptr(K), _ptr(V), _ptr(eta), ctypes.c_float(eta_scalar),
+                                 _ptr(dS), B, H, T, d, C, _dtype_code(K), _stream_ptr(stream))
+    _check("ttt_assoc_state_fwd", st)
+    return dS
+
+
+def ttt_state_prefix_sum(S0, increments, upto: int, *, out=None, stream=None):
+    """out = S0 + sum_{r < upto} increments[r]; increments [R, B, H, d, d] fp32."""
+    import torch
+
+    lib = load_library()
+    _require(increments.dim() == 5 and increments.dtype == torch.float32 and
+             increments.is_cuda and increments.is_contiguous(),
+             "increments must be a contiguous fp32 CUDA tensor [R, B, H, d, d]")
+    R, B, H, d, _ = increments.shape
+    if S0 is not None:
+        _require(S0.is_cuda and S0.dtype == torch.float32 and S0.is_contiguous() and
+                 tuple(S0.shape) == (B, H, d, d), "S0 must be fp32 [B, H, d, d]")
+    if out is None:
+        out = torch.empty((B, H, d, d), device=increments.device, dtype=torch.float32)
+    st = lib.ttt_state_prefix_sum(_ptr(S0), _ptr(increments), R, upto, B, H, d, _ptr(out),
+                                  _stream_ptr(stream))
+    _check("ttt_state_prefix_sum", st)
+    return out
 
 
 def inplace_ttt_chunk_fwd(Z, Vhat, W0, eta: float, *, C: int, O=None, W_out=None,

@@ -487,6 +487,33 @@ int launch_chunk(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
 
 bool assoc_supported(int d, int C_, int dt) { return dt == 1 && d == D && C_ == C; }
 
+int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
+  // Pass 1 over the whole sequence as a single superchunk: S_out = sum_t eta_t k_t^T v_t.
+  const int BH = a.B * a.H;
+  CUtensorMap tq, tk, tv, to;
+  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.T, (uint64_t)BH};
+  const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)a.T * D * 2};
+  const uint32_t box[3] = {64, (uint32_t)C, 1};
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_tmap_3d(&tk, a.K, bf, dims, strides, box, sw, ctx.msg) ||
+      !make_tmap_3d(&tv, a.V, bf, dims, strides, box, sw, ctx.msg))
+    return kCuda;
+  tq = tk;  // unused in state-only mode
+  to = tk;
+  AssocParams p;
+  p.eta = a.eta;
+  p.eta_scalar = a.eta_scalar;
+  p.S0 = nullptr;
+  p.S_start = nullptr;
+  p.S_dst = a.S_out;
+  p.T = a.T;
+  p.P = 2;             // parts 0 .. P-2 = the single part [0, T)
+  p.part_len = a.T;
+  p.err = ctx.err;
+  return launch_chunk<true>(tq, tk, tv, to, p, BH * 2, ctx);
+}
+
 size_t assoc_workspace_bytes(int B, int H, int T, int d, int C_) {
   if (d != D || C_ != C || T % C != 0) return 0;
   const int P = choose_parts(B * H, T);

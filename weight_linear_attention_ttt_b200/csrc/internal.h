@@ -67,6 +67,7 @@ int launch_dual_simt(const StateArgs& a, const LaunchCtx& ctx);
 size_t assoc_workspace_bytes(int B, int H, int T, int d, int C);
 bool assoc_supported(int d, int C, int dt);
 int launch_assoc(const StateArgs& a, const LaunchCtx& ctx);
+int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx);
 
 // In-Place W_down.
 size_t inplace_workspace_bytes(int T, int Dff, int D, int C);

@@ -223,6 +223,35 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
   return finish(launch_assoc(a, ctx), msg);
 }
 
+int ttt_assoc_state_fwd(const void* K, const void* V, const float* eta, float eta_scalar,
+                        float* dS, int B, int H, int T, int d, int C, int dt,
+                        cudaStream_t stream) {
+  const std::string f("ttt_assoc_state_fwd");
+  if (!K || !V || !dS) return fail(TTT_ERR_INVALID_ARG, f + ": K, V and dS must be non-null");
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0)
+    return fail(TTT_ERR_INVALID_ARG, f + ": B, H, T, d and C must be positive");
+  if (T % C != 0) return fail(TTT_ERR_INVALID_ARG, f + ": T must be a multiple of C");
+  if (dt != TTT_DTYPE_F32 && dt != TTT_DTYPE_BF16)
+    return fail(TTT_ERR_INVALID_ARG, f + ": dtype must be TTT_DTYPE_F32 or TTT_DTYPE_BF16");
+  const void* ptrs[] = {K, V, eta, dS};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p))
+      return fail(TTT_ERR_INVALID_ARG, f + ": every device pointer must be 16-byte aligned");
+  if (!assoc_supported(d, C, dt))
+    return fail(TTT_ERR_UNSUPPORTED, f + ": supported bf16, d == 128, C == 64");
+  const size_t nx = (size_t)B * H * T * d * 2, ns = (size_t)B * H * d * d * 4;
+  const size_t ne = (size_t)B * H * T * 4;
+  if (overlap(dS, ns, K, nx) || overlap(dS, ns, V, nx) || overlap(dS, ns, eta, ne))
+    return fail(TTT_ERR_INVALID_ARG, f + ": dS must not overlap K, V or eta");
+  StateArgs a{nullptr, K, V, eta, eta_scalar, nullptr, nullptr, dS, B, H, T, d, C, dt,
+              nullptr, 0};
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  return finish(launch_assoc_state(a, ctx), msg);
+}
+
 size_t inplace_ttt_workspace_size(int T, int Dff, int D, int C) {
   if (T <= 0 || Dff <= 0 || D <= 0 || C <= 0) return 0;
   return inplace_workspace_bytes(T, Dff, D, C);
