@@ -13,22 +13,25 @@
 // T/P tokens. Pass 1 (assoc_chunk_kernel<true>) computes every part's state increment except
 // the last; assoc_scan_kernel turns them, with S0, into each part's starting state; pass 2
 // (assoc_chunk_kernel<false>) runs every part from its start, chunk by chunk, and the last part
-// writes S_out. P is chosen so that streams x parts x 2 column halves fill the GPU; with P = 1
-// pass 1 and the scan vanish.
+// writes S_out. With P = 1 pass 1 and the scan vanish.
 //
-// Pass-2 CTA = (stream, part, half of the output columns). The state S^T[half] (64 x 128 fp32)
-// stays in TMEM (M = 64 accumulator) for the whole part. Per chunk:
-//   MMA-S  D_P = Q_c K_c^T                        (A = Q, B = K; both K-major TMA tiles)
-//   warps  mask D_P (s <= t) -> bf16 P tile; eta-scale the V half -> bf16 EV tile
-//   MMA-O  D_O = Q_c bf16(S) + P * EV             (B = bf16 copy of S^T, K-major)
-//   MMA-U  D_S += EV^T K_c                        (A = EV, MN-major; B = K, MN-major)
-//   warps  D_S -> bf16 copy of S^T for the next chunk; D_O -> bf16 O tile -> TMA store
-// Warp 0 issues TMA loads (3-stage ring); warp 1 owns TMEM and issues the MMAs from one thread;
-// warps 2-5 ("attention" group) turn scores into the masked P tile, scale V by eta and drain O;
-// warps 6-9 ("state" group) only refresh the bf16 copy of S after each update. The serial
-// chain per chunk is therefore MMA-U -> S readout -> MMA-U; the attention work of the next
-// chunk and the outputs of this one run beside it. Each group has one warp per TMEM
-// sub-partition.
+// One CTA per (stream, part) holds the whole state. Every d-sized dimension of the chunk
+// contractions is put on the 128-row M side of the tensor core by computing the outputs
+// transposed: with EV = diag(eta) V and P = tril(Q K^T),
+//     O^T = S^T Q^T + EV^T P^T          (M = d_out, N = 64 tokens)
+//     S^T += EV^T K                     (M = d_out, N = d_in, K = 64 tokens)
+// Operands that the CTA itself produces live in TMEM as bf16 and feed the MMAs as the A
+// operand: the bf16 copy of S^T (refreshed after every update) and EV^T (written by the
+// operand warps from the V tile). Only Q, K and the masked score tile P are read from shared
+// memory by the tensor core. TMEM columns: S^T fp32 [0,128), bf16 S^T [128,192), EV^T (x2)
+// [192,256), O^T (x2) [256,384), scores Q K^T (x2, M = 64) [384,512).
+//
+// Warp roles: warp 0 issues the TMA loads (3-stage ring of Q/K/V/eta tiles); warp 1 owns TMEM
+// and issues the MMAs from one thread; warps 2-5 (operand group) write EV^T to TMEM and turn
+// the scores into the masked bf16 P tile; warps 6-9 (state group) convert S^T to its bf16 copy
+// after each update; warps 10-13 (output group) drain O^T through a shared tile and TMA-store
+// it. Each group has one warp per TMEM sub-partition. The serial chain per chunk is
+// update -> bf16 copy -> update; everything else overlaps it.
 #include <algorithm>
 #include <cstdlib>
 
@@ -39,30 +42,34 @@
 namespace ttt {
 namespace {
 
-constexpr int D = 128;       // head dim
-constexpr int C = 64;        // chunk
-constexpr int HALF = 64;     // output columns per CTA
-constexpr int THREADS = 320;   // TMA warp, MMA warp, 4 attention warps, 4 state warps
-constexpr int STAGES = 3;
+constexpr int D = 128;         // head dim
+constexpr int C = 64;          // chunk
+constexpr int THREADS = 448;   // TMA warp, MMA warp, operand / state / output groups of 4 warps
 
-// shared-memory map (bytes from the 1024-aligned base)
-constexpr int Q_BYTES = C * D * 2;        // two [64][64] sub-tiles
-constexpr int K_BYTES = C * D * 2;
-constexpr int V_BYTES = C * HALF * 2;     // one [64][64] sub-tile
-constexpr int ETA_BYTES = 1024;
-constexpr int STAGE_BYTES = Q_BYTES + K_BYTES + V_BYTES + ETA_BYTES;
-constexpr int P_OFF = STAGES * STAGE_BYTES;              // 2 x [64 t][64 s] bf16
-constexpr int EV_OFF = P_OFF + 2 * 8192;                 // 2 x [64 s][64 dout] bf16
-constexpr int SB_OFF = EV_OFF + 2 * 8192;                // 2 x S^T bf16 [64 dout][128 din]
-constexpr int O_OFF = SB_OFF + 2 * 16384;                // 2 x [64 t][64 dout] bf16
-constexpr int BAR_OFF = O_OFF + 2 * 8192;
-constexpr int SMEM = 1024 + BAR_OFF + 256;
-static_assert(SMEM <= 227 * 1024, "shared memory");
+// shared-memory map (bytes from the 1024-aligned base); pass 1 loads no Q and writes no O
+template <bool SO>
+struct Smem {
+  static constexpr int Q_BYTES = SO ? 0 : C * D * 2;   // two [64 t][64 d_in] sub-tiles
+  static constexpr int K_BYTES = C * D * 2;            // two [64 s][64 d_in] sub-tiles
+  static constexpr int V_BYTES = C * D * 2;            // two [64 s][64 d_out] sub-tiles
+  static constexpr int K_OFF = Q_BYTES;
+  static constexpr int V_OFF = K_OFF + K_BYTES;
+  static constexpr int ETA_OFF = V_OFF + V_BYTES;
+  static constexpr int STAGE = ETA_OFF + 1024;         // eta (256 B) padded to keep alignment
+  static constexpr int STAGES = SO ? 5 : 3;
+  static constexpr int P_OFF = STAGES * STAGE;                // 2 x [64 t][64 s] bf16
+  static constexpr int O_OFF = P_OFF + (SO ? 0 : 2 * 8192);   // 2 x [64 t][128 d_out] bf16
+  static constexpr int BAR_OFF = O_OFF + (SO ? 0 : 2 * 16384);
+  static constexpr int BYTES = 1024 + BAR_OFF + 256;
+  static_assert(BYTES <= 227 * 1024, "shared memory");
+};
 
 // TMEM columns
-constexpr uint32_t TM_S = 0;     // 128 columns: S^T half (M = 64)
-constexpr uint32_t TM_P = 128;   // 2 x 64: scores
-constexpr uint32_t TM_O = 256;   // 2 x 64: outputs
+constexpr uint32_t TM_S = 0;      // S^T fp32, lanes = d_out, columns = d_in
+constexpr uint32_t TM_SBF = 128;  // bf16 S^T (64 columns of d_in pairs)
+constexpr uint32_t TM_EV = 192;   // 2 x 32: bf16 EV^T (token pairs)
+constexpr uint32_t TM_O = 256;    // 2 x 64: O^T fp32, lanes = d_out, columns = tokens
+constexpr uint32_t TM_P = 384;    // 2 x 64: Q K^T (M = 64)
 constexpr uint32_t TM_COLS = 512;
 
 struct AssocParams {
@@ -78,232 +85,341 @@ struct AssocParams {
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
+// Barrier over `threads` threads that also returns whether any of them passed `pred` = true.
+__device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
 
-// Row r (0..63) of an M = 64 accumulator lives in TMEM lane 32 * (r / 16) + r % 16: compute
-// warp with sub-partition q holds rows 16q .. 16q+15 in its threads 0..15.
-template <bool STATE_ONLY>
+template <bool SO>
 __global__ void __launch_bounds__(THREADS, 1)
     assoc_chunk_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
                        const __grid_constant__ CUtensorMap tmO, const AssocParams p) {
+  using L = Smem<SO>;
+  constexpr int ST = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar = sbase + BAR_OFF;
-  const uint32_t full = bar, empty = bar + 8 * STAGES;          // stage ring
-  const uint32_t pfull = bar + 48, pempty = bar + 64;           // score accumulators
-  const uint32_t aready = bar + 80;                             // P / EV tiles written
-  const uint32_t sdone = bar + 96;                              // state update finished
-  const uint32_t sready = bar + 104;                            // bf16 S copy written (x2)
-  const uint32_t ofull = bar + 120, oempty = bar + 136;         // output accumulators
-  const uint32_t tslot = bar + 160;
-  const uint32_t evfree = bar + 168;                            // pass 1: EV tile reusable (x2)
+  const uint32_t bar = sbase + L::BAR_OFF;
+  const uint32_t full = bar, empty = bar + 40;                  // stage ring (up to 5)
+  const uint32_t pfull = bar + 80;                              // score accumulators (x2)
+  const uint32_t pready = bar + 112;                            // P tile written (x2)
+  const uint32_t evready = bar + 128;                           // EV^T written (x2)
+  const uint32_t afree = bar + 144;                             // EV^T and P tile reusable (x2)
+  const uint32_t ofull = bar + 160, oempty = bar + 176;         // output accumulators (x2)
+  const uint32_t sdone = bar + 192;                             // state update finished
+  const uint32_t sready = bar + 200;                            // bf16 S^T written
+  const uint32_t tslot = bar + 208;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // pass 2: blockIdx = (stream * P + part) * 2 + half; pass 1 only covers parts 0 .. P-2
-  const int nparts = STATE_ONLY ? p.P - 1 : p.P;
-  const int half = blockIdx.x & 1;
-  const int sp = blockIdx.x >> 1;
-  const int stream = sp / nparts, part = sp % nparts;
+  // blockIdx = stream * nparts + part; pass 1 only covers parts 0 .. P-2
+  const int nparts = SO ? p.P - 1 : p.P;
+  const int stream = blockIdx.x / nparts, part = blockIdx.x % nparts;
   const int tok0 = part * p.part_len;
   const int nch = p.part_len / C;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < ST; ++s) {
       mbar_init(full + 8 * s, 1);
-      mbar_init(empty + 8 * s, 5);  // MMA commit + 4 compute warps
+      mbar_init(empty + 8 * s, 5);  // MMA commit + 4 operand warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(pfull + 8 * b, 1);
-      mbar_init(pempty + 8 * b, 4);
-      mbar_init(aready + 8 * b, 4);
-      mbar_init(sready + 8 * b, 4);
+      mbar_init(pready + 8 * b, 4);
+      mbar_init(evready + 8 * b, 4);
+      mbar_init(afree + 8 * b, 1);
       mbar_init(ofull + 8 * b, 1);
       mbar_init(oempty + 8 * b, 4);
     }
     mbar_init(sdone, 1);
-    mbar_init(evfree, 1);
-    mbar_init(evfree + 8, 1);
+    mbar_init(sready, 4);
     fence_mbar_init();
   }
   if (warp == 1) umma::tmem_alloc(tslot, TM_COLS);
   umma::fence_before();
   __syncthreads();
   umma::fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + BAR_OFF + 160);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::BAR_OFF + 208);
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      if (!STATE_ONLY) prefetch_tmap(&tmQ);
-      const uint32_t bytes = K_BYTES + V_BYTES + (STATE_ONLY ? 0 : Q_BYTES) + (p.eta ? C * 4 : 0);
+      if (!SO) prefetch_tmap(&tmQ);
+      const uint32_t bytes = L::Q_BYTES + L::K_BYTES + L::V_BYTES + (p.eta ? C * 4 : 0);
       for (int c = 0; c < nch; ++c) {
-        const int s = c % STAGES;
-        if (c >= STAGES && !mbar_wait(empty + 8 * s, ((c / STAGES) - 1) & 1, p.err)) break;
+        const int s = c % ST;
+        if (c >= ST && !mbar_wait(empty + 8 * s, ((c / ST) - 1) & 1, p.err)) break;
         const uint32_t fb = full + 8 * s;
-        const uint32_t st = sbase + s * STAGE_BYTES;
+        const uint32_t st = sbase + s * L::STAGE;
         const int t0 = tok0 + c * C;
         mbar_arrive_expect_tx(fb, bytes);
-        if (!STATE_ONLY) {
+        if (!SO) {
           tma_load_3d(st, &tmQ, fb, 0, t0, stream);
           tma_load_3d(st + 8192, &tmQ, fb, 64, t0, stream);
         }
-        tma_load_3d(st + Q_BYTES, &tmK, fb, 0, t0, stream);
-        tma_load_3d(st + Q_BYTES + 8192, &tmK, fb, 64, t0, stream);
-        tma_load_3d(st + Q_BYTES + K_BYTES, &tmV, fb, HALF * half, t0, stream);
+        tma_load_3d(st + L::K_OFF, &tmK, fb, 0, t0, stream);
+        tma_load_3d(st + L::K_OFF + 8192, &tmK, fb, 64, t0, stream);
+        tma_load_3d(st + L::V_OFF, &tmV, fb, 0, t0, stream);
+        tma_load_3d(st + L::V_OFF + 8192, &tmV, fb, 64, t0, stream);
         if (p.eta)
-          bulk_load(st + Q_BYTES + K_BYTES + V_BYTES, p.eta + (size_t)stream * p.T + t0, C * 4,
-                    fb);
+          bulk_load(st + L::ETA_OFF, p.eta + (size_t)stream * p.T + t0, C * 4, fb);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t id_s = umma::idesc_bf16(64, 64, false, false);   // Q K^T
-      const uint32_t id_o1 = umma::idesc_bf16(64, 64, false, false);  // Q S
-      const uint32_t id_o2 = umma::idesc_bf16(64, 64, false, true);   // P EV
-      const uint32_t id_u = umma::idesc_bf16(64, 128, true, true);    // EV^T K
-      auto mma_scores = [&](int c) -> bool {
-        const int s = c % STAGES, b = c & 1;
-        if (!mbar_wait(full + 8 * s, (c / STAGES) & 1, p.err)) return false;
-        if (c >= 2 && !mbar_wait(pempty + 8 * b, ((c >> 1) - 1) & 1, p.err)) return false;
-        umma::fence_after();
-        const uint32_t sQ = sbase + s * STAGE_BYTES, sK = sQ + Q_BYTES;
+    // The whole warp runs this loop: every lane waits, the wait results are made warp-uniform,
+    // and one elected lane issues each MMA / commit, so no divergent branch surrounds them.
+    const uint32_t id_s = umma::idesc_bf16(64, 64, false, false);    // Q K^T
+    const uint32_t id_o = umma::idesc_bf16(128, 64, false, false);   // S^T Q^T, EV^T P^T
+    const uint32_t id_u = umma::idesc_bf16(128, 128, false, true);   // EV^T K
+    auto wait = [&](uint32_t b_, uint32_t parity) -> bool {
+      return mbar_wait_warp(b_, parity, p.err);
+    };
+    auto scores = [&](int c) {
+      const int s = c % ST, b = c & 1;
+      const uint32_t sQ = sbase + s * L::STAGE, sK = sQ + L::K_OFF;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
-          umma::mma_ss(tmem + TM_P + 64 * b, umma::desc_kmajor(sQ + o), umma::desc_kmajor(sK + o),
-                       id_s, ks > 0);
-        }
-        umma::commit(pfull + 8 * b);
-        return true;
-      };
-      bool ok = true;
-      if (!STATE_ONLY) {
-        ok = mma_scores(0);
-        if (ok && nch > 1) ok = mma_scores(1);
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
+        umma::mma_ss_elect(tmem + TM_P + 64 * b, umma::desc_kmajor(sQ + o),
+                           umma::desc_kmajor(sK + o), id_s, ks > 0);
       }
-      for (int c = 0; ok && c < nch; ++c) {
-        const int s = c % STAGES, b = c & 1;
-        const uint32_t sQ = sbase + s * STAGE_BYTES, sK = sQ + Q_BYTES;
-        const uint32_t sEV = sbase + EV_OFF + 8192 * b;
-        if (STATE_ONLY && !mbar_wait(full + 8 * s, (c / STAGES) & 1, p.err)) break;
-        if (!mbar_wait(aready + 8 * b, (c >> 1) & 1, p.err)) break;
-        if (!STATE_ONLY && !mbar_wait(sready + 8 * b, (c >> 1) & 1, p.err)) break;
+      umma::commit_elect(pfull + 8 * b);
+    };
+    bool ok = true;
+    if (!SO) {
+      ok = wait(full, 0);
+      if (ok) {
         umma::fence_after();
-        // state update first: it heads the serial chain
+        scores(0);
+      }
+    }
+    for (int c = 0; ok && c < nch; ++c) {
+      const int s = c % ST, b = c & 1;
+      const uint32_t sQ = sbase + s * L::STAGE, sK = sQ + L::K_OFF;
+      const uint32_t aEV = tmem + TM_EV + 32 * b;
+      const uint32_t dO = tmem + TM_O + 64 * b;
+      if (SO) ok = wait(full + 8 * s, (c / ST) & 1);
+      ok = ok && wait(evready + 8 * b, (c >> 1) & 1);
+      if (!SO) {
+        ok = ok && wait(sready, c & 1);
+        if (c >= 2) ok = ok && wait(oempty + 8 * b, ((c >> 1) - 1) & 1);
+      }
+      if (!ok) break;
+      umma::fence_after();
+      if (!SO) {
+        // O^T = S^T Q^T: reads the bf16 copy of S before this chunk's update
 #pragma unroll
-        for (int ks = 0; ks < C / 16; ++ks)
-          umma::mma_ss(tmem + TM_S, umma::desc_mnmajor(sEV + 2048 * ks, 8192),
-                       umma::desc_mnmajor(sK + 2048 * ks, 8192), id_u,
-                       STATE_ONLY ? (c > 0 || ks > 0) : true);
-        // Pass 2 signals every update (the state warps refresh the bf16 copy); pass 1 only
-        // frees the EV tile per chunk and signals the final update.
-        if (!STATE_ONLY || c + 1 == nch) umma::commit(sdone);
-        if (STATE_ONLY) umma::commit(evfree + 8 * b);
-        if (!STATE_ONLY) {
-          if (c >= 2 && !mbar_wait(oempty + 8 * b, ((c >> 1) - 1) & 1, p.err)) break;
-          umma::fence_after();
-          const uint32_t sS = sbase + SB_OFF + 16384 * b, sP = sbase + P_OFF + 8192 * b;
-          const uint32_t dO = tmem + TM_O + 64 * b;
+        for (int ks = 0; ks < D / 16; ++ks)
+          umma::mma_ts_elect(dO, tmem + TM_SBF + 8 * ks,
+                             umma::desc_kmajor(sQ + (ks >> 2) * 8192 + (ks & 3) * 32), id_o,
+                             ks > 0);
+      }
+      // S^T += EV^T K (heads the serial chain)
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
-            umma::mma_ss(dO, umma::desc_kmajor(sQ + o), umma::desc_kmajor(sS + o), id_o1, ks > 0);
-          }
+      for (int ks = 0; ks < C / 16; ++ks)
+        umma::mma_ts_elect(tmem + TM_S, aEV + 8 * ks, umma::desc_mnmajor(sK + 2048 * ks, 8192),
+                           id_u, SO ? (c > 0 || ks > 0) : true);
+      if (SO) {
+        // pass 1 signals only the final update
+        if (c + 1 == nch) umma::commit_elect(sdone);
+        umma::commit_elect(afree + 8 * b);
+        umma::commit_elect(empty + 8 * s);
+        continue;
+      }
+      umma::commit_elect(sdone);   // the state warps refresh the bf16 copy
+      if (!wait(pready + 8 * b, (c >> 1) & 1)) break;
+      umma::fence_after();
+      const uint32_t sP = sbase + L::P_OFF + 8192 * b;
+      // O^T += EV^T P^T
 #pragma unroll
-          for (int ks = 0; ks < C / 16; ++ks)
-            umma::mma_ss(dO, umma::desc_kmajor(sP + 32 * ks),
-                         umma::desc_mnmajor(sEV + 2048 * ks, 8192), id_o2, true);
-          umma::commit(ofull + 8 * b);
-        }
-        umma::commit(empty + 8 * s);
-        if (!STATE_ONLY && c + 2 < nch && !mma_scores(c + 2)) break;
+      for (int ks = 0; ks < C / 16; ++ks)
+        umma::mma_ts_elect(dO, aEV + 8 * ks, umma::desc_kmajor(sP + 32 * ks), id_o, true);
+      umma::commit_elect(ofull + 8 * b);
+      umma::commit_elect(afree + 8 * b);
+      umma::commit_elect(empty + 8 * s);
+      if (c + 1 < nch) {
+        // The score buffer of chunk c+1 was last read for chunk c-1; those reads finished
+        // before the operand warps signalled pready(c-1), which this warp has seen.
+        const int s1 = (c + 1) % ST;
+        if (!wait(full + 8 * s1, ((c + 1) / ST) & 1)) break;
+        umma::fence_after();
+        scores(c + 1);
       }
     }
   } else if (warp < 6) {
-    // ---------------------------------------------------------------- attention warps 2..5
+    // ---------------------------------------------------------------- operand warps 2..5
     const int q = warp & 3;
-    const int ctid = threadIdx.x - 64;        // 0..127
-    const bool rowthr = lane < 16;            // holds an M = 64 accumulator row
-    const int r = 16 * q + lane;              // that row (token t of the chunk)
+    const int dout = 32 * q + lane;           // TMEM lane = output column
     const uint32_t tl = (uint32_t)(32 * q) << 16;
-
-    // Produce chunk c's operands: masked scores -> P tile, eta * V half -> EV tile.
-    auto produce = [&](int c) -> bool {
-      const int s = c % STAGES, b = c & 1;
-      const uint8_t* stg = smem + s * STAGE_BYTES;
-      if (!STATE_ONLY) {
-        if (!mbar_wait(pfull + 8 * b, (c >> 1) & 1, p.err)) return false;
-        umma::fence_after();
-        uint32_t v0[32], v1[32];
-        umma::ld32x32(tmem + tl + TM_P + 64 * b, v0);
-        umma::ld32x32(tmem + tl + TM_P + 64 * b + 32, v1);
-        umma::wait_ld();
-        umma::reg_fence(v0);
-        umma::reg_fence(v1);
-        umma::fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(pempty + 8 * b);
-        if (rowthr) {
-          const uint32_t prow = sbase + P_OFF + 8192 * b;
-#pragma unroll
-          for (int j = 0; j < 64; j += 8) {
-            float f[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int sidx = j + e;
-              const float x = __uint_as_float(sidx < 32 ? v0[sidx] : v1[sidx - 32]);
-              f[e] = sidx <= r ? x : 0.f;
-            }
-            sts128(prow + swz<128>(r * 128 + 2 * j),
-                   make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
-                              pack_bf16(f[6], f[7])));
-          }
-        }
-      }
-      if (!mbar_wait(full + 8 * s, (c / STAGES) & 1, p.err)) return false;
+    const bool rowthr = lane < 16;            // holds an M = 64 score row
+    const int r = 16 * q + lane;              // that row (token t of the chunk)
+    for (int c = 0; c < nch; ++c) {
+      const int s = c % ST, b = c & 1;
+      const uint32_t stg = sbase + s * L::STAGE;
+      if (!mbar_wait(full + 8 * s, (c / ST) & 1, p.err)) break;
+      if (c >= 2 && !mbar_wait(afree + 8 * b, ((c >> 1) - 1) & 1, p.err)) break;
+      // EV^T: column j of this lane holds (eta_2j v_2j, eta_2j+1 v_2j+1)[dout]
       {
-        const uint32_t vt = sbase + s * STAGE_BYTES + Q_BYTES + K_BYTES;
-        const uint32_t et = vt + V_BYTES;
-        const uint32_t ev = sbase + EV_OFF + 8192 * b;
-        // 8192 bytes = 512 x 16-byte pieces; piece i covers row (i / 8), eight columns; the
-        // EV tile uses the same swizzled layout as the TMA tile.
-        uint4 x[4];
-        float e[4];
+        const uint32_t vcol = stg + L::V_OFF + (dout >> 6) * 8192;
+        const uint32_t cb = 2 * (dout & 63);
+        uint32_t ev[32];
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          const int i = ctid + 128 * it;
-          x[it] = lds128(vt + swz<128>((i >> 3) * 128 + (i & 7) * 16));
-          e[it] = p.eta ? ldsf(et + 4 * (i >> 3)) : p.eta_scalar;
+        for (int j4 = 0; j4 < C / 4; ++j4) {
+          float e[4];
+          if (p.eta) {
+            const uint4 ee = lds128(stg + L::ETA_OFF + 16 * j4);
+            e[0] = __uint_as_float(ee.x);
+            e[1] = __uint_as_float(ee.y);
+            e[2] = __uint_as_float(ee.z);
+            e[3] = __uint_as_float(ee.w);
+          } else {
+            e[0] = e[1] = e[2] = e[3] = p.eta_scalar;
+          }
+          float f[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int tok = 4 * j4 + u;
+            f[u] = __uint_as_float(ldsu16(vcol + swz<128>(tok * 128 + cb)) << 16) * e[u];
+          }
+          ev[2 * j4] = pack_bf16(f[0], f[1]);
+          ev[2 * j4 + 1] = pack_bf16(f[2], f[3]);
         }
+        umma::st32x32(tmem + tl + TM_EV + 32 * b, ev);
+        umma::wait_st();
+      }
+      umma::fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(evready + 8 * b);
+        mbar_arrive(empty + 8 * s);
+      }
+      if (SO) continue;
+      // masked scores -> P tile [t][s]
+      if (!mbar_wait(pfull + 8 * b, (c >> 1) & 1, p.err)) break;
+      umma::fence_after();
+      uint32_t v0[32], v1[32];
+      umma::ld32x32(tmem + tl + TM_P + 64 * b, v0);
+      umma::ld32x32(tmem + tl + TM_P + 64 * b + 32, v1);
+      umma::wait_ld();
+      umma::reg_fence(v0);
+      umma::reg_fence(v1);
+      umma::fence_before();
+      if (rowthr) {
+        const uint32_t prow = sbase + L::P_OFF + 8192 * b;
 #pragma unroll
-        for (int it = 0; it < 4; ++it) {
-          const int i = ctid + 128 * it;
-          const float f = e[it];
-          sts128(ev + swz<128>((i >> 3) * 128 + (i & 7) * 16),
-                 make_uint4(pack_bf16(bf16_lo(x[it].x) * f, bf16_hi(x[it].x) * f),
-                            pack_bf16(bf16_lo(x[it].y) * f, bf16_hi(x[it].y) * f),
-                            pack_bf16(bf16_lo(x[it].z) * f, bf16_hi(x[it].z) * f),
-                            pack_bf16(bf16_lo(x[it].w) * f, bf16_hi(x[it].w) * f)));
+        for (int j = 0; j < 64; j += 8) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int sidx = j + e;
+            const float x = __uint_as_float(sidx < 32 ? v0[sidx] : v1[sidx - 32]);
+            f[e] = sidx <= r ? x : 0.f;
+          }
+          sts128(prow + swz<128>(r * 128 + 2 * j),
+                 make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
+                            pack_bf16(f[6], f[7])));
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(aready + 8 * b);
-        mbar_arrive(empty + 8 * s);
+      if (lane == 0) mbar_arrive(pready + 8 * b);
+    }
+  } else if (warp < 10) {
+    // ---------------------------------------------------------------- state warps 6..9
+    const int q = warp & 3;
+    const int dout = 32 * q + lane;
+    const uint32_t tl = (uint32_t)(32 * q) << 16;
+
+    // fp32 S^T row (this lane) -> bf16 copy used as the A operand of O^T = S^T Q^T
+    auto refresh = [&]() {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t a0[32], a1[32], o[32];
+        umma::ld32x32(tmem + tl + TM_S + 64 * h, a0);
+        umma::ld32x32(tmem + tl + TM_S + 64 * h + 32, a1);
+        umma::wait_ld();
+        umma::reg_fence(a0);
+        umma::reg_fence(a1);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          o[j] = pack_bf16(__uint_as_float(a0[2 * j]), __uint_as_float(a0[2 * j + 1]));
+          o[16 + j] = pack_bf16(__uint_as_float(a1[2 * j]), __uint_as_float(a1[2 * j + 1]));
+        }
+        umma::st32x32(tmem + tl + TM_SBF + 32 * h, o);
       }
-      return true;
+      umma::wait_st();
+      umma::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sready);
     };
-    // Drain chunk c's outputs: D_O -> bf16 O tile -> TMA store.
-    auto consume = [&](int c) -> bool {
+
+    bool ok = true;
+    if (!SO) {
+      // starting state S (d_in x d_out, row-major) -> S^T in TMEM and its bf16 copy
+      const float* src = nullptr;
+      if (part == 0) src = p.S0 ? p.S0 + (size_t)stream * D * D : nullptr;
+      else src = p.S_start + ((size_t)stream * (p.P - 1) + (part - 1)) * D * D;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          v[j] = __float_as_uint(src ? src[(32 * cc + j) * D + dout] : 0.f);
+        umma::st32x32(tmem + tl + TM_S + 32 * cc, v);
+      }
+      umma::wait_st();
+      refresh();
+      for (int c = 0; c < nch; ++c) {
+        if (!mbar_wait(sdone, c & 1, p.err)) { ok = false; break; }
+        umma::fence_after();
+        if (c + 1 < nch) refresh();
+      }
+    } else {
+      ok = mbar_wait(sdone, 0, p.err);
+      umma::fence_after();
+    }
+    // ---- final state of the part: increment (pass 1) or S_out (pass 2, last part)
+    if (ok && (SO || part == p.P - 1)) {
+      float* dst = SO ? p.S_dst + ((size_t)stream * (p.P - 1) + part) * D * D
+                      : p.S_dst + (size_t)stream * D * D;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        umma::ld32x32(tmem + tl + TM_S + 32 * cc, v);
+        umma::wait_ld();
+        umma::reg_fence(v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dst[(32 * cc + j) * D + dout] = __uint_as_float(v[j]);
+      }
+    }
+  } else if (!SO) {
+    // ---------------------------------------------------------------- output warps 10..13
+    const int q = warp & 3;
+    const int dout = 32 * q + lane;
+    const uint32_t tl = (uint32_t)(32 * q) << 16;
+    const int otid = threadIdx.x - 320;        // 0..127
+    const bool odd = lane & 1;
+    // Lane pairs (2i, 2i+1) exchange one value per token pair (t, t+4) so that each lane
+    // stores a 32-bit word of two adjacent output columns: the even lane row t, the odd lane
+    // row t+4 (the two rows fall in disjoint bank halves of the swizzled tile).
+    const uint32_t ocol = (dout >> 6) * 8192;
+    const uint32_t cb = 2 * ((dout & 63) & ~1);
+    for (int c = 0; c < nch; ++c) {
       const int b = c & 1;
-      if (!mbar_wait(ofull + 8 * b, (c >> 1) & 1, p.err)) return false;
+      const bool got = mbar_wait(ofull + 8 * b, (c >> 1) & 1, p.err);
+      if (named_bar_or(2, 128, !got)) break;
       umma::fence_after();
       uint32_t v0[32], v1[32];
       umma::ld32x32(tmem + tl + TM_O + 64 * b, v0);
@@ -314,122 +430,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       umma::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(oempty + 8 * b);
-      if (rowthr) {
-        const uint32_t orow = sbase + O_OFF + 8192 * b;
+      const uint32_t so = sbase + L::O_OFF + 16384 * b + ocol;
 #pragma unroll
-        for (int j = 0; j < 64; j += 8) {
-          const uint32_t* vv = j < 32 ? v0 + j : v1 + (j - 32);
-          sts128(orow + swz<128>(r * 128 + 2 * j),
-                 make_uint4(pack_bf16(__uint_as_float(vv[0]), __uint_as_float(vv[1])),
-                            pack_bf16(__uint_as_float(vv[2]), __uint_as_float(vv[3])),
-                            pack_bf16(__uint_as_float(vv[4]), __uint_as_float(vv[5])),
-                            pack_bf16(__uint_as_float(vv[6]), __uint_as_float(vv[7]))));
-        }
+      for (int t = 0; t < C; ++t) {
+        if (t & 4) continue;
+        const uint32_t* vv = t < 32 ? v0 : v1;
+        const int tt = t & 31;
+        const float a = __uint_as_float(vv[tt]), a4 = __uint_as_float(vv[tt + 4]);
+        const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
+        const uint32_t w = odd ? pack_bf16(y, a4) : pack_bf16(a, y);
+        const int row = odd ? t + 4 : t;
+        sts32(so + swz<128>(row * 128 + cb), w);
       }
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (ctid == 0) {
-        tma_store_3d(&tmO, sbase + O_OFF + 8192 * b, HALF * half, tok0 + c * C, stream);
+      named_bar_sync(2, 128);
+      if (otid == 0) {
+        const uint32_t sO = sbase + L::O_OFF + 16384 * b;
+        tma_store_3d(&tmO, sO, 0, tok0 + c * C, stream);
+        tma_store_3d(&tmO, sO + 8192, 64, tok0 + c * C, stream);
         bulk_commit();
-        bulk_wait_read<1>();
+        bulk_wait_read<1>();  // the other staging buffer is free again
       }
-      named_bar_sync(1, 128);
-      return true;
-    };
-    // Chunk c+1's operands are produced before chunk c's outputs are drained, so the MMA
-    // thread always has the next chunk's P / EV when the state chain allows it to go on.
-    // Buffer (c+1) % 2 is free: chunk c-1's MMAs finished before its outputs were drained.
-    bool ok = produce(0);
-    for (int c = 0; ok && c < nch; ++c) {
-      // pass 1 has no outputs to wait for: wait until the update of chunk c-1 released its
-      // EV tile instead.
-      if (STATE_ONLY && c >= 1 && c + 1 < nch &&
-          !mbar_wait(evfree + 8 * ((c + 1) & 1), (((c + 1) >> 1) - 1) & 1, p.err))
-        break;
-      if (c + 1 < nch && !produce(c + 1)) break;
-      if (!STATE_ONLY && !consume(c)) break;
+      named_bar_sync(2, 128);
     }
-    if (ctid == 0) bulk_wait<0>();
-  } else {
-    // ---------------------------------------------------------------- state warps 6..9
-    const int q = warp & 3;
-    const bool rowthr = lane < 16;
-    const int r = 16 * q + lane;              // row of S^T[half] = output column index
-    const uint32_t tl = (uint32_t)(32 * q) << 16;
-    const int dcol = HALF * half + r;         // global output column of S row r
-
-    // Writes the fp32 state rows in TMEM as the bf16 copy (K-major [64 dout][128 din]).
-    auto to_bf16 = [&](int nb) {
-      const uint32_t sb = sbase + SB_OFF + 16384 * nb;
-      uint32_t v[2][32];
-      umma::ld32x32(tmem + tl + TM_S, v[0]);
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        umma::wait_ld();
-        umma::reg_fence(v[cc & 1]);
-        if (cc + 1 < 4) umma::ld32x32(tmem + tl + TM_S + 32 * (cc + 1), v[(cc + 1) & 1]);
-        const uint32_t* vv = v[cc & 1];
-        if (rowthr) {
-          const uint32_t row = sb + (cc >> 1) * 8192;
-#pragma unroll
-          for (int j = 0; j < 32; j += 8) {
-            const int k = (32 * cc + j) & 63;
-            sts128(row + swz<128>(r * 128 + 2 * k),
-                   make_uint4(pack_bf16(__uint_as_float(vv[j]), __uint_as_float(vv[j + 1])),
-                              pack_bf16(__uint_as_float(vv[j + 2]), __uint_as_float(vv[j + 3])),
-                              pack_bf16(__uint_as_float(vv[j + 4]), __uint_as_float(vv[j + 5])),
-                              pack_bf16(__uint_as_float(vv[j + 6]), __uint_as_float(vv[j + 7]))));
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      umma::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sready + 8 * nb);
-    };
-
-    // Initial state S^T[half] -> TMEM (fp32) and its bf16 copy for chunk 0.
-    if (!STATE_ONLY) {
-      const float* src = nullptr;
-      if (part == 0) src = p.S0 ? p.S0 + (size_t)stream * D * D : nullptr;
-      else src = p.S_start + ((size_t)stream * (p.P - 1) + (part - 1)) * D * D;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          v[j] = __float_as_uint((rowthr && src) ? src[(32 * cc + j) * D + dcol] : 0.f);
-        umma::st32x32(tmem + tl + TM_S + 32 * cc, v);
-      }
-      umma::wait_st();
-      to_bf16(0);
-    }
-    bool ok = true;
-    if (STATE_ONLY) {
-      ok = mbar_wait(sdone, 0, p.err);
-      umma::fence_after();
-    } else {
-      for (int c = 0; c < nch; ++c) {
-        if (!mbar_wait(sdone, c & 1, p.err)) { ok = false; break; }
-        umma::fence_after();
-        if (c + 1 < nch) to_bf16((c + 1) & 1);
-      }
-    }
-    // ---- final state of the part: increment (pass 1) or S_out (pass 2, last part)
-    if (ok && (STATE_ONLY || part == p.P - 1)) {
-      float* dst = STATE_ONLY ? p.S_dst + ((size_t)stream * (p.P - 1) + part) * D * D
-                              : p.S_dst + (size_t)stream * D * D;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        umma::ld32x32(tmem + tl + TM_S + 32 * cc, v);
-        umma::wait_ld();
-        umma::reg_fence(v);
-        if (rowthr)
-#pragma unroll
-          for (int j = 0; j < 32; ++j) dst[(32 * cc + j) * D + dcol] = __uint_as_float(v[j]);
-      }
-    }
+    if (otid == 0) bulk_wait<0>();
   }
   umma::fence_before();
   __syncthreads();
@@ -460,7 +484,7 @@ int choose_parts(int streams, int T) {
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   int P = 1;
-  while (nchunks % (2 * P) == 0 && streams * 2 * (2 * P) <= sms) P *= 2;
+  while (nchunks % (2 * P) == 0 && streams * (2 * P) <= sms) P *= 2;
   return P;
 }
 
@@ -468,12 +492,13 @@ template <bool STATE_ONLY>
 int launch_chunk(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const CUtensorMap& to, const AssocParams& p, int grid, const LaunchCtx& ctx) {
   auto kern = assoc_chunk_kernel<STATE_ONLY>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Smem<STATE_ONLY>::BYTES);
   if (e != cudaSuccess) {
     *ctx.msg = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
     return kCuda;
   }
-  kern<<<grid, THREADS, SMEM, ctx.stream>>>(tq, tk, tv, to, p);
+  kern<<<grid, THREADS, Smem<STATE_ONLY>::BYTES, ctx.stream>>>(tq, tk, tv, to, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *ctx.msg = std::string("assoc launch: ") + cudaGetErrorString(e);
@@ -511,7 +536,7 @@ int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
   p.P = 2;             // parts 0 .. P-2 = the single part [0, T)
   p.part_len = a.T;
   p.err = ctx.err;
-  return launch_chunk<true>(tq, tk, tv, to, p, BH * 2, ctx);
+  return launch_chunk<true>(tq, tk, tv, to, p, BH, ctx);
 }
 
 size_t assoc_workspace_bytes(int B, int H, int T, int d, int C_) {
@@ -550,7 +575,7 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   p.err = ctx.err;
   if (P > 1) {
     p.S_dst = static_cast<float*>(a.ws);
-    int st = launch_chunk<true>(tq, tk, tv, to, p, BH * (P - 1) * 2, ctx);
+    int st = launch_chunk<true>(tq, tk, tv, to, p, BH * (P - 1), ctx);
     if (st != kOk) return st;
     assoc_scan_kernel<<<dim3(D * D / 256, BH), 256, 0, ctx.stream>>>(a.S0, p.S_dst, P);
     cudaError_t e = cudaGetLastError();
@@ -561,7 +586,7 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
     count_launch();
   }
   p.S_dst = a.S_out;
-  return launch_chunk<false>(tq, tk, tv, to, p, BH * P * 2, ctx);
+  return launch_chunk<false>(tq, tk, tv, to, p, BH * P, ctx);
 }
 
 }  // namespace ttt

@@ -47,11 +47,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete. Gives up after `limit_ns` of
-// global time, raises the error word and returns false; the caller then leaves its loop.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err,
-                                          uint64_t limit_ns = 4000000000ull) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of a bounded wait: spins until the phase with the given parity completes or
+// `limit_ns` of global time passes, then raises the error word and returns false. Kept out of
+// line so that the inline fast path of mbar_wait is one try_wait and a branch.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, unsigned* err,
+                                                   uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (global_timer_ns() - t0 > limit_ns) {
@@ -60,6 +60,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
     }
   }
   return true;
+}
+// Bounded wait for the phase with the given parity to complete. Gives up after `limit_ns` of
+// global time, raises the error word and returns false; the caller then leaves its loop.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned* err,
+                                          uint64_t limit_ns = 4000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, err, limit_ns);
+}
+// The same wait taken by all 32 lanes of a converged warp; the result is warp-uniform.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, unsigned* err,
+                                               uint64_t limit_ns = 4000000000ull) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  return __all_sync(0xffffffffu, mbar_wait_slow(bar, parity, err, limit_ns));
 }
 
 // ------------------------------------------------------------------------------ TMA
@@ -124,6 +137,14 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
                : "memory");
+}
+__device__ __forceinline__ uint32_t ldsu16(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 __device__ __forceinline__ float ldsf(uint32_t a) {
   float v;
