@@ -27,11 +27,12 @@
 // [192,256), O^T (x2) [256,384), scores Q K^T (x2, M = 64) [384,512).
 //
 // Warp roles: warp 0 issues the TMA loads (3-stage ring of Q/K/V/eta tiles); warp 1 owns TMEM
-// and issues the MMAs from one thread; warps 2-5 (operand group) write EV^T to TMEM and turn
-// the scores into the masked bf16 P tile; warps 6-9 (state group) convert S^T to its bf16 copy
-// after each update; warps 10-13 (output group) drain O^T through a shared tile and TMA-store
-// it. Each group has one warp per TMEM sub-partition. The serial chain per chunk is
-// update -> bf16 copy -> update; everything else overlaps it.
+// and issues the output and update MMAs; warp 14 issues the score MMAs Q K^T as soon as a stage
+// lands; warps 2-5 (operand group) write EV^T to TMEM and turn the scores into the masked bf16
+// P tile; warps 6-9 (state group) convert S^T to its bf16 copy after each update; warps 10-13
+// (output group) drain O^T through a shared tile and TMA-store it. Each group has one warp per
+// TMEM sub-partition. The MMA-issuing warps run converged and issue through elect.sync. The
+// serial chain per chunk is update -> bf16 copy -> update; everything else overlaps it.
 #include <algorithm>
 #include <cstdlib>
 
@@ -44,7 +45,7 @@ namespace {
 
 constexpr int D = 128;         // head dim
 constexpr int C = 64;          // chunk
-constexpr int THREADS = 448;   // TMA warp, MMA warp, operand / state / output groups of 4 warps
+constexpr int THREADS = 480;   // TMA warp, MMA warp, 3 groups of 4 warps, score warp
 
 // shared-memory map (bytes from the 1024-aligned base); pass 1 loads no Q and writes no O
 template <bool SO>
@@ -112,13 +113,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t bar = sbase + L::BAR_OFF;
   const uint32_t full = bar, empty = bar + 40;                  // stage ring (up to 5)
   const uint32_t pfull = bar + 80;                              // score accumulators (x2)
-  const uint32_t pready = bar + 112;                            // P tile written (x2)
-  const uint32_t evready = bar + 128;                           // EV^T written (x2)
-  const uint32_t afree = bar + 144;                             // EV^T and P tile reusable (x2)
-  const uint32_t ofull = bar + 160, oempty = bar + 176;         // output accumulators (x2)
-  const uint32_t sdone = bar + 192;                             // state update finished
-  const uint32_t sready = bar + 200;                            // bf16 S^T written
-  const uint32_t tslot = bar + 208;
+  const uint32_t pready = bar + 96;                             // P tile written (x2)
+  const uint32_t go = bar + 112;                                // chunk operands ready (x2)
+  const uint32_t afree = bar + 128;                             // EV^T and P tile reusable (x2)
+  const uint32_t ofull = bar + 144;                             // output accumulators (x2)
+  const uint32_t sdone = bar + 160;                             // state update finished
+  const uint32_t tslot = bar + 168;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // blockIdx = stream * nparts + part; pass 1 only covers parts 0 .. P-2
@@ -130,25 +130,27 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(full + 8 * s, 1);
-      mbar_init(empty + 8 * s, 5);  // MMA commit + 4 operand warps
+      // MMA warp + 4 operand warps (+ the score warp in pass 2)
+      mbar_init(empty + 8 * s, SO ? 5 : 6);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(pfull + 8 * b, 1);
       mbar_init(pready + 8 * b, 4);
-      mbar_init(evready + 8 * b, 4);
+      // chunk c may start once EV^T(c) is written (4 operand warps), and in pass 2 once the
+      // bf16 copy of S holds the state before c (4 state warps) and O^T(c-2) has been read
+      // out (4 output warps)
+      mbar_init(go + 8 * b, SO ? 4 : 12);
       mbar_init(afree + 8 * b, 1);
       mbar_init(ofull + 8 * b, 1);
-      mbar_init(oempty + 8 * b, 4);
     }
     mbar_init(sdone, 1);
-    mbar_init(sready, 4);
     fence_mbar_init();
   }
   if (warp == 1) umma::tmem_alloc(tslot, TM_COLS);
   umma::fence_before();
   __syncthreads();
   umma::fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::BAR_OFF + 208);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::BAR_OFF + 168);
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -177,46 +179,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    // The whole warp runs this loop: every lane waits, the wait results are made warp-uniform,
-    // and one elected lane issues each MMA / commit, so no divergent branch surrounds them.
-    const uint32_t id_s = umma::idesc_bf16(64, 64, false, false);    // Q K^T
+    // ---------------------------------------------------------------- chain MMA warp
+    // The whole warp runs this loop: every lane waits (warp-uniform results) and one elected
+    // lane issues each MMA / commit, so no divergent branch surrounds them.
     const uint32_t id_o = umma::idesc_bf16(128, 64, false, false);   // S^T Q^T, EV^T P^T
     const uint32_t id_u = umma::idesc_bf16(128, 128, false, true);   // EV^T K
-    auto wait = [&](uint32_t b_, uint32_t parity) -> bool {
-      return mbar_wait_warp(b_, parity, p.err);
-    };
-    auto scores = [&](int c) {
-      const int s = c % ST, b = c & 1;
-      const uint32_t sQ = sbase + s * L::STAGE, sK = sQ + L::K_OFF;
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
-        umma::mma_ss_elect(tmem + TM_P + 64 * b, umma::desc_kmajor(sQ + o),
-                           umma::desc_kmajor(sK + o), id_s, ks > 0);
-      }
-      umma::commit_elect(pfull + 8 * b);
-    };
-    bool ok = true;
-    if (!SO) {
-      ok = wait(full, 0);
-      if (ok) {
-        umma::fence_after();
-        scores(0);
-      }
-    }
-    for (int c = 0; ok && c < nch; ++c) {
+    for (int c = 0; c < nch; ++c) {
       const int s = c % ST, b = c & 1;
       const uint32_t sQ = sbase + s * L::STAGE, sK = sQ + L::K_OFF;
       const uint32_t aEV = tmem + TM_EV + 32 * b;
       const uint32_t dO = tmem + TM_O + 64 * b;
-      if (SO) ok = wait(full + 8 * s, (c / ST) & 1);
-      ok = ok && wait(evready + 8 * b, (c >> 1) & 1);
-      if (!SO) {
-        ok = ok && wait(sready, c & 1);
-        if (c >= 2) ok = ok && wait(oempty + 8 * b, ((c >> 1) - 1) & 1);
-      }
-      if (!ok) break;
+      if (!mbar_wait_warp(full + 8 * s, (c / ST) & 1, p.err)) break;
+      if (!mbar_wait_warp(go + 8 * b, (c >> 1) & 1, p.err)) break;
       umma::fence_after();
       if (!SO) {
         // O^T = S^T Q^T: reads the bf16 copy of S before this chunk's update
@@ -231,15 +205,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int ks = 0; ks < C / 16; ++ks)
         umma::mma_ts_elect(tmem + TM_S, aEV + 8 * ks, umma::desc_mnmajor(sK + 2048 * ks, 8192),
                            id_u, SO ? (c > 0 || ks > 0) : true);
+      // Pass 2 signals every update (the state warps refresh the bf16 copy); pass 1 only the
+      // final one.
+      if (!SO || c + 1 == nch) umma::commit_elect(sdone);
+      umma::commit_elect(empty + 8 * s);   // Q and K of this stage are no longer needed here
       if (SO) {
-        // pass 1 signals only the final update
-        if (c + 1 == nch) umma::commit_elect(sdone);
         umma::commit_elect(afree + 8 * b);
-        umma::commit_elect(empty + 8 * s);
         continue;
       }
-      umma::commit_elect(sdone);   // the state warps refresh the bf16 copy
-      if (!wait(pready + 8 * b, (c >> 1) & 1)) break;
+      if (!mbar_wait_warp(pready + 8 * b, (c >> 1) & 1, p.err)) break;
       umma::fence_after();
       const uint32_t sP = sbase + L::P_OFF + 8192 * b;
       // O^T += EV^T P^T
@@ -248,15 +222,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma::mma_ts_elect(dO, aEV + 8 * ks, umma::desc_kmajor(sP + 32 * ks), id_o, true);
       umma::commit_elect(ofull + 8 * b);
       umma::commit_elect(afree + 8 * b);
-      umma::commit_elect(empty + 8 * s);
-      if (c + 1 < nch) {
-        // The score buffer of chunk c+1 was last read for chunk c-1; those reads finished
-        // before the operand warps signalled pready(c-1), which this warp has seen.
-        const int s1 = (c + 1) % ST;
-        if (!wait(full + 8 * s1, ((c + 1) / ST) & 1)) break;
-        umma::fence_after();
-        scores(c + 1);
-      }
     }
   } else if (warp < 6) {
     // ---------------------------------------------------------------- operand warps 2..5
@@ -265,6 +230,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tl = (uint32_t)(32 * q) << 16;
     const bool rowthr = lane < 16;            // holds an M = 64 score row
     const int r = 16 * q + lane;              // that row (token t of the chunk)
+    // byte offset of this lane's column in token row `tok` of a swizzled V sub-tile is
+    // 128 * tok + (cb ^ 16 * (tok % 8))
+    const uint32_t cb = 2 * (dout & 63);
+    uint32_t cbx[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) cbx[k] = cb ^ (16u * k);
     for (int c = 0; c < nch; ++c) {
       const int s = c % ST, b = c & 1;
       const uint32_t stg = sbase + s * L::STAGE;
@@ -273,7 +244,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       // EV^T: column j of this lane holds (eta_2j v_2j, eta_2j+1 v_2j+1)[dout]
       {
         const uint32_t vcol = stg + L::V_OFF + (dout >> 6) * 8192;
-        const uint32_t cb = 2 * (dout & 63);
         uint32_t ev[32];
 #pragma unroll
         for (int j4 = 0; j4 < C / 4; ++j4) {
@@ -291,7 +261,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int tok = 4 * j4 + u;
-            f[u] = __uint_as_float(ldsu16(vcol + swz<128>(tok * 128 + cb)) << 16) * e[u];
+            f[u] = __uint_as_float(ldsu16(vcol + cbx[tok & 7] + 128 * tok) << 16) * e[u];
           }
           ev[2 * j4] = pack_bf16(f[0], f[1]);
           ev[2 * j4 + 1] = pack_bf16(f[2], f[3]);
@@ -302,7 +272,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       umma::fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(evready + 8 * b);
+        mbar_arrive(go + 8 * b);
         mbar_arrive(empty + 8 * s);
       }
       if (SO) continue;
@@ -334,6 +304,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
+      // pready(c) also tells the score warp that the score buffer of chunk c is read
       if (lane == 0) mbar_arrive(pready + 8 * b);
     }
   } else if (warp < 10) {
@@ -342,8 +313,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int dout = 32 * q + lane;
     const uint32_t tl = (uint32_t)(32 * q) << 16;
 
-    // fp32 S^T row (this lane) -> bf16 copy used as the A operand of O^T = S^T Q^T
-    auto refresh = [&]() {
+    // fp32 S^T row (this lane) -> bf16 copy used as the A operand of O^T = S^T Q^T; signals
+    // go(chunk)
+    auto refresh = [&](int chunk) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t a0[32], a1[32], o[32];
@@ -362,7 +334,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       umma::wait_st();
       umma::fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sready);
+      if (lane == 0) mbar_arrive(go + 8 * (chunk & 1));
     };
 
     bool ok = true;
@@ -380,11 +352,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma::st32x32(tmem + tl + TM_S + 32 * cc, v);
       }
       umma::wait_st();
-      refresh();
+      refresh(0);
       for (int c = 0; c < nch; ++c) {
         if (!mbar_wait(sdone, c & 1, p.err)) { ok = false; break; }
         umma::fence_after();
-        if (c + 1 < nch) refresh();
+        if (c + 1 < nch) refresh(c + 1);
       }
     } else {
       ok = mbar_wait(sdone, 0, p.err);
@@ -404,8 +376,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int j = 0; j < 32; ++j) dst[(32 * cc + j) * D + dout] = __uint_as_float(v[j]);
       }
     }
-  } else if (!SO) {
+  } else if (warp < 14) {
     // ---------------------------------------------------------------- output warps 10..13
+    if (SO) goto done;   // pass 1 has no outputs
+    {
     const int q = warp & 3;
     const int dout = 32 * q + lane;
     const uint32_t tl = (uint32_t)(32 * q) << 16;
@@ -416,6 +390,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     // row t+4 (the two rows fall in disjoint bank halves of the swizzled tile).
     const uint32_t ocol = (dout >> 6) * 8192;
     const uint32_t cb = 2 * ((dout & 63) & ~1);
+    // the output buffers of chunks 0 and 1 start free
+    if (lane == 0) {
+      mbar_arrive(go);
+      mbar_arrive(go + 8);
+    }
     for (int c = 0; c < nch; ++c) {
       const int b = c & 1;
       const bool got = mbar_wait(ofull + 8 * b, (c >> 1) & 1, p.err);
@@ -429,7 +408,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       umma::reg_fence(v1);
       umma::fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(oempty + 8 * b);
+      if (lane == 0 && c + 2 < nch) mbar_arrive(go + 8 * b);   // O^T buffer free for c+2
       const uint32_t so = sbase + L::O_OFF + 16384 * b + ocol;
 #pragma unroll
       for (int t = 0; t < C; ++t) {
@@ -454,7 +433,29 @@ __global__ void __launch_bounds__(THREADS, 1)
       named_bar_sync(2, 128);
     }
     if (otid == 0) bulk_wait<0>();
+    }
+  } else if (!SO) {
+    // ---------------------------------------------------------------- score warp 14
+    // D_P(c) = Q_c K_c^T into score buffer c % 2, issued as soon as the tiles land.
+    const uint32_t id_s = umma::idesc_bf16(64, 64, false, false);
+    for (int c = 0; c < nch; ++c) {
+      const int s = c % ST, b = c & 1;
+      if (!mbar_wait_warp(full + 8 * s, (c / ST) & 1, p.err)) break;
+      // score buffer b was last read for chunk c-2, before pready(c-2)
+      if (c >= 2 && !mbar_wait_warp(pready + 8 * b, ((c >> 1) - 1) & 1, p.err)) break;
+      umma::fence_after();
+      const uint32_t sQ = sbase + s * L::STAGE, sK = sQ + L::K_OFF;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
+        umma::mma_ss_elect(tmem + TM_P + 64 * b, umma::desc_kmajor(sQ + o),
+                           umma::desc_kmajor(sK + o), id_s, ks > 0);
+      }
+      umma::commit_elect(pfull + 8 * b);
+      umma::commit_elect(empty + 8 * s);
+    }
   }
+done:
   umma::fence_before();
   __syncthreads();
   if (warp == 1) umma::tmem_dealloc(tmem, TM_COLS);
