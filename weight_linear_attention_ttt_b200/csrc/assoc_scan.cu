@@ -20,19 +20,19 @@
 // transposed: with EV = diag(eta) V and P = tril(Q K^T),
 //     O^T = S^T Q^T + EV^T P^T          (M = d_out, N = 64 tokens)
 //     S^T += EV^T K                     (M = d_out, N = d_in, K = 64 tokens)
-// Operands that the CTA itself produces live in TMEM as bf16 and feed the MMAs as the A
-// operand: the bf16 copy of S^T (refreshed after every update) and EV^T (written by the
-// operand warps from the V tile). Only Q, K and the masked score tile P are read from shared
-// memory by the tensor core. TMEM columns: S^T fp32 [0,128), bf16 S^T [128,192), EV^T (x2)
-// [192,256), O^T (x2) [256,384), scores Q K^T (x2, M = 64) [384,512).
+// The bf16 copy of S^T (refreshed after every update) lives in TMEM and feeds O^T = S^T Q^T as
+// the A operand; EV is the V tile scaled by eta in place in shared memory and feeds the other
+// two products as an MN-major A operand. TMEM columns: S^T fp32 [0,128), bf16 S^T (x2)
+// [128,256), O^T (x2) [256,384), scores Q K^T (x2, M = 64) [384,512).
 //
 // Warp roles: warp 0 issues the TMA loads (3-stage ring of Q/K/V/eta tiles); warp 1 owns TMEM
-// and issues the output and update MMAs; warp 14 issues the score MMAs Q K^T as soon as a stage
-// lands; warps 2-5 (operand group) write EV^T to TMEM and turn the scores into the masked bf16
-// P tile; warps 6-9 (state group) convert S^T to its bf16 copy after each update; warps 10-13
-// (output group) drain O^T through a shared tile and TMA-store it. Each group has one warp per
-// TMEM sub-partition. The MMA-issuing warps run converged and issue through elect.sync. The
-// serial chain per chunk is update -> bf16 copy -> update; everything else overlaps it.
+// and issues the update and output MMAs; warp 14 issues the score MMAs Q K^T as soon as a stage
+// lands; warps 2-5 (operand group) scale V by eta in place and turn the scores into the masked
+// bf16 P tile; warps 6-9 (state group) and 10-13 (output group) each convert half of S^T to its
+// bf16 copy after every update, and the output group drains O^T through a shared tile and
+// TMA-stores it. Each group has one warp per TMEM sub-partition. The MMA-issuing warps run
+// converged and issue through elect.sync. The serial chain per chunk is
+// update -> bf16 copy -> update; everything else overlaps it.
 #include <algorithm>
 #include <cstdlib>
 
@@ -67,8 +67,7 @@ struct Smem {
 
 // TMEM columns
 constexpr uint32_t TM_S = 0;      // S^T fp32, lanes = d_out, columns = d_in
-constexpr uint32_t TM_SBF = 128;  // bf16 S^T (64 columns of d_in pairs)
-constexpr uint32_t TM_EV = 192;   // 2 x 32: bf16 EV^T (token pairs)
+constexpr uint32_t TM_SBF = 128;  // 2 x 64: bf16 S^T (d_in pairs), one per chunk parity
 constexpr uint32_t TM_O = 256;    // 2 x 64: O^T fp32, lanes = d_out, columns = tokens
 constexpr uint32_t TM_P = 384;    // 2 x 64: Q K^T (M = 64)
 constexpr uint32_t TM_COLS = 512;
@@ -115,7 +114,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t pfull = bar + 80;                              // score accumulators (x2)
   const uint32_t pready = bar + 96;                             // P tile written (x2)
   const uint32_t go = bar + 112;                                // chunk operands ready (x2)
-  const uint32_t afree = bar + 128;                             // EV^T and P tile reusable (x2)
+  const uint32_t afree = bar + 128;                             // P tile reusable (x2)
   const uint32_t ofull = bar + 144;                             // output accumulators (x2)
   const uint32_t sdone = bar + 160;                             // state update finished
   const uint32_t tslot = bar + 168;
@@ -136,9 +135,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(pfull + 8 * b, 1);
       mbar_init(pready + 8 * b, 4);
-      // chunk c may start once EV^T(c) is written (4 operand warps), and in pass 2 once the
-      // bf16 copy of S holds the state before c (4 state warps) and O^T(c-2) has been read
-      // out (4 output warps)
+      // Chunk c may start once EV(c) is written (4 operand warps) and, in pass 2, once the
+      // bf16 copy of the state before c is written (state and output warps, half each; the
+      // output warps also have read out O^T(c-2) by then).
       mbar_init(go + 8 * b, SO ? 4 : 12);
       mbar_init(afree + 8 * b, 1);
       mbar_init(ofull + 8 * b, 1);
@@ -151,6 +150,44 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   umma::fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::BAR_OFF + 168);
+
+  // State and output warps (pass 2): bf16 copy of 64 of the 128 state columns for `chunk`.
+  // Lane = d_out row of S^T; `half` selects d_in columns [64 half, 64 half + 64).
+  auto refresh = [&](int chunk, int half, uint32_t tl) {
+    uint32_t a0[32], a1[32], o[32];
+    umma::ld32x32(tmem + tl + TM_S + 64 * half, a0);
+    umma::ld32x32(tmem + tl + TM_S + 64 * half + 32, a1);
+    umma::wait_ld();
+    umma::reg_fence(a0);
+    umma::reg_fence(a1);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      o[j] = pack_bf16(__uint_as_float(a0[2 * j]), __uint_as_float(a0[2 * j + 1]));
+      o[16 + j] = pack_bf16(__uint_as_float(a1[2 * j]), __uint_as_float(a1[2 * j + 1]));
+    }
+    umma::st32x32(tmem + tl + TM_SBF + 64 * (chunk & 1) + 32 * half, o);
+    umma::wait_st();
+    umma::fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(go + 8 * (chunk & 1));
+  };
+  // Starting state S (d_in x d_out, row-major) of this part, columns [64 half, 64 half + 64)
+  // of S^T, into TMEM.
+  auto load_state = [&](int half, uint32_t tl, int dout) {
+    const float* src = nullptr;
+    if (part == 0) src = p.S0 ? p.S0 + (size_t)stream * D * D : nullptr;
+    else src = p.S_start + ((size_t)stream * (p.P - 1) + (part - 1)) * D * D;
+#pragma unroll 1
+    for (int cc = 0; cc < 2; ++cc) {
+      uint32_t v[32];
+      const int din0 = 64 * half + 32 * cc;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        v[j] = __float_as_uint(src ? src[(din0 + j) * D + dout] : 0.f);
+      umma::st32x32(tmem + tl + TM_S + din0, v);
+    }
+    umma::wait_st();
+  };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -182,102 +219,95 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---------------------------------------------------------------- chain MMA warp
     // The whole warp runs this loop: every lane waits (warp-uniform results) and one elected
     // lane issues each MMA / commit, so no divergent branch surrounds them.
-    const uint32_t id_o = umma::idesc_bf16(128, 64, false, false);   // S^T Q^T, EV^T P^T
-    const uint32_t id_u = umma::idesc_bf16(128, 128, false, true);   // EV^T K
+    const uint32_t id_o1 = umma::idesc_bf16(128, 64, false, false);  // S^T Q^T (A in TMEM)
+    const uint32_t id_o2 = umma::idesc_bf16(128, 64, true, false);   // EV^T P^T
+    const uint32_t id_u = umma::idesc_bf16(128, 128, true, true);    // EV^T K
     for (int c = 0; c < nch; ++c) {
       const int s = c % ST, b = c & 1;
       const uint32_t sQ = sbase + s * L::STAGE, sK = sQ + L::K_OFF;
-      const uint32_t aEV = tmem + TM_EV + 32 * b;
+      const uint32_t sEV = sQ + L::V_OFF;
       const uint32_t dO = tmem + TM_O + 64 * b;
       if (!mbar_wait_warp(full + 8 * s, (c / ST) & 1, p.err)) break;
       if (!mbar_wait_warp(go + 8 * b, (c >> 1) & 1, p.err)) break;
       umma::fence_after();
-      if (!SO) {
-        // O^T = S^T Q^T: reads the bf16 copy of S before this chunk's update
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks)
-          umma::mma_ts_elect(dO, tmem + TM_SBF + 8 * ks,
-                             umma::desc_kmajor(sQ + (ks >> 2) * 8192 + (ks & 3) * 32), id_o,
-                             ks > 0);
-      }
-      // S^T += EV^T K (heads the serial chain)
+      // S^T += EV^T K: heads the serial chain, so it is issued first
 #pragma unroll
       for (int ks = 0; ks < C / 16; ++ks)
-        umma::mma_ts_elect(tmem + TM_S, aEV + 8 * ks, umma::desc_mnmajor(sK + 2048 * ks, 8192),
-                           id_u, SO ? (c > 0 || ks > 0) : true);
-      // Pass 2 signals every update (the state warps refresh the bf16 copy); pass 1 only the
-      // final one.
+        umma::mma_ss_elect(tmem + TM_S, umma::desc_mnmajor(sEV + 2048 * ks, 8192),
+                           umma::desc_mnmajor(sK + 2048 * ks, 8192), id_u,
+                           SO ? (c > 0 || ks > 0) : true);
+      // Pass 2 signals every update (the state and output warps refresh the bf16 copy);
+      // pass 1 only the final one.
       if (!SO || c + 1 == nch) umma::commit_elect(sdone);
-      umma::commit_elect(empty + 8 * s);   // Q and K of this stage are no longer needed here
       if (SO) {
-        umma::commit_elect(afree + 8 * b);
+        umma::commit_elect(empty + 8 * s);
         continue;
       }
+      // O^T = S^T Q^T with the bf16 copy of the state before this chunk
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks)
+        umma::mma_ts_elect(dO, tmem + TM_SBF + 64 * b + 8 * ks,
+                           umma::desc_kmajor(sQ + (ks >> 2) * 8192 + (ks & 3) * 32), id_o1,
+                           ks > 0);
       if (!mbar_wait_warp(pready + 8 * b, (c >> 1) & 1, p.err)) break;
       umma::fence_after();
       const uint32_t sP = sbase + L::P_OFF + 8192 * b;
       // O^T += EV^T P^T
 #pragma unroll
       for (int ks = 0; ks < C / 16; ++ks)
-        umma::mma_ts_elect(dO, aEV + 8 * ks, umma::desc_kmajor(sP + 32 * ks), id_o, true);
+        umma::mma_ss_elect(dO, umma::desc_mnmajor(sEV + 2048 * ks, 8192),
+                           umma::desc_kmajor(sP + 32 * ks), id_o2, true);
       umma::commit_elect(ofull + 8 * b);
       umma::commit_elect(afree + 8 * b);
+      umma::commit_elect(empty + 8 * s);   // the stage (Q, K, EV) is no longer needed
     }
   } else if (warp < 6) {
     // ---------------------------------------------------------------- operand warps 2..5
     const int q = warp & 3;
-    const int dout = 32 * q + lane;           // TMEM lane = output column
     const uint32_t tl = (uint32_t)(32 * q) << 16;
     const bool rowthr = lane < 16;            // holds an M = 64 score row
     const int r = 16 * q + lane;              // that row (token t of the chunk)
-    // byte offset of this lane's column in token row `tok` of a swizzled V sub-tile is
-    // 128 * tok + (cb ^ 16 * (tok % 8))
-    const uint32_t cb = 2 * (dout & 63);
-    uint32_t cbx[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) cbx[k] = cb ^ (16u * k);
+    const int otid = threadIdx.x - 64;       // 0..127
     for (int c = 0; c < nch; ++c) {
       const int s = c % ST, b = c & 1;
       const uint32_t stg = sbase + s * L::STAGE;
       if (!mbar_wait(full + 8 * s, (c / ST) & 1, p.err)) break;
-      if (c >= 2 && !mbar_wait(afree + 8 * b, ((c >> 1) - 1) & 1, p.err)) break;
-      // EV^T: column j of this lane holds (eta_2j v_2j, eta_2j+1 v_2j+1)[dout]
+      // EV = diag(eta) V in place: the V tile is 1024 16-byte pieces (row = token, eight
+      // columns each); piece i is row i / 16 of the two sub-tiles' swizzled layout.
       {
-        const uint32_t vcol = stg + L::V_OFF + (dout >> 6) * 8192;
-        uint32_t ev[32];
+        const uint32_t vt = stg + L::V_OFF;
+        uint4 x[8];
+        float e[8];
 #pragma unroll
-        for (int j4 = 0; j4 < C / 4; ++j4) {
-          float e[4];
-          if (p.eta) {
-            const uint4 ee = lds128(stg + L::ETA_OFF + 16 * j4);
-            e[0] = __uint_as_float(ee.x);
-            e[1] = __uint_as_float(ee.y);
-            e[2] = __uint_as_float(ee.z);
-            e[3] = __uint_as_float(ee.w);
-          } else {
-            e[0] = e[1] = e[2] = e[3] = p.eta_scalar;
-          }
-          float f[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int tok = 4 * j4 + u;
-            f[u] = __uint_as_float(ldsu16(vcol + cbx[tok & 7] + 128 * tok) << 16) * e[u];
-          }
-          ev[2 * j4] = pack_bf16(f[0], f[1]);
-          ev[2 * j4 + 1] = pack_bf16(f[2], f[3]);
+        for (int it = 0; it < 8; ++it) {
+          const int i = otid + 128 * it;                // 0..1023
+          const int sub = i >> 9, w = i & 511;          // sub-tile, piece within it
+          const uint32_t a = vt + sub * 8192 + swz<128>((w >> 3) * 128 + (w & 7) * 16);
+          x[it] = lds128(a);
+          e[it] = p.eta ? ldsf(stg + L::ETA_OFF + 4 * (w >> 3)) : p.eta_scalar;
         }
-        umma::st32x32(tmem + tl + TM_EV + 32 * b, ev);
-        umma::wait_st();
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int i = otid + 128 * it;
+          const int sub = i >> 9, w = i & 511;
+          const uint32_t a = vt + sub * 8192 + swz<128>((w >> 3) * 128 + (w & 7) * 16);
+          const float f = e[it];
+          sts128(a, make_uint4(pack_bf16(bf16_lo(x[it].x) * f, bf16_hi(x[it].x) * f),
+                               pack_bf16(bf16_lo(x[it].y) * f, bf16_hi(x[it].y) * f),
+                               pack_bf16(bf16_lo(x[it].z) * f, bf16_hi(x[it].z) * f),
+                               pack_bf16(bf16_lo(x[it].w) * f, bf16_hi(x[it].w) * f)));
+        }
       }
-      umma::fence_before();
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(go + 8 * b);
         mbar_arrive(empty + 8 * s);
       }
       if (SO) continue;
-      // masked scores -> P tile [t][s]
+      // masked scores -> P tile [t][s]; P tile b was last read by the MMAs of chunk c-2
       if (!mbar_wait(pfull + 8 * b, (c >> 1) & 1, p.err)) break;
+      if (c >= 2 && !mbar_wait(afree + 8 * b, ((c >> 1) - 1) & 1, p.err)) break;
       umma::fence_after();
       uint32_t v0[32], v1[32];
       umma::ld32x32(tmem + tl + TM_P + 64 * b, v0);
@@ -304,7 +334,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      // pready(c) also tells the score warp that the score buffer of chunk c is read
+      // pready(c) also tells the score warp that score buffer b has been read
       if (lane == 0) mbar_arrive(pready + 8 * b);
     }
   } else if (warp < 10) {
@@ -312,51 +342,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;
     const int dout = 32 * q + lane;
     const uint32_t tl = (uint32_t)(32 * q) << 16;
-
-    // fp32 S^T row (this lane) -> bf16 copy used as the A operand of O^T = S^T Q^T; signals
-    // go(chunk)
-    auto refresh = [&](int chunk) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t a0[32], a1[32], o[32];
-        umma::ld32x32(tmem + tl + TM_S + 64 * h, a0);
-        umma::ld32x32(tmem + tl + TM_S + 64 * h + 32, a1);
-        umma::wait_ld();
-        umma::reg_fence(a0);
-        umma::reg_fence(a1);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          o[j] = pack_bf16(__uint_as_float(a0[2 * j]), __uint_as_float(a0[2 * j + 1]));
-          o[16 + j] = pack_bf16(__uint_as_float(a1[2 * j]), __uint_as_float(a1[2 * j + 1]));
-        }
-        umma::st32x32(tmem + tl + TM_SBF + 32 * h, o);
-      }
-      umma::wait_st();
-      umma::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(go + 8 * (chunk & 1));
-    };
-
     bool ok = true;
     if (!SO) {
-      // starting state S (d_in x d_out, row-major) -> S^T in TMEM and its bf16 copy
-      const float* src = nullptr;
-      if (part == 0) src = p.S0 ? p.S0 + (size_t)stream * D * D : nullptr;
-      else src = p.S_start + ((size_t)stream * (p.P - 1) + (part - 1)) * D * D;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          v[j] = __float_as_uint(src ? src[(32 * cc + j) * D + dout] : 0.f);
-        umma::st32x32(tmem + tl + TM_S + 32 * cc, v);
-      }
-      umma::wait_st();
-      refresh(0);
+      load_state(0, tl, dout);
+      refresh(0, 0, tl);
       for (int c = 0; c < nch; ++c) {
         if (!mbar_wait(sdone, c & 1, p.err)) { ok = false; break; }
         umma::fence_after();
-        if (c + 1 < nch) refresh(c + 1);
+        if (c + 1 < nch) refresh(c + 1, 0, tl);
       }
     } else {
       ok = mbar_wait(sdone, 0, p.err);
@@ -380,68 +373,70 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---------------------------------------------------------------- output warps 10..13
     if (SO) goto done;   // pass 1 has no outputs
     {
-    const int q = warp & 3;
-    const int dout = 32 * q + lane;
-    const uint32_t tl = (uint32_t)(32 * q) << 16;
-    const int otid = threadIdx.x - 320;        // 0..127
-    const bool odd = lane & 1;
-    // Lane pairs (2i, 2i+1) exchange one value per token pair (t, t+4) so that each lane
-    // stores a 32-bit word of two adjacent output columns: the even lane row t, the odd lane
-    // row t+4 (the two rows fall in disjoint bank halves of the swizzled tile).
-    const uint32_t ocol = (dout >> 6) * 8192;
-    const uint32_t cb = 2 * ((dout & 63) & ~1);
-    // the output buffers of chunks 0 and 1 start free
-    if (lane == 0) {
-      mbar_arrive(go);
-      mbar_arrive(go + 8);
-    }
-    for (int c = 0; c < nch; ++c) {
-      const int b = c & 1;
-      const bool got = mbar_wait(ofull + 8 * b, (c >> 1) & 1, p.err);
-      if (named_bar_or(2, 128, !got)) break;
-      umma::fence_after();
-      uint32_t v0[32], v1[32];
-      umma::ld32x32(tmem + tl + TM_O + 64 * b, v0);
-      umma::ld32x32(tmem + tl + TM_O + 64 * b + 32, v1);
-      umma::wait_ld();
-      umma::reg_fence(v0);
-      umma::reg_fence(v1);
-      umma::fence_before();
-      __syncwarp();
-      if (lane == 0 && c + 2 < nch) mbar_arrive(go + 8 * b);   // O^T buffer free for c+2
-      const uint32_t so = sbase + L::O_OFF + 16384 * b + ocol;
+      const int q = warp & 3;
+      const int dout = 32 * q + lane;
+      const uint32_t tl = (uint32_t)(32 * q) << 16;
+      const int otid = threadIdx.x - 320;        // 0..127
+      const bool odd = lane & 1;
+      // Lane pairs (2i, 2i+1) exchange one value per token pair (t, t+4) so that each lane
+      // stores a 32-bit word of two adjacent output columns: the even lane row t, the odd
+      // lane row t+4 (the two rows fall in disjoint bank halves of the swizzled tile).
+      const uint32_t ocol = (dout >> 6) * 8192;
+      const uint32_t cb = 2 * ((dout & 63) & ~1);
+      load_state(1, tl, dout);
+      refresh(0, 1, tl);
+      for (int c = 0; c < nch; ++c) {
+        const int b = c & 1;
+        // second half of the bf16 state copy for chunk c+1; the go(c+1) arrival also says
+        // that O^T(c-1) has been read out
+        bool got = mbar_wait(sdone, c & 1, p.err);
+        if (got) {
+          umma::fence_after();
+          if (c + 1 < nch) refresh(c + 1, 1, tl);
+          got = mbar_wait(ofull + 8 * b, (c >> 1) & 1, p.err);
+        }
+        if (named_bar_or(2, 128, !got)) break;
+        umma::fence_after();
+        uint32_t v0[32], v1[32];
+        umma::ld32x32(tmem + tl + TM_O + 64 * b, v0);
+        umma::ld32x32(tmem + tl + TM_O + 64 * b + 32, v1);
+        umma::wait_ld();
+        umma::reg_fence(v0);
+        umma::reg_fence(v1);
+        umma::fence_before();
+        const uint32_t so = sbase + L::O_OFF + 16384 * b + ocol;
 #pragma unroll
-      for (int t = 0; t < C; ++t) {
-        if (t & 4) continue;
-        const uint32_t* vv = t < 32 ? v0 : v1;
-        const int tt = t & 31;
-        const float a = __uint_as_float(vv[tt]), a4 = __uint_as_float(vv[tt + 4]);
-        const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
-        const uint32_t w = odd ? pack_bf16(y, a4) : pack_bf16(a, y);
-        const int row = odd ? t + 4 : t;
-        sts32(so + swz<128>(row * 128 + cb), w);
+        for (int t = 0; t < C; ++t) {
+          if (t & 4) continue;
+          const uint32_t* vv = t < 32 ? v0 : v1;
+          const int tt = t & 31;
+          const float a = __uint_as_float(vv[tt]), a4 = __uint_as_float(vv[tt + 4]);
+          const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
+          const uint32_t w = odd ? pack_bf16(y, a4) : pack_bf16(a, y);
+          const int row = odd ? t + 4 : t;
+          sts32(so + swz<128>(row * 128 + cb), w);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(2, 128);
+        if (otid == 0) {
+          const uint32_t sO = sbase + L::O_OFF + 16384 * b;
+          tma_store_3d(&tmO, sO, 0, tok0 + c * C, stream);
+          tma_store_3d(&tmO, sO + 8192, 64, tok0 + c * C, stream);
+          bulk_commit();
+          bulk_wait_read<1>();  // the other staging buffer is free again
+        }
+        named_bar_sync(2, 128);
       }
-      fence_proxy_async_smem();
-      named_bar_sync(2, 128);
-      if (otid == 0) {
-        const uint32_t sO = sbase + L::O_OFF + 16384 * b;
-        tma_store_3d(&tmO, sO, 0, tok0 + c * C, stream);
-        tma_store_3d(&tmO, sO + 8192, 64, tok0 + c * C, stream);
-        bulk_commit();
-        bulk_wait_read<1>();  // the other staging buffer is free again
-      }
-      named_bar_sync(2, 128);
-    }
-    if (otid == 0) bulk_wait<0>();
+      if (otid == 0) bulk_wait<0>();
     }
   } else if (!SO) {
     // ---------------------------------------------------------------- score warp 14
-    // D_P(c) = Q_c K_c^T into score buffer c % 2, issued as soon as the tiles land.
+    // D_P(c) = Q_c K_c^T into score buffer c % 2, issued as soon as the tiles land and the
+    // operand warps have read the scores of chunk c-2.
     const uint32_t id_s = umma::idesc_bf16(64, 64, false, false);
     for (int c = 0; c < nch; ++c) {
       const int s = c % ST, b = c & 1;
       if (!mbar_wait_warp(full + 8 * s, (c / ST) & 1, p.err)) break;
-      // score buffer b was last read for chunk c-2, before pready(c-2)
       if (c >= 2 && !mbar_wait_warp(pready + 8 * b, ((c >> 1) - 1) & 1, p.err)) break;
       umma::fence_after();
       const uint32_t sQ = sbase + s * L::STAGE, sK = sQ + L::K_OFF;
