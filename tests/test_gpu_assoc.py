@@ -64,7 +64,15 @@ def test_forced_superchunk_counts_agree(cuda_lib, monkeypatch, parts):
     n0 = ttt.launch_count()
     O, S = run(x, S0)
     assert ttt.launch_count() - n0 == (1 if parts == "1" else 3)
-    check(x, O, S, S0)
+    eo, es = check(x, O, S, S0)
+    assert eo <= RACE_TRIPWIRE and es <= RACE_TRIPWIRE, (eo, es)
+
+
+# The kernel's own error on these inputs is bf16 rounding of Q, K, eta*V, the bf16 state copy and
+# the score tile: about 3e-3 for O and 2e-3 for S. A chunk that reads a stale or half-written
+# operand (a synchronisation fault between the warp groups) raises it well above that while
+# often staying under the 1e-2 parity bar, so these cases also check a bound of twice the level.
+RACE_TRIPWIRE = 6e-3
 
 
 def test_full_associative_workload_sampled_streams(cuda_lib):
@@ -74,6 +82,7 @@ def test_full_associative_workload_sampled_streams(cuda_lib):
     streams = [(0, 0), (1, 7), (3, 15)]
     eo, es = check(x, O, S, streams=streams)
     print(f"associative workload (3 sampled streams): max rel L2 O {eo:.2e} S {es:.2e}")
+    assert eo <= RACE_TRIPWIRE and es <= RACE_TRIPWIRE, (eo, es)
     assert torch.isfinite(O.float()).all() and torch.isfinite(S).all()
     assert ttt.read_device_error() == 0
 

@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t pfull = bar + 80;                              // score accumulators (x2)
   const uint32_t pready = bar + 96;                             // P tile written (x2)
   const uint32_t go = bar + 112;                                // chunk operands ready (x2)
-  const uint32_t afree = bar + 128;                             // P tile reusable (x2)
+  const uint32_t afree = bar + 128;                             // chunk c's MMAs done (x2)
   const uint32_t ofull = bar + 144;                             // output accumulators (x2)
   const uint32_t sdone = bar + 160;                             // state update finished
   const uint32_t tslot = bar + 168;
@@ -241,6 +241,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!SO || c + 1 == nch) umma::commit_elect(sdone);
       if (SO) {
         umma::commit_elect(empty + 8 * s);
+        umma::commit_elect(afree + 8 * b);
         continue;
       }
       // O^T = S^T Q^T with the bf16 copy of the state before this chunk
@@ -272,6 +273,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int s = c % ST, b = c & 1;
       const uint32_t stg = sbase + s * L::STAGE;
       if (!mbar_wait(full + 8 * s, (c / ST) & 1, p.err)) break;
+      // The arrival on go(c) below must not come before go(c-2) has been consumed, or it
+      // would complete that phase in place of the state warps: the MMAs of chunk c-2
+      // finishing (afree(c-2)) shows that it has.
+      if (c >= 2 && !mbar_wait(afree + 8 * b, ((c >> 1) - 1) & 1, p.err)) break;
       // EV = diag(eta) V in place: the V tile is 1024 16-byte pieces (row = token, eight
       // columns each); piece i is row i / 16 of the two sub-tiles' swizzled layout.
       {
@@ -307,7 +312,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (SO) continue;
       // masked scores -> P tile [t][s]; P tile b was last read by the MMAs of chunk c-2
       if (!mbar_wait(pfull + 8 * b, (c >> 1) & 1, p.err)) break;
-      if (c >= 2 && !mbar_wait(afree + 8 * b, ((c >> 1) - 1) & 1, p.err)) break;
       umma::fence_after();
       uint32_t v0[32], v1[32];
       umma::ld32x32(tmem + tl + TM_P + 64 * b, v0);
