@@ -191,14 +191,31 @@ def test_invalid_calls_raise_before_launch(cuda_lib):
     assert ttt.launch_count() == n0
 
 
+@pytest.mark.parametrize("form", ["single", "pair"])
 @pytest.mark.parametrize("warp_cols", ["8", "16"])
 @pytest.mark.parametrize("split", ["1", "2"])
-def test_kernel_variants_match_oracle(cuda_lib, monkeypatch, warp_cols, split):
-    """Every tensor-core variant (8 or 16 output columns per warp, one or two CTAs per stream)
-    meets the bf16 tolerance on full and partial pipeline stages."""
+def test_kernel_variants_match_oracle(cuda_lib, monkeypatch, warp_cols, split, form):
+    """Every tensor-core variant (8 or 16 output columns per warp, one or two CTAs per stream,
+    chain and outputs on one warp or on a warp pair) meets the bf16 tolerance on full and partial
+    pipeline stages."""
+    if form == "pair" and warp_cols == "8":
+        pytest.skip("the warp-pair form exists for 16-column warps")
     monkeypatch.setenv("TTT_DUAL_WARP_COLS", warp_cols)
     monkeypatch.setenv("TTT_DUAL_COLUMN_SPLIT", split)
+    monkeypatch.setenv("TTT_DUAL_KERNEL", form)
     for T in (144, 512):
         x = inp.dual_or_assoc_inputs(2, 3, T, 64, seed=T + 3, device="cuda", normalise=("K", "V"))
         O, W = run(x, 16)
         check(x, 16, O, W, TOL["bf16"])
+
+
+def test_pair_and_single_forms_agree_bitwise(cuda_lib, monkeypatch):
+    """The warp-pair form performs the single-warp form's arithmetic in the same order."""
+    x = inp.dual_or_assoc_inputs(2, 3, 400, 64, seed=21, device="cuda", normalise=("K", "V"))
+    for split in ("1", "2"):
+        monkeypatch.setenv("TTT_DUAL_COLUMN_SPLIT", split)
+        outs = []
+        for form in ("single", "pair"):
+            monkeypatch.setenv("TTT_DUAL_KERNEL", form)
+            outs.append(run(x, 16))
+        assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])

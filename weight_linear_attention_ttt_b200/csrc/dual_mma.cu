@@ -31,6 +31,8 @@
 #include <algorithm>
 #include <cstdlib>
 
+#include <string>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -624,6 +626,13 @@ int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
       const char* env = getenv("TTT_DUAL_STAGE_CHUNKS");  // tuning override: 4 or 8
       const char* wenv = getenv("TTT_DUAL_WARP_COLS");    // tuning override: 8 or 16
       const int wcols = wenv ? atoi(wenv) : 16;
+      // Chain and output products on paired warps (dual_pair.cu) measured faster when a stream
+      // is split over two CTAs (two warp pairs per SM) and slower with one CTA per stream (four
+      // pairs per SM: the hand-off and the output warps' own Q/K loads double the shared-memory
+      // traffic). Either form can be forced.
+      const char* kenv = getenv("TTT_DUAL_KERNEL");      // tuning override: pair or single
+      const bool pair = kenv ? std::string(kenv) == "pair" : split == 2;
+      if (wcols == 16 && pair) return launch_dual_pair(a, ctx, split);
       if (wcols == 16)
         return split == 2 ? launch_cfg<64, 2, 8, 16>(a, ctx) : launch_cfg<64, 4, 8, 16>(a, ctx);
       if (env && atoi(env) == 4)

@@ -61,6 +61,7 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
 // Dual form.
 bool dual_mma_supported(int d, int C, int dt);
 int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx);
+int launch_dual_pair(const StateArgs& a, const LaunchCtx& ctx, int split);
 int launch_dual_simt(const StateArgs& a, const LaunchCtx& ctx);
 
 // Associative mode.
