@@ -38,8 +38,9 @@ Pins (tests/test_oracle_pins.py): per-token SGD from autograd gradients at C=1; 
 gradient descent from autograd gradients at any C; the causal-linear-attention closed form at
 W0 = 0; o = q(S0 + k^T v) for one token; the sequential recurrence vs. the chunked and two-pass
 forms; eta folded into V; the In-Place block-causal linear-attention form and its one-chunk closed
-form; autograd ascent steps for the associative and In-Place deltas; hand-worked golden examples.
-Every function below has at least one pin.
+form; autograd ascent steps for the associative and In-Place deltas; hand-worked golden examples;
+the associative backward against central finite differences of the forward definition and
+against autograd of an independent torch restatement. Every function below has at least one pin.
 """
 from __future__ import annotations
 
@@ -198,6 +199,57 @@ def assoc_scan(Q, K, V, eta, S0, *, threads: int = 1, streams=None, form: str = 
         O = O.reshape(B, H, T, d)
         S = S.reshape(B, H, d, d)
     return O, S
+
+
+def assoc_backward_stream(Q, K, V, eta, S0, dO, dS_out):
+    """Gradients of  L = sum_t <dO_t, o_t> + <dS_out, S_T>  through the associative recurrence
+    S_t = S_(t-1) + eta_t k_t^T v_t, o_t = q_t S_t (the backward pass that outer-loop training
+    of the layer needs).
+
+    Written as the adjoint of the recurrence, one token at a time. A forward sweep recomputes
+    S_t and gives dq_t = dO_t S_t^T. A reverse sweep carries the state adjoint A (the gradient
+    of L with respect to S_t): A starts at dS_out; token t first adds q_t^T dO_t (o_t reads S_t),
+    then dv_t = eta_t k_t A, dk_t = eta_t v_t A^T and deta_t = k_t A v_t^T; A passes to S_(t-1)
+    unchanged because S_t = S_(t-1) + ... . After token 0, A is dS0.
+    Returns (dQ, dK, dV [T, d], deta [T] (per-token rates; their sum when eta is a scalar),
+    dS0 [d, d])."""
+    Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    T, d = Q.shape
+    e = _eta_stream(eta, T)
+    S = np.zeros((d, d)) if S0 is None else _f64(S0).copy()
+    dQ = np.empty((T, d))
+    for t in range(T):                                    # forward sweep
+        S += e[t] * np.outer(K[t], V[t])
+        dQ[t] = dO[t] @ S.T
+    A = np.zeros((d, d)) if dS_out is None else _f64(dS_out).copy()
+    dK, dV, deta = np.empty((T, d)), np.empty((T, d)), np.empty(T)
+    for t in range(T - 1, -1, -1):                        # reverse sweep
+        A += np.outer(Q[t], dO[t])
+        kA = K[t] @ A
+        dV[t] = e[t] * kA
+        dK[t] = e[t] * (A @ V[t])
+        deta[t] = kA @ V[t]
+    return dQ, dK, dV, deta, A
+
+
+def assoc_scan_bwd(Q, K, V, eta, S0, dO, dS_out, *, threads: int = 1, streams=None):
+    """All streams of [B, H, T, d] inputs (eta [B, H, T] or scalar, S0 / dS_out [B, H, d, d] or
+    None). Returns (dQ, dK, dV, deta, dS0); deta is per token even for a scalar eta."""
+    B, H, T, d = np.shape(Q)
+
+    def one(b, h):
+        e = eta if np.ndim(eta) == 0 else np.asarray(eta)[b, h]
+        s0 = None if S0 is None else np.asarray(S0)[b, h]
+        g = None if dS_out is None else np.asarray(dS_out)[b, h]
+        return assoc_backward_stream(np.asarray(Q)[b, h], np.asarray(K)[b, h],
+                                     np.asarray(V)[b, h], e, s0, np.asarray(dO)[b, h], g)
+
+    idx, res = _streams(one, None, B, H, threads, streams)
+    out = [np.stack([r[i] for r in res]) for i in range(5)]
+    if streams is None:
+        shapes = [(B, H, T, d)] * 3 + [(B, H, T), (B, H, d, d)]
+        out = [o.reshape(sh) for o, sh in zip(out, shapes)]
+    return tuple(out)
 
 
 # --------------------------------------------------------------------------------------------

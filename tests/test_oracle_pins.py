@@ -324,3 +324,101 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     assert np.allclose(variant(0, False, -1), O_ref, rtol=1e-11, atol=1e-12)
     for bad in ((-1, False, -1), (0, True, -1), (0, False, +1)):
         assert not np.allclose(variant(*bad), O_ref, rtol=1e-6, atol=1e-8)
+
+
+# ----------------------------------------------------------------------------- associative backward
+def _assoc_loss(Q, K, V, eta, S0, dO, G):
+    """The scalar whose gradients the backward returns, from the forward definition only."""
+    O, S = orc.assoc_recurrence_stream(Q, K, V, eta, S0)
+    return float(np.sum(dO * O) + np.sum(G * S))
+
+
+def _bwd_case(T, d, scalar_eta=False):
+    Q, K, V, dO = _rand(T, d), _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = 0.3 if scalar_eta else rng.uniform(0.05, 0.9, T)
+    S0, G = _rand(d, d, scale=0.5), _rand(d, d, scale=0.5)
+    return Q, K, V, eta, S0, dO, G
+
+
+def test_assoc_backward_matches_central_finite_differences():
+    """Every gradient of the adjoint sweep against central differences of the forward
+    definition (the loss is quadratic in each input, so the difference is exact up to
+    rounding)."""
+    Q, K, V, eta, S0, dO, G = _bwd_case(5, 3)
+    dQ, dK, dV, deta, dS0 = orc.assoc_backward_stream(Q, K, V, eta, S0, dO, G)
+    h = 1e-4
+    args = [Q, K, V, eta, S0]
+    for i, grad in enumerate((dQ, dK, dV, deta, dS0)):
+        fd = np.empty_like(grad)
+        for idx in np.ndindex(grad.shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[i][idx] += h
+            minus[i][idx] -= h
+            fd[idx] = (_assoc_loss(*plus, dO, G) - _assoc_loss(*minus, dO, G)) / (2 * h)
+        assert np.allclose(grad, fd, rtol=1e-7, atol=1e-8), i
+
+
+@pytest.mark.parametrize("scalar_eta", [False, True])
+def test_assoc_backward_matches_autograd(scalar_eta):
+    """Against torch autograd of an independent restatement of the recurrence (float64)."""
+    T, d = 24, 6
+    Q, K, V, eta, S0, dO, G = _bwd_case(T, d, scalar_eta)
+    dQ, dK, dV, deta, dS0 = orc.assoc_backward_stream(Q, K, V, eta, S0, dO, G)
+    tq, tk, tv, ts0 = (torch.tensor(a, requires_grad=True) for a in (Q, K, V, S0))
+    te = torch.tensor(np.full(T, eta) if scalar_eta else eta, requires_grad=True)
+    S = ts0
+    outs = []
+    for t in range(T):
+        S = S + te[t] * torch.outer(tk[t], tv[t])
+        outs.append(tq[t] @ S)
+    L = (torch.stack(outs) * torch.tensor(dO)).sum() + (S * torch.tensor(G)).sum()
+    L.backward()
+    for ours, ref in ((dQ, tq.grad), (dK, tk.grad), (dV, tv.grad), (deta, te.grad),
+                      (dS0, ts0.grad)):
+        assert np.allclose(ours, ref.numpy(), rtol=1e-10, atol=1e-11)
+
+
+def test_assoc_backward_all_streams_helper_and_zero_inputs():
+    """The batched helper equals the per-stream sweep; with dO = 0 and dS_out = 0 every gradient
+    vanishes; with dO = 0 the state adjoint is dS_out throughout (dS0 = dS_out)."""
+    B, H, T, d = 2, 2, 8, 3
+    Q, K, V, dO = (_rand(B, H, T, d) for _ in range(4))
+    eta = rng.uniform(0.1, 0.5, (B, H, T))
+    G = _rand(B, H, d, d)
+    out = orc.assoc_scan_bwd(Q, K, V, eta, None, dO, G)
+    one = orc.assoc_backward_stream(Q[1, 0], K[1, 0], V[1, 0], eta[1, 0], None, dO[1, 0],
+                                    G[1, 0])
+    for a, b in zip(out, one):
+        assert np.allclose(a[1, 0], b, rtol=0, atol=0)
+    zero = orc.assoc_scan_bwd(Q, K, V, eta, None, np.zeros_like(dO), None)
+    assert all(np.all(z == 0) for z in zero)
+    only_g = orc.assoc_scan_bwd(Q, K, V, eta, None, np.zeros_like(dO), G)
+    assert np.allclose(only_g[4], G) and np.all(only_g[0] == 0)
+
+
+def test_assoc_backward_pins_catch_planted_mistakes():
+    """Plausible slips in the adjoint (adding q_t^T dO_t after the token's gradients instead of
+    before, a transposed state adjoint in dK, eta left out of dV) must fail the
+    finite-difference pin. Planted in a copy of the reverse sweep, on the CPU."""
+    Q, K, V, eta, S0, dO, G = _bwd_case(6, 3)
+    ref = orc.assoc_backward_stream(Q, K, V, eta, S0, dO, G)
+
+    def sweep(late_add, transpose_dk, drop_eta):
+        A = G.copy()
+        dK, dV = np.empty_like(K), np.empty_like(V)
+        for t in range(len(Q) - 1, -1, -1):
+            if not late_add:
+                A += np.outer(Q[t], dO[t])
+            kA = K[t] @ A
+            dV[t] = (1.0 if drop_eta else eta[t]) * kA
+            dK[t] = eta[t] * ((A.T if transpose_dk else A) @ V[t])
+            if late_add:
+                A += np.outer(Q[t], dO[t])
+        return dK, dV
+
+    good = sweep(False, False, False)
+    assert np.allclose(good[0], ref[1]) and np.allclose(good[1], ref[2])
+    for bad in ((True, False, False), (False, True, False), (False, False, True)):
+        dK, dV = sweep(*bad)
+        assert not (np.allclose(dK, ref[1], rtol=1e-6) and np.allclose(dV, ref[2], rtol=1e-6))
