@@ -120,6 +120,31 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
                        cudaStream_t stream);
 
 /* --------------------------------------------------------------------------------------------
+ * Backward of the associative mode (the gradients that outer-loop training of the layer needs,
+ * "KV 바인딩 기반 테스트 시간 학습은 사실상 선형 어텐션이다": the layer is trained end to end
+ * through its inner updates). For the forward above and a scalar loss L with
+ *     dL/dO = dO,   dL/dS_out = dS_out,
+ *  returns dQ = dL/dQ, dK, dV, deta (per token) and dS0. With A_t = dS_out + sum_{u>=t} q_u^T dO_u:
+ *     dq_t = dO_t S_t^T,  dv_t = eta_t k_t A_t,  dk_t = eta_t v_t A_t^T,  deta_t = k_t A_t v_t^T,
+ *     dS0 = A_0.
+ *  Q, K, V, dO [B,H,T,d] bf16; eta [B,H,T] fp32 or NULL (eta_scalar for every token); S0 and
+ *  dS_out [B,H,d,d] fp32 or NULL (zeros). Outputs: dQ, dK, dV [B,H,T,d] bf16; deta [B,H,T]
+ *  fp32 (per token also when eta is NULL: the scalar's gradient is their sum); dS0 [B,H,d,d]
+ *  fp32. Outputs must not overlap the inputs or each other.
+ *  Supported: bf16, d == 128, C == 64, T % C == 0. C is the evaluation granularity; the
+ *  gradients do not depend on it beyond rounding.
+ *  Workspace: ttt_assoc_scan_bwd_workspace_size() bytes.
+ *  Runs as three passes of the forward kernel (dQ in forward order; dV and dK through the
+ *  reverse-order recurrence of the state gradient) and one elementwise pass.
+ * ------------------------------------------------------------------------------------------ */
+size_t ttt_assoc_scan_bwd_workspace_size(int B, int H, int T, int d, int C, int dt);
+int ttt_assoc_scan_bwd(const void* Q, const void* K, const void* V, const float* eta,
+                       float eta_scalar, const float* S0, const void* dO, const float* dS_out,
+                       void* dQ, void* dK, void* dV, float* deta, float* dS0, int B, int H,
+                       int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
+
+/* --------------------------------------------------------------------------------------------
  * State increment of a sequence slice in the associative mode (the first pass of the prefix
  * scan over states, "KV 바인딩 기반 테스트 시간 학습은 사실상 선형 어텐션이다", associativity
  * paragraph; per-chunk deltas combined by a prefix sum for context parallelism, "In-Place

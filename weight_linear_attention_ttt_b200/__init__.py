@@ -25,6 +25,7 @@ EXPORTED_SYMBOLS = (
     "ttt_read_device_error",
     "ttt_linear_dual_workspace_size", "ttt_linear_dual_fwd",
     "ttt_assoc_scan_workspace_size", "ttt_assoc_scan_fwd", "ttt_assoc_state_fwd",
+    "ttt_assoc_scan_bwd_workspace_size", "ttt_assoc_scan_bwd",
     "ttt_state_prefix_sum",
     "inplace_ttt_workspace_size", "inplace_ttt_chunk_fwd",
     "inplace_ttt_noalloc_max_scratch_bytes", "inplace_ttt_chunk_fwd_noalloc",
@@ -67,9 +68,13 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     for name in ("ttt_linear_dual_fwd", "ttt_assoc_scan_fwd"):
         getattr(lib, name).restype = c_int
         getattr(lib, name).argtypes = state_args
-    for name in ("ttt_linear_dual_workspace_size", "ttt_assoc_scan_workspace_size"):
+    for name in ("ttt_linear_dual_workspace_size", "ttt_assoc_scan_workspace_size",
+                 "ttt_assoc_scan_bwd_workspace_size"):
         getattr(lib, name).restype = c_size
         getattr(lib, name).argtypes = [c_int] * 6
+    lib.ttt_assoc_scan_bwd.restype = c_int
+    lib.ttt_assoc_scan_bwd.argtypes = [vp, vp, vp, fp, c_float, fp, vp, fp, vp, vp, vp, fp, fp,
+                                       c_int, c_int, c_int, c_int, c_int, c_int, vp, c_size, vp]
     lib.ttt_assoc_state_fwd.restype = c_int
     lib.ttt_assoc_state_fwd.argtypes = [vp, vp, fp, c_float, fp, c_int, c_int, c_int, c_int,
                                         c_int, c_int, vp]
@@ -165,6 +170,47 @@ def ttt_assoc_scan_fwd(Q, K, V, eta=None, S0=None, *, C: int, eta_scalar: float 
     """Associative (gradient-ascent) linear-attention mode. Returns (O, S_out)."""
     return _state_call("ttt_assoc_scan_fwd", "ttt_assoc_scan_workspace_size", Q, K, V, eta,
                        eta_scalar, S0, C, O, S_out, workspace, stream)
+
+
+def ttt_assoc_scan_bwd(Q, K, V, eta, S0, dO, dS_out=None, *, C: int, eta_scalar: float = 0.0,
+                       dQ=None, dK=None, dV=None, deta=None, dS0=None, workspace=None,
+                       stream=None) -> Tuple:
+    """Backward of the associative mode: gradients of a loss whose gradients with respect to the
+    forward's O and S_out are dO and dS_out (None: zeros). Returns (dQ, dK, dV, deta, dS0);
+    deta is per token even when eta is None (the scalar rate's gradient is its sum)."""
+    import torch
+
+    lib = load_library()
+    _require(Q.dim() == 4, "Q, K, V, dO must be [B, H, T, d]")
+    B, H, T, d = Q.shape
+    for t in (Q, K, V, dO):
+        _require(t.is_cuda and t.is_contiguous() and t.shape == Q.shape and t.dtype == Q.dtype,
+                 "Q, K, V, dO must be contiguous CUDA tensors of one shape and dtype")
+    dt = _dtype_code(Q)
+    if eta is not None:
+        _require(eta.is_cuda and eta.dtype == torch.float32 and eta.is_contiguous() and
+                 tuple(eta.shape) == (B, H, T), "eta must be a contiguous fp32 [B, H, T] tensor")
+    for t in (S0, dS_out):
+        if t is not None:
+            _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
+                     tuple(t.shape) == (B, H, d, d), "states must be fp32 [B, H, d, d]")
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(Q) if dK is None else dK
+    dV = torch.empty_like(Q) if dV is None else dV
+    if deta is None:
+        deta = torch.empty((B, H, T), device=Q.device, dtype=torch.float32)
+    if dS0 is None:
+        dS0 = torch.empty((B, H, d, d), device=Q.device, dtype=torch.float32)
+    ws_bytes = lib.ttt_assoc_scan_bwd_workspace_size(B, H, T, d, C, dt)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, device=Q.device, dtype=torch.uint8)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.ttt_assoc_scan_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta), ctypes.c_float(eta_scalar),
+                                _ptr(S0), _ptr(dO), _ptr(dS_out), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                _ptr(deta), _ptr(dS0), B, H, T, d, C, dt, _ptr(workspace), wsz,
+                                _stream_ptr(stream))
+    _check("ttt_assoc_scan_bwd", st)
+    return dQ, dK, dV, deta, dS0
 
 
 def ttt_assoc_state_fwd(K, V, eta=None, *, C: int, eta_scalar: float = 0.0, dS=None,

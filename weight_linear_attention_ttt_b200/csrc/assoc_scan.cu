@@ -79,6 +79,7 @@ struct AssocParams {
   const float* S_start;     // [BH, P-1, D, D] starting states of parts 1.. (pass 2, P > 1)
   float* S_dst;             // pass 1: [BH, P-1, D, D] increments; pass 2: S_out [BH, D, D]
   int T, P, part_len;
+  int reverse;              // chunks last to first, transposed causal mask
   unsigned* err;
 };
 
@@ -125,6 +126,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int stream = blockIdx.x / nparts, part = blockIdx.x % nparts;
   const int tok0 = part * p.part_len;
   const int nch = p.part_len / C;
+  // first token of the c-th chunk this CTA processes (in reverse mode the sequence is walked
+  // from its end, and part 0 is the last superchunk)
+  auto tok = [&](int c) { return p.reverse ? p.T - C - (tok0 + c * C) : tok0 + c * C; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -201,7 +205,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (c >= ST && !mbar_wait(empty + 8 * s, ((c / ST) - 1) & 1, p.err)) break;
         const uint32_t fb = full + 8 * s;
         const uint32_t st = sbase + s * L::STAGE;
-        const int t0 = tok0 + c * C;
+        const int t0 = tok(c);
         mbar_arrive_expect_tx(fb, bytes);
         if (!SO) {
           tma_load_3d(st, &tmQ, fb, 0, t0, stream);
@@ -329,7 +333,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int e = 0; e < 8; ++e) {
             const int sidx = j + e;
             const float x = __uint_as_float(sidx < 32 ? v0[sidx] : v1[sidx - 32]);
-            f[e] = sidx <= r ? x : 0.f;
+            f[e] = (p.reverse ? sidx >= r : sidx <= r) ? x : 0.f;
           }
           sts128(prow + swz<128>(r * 128 + 2 * j),
                  make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
@@ -424,8 +428,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         named_bar_sync(2, 128);
         if (otid == 0) {
           const uint32_t sO = sbase + L::O_OFF + 16384 * b;
-          tma_store_3d(&tmO, sO, 0, tok0 + c * C, stream);
-          tma_store_3d(&tmO, sO + 8192, 64, tok0 + c * C, stream);
+          tma_store_3d(&tmO, sO, 0, tok(c), stream);
+          tma_store_3d(&tmO, sO + 8192, 64, tok(c), stream);
           bulk_commit();
           bulk_wait_read<1>();  // the other staging buffer is free again
         }
@@ -535,6 +539,7 @@ int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
   p.T = a.T;
   p.P = 2;             // parts 0 .. P-2 = the single part [0, T)
   p.part_len = a.T;
+  p.reverse = a.reverse;
   p.err = ctx.err;
   return launch_chunk<true>(tq, tk, tv, to, p, BH, ctx);
 }
@@ -572,6 +577,7 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   p.T = a.T;
   p.P = P;
   p.part_len = a.T / P;
+  p.reverse = a.reverse;
   p.err = ctx.err;
   if (P > 1) {
     p.S_dst = static_cast<float*>(a.ws);

@@ -24,6 +24,9 @@ struct StateArgs {
   int dt;            // 0 = fp32, 1 = bf16
   void* ws;
   size_t ws_bytes;
+  // Associative mode only: run the chunks from the last to the first and keep, inside a chunk,
+  // the pairs with key token >= query token (the transposed causal mask). Used by the backward.
+  int reverse = 0;
 };
 
 struct InplaceArgs {
@@ -69,6 +72,26 @@ size_t assoc_workspace_bytes(int B, int H, int T, int d, int C);
 bool assoc_supported(int d, int C, int dt);
 int launch_assoc(const StateArgs& a, const LaunchCtx& ctx);
 int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx);
+size_t assoc_bwd_workspace_bytes(int B, int H, int T, int d, int C);
+struct AssocBwdArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const float* eta;  // [B,H,T] or nullptr
+  float eta_scalar;
+  const float* S0;   // [B,H,d,d] or nullptr
+  const void* dO;
+  const float* dS_out;  // [B,H,d,d] or nullptr
+  void* dQ;
+  void* dK;
+  void* dV;
+  float* deta;       // [B,H,T]
+  float* dS0;        // [B,H,d,d]
+  int B, H, T, d, C;
+  void* ws;
+  size_t ws_bytes;
+};
+int launch_assoc_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx);
 
 // In-Place W_down.
 size_t inplace_workspace_bytes(int T, int Dff, int D, int C);

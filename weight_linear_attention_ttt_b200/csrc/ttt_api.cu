@@ -223,6 +223,58 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
   return finish(launch_assoc(a, ctx), msg);
 }
 
+size_t ttt_assoc_scan_bwd_workspace_size(int B, int H, int T, int d, int C, int dt) {
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0 ||
+      !assoc_supported(d, C, dt))
+    return 0;
+  return assoc_bwd_workspace_bytes(B, H, T, d, C);
+}
+
+int ttt_assoc_scan_bwd(const void* Q, const void* K, const void* V, const float* eta,
+                       float eta_scalar, const float* S0, const void* dO, const float* dS_out,
+                       void* dQ, void* dK, void* dV, float* deta, float* dS0, int B, int H,
+                       int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
+  const std::string f("ttt_assoc_scan_bwd");
+  if (!Q || !K || !V || !dO || !dQ || !dK || !dV || !deta || !dS0)
+    return fail(TTT_ERR_INVALID_ARG, f + ": Q, K, V, dO and every output must be non-null");
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0)
+    return fail(TTT_ERR_INVALID_ARG, f + ": B, H, T, d and C must be positive");
+  if (T % C != 0) return fail(TTT_ERR_INVALID_ARG, f + ": T must be a multiple of C");
+  if (dt != TTT_DTYPE_F32 && dt != TTT_DTYPE_BF16)
+    return fail(TTT_ERR_INVALID_ARG, f + ": dtype must be TTT_DTYPE_F32 or TTT_DTYPE_BF16");
+  const void* ptrs[] = {Q, K, V, eta, S0, dO, dS_out, dQ, dK, dV, deta, dS0, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p))
+      return fail(TTT_ERR_INVALID_ARG, f + ": every device pointer must be 16-byte aligned");
+  if (!assoc_supported(d, C, dt))
+    return fail(TTT_ERR_UNSUPPORTED, f + ": supported bf16, d == 128, C == 64");
+  const size_t need = assoc_bwd_workspace_bytes(B, H, T, d, C);
+  if (!workspace || workspace_bytes < need)
+    return fail(TTT_ERR_WORKSPACE, f + ": workspace smaller than ttt_assoc_scan_bwd_workspace_size()");
+  const size_t nx = (size_t)B * H * T * d * 2, ns = (size_t)B * H * d * d * 4;
+  const size_t ne = (size_t)B * H * T * 4;
+  struct R { const void* p; size_t n; };
+  const R ins[] = {{Q, nx}, {K, nx}, {V, nx}, {dO, nx}, {eta, ne}, {S0, ns}, {dS_out, ns}};
+  const R outs[] = {{dQ, nx}, {dK, nx}, {dV, nx}, {deta, ne}, {dS0, ns},
+                    {workspace, workspace_bytes}};
+  for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+    for (const R& in : ins)
+      if (in.p && overlap(outs[i].p, outs[i].n, in.p, in.n))
+        return fail(TTT_ERR_INVALID_ARG, f + ": outputs and workspace must not overlap inputs");
+    for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+      if (overlap(outs[i].p, outs[i].n, outs[j].p, outs[j].n))
+        return fail(TTT_ERR_INVALID_ARG, f + ": outputs and workspace must not overlap");
+  }
+  AssocBwdArgs a{Q, K, V, eta, eta_scalar, S0, dO, dS_out, dQ, dK, dV, deta, dS0, B, H, T, d, C,
+                 workspace, workspace_bytes};
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  return finish(launch_assoc_bwd(a, ctx), msg);
+}
+
 int ttt_assoc_state_fwd(const void* K, const void* V, const float* eta, float eta_scalar,
                         float* dS, int B, int H, int T, int d, int C, int dt,
                         cudaStream_t stream) {
