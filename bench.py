@@ -30,11 +30,18 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "TTT-layer fwd tokens/s on 1 B200; % of bf16 tensor-peak/HBM roofline"
+# the backward of the associative mode is measured the same way, as backward tokens/s
+METRIC_BWD = "TTT-layer bwd tokens/s on 1 B200; % of bf16 tensor-peak/HBM roofline"
+
+
+def metric_of(w) -> str:
+    return METRIC_BWD if w.kind.endswith("_bwd") else METRIC
 DEFAULT_WORKLOAD = "dual_bf16_B8H12T2048_d64C16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DOMINANT_KERNEL = {"dual": ("dual_mma_kernel", "dual_mma.cu"),
                    "assoc": ("assoc_chunk_kernel", "assoc_scan.cu"),
-                   "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu")}
+                   "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu"),
+                   "assoc_bwd": ("assoc_chunk_kernel", "assoc_scan.cu")}
 
 
 def peaks():
@@ -150,6 +157,18 @@ def make_call(w, x, stream_outputs=None):
         return lambda: ttt.ttt_assoc_scan_fwd(x["Q"], x["K"], x["V"], x["eta"], None, C=w.C,
                                               eta_scalar=x["eta_scalar"], O=O, S_out=S,
                                               workspace=ws)
+    if w.kind == "assoc_bwd":
+        dev = x["Q"].device
+        outs = dict(dQ=torch.empty_like(x["Q"]), dK=torch.empty_like(x["Q"]),
+                    dV=torch.empty_like(x["Q"]),
+                    deta=torch.empty((w.B, w.H, w.T), device=dev, dtype=torch.float32),
+                    dS0=torch.empty((w.B, w.H, w.d, w.d), device=dev, dtype=torch.float32))
+        lib = ttt.load_library()
+        nbytes = lib.ttt_assoc_scan_bwd_workspace_size(w.B, w.H, w.T, w.d, w.C, 1)
+        ws = torch.empty(max(nbytes, 16), device=dev, dtype=torch.uint8)
+        return lambda: ttt.ttt_assoc_scan_bwd(x["Q"], x["K"], x["V"], x["eta"], None, x["dO"],
+                                              x["dS_out"], C=w.C, eta_scalar=x["eta_scalar"],
+                                              workspace=ws, **outs)
     if w.kind == "inplace":
         O = torch.empty((w.T, w.D), device=x["Z"].device, dtype=torch.bfloat16)
         Wf = torch.empty((w.Dff, w.D), device=x["Z"].device, dtype=torch.float32)
@@ -173,6 +192,9 @@ def e2e_measure(w, x, steps: int, warmup: int):
     scal = {k: v for k, v in x.items() if not torch.is_tensor(v)}
     if w.kind == "inplace":
         out_shapes = [((w.T, w.D), torch.bfloat16), ((w.Dff, w.D), torch.float32)]
+    elif w.kind == "assoc_bwd":
+        out_shapes = [((w.B, w.H, w.T, w.d), x["Q"].dtype)] * 3 + [
+            ((w.B, w.H, w.T), torch.float32), ((w.B, w.H, w.d, w.d), torch.float32)]
     else:
         out_shapes = [((w.B, w.H, w.T, w.d), x["Q"].dtype), ((w.B, w.H, w.d, w.d), torch.float32)]
     outs_h = [torch.empty(s, dtype=dt).pin_memory() for s, dt in out_shapes]
@@ -214,11 +236,14 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
 
     threads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    if w.kind in ("dual", "assoc"):
+    if w.kind in ("dual", "assoc", "assoc_bwd"):
         streams = [(b, h) for b in range(w.B) for h in range(w.H)]
         Q, K, V = (x[k].float().cpu().numpy() for k in ("Q", "K", "V"))
         eta = None if x["eta"] is None else x["eta"].cpu().numpy()
         W0 = x["W0"].cpu().numpy()
+        if w.kind == "assoc_bwd":
+            dO = x["dO"].float().cpu().numpy()
+            G = x["dS_out"].cpu().numpy()
         # probe the cost of one chunk-run of one stream to size the sample
         tok = 0
         n_streams = 0
@@ -230,6 +255,9 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
             if w.kind == "dual":
                 orc.dual_form_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
                                      W0[b, h], w.C)
+            elif w.kind == "assoc_bwd":
+                orc.assoc_backward_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
+                                          None, dO[b, h, :ncol], G[b, h])
             else:
                 orc.assoc_recurrence_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
                                             None)
@@ -238,7 +266,7 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
             if time.perf_counter() - t0 >= budget_s or n_streams >= len(streams):
                 break
         desc = (f"{n_streams} (b,h) stream(s) x {ncol} tokens of the workload, "
-                f"{'dual-form per-chunk loop' if w.kind == 'dual' else 'sequential recurrence'}"
+                f"{ {'dual': 'dual-form per-chunk loop', 'assoc': 'sequential recurrence'}.get(w.kind, 'adjoint sweeps of the recurrence')}"
                 f", numpy fp64, 1 thread")
         return tok / w.H, time.perf_counter() - t0, 1, desc
     # In-Place: every 80th output column over all chunks (columns are independent)
@@ -276,7 +304,7 @@ def run_reference(args, w, rank, world):
         sec_total += sec
     value = tok_total / sec_total
     ms = 1e3 * sec_total / args.steps
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+    line = {"impl": "reference", "metric": metric_of(w), "value": value, "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
@@ -357,7 +385,7 @@ def run_ours(args, w, rank, world, local_rank):
                  "duration_us": 1e3 * ms_per_step / max(1.0, launches_per_step)
                  if w.kind == "dual" else None})
 
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+    line = {"metric": metric_of(w), "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",

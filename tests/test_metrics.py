@@ -11,6 +11,7 @@ from weight_linear_attention_ttt_b200.shard import split_range
     ("dual_bf16_B2H32T32768_d64C16", 60.13e9, 1084.0, "hbm"),
     ("assoc_bf16_B4H16T65536_d128C64", 412.3e9, 4316.0, "hbm"),
     ("inplace_bf16_T32768_Dff9728_D2560_C1024", 3.264e12, 1122.5, "tensor"),
+    ("assoc_bwd_bf16_B4H16T65536_d128C64", 1.2370e12, 7558.1, "hbm"),
 ])
 def test_algorithmic_counts(name, flops, mbytes, bound):
     w = inp.WORKLOADS[name]

@@ -52,7 +52,8 @@ class Workload:
         return self.B * self.T if self.kind != "inplace" else self.T
 
 
-# The five workloads; index i uses seed 1000 + i.
+# The five workloads of the forward path use seeds 1000 + i; the backward of the associative
+# mode on the associative workload's shape uses 1005.
 WORKLOADS = {
     "dual_f32_B1H2T256_d32C16": Workload(
         "dual_f32_B1H2T256_d32C16", "dual", 1000, B=1, H=2, T=256, d=32, C=16, dtype="f32",
@@ -69,6 +70,9 @@ WORKLOADS = {
     "inplace_bf16_T32768_Dff9728_D2560_C1024": Workload(
         "inplace_bf16_T32768_Dff9728_D2560_C1024", "inplace", 1004, T=32768, C=1024,
         Dff=9728, D=2560, eta="const", eta_const=1e-3),
+    "assoc_bwd_bf16_B4H16T65536_d128C64": Workload(
+        "assoc_bwd_bf16_B4H16T65536_d128C64", "assoc_bwd", 1005, B=4, H=16, T=65536, d=128,
+        C=64, normalise=("Q", "K"), eta="sigmoid", w0="zero"),
 }
 WORKLOAD_ORDER = list(WORKLOADS)
 
@@ -138,6 +142,20 @@ def inplace_inputs(T: int, Dff: int, D: int, *, seed: int, device="cpu",
     return {"Z": Z, "Vhat": Vhat, "W0": W0, "eta": float(eta)}
 
 
+def assoc_bwd_inputs(B: int, H: int, T: int, d: int, *, seed: int, device="cpu",
+                     **recipe) -> dict:
+    """The associative inputs of ``dual_or_assoc_inputs`` (S0 = 0) plus the incoming gradients:
+    dO [B,H,T,d] bf16 ~ N(0,1) and dS_out [B,H,d,d] fp32 ~ N(0, 0.05^2), drawn in that order
+    from a generator seeded with seed + 1."""
+    out = dual_or_assoc_inputs(B, H, T, d, seed=seed, device=device, **recipe)
+    g = _gen(seed + 1, device)
+    out["dO"] = torch.randn((B, H, T, d), generator=g, device=device,
+                            dtype=torch.float32).to(torch.bfloat16).contiguous()
+    out["dS_out"] = (torch.randn((B, H, d, d), generator=g, device=device,
+                                 dtype=torch.float32) * 0.05).contiguous()
+    return out
+
+
 def make_inputs(w: Workload, device="cpu", *, seed: Optional[int] = None, **overrides) -> dict:
     """Inputs of a named workload (optionally with shape overrides for reduced cases)."""
     if overrides:
@@ -147,6 +165,10 @@ def make_inputs(w: Workload, device="cpu", *, seed: Optional[int] = None, **over
         return dual_or_assoc_inputs(w.B, w.H, w.T, w.d, seed=s, device=device, dtype=w.dtype,
                                     qkv=w.qkv, normalise=w.normalise, eta=w.eta,
                                     eta_const=w.eta_const, w0=w.w0)
+    if w.kind == "assoc_bwd":
+        return assoc_bwd_inputs(w.B, w.H, w.T, w.d, seed=s, device=device, dtype=w.dtype,
+                                qkv=w.qkv, normalise=w.normalise, eta=w.eta,
+                                eta_const=w.eta_const, w0=w.w0)
     if w.kind == "inplace":
         return inplace_inputs(w.T, w.Dff, w.D, seed=s, device=device, eta=w.eta_const)
     raise ValueError(w.kind)

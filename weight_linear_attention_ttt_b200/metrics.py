@@ -28,6 +28,14 @@ def algorithmic(w: Workload) -> dict:
         return {"flops": th * per_tok,
                 "bytes": th * (4 * w.d * e + eta_bytes) + w.B * w.H * state_bytes,
                 "tokens": w.B * w.T}
+    if w.kind == "assoc_bwd":
+        # three passes of the forward recurrence (dQ, and dV / dK through the state gradient);
+        # bytes: Q, K, V, dO in and dQ, dK, dV out (bf16), eta in and deta out (fp32), per
+        # stream dS_out in and dS0 out (the initial state is zero)
+        th = w.B * w.H * w.T
+        return {"flops": 3 * th * (4 * w.d * w.d + 4 * w.C * w.d),
+                "bytes": th * (7 * w.d * 2 + 8) + w.B * w.H * 2 * w.d * w.d * 4,
+                "tokens": w.B * w.T}
     if w.kind == "inplace":
         T, F, D = w.T, w.Dff, w.D
         return {"flops": 4 * F * D * T,
