@@ -40,7 +40,9 @@ W0 = 0; o = q(S0 + k^T v) for one token; the sequential recurrence vs. the chunk
 forms; eta folded into V; the In-Place block-causal linear-attention form and its one-chunk closed
 form; autograd ascent steps for the associative and In-Place deltas; hand-worked golden examples;
 the associative backward against central finite differences of the forward definition and
-against autograd of an independent torch restatement. Every function below has at least one pin.
+against autograd of an independent torch restatement; the momentum recurrence against the plain
+one at beta = 0, against its closed weighted-sum form and against hand-worked tokens. Every
+function below has at least one pin.
 """
 from __future__ import annotations
 
@@ -199,6 +201,44 @@ def assoc_scan(Q, K, V, eta, S0, *, threads: int = 1, streams=None, form: str = 
         O = O.reshape(B, H, T, d)
         S = S.reshape(B, H, d, d)
     return O, S
+
+
+def assoc_momentum_stream(Q, K, V, eta, beta: float, S0, M0):
+    """Associative mode with a momentum inner loop [KVB, momentum paragraph: with momentum SGD
+    the layer is still a weighted sum of linear-attention terms], one token at a time:
+        M_t = beta M_(t-1) + eta_t k_t^T v_t,   S_t = S_(t-1) + M_t,   o_t = q_t S_t
+    (the ascent gradient of <k S, v> is k^T v; the rate scales each token's gradient before it
+    enters the momentum; M_0 = M0, zeros by default). Returns (O [T, d], S_T, M_T)."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    T, d = Q.shape
+    e = _eta_stream(eta, T)
+    S = np.zeros((d, d)) if S0 is None else _f64(S0).copy()
+    M = np.zeros((d, d)) if M0 is None else _f64(M0).copy()
+    O = np.empty((T, d))
+    for t in range(T):
+        M = beta * M + e[t] * np.outer(K[t], V[t])
+        S = S + M
+        O[t] = Q[t] @ S
+    return O, S, M
+
+
+def assoc_momentum(Q, K, V, eta, beta: float, S0, M0, *, threads: int = 1, streams=None):
+    """All streams of [B, H, T, d] inputs; S0 / M0 [B, H, d, d] or None. Returns (O, S_T, M_T)."""
+    B, H, T, d = np.shape(Q)
+
+    def one(b, h):
+        e = eta if np.ndim(eta) == 0 else np.asarray(eta)[b, h]
+        s0 = None if S0 is None else np.asarray(S0)[b, h]
+        m0 = None if M0 is None else np.asarray(M0)[b, h]
+        return assoc_momentum_stream(np.asarray(Q)[b, h], np.asarray(K)[b, h],
+                                     np.asarray(V)[b, h], e, beta, s0, m0)
+
+    idx, res = _streams(one, None, B, H, threads, streams)
+    out = [np.stack([r[i] for r in res]) for i in range(3)]
+    if streams is None:
+        out = [out[0].reshape(B, H, T, d), out[1].reshape(B, H, d, d),
+               out[2].reshape(B, H, d, d)]
+    return tuple(out)
 
 
 def assoc_backward_stream(Q, K, V, eta, S0, dO, dS_out):

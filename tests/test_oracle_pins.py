@@ -422,3 +422,54 @@ def test_assoc_backward_pins_catch_planted_mistakes():
     for bad in ((True, False, False), (False, True, False), (False, False, True)):
         dK, dV = sweep(*bad)
         assert not (np.allclose(dK, ref[1], rtol=1e-6) and np.allclose(dV, ref[2], rtol=1e-6))
+
+
+# ----------------------------------------------------------------------------- momentum
+def test_momentum_beta_zero_is_the_plain_recurrence():
+    T, d = 20, 5
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.1, 0.6, T)
+    S0 = _rand(d, d)
+    O, S, M = orc.assoc_momentum_stream(Q, K, V, eta, 0.0, S0, None)
+    Or, Sr = orc.assoc_recurrence_stream(Q, K, V, eta, S0)
+    assert np.allclose(O, Or, rtol=1e-12, atol=1e-12) and np.allclose(S, Sr, rtol=1e-12)
+    assert np.allclose(M, eta[-1] * np.outer(K[-1], V[-1]), rtol=1e-12)
+
+
+@pytest.mark.parametrize("beta", [0.5, 0.9, 0.99])
+def test_momentum_closed_weighted_sum(beta):
+    """Unrolled, the momentum form is a linear-attention sum with weights
+    (1 - beta^(t-s+1)) / (1 - beta) on token s's update, plus the initial momentum's
+    contribution beta (1 - beta^t) / (1 - beta) M0 after t tokens (t counted from 1)."""
+    T, d = 17, 4
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.1, 0.6, T)
+    S0, M0 = _rand(d, d), _rand(d, d)
+    O, S, M = orc.assoc_momentum_stream(Q, K, V, eta, beta, S0, M0)
+    for t in range(T):
+        n = t + 1
+        St = S0 + beta * (1 - beta ** n) / (1 - beta) * M0
+        for s_ in range(t + 1):
+            St = St + (1 - beta ** (t - s_ + 1)) / (1 - beta) * eta[s_] * np.outer(K[s_], V[s_])
+        assert np.allclose(O[t], Q[t] @ St, rtol=1e-10, atol=1e-12)
+    Mt = beta ** T * M0 + sum(beta ** (T - 1 - s_) * eta[s_] * np.outer(K[s_], V[s_])
+                              for s_ in range(T))
+    assert np.allclose(M, Mt, rtol=1e-10, atol=1e-12)
+
+
+def test_momentum_two_tokens_by_hand():
+    """d = 1: q = (1, 2), k = (1, 1), v = (3, 5), eta = (0.5, 1), beta = 0.5, S0 = M0 = 0.
+    M1 = 1.5, S1 = 1.5, o1 = 1.5; M2 = 0.75 + 5 = 5.75, S2 = 7.25, o2 = 14.5."""
+    O, S, M = orc.assoc_momentum_stream([[1.0], [2.0]], [[1.0], [1.0]], [[3.0], [5.0]],
+                                        [0.5, 1.0], 0.5, None, None)
+    assert np.allclose(O[:, 0], [1.5, 14.5]) and np.isclose(S[0, 0], 7.25)
+    assert np.isclose(M[0, 0], 5.75)
+
+
+def test_momentum_all_streams_helper():
+    B, H, T, d = 2, 3, 6, 3
+    Q, K, V = _rand(B, H, T, d), _rand(B, H, T, d), _rand(B, H, T, d)
+    O, S, M = orc.assoc_momentum(Q, K, V, 0.25, 0.8, None, None)
+    o, s_, m = orc.assoc_momentum_stream(Q[1, 2], K[1, 2], V[1, 2], 0.25, 0.8, None, None)
+    assert np.array_equal(O[1, 2], o) and np.array_equal(S[1, 2], s_)
+    assert np.array_equal(M[1, 2], m)
