@@ -120,6 +120,27 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
                        cudaStream_t stream);
 
 /* --------------------------------------------------------------------------------------------
+ * Associative mode with a momentum inner loop ("KV 바인딩 기반 테스트 시간 학습은 사실상 선형
+ * 어텐션이다", momentum paragraph: with momentum SGD the layer remains a weighted sum of
+ * linear-attention terms), per stream:
+ *     M_t = beta M_(t-1) + eta_t k_t^T v_t,   S_t = S_(t-1) + M_t,   o_t = q_t S_t
+ *  (M_0 = M0, S_0 = S0; the rate scales each token's gradient before it enters the momentum).
+ *  Q, K, V, O [B,H,T,d] bf16; eta [B,H,T] fp32 or NULL (eta_scalar); S0, M0 [B,H,d,d] fp32 or
+ *  NULL (zeros); S_out, M_out [B,H,d,d] fp32 (S_out may equal S0, M_out may equal M0).
+ *  beta in [0.25, 0.9] (beta = 0 is ttt_assoc_scan_fwd; the two-pass evaluation subtracts
+ *  outputs of size ~1/(1 - beta), which bounds beta for bf16 outputs). Supported: bf16,
+ *  d == 128, C == 64.
+ *  Workspace: ttt_assoc_momentum_workspace_size() bytes. Runs as one plain associative pass, one
+ *  decayed pass and an elementwise combination (see assoc_momentum.cu).
+ * ------------------------------------------------------------------------------------------ */
+size_t ttt_assoc_momentum_workspace_size(int B, int H, int T, int d, int C, int dt);
+int ttt_assoc_momentum_fwd(const void* Q, const void* K, const void* V, const float* eta,
+                           float eta_scalar, float beta, const float* S0, const float* M0,
+                           void* O, float* S_out, float* M_out, int B, int H, int T, int d,
+                           int C, int dt, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/* --------------------------------------------------------------------------------------------
  * Backward of the associative mode (the gradients that outer-loop training of the layer needs,
  * "KV 바인딩 기반 테스트 시간 학습은 사실상 선형 어텐션이다": the layer is trained end to end
  * through its inner updates). For the forward above and a scalar loss L with

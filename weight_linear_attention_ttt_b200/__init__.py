@@ -26,6 +26,7 @@ EXPORTED_SYMBOLS = (
     "ttt_linear_dual_workspace_size", "ttt_linear_dual_fwd",
     "ttt_assoc_scan_workspace_size", "ttt_assoc_scan_fwd", "ttt_assoc_state_fwd",
     "ttt_assoc_scan_bwd_workspace_size", "ttt_assoc_scan_bwd",
+    "ttt_assoc_momentum_workspace_size", "ttt_assoc_momentum_fwd",
     "ttt_state_prefix_sum",
     "inplace_ttt_workspace_size", "inplace_ttt_chunk_fwd",
     "inplace_ttt_noalloc_max_scratch_bytes", "inplace_ttt_chunk_fwd_noalloc",
@@ -69,12 +70,16 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         getattr(lib, name).restype = c_int
         getattr(lib, name).argtypes = state_args
     for name in ("ttt_linear_dual_workspace_size", "ttt_assoc_scan_workspace_size",
-                 "ttt_assoc_scan_bwd_workspace_size"):
+                 "ttt_assoc_scan_bwd_workspace_size", "ttt_assoc_momentum_workspace_size"):
         getattr(lib, name).restype = c_size
         getattr(lib, name).argtypes = [c_int] * 6
     lib.ttt_assoc_scan_bwd.restype = c_int
     lib.ttt_assoc_scan_bwd.argtypes = [vp, vp, vp, fp, c_float, fp, vp, fp, vp, vp, vp, fp, fp,
                                        c_int, c_int, c_int, c_int, c_int, c_int, vp, c_size, vp]
+    lib.ttt_assoc_momentum_fwd.restype = c_int
+    lib.ttt_assoc_momentum_fwd.argtypes = [vp, vp, vp, fp, c_float, c_float, fp, fp, vp, fp, fp,
+                                           c_int, c_int, c_int, c_int, c_int, c_int, vp, c_size,
+                                           vp]
     lib.ttt_assoc_state_fwd.restype = c_int
     lib.ttt_assoc_state_fwd.argtypes = [vp, vp, fp, c_float, fp, c_int, c_int, c_int, c_int,
                                         c_int, c_int, vp]
@@ -211,6 +216,44 @@ def ttt_assoc_scan_bwd(Q, K, V, eta, S0, dO, dS_out=None, *, C: int, eta_scalar:
                                 _stream_ptr(stream))
     _check("ttt_assoc_scan_bwd", st)
     return dQ, dK, dV, deta, dS0
+
+
+def ttt_assoc_momentum_fwd(Q, K, V, eta, beta: float, S0=None, M0=None, *, C: int,
+                           eta_scalar: float = 0.0, O=None, S_out=None, M_out=None,
+                           workspace=None, stream=None) -> Tuple:
+    """Associative mode with a momentum inner loop (M = beta M + eta k^T v, S += M, o = q S).
+    Returns (O, S_out, M_out); see include/ttt.h."""
+    import torch
+
+    lib = load_library()
+    _require(Q.dim() == 4, "Q, K, V must be [B, H, T, d]")
+    B, H, T, d = Q.shape
+    for t in (Q, K, V):
+        _require(t.is_cuda and t.is_contiguous() and t.shape == Q.shape and t.dtype == Q.dtype,
+                 "Q, K, V must be contiguous CUDA tensors of one shape and dtype")
+    dt = _dtype_code(Q)
+    if eta is not None:
+        _require(eta.is_cuda and eta.dtype == torch.float32 and eta.is_contiguous() and
+                 tuple(eta.shape) == (B, H, T), "eta must be a contiguous fp32 [B, H, T] tensor")
+    for t in (S0, M0):
+        if t is not None:
+            _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
+                     tuple(t.shape) == (B, H, d, d), "states must be fp32 [B, H, d, d]")
+    O = torch.empty_like(Q) if O is None else O
+    if S_out is None:
+        S_out = torch.empty((B, H, d, d), device=Q.device, dtype=torch.float32)
+    if M_out is None:
+        M_out = torch.empty((B, H, d, d), device=Q.device, dtype=torch.float32)
+    ws_bytes = lib.ttt_assoc_momentum_workspace_size(B, H, T, d, C, dt)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, device=Q.device, dtype=torch.uint8)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.ttt_assoc_momentum_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta),
+                                    ctypes.c_float(eta_scalar), ctypes.c_float(beta), _ptr(S0),
+                                    _ptr(M0), _ptr(O), _ptr(S_out), _ptr(M_out), B, H, T, d, C,
+                                    dt, _ptr(workspace), wsz, _stream_ptr(stream))
+    _check("ttt_assoc_momentum_fwd", st)
+    return O, S_out, M_out
 
 
 def ttt_assoc_state_fwd(K, V, eta=None, *, C: int, eta_scalar: float = 0.0, dS=None,

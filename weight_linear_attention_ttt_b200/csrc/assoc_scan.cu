@@ -45,6 +45,7 @@ namespace {
 
 constexpr int D = 128;         // head dim
 constexpr int C = 64;          // chunk
+constexpr float H_MID = 0.5f * (C - 1);   // middle of a chunk (decay mode)
 constexpr int THREADS = 480;   // TMA warp, MMA warp, 3 groups of 4 warps, score warp
 
 // shared-memory map (bytes from the 1024-aligned base); pass 1 loads no Q and writes no O
@@ -61,7 +62,7 @@ struct Smem {
   static constexpr int P_OFF = STAGES * STAGE;                // 2 x [64 t][64 s] bf16
   static constexpr int O_OFF = P_OFF + (SO ? 0 : 2 * 8192);   // 2 x [64 t][128 d_out] bf16
   static constexpr int BAR_OFF = O_OFF + (SO ? 0 : 2 * 16384);
-  static constexpr int BYTES = 1024 + BAR_OFF + 256;
+  static constexpr int BYTES = 1024 + BAR_OFF + 768;   // barriers, then two 64-float tables
   static_assert(BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -80,6 +81,14 @@ struct AssocParams {
   float* S_dst;             // pass 1: [BH, P-1, D, D] increments; pass 2: S_out [BH, D, D]
   int T, P, part_len;
   int reverse;              // chunks last to first, transposed causal mask
+  float eta_mul;            // every rate multiplied by this
+  // Decay mode (one superchunk): the state follows M_t = beta M_(t-1) + eta_t k_t^T v_t and
+  // o_t = q_t M_t (momentum). In a chunk with local token index i and h = (C - 1) / 2 the
+  // kernel runs the plain chunk step on values scaled by beta^(h - i) from a state holding
+  // beta^(h+1) M, multiplies output row i by beta^(i - h) and the state by beta^C after each
+  // update; the final state is beta^h times what TMEM holds.
+  int decay;
+  float beta;
   unsigned* err;
 };
 
@@ -98,7 +107,7 @@ __device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
   return r != 0;
 }
 
-template <bool SO>
+template <bool SO, bool DECAY = false>
 __global__ void __launch_bounds__(THREADS, 1)
     assoc_chunk_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -149,11 +158,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(sdone, 1);
     fence_mbar_init();
   }
+  if (DECAY && threadIdx.x < C) {
+    const float x = (float)threadIdx.x - H_MID;
+    reinterpret_cast<float*>(smem + L::BAR_OFF + 256)[threadIdx.x] = powf(p.beta, -x);
+    reinterpret_cast<float*>(smem + L::BAR_OFF + 512)[threadIdx.x] = powf(p.beta, x);
+  }
   if (warp == 1) umma::tmem_alloc(tslot, TM_COLS);
   umma::fence_before();
   __syncthreads();
   umma::fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::BAR_OFF + 168);
+  // decay-mode factors by local token index: beta^(h - i) on values, beta^(i - h) on outputs
+  const uint32_t evfac = bar + 256, ocfac = bar + 512;
 
   // State and output warps (pass 2): bf16 copy of 64 of the 128 state columns for `chunk`.
   // Lane = d_out row of S^T; `half` selects d_in columns [64 half, 64 half + 64).
@@ -164,6 +180,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     umma::wait_ld();
     umma::reg_fence(a0);
     umma::reg_fence(a1);
+    if (DECAY && chunk > 0) {
+      // state of the next chunk: beta^C times the updated one, written back in place
+      const float bc = powf(p.beta, (float)C);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        a0[j] = __float_as_uint(__uint_as_float(a0[j]) * bc);
+        a1[j] = __float_as_uint(__uint_as_float(a1[j]) * bc);
+      }
+      umma::st32x32(tmem + tl + TM_S + 64 * half, a0);
+      umma::st32x32(tmem + tl + TM_S + 64 * half + 32, a1);
+    }
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       o[j] = pack_bf16(__uint_as_float(a0[2 * j]), __uint_as_float(a0[2 * j + 1]));
@@ -181,13 +208,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     const float* src = nullptr;
     if (part == 0) src = p.S0 ? p.S0 + (size_t)stream * D * D : nullptr;
     else src = p.S_start + ((size_t)stream * (p.P - 1) + (part - 1)) * D * D;
+    const float sc = DECAY ? powf(p.beta, H_MID + 1.f) : 1.f;
 #pragma unroll 1
     for (int cc = 0; cc < 2; ++cc) {
       uint32_t v[32];
       const int din0 = 64 * half + 32 * cc;
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        v[j] = __float_as_uint(src ? src[(din0 + j) * D + dout] : 0.f);
+        v[j] = __float_as_uint(src ? sc * src[(din0 + j) * D + dout] : 0.f);
       umma::st32x32(tmem + tl + TM_S + din0, v);
     }
     umma::wait_st();
@@ -300,7 +328,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int i = otid + 128 * it;
           const int sub = i >> 9, w = i & 511;
           const uint32_t a = vt + sub * 8192 + swz<128>((w >> 3) * 128 + (w & 7) * 16);
-          const float f = e[it];
+          const float f = e[it] * p.eta_mul * (DECAY ? ldsf(evfac + 4 * (w >> 3)) : 1.f);
           sts128(a, make_uint4(pack_bf16(bf16_lo(x[it].x) * f, bf16_hi(x[it].x) * f),
                                pack_bf16(bf16_lo(x[it].y) * f, bf16_hi(x[it].y) * f),
                                pack_bf16(bf16_lo(x[it].z) * f, bf16_hi(x[it].z) * f),
@@ -367,6 +395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (ok && (SO || part == p.P - 1)) {
       float* dst = SO ? p.S_dst + ((size_t)stream * (p.P - 1) + part) * D * D
                       : p.S_dst + (size_t)stream * D * D;
+      const float sc = DECAY ? powf(p.beta, H_MID) : 1.f;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t v[32];
@@ -374,7 +403,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma::wait_ld();
         umma::reg_fence(v);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(32 * cc + j) * D + dout] = __uint_as_float(v[j]);
+        for (int j = 0; j < 32; ++j) dst[(32 * cc + j) * D + dout] = sc * __uint_as_float(v[j]);
       }
     }
   } else if (warp < 14) {
@@ -418,7 +447,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (t & 4) continue;
           const uint32_t* vv = t < 32 ? v0 : v1;
           const int tt = t & 31;
-          const float a = __uint_as_float(vv[tt]), a4 = __uint_as_float(vv[tt + 4]);
+          float a = __uint_as_float(vv[tt]), a4 = __uint_as_float(vv[tt + 4]);
+          if (DECAY) {
+            a *= ldsf(ocfac + 4 * t);
+            a4 *= ldsf(ocfac + 4 * (t + 4));
+          }
           const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
           const uint32_t w = odd ? pack_bf16(y, a4) : pack_bf16(a, y);
           const int row = odd ? t + 4 : t;
@@ -495,7 +528,8 @@ int choose_parts(int streams, int T) {
 template <bool STATE_ONLY>
 int launch_chunk(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const CUtensorMap& to, const AssocParams& p, int grid, const LaunchCtx& ctx) {
-  auto kern = assoc_chunk_kernel<STATE_ONLY>;
+  auto kern = (!STATE_ONLY && p.decay) ? assoc_chunk_kernel<STATE_ONLY, true>
+                                       : assoc_chunk_kernel<STATE_ONLY, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Smem<STATE_ONLY>::BYTES);
   if (e != cudaSuccess) {
@@ -540,6 +574,9 @@ int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
   p.P = 2;             // parts 0 .. P-2 = the single part [0, T)
   p.part_len = a.T;
   p.reverse = a.reverse;
+  p.eta_mul = a.eta_mul;
+  p.decay = a.decay;
+  p.beta = a.beta;
   p.err = ctx.err;
   return launch_chunk<true>(tq, tk, tv, to, p, BH, ctx);
 }
@@ -552,7 +589,7 @@ size_t assoc_workspace_bytes(int B, int H, int T, int d, int C_) {
 
 int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   const int BH = a.B * a.H;
-  const int P = choose_parts(BH, a.T);
+  const int P = a.decay ? 1 : choose_parts(BH, a.T);   // decay mode: one superchunk
   const size_t need = (size_t)BH * (P - 1) * D * D * sizeof(float);
   if (a.ws_bytes < need) {
     *ctx.msg = "ttt_assoc_scan_fwd: workspace smaller than ttt_assoc_scan_workspace_size()";
@@ -578,6 +615,9 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   p.P = P;
   p.part_len = a.T / P;
   p.reverse = a.reverse;
+  p.eta_mul = a.eta_mul;
+  p.decay = a.decay;
+  p.beta = a.beta;
   p.err = ctx.err;
   if (P > 1) {
     p.S_dst = static_cast<float*>(a.ws);

@@ -27,6 +27,11 @@ struct StateArgs {
   // Associative mode only: run the chunks from the last to the first and keep, inside a chunk,
   // the pairs with key token >= query token (the transposed causal mask). Used by the backward.
   int reverse = 0;
+  // Associative mode only: every rate multiplied by eta_mul; decay != 0 runs the momentum
+  // (decayed) recurrence M_t = beta M_(t-1) + eta_t k_t^T v_t, o_t = q_t M_t.
+  float eta_mul = 1.f;
+  int decay = 0;
+  float beta = 0.f;
 };
 
 struct InplaceArgs {
@@ -92,6 +97,24 @@ struct AssocBwdArgs {
   size_t ws_bytes;
 };
 int launch_assoc_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx);
+size_t assoc_momentum_workspace_bytes(int B, int H, int T, int d, int C);
+struct AssocMomentumArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const float* eta;
+  float eta_scalar;
+  float beta;
+  const float* S0;   // [B,H,d,d] or nullptr
+  const float* M0;   // [B,H,d,d] or nullptr
+  void* O;
+  float* S_out;
+  float* M_out;
+  int B, H, T, d, C;
+  void* ws;
+  size_t ws_bytes;
+};
+int launch_assoc_momentum(const AssocMomentumArgs& a, const LaunchCtx& ctx);
 
 // In-Place W_down.
 size_t inplace_workspace_bytes(int T, int Dff, int D, int C);

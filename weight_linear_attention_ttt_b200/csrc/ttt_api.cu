@@ -223,6 +223,64 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
   return finish(launch_assoc(a, ctx), msg);
 }
 
+size_t ttt_assoc_momentum_workspace_size(int B, int H, int T, int d, int C, int dt) {
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0 ||
+      !assoc_supported(d, C, dt))
+    return 0;
+  return assoc_momentum_workspace_bytes(B, H, T, d, C);
+}
+
+int ttt_assoc_momentum_fwd(const void* Q, const void* K, const void* V, const float* eta,
+                           float eta_scalar, float beta, const float* S0, const float* M0,
+                           void* O, float* S_out, float* M_out, int B, int H, int T, int d,
+                           int C, int dt, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+  const char* fn = "ttt_assoc_momentum_fwd";
+  const std::string f(fn);
+  StateArgs a{Q, K, V, eta, eta_scalar, S0, O, S_out, B, H, T, d, C, dt, workspace,
+              workspace_bytes};
+  int st = check_state_args(fn, a, 0);
+  if (st != TTT_OK) return st;
+  if (!M_out) return fail(TTT_ERR_INVALID_ARG, f + ": M_out must be non-null");
+  // The two-pass form subtracts two bf16 outputs of size ~1/(1 - beta) times the result
+  // early in a sequence; up to beta = 0.9 that stays within the bf16 accuracy bar.
+  if (!(beta >= 0.25f && beta <= 0.9f))
+    return fail(TTT_ERR_UNSUPPORTED, f + ": momentum coefficient must lie in [0.25, 0.9] (0 is "
+                                         "the plain associative mode)");
+  if (!assoc_supported(d, C, dt))
+    return fail(TTT_ERR_UNSUPPORTED, f + ": supported bf16, d == 128, C == 64");
+  st = check_state_args(fn, a, assoc_momentum_workspace_bytes(B, H, T, d, C));
+  if (st != TTT_OK) return st;
+  const void* extra[] = {M0, M_out};
+  for (const void* p : extra)
+    if (p && !aligned16(p))
+      return fail(TTT_ERR_INVALID_ARG, f + ": every device pointer must be 16-byte aligned");
+  const size_t nx = (size_t)B * H * T * d * 2, ns = (size_t)B * H * d * d * 4;
+  const size_t ne = (size_t)B * H * T * 4;
+  struct R { const void* p; size_t n; };
+  const R others[] = {{Q, nx}, {K, nx}, {V, nx}, {eta, ne}, {O, nx}, {S_out, ns}, {S0, ns},
+                      {workspace, workspace_bytes}};
+  for (const R& o : others)
+    if (o.p && overlap(M_out, ns, o.p, o.n))
+      return fail(TTT_ERR_INVALID_ARG, f + ": M_out must not overlap another argument");
+  if (M0 && M0 != M_out) {
+    const R outs[] = {{O, nx}, {S_out, ns}, {workspace, workspace_bytes}};
+    for (const R& o : outs)
+      if (overlap(M0, ns, o.p, o.n))
+        return fail(TTT_ERR_INVALID_ARG, f + ": M0 must not overlap O, S_out or the workspace");
+  }
+  if (overlap(workspace, workspace_bytes, O, nx) ||
+      overlap(workspace, workspace_bytes, S_out, ns))
+    return fail(TTT_ERR_INVALID_ARG, f + ": workspace overlaps an output");
+  AssocMomentumArgs m{Q, K, V, eta, eta_scalar, beta, S0, M0, O, S_out, M_out, B, H, T, d, C,
+                      workspace, workspace_bytes};
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  return finish(launch_assoc_momentum(m, ctx), msg);
+}
+
 size_t ttt_assoc_scan_bwd_workspace_size(int B, int H, int T, int d, int C, int dt) {
   if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0 ||
       !assoc_supported(d, C, dt))
