@@ -41,7 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 DOMINANT_KERNEL = {"dual": ("dual_mma_kernel", "dual_mma.cu"),
                    "assoc": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu"),
-                   "assoc_bwd": ("assoc_chunk_kernel", "assoc_scan.cu")}
+                   "assoc_bwd": ("assoc_chunk_kernel", "assoc_scan.cu"),
+                   "assoc_momentum": ("assoc_chunk_kernel", "assoc_scan.cu")}
 
 
 def peaks():
@@ -142,6 +143,7 @@ def make_call(w, x, stream_outputs=None):
     import torch
 
     import weight_linear_attention_ttt_b200 as ttt
+    from weight_linear_attention_ttt_b200 import inputs as inp
 
     if w.kind == "dual":
         O = torch.empty_like(x["Q"])
@@ -157,6 +159,18 @@ def make_call(w, x, stream_outputs=None):
         return lambda: ttt.ttt_assoc_scan_fwd(x["Q"], x["K"], x["V"], x["eta"], None, C=w.C,
                                               eta_scalar=x["eta_scalar"], O=O, S_out=S,
                                               workspace=ws)
+    if w.kind == "assoc_momentum":
+        dev = x["Q"].device
+        O = torch.empty_like(x["Q"])
+        S = torch.empty((w.B, w.H, w.d, w.d), device=dev, dtype=torch.float32)
+        M = torch.empty_like(S)
+        lib = ttt.load_library()
+        nbytes = lib.ttt_assoc_momentum_workspace_size(w.B, w.H, w.T, w.d, w.C, 1)
+        ws = torch.empty(max(nbytes, 16), device=dev, dtype=torch.uint8)
+        return lambda: ttt.ttt_assoc_momentum_fwd(x["Q"], x["K"], x["V"], x["eta"],
+                                                  inp.MOMENTUM_BETA, None, None, C=w.C,
+                                                  eta_scalar=x["eta_scalar"], O=O, S_out=S,
+                                                  M_out=M, workspace=ws)
     if w.kind == "assoc_bwd":
         dev = x["Q"].device
         outs = dict(dQ=torch.empty_like(x["Q"]), dK=torch.empty_like(x["Q"]),
@@ -192,6 +206,9 @@ def e2e_measure(w, x, steps: int, warmup: int):
     scal = {k: v for k, v in x.items() if not torch.is_tensor(v)}
     if w.kind == "inplace":
         out_shapes = [((w.T, w.D), torch.bfloat16), ((w.Dff, w.D), torch.float32)]
+    elif w.kind == "assoc_momentum":
+        out_shapes = [((w.B, w.H, w.T, w.d), x["Q"].dtype), ((w.B, w.H, w.d, w.d), torch.float32),
+                      ((w.B, w.H, w.d, w.d), torch.float32)]
     elif w.kind == "assoc_bwd":
         out_shapes = [((w.B, w.H, w.T, w.d), x["Q"].dtype)] * 3 + [
             ((w.B, w.H, w.T), torch.float32), ((w.B, w.H, w.d, w.d), torch.float32)]
@@ -233,10 +250,11 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
     import numpy as np
 
     from oracle import ttt_oracle as orc
+    from weight_linear_attention_ttt_b200 import inputs as inp
 
     threads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    if w.kind in ("dual", "assoc", "assoc_bwd"):
+    if w.kind in ("dual", "assoc", "assoc_bwd", "assoc_momentum"):
         streams = [(b, h) for b in range(w.B) for h in range(w.H)]
         Q, K, V = (x[k].float().cpu().numpy() for k in ("Q", "K", "V"))
         eta = None if x["eta"] is None else x["eta"].cpu().numpy()
@@ -255,6 +273,9 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
             if w.kind == "dual":
                 orc.dual_form_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
                                      W0[b, h], w.C)
+            elif w.kind == "assoc_momentum":
+                orc.assoc_momentum_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
+                                          inp.MOMENTUM_BETA, None, None)
             elif w.kind == "assoc_bwd":
                 orc.assoc_backward_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
                                           None, dO[b, h, :ncol], G[b, h])
@@ -266,7 +287,7 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
             if time.perf_counter() - t0 >= budget_s or n_streams >= len(streams):
                 break
         desc = (f"{n_streams} (b,h) stream(s) x {ncol} tokens of the workload, "
-                f"{ {'dual': 'dual-form per-chunk loop', 'assoc': 'sequential recurrence'}.get(w.kind, 'adjoint sweeps of the recurrence')}"
+                f"{ {'dual': 'dual-form per-chunk loop', 'assoc': 'sequential recurrence', 'assoc_momentum': 'momentum recurrence'}.get(w.kind, 'adjoint sweeps of the recurrence')}"
                 f", numpy fp64, 1 thread")
         return tok / w.H, time.perf_counter() - t0, 1, desc
     # In-Place: every 80th output column over all chunks (columns are independent)

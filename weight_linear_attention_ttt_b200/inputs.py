@@ -53,7 +53,8 @@ class Workload:
 
 
 # The five workloads of the forward path use seeds 1000 + i; the backward of the associative
-# mode on the associative workload's shape uses 1005.
+# mode and its momentum form, on the associative workload's shape, use 1005 and 1007.
+MOMENTUM_BETA = 0.9   # momentum coefficient of the momentum workload
 WORKLOADS = {
     "dual_f32_B1H2T256_d32C16": Workload(
         "dual_f32_B1H2T256_d32C16", "dual", 1000, B=1, H=2, T=256, d=32, C=16, dtype="f32",
@@ -70,6 +71,9 @@ WORKLOADS = {
     "inplace_bf16_T32768_Dff9728_D2560_C1024": Workload(
         "inplace_bf16_T32768_Dff9728_D2560_C1024", "inplace", 1004, T=32768, C=1024,
         Dff=9728, D=2560, eta="const", eta_const=1e-3),
+    "assoc_momentum_bf16_B4H16T65536_d128C64": Workload(
+        "assoc_momentum_bf16_B4H16T65536_d128C64", "assoc_momentum", 1007, B=4, H=16, T=65536,
+        d=128, C=64, normalise=("Q", "K"), eta="sigmoid", w0="zero"),
     "assoc_bwd_bf16_B4H16T65536_d128C64": Workload(
         "assoc_bwd_bf16_B4H16T65536_d128C64", "assoc_bwd", 1005, B=4, H=16, T=65536, d=128,
         C=64, normalise=("Q", "K"), eta="sigmoid", w0="zero"),
@@ -161,7 +165,7 @@ def make_inputs(w: Workload, device="cpu", *, seed: Optional[int] = None, **over
     if overrides:
         w = dataclasses.replace(w, **overrides)
     s = w.seed if seed is None else seed
-    if w.kind in ("dual", "assoc"):
+    if w.kind in ("dual", "assoc", "assoc_momentum"):
         return dual_or_assoc_inputs(w.B, w.H, w.T, w.d, seed=s, device=device, dtype=w.dtype,
                                     qkv=w.qkv, normalise=w.normalise, eta=w.eta,
                                     eta_const=w.eta_const, w0=w.w0)

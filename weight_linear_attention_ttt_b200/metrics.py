@@ -14,11 +14,19 @@ Vhat, W0 (bf16), O (bf16) and the final fp32 W once each.
 """
 from __future__ import annotations
 
+import dataclasses
+
 from .inputs import Workload
 
 
 def algorithmic(w: Workload) -> dict:
     """{'flops': F, 'bytes': B, 'tokens': N} for one call of the workload."""
+    if w.kind == "assoc_momentum":
+        # the momentum recurrence reads and writes what the plain one does, plus the momentum
+        # state (in and out); flops: the plain and the decayed chunk steps
+        a = algorithmic(dataclasses.replace(w, kind="assoc"))
+        return {"flops": 2 * a["flops"], "bytes": a["bytes"] + w.B * w.H * 2 * w.d * w.d * 4,
+                "tokens": a["tokens"]}
     if w.kind in ("dual", "assoc"):
         e = 4 if w.dtype == "f32" else 2
         th = w.B * w.H * w.T
