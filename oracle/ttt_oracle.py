@@ -317,3 +317,22 @@ def inplace_chunks(Z, Vhat, W0, eta: float, C: int, cols=None):
         O[c0:c0 + C] = z @ W
         W = W + eta * (z.T @ _f64(Vh[c0:c0 + C]))
     return O, W
+
+
+# --------------------------------------------------------------------------------------------
+# LM-aligned target for the In-Place update  [IPT, LM-aligned objective paragraph]
+# --------------------------------------------------------------------------------------------
+def lm_target(X, Wc, Wp):
+    """Vhat = conv(X) Wp: a depthwise 1D convolution over tokens that reaches one token ahead,
+    then a bias-free projection [IPT: the target is made from the token embeddings by a 1D
+    convolution and a projection and carries the next token's information].
+    X [T, Dm]; Wc [k, Dm] (tap i multiplies token t + 1 - i: the next token, the current one and
+    k - 2 before it; tokens outside [0, T) count as zero); Wp [Dm, D]. Returns Vhat [T, D]."""
+    X, Wc, Wp = _f64(X), _f64(Wc), _f64(Wp)
+    T, Dm = X.shape
+    U = np.zeros((T, Dm))
+    for i in range(Wc.shape[0]):
+        shift = 1 - i                      # U[t] += Wc[i] * X[t + shift]
+        lo, hi = max(0, -shift), min(T, T - shift)
+        U[lo:hi] += Wc[i][None, :] * X[lo + shift:hi + shift]
+    return U @ Wp

@@ -473,3 +473,43 @@ def test_momentum_all_streams_helper():
     o, s_, m = orc.assoc_momentum_stream(Q[1, 2], K[1, 2], V[1, 2], 0.25, 0.8, None, None)
     assert np.array_equal(O[1, 2], o) and np.array_equal(S[1, 2], s_)
     assert np.array_equal(M[1, 2], m)
+
+
+# ----------------------------------------------------------------------------- LM-aligned target
+def test_lm_target_brute_force():
+    """Against the definition written as plain loops on a tiny case."""
+    T, Dm, D, k = 7, 3, 2, 4
+    X, Wc, Wp = _rand(T, Dm), _rand(k, Dm), _rand(Dm, D)
+    got = orc.lm_target(X, Wc, Wp)
+    ref = np.zeros((T, D))
+    for t in range(T):
+        for n in range(D):
+            acc = 0.0
+            for j in range(Dm):
+                for i in range(k):
+                    tt = t + 1 - i
+                    if 0 <= tt < T:
+                        acc += Wc[i, j] * X[tt, j] * Wp[j, n]
+            ref[t, n] = acc
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_lm_target_single_taps_and_causality():
+    """Tap 1 alone reads the current token (Vhat = X Wp); tap 0 alone reads the next one (and
+    zero at the last token); Vhat_t changes with X_(t+1) but not with X_(t+2)."""
+    T, Dm, D = 9, 4, 3
+    X, Wp = _rand(T, Dm), _rand(Dm, D)
+    cur = np.zeros((4, Dm))
+    cur[1] = 1.0
+    assert np.allclose(orc.lm_target(X, cur, Wp), X @ Wp, rtol=1e-12)
+    nxt = np.zeros((4, Dm))
+    nxt[0] = 1.0
+    ref = np.vstack([X[1:] @ Wp, np.zeros((1, D))])
+    assert np.allclose(orc.lm_target(X, nxt, Wp), ref, rtol=1e-12, atol=1e-14)
+    Wc = _rand(4, Dm)
+    base = orc.lm_target(X, Wc, Wp)
+    X2 = X.copy()
+    X2[5] += 1.0
+    d = orc.lm_target(X2, Wc, Wp) - base
+    assert np.abs(d[4]).max() > 1e-6           # token 4 sees token 5 (the next one)
+    assert np.abs(d[:4]).max() == 0.0           # earlier tokens do not see two ahead
