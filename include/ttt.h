@@ -233,6 +233,32 @@ int inplace_ttt_chunk_fwd_noalloc(const void* Z, const void* Vhat, const void* W
                                   void* O, float* W_out, int T, int Dff, int D, int C,
                                   cudaStream_t stream);
 
+/* --------------------------------------------------------------------------------------------
+ * LM-aligned target of the In-Place update ("In-Place 테스트 시점 학습", LM-aligned objective
+ * paragraph: the target is made from the token embeddings by a 1D convolution and a projection
+ * and carries the next token's information). Reading: a depthwise convolution over tokens whose
+ * tap i multiplies token t + 1 - i (tokens outside [0, T) are zero), then a bias-free projection:
+ *     Vhat[t, :] = (sum_i Wc[i, :] * X[t + 1 - i, :]) Wp
+ *  X [T, Dm] bf16; Wc [k, Dm] fp32; Wp [Dm, D] bf16; Vhat [T, D] bf16 (output).
+ *  Supported: T % 128 == 0, Dm % 128 == 0, D % 64 == 0, 1 <= k <= 8.
+ *  Workspace: ttt_lm_target_workspace_size() bytes (the convolved embeddings, bf16).
+ *  Errors: TTT_ERR_INVALID_ARG (null/misaligned/overlapping pointers), TTT_ERR_UNSUPPORTED
+ *  (shape), TTT_ERR_WORKSPACE, TTT_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------ */
+size_t ttt_lm_target_workspace_size(int T, int Dm, int D, int k);
+int ttt_lm_target_fwd(const void* X, const float* Wc, const void* Wp, void* Vhat, int T, int Dm,
+                      int D, int k, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream);
+
+/* The In-Place chunk update with its LM-aligned target formed in front of it: Vhat as above
+ *  (into the workspace), then inplace_ttt_chunk_fwd(Z, Vhat, W0, eta, O, W_out, T, Dff, D, C).
+ *  Arguments as for the two calls; workspace: inplace_ttt_lm_workspace_size() bytes. */
+size_t inplace_ttt_lm_workspace_size(int T, int Dff, int D, int Dm, int C, int k);
+int inplace_ttt_lm_chunk_fwd(const void* Z, const void* X, const float* Wc, const void* Wp,
+                             const void* W0, float eta, void* O, float* W_out, int T, int Dff,
+                             int D, int Dm, int C, int k, void* workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

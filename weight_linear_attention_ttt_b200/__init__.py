@@ -30,6 +30,8 @@ EXPORTED_SYMBOLS = (
     "ttt_state_prefix_sum",
     "inplace_ttt_workspace_size", "inplace_ttt_chunk_fwd",
     "inplace_ttt_noalloc_max_scratch_bytes", "inplace_ttt_chunk_fwd_noalloc",
+    "ttt_lm_target_workspace_size", "ttt_lm_target_fwd",
+    "inplace_ttt_lm_workspace_size", "inplace_ttt_lm_chunk_fwd",
 )
 
 _LIB: Optional[ctypes.CDLL] = None
@@ -95,6 +97,15 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.inplace_ttt_chunk_fwd_noalloc.restype = c_int
     lib.inplace_ttt_chunk_fwd_noalloc.argtypes = [vp, vp, vp, c_float, vp, fp, c_int, c_int,
                                                   c_int, c_int, vp]
+    lib.ttt_lm_target_workspace_size.restype = c_size
+    lib.ttt_lm_target_workspace_size.argtypes = [c_int] * 4
+    lib.ttt_lm_target_fwd.restype = c_int
+    lib.ttt_lm_target_fwd.argtypes = [vp, fp, vp, vp, c_int, c_int, c_int, c_int, vp, c_size, vp]
+    lib.inplace_ttt_lm_workspace_size.restype = c_size
+    lib.inplace_ttt_lm_workspace_size.argtypes = [c_int] * 6
+    lib.inplace_ttt_lm_chunk_fwd.restype = c_int
+    lib.inplace_ttt_lm_chunk_fwd.argtypes = [vp, vp, fp, vp, vp, c_float, vp, fp, c_int, c_int,
+                                             c_int, c_int, c_int, c_int, vp, c_size, vp]
     if path is None:
         _LIB = lib
     return lib
@@ -363,3 +374,63 @@ def read_device_error() -> int:
     v = ctypes.c_uint(0)
     _check("ttt_read_device_error", load_library().ttt_read_device_error(ctypes.byref(v)))
     return int(v.value)
+
+
+def _lm_checks(X, Wc, Wp):
+    import torch
+
+    _require(X.dim() == 2 and X.is_cuda and X.is_contiguous() and X.dtype == torch.bfloat16,
+             "X must be a contiguous bf16 [T, Dm] CUDA tensor")
+    _require(Wc.dim() == 2 and Wc.is_cuda and Wc.is_contiguous() and Wc.dtype == torch.float32
+             and Wc.shape[1] == X.shape[1], "Wc must be a contiguous fp32 [k, Dm] CUDA tensor")
+    _require(Wp.dim() == 2 and Wp.is_cuda and Wp.is_contiguous() and Wp.dtype == torch.bfloat16
+             and Wp.shape[0] == X.shape[1], "Wp must be a contiguous bf16 [Dm, D] CUDA tensor")
+
+
+def ttt_lm_target_fwd(X, Wc, Wp, *, Vhat=None, workspace=None, stream=None):
+    """LM-aligned target Vhat = conv(X; Wc) Wp (see include/ttt.h). Returns Vhat [T, D] bf16."""
+    import torch
+
+    lib = load_library()
+    _lm_checks(X, Wc, Wp)
+    T, Dm = X.shape
+    k, D = Wc.shape[0], Wp.shape[1]
+    if Vhat is None:
+        Vhat = torch.empty((T, D), device=X.device, dtype=torch.bfloat16)
+    nbytes = lib.ttt_lm_target_workspace_size(T, Dm, D, k)
+    if workspace is None and nbytes:
+        workspace = torch.empty(nbytes, device=X.device, dtype=torch.uint8)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.ttt_lm_target_fwd(_ptr(X), _ptr(Wc), _ptr(Wp), _ptr(Vhat), T, Dm, D, k,
+                               _ptr(workspace), wsz, _stream_ptr(stream))
+    _check("ttt_lm_target_fwd", st)
+    return Vhat
+
+
+def inplace_ttt_lm_chunk_fwd(Z, X, Wc, Wp, W0, eta: float, *, C: int, O=None, W_out=None,
+                             workspace=None, stream=None) -> Tuple:
+    """In-Place chunk update whose target is the LM-aligned Vhat formed in front of it.
+    Returns (O, W_out); see include/ttt.h."""
+    import torch
+
+    lib = load_library()
+    _lm_checks(X, Wc, Wp)
+    _require(Z.dim() == 2 and Z.is_cuda and Z.is_contiguous() and Z.dtype == torch.bfloat16
+             and Z.shape[0] == X.shape[0], "Z must be a contiguous bf16 [T, Dff] CUDA tensor")
+    T, Dff = Z.shape
+    Dm, k, D = X.shape[1], Wc.shape[0], Wp.shape[1]
+    _require(tuple(W0.shape) == (Dff, D) and W0.dtype == torch.bfloat16 and W0.is_contiguous(),
+             "W0 must be a contiguous bf16 [Dff, D] tensor")
+    if O is None:
+        O = torch.empty((T, D), device=Z.device, dtype=torch.bfloat16)
+    if W_out is None:
+        W_out = torch.empty((Dff, D), device=Z.device, dtype=torch.float32)
+    nbytes = lib.inplace_ttt_lm_workspace_size(T, Dff, D, Dm, C, k)
+    if workspace is None and nbytes:
+        workspace = torch.empty(nbytes, device=Z.device, dtype=torch.uint8)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.inplace_ttt_lm_chunk_fwd(_ptr(Z), _ptr(X), _ptr(Wc), _ptr(Wp), _ptr(W0),
+                                      ctypes.c_float(eta), _ptr(O), _ptr(W_out), T, Dff, D, Dm,
+                                      C, k, _ptr(workspace), wsz, _stream_ptr(stream))
+    _check("inplace_ttt_lm_chunk_fwd", st)
+    return O, W_out

@@ -386,6 +386,64 @@ int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
   return kOk;
 }
 
+// Plain projection Out[M, N] = A[M, K] B[K, N] (bf16 in, fp32 accumulate, bf16 out) on the read
+// tiles of the kernel above: one "chunk" of M rows whose tile list has no update tiles.
+template <int BN>
+int launch_proj_bn(const void* A, const void* B, void* Out, int M, int K, int N, int* counter,
+                   const LaunchCtx& ctx) {
+  using Cfg = IpCfg<BN>;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  CUtensorMap tak, tam, tb, tunused;
+  const uint64_t da[2] = {(uint64_t)K, (uint64_t)M};
+  const uint64_t db[2] = {(uint64_t)N, (uint64_t)K};
+  const uint32_t bk[2] = {64, 128}, bm[2] = {64, 64}, bwf[2] = {32, 128};
+  if (!make_tmap_2d(&tak, A, bf, da, (uint64_t)K * 2, bk, sw, ctx.msg) ||
+      !make_tmap_2d(&tam, A, bf, da, (uint64_t)K * 2, bm, sw, ctx.msg) ||
+      !make_tmap_2d(&tb, B, bf, db, (uint64_t)N * 2, bm, sw, ctx.msg))
+    return kCuda;
+  // the update-tile maps are never used without update tiles; an fp32 view of B fills the slot
+  const uint64_t dw[2] = {(uint64_t)(N / 2), (uint64_t)K};
+  if (!make_tmap_2d(&tunused, B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dw, (uint64_t)N * 2, bwf, sw,
+                    ctx.msg))
+    return kCuda;
+  auto kern = inplace_chunk_kernel<BN>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+  if (e == cudaSuccess) e = cudaMemsetAsync(counter, 0, sizeof(int), ctx.stream);
+  if (e != cudaSuccess) {
+    *ctx.msg = std::string("projection setup: ") + cudaGetErrorString(e);
+    return kCuda;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  IpParams p;
+  p.W0 = static_cast<const __nv_bfloat16*>(B);
+  p.Wout = nullptr;
+  p.Wbf_next = nullptr;
+  p.O = static_cast<__nv_bfloat16*>(Out);
+  p.eta = 0.f;
+  p.first = 1;
+  p.tok0 = 0;
+  p.C = M;
+  p.Dff = K;
+  p.D = N;
+  p.n_read = (M / BM) * (N / BN);
+  p.n_total = p.n_read;
+  p.counter = counter;
+  p.err = ctx.err;
+  kern<<<std::min(sms, p.n_read), THREADS, Cfg::SMEM, ctx.stream>>>(tak, tam, tb, tam, tunused,
+                                                                     p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    *ctx.msg = std::string("projection launch: ") + cudaGetErrorString(e);
+    return kCuda;
+  }
+  count_launch();
+  return kOk;
+}
+
 }  // namespace
 
 size_t inplace_workspace_bytes(int T, int Dff, int D, int C) {
@@ -413,6 +471,15 @@ bool inplace_supported(int T, int Dff, int D, int C, std::string* why) {
     return false;
   }
   return true;
+}
+
+int launch_projection(const void* A, const void* B, void* Out, int M, int K, int N, int* counter,
+                      const LaunchCtx& ctx) {
+  switch (pick_bn(N)) {
+    case 256: return launch_proj_bn<256>(A, B, Out, M, K, N, counter, ctx);
+    case 128: return launch_proj_bn<128>(A, B, Out, M, K, N, counter, ctx);
+    default: return launch_proj_bn<64>(A, B, Out, M, K, N, counter, ctx);
+  }
 }
 
 int launch_inplace(const InplaceArgs& a, const LaunchCtx& ctx) {

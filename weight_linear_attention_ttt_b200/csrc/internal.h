@@ -115,6 +115,13 @@ struct AssocMomentumArgs {
   size_t ws_bytes;
 };
 int launch_assoc_momentum(const AssocMomentumArgs& a, const LaunchCtx& ctx);
+// Out[M, N] = A[M, K] B[K, N], bf16, on the In-Place kernel's read tiles (M % 128 == 0,
+// K % 64 == 0, N % 64 == 0); `counter` is one int of device memory.
+int launch_projection(const void* A, const void* B, void* Out, int M, int K, int N, int* counter,
+                      const LaunchCtx& ctx);
+size_t lm_target_workspace_bytes(int T, int Dm, int D, int k);
+int launch_lm_target(const void* X, const float* Wc, const void* Wp, void* Vhat, int T, int Dm,
+                     int D, int k, void* ws, size_t ws_bytes, const LaunchCtx& ctx);
 
 // In-Place W_down.
 size_t inplace_workspace_bytes(int T, int Dff, int D, int C);

@@ -2,6 +2,7 @@
 // Declarations and the contract of every entry point live in include/ttt.h.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -403,6 +404,110 @@ int inplace_ttt_chunk_fwd(const void* Z, const void* Vhat, const void* W0, float
   if (!err) return fail(TTT_ERR_CUDA, msg);
   LaunchCtx ctx{stream, err, &msg};
   InplaceArgs a{Z, Vhat, W0, eta, O, W_out, T, Dff, D, C, workspace, workspace_bytes};
+  return finish(launch_inplace(a, ctx), msg);
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static int check_lm_shapes(const std::string& f, int T, int Dm, int D, int k) {
+  if (T <= 0 || Dm <= 0 || D <= 0 || k <= 0)
+    return fail(TTT_ERR_INVALID_ARG, f + ": T, Dm, D and k must be positive");
+  if (T % 128 != 0 || Dm % 128 != 0 || D % 64 != 0 || k > 8)
+    return fail(TTT_ERR_UNSUPPORTED,
+                f + ": supported T % 128 == 0, Dm % 128 == 0, D % 64 == 0, 1 <= k <= 8");
+  if ((long long)T * std::max(Dm, D) >= (1ll << 40))
+    return fail(TTT_ERR_UNSUPPORTED, f + ": too large");
+  return TTT_OK;
+}
+
+size_t ttt_lm_target_workspace_size(int T, int Dm, int D, int k) {
+  if (T <= 0 || Dm <= 0 || D <= 0 || k <= 0) return 0;
+  return lm_target_workspace_bytes(T, Dm, D, k);
+}
+
+int ttt_lm_target_fwd(const void* X, const float* Wc, const void* Wp, void* Vhat, int T, int Dm,
+                      int D, int k, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream) {
+  const std::string f("ttt_lm_target_fwd");
+  if (!X || !Wc || !Wp || !Vhat)
+    return fail(TTT_ERR_INVALID_ARG, f + ": X, Wc, Wp and Vhat must be non-null");
+  int st = check_lm_shapes(f, T, Dm, D, k);
+  if (st != TTT_OK) return st;
+  const void* ptrs[] = {X, Wc, Wp, Vhat, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p))
+      return fail(TTT_ERR_INVALID_ARG, f + ": pointers must be 16-byte aligned");
+  const size_t need = lm_target_workspace_bytes(T, Dm, D, k);
+  if (!workspace || workspace_bytes < need)
+    return fail(TTT_ERR_WORKSPACE, f + ": workspace of at least " + std::to_string(need) +
+                                       " bytes required");
+  const size_t nx = (size_t)T * Dm * 2, nc = (size_t)k * Dm * 4, np = (size_t)Dm * D * 2;
+  const size_t nv = (size_t)T * D * 2;
+  const void* ins[] = {X, Wc, Wp};
+  const size_t nin[] = {nx, nc, np};
+  for (int i = 0; i < 3; ++i)
+    if (overlap(Vhat, nv, ins[i], nin[i]) || overlap(workspace, workspace_bytes, ins[i], nin[i]))
+      return fail(TTT_ERR_INVALID_ARG, f + ": output/workspace overlap an input");
+  if (overlap(Vhat, nv, workspace, workspace_bytes))
+    return fail(TTT_ERR_INVALID_ARG, f + ": output overlaps the workspace");
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  return finish(launch_lm_target(X, Wc, Wp, Vhat, T, Dm, D, k, workspace, workspace_bytes, ctx),
+                msg);
+}
+
+size_t inplace_ttt_lm_workspace_size(int T, int Dff, int D, int Dm, int C, int k) {
+  if (T <= 0 || Dff <= 0 || D <= 0 || Dm <= 0 || C <= 0 || k <= 0 || T % C != 0) return 0;
+  return align256(lm_target_workspace_bytes(T, Dm, D, k)) + align256((size_t)T * D * 2) +
+         inplace_workspace_bytes(T, Dff, D, C);
+}
+
+int inplace_ttt_lm_chunk_fwd(const void* Z, const void* X, const float* Wc, const void* Wp,
+                             const void* W0, float eta, void* O, float* W_out, int T, int Dff,
+                             int D, int Dm, int C, int k, void* workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
+  const std::string f("inplace_ttt_lm_chunk_fwd");
+  if (!Z || !X || !Wc || !Wp || !W0 || !O || !W_out)
+    return fail(TTT_ERR_INVALID_ARG, f + ": every pointer but the workspace must be non-null");
+  int st = check_lm_shapes(f, T, Dm, D, k);
+  if (st != TTT_OK) return st;
+  if (Dff <= 0 || C <= 0 || T % C != 0)
+    return fail(TTT_ERR_INVALID_ARG, f + ": Dff and C must be positive, T a multiple of C");
+  std::string why;
+  if (!inplace_supported(T, Dff, D, C, &why)) return fail(TTT_ERR_UNSUPPORTED, f + ": " + why);
+  const void* ptrs[] = {Z, X, Wc, Wp, W0, O, W_out, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p))
+      return fail(TTT_ERR_INVALID_ARG, f + ": pointers must be 16-byte aligned");
+  const size_t need = inplace_ttt_lm_workspace_size(T, Dff, D, Dm, C, k);
+  if (!workspace || workspace_bytes < need)
+    return fail(TTT_ERR_WORKSPACE, f + ": workspace of at least " + std::to_string(need) +
+                                       " bytes required");
+  const size_t sizes_in[] = {(size_t)T * Dff * 2, (size_t)T * Dm * 2, (size_t)k * Dm * 4,
+                             (size_t)Dm * D * 2, (size_t)Dff * D * 2};
+  const void* ins[] = {Z, X, Wc, Wp, W0};
+  const size_t no = (size_t)T * D * 2, nwo = (size_t)Dff * D * 4;
+  for (int i = 0; i < 5; ++i)
+    if (overlap(O, no, ins[i], sizes_in[i]) || overlap(W_out, nwo, ins[i], sizes_in[i]) ||
+        overlap(workspace, workspace_bytes, ins[i], sizes_in[i]))
+      return fail(TTT_ERR_INVALID_ARG, f + ": outputs/workspace overlap an input");
+  if (overlap(O, no, W_out, nwo) || overlap(workspace, workspace_bytes, O, no) ||
+      overlap(workspace, workspace_bytes, W_out, nwo))
+    return fail(TTT_ERR_INVALID_ARG, f + ": outputs/workspace overlap");
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t lm = align256(lm_target_workspace_bytes(T, Dm, D, k));
+  void* Vhat = ws + lm;
+  const size_t vb = align256((size_t)T * D * 2);
+  int r = launch_lm_target(X, Wc, Wp, Vhat, T, Dm, D, k, ws, lm, ctx);
+  if (r != kOk) return finish(r, msg);
+  InplaceArgs a{Z, Vhat, W0, eta, O, W_out, T, Dff, D, C, ws + lm + vb,
+                workspace_bytes - lm - vb};
   return finish(launch_inplace(a, ctx), msg);
 }
 

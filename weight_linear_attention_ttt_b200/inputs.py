@@ -46,10 +46,13 @@ class Workload:
     # in-place recipe
     Dff: int = 0
     D: int = 0
+    # LM-aligned target (in-place with its target formed from embeddings)
+    Dm: int = 0
+    k: int = 0
 
     @property
     def tokens(self) -> int:
-        return self.B * self.T if self.kind != "inplace" else self.T
+        return self.B * self.T if not self.kind.startswith("inplace") else self.T
 
 
 # The five workloads of the forward path use seeds 1000 + i; the backward of the associative
@@ -74,6 +77,9 @@ WORKLOADS = {
     "assoc_momentum_bf16_B4H16T65536_d128C64": Workload(
         "assoc_momentum_bf16_B4H16T65536_d128C64", "assoc_momentum", 1007, B=4, H=16, T=65536,
         d=128, C=64, normalise=("Q", "K"), eta="sigmoid", w0="zero"),
+    "inplace_lm_bf16_T32768_Dff9728_D2560_Dm2560_C1024": Workload(
+        "inplace_lm_bf16_T32768_Dff9728_D2560_Dm2560_C1024", "inplace_lm", 1008, T=32768,
+        C=1024, Dff=9728, D=2560, Dm=2560, k=4, eta="const", eta_const=1e-3),
     "assoc_bwd_bf16_B4H16T65536_d128C64": Workload(
         "assoc_bwd_bf16_B4H16T65536_d128C64", "assoc_bwd", 1005, B=4, H=16, T=65536, d=128,
         C=64, normalise=("Q", "K"), eta="sigmoid", w0="zero"),
@@ -160,6 +166,25 @@ def assoc_bwd_inputs(B: int, H: int, T: int, d: int, *, seed: int, device="cpu",
     return out
 
 
+def inplace_lm_inputs(T: int, Dff: int, D: int, Dm: int, k: int, *, seed: int, device="cpu",
+                      eta: float = 1e-3) -> dict:
+    """The In-Place inputs of ``inplace_inputs`` (its Vhat is not used) plus the embeddings and
+    target weights: X [T, Dm] bf16 ~ N(0,1); Wc [k, Dm] fp32 ~ N(0, 1/k) (so the convolved
+    embeddings have unit variance); Wp [Dm, D] bf16 ~ N(0, 0.02^2 / Dm) (so Vhat has the
+    N(0, 0.02^2) scale of the plain recipe), drawn in that order from a generator seeded
+    seed + 1."""
+    out = inplace_inputs(T, Dff, D, seed=seed, device=device, eta=eta)
+    del out["Vhat"]
+    g = _gen(seed + 1, device)
+    out["X"] = torch.randn((T, Dm), generator=g, device=device,
+                           dtype=torch.float32).to(torch.bfloat16)
+    out["Wc"] = (torch.randn((k, Dm), generator=g, device=device, dtype=torch.float32)
+                 * (1.0 / k) ** 0.5).contiguous()
+    out["Wp"] = (torch.randn((Dm, D), generator=g, device=device, dtype=torch.float32)
+                 * (0.02 / Dm ** 0.5)).to(torch.bfloat16)
+    return out
+
+
 def make_inputs(w: Workload, device="cpu", *, seed: Optional[int] = None, **overrides) -> dict:
     """Inputs of a named workload (optionally with shape overrides for reduced cases)."""
     if overrides:
@@ -175,4 +200,7 @@ def make_inputs(w: Workload, device="cpu", *, seed: Optional[int] = None, **over
                                 eta_const=w.eta_const, w0=w.w0)
     if w.kind == "inplace":
         return inplace_inputs(w.T, w.Dff, w.D, seed=s, device=device, eta=w.eta_const)
+    if w.kind == "inplace_lm":
+        return inplace_lm_inputs(w.T, w.Dff, w.D, w.Dm, w.k, seed=s, device=device,
+                                 eta=w.eta_const)
     raise ValueError(w.kind)
