@@ -42,7 +42,8 @@ DOMINANT_KERNEL = {"dual": ("dual_mma_kernel", "dual_mma.cu"),
                    "assoc": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu"),
                    "assoc_bwd": ("assoc_chunk_kernel", "assoc_scan.cu"),
-                   "assoc_momentum": ("assoc_chunk_kernel", "assoc_scan.cu")}
+                   "assoc_momentum": ("assoc_chunk_kernel", "assoc_scan.cu"),
+                   "inplace_lm": ("inplace_chunk_kernel", "inplace_ttt.cu")}
 
 
 def peaks():
@@ -183,6 +184,14 @@ def make_call(w, x, stream_outputs=None):
         return lambda: ttt.ttt_assoc_scan_bwd(x["Q"], x["K"], x["V"], x["eta"], None, x["dO"],
                                               x["dS_out"], C=w.C, eta_scalar=x["eta_scalar"],
                                               workspace=ws, **outs)
+    if w.kind == "inplace_lm":
+        O = torch.empty((w.T, w.D), device=x["Z"].device, dtype=torch.bfloat16)
+        Wf = torch.empty((w.Dff, w.D), device=x["Z"].device, dtype=torch.float32)
+        lib = ttt.load_library()
+        nbytes = lib.inplace_ttt_lm_workspace_size(w.T, w.Dff, w.D, w.Dm, w.C, w.k)
+        ws = torch.empty(max(nbytes, 16), device=x["Z"].device, dtype=torch.uint8)
+        return lambda: ttt.inplace_ttt_lm_chunk_fwd(x["Z"], x["X"], x["Wc"], x["Wp"], x["W0"],
+                                                    x["eta"], C=w.C, O=O, W_out=Wf, workspace=ws)
     if w.kind == "inplace":
         O = torch.empty((w.T, w.D), device=x["Z"].device, dtype=torch.bfloat16)
         Wf = torch.empty((w.Dff, w.D), device=x["Z"].device, dtype=torch.float32)
@@ -204,7 +213,7 @@ def e2e_measure(w, x, steps: int, warmup: int):
     host = {k: v.cpu().pin_memory() for k, v in x.items() if torch.is_tensor(v)}
     dev = {k: torch.empty_like(v) for k, v in x.items() if torch.is_tensor(v)}
     scal = {k: v for k, v in x.items() if not torch.is_tensor(v)}
-    if w.kind == "inplace":
+    if w.kind in ("inplace", "inplace_lm"):
         out_shapes = [((w.T, w.D), torch.bfloat16), ((w.Dff, w.D), torch.float32)]
     elif w.kind == "assoc_momentum":
         out_shapes = [((w.B, w.H, w.T, w.d), x["Q"].dtype), ((w.B, w.H, w.d, w.d), torch.float32),
@@ -218,7 +227,7 @@ def e2e_measure(w, x, steps: int, warmup: int):
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in outs_h)
     xd = dict(dev, **scal)
-    if w.kind != "inplace" and x.get("eta") is None:
+    if not w.kind.startswith("inplace") and x.get("eta") is None:
         xd["eta"] = None
     call = make_call(w, xd)
 
@@ -294,9 +303,14 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
     cols = np.arange(cursor[0] % 80, w.D, 80)
     cursor[0] += 1
     Z = x["Z"].float().cpu().numpy()
-    Vh = x["Vhat"].float().cpu().numpy()[:, cols]
     W0 = x["W0"].float().cpu().numpy()[:, cols]
-    t0 = time.perf_counter()
+    if w.kind == "inplace_lm":
+        Xh, Wc, Wp = (x[k].float().cpu().numpy() for k in ("X", "Wc", "Wp"))
+        t0 = time.perf_counter()
+        Vh = orc.lm_target(Xh, Wc, Wp[:, cols])
+    else:
+        Vh = x["Vhat"].float().cpu().numpy()[:, cols]
+        t0 = time.perf_counter()
     orc.inplace_chunks(Z, Vh, W0, x["eta"], w.C)
     dt = time.perf_counter() - t0
     frac = len(cols) / w.D
@@ -388,7 +402,7 @@ def run_ours(args, w, rank, world, local_rank):
     pk, pk_kind = peaks()
     kname, ksrc = DOMINANT_KERNEL[w.kind]
     launches_per_step = launches / args.steps
-    if w.kind == "inplace":
+    if w.kind.startswith("inplace"):
         achieved = algo["flops"] / (ms_per_step / 1e3) / 1e12
         peak = pk["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

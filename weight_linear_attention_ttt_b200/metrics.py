@@ -44,6 +44,14 @@ def algorithmic(w: Workload) -> dict:
         return {"flops": 3 * th * (4 * w.d * w.d + 4 * w.C * w.d),
                 "bytes": th * (7 * w.d * 2 + 8) + w.B * w.H * 2 * w.d * w.d * 4,
                 "tokens": w.B * w.T}
+    if w.kind == "inplace_lm":
+        # the In-Place update plus the target: convolution (2 k Dm flops per token) and
+        # projection (2 Dm D per token); bytes: the update's with Vhat replaced by X, Wc, Wp
+        a = algorithmic(dataclasses.replace(w, kind="inplace"))
+        T, Dm, D = w.T, w.Dm, w.D
+        return {"flops": a["flops"] + T * (2 * w.k * Dm + 2 * Dm * D),
+                "bytes": a["bytes"] - T * D * 2 + T * Dm * 2 + w.k * Dm * 4 + Dm * D * 2,
+                "tokens": T}
     if w.kind == "inplace":
         T, F, D = w.T, w.Dff, w.D
         return {"flops": 4 * F * D * T,
