@@ -7,9 +7,10 @@
 // state) and M_t the momentum itself,
 //     S_t = S0 + (beta M0 + A_t - beta M_t) / (1 - beta),
 // so the layer is one plain associative pass with rates eta / (1 - beta) from
-// S0 + beta M0 / (1 - beta), one decayed pass (the chunk kernel's decay mode) giving q_t M_t and
-// M_T, and an elementwise combination O = O_plain - beta / (1 - beta) O_decay,
-// S_T = S_plain - beta / (1 - beta) M_T.
+// S0 + beta M0 / (1 - beta), then one decayed pass (the chunk kernel's decay mode) that forms
+// q_t M_t and M_T and writes O = O_plain - beta / (1 - beta) q_t M_t in its epilogue (the
+// decayed output is not rounded before the subtraction); S_T = S_plain - beta / (1 - beta) M_T
+// elementwise.
 #include <cuda_bf16.h>
 
 #include <string>
@@ -27,48 +28,25 @@ __global__ void axpy_states_kernel(const float* a, const float* __restrict__ b, 
     out[i] = (a ? a[i] : 0.f) + c * b[i];
 }
 
-// O += c * Od over n bf16 elements, eight at a time (fp32 arithmetic, one rounding)
-__global__ void axpy_bf16_kernel(uint4* O, const uint4* __restrict__ Od, float c, size_t n8) {
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
-       i += (size_t)gridDim.x * blockDim.x) {
-    uint4 x = O[i];
-    const uint4 y = Od[i];
-    uint32_t* xs = reinterpret_cast<uint32_t*>(&x);
-    const uint32_t* ys = reinterpret_cast<const uint32_t*>(&y);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float lo = __uint_as_float(xs[k] << 16) + c * __uint_as_float(ys[k] << 16);
-      const float hi =
-          __uint_as_float(xs[k] & 0xffff0000u) + c * __uint_as_float(ys[k] & 0xffff0000u);
-      const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-      xs[k] = *reinterpret_cast<const uint32_t*>(&v);
-    }
-    O[i] = x;
-  }
-}
-
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
 size_t assoc_momentum_workspace_bytes(int B, int H, int T, int d, int C) {
   const size_t BH = (size_t)B * H;
-  return align256(assoc_workspace_bytes(B, H, T, d, C)) + align256(BH * T * d * 2) +
-         BH * d * d * sizeof(float);
+  return align256(assoc_workspace_bytes(B, H, T, d, C)) + BH * d * d * sizeof(float);
 }
 
 int launch_assoc_momentum(const AssocMomentumArgs& a, const LaunchCtx& ctx) {
   const size_t BH = (size_t)a.B * a.H, d = a.d;
   const size_t fwd = align256(assoc_workspace_bytes(a.B, a.H, a.T, a.d, a.C));
-  const size_t od = align256(BH * a.T * d * 2);
-  if (a.ws_bytes < fwd + od + BH * d * d * sizeof(float)) {
+  if (a.ws_bytes < fwd + BH * d * d * sizeof(float)) {
     *ctx.msg = "ttt_assoc_momentum_fwd: workspace smaller than "
                "ttt_assoc_momentum_workspace_size()";
     return kWorkspace;
   }
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
-  void* Od = ws + fwd;
-  float* S0p = reinterpret_cast<float*>(ws + fwd + od);
+  float* S0p = reinterpret_cast<float*>(ws + fwd);
   const float inv = 1.f / (1.f - a.beta), c = -a.beta * inv;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -85,17 +63,16 @@ int launch_assoc_momentum(const AssocMomentumArgs& a, const LaunchCtx& ctx) {
   plain.eta_mul = inv;
   int r = launch_assoc(plain, ctx);
   if (r != kOk) return r;
-  StateArgs decay{a.Q, a.K, a.V, a.eta, a.eta_scalar, a.M0, Od, a.M_out, a.B, a.H, a.T, a.d,
+  StateArgs decay{a.Q, a.K, a.V, a.eta, a.eta_scalar, a.M0, a.O, a.M_out, a.B, a.H, a.T, a.d,
                   a.C, 1, a.ws, fwd};
   decay.decay = 1;
   decay.beta = a.beta;
+  decay.Oadd = a.O;         // read back, combined and rewritten row by row in the epilogue
+  decay.add_scale = c;
   r = launch_assoc(decay, ctx);
   if (r != kOk) return r;
-  axpy_bf16_kernel<<<sms * 8, 256, 0, ctx.stream>>>(static_cast<uint4*>(a.O),
-                                                    static_cast<const uint4*>(Od), c,
-                                                    BH * a.T * d / 8);
   axpy_states_kernel<<<sms * 4, 256, 0, ctx.stream>>>(a.S_out, a.M_out, c, a.S_out, BH * d * d);
-  count_launch(2);
+  count_launch();
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     *ctx.msg = std::string("assoc momentum launch: ") + cudaGetErrorString(e);

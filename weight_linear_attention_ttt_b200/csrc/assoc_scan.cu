@@ -87,8 +87,13 @@ struct AssocParams {
   // kernel runs the plain chunk step on values scaled by beta^(h - i) from a state holding
   // beta^(h+1) M, multiplies output row i by beta^(i - h) and the state by beta^C after each
   // update; the final state is beta^h times what TMEM holds.
+  // Pass 1 in decay mode sums a superchunk's increment with weights beta^(L - 1 - s) (L the
+  // superchunk length, s the token index in it): per chunk c a factor beta^(L - C - cC) times
+  // beta^(C - 1 - i) by local index i; the prefix over superchunks applies beta^L.
   int decay;
   float beta;
+  const uint16_t* Oadd;     // pass 2, decay mode: O = Oadd + add_scale * (decayed output)
+  float add_scale;
   unsigned* err;
 };
 
@@ -160,7 +165,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (DECAY && threadIdx.x < C) {
     const float x = (float)threadIdx.x - H_MID;
-    reinterpret_cast<float*>(smem + L::BAR_OFF + 256)[threadIdx.x] = powf(p.beta, -x);
+    reinterpret_cast<float*>(smem + L::BAR_OFF + 256)[threadIdx.x] =
+        SO ? powf(p.beta, (float)(C - 1 - (int)threadIdx.x)) : powf(p.beta, -x);
     reinterpret_cast<float*>(smem + L::BAR_OFF + 512)[threadIdx.x] = powf(p.beta, x);
   }
   if (warp == 1) umma::tmem_alloc(tslot, TM_COLS);
@@ -312,6 +318,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // EV = diag(eta) V in place: the V tile is 1024 16-byte pieces (row = token, eight
       // columns each); piece i is row i / 16 of the two sub-tiles' swizzled layout.
       {
+        const float cf = (DECAY && SO) ? powf(p.beta, (float)(p.part_len - C - c * C)) : 1.f;
         const uint32_t vt = stg + L::V_OFF;
         uint4 x[8];
         float e[8];
@@ -328,7 +335,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int i = otid + 128 * it;
           const int sub = i >> 9, w = i & 511;
           const uint32_t a = vt + sub * 8192 + swz<128>((w >> 3) * 128 + (w & 7) * 16);
-          const float f = e[it] * p.eta_mul * (DECAY ? ldsf(evfac + 4 * (w >> 3)) : 1.f);
+          const float f = e[it] * p.eta_mul * (DECAY ? cf * ldsf(evfac + 4 * (w >> 3)) : 1.f);
           sts128(a, make_uint4(pack_bf16(bf16_lo(x[it].x) * f, bf16_hi(x[it].x) * f),
                                pack_bf16(bf16_lo(x[it].y) * f, bf16_hi(x[it].y) * f),
                                pack_bf16(bf16_lo(x[it].z) * f, bf16_hi(x[it].z) * f),
@@ -395,7 +402,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (ok && (SO || part == p.P - 1)) {
       float* dst = SO ? p.S_dst + ((size_t)stream * (p.P - 1) + part) * D * D
                       : p.S_dst + (size_t)stream * D * D;
-      const float sc = DECAY ? powf(p.beta, H_MID) : 1.f;
+      // pass 2 in decay mode holds beta^(h+1) M and ends with beta^h times the state; pass 1
+      // accumulates the weighted increment itself
+      const float sc = (DECAY && !SO) ? powf(p.beta, H_MID) : 1.f;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t v[32];
@@ -424,6 +433,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       refresh(0, 1, tl);
       for (int c = 0; c < nch; ++c) {
         const int b = c & 1;
+        // decay mode: the words this lane rewrites, read back before the waits below (all
+        // loads in flight at once; each word is read once, before this kernel stores that row)
+        uint32_t oadd[DECAY ? 32 : 1];
+        if (DECAY && p.Oadd) {
+          const uint32_t* ob = reinterpret_cast<const uint32_t*>(
+              p.Oadd + ((size_t)stream * p.T + tok(c)) * D + (dout & ~1));
+#pragma unroll
+          for (int t = 0; t < C; ++t) {
+            if (t & 4) continue;
+            oadd[(t >> 3) * 4 + (t & 3)] = ob[(size_t)(odd ? t + 4 : t) * (D / 2)];
+          }
+        }
         // second half of the bf16 state copy for chunk c+1; the go(c+1) arrival also says
         // that O^T(c-1) has been read out
         bool got = mbar_wait(sdone, c & 1, p.err);
@@ -453,8 +474,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             a4 *= ldsf(ocfac + 4 * (t + 4));
           }
           const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
-          const uint32_t w = odd ? pack_bf16(y, a4) : pack_bf16(a, y);
+          float lo = odd ? y : a, hi = odd ? a4 : y;   // columns (dout & ~1) and (dout | 1)
           const int row = odd ? t + 4 : t;
+          if (DECAY && p.Oadd) {
+            const uint32_t base = oadd[(t >> 3) * 4 + (t & 3)];
+            lo = __uint_as_float(base << 16) + p.add_scale * lo;
+            hi = __uint_as_float(base & 0xffff0000u) + p.add_scale * hi;
+          }
+          const uint32_t w = pack_bf16(lo, hi);
           sts32(so + swz<128>(row * 128 + cb), w);
         }
         fence_proxy_async_smem();
@@ -498,14 +525,15 @@ done:
 }
 
 // Exclusive prefix over the parts' increments, in place: slot p-1 becomes the start of part p.
-__global__ void assoc_scan_kernel(const float* __restrict__ S0, float* inc, int P) {
+// (decay mode: each step first multiplies the running state by decay_L = beta^L.)
+__global__ void assoc_scan_kernel(const float* __restrict__ S0, float* inc, int P, float decay_L) {
   const int stream = blockIdx.y;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;   // element of the d x d state
   if (e >= D * D) return;
   float run = S0 ? S0[(size_t)stream * D * D + e] : 0.f;
   float* base = inc + (size_t)stream * (P - 1) * D * D + e;
   for (int pp = 0; pp < P - 1; ++pp) {
-    run += base[(size_t)pp * D * D];
+    run = decay_L * run + base[(size_t)pp * D * D];
     base[(size_t)pp * D * D] = run;
   }
 }
@@ -528,8 +556,7 @@ int choose_parts(int streams, int T) {
 template <bool STATE_ONLY>
 int launch_chunk(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const CUtensorMap& to, const AssocParams& p, int grid, const LaunchCtx& ctx) {
-  auto kern = (!STATE_ONLY && p.decay) ? assoc_chunk_kernel<STATE_ONLY, true>
-                                       : assoc_chunk_kernel<STATE_ONLY, false>;
+  auto kern = p.decay ? assoc_chunk_kernel<STATE_ONLY, true> : assoc_chunk_kernel<STATE_ONLY, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Smem<STATE_ONLY>::BYTES);
   if (e != cudaSuccess) {
@@ -577,6 +604,8 @@ int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
   p.eta_mul = a.eta_mul;
   p.decay = a.decay;
   p.beta = a.beta;
+  p.Oadd = static_cast<const uint16_t*>(a.Oadd);
+  p.add_scale = a.add_scale;
   p.err = ctx.err;
   return launch_chunk<true>(tq, tk, tv, to, p, BH, ctx);
 }
@@ -589,7 +618,7 @@ size_t assoc_workspace_bytes(int B, int H, int T, int d, int C_) {
 
 int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   const int BH = a.B * a.H;
-  const int P = a.decay ? 1 : choose_parts(BH, a.T);   // decay mode: one superchunk
+  const int P = choose_parts(BH, a.T);
   const size_t need = (size_t)BH * (P - 1) * D * D * sizeof(float);
   if (a.ws_bytes < need) {
     *ctx.msg = "ttt_assoc_scan_fwd: workspace smaller than ttt_assoc_scan_workspace_size()";
@@ -618,12 +647,15 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   p.eta_mul = a.eta_mul;
   p.decay = a.decay;
   p.beta = a.beta;
+  p.Oadd = static_cast<const uint16_t*>(a.Oadd);
+  p.add_scale = a.add_scale;
   p.err = ctx.err;
   if (P > 1) {
     p.S_dst = static_cast<float*>(a.ws);
     int st = launch_chunk<true>(tq, tk, tv, to, p, BH * (P - 1), ctx);
     if (st != kOk) return st;
-    assoc_scan_kernel<<<dim3(D * D / 256, BH), 256, 0, ctx.stream>>>(a.S0, p.S_dst, P);
+    const float decay_L = a.decay ? powf(a.beta, (float)p.part_len) : 1.f;
+    assoc_scan_kernel<<<dim3(D * D / 256, BH), 256, 0, ctx.stream>>>(a.S0, p.S_dst, P, decay_L);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
       *ctx.msg = std::string("assoc scan launch: ") + cudaGetErrorString(e);

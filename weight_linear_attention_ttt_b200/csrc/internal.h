@@ -32,6 +32,9 @@ struct StateArgs {
   float eta_mul = 1.f;
   int decay = 0;
   float beta = 0.f;
+  // decay mode: O = Oadd + add_scale * (decayed output), Oadd [B,H,T,d] bf16 (may equal O)
+  const void* Oadd = nullptr;
+  float add_scale = 0.f;
 };
 
 struct InplaceArgs {
