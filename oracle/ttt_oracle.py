@@ -40,9 +40,10 @@ W0 = 0; o = q(S0 + k^T v) for one token; the sequential recurrence vs. the chunk
 forms; eta folded into V; the In-Place block-causal linear-attention form and its one-chunk closed
 form; autograd ascent steps for the associative and In-Place deltas; hand-worked golden examples;
 the associative backward against central finite differences of the forward definition and
-against autograd of an independent torch restatement; the momentum recurrence against the plain
-one at beta = 0, against its closed weighted-sum form and against hand-worked tokens. Every
-function below has at least one pin.
+against autograd of an independent torch restatement; the dual-form backward against central
+finite differences and against autograd through mini-batch gradient steps that autograd itself
+takes; the momentum recurrence against the plain one at beta = 0, against its closed
+weighted-sum form and against hand-worked tokens. Every function below has at least one pin.
 """
 from __future__ import annotations
 
@@ -121,6 +122,89 @@ def dual_form(Q, K, V, eta, W0, C: int, *, threads: int = 1, streams=None):
         O = O.reshape(B, H, T, d)
         W = W.reshape(B, H, d, d)
     return O, W
+
+
+def dual_backward_stream(Q, K, V, eta, W0, dO, dW_out, C: int):
+    """Gradients of  L = sum_t <dO_t, o_t> + <dW_out, W_T>  through the dual form of
+    ``dual_form_stream`` (the backward pass that outer-loop training of the layer needs
+    [TTT-read, "gradient를 효율적인 layer로 만드는 작업"]: the inner updates are differentiated
+    like any other layer).
+
+    A forward sweep recomputes the chunk-start states W_c. A reverse sweep carries X, the
+    gradient of L with respect to the state after the chunk (dW_out after the last one), and
+    differentiates the chunk's three statements in reverse order:
+        W' = W - K^T diag(eta) G :  dW += X,  dG = -diag(eta) K X,
+                                    dk_s = -eta_s g_s X^T,  deta_s = -k_s X g_s^T
+        O  = Q W - A G, A = tril(Q K^T) diag(eta) :
+                                    dW += Q^T dO,  dG += -A^T dO,
+                                    dA = -tril(dO G^T)  (entries s > t of A are zero),
+                                    d(QK^T) = dA diag(eta) -> dQ += d(QK^T) K, dK += d(QK^T)^T Q,
+                                    deta_s += sum_t dA[t, s] (Q K^T)[t, s]
+        G  = K W - V :              dW += K^T dG,  dK += dG W^T,  dV = -dG
+    and the total dW is X for the chunk before. After chunk 0, X is dW0.
+    Returns (dQ, dK, dV [T, d], deta [T] (per token; their sum when eta is a scalar),
+    dW0 [d, d])."""
+    Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    T, d = Q.shape
+    if C <= 0 or T % C:
+        raise ValueError("T must be a positive multiple of C")
+    e_all = _eta_stream(eta, T)
+    W = np.zeros((d, d)) if W0 is None else _f64(W0).copy()
+    starts = []
+    for c0 in range(0, T, C):                             # forward sweep: chunk-start states
+        starts.append(W.copy())
+        k, v, e = K[c0:c0 + C], V[c0:c0 + C], e_all[c0:c0 + C]
+        W = W - k.T @ (e[:, None] * (k @ W - v))
+    X = np.zeros((d, d)) if dW_out is None else _f64(dW_out).copy()
+    dQ, dK, dV, deta = np.empty((T, d)), np.empty((T, d)), np.empty((T, d)), np.empty(T)
+    mask = np.tril(np.ones((C, C)))
+    for ci in range(T // C - 1, -1, -1):                  # reverse sweep
+        c0 = ci * C
+        sl = slice(c0, c0 + C)
+        q, k, v, e, do = Q[sl], K[sl], V[sl], e_all[sl], dO[sl]
+        W = starts[ci]
+        G = k @ W - v
+        QK = q @ k.T
+        A = QK * mask * e[None, :]
+        # W' = W - K^T diag(eta) G
+        kX = k @ X
+        dG = -e[:, None] * kX
+        dk = -e[:, None] * (G @ X.T)
+        de = -np.sum(kX * G, axis=1)
+        # O = Q W - A G
+        dW = X + q.T @ do
+        dG = dG - A.T @ do
+        dA = -(do @ G.T) * mask
+        dQK = dA * e[None, :]
+        dq = do @ W.T + dQK @ k
+        dk = dk + dQK.T @ q
+        de = de + np.sum(dA * QK, axis=0)
+        # G = K W - V
+        dW = dW + k.T @ dG
+        dk = dk + dG @ W.T
+        dQ[sl], dK[sl], dV[sl], deta[sl] = dq, dk, -dG, de
+        X = dW
+    return dQ, dK, dV, deta, X
+
+
+def dual_form_bwd(Q, K, V, eta, W0, dO, dW_out, C: int, *, threads: int = 1, streams=None):
+    """All streams of [B, H, T, d] inputs (eta [B, H, T] or scalar; W0 / dW_out [B, H, d, d] or
+    None). Returns (dQ, dK, dV, deta, dW0); deta is per token even for a scalar eta."""
+    B, H, T, d = np.shape(Q)
+
+    def one(b, h):
+        e = eta if np.ndim(eta) == 0 else np.asarray(eta)[b, h]
+        w0 = None if W0 is None else np.asarray(W0)[b, h]
+        g = None if dW_out is None else np.asarray(dW_out)[b, h]
+        return dual_backward_stream(np.asarray(Q)[b, h], np.asarray(K)[b, h],
+                                    np.asarray(V)[b, h], e, w0, np.asarray(dO)[b, h], g, C)
+
+    idx, res = _streams(one, None, B, H, threads, streams)
+    out = [np.stack([r[i] for r in res]) for i in range(5)]
+    if streams is None:
+        shapes = [(B, H, T, d)] * 3 + [(B, H, T), (B, H, d, d)]
+        out = [o.reshape(sh) for o, sh in zip(out, shapes)]
+    return tuple(out)
 
 
 # --------------------------------------------------------------------------------------------

@@ -424,6 +424,142 @@ def test_assoc_backward_pins_catch_planted_mistakes():
         assert not (np.allclose(dK, ref[1], rtol=1e-6) and np.allclose(dV, ref[2], rtol=1e-6))
 
 
+# ----------------------------------------------------------------------------- dual-form backward
+def _dual_loss(Q, K, V, eta, W0, dO, G, C):
+    """The scalar whose gradients the dual-form backward returns, from the forward only."""
+    O, W = orc.dual_form_stream(Q, K, V, eta, W0, C)
+    return float(np.sum(dO * O) + np.sum(G * W))
+
+
+def _dual_bwd_case(T, d, scalar_eta=False, scale=0.6):
+    Q, K, V, dO = (_rand(T, d, scale=scale) for _ in range(4))
+    eta = 0.2 if scalar_eta else rng.uniform(0.05, 0.5, T)
+    W0, G = _rand(d, d, scale=0.4), _rand(d, d, scale=0.5)
+    return Q, K, V, eta, W0, dO, G
+
+
+@pytest.mark.parametrize("T,d,C", [(6, 3, 3), (6, 2, 2), (4, 3, 4)])
+def test_dual_backward_matches_central_finite_differences(T, d, C):
+    """Every gradient of the chunk-wise adjoint against central differences of the forward
+    (the loss is a polynomial in each input; h = 1e-5 leaves an O(h^2) truncation error)."""
+    Q, K, V, eta, W0, dO, G = _dual_bwd_case(T, d)
+    grads = orc.dual_backward_stream(Q, K, V, eta, W0, dO, G, C)
+    h = 1e-5
+    args = [Q, K, V, eta, W0]
+    for i, grad in enumerate(grads):
+        fd = np.empty_like(grad)
+        for idx in np.ndindex(grad.shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[i][idx] += h
+            minus[i][idx] -= h
+            fd[idx] = (_dual_loss(*plus, dO, G, C) - _dual_loss(*minus, dO, G, C)) / (2 * h)
+        assert np.allclose(grad, fd, rtol=1e-6, atol=1e-8), i
+
+
+def _inner_grad_graph(W, k, v):
+    """Gradient of 1/2 ||k W - v||^2 at W by autograd, kept in the graph so that the outer
+    loss can be differentiated through it."""
+    loss = 0.5 * ((k @ W - v) ** 2).sum()
+    (g,) = torch.autograd.grad(loss, W, create_graph=True)
+    return g
+
+
+@pytest.mark.parametrize("scalar_eta", [False, True])
+@pytest.mark.parametrize("T,d,C", [(16, 4, 4), (12, 5, 3), (8, 3, 8)])
+def test_dual_backward_matches_autograd_through_minibatch_steps(T, d, C, scalar_eta):
+    """Against torch autograd of mini-batch TTT written by definition (every inner gradient
+    taken by autograd at the chunk-start weight, every W_t formed explicitly), float64."""
+    Q, K, V, eta, W0, dO, G = _dual_bwd_case(T, d, scalar_eta)
+    grads = orc.dual_backward_stream(Q, K, V, eta, W0, dO, G, C)
+    tq, tk, tv, tw = (torch.tensor(a, requires_grad=True) for a in (Q, K, V, W0))
+    te = torch.tensor(np.full(T, eta) if scalar_eta else eta, requires_grad=True)
+    W = tw
+    outs = []
+    for c0 in range(0, T, C):
+        steps = [te[s] * _inner_grad_graph(W, tk[s], tv[s]) for s in range(c0, c0 + C)]
+        for t in range(c0, c0 + C):
+            outs.append(tq[t] @ (W - sum(steps[: t - c0 + 1])))
+        W = W - sum(steps)
+    L = (torch.stack(outs) * torch.tensor(dO)).sum() + (W * torch.tensor(G)).sum()
+    L.backward()
+    for ours, ref in zip(grads, (tq.grad, tk.grad, tv.grad, te.grad, tw.grad)):
+        assert np.allclose(ours, ref.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_dual_backward_zero_keys_closed_form_and_helper():
+    """With K = 0 the state never moves: dQ = dO W0^T, dV = 0, deta = 0 and
+    dW0 = dW_out + Q^T dO. The batched helper equals the per-stream sweep, and zero output
+    gradients give zero everywhere."""
+    T, d, C = 12, 4, 4
+    Q, _, V, eta, W0, dO, G = _dual_bwd_case(T, d)
+    dQ, dK, dV, deta, dW0 = orc.dual_backward_stream(Q, np.zeros((T, d)), V, eta, W0, dO, G, C)
+    assert np.allclose(dQ, dO @ W0.T, rtol=1e-13, atol=1e-13)
+    assert np.all(dV == 0) and np.allclose(deta, 0, atol=1e-15)
+    assert np.allclose(dW0, G + Q.T @ dO, rtol=1e-13, atol=1e-13)
+    B, H = 2, 2
+    Qb, Kb, Vb, dOb = (_rand(B, H, T, d, scale=0.5) for _ in range(4))
+    eb = rng.uniform(0.1, 0.5, (B, H, T))
+    Gb = _rand(B, H, d, d)
+    out = orc.dual_form_bwd(Qb, Kb, Vb, eb, None, dOb, Gb, C)
+    one = orc.dual_backward_stream(Qb[1, 0], Kb[1, 0], Vb[1, 0], eb[1, 0], None, dOb[1, 0],
+                                   Gb[1, 0], C)
+    for a, b in zip(out, one):
+        assert np.array_equal(a[1, 0], b)
+    zero = orc.dual_form_bwd(Qb, Kb, Vb, eb, None, np.zeros_like(dOb), None, C)
+    assert all(np.all(z == 0) for z in zero)
+
+
+def test_dual_backward_pins_catch_planted_mistakes():
+    """Plausible slips in the chunk adjoint (the causal mask without its diagonal, the -A^T dO
+    term left out of dG, the state after the chunk used in place of the chunk-start state) must
+    fail the finite-difference pin. Planted in a copy of the reverse sweep, on the CPU."""
+    T, d, C = 6, 3, 3
+    Q, K, V, eta, W0, dO, G = _dual_bwd_case(T, d)
+    fd_dq = np.empty((T, d))
+    for idx in np.ndindex(T, d):
+        plus, minus = Q.copy(), Q.copy()
+        plus[idx] += 1e-5
+        minus[idx] -= 1e-5
+        fd_dq[idx] = (_dual_loss(plus, K, V, eta, W0, dO, G, C)
+                      - _dual_loss(minus, K, V, eta, W0, dO, G, C)) / 2e-5
+    fd_w0 = np.empty((d, d))
+    for idx in np.ndindex(d, d):
+        plus, minus = W0.copy(), W0.copy()
+        plus[idx] += 1e-5
+        minus[idx] -= 1e-5
+        fd_w0[idx] = (_dual_loss(Q, K, V, eta, plus, dO, G, C)
+                      - _dual_loss(Q, K, V, eta, minus, dO, G, C)) / 2e-5
+
+    def sweep(strict_mask, drop_at_do, end_state):
+        W, starts = W0.copy(), []
+        for c0 in range(0, T, C):
+            starts.append(W.copy())
+            k, v, e = K[c0:c0 + C], V[c0:c0 + C], eta[c0:c0 + C]
+            W = W - k.T @ (e[:, None] * (k @ W - v))
+        starts.append(W)
+        mask = np.tril(np.ones((C, C)), -1 if strict_mask else 0)
+        X, dq_all = G.copy(), np.empty((T, d))
+        for ci in range(T // C - 1, -1, -1):
+            sl = slice(ci * C, ci * C + C)
+            q, k, v, e, do = Q[sl], K[sl], V[sl], eta[sl], dO[sl]
+            W = starts[ci + 1] if end_state else starts[ci]
+            Gc = k @ W - v
+            A = (q @ k.T) * mask * e[None, :]
+            dG = -e[:, None] * (k @ X) - (0 if drop_at_do else A.T @ do)
+            dQK = -(do @ Gc.T) * mask * e[None, :]
+            dq_all[sl] = do @ W.T + dQK @ k
+            X = X + q.T @ do + k.T @ dG
+        return dq_all, X
+
+    good = sweep(False, False, False)
+    assert np.allclose(good[0], fd_dq, rtol=1e-6, atol=1e-8)
+    assert np.allclose(good[1], fd_w0, rtol=1e-6, atol=1e-8)
+    for bad in ((True, False, False), (False, True, False), (False, False, True)):
+        dq, dw0 = sweep(*bad)
+        assert not (np.allclose(dq, fd_dq, rtol=1e-4) and np.allclose(dw0, fd_w0, rtol=1e-4))
+
+
 # ----------------------------------------------------------------------------- momentum
 def test_momentum_beta_zero_is_the_plain_recurrence():
     T, d = 20, 5
