@@ -42,6 +42,7 @@ DOMINANT_KERNEL = {"dual": ("dual_mma_kernel", "dual_mma.cu"),
                    "assoc": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu"),
                    "assoc_bwd": ("assoc_chunk_kernel", "assoc_scan.cu"),
+                   "dual_bwd": ("dual_bwd_kernel", "dual_bwd.cu"),
                    "assoc_momentum": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "inplace_lm": ("inplace_chunk_kernel", "inplace_ttt.cu")}
 
@@ -184,6 +185,18 @@ def make_call(w, x, stream_outputs=None):
         return lambda: ttt.ttt_assoc_scan_bwd(x["Q"], x["K"], x["V"], x["eta"], None, x["dO"],
                                               x["dS_out"], C=w.C, eta_scalar=x["eta_scalar"],
                                               workspace=ws, **outs)
+    if w.kind == "dual_bwd":
+        dev = x["Q"].device
+        outs = dict(dQ=torch.empty_like(x["Q"]), dK=torch.empty_like(x["Q"]),
+                    dV=torch.empty_like(x["Q"]),
+                    deta=torch.empty((w.B, w.H, w.T), device=dev, dtype=torch.float32),
+                    dW0=torch.empty((w.B, w.H, w.d, w.d), device=dev, dtype=torch.float32))
+        lib = ttt.load_library()
+        nbytes = lib.ttt_linear_dual_bwd_workspace_size(w.B, w.H, w.T, w.d, w.C, 1)
+        ws = torch.empty(max(nbytes, 16), device=dev, dtype=torch.uint8)
+        return lambda: ttt.ttt_linear_dual_bwd(x["Q"], x["K"], x["V"], x["eta"], x["W0"],
+                                               x["dO"], x["dW_out"], C=w.C,
+                                               eta_scalar=x["eta_scalar"], workspace=ws, **outs)
     if w.kind == "inplace_lm":
         O = torch.empty((w.T, w.D), device=x["Z"].device, dtype=torch.bfloat16)
         Wf = torch.empty((w.Dff, w.D), device=x["Z"].device, dtype=torch.float32)
@@ -218,7 +231,7 @@ def e2e_measure(w, x, steps: int, warmup: int):
     elif w.kind == "assoc_momentum":
         out_shapes = [((w.B, w.H, w.T, w.d), x["Q"].dtype), ((w.B, w.H, w.d, w.d), torch.float32),
                       ((w.B, w.H, w.d, w.d), torch.float32)]
-    elif w.kind == "assoc_bwd":
+    elif w.kind in ("assoc_bwd", "dual_bwd"):
         out_shapes = [((w.B, w.H, w.T, w.d), x["Q"].dtype)] * 3 + [
             ((w.B, w.H, w.T), torch.float32), ((w.B, w.H, w.d, w.d), torch.float32)]
     else:
@@ -263,18 +276,18 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
 
     threads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    if w.kind in ("dual", "assoc", "assoc_bwd", "assoc_momentum"):
+    if w.kind in ("dual", "assoc", "assoc_bwd", "assoc_momentum", "dual_bwd"):
         streams = [(b, h) for b in range(w.B) for h in range(w.H)]
         Q, K, V = (x[k].float().cpu().numpy() for k in ("Q", "K", "V"))
         eta = None if x["eta"] is None else x["eta"].cpu().numpy()
         W0 = x["W0"].cpu().numpy()
-        if w.kind == "assoc_bwd":
+        if w.kind in ("assoc_bwd", "dual_bwd"):
             dO = x["dO"].float().cpu().numpy()
-            G = x["dS_out"].cpu().numpy()
+            G = x["dS_out" if w.kind == "assoc_bwd" else "dW_out"].cpu().numpy()
         # probe the cost of one chunk-run of one stream to size the sample
         tok = 0
         n_streams = 0
-        ncol = w.T if w.kind == "dual" else min(w.T, 4096)
+        ncol = w.T if w.kind in ("dual", "dual_bwd") else min(w.T, 4096)
         while True:
             b, h = streams[cursor[0] % len(streams)]
             cursor[0] += 1
@@ -285,6 +298,9 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
             elif w.kind == "assoc_momentum":
                 orc.assoc_momentum_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
                                           inp.MOMENTUM_BETA, None, None)
+            elif w.kind == "dual_bwd":
+                orc.dual_backward_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
+                                         W0[b, h], dO[b, h, :ncol], G[b, h], w.C)
             elif w.kind == "assoc_bwd":
                 orc.assoc_backward_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
                                           None, dO[b, h, :ncol], G[b, h])
@@ -296,7 +312,7 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
             if time.perf_counter() - t0 >= budget_s or n_streams >= len(streams):
                 break
         desc = (f"{n_streams} (b,h) stream(s) x {ncol} tokens of the workload, "
-                f"{ {'dual': 'dual-form per-chunk loop', 'assoc': 'sequential recurrence', 'assoc_momentum': 'momentum recurrence'}.get(w.kind, 'adjoint sweeps of the recurrence')}"
+                f"{ {'dual': 'dual-form per-chunk loop', 'assoc': 'sequential recurrence', 'assoc_momentum': 'momentum recurrence', 'dual_bwd': 'dual-form chunk adjoint sweeps'}.get(w.kind, 'adjoint sweeps of the recurrence')}"
                 f", numpy fp64, 1 thread")
         return tok / w.H, time.perf_counter() - t0, 1, desc
     # In-Place: every 80th output column over all chunks (columns are independent)
@@ -418,7 +434,7 @@ def run_ours(args, w, rank, world, local_rank):
                  else "fallback", "launches_per_step": launches_per_step,
                  "kernel_source_sha": sha,
                  "duration_us": 1e3 * ms_per_step / max(1.0, launches_per_step)
-                 if w.kind == "dual" else None})
+                 if w.kind in ("dual", "dual_bwd") else None})
 
     line = {"metric": metric_of(w), "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,

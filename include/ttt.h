@@ -130,8 +130,9 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
  *  beta in [0.25, 0.9] (beta = 0 is ttt_assoc_scan_fwd; the two-pass evaluation subtracts
  *  outputs of size ~1/(1 - beta), which bounds beta for bf16 outputs). Supported: bf16,
  *  d == 128, C == 64.
- *  Workspace: ttt_assoc_momentum_workspace_size() bytes. Runs as one plain associative pass, one
- *  decayed pass and an elementwise combination (see assoc_momentum.cu).
+ *  Workspace: ttt_assoc_momentum_workspace_size() bytes. Runs as one plain associative pass and
+ *  one decayed pass whose output stage combines the two outputs, then an elementwise
+ *  combination of the states (see assoc_momentum.cu).
  * ------------------------------------------------------------------------------------------ */
 size_t ttt_assoc_momentum_workspace_size(int B, int H, int T, int d, int C, int dt);
 int ttt_assoc_momentum_fwd(const void* Q, const void* K, const void* V, const float* eta,
@@ -164,6 +165,34 @@ int ttt_assoc_scan_bwd(const void* Q, const void* K, const void* V, const float*
                        void* dQ, void* dK, void* dV, float* deta, float* dS0, int B, int H,
                        int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
                        cudaStream_t stream);
+
+/* --------------------------------------------------------------------------------------------
+ * Backward of the TTT-Linear dual form ("RNN의 기억을 작은 모델로 바꾼다면: Test-Time Training
+ * 읽기", section "gradient를 효율적인 layer로 만드는 작업": the mini-batch inner updates are part
+ * of the layer and are differentiated with it in outer-loop training). For ttt_linear_dual_fwd
+ * and a scalar loss L with dL/dO = dO and dL/dW_out = dW_out, returns dQ, dK, dV, deta (per
+ * token) and dW0. Per chunk, with X the gradient of the state after the chunk (dW_out after the
+ * last), W the chunk-start state, G = K W - V and A = tril(Q K^T) diag(eta):
+ *     dG = -A^T dO - diag(eta) K X,   dV = -dG,   dA = -tril(dO G^T),   dS = dA diag(eta),
+ *     dQ = dO W^T + dS K,   dK = dS^T Q - diag(eta) G X^T + dG W^T,
+ *     deta_s = sum_t dA[t,s] (Q K^T)[t,s] - (K X)_s . G_s,   X <- X + Q^T dO + K^T dG;
+ *  dW0 is X after the first chunk.
+ *  Q, K, V, dO [B,H,T,d] bf16; eta [B,H,T] fp32 or NULL (eta_scalar for every token); W0 and
+ *  dW_out [B,H,d,d] fp32 or NULL (zeros). Outputs: dQ, dK, dV [B,H,T,d] bf16; deta [B,H,T]
+ *  fp32 (per token also when eta is NULL); dW0 [B,H,d,d] fp32. Outputs and workspace must not
+ *  overlap the inputs or each other.
+ *  Supported: bf16, C == 16, d in {32, 64, 128}, T % C == 0 (C changes the result: it is the
+ *  mini-batch size of the forward).
+ *  Workspace: ttt_linear_dual_bwd_workspace_size() bytes (one bf16 d x d state per chunk:
+ *  B*H*(T/16)*d*d*2). One kernel launch: a forward sweep recomputes the chunk-start states,
+ *  a reverse sweep forms the gradients (see dual_bwd.cu).
+ * ------------------------------------------------------------------------------------------ */
+size_t ttt_linear_dual_bwd_workspace_size(int B, int H, int T, int d, int C, int dt);
+int ttt_linear_dual_bwd(const void* Q, const void* K, const void* V, const float* eta,
+                        float eta_scalar, const float* W0, const void* dO, const float* dW_out,
+                        void* dQ, void* dK, void* dV, float* deta, float* dW0, int B, int H,
+                        int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
 
 /* --------------------------------------------------------------------------------------------
  * State increment of a sequence slice in the associative mode (the first pass of the prefix

@@ -53,6 +53,16 @@ def test_momentum_matches_oracle(cuda_lib, B, H, T, beta):
     assert ttt.read_device_error() == 0
 
 
+@pytest.mark.parametrize("parts", ["1", "2", "4", "16"])
+def test_forced_superchunk_counts(cuda_lib, monkeypatch, parts):
+    """Both passes split into superchunks (the decayed one carrying its state across them with
+    the superchunk decay) give the oracle's results for every split."""
+    monkeypatch.setenv("TTT_ASSOC_PARTS", parts)
+    x = make(1, 2, 1024, seed=31)
+    check(x, 0.9, run(x, 0.9))
+    assert ttt.read_device_error() == 0
+
+
 def test_scalar_eta_zero_states_and_state_aliasing(cuda_lib):
     x = make(1, 2, 256, seed=4, eta="const", states=False)
     check(x, 0.8, run(x, 0.8))

@@ -100,6 +100,11 @@ struct AssocBwdArgs {
   size_t ws_bytes;
 };
 int launch_assoc_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx);
+// Dual-form backward (one kernel; S0 / dS_out / dS0 of the arguments are W0 / dW_out / dW0; the
+// workspace holds one bf16 d x d checkpoint per chunk).
+bool dual_bwd_supported(int d, int C, int dt);
+size_t dual_bwd_workspace_bytes(int B, int H, int T, int d);
+int launch_dual_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx);
 size_t assoc_momentum_workspace_bytes(int B, int H, int T, int d, int C);
 struct AssocMomentumArgs {
   const void* Q;

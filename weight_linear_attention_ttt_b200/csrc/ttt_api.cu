@@ -334,6 +334,58 @@ int ttt_assoc_scan_bwd(const void* Q, const void* K, const void* V, const float*
   return finish(launch_assoc_bwd(a, ctx), msg);
 }
 
+size_t ttt_linear_dual_bwd_workspace_size(int B, int H, int T, int d, int C, int dt) {
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0 ||
+      !dual_bwd_supported(d, C, dt))
+    return 0;
+  return dual_bwd_workspace_bytes(B, H, T, d);
+}
+
+int ttt_linear_dual_bwd(const void* Q, const void* K, const void* V, const float* eta,
+                        float eta_scalar, const float* W0, const void* dO, const float* dW_out,
+                        void* dQ, void* dK, void* dV, float* deta, float* dW0, int B, int H,
+                        int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+  const std::string f("ttt_linear_dual_bwd");
+  if (!Q || !K || !V || !dO || !dQ || !dK || !dV || !deta || !dW0)
+    return fail(TTT_ERR_INVALID_ARG, f + ": Q, K, V, dO and every output must be non-null");
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0)
+    return fail(TTT_ERR_INVALID_ARG, f + ": B, H, T, d and C must be positive");
+  if (T % C != 0) return fail(TTT_ERR_INVALID_ARG, f + ": T must be a multiple of C");
+  if (dt != TTT_DTYPE_F32 && dt != TTT_DTYPE_BF16)
+    return fail(TTT_ERR_INVALID_ARG, f + ": dtype must be TTT_DTYPE_F32 or TTT_DTYPE_BF16");
+  const void* ptrs[] = {Q, K, V, eta, W0, dO, dW_out, dQ, dK, dV, deta, dW0, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p))
+      return fail(TTT_ERR_INVALID_ARG, f + ": every device pointer must be 16-byte aligned");
+  if (!dual_bwd_supported(d, C, dt))
+    return fail(TTT_ERR_UNSUPPORTED, f + ": supported bf16, C == 16, d in {32, 64, 128}");
+  const size_t need = dual_bwd_workspace_bytes(B, H, T, d);
+  if (!workspace || workspace_bytes < need)
+    return fail(TTT_ERR_WORKSPACE, f + ": workspace smaller than ttt_linear_dual_bwd_workspace_size()");
+  const size_t nx = (size_t)B * H * T * d * 2, ns = (size_t)B * H * d * d * 4;
+  const size_t ne = (size_t)B * H * T * 4;
+  struct R { const void* p; size_t n; };
+  const R ins[] = {{Q, nx}, {K, nx}, {V, nx}, {dO, nx}, {eta, ne}, {W0, ns}, {dW_out, ns}};
+  const R outs[] = {{dQ, nx}, {dK, nx}, {dV, nx}, {deta, ne}, {dW0, ns},
+                    {workspace, workspace_bytes}};
+  for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+    for (const R& in : ins)
+      if (in.p && overlap(outs[i].p, outs[i].n, in.p, in.n))
+        return fail(TTT_ERR_INVALID_ARG, f + ": outputs and workspace must not overlap inputs");
+    for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+      if (overlap(outs[i].p, outs[i].n, outs[j].p, outs[j].n))
+        return fail(TTT_ERR_INVALID_ARG, f + ": outputs and workspace must not overlap");
+  }
+  AssocBwdArgs a{Q, K, V, eta, eta_scalar, W0, dO, dW_out, dQ, dK, dV, deta, dW0, B, H, T, d, C,
+                 workspace, workspace_bytes};
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  return finish(launch_dual_bwd(a, ctx), msg);
+}
+
 int ttt_assoc_state_fwd(const void* K, const void* V, const float* eta, float eta_scalar,
                         float* dS, int B, int H, int T, int d, int C, int dt,
                         cudaStream_t stream) {

@@ -80,6 +80,9 @@ WORKLOADS = {
     "inplace_lm_bf16_T32768_Dff9728_D2560_Dm2560_C1024": Workload(
         "inplace_lm_bf16_T32768_Dff9728_D2560_Dm2560_C1024", "inplace_lm", 1008, T=32768,
         C=1024, Dff=9728, D=2560, Dm=2560, k=4, eta="const", eta_const=1e-3),
+    "dual_bwd_bf16_B8H12T2048_d64C16": Workload(
+        "dual_bwd_bf16_B8H12T2048_d64C16", "dual_bwd", 1006, B=8, H=12, T=2048, d=64, C=16,
+        normalise=("K", "V")),
     "assoc_bwd_bf16_B4H16T65536_d128C64": Workload(
         "assoc_bwd_bf16_B4H16T65536_d128C64", "assoc_bwd", 1005, B=4, H=16, T=65536, d=128,
         C=64, normalise=("Q", "K"), eta="sigmoid", w0="zero"),
@@ -166,6 +169,20 @@ def assoc_bwd_inputs(B: int, H: int, T: int, d: int, *, seed: int, device="cpu",
     return out
 
 
+def dual_bwd_inputs(B: int, H: int, T: int, d: int, *, seed: int, device="cpu",
+                    **recipe) -> dict:
+    """The dual-form inputs of ``dual_or_assoc_inputs`` plus the incoming gradients:
+    dO [B,H,T,d] bf16 ~ N(0,1) and dW_out [B,H,d,d] fp32 ~ N(0, 0.05^2), drawn in that order
+    from a generator seeded with seed + 1."""
+    out = dual_or_assoc_inputs(B, H, T, d, seed=seed, device=device, **recipe)
+    g = _gen(seed + 1, device)
+    out["dO"] = torch.randn((B, H, T, d), generator=g, device=device,
+                            dtype=torch.float32).to(torch.bfloat16).contiguous()
+    out["dW_out"] = (torch.randn((B, H, d, d), generator=g, device=device,
+                                 dtype=torch.float32) * 0.05).contiguous()
+    return out
+
+
 def inplace_lm_inputs(T: int, Dff: int, D: int, Dm: int, k: int, *, seed: int, device="cpu",
                       eta: float = 1e-3) -> dict:
     """The In-Place inputs of ``inplace_inputs`` (its Vhat is not used) plus the embeddings and
@@ -198,6 +215,10 @@ def make_inputs(w: Workload, device="cpu", *, seed: Optional[int] = None, **over
         return assoc_bwd_inputs(w.B, w.H, w.T, w.d, seed=s, device=device, dtype=w.dtype,
                                 qkv=w.qkv, normalise=w.normalise, eta=w.eta,
                                 eta_const=w.eta_const, w0=w.w0)
+    if w.kind == "dual_bwd":
+        return dual_bwd_inputs(w.B, w.H, w.T, w.d, seed=s, device=device, dtype=w.dtype,
+                               qkv=w.qkv, normalise=w.normalise, eta=w.eta,
+                               eta_const=w.eta_const, w0=w.w0)
     if w.kind == "inplace":
         return inplace_inputs(w.T, w.Dff, w.D, seed=s, device=device, eta=w.eta_const)
     if w.kind == "inplace_lm":

@@ -9,6 +9,9 @@ and O out (d elements each) plus one fp32 learning rate, and per stream the fp32
 Associative mode, per token and head: Q S and K^T V (2 d^2 each) plus the causal C x C terms
 (4 C d, counted dense): 4 d^2 + 4 C d flops; bytes as the dual form.
 
+Dual-form backward, per token and head: 14 d^2 + 10 C d flops (see ``algorithmic``); bytes: Q, K,
+V, dO in, dQ, dK, dV out, eta in, deta out, and per stream three fp32 d x d states.
+
 In-Place, per token: the read Z_i W and the update Z_i^T Vhat_i, 2 Dff D flops each; bytes: Z,
 Vhat, W0 (bf16), O (bf16) and the final fp32 W once each.
 """
@@ -43,6 +46,16 @@ def algorithmic(w: Workload) -> dict:
         th = w.B * w.H * w.T
         return {"flops": 3 * th * (4 * w.d * w.d + 4 * w.C * w.d),
                 "bytes": th * (7 * w.d * 2 + 8) + w.B * w.H * 2 * w.d * w.d * 4,
+                "tokens": w.B * w.T}
+    if w.kind == "dual_bwd":
+        # the chunk adjoint's products: K W, K X, dO W^T, dG W^T, diag(eta) G X^T, Q^T dO and
+        # K^T dG (2 d^2 each) plus the C x C terms Q K^T, dO G^T, A^T dO, dS K, dS^T Q (2 C d
+        # each); recomputing the chunk-start states is overhead and not counted. Bytes: Q, K,
+        # V, dO in and dQ, dK, dV out (bf16), eta in and deta out (fp32), per stream W0 and
+        # dW_out in and dW0 out (fp32)
+        th = w.B * w.H * w.T
+        return {"flops": th * (14 * w.d * w.d + 10 * w.C * w.d),
+                "bytes": th * (7 * w.d * 2 + 8) + w.B * w.H * 3 * w.d * w.d * 4,
                 "tokens": w.B * w.T}
     if w.kind == "inplace_lm":
         # the In-Place update plus the target: convolution (2 k Dm flops per token) and
