@@ -14,12 +14,14 @@
 //   1. forward: the chunk-start states W_c are recomputed (fp32 in registers, bf16 operand copy
 //      in shared memory, exactly the products of the forward kernel) and written to the
 //      workspace as bf16, one d x d checkpoint per chunk;
-//   2. reverse: chunks from last to first; the checkpoint and the chunk's Q/K/V/dO/eta tiles
-//      are prefetched with cp.async one chunk ahead; X stays in fp32 registers (its bf16 copy
+//   2. reverse: chunks from last to first; X stays in fp32 registers (its bf16 copy
 //      double-buffered in shared memory), and the chunk's twelve products run on mma.sync
 //      m16n8k16 (bf16 operands, fp32 accumulation) in four phases separated by block barriers.
-// Work split over 8 warps: a 16 x d result is cut into d/8 column tiles (n8), a d x d state into
-// (d/16) x (d/8) m16n8 tiles, both dealt round-robin to the warps.
+// Inputs (and in sweep 2 the checkpoints) stream through a ring of shared-memory slots filled by
+// cp.async up to three chunks ahead, so that the serial chunk loop does not wait on HBM latency.
+// Work split over 8 warps: a 16 x d result is cut into d/8 column tiles (n8) dealt round-robin
+// to the warps; a warp owns the same columns of the state (all d/16 row tiles), so the state
+// recurrences (column-independent) need no barrier of their own.
 // Precision: W, X and all accumulations are fp32; operands (W_c, X, G, dG, A, dS) are rounded to
 // bf16 once per chunk for the tensor cores.
 #include <cuda_bf16.h>
@@ -43,8 +45,9 @@ struct BwdCfg {
   static constexpr int IN_Q = 0, IN_K = TILE, IN_V = 2 * TILE, IN_DO = 3 * TILE;
   static constexpr int IN_W = 4 * TILE;
   static constexpr int IN_ETA = IN_W + WBYTES;
-  static constexpr int IN_BYTES = IN_ETA + 64;     // one chunk's inputs (double-buffered)
-  static constexpr int XB = 2 * IN_BYTES;          // two bf16 state copies
+  static constexpr int IN_BYTES = IN_ETA + 64;     // one chunk's inputs
+  static constexpr int NBUF = D <= 64 ? 4 : 2;     // input ring: NBUF - 1 chunks in flight
+  static constexpr int XB = NBUF * IN_BYTES;       // two bf16 state copies
   static constexpr int SG = XB + 2 * WBYTES;       // G (bf16)
   static constexpr int SEG = SG + TILE;            // diag(eta) G (bf16; negated in sweep 1)
   static constexpr int SDG = SEG + TILE;           // dG (bf16)
@@ -57,8 +60,6 @@ struct BwdCfg {
   static constexpr int SMEM = SDE1 + 64;
   static constexpr int NT = D / 8, MT = D / 16, KS = D / 16;
   static constexpr int CT = (NT + NWARP - 1) / NWARP;  // column tiles per warp
-  static constexpr int ST = MT * NT / NWARP;           // state tiles per warp
-  static_assert(MT * NT % NWARP == 0, "state tiles");
   static_assert(IN_BYTES % 16 == 0 && RS % 16 == 0, "16-byte cp.async rows");
 };
 
@@ -118,31 +119,45 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
   const size_t s_tok = (size_t)blockIdx.x * p.T;           // first token row of this stream
   uint16_t* ck = p.ckpt + (size_t)blockIdx.x * n * D * D;
 
-  float st[L::ST][4];   // state tiles: W in sweep 1, X in sweep 2
+  // State tiles (W in sweep 1, X in sweep 2): warp w owns whole column tiles nt = w + 8 ct
+  // (all d/16 row tiles of each). Columns of both recurrences are independent, so each warp
+  // carries its own columns from chunk to chunk without block barriers.
+  float st[L::CT][L::MT][4];
   auto load_state = [&](const float* src) {
 #pragma unroll
-    for (int r = 0; r < L::ST; ++r) {
-      const int tau = warp + NWARP * r, row = (tau / L::NT) * 16 + g, col = (tau % L::NT) * 8 + 2 * tq;
-      if (src) {
-        const float* s = src + (size_t)blockIdx.x * D * D;
-        const float2 u = *reinterpret_cast<const float2*>(s + row * D + col);
-        const float2 v = *reinterpret_cast<const float2*>(s + (row + 8) * D + col);
-        st[r][0] = u.x, st[r][1] = u.y, st[r][2] = v.x, st[r][3] = v.y;
-      } else {
-        st[r][0] = st[r][1] = st[r][2] = st[r][3] = 0.f;
+    for (int ct = 0; ct < L::CT; ++ct) {
+      const int nt = warp + NWARP * ct;
+#pragma unroll
+      for (int mt = 0; mt < L::MT; ++mt) {
+        const int row = mt * 16 + g, col = nt * 8 + 2 * tq;
+        if (src && nt < L::NT) {
+          const float* s = src + (size_t)blockIdx.x * D * D;
+          const float2 u = *reinterpret_cast<const float2*>(s + row * D + col);
+          const float2 v = *reinterpret_cast<const float2*>(s + (row + 8) * D + col);
+          st[ct][mt][0] = u.x, st[ct][mt][1] = u.y, st[ct][mt][2] = v.x, st[ct][mt][3] = v.y;
+        } else {
+          st[ct][mt][0] = st[ct][mt][1] = st[ct][mt][2] = st[ct][mt][3] = 0.f;
+        }
       }
     }
   };
   auto put_state = [&](uint32_t dst, uint16_t* gdst) {   // bf16 copy (shared, and a checkpoint)
 #pragma unroll
-    for (int r = 0; r < L::ST; ++r) {
-      const int tau = warp + NWARP * r, row = (tau / L::NT) * 16 + g, col = (tau % L::NT) * 8 + 2 * tq;
-      const uint32_t w0 = pack_bf16(st[r][0], st[r][1]), w1 = pack_bf16(st[r][2], st[r][3]);
-      sts32(dst + row * RS + col * 2, w0);
-      sts32(dst + (row + 8) * RS + col * 2, w1);
-      if (gdst) {
-        *reinterpret_cast<uint32_t*>(gdst + row * D + col) = w0;
-        *reinterpret_cast<uint32_t*>(gdst + (row + 8) * D + col) = w1;
+    for (int ct = 0; ct < L::CT; ++ct) {
+      const int nt = warp + NWARP * ct;
+      if (nt < L::NT) {
+#pragma unroll
+        for (int mt = 0; mt < L::MT; ++mt) {
+          const int row = mt * 16 + g, col = nt * 8 + 2 * tq;
+          const uint32_t w0 = pack_bf16(st[ct][mt][0], st[ct][mt][1]);
+          const uint32_t w1 = pack_bf16(st[ct][mt][2], st[ct][mt][3]);
+          sts32(dst + row * RS + col * 2, w0);
+          sts32(dst + (row + 8) * RS + col * 2, w1);
+          if (gdst) {
+            *reinterpret_cast<uint32_t*>(gdst + row * D + col) = w0;
+            *reinterpret_cast<uint32_t*>(gdst + (row + 8) * D + col) = w1;
+          }
+        }
       }
     }
   };
@@ -162,24 +177,26 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
   };
 
   // ---------------------------------------------------------------- sweep 1: chunk-start states
+  auto load_kv = [&](int c) {
+    const uint32_t buf = sb + (c % L::NBUF) * L::IN_BYTES;
+    cp_rows(buf + L::IN_K, p.K + (s_tok + (size_t)c * BC) * D, BC);
+    cp_rows(buf + L::IN_V, p.V + (s_tok + (size_t)c * BC) * D, BC);
+    cp_eta(buf + L::IN_ETA, c);
+  };
   load_state(p.W0);
   put_state(sb + L::XB, ck);
-  cp_rows(sb + L::IN_K, p.K + s_tok * D, BC);
-  cp_rows(sb + L::IN_V, p.V + s_tok * D, BC);
-  cp_eta(sb + L::IN_ETA, 0);
-  cp_async_commit();
+#pragma unroll
+  for (int s = 0; s < L::NBUF - 1; ++s) {   // one commit group per ring slot, empty past the end
+    if (s < n) load_kv(s);
+    cp_async_commit();
+  }
   for (int c = 0; c < n; ++c) {
-    const uint32_t in = sb + (c & 1) * L::IN_BYTES;
+    const uint32_t in = sb + (c % L::NBUF) * L::IN_BYTES;
     const uint32_t wb = sb + L::XB + (c & 1) * L::WBYTES;
     const uint32_t wn = sb + L::XB + ((c + 1) & 1) * L::WBYTES;
-    cp_async_wait_all();
-    __syncthreads();
-    if (c + 1 < n) {
-      const uint32_t nx = sb + ((c + 1) & 1) * L::IN_BYTES;
-      cp_rows(nx + L::IN_K, p.K + (s_tok + (c + 1) * BC) * D, BC);
-      cp_rows(nx + L::IN_V, p.V + (s_tok + (c + 1) * BC) * D, BC);
-      cp_eta(nx + L::IN_ETA, c + 1);
-    }
+    cp_async_wait<L::NBUF - 2>();   // chunk c's group has landed (this thread's part)
+    __syncthreads();                // ... and every thread's; slot (c - 1) % NBUF is free
+    if (c + L::NBUF - 1 < n) load_kv(c + L::NBUF - 1);
     cp_async_commit();
     // -diag(eta) G = diag(eta) (V - K W), column tiles
 #pragma unroll
@@ -204,15 +221,20 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
               pack_bf16(e1 * (bf16_lo(v1) - acc[2]), e1 * (bf16_hi(v1) - acc[3])));
       }
     }
-    __syncthreads();
-    // W += K^T (-diag(eta) G), state tiles
+    __syncwarp();   // the update below reads only this warp's columns of -diag(eta) G
+    // W += K^T (-diag(eta) G), own columns
 #pragma unroll
-    for (int r = 0; r < L::ST; ++r) {
-      const int tau = warp + NWARP * r, mt = tau / L::NT, nt = tau % L::NT;
-      uint32_t a[4], b[2];
-      frag_a_t(in + L::IN_K, RS, 16 * mt, 0, a);
-      frag_b_t(sb + L::SEG, RS, 0, 8 * nt, b);
-      mma(st[r], a, b);
+    for (int ct = 0; ct < L::CT; ++ct) {
+      const int nt = warp + NWARP * ct;
+      if (nt < L::NT) {
+#pragma unroll
+        for (int mt = 0; mt < L::MT; ++mt) {
+          uint32_t a[4], b[2];
+          frag_a_t(in + L::IN_K, RS, 16 * mt, 0, a);
+          frag_b_t(sb + L::SEG, RS, 0, 8 * nt, b);
+          mma(st[ct][mt], a, b);
+        }
+      }
     }
     put_state(wn, c + 1 < n ? ck + (size_t)(c + 1) * D * D : nullptr);
   }
@@ -231,17 +253,21 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
   };
   load_state(p.dW_out);
   put_state(sb + L::XB, nullptr);
-  prefetch(sb, n - 1);
-  cp_async_commit();
+#pragma unroll
+  for (int s = 0; s < L::NBUF - 1; ++s) {
+    if (s < n) prefetch(sb + s * L::IN_BYTES, n - 1 - s);
+    cp_async_commit();
+  }
   for (int i = 0; i < n; ++i) {
     const int c = n - 1 - i;
     const size_t row0 = s_tok + (size_t)c * BC;
-    const uint32_t in = sb + (i & 1) * L::IN_BYTES;
+    const uint32_t in = sb + (i % L::NBUF) * L::IN_BYTES;
     const uint32_t xb = sb + L::XB + (i & 1) * L::WBYTES;
     const uint32_t xn = sb + L::XB + ((i + 1) & 1) * L::WBYTES;
-    cp_async_wait_all();
+    cp_async_wait<L::NBUF - 2>();
     __syncthreads();
-    if (i + 1 < n) prefetch(sb + ((i + 1) & 1) * L::IN_BYTES, c - 1);
+    if (i + L::NBUF - 1 < n)
+      prefetch(sb + ((i + L::NBUF - 1) % L::NBUF) * L::IN_BYTES, c - (L::NBUF - 1));
     cp_async_commit();
     const float e_g = ldsf(in + L::IN_ETA + 4 * g), e_g8 = ldsf(in + L::IN_ETA + 4 * (g + 8));
 
@@ -408,25 +434,37 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
       }
     }
 #pragma unroll
-    for (int r = 0; r < L::ST; ++r) {
-      const int tau = warp + NWARP * r, mt = tau / L::NT, nt = tau % L::NT;
-      uint32_t a[4], b[2];
-      frag_a_t(in + L::IN_K, RS, 16 * mt, 0, a);
-      frag_b_t(sb + L::SDG, RS, 0, 8 * nt, b);
-      mma(st[r], a, b);
-      frag_a_t(in + L::IN_Q, RS, 16 * mt, 0, a);
-      frag_b_t(in + L::IN_DO, RS, 0, 8 * nt, b);
-      mma(st[r], a, b);
+    for (int ct = 0; ct < L::CT; ++ct) {
+      const int nt = warp + NWARP * ct;
+      if (nt < L::NT) {
+#pragma unroll
+        for (int mt = 0; mt < L::MT; ++mt) {
+          uint32_t a[4], b[2];
+          frag_a_t(in + L::IN_K, RS, 16 * mt, 0, a);
+          frag_b_t(sb + L::SDG, RS, 0, 8 * nt, b);
+          mma(st[ct][mt], a, b);
+          frag_a_t(in + L::IN_Q, RS, 16 * mt, 0, a);
+          frag_b_t(in + L::IN_DO, RS, 0, 8 * nt, b);
+          mma(st[ct][mt], a, b);
+        }
+      }
     }
     put_state(xn, nullptr);
   }
   // dW0 (fp32)
+  float* dw = p.dW0 + (size_t)blockIdx.x * D * D;
 #pragma unroll
-  for (int r = 0; r < L::ST; ++r) {
-    const int tau = warp + NWARP * r, row = (tau / L::NT) * 16 + g, col = (tau % L::NT) * 8 + 2 * tq;
-    float* d = p.dW0 + (size_t)blockIdx.x * D * D;
-    *reinterpret_cast<float2*>(d + row * D + col) = make_float2(st[r][0], st[r][1]);
-    *reinterpret_cast<float2*>(d + (row + 8) * D + col) = make_float2(st[r][2], st[r][3]);
+  for (int ct = 0; ct < L::CT; ++ct) {
+    const int nt = warp + NWARP * ct;
+    if (nt < L::NT) {
+#pragma unroll
+      for (int mt = 0; mt < L::MT; ++mt) {
+        const int row = mt * 16 + g, col = nt * 8 + 2 * tq;
+        *reinterpret_cast<float2*>(dw + row * D + col) = make_float2(st[ct][mt][0], st[ct][mt][1]);
+        *reinterpret_cast<float2*>(dw + (row + 8) * D + col) =
+            make_float2(st[ct][mt][2], st[ct][mt][3]);
+      }
+    }
   }
 }
 
