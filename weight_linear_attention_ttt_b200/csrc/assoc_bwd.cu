@@ -15,8 +15,9 @@
 //     Y : queries K,  keys Q, values dO, rate 1,   start dS_out         (reverse order)
 //     Z : queries V,  keys dO, values Q, rate 1,   start dS_out^T       (reverse order)
 // where reverse order walks the chunks from the last and keeps, inside a chunk, key tokens at
-// or after the query token. The state the Y pass ends with is dS0. A last elementwise pass
-// scales Y and Z by eta in place and forms deta.
+// or after the query token. The state the Y pass ends with is dS0. The Z pass scales its output
+// rows by eta in its own epilogue (it writes dK); a last elementwise pass scales Y by eta in
+// place and forms deta = Y . v.
 #include <cuda_bf16.h>
 
 #include <string>
@@ -47,10 +48,9 @@ __device__ __forceinline__ uint16_t f_to_bf16(float f) {
   return *reinterpret_cast<const uint16_t*>(&b);
 }
 
-// One warp per token row of d = 128 values (four per lane): dV = eta Y and dK = eta Z in place,
-// deta = Y . V.
+// One warp per token row of d = 128 values (four per lane): dV = eta Y in place, deta = Y . V.
 __global__ void assoc_bwd_finish_kernel(const uint16_t* __restrict__ V, const float* eta,
-                                        float eta_scalar, uint16_t* dK, uint16_t* dV,
+                                        float eta_scalar, uint16_t* dV,
                                         float* __restrict__ deta, size_t rows) {
   const int lane = threadIdx.x & 31;
   const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
@@ -58,25 +58,20 @@ __global__ void assoc_bwd_finish_kernel(const uint16_t* __restrict__ V, const fl
        row += warps) {
     const size_t o = row * 128 + 4 * lane;
     const uint2 y = *reinterpret_cast<const uint2*>(dV + o);
-    const uint2 z = *reinterpret_cast<const uint2*>(dK + o);
     const uint2 v = *reinterpret_cast<const uint2*>(V + o);
     const float e = eta ? eta[row] : eta_scalar;
     const uint16_t* yh = reinterpret_cast<const uint16_t*>(&y);
-    const uint16_t* zh = reinterpret_cast<const uint16_t*>(&z);
     const uint16_t* vh = reinterpret_cast<const uint16_t*>(&v);
-    uint2 ov, ok;
+    uint2 ov;
     uint16_t* ovh = reinterpret_cast<uint16_t*>(&ov);
-    uint16_t* okh = reinterpret_cast<uint16_t*>(&ok);
     float dot = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float yf = bf16_to_f(yh[i]);
       dot += yf * bf16_to_f(vh[i]);
       ovh[i] = f_to_bf16(e * yf);
-      okh[i] = f_to_bf16(e * bf16_to_f(zh[i]));
     }
     *reinterpret_cast<uint2*>(dV + o) = ov;
-    *reinterpret_cast<uint2*>(dK + o) = ok;
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, s);
     if (lane == 0) deta[row] = dot;
@@ -132,14 +127,16 @@ int launch_assoc_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx) {
   StateArgs z{a.V, a.dO, a.Q, nullptr, 1.0f, a.dS_out ? gt : nullptr, a.dK, junk, a.B, a.H, a.T,
               d, a.C, 1, a.ws, fwd};
   z.reverse = 1;
+  z.orow = a.eta;                              // dK = eta Z, scaled in the pass's epilogue
+  z.oscale = a.eta ? 1.f : a.eta_scalar;
   r = launch_assoc(z, ctx);
   if (r != kOk) return r;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   assoc_bwd_finish_kernel<<<sms * 8, 256, 0, ctx.stream>>>(
-      static_cast<const uint16_t*>(a.V), a.eta, a.eta_scalar, static_cast<uint16_t*>(a.dK),
-      static_cast<uint16_t*>(a.dV), a.deta, (size_t)BH * a.T);
+      static_cast<const uint16_t*>(a.V), a.eta, a.eta_scalar, static_cast<uint16_t*>(a.dV),
+      a.deta, (size_t)BH * a.T);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *ctx.msg = std::string("assoc bwd finish launch: ") + cudaGetErrorString(e);

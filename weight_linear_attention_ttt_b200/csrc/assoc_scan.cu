@@ -35,6 +35,7 @@
 // update -> bf16 copy -> update; everything else overlaps it.
 #include <algorithm>
 #include <cstdlib>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -62,7 +63,7 @@ struct Smem {
   static constexpr int P_OFF = STAGES * STAGE;                // 2 x [64 t][64 s] bf16
   static constexpr int O_OFF = P_OFF + (SO ? 0 : 2 * 8192);   // 2 x [64 t][128 d_out] bf16
   static constexpr int BAR_OFF = O_OFF + (SO ? 0 : 2 * 16384);
-  static constexpr int BYTES = 1024 + BAR_OFF + 768;   // barriers, then two 64-float tables
+  static constexpr int BYTES = 1024 + BAR_OFF + 1024;  // barriers, then three 64-float tables
   static_assert(BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -94,6 +95,8 @@ struct AssocParams {
   float beta;
   const uint16_t* Oadd;     // pass 2, decay mode: O = Oadd + add_scale * (decayed output)
   float add_scale;
+  const float* orow;        // pass 2: output row of token t scaled by oscale * orow[t] (or null)
+  float oscale;
   unsigned* err;
 };
 
@@ -112,7 +115,10 @@ __device__ __forceinline__ bool named_bar_or(int id, int threads, bool pred) {
   return r != 0;
 }
 
-template <bool SO, bool DECAY = false>
+// REV (chunks last to first, transposed mask) and ROWSC (output row scales) are template
+// parameters, not runtime flags: as runtime branches they measured 37% slower each on the plain
+// forward (the kernel's warp roles are balanced to a few hundred cycles per chunk).
+template <bool SO, bool DECAY = false, bool REV = false, bool ROWSC = false>
 __global__ void __launch_bounds__(THREADS, 1)
     assoc_chunk_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -142,7 +148,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int nch = p.part_len / C;
   // first token of the c-th chunk this CTA processes (in reverse mode the sequence is walked
   // from its end, and part 0 is the last superchunk)
-  auto tok = [&](int c) { return p.reverse ? p.T - C - (tok0 + c * C) : tok0 + c * C; };
+  auto tok = [&](int c) { return REV ? p.T - C - (tok0 + c * C) : tok0 + c * C; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -176,6 +182,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + L::BAR_OFF + 168);
   // decay-mode factors by local token index: beta^(h - i) on values, beta^(i - h) on outputs
   const uint32_t evfac = bar + 256, ocfac = bar + 512;
+  const uint32_t rtab = bar + 768;   // pass 2: the current chunk's output row scales
 
   // State and output warps (pass 2): bf16 copy of 64 of the 128 state columns for `chunk`.
   // Lane = d_out row of S^T; `half` selects d_in columns [64 half, 64 half + 64).
@@ -368,7 +375,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int e = 0; e < 8; ++e) {
             const int sidx = j + e;
             const float x = __uint_as_float(sidx < 32 ? v0[sidx] : v1[sidx - 32]);
-            f[e] = (p.reverse ? sidx >= r : sidx <= r) ? x : 0.f;
+            f[e] = (REV ? sidx >= r : sidx <= r) ? x : 0.f;
           }
           sts128(prow + swz<128>(r * 128 + 2 * j),
                  make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]),
@@ -429,10 +436,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       // lane row t+4 (the two rows fall in disjoint bank halves of the swizzled tile).
       const uint32_t ocol = (dout >> 6) * 8192;
       const uint32_t cb = 2 * ((dout & 63) & ~1);
+      // Row scales (p.orow): chunk c+1's are loaded into registers at the top of iteration c
+      // and written to the table after iteration c's epilogue has read chunk c's, so the load
+      // never stalls the half refresh these warps run on the chain; the barrier that ends the
+      // iteration publishes them.
+      const bool rows_scaled = ROWSC && p.orow && otid < C / 4;
+      auto load_rows = [&](int c) {   // volatile asm: stays where it is issued
+        uint4 v;
+        asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "l"(p.orow + (size_t)stream * p.T + tok(c) + 4 * otid));
+        return v;
+      };
+      uint4 rnext = make_uint4(0u, 0u, 0u, 0u);
+      if (rows_scaled) sts128(rtab + 16 * otid, load_rows(0));
       load_state(1, tl, dout);
       refresh(0, 1, tl);
       for (int c = 0; c < nch; ++c) {
         const int b = c & 1;
+        if (rows_scaled && c + 1 < nch) rnext = load_rows(c + 1);
         // decay mode: the words this lane rewrites, read back before the waits below (all
         // loads in flight at once; each word is read once, before this kernel stores that row)
         uint32_t oadd[DECAY ? 32 : 1];
@@ -442,7 +464,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int t = 0; t < C; ++t) {
             if (t & 4) continue;
-            oadd[(t >> 3) * 4 + (t & 3)] = ob[(size_t)(odd ? t + 4 : t) * (D / 2)];
+            // volatile asm keeps the load here, ahead of the waits, instead of at its use
+            asm volatile("ld.global.u32 %0, [%1];"
+                         : "=r"(oadd[(t >> 3) * 4 + (t & 3)])
+                         : "l"(ob + (size_t)(odd ? t + 4 : t) * (D / 2)));
           }
         }
         // second half of the bf16 state copy for chunk c+1; the go(c+1) arrival also says
@@ -463,27 +488,35 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma::reg_fence(v1);
         umma::fence_before();
         const uint32_t so = sbase + L::O_OFF + 16384 * b + ocol;
+        auto epilogue = [&](auto scaled_c) {
+          constexpr bool SCALED = decltype(scaled_c)::value;
 #pragma unroll
-        for (int t = 0; t < C; ++t) {
-          if (t & 4) continue;
-          const uint32_t* vv = t < 32 ? v0 : v1;
-          const int tt = t & 31;
-          float a = __uint_as_float(vv[tt]), a4 = __uint_as_float(vv[tt + 4]);
-          if (DECAY) {
-            a *= ldsf(ocfac + 4 * t);
-            a4 *= ldsf(ocfac + 4 * (t + 4));
+          for (int t = 0; t < C; ++t) {
+            if (t & 4) continue;
+            const uint32_t* vv = t < 32 ? v0 : v1;
+            const int tt = t & 31;
+            float a = __uint_as_float(vv[tt]), a4 = __uint_as_float(vv[tt + 4]);
+            if (DECAY) {
+              a *= ldsf(ocfac + 4 * t);
+              a4 *= ldsf(ocfac + 4 * (t + 4));
+            }
+            const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
+            float lo = odd ? y : a, hi = odd ? a4 : y;   // columns (dout & ~1) and (dout | 1)
+            const int row = odd ? t + 4 : t;
+            if constexpr (SCALED) {
+              const float sr = p.oscale * (p.orow ? ldsf(rtab + 4 * row) : 1.f);
+              lo *= sr, hi *= sr;
+            }
+            if (DECAY && p.Oadd) {
+              const uint32_t base = oadd[(t >> 3) * 4 + (t & 3)];
+              lo = __uint_as_float(base << 16) + p.add_scale * lo;
+              hi = __uint_as_float(base & 0xffff0000u) + p.add_scale * hi;
+            }
+            const uint32_t w = pack_bf16(lo, hi);
+            sts32(so + swz<128>(row * 128 + cb), w);
           }
-          const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
-          float lo = odd ? y : a, hi = odd ? a4 : y;   // columns (dout & ~1) and (dout | 1)
-          const int row = odd ? t + 4 : t;
-          if (DECAY && p.Oadd) {
-            const uint32_t base = oadd[(t >> 3) * 4 + (t & 3)];
-            lo = __uint_as_float(base << 16) + p.add_scale * lo;
-            hi = __uint_as_float(base & 0xffff0000u) + p.add_scale * hi;
-          }
-          const uint32_t w = pack_bf16(lo, hi);
-          sts32(so + swz<128>(row * 128 + cb), w);
-        }
+        };
+        epilogue(std::integral_constant<bool, ROWSC>{});
         fence_proxy_async_smem();
         named_bar_sync(2, 128);
         if (otid == 0) {
@@ -493,6 +526,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           bulk_commit();
           bulk_wait_read<1>();  // the other staging buffer is free again
         }
+        if (rows_scaled && c + 1 < nch) sts128(rtab + 16 * otid, rnext);
         named_bar_sync(2, 128);
       }
       if (otid == 0) bulk_wait<0>();
@@ -556,7 +590,18 @@ int choose_parts(int streams, int T) {
 template <bool STATE_ONLY>
 int launch_chunk(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                  const CUtensorMap& to, const AssocParams& p, int grid, const LaunchCtx& ctx) {
-  auto kern = p.decay ? assoc_chunk_kernel<STATE_ONLY, true> : assoc_chunk_kernel<STATE_ONLY, false>;
+  using Kern = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, AssocParams);
+  Kern kern = assoc_chunk_kernel<STATE_ONLY, false, false, false>;
+  const bool rows = !STATE_ONLY && (p.orow || p.oscale != 1.f);
+  if (p.decay) {
+    kern = assoc_chunk_kernel<STATE_ONLY, true, false, false>;
+  } else if (p.reverse) {
+    kern = assoc_chunk_kernel<STATE_ONLY, false, true, false>;
+    if constexpr (!STATE_ONLY)
+      if (rows) kern = assoc_chunk_kernel<false, false, true, true>;
+  } else if constexpr (!STATE_ONLY) {
+    if (rows) kern = assoc_chunk_kernel<false, false, false, true>;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Smem<STATE_ONLY>::BYTES);
   if (e != cudaSuccess) {
@@ -606,6 +651,8 @@ int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
   p.beta = a.beta;
   p.Oadd = static_cast<const uint16_t*>(a.Oadd);
   p.add_scale = a.add_scale;
+  p.orow = a.orow;
+  p.oscale = a.oscale;
   p.err = ctx.err;
   return launch_chunk<true>(tq, tk, tv, to, p, BH, ctx);
 }
@@ -649,6 +696,8 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   p.beta = a.beta;
   p.Oadd = static_cast<const uint16_t*>(a.Oadd);
   p.add_scale = a.add_scale;
+  p.orow = a.orow;
+  p.oscale = a.oscale;
   p.err = ctx.err;
   if (P > 1) {
     p.S_dst = static_cast<float*>(a.ws);

@@ -26,6 +26,8 @@
 // bf16 once per chunk for the tensor cores.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -161,13 +163,18 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
       }
     }
   };
-  auto cp_rows = [&](uint32_t dst, const uint16_t* src, int rows) {   // rows x d bf16, dense
-    constexpr int PPR = D / 8;
-    for (int i = threadIdx.x; i < rows * PPR; i += THREADS) {
-      const int r = i / PPR, q = i % PPR;
-      cp_async16(dst + r * RS + q * 16, src + (size_t)r * D + q * 8);
+  // ROWS x d bf16 rows, dense in global memory, into padded shared rows (16-byte pieces)
+  auto cp_rows = [&](auto rows_c, uint32_t dst, const uint16_t* src) {
+    constexpr int ROWS = decltype(rows_c)::value, PPR = D / 8, N = ROWS * PPR;
+#pragma unroll
+    for (int k = 0; k < (N + THREADS - 1) / THREADS; ++k) {
+      const int i = threadIdx.x + k * THREADS;
+      if (N % THREADS == 0 || i < N)
+        cp_async16(dst + (i / PPR) * RS + (i % PPR) * 16, src + (size_t)(i / PPR) * D + (i % PPR) * 8);
     }
   };
+  using Rows16 = std::integral_constant<int, BC>;
+  using RowsD = std::integral_constant<int, D>;
   auto cp_eta = [&](uint32_t dst, int c) {
     if (p.eta) {
       if (threadIdx.x < 4) cp_async16(dst + threadIdx.x * 16, p.eta + s_tok + c * BC + threadIdx.x * 4);
@@ -179,8 +186,8 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
   // ---------------------------------------------------------------- sweep 1: chunk-start states
   auto load_kv = [&](int c) {
     const uint32_t buf = sb + (c % L::NBUF) * L::IN_BYTES;
-    cp_rows(buf + L::IN_K, p.K + (s_tok + (size_t)c * BC) * D, BC);
-    cp_rows(buf + L::IN_V, p.V + (s_tok + (size_t)c * BC) * D, BC);
+    cp_rows(Rows16{}, buf + L::IN_K, p.K + (s_tok + (size_t)c * BC) * D);
+    cp_rows(Rows16{}, buf + L::IN_V, p.V + (s_tok + (size_t)c * BC) * D);
     cp_eta(buf + L::IN_ETA, c);
   };
   load_state(p.W0);
@@ -203,14 +210,17 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
     for (int ct = 0; ct < L::CT; ++ct) {
       const int nt = warp + NWARP * ct;
       if (nt < L::NT) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        // two accumulators (even / odd k-steps) halve the dependent MMA chain
+        float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int ks = 0; ks < L::KS; ++ks) {
           uint32_t a[4], b[2];
           frag_a(in + L::IN_K, RS, 0, 16 * ks, a);
           frag_b_t(wb, RS, 16 * ks, 8 * nt, b);
-          mma(acc, a, b);
+          mma((ks & 1) ? acc2 : acc, a, b);
         }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] += acc2[j];
         const int col = 8 * nt + 2 * tq;
         const uint32_t v0 = ldsu32(in + L::IN_V + g * RS + col * 2);
         const uint32_t v1 = ldsu32(in + L::IN_V + (g + 8) * RS + col * 2);
@@ -244,11 +254,11 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
   // ---------------------------------------------------------------- sweep 2: adjoint, reversed
   auto prefetch = [&](uint32_t buf, int c) {
     const size_t row = s_tok + (size_t)c * BC;
-    cp_rows(buf + L::IN_Q, p.Q + row * D, BC);
-    cp_rows(buf + L::IN_K, p.K + row * D, BC);
-    cp_rows(buf + L::IN_V, p.V + row * D, BC);
-    cp_rows(buf + L::IN_DO, p.dO + row * D, BC);
-    cp_rows(buf + L::IN_W, ck + (size_t)c * D * D, D);
+    cp_rows(Rows16{}, buf + L::IN_Q, p.Q + row * D);
+    cp_rows(Rows16{}, buf + L::IN_K, p.K + row * D);
+    cp_rows(Rows16{}, buf + L::IN_V, p.V + row * D);
+    cp_rows(Rows16{}, buf + L::IN_DO, p.dO + row * D);
+    cp_rows(RowsD{}, buf + L::IN_W, ck + (size_t)c * D * D);
     cp_eta(buf + L::IN_ETA, c);
   };
   load_state(p.dW_out);
@@ -332,14 +342,16 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
 
     // Phase B (warps 0-1, score columns 8w..8w+7): dA = -tril(dO G^T), dS, A, deta's first term
     if (warp < 2) {
-      float pacc[4] = {0.f, 0.f, 0.f, 0.f};
+      float pacc[4] = {0.f, 0.f, 0.f, 0.f}, pacc2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ks = 0; ks < L::KS; ++ks) {
         uint32_t a[4], b[2];
         frag_a(in + L::IN_DO, RS, 0, 16 * ks, a);
         frag_b(sb + L::SG, RS, 8 * warp, 16 * ks, b);
-        mma(pacc, a, b);
+        mma((ks & 1) ? pacc2 : pacc, a, b);
       }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) pacc[j] += pacc2[j];
       float col_sum[2] = {0.f, 0.f};
       float dsv[4], av[4];
 #pragma unroll

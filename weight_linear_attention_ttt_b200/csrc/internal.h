@@ -35,6 +35,10 @@ struct StateArgs {
   // decay mode: O = Oadd + add_scale * (decayed output), Oadd [B,H,T,d] bf16 (may equal O)
   const void* Oadd = nullptr;
   float add_scale = 0.f;
+  // output row i of token t (pass 2) multiplied by oscale * orow[t] (orow [B,H,T] fp32 or
+  // nullptr), before any Oadd combination
+  const float* orow = nullptr;
+  float oscale = 1.f;
 };
 
 struct InplaceArgs {
