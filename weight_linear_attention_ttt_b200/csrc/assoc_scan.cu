@@ -314,6 +314,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool rowthr = lane < 16;            // holds an M = 64 score row
     const int r = 16 * q + lane;              // that row (token t of the chunk)
     const int otid = threadIdx.x - 64;       // 0..127
+    // decay mode: the value factor of each of this thread's four token rows (rows of pieces
+    // it and it + 4 coincide), read from the table once instead of per chunk
+    float vfac[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      vfac[j] = DECAY ? ldsf(evfac + 4 * (((otid + 128 * j) & 511) >> 3)) : 1.f;
     for (int c = 0; c < nch; ++c) {
       const int s = c % ST, b = c & 1;
       const uint32_t stg = sbase + s * L::STAGE;
@@ -342,7 +348,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int i = otid + 128 * it;
           const int sub = i >> 9, w = i & 511;
           const uint32_t a = vt + sub * 8192 + swz<128>((w >> 3) * 128 + (w & 7) * 16);
-          const float f = e[it] * p.eta_mul * (DECAY ? cf * ldsf(evfac + 4 * (w >> 3)) : 1.f);
+          const float f = e[it] * p.eta_mul * (DECAY ? cf * vfac[it & 3] : 1.f);
           sts128(a, make_uint4(pack_bf16(bf16_lo(x[it].x) * f, bf16_hi(x[it].x) * f),
                                pack_bf16(bf16_lo(x[it].y) * f, bf16_hi(x[it].y) * f),
                                pack_bf16(bf16_lo(x[it].z) * f, bf16_hi(x[it].z) * f),
@@ -490,15 +496,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t so = sbase + L::O_OFF + 16384 * b + ocol;
         auto epilogue = [&](auto scaled_c) {
           constexpr bool SCALED = decltype(scaled_c)::value;
+          uint4 of0 = make_uint4(0u, 0u, 0u, 0u), of4 = of0;
 #pragma unroll
           for (int t = 0; t < C; ++t) {
             if (t & 4) continue;
             const uint32_t* vv = t < 32 ? v0 : v1;
             const int tt = t & 31;
             float a = __uint_as_float(vv[tt]), a4 = __uint_as_float(vv[tt + 4]);
-            if (DECAY) {
-              a *= ldsf(ocfac + 4 * t);
-              a4 *= ldsf(ocfac + 4 * (t + 4));
+            if (DECAY) {   // row factors of rows t0..t0+3 and t0+4..t0+7, four per load
+              if ((t & 3) == 0) {
+                of0 = lds128(ocfac + 4 * t);
+                of4 = lds128(ocfac + 4 * (t + 4));
+              }
+              const int k = t & 3;
+              a *= __uint_as_float(k == 0 ? of0.x : k == 1 ? of0.y : k == 2 ? of0.z : of0.w);
+              a4 *= __uint_as_float(k == 0 ? of4.x : k == 1 ? of4.y : k == 2 ? of4.z : of4.w);
             }
             const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
             float lo = odd ? y : a, hi = odd ? a4 : y;   // columns (dout & ~1) and (dout | 1)
