@@ -172,8 +172,12 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS, WC>::THREADS, 1)
         const int rows = min(R, T - j * R);
         const uint32_t bytes = 3 * Cfg::TILE_BYTES + (p.eta ? rows * 4 : 0);
         const uint32_t fb = full_bar + 8 * s;
-        mbar_arrive_expect_tx(fb, bytes);
         const uint32_t st = sbase + s * Cfg::STAGE_BYTES;
+        // a scalar rate is written into the stage's rate slot, so the compute warps read the
+        // slot unconditionally (the arrival below releases these stores)
+        if (!p.eta)
+          for (int i = 0; i < R; ++i) stsf(st + 3 * Cfg::TILE_BYTES + 4 * i, p.eta_scalar);
+        mbar_arrive_expect_tx(fb, bytes);
 #pragma unroll
         for (int sub = 0; sub < Cfg::NSUB; ++sub) {
           tma_load_3d(st + sub * Cfg::SUB_BYTES, &tmQ, fb, sub * Cfg::SUB, j * R, stream);
@@ -320,12 +324,8 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS, WC>::THREADS, 1)
       }
       o.v0 = ld_shared_u32(sV + cb + o_v0);
       o.v1 = ld_shared_u32(sV + cb + o_v1);
-      if (p.eta) {
-        o.eg = ld_shared_f32(sEta + 4 * (16 * c + g));
-        o.eg8 = ld_shared_f32(sEta + 4 * (16 * c + g + 8));
-      } else {
-        o.eg = o.eg8 = p.eta_scalar;
-      }
+      o.eg = ld_shared_f32(sEta + 4 * (16 * c + g));
+      o.eg8 = ld_shared_f32(sEta + 4 * (16 * c + g + 8));
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) ldsm_x4(sQ + cb + o_arow[ks], o.qa[ks]);
       ld_shared_v4(sL + c * 512 + lane * 16, o.la);
@@ -407,14 +407,10 @@ __global__ void __launch_bounds__(DualCfg<D, NW, CPS, WC>::THREADS, 1)
         ldsm_x4_t(sK + cb + o_btrn[ks], o.kt[ks]);
       }
       ldsm_x4_t(sV + cb + o_vt, o.vt);
-      if (p.eta) {
-        o.e0 = ld_shared_f32(sEta + 4 * (16 * c + 2 * tq));
-        o.e1 = ld_shared_f32(sEta + 4 * (16 * c + 2 * tq + 1));
-        o.e8 = ld_shared_f32(sEta + 4 * (16 * c + 8 + 2 * tq));
-        o.e9 = ld_shared_f32(sEta + 4 * (16 * c + 9 + 2 * tq));
-      } else {
-        o.e0 = o.e1 = o.e8 = o.e9 = p.eta_scalar;
-      }
+      o.e0 = ld_shared_f32(sEta + 4 * (16 * c + 2 * tq));
+      o.e1 = ld_shared_f32(sEta + 4 * (16 * c + 2 * tq + 1));
+      o.e8 = ld_shared_f32(sEta + 4 * (16 * c + 8 + 2 * tq));
+      o.e9 = ld_shared_f32(sEta + 4 * (16 * c + 9 + 2 * tq));
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) ldsm_x4(sQ + cb + o_arow[ks], o.qa[ks]);
     };

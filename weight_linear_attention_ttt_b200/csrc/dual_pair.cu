@@ -138,8 +138,12 @@ __global__ void __launch_bounds__(PairCfg<D, NP, CPS>::THREADS, 1)
         const int rows = min(R, T - j * R);
         const uint32_t bytes = 3 * Cfg::TILE_BYTES + (p.eta ? rows * 4 : 0);
         const uint32_t fb = full_bar + 8 * s;
-        mbar_arrive_expect_tx(fb, bytes);
         const uint32_t st = sbase + s * Cfg::STAGE_BYTES;
+        // a scalar rate is written into the stage's rate slot, so the compute warps read the
+        // slot unconditionally (the arrival below releases these stores)
+        if (!p.eta)
+          for (int i = 0; i < R; ++i) stsf(st + 3 * Cfg::TILE_BYTES + 4 * i, p.eta_scalar);
+        mbar_arrive_expect_tx(fb, bytes);
 #pragma unroll
         for (int sub = 0; sub < Cfg::NSUB; ++sub) {
           tma_load_3d(st + sub * Cfg::SUB_BYTES, &tmQ, fb, sub * Cfg::SUB, j * R, stream);
@@ -228,14 +232,10 @@ __global__ void __launch_bounds__(PairCfg<D, NP, CPS>::THREADS, 1)
           ldsm_x4_t(sK + cb + o_btrn[ks], o.kt[ks]);
         }
         ldsm_x4_t(sV + cb + o_vt, o.vt);
-        if (p.eta) {
-          o.e0 = lds_f32(sEta + 4 * (16 * c + 2 * tq));
-          o.e1 = lds_f32(sEta + 4 * (16 * c + 2 * tq + 1));
-          o.e8 = lds_f32(sEta + 4 * (16 * c + 8 + 2 * tq));
-          o.e9 = lds_f32(sEta + 4 * (16 * c + 9 + 2 * tq));
-        } else {
-          o.e0 = o.e1 = o.e8 = o.e9 = p.eta_scalar;
-        }
+        o.e0 = lds_f32(sEta + 4 * (16 * c + 2 * tq));
+        o.e1 = lds_f32(sEta + 4 * (16 * c + 2 * tq + 1));
+        o.e8 = lds_f32(sEta + 4 * (16 * c + 8 + 2 * tq));
+        o.e9 = lds_f32(sEta + 4 * (16 * c + 9 + 2 * tq));
       };
       // bf16(W^T) -> P^T = W^T K^T -> E^T -> W^T -= E^T K; hands bf16(W^T) and bf16(E^T) over.
       auto step = [&](const Ops& o) {
