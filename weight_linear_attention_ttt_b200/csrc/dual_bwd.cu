@@ -19,6 +19,8 @@
 //      m16n8k16 (bf16 operands, fp32 accumulation) in four phases separated by block barriers.
 // Inputs (and in sweep 2 the checkpoints) stream through a ring of shared-memory slots filled by
 // cp.async up to three chunks ahead, so that the serial chunk loop does not wait on HBM latency.
+// Results (checkpoints, dQ, dK, dV) are staged in shared memory and leave as whole 16-byte
+// pieces: written straight from the MMA fragments, every row would be an 8-byte scatter.
 // Work split over 8 warps: a 16 x d result is cut into d/8 column tiles (n8) dealt round-robin
 // to the warps; a warp owns the same columns of the state (all d/16 row tiles), so the state
 // recurrences (column-independent) need no barrier of their own.
@@ -26,6 +28,7 @@
 // bf16 once per chunk for the tensor cores.
 #include <cuda_bf16.h>
 
+#include <string>
 #include <type_traits>
 
 #include "internal.h"
@@ -59,7 +62,10 @@ struct BwdCfg {
   static constexpr int SDS = SA + BC * SRS;        // dS (bf16 [16][24])
   static constexpr int SDE2 = SDS + BC * SRS;      // per column tile: -sum_j U G  [NT][16]
   static constexpr int SDE1 = SDE2 + (D / 8) * 64; // sum_t dA (Q K^T)  [16]
-  static constexpr int SMEM = SDE1 + 64;
+  static constexpr int SOQ = SDE1 + 64;            // dQ, dV, dK staged for coalesced stores
+  static constexpr int SOV = SOQ + TILE;
+  static constexpr int SOK = SOV + TILE;
+  static constexpr int SMEM = SOK + TILE;
   static constexpr int NT = D / 8, MT = D / 16, KS = D / 16;
   static constexpr int CT = (NT + NWARP - 1) / NWARP;  // column tiles per warp
   static_assert(IN_BYTES % 16 == 0 && RS % 16 == 0, "16-byte cp.async rows");
@@ -108,6 +114,20 @@ __device__ __forceinline__ void frag_b_t(uint32_t base, int rs, int k0, int n0,
 }
 __device__ __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
   mma16816(d, a[0], a[1], a[2], a[3], b[0], b[1]);
+}
+
+// rows x d bf16 from a padded shared tile (row stride rs bytes) to dense global rows, one
+// 16-byte piece per thread and step (a warp writes four whole 128-byte rows at d = 64)
+template <int D, int ROWS, int NTHR>
+__device__ __forceinline__ void copy_out(uint32_t src, int rs, uint16_t* dst, int tid) {
+  constexpr int PPR = D / 8, N = ROWS * PPR;
+#pragma unroll
+  for (int k = 0; k < (N + NTHR - 1) / NTHR; ++k) {
+    const int i = tid + k * NTHR;
+    if (N % NTHR == 0 || i < N)
+      *reinterpret_cast<uint4*>(dst + (size_t)(i / PPR) * D + (i % PPR) * 8) =
+          lds128(src + (i / PPR) * rs + (i % PPR) * 16);
+  }
 }
 
 template <int D>
@@ -191,7 +211,7 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
     cp_eta(buf + L::IN_ETA, c);
   };
   load_state(p.W0);
-  put_state(sb + L::XB, ck);
+  put_state(sb + L::XB, nullptr);
 #pragma unroll
   for (int s = 0; s < L::NBUF - 1; ++s) {   // one commit group per ring slot, empty past the end
     if (s < n) load_kv(s);
@@ -205,6 +225,8 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
     __syncthreads();                // ... and every thread's; slot (c - 1) % NBUF is free
     if (c + L::NBUF - 1 < n) load_kv(c + L::NBUF - 1);
     cp_async_commit();
+    // checkpoint W_c (complete in wb since the barrier above), coalesced 16-byte stores
+    copy_out<D, D, THREADS>(wb, RS, ck + (size_t)c * D * D, threadIdx.x);
     // -diag(eta) G = diag(eta) (V - K W), column tiles
 #pragma unroll
     for (int ct = 0; ct < L::CT; ++ct) {
@@ -246,7 +268,7 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
         }
       }
     }
-    put_state(wn, c + 1 < n ? ck + (size_t)(c + 1) * D * D : nullptr);
+    put_state(wn, nullptr);
   }
   cp_async_wait_all();
   __syncthreads();   // checkpoints written above are read back below through cp.async
@@ -280,6 +302,8 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
       prefetch(sb + ((i + L::NBUF - 1) % L::NBUF) * L::IN_BYTES, c - (L::NBUF - 1));
     cp_async_commit();
     const float e_g = ldsf(in + L::IN_ETA + 4 * g), e_g8 = ldsf(in + L::IN_ETA + 4 * (g + 8));
+    if (i > 0)   // dK of the previous chunk (c + 1), staged in its phase D
+      copy_out<D, BC, THREADS>(sb + L::SOK, RS, p.dK + (row0 + BC) * D, threadIdx.x);
 
     // Phase A: G = K W - V, U = K X, dO W^T (column tiles); scores Q K^T (warps 0-1)
     float G[L::CT][4], U[L::CT][4], T1[L::CT][4];
@@ -404,11 +428,10 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
         const int col = 8 * nt + 2 * tq;
         sts32(sb + L::SDG + g * RS + col * 2, pack_bf16(dg[0], dg[1]));
         sts32(sb + L::SDG + (g + 8) * RS + col * 2, pack_bf16(dg[2], dg[3]));
-        const size_t o0 = (row0 + g) * D + col, o1 = (row0 + g + 8) * D + col;
-        *reinterpret_cast<uint32_t*>(p.dV + o0) = pack_bf16(-dg[0], -dg[1]);
-        *reinterpret_cast<uint32_t*>(p.dV + o1) = pack_bf16(-dg[2], -dg[3]);
-        *reinterpret_cast<uint32_t*>(p.dQ + o0) = pack_bf16(T1[ct][0], T1[ct][1]);
-        *reinterpret_cast<uint32_t*>(p.dQ + o1) = pack_bf16(T1[ct][2], T1[ct][3]);
+        sts32(sb + L::SOV + g * RS + col * 2, pack_bf16(-dg[0], -dg[1]));
+        sts32(sb + L::SOV + (g + 8) * RS + col * 2, pack_bf16(-dg[2], -dg[3]));
+        sts32(sb + L::SOQ + g * RS + col * 2, pack_bf16(T1[ct][0], T1[ct][1]));
+        sts32(sb + L::SOQ + (g + 8) * RS + col * 2, pack_bf16(T1[ct][2], T1[ct][3]));
       }
     }
     if (warp == NWARP - 1 && lane < BC) {
@@ -420,6 +443,8 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
     __syncthreads();
 
     // Phase D: dK = dS^T Q + dG W^T - diag(eta) G X^T (column tiles); X += Q^T dO + K^T dG
+    copy_out<D, BC, THREADS>(sb + L::SOV, RS, p.dV + row0 * D, threadIdx.x);
+    copy_out<D, BC, THREADS>(sb + L::SOQ, RS, p.dQ + row0 * D, threadIdx.x);
 #pragma unroll
     for (int ct = 0; ct < L::CT; ++ct) {
       const int nt = warp + NWARP * ct;
@@ -439,10 +464,8 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
           mma(k2, a, b);
         }
         const int col = 8 * nt + 2 * tq;
-        *reinterpret_cast<uint32_t*>(p.dK + (row0 + g) * D + col) =
-            pack_bf16(k1[0] - k2[0], k1[1] - k2[1]);
-        *reinterpret_cast<uint32_t*>(p.dK + (row0 + g + 8) * D + col) =
-            pack_bf16(k1[2] - k2[2], k1[3] - k2[3]);
+        sts32(sb + L::SOK + g * RS + col * 2, pack_bf16(k1[0] - k2[0], k1[1] - k2[1]));
+        sts32(sb + L::SOK + (g + 8) * RS + col * 2, pack_bf16(k1[2] - k2[2], k1[3] - k2[3]));
       }
     }
 #pragma unroll
@@ -463,6 +486,8 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
     }
     put_state(xn, nullptr);
   }
+  __syncthreads();   // dK of chunk 0
+  copy_out<D, BC, THREADS>(sb + L::SOK, RS, p.dK + s_tok * D, threadIdx.x);
   // dW0 (fp32)
   float* dw = p.dW0 + (size_t)blockIdx.x * D * D;
 #pragma unroll
