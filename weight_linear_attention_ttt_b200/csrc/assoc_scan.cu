@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // State and output warps (pass 2): bf16 copy of 64 of the 128 state columns for `chunk`.
   // Lane = d_out row of S^T; `half` selects d_in columns [64 half, 64 half + 64).
+  const float beta_c = DECAY ? powf(p.beta, (float)C) : 1.f;   // decay of the state per chunk
   auto refresh = [&](int chunk, int half, uint32_t tl) {
     uint32_t a0[32], a1[32], o[32];
     umma::ld32x32(tmem + tl + TM_S + 64 * half, a0);
@@ -195,11 +196,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     umma::reg_fence(a1);
     if (DECAY && chunk > 0) {
       // state of the next chunk: beta^C times the updated one, written back in place
-      const float bc = powf(p.beta, (float)C);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        a0[j] = __float_as_uint(__uint_as_float(a0[j]) * bc);
-        a1[j] = __float_as_uint(__uint_as_float(a1[j]) * bc);
+        a0[j] = __float_as_uint(__uint_as_float(a0[j]) * beta_c);
+        a1[j] = __float_as_uint(__uint_as_float(a1[j]) * beta_c);
       }
       umma::st32x32(tmem + tl + TM_S + 64 * half, a0);
       umma::st32x32(tmem + tl + TM_S + 64 * half + 32, a1);
