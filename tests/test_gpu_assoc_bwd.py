@@ -61,6 +61,20 @@ def test_scalar_eta_and_zero_states(cuda_lib):
     check(x, run(x))
 
 
+def test_zero_and_tiny_rates(cuda_lib):
+    """Rows whose rate is zero or tiny get the oracle's dV and deta like every other row; a zero
+    scalar rate gives exactly zero dK and dV."""
+    x = make(1, 2, 512, seed=21)
+    x["eta"][:, :, ::7] = 0.0
+    x["eta"][:, :, 3::11] = 1e-30
+    check(x, run(x))
+    x = make(1, 1, 256, seed=22, eta="const", states=False)
+    x["eta_scalar"] = 0.0
+    got = run(x)
+    assert torch.count_nonzero(got[2]) == 0 and torch.count_nonzero(got[1]) == 0
+    check(x, got)
+
+
 @pytest.mark.parametrize("parts", ["1", "2", "4", "16"])
 def test_forced_superchunk_counts(cuda_lib, monkeypatch, parts):
     """The reverse-order passes split into superchunks give the oracle's gradients for every P."""

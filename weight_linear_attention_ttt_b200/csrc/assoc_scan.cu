@@ -334,21 +334,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float cf = (DECAY && SO) ? powf(p.beta, (float)(p.part_len - C - c * C)) : 1.f;
         const uint32_t vt = stg + L::V_OFF;
         uint4 x[8];
-        float e[8];
+        float e[4];
 #pragma unroll
         for (int it = 0; it < 8; ++it) {
           const int i = otid + 128 * it;                // 0..1023
           const int sub = i >> 9, w = i & 511;          // sub-tile, piece within it
           const uint32_t a = vt + sub * 8192 + swz<128>((w >> 3) * 128 + (w & 7) * 16);
           x[it] = lds128(a);
-          e[it] = p.eta ? ldsf(stg + L::ETA_OFF + 4 * (w >> 3)) : p.eta_scalar;
+          // pieces it and it + 4 share a token row: four rate loads per thread, not eight
+          if (it < 4) e[it] = p.eta ? ldsf(stg + L::ETA_OFF + 4 * (w >> 3)) : p.eta_scalar;
         }
 #pragma unroll
         for (int it = 0; it < 8; ++it) {
           const int i = otid + 128 * it;
           const int sub = i >> 9, w = i & 511;
           const uint32_t a = vt + sub * 8192 + swz<128>((w >> 3) * 128 + (w & 7) * 16);
-          const float f = e[it] * p.eta_mul * (DECAY ? cf * vfac[it & 3] : 1.f);
+          const float f = e[it & 3] * p.eta_mul * (DECAY ? cf * vfac[it & 3] : 1.f);
           sts128(a, make_uint4(pack_bf16(bf16_lo(x[it].x) * f, bf16_hi(x[it].x) * f),
                                pack_bf16(bf16_lo(x[it].y) * f, bf16_hi(x[it].y) * f),
                                pack_bf16(bf16_lo(x[it].z) * f, bf16_hi(x[it].z) * f),
