@@ -103,3 +103,77 @@ def test_python_binding_rejects_non_cuda_tensors(lib):
     x = torch.zeros(1, 1, 16, 32)
     with pytest.raises(ValueError):
         ttt.ttt_linear_dual_fwd(x, x, x, C=16)
+
+
+def _bwd(lib, fn, **kw):
+    """Backward entry points (associative and dual form) share one argument list."""
+    args = dict(Q=A, K=2 * A, V=3 * A, eta=4 * A, eta_scalar=0.0, S0=5 * A, dO=6 * A,
+                dS_out=7 * A, dQ=8 * A, dK=9 * A, dV=10 * A, deta=11 * A, dS0=12 * A,
+                B=1, H=1, T=64, d=128, C=64, dt=1, ws=13 * A, ws_bytes=1 << 19, stream=0)
+    args.update(kw)
+    v = ctypes.c_void_p
+    return getattr(lib, fn)(
+        v(args["Q"]), v(args["K"]), v(args["V"]), v(args["eta"]),
+        ctypes.c_float(args["eta_scalar"]), v(args["S0"]), v(args["dO"]), v(args["dS_out"]),
+        v(args["dQ"]), v(args["dK"]), v(args["dV"]), v(args["deta"]), v(args["dS0"]),
+        args["B"], args["H"], args["T"], args["d"], args["C"], args["dt"], v(args["ws"]),
+        args["ws_bytes"], v(args["stream"]))
+
+
+@pytest.mark.parametrize("fn,base", [
+    ("ttt_assoc_scan_bwd", dict(d=128, C=64, T=128)),
+    ("ttt_linear_dual_bwd", dict(d=64, C=16, T=64)),
+])
+@pytest.mark.parametrize("kw,status", [
+    (dict(dQ=0), 1), (dict(dO=0), 1), (dict(deta=0), 1),
+    (dict(V=3 * A + 8), 1),                  # misaligned
+    (dict(T=100), 1),                        # T % C != 0
+    (dict(H=0), 1), (dict(dt=5), 1),
+    (dict(d=48), 2),                         # unsupported head dim
+    (dict(ws_bytes=16), 3),                  # workspace too small
+    (dict(ws=0), 3),
+    (dict(dK=2 * A), 1),                     # an output on an input
+    (dict(dQ=8 * A, dK=8 * A + 64), 1),      # two outputs overlap
+])
+def test_backward_validation(lib, fn, base, kw, status):
+    ws = {"ws_bytes": 1 << 30}
+    assert _bwd(lib, fn, **dict(base, **dict(ws, **kw))) == status
+    assert lib.ttt_last_error_message() != b""
+    assert lib.ttt_launch_count() == 0
+
+
+def test_backward_chunk_size_rules(lib):
+    # the dual form's backward runs the C = 16 mini-batch only; the associative one C = 64
+    assert _bwd(lib, "ttt_linear_dual_bwd", d=64, C=32, T=64, ws_bytes=1 << 30) == 2
+    assert _bwd(lib, "ttt_assoc_scan_bwd", d=128, C=16, T=64, ws_bytes=1 << 30) == 2
+    assert lib.ttt_launch_count() == 0
+
+
+def test_workspace_size_queries(lib):
+    # dual-form backward: one bf16 d x d checkpoint per chunk and stream
+    assert lib.ttt_linear_dual_bwd_workspace_size(8, 12, 2048, 64, 16, 1) == 8 * 12 * 128 * 64 * 64 * 2
+    assert lib.ttt_linear_dual_bwd_workspace_size(8, 12, 2048, 64, 32, 1) == 0   # C unsupported
+    assert lib.ttt_linear_dual_bwd_workspace_size(8, 12, 2040, 64, 16, 1) == 0   # T % C
+    assert lib.ttt_linear_dual_bwd_workspace_size(1, 1, 64, 64, 16, 0) == 0      # fp32
+    assert lib.ttt_assoc_scan_bwd_workspace_size(4, 16, 65536, 128, 64, 1) > 0
+    assert lib.ttt_assoc_scan_bwd_workspace_size(4, 16, 65536, 64, 64, 1) == 0
+    assert lib.ttt_assoc_momentum_workspace_size(4, 16, 65536, 128, 64, 1) > 0
+    assert lib.ttt_assoc_momentum_workspace_size(4, 16, 100, 128, 64, 1) == 0
+    # the convolved embeddings (bf16, 256-byte aligned) and one 256-byte counter slot
+    assert lib.ttt_lm_target_workspace_size(32768, 2560, 2560, 4) == 32768 * 2560 * 2 + 256
+    assert lib.ttt_lm_target_workspace_size(0, 2560, 2560, 4) == 0
+
+
+def test_momentum_validation(lib):
+    v = ctypes.c_void_p
+
+    def mom(beta, M_out=9 * A, d=128):
+        return lib.ttt_assoc_momentum_fwd(v(A), v(2 * A), v(3 * A), None, ctypes.c_float(1.0),
+                                          ctypes.c_float(beta), None, None, v(6 * A), v(7 * A),
+                                          v(M_out), 1, 1, 128, d, 64, 1, v(10 * A), 1 << 30, None)
+
+    assert mom(0.95) == 2 and mom(0.1) == 2 and mom(1.0) == 2   # outside [0.25, 0.9]
+    assert mom(0.5, M_out=0) == 1
+    assert mom(0.5, d=64) == 2
+    assert mom(0.5, M_out=6 * A + 64) == 1                      # M_out overlaps O
+    assert lib.ttt_launch_count() == 0
