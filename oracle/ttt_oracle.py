@@ -43,7 +43,9 @@ the associative backward against central finite differences of the forward defin
 against autograd of an independent torch restatement; the dual-form backward against central
 finite differences and against autograd through mini-batch gradient steps that autograd itself
 takes; the momentum recurrence against the plain one at beta = 0, against its closed
-weighted-sum form and against hand-worked tokens. Every function below has at least one pin.
+weighted-sum form and against hand-worked tokens; the segment maps of the dual form against
+the product of the chunk matrices and the zero-start dual form, and the segmented evaluation
+against the sequential chunk loop. Every function below has at least one pin.
 """
 from __future__ import annotations
 
@@ -122,6 +124,49 @@ def dual_form(Q, K, V, eta, W0, C: int, *, threads: int = 1, streams=None):
         O = O.reshape(B, H, T, d)
         W = W.reshape(B, H, d, d)
     return O, W
+
+
+def dual_segment_maps_stream(K, V, eta, C: int):
+    """The chunk updates of one segment of tokens composed into one affine map
+    W_end = A W_start + B [KVB, associativity paragraph: without weight normalisation the
+    update is associative; applied here to the dual form's affine chunk update
+    W' = (I - K^T diag(eta) K) W + K^T diag(eta) V]. Propagates the pair (A, B) from (I, 0)
+    through the segment's chunks in order. Returns (A [d, d], B [d, d])."""
+    K, V = _f64(K), _f64(V)
+    T, d = K.shape
+    if C <= 0 or T % C:
+        raise ValueError("T must be a positive multiple of C")
+    e_all = _eta_stream(eta, T)
+    A, B = np.eye(d), np.zeros((d, d))
+    for c0 in range(0, T, C):
+        k, v, e = K[c0:c0 + C], V[c0:c0 + C], e_all[c0:c0 + C]
+        A = A - k.T @ (e[:, None] * (k @ A))
+        B = B - k.T @ (e[:, None] * (k @ B - v))
+    return A, B
+
+
+def dual_form_segmented_stream(Q, K, V, eta, W0, C: int, L: int):
+    """Sequence-parallel evaluation of ``dual_form_stream``: the sequence is cut into segments of
+    L tokens (L a multiple of C); each segment's map (A_s, B_s) comes from
+    ``dual_segment_maps_stream``; the segment start states follow by folding the maps in order,
+    W_start(s+1) = A_s W_start(s) + B_s; every segment then runs the dual form from its start
+    state. Returns (O [T, d], W_final [d, d]); equal to ``dual_form_stream`` up to rounding."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    T, d = Q.shape
+    if L <= 0 or L % C or T % L:
+        raise ValueError("L must be a positive multiple of C that divides T")
+    e_all = _eta_stream(eta, T)
+    W = np.zeros((d, d)) if W0 is None else _f64(W0).copy()
+    starts = []
+    for s0 in range(0, T, L):
+        starts.append(W.copy())
+        A, B = dual_segment_maps_stream(K[s0:s0 + L], V[s0:s0 + L], e_all[s0:s0 + L], C)
+        W = A @ W + B
+    O = np.empty((T, d))
+    for i, s0 in enumerate(range(0, T, L)):
+        O[s0:s0 + L], W_end = dual_form_stream(Q[s0:s0 + L], K[s0:s0 + L], V[s0:s0 + L],
+                                               e_all[s0:s0 + L], starts[i], C)
+    return O, W_end
 
 
 def dual_backward_stream(Q, K, V, eta, W0, dO, dW_out, C: int):

@@ -424,6 +424,48 @@ def test_assoc_backward_pins_catch_planted_mistakes():
         assert not (np.allclose(dK, ref[1], rtol=1e-6) and np.allclose(dV, ref[2], rtol=1e-6))
 
 
+# ----------------------------------------------------------------------------- segment-affine scan
+def test_dual_segment_maps_are_the_chunk_products_and_the_zero_start_run():
+    """A is the product of the chunk matrices I - K_c^T diag(eta_c) K_c (latest on the left),
+    formed here by a separate loop; B is the final state of the dual form started from W = 0;
+    and for any start W the segment ends at A W + B."""
+    T, d, C = 24, 5, 4
+    K, V = _rand(T, d, scale=0.5), _rand(T, d)
+    eta = rng.uniform(0.05, 0.6, T)
+    A, B = orc.dual_segment_maps_stream(K, V, eta, C)
+    P = np.eye(d)
+    for c0 in range(0, T, C):
+        k, e = K[c0:c0 + C], eta[c0:c0 + C]
+        P = (np.eye(d) - k.T @ np.diag(e) @ k) @ P
+    np.testing.assert_allclose(A, P, rtol=1e-12, atol=1e-13)
+    Q = _rand(T, d)
+    _, Wz = orc.dual_form_stream(Q, K, V, eta, None, C)
+    np.testing.assert_allclose(B, Wz, rtol=1e-12, atol=1e-13)
+    W0 = _rand(d, d)
+    _, W = orc.dual_form_stream(Q, K, V, eta, W0, C)
+    np.testing.assert_allclose(A @ W0 + B, W, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("T,d,C,L", [(32, 4, 4, 8), (48, 6, 8, 16), (30, 3, 3, 6), (16, 4, 16, 16)])
+def test_dual_segmented_equals_sequential(T, d, C, L):
+    """Segment-affine composition equals the sequential chunk loop (any segment length that is
+    a multiple of C), per-token and scalar rates, with and without W0."""
+    Q, K, V = _rand(T, d), _rand(T, d, scale=0.5), _rand(T, d)
+    for eta in (rng.uniform(0.05, 0.6, T), 0.3):
+        for W0 in (None, _rand(d, d)):
+            O, W = orc.dual_form_segmented_stream(Q, K, V, eta, W0, C, L)
+            O_ref, W_ref = orc.dual_form_stream(Q, K, V, eta, W0, C)
+            np.testing.assert_allclose(O, O_ref, rtol=1e-10, atol=1e-11)
+            np.testing.assert_allclose(W, W_ref, rtol=1e-10, atol=1e-11)
+
+
+def test_dual_segmented_rejects_bad_segment_lengths():
+    Q = K = V = np.zeros((16, 2))
+    for L in (0, 6, 32):   # not a positive multiple of C = 4 dividing T
+        with pytest.raises(ValueError):
+            orc.dual_form_segmented_stream(Q, K, V, 0.1, None, 4, L)
+
+
 # ----------------------------------------------------------------------------- dual-form backward
 def _dual_loss(Q, K, V, eta, W0, dO, G, C):
     """The scalar whose gradients the dual-form backward returns, from the forward only."""
