@@ -39,6 +39,7 @@ def metric_of(w) -> str:
 DEFAULT_WORKLOAD = "dual_bf16_B8H12T2048_d64C16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DOMINANT_KERNEL = {"dual": ("dual_mma_kernel", "dual_mma.cu"),
+                   "dual_seg": ("dual_mma_kernel", "dual_mma.cu"),
                    "assoc": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu"),
                    "assoc_bwd": ("assoc_chunk_kernel", "assoc_scan.cu"),
@@ -152,6 +153,16 @@ def make_call(w, x, stream_outputs=None):
         W = torch.empty((w.B, w.H, w.d, w.d), device=x["Q"].device, dtype=torch.float32)
         return lambda: ttt.ttt_linear_dual_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W0"], C=w.C,
                                                eta_scalar=x["eta_scalar"], O=O, W_out=W)
+    if w.kind == "dual_seg":
+        O = torch.empty_like(x["Q"])
+        W = torch.empty((w.B, w.H, w.d, w.d), device=x["Q"].device, dtype=torch.float32)
+        lib = ttt.load_library()
+        nbytes = lib.ttt_linear_dual_seg_workspace_size(w.B, w.H, w.T, w.d, w.C, 1, 0)
+        ws = torch.empty(max(nbytes, 16), device=x["Q"].device, dtype=torch.uint8)
+        return lambda: ttt.ttt_linear_dual_seg_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W0"],
+                                                   C=w.C, segments=0,
+                                                   eta_scalar=x["eta_scalar"], O=O, W_out=W,
+                                                   workspace=ws)
     if w.kind == "assoc":
         O = torch.empty_like(x["Q"])
         S = torch.empty((w.B, w.H, w.d, w.d), device=x["Q"].device, dtype=torch.float32)
@@ -276,7 +287,7 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
 
     threads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    if w.kind in ("dual", "assoc", "assoc_bwd", "assoc_momentum", "dual_bwd"):
+    if w.kind in ("dual", "dual_seg", "assoc", "assoc_bwd", "assoc_momentum", "dual_bwd"):
         streams = [(b, h) for b in range(w.B) for h in range(w.H)]
         Q, K, V = (x[k].float().cpu().numpy() for k in ("Q", "K", "V"))
         eta = None if x["eta"] is None else x["eta"].cpu().numpy()
@@ -287,12 +298,12 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
         # probe the cost of one chunk-run of one stream to size the sample
         tok = 0
         n_streams = 0
-        ncol = w.T if w.kind in ("dual", "dual_bwd") else min(w.T, 4096)
+        ncol = w.T if w.kind in ("dual", "dual_seg", "dual_bwd") else min(w.T, 4096)
         while True:
             b, h = streams[cursor[0] % len(streams)]
             cursor[0] += 1
             e = w.eta_const if eta is None else eta[b, h, :ncol]
-            if w.kind == "dual":
+            if w.kind in ("dual", "dual_seg"):
                 orc.dual_form_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
                                      W0[b, h], w.C)
             elif w.kind == "assoc_momentum":
@@ -312,7 +323,7 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
             if time.perf_counter() - t0 >= budget_s or n_streams >= len(streams):
                 break
         desc = (f"{n_streams} (b,h) stream(s) x {ncol} tokens of the workload, "
-                f"{ {'dual': 'dual-form per-chunk loop', 'assoc': 'sequential recurrence', 'assoc_momentum': 'momentum recurrence', 'dual_bwd': 'dual-form chunk adjoint sweeps'}.get(w.kind, 'adjoint sweeps of the recurrence')}"
+                f"{ {'dual': 'dual-form per-chunk loop', 'dual_seg': 'dual-form per-chunk loop', 'assoc': 'sequential recurrence', 'assoc_momentum': 'momentum recurrence', 'dual_bwd': 'dual-form chunk adjoint sweeps'}.get(w.kind, 'adjoint sweeps of the recurrence')}"
                 f", numpy fp64, 1 thread")
         return tok / w.H, time.perf_counter() - t0, 1, desc
     # In-Place: every 80th output column over all chunks (columns are independent)

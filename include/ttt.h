@@ -103,6 +103,28 @@ int ttt_linear_dual_fwd(const void* Q, const void* K, const void* V, const float
                         cudaStream_t stream);
 
 /* --------------------------------------------------------------------------------------------
+ * Sequence-parallel dual form (the segment-affine scan). Same operation, arguments, layouts
+ * and results as ttt_linear_dual_fwd, evaluated differently: without weight normalisation the
+ * chunk update W' = (I - K^T diag(eta) K) W + K^T diag(eta) V is affine in W ("KV 바인딩 기반
+ * 테스트 시간 학습은 사실상 선형 어텐션이다", associativity paragraph), so each stream is cut
+ * into `segments` segments of T / segments tokens whose maps W_end = A_s W_start + B_s are
+ * computed in parallel (two dual-form passes over the segments, from W = 0 and W = I), folded in
+ * order in fp32 to give every segment's start state, and a third pass produces O and W_out.
+ * Three passes of work over segments-times as many chains: for few streams (B*H well below
+ * the SM count) and long sequences.
+ *  segments: 0 picks the count (the most segments that keep B*H*segments chains within the SM
+ *  count, at least 4, else 1 = the sequential kernel); otherwise it must divide T / C.
+ *  Workspace: ttt_linear_dual_seg_workspace_size() bytes (5 fp32 d x d states per segment;
+ *  0 when the choice is 1). Returns TTT_ERR_INVALID_ARG when segments does not divide T / C.
+ * ------------------------------------------------------------------------------------------ */
+size_t ttt_linear_dual_seg_workspace_size(int B, int H, int T, int d, int C, int dt,
+                                          int segments);
+int ttt_linear_dual_seg_fwd(const void* Q, const void* K, const void* V, const float* eta,
+                            float eta_scalar, const float* W0, void* O, float* W_out, int B,
+                            int H, int T, int d, int C, int dt, int segments, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------------------------
  * Associative (gradient-ascent, weight-norm-free) linear-attention mode, per stream:
  *     S_t = S_(t-1) + eta_t k_t^T v_t,   o_t = q_t S_t      (S_0 = S0)
  *  computed per chunk of C tokens as O_c = Q_c S + (tril(Q_c K_c^T) diag(eta_c)) V_c,

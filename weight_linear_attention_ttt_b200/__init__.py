@@ -24,6 +24,7 @@ EXPORTED_SYMBOLS = (
     "ttt_status_string", "ttt_last_error_message", "ttt_version", "ttt_launch_count",
     "ttt_read_device_error",
     "ttt_linear_dual_workspace_size", "ttt_linear_dual_fwd",
+    "ttt_linear_dual_seg_workspace_size", "ttt_linear_dual_seg_fwd",
     "ttt_assoc_scan_workspace_size", "ttt_assoc_scan_fwd", "ttt_assoc_state_fwd",
     "ttt_assoc_scan_bwd_workspace_size", "ttt_assoc_scan_bwd",
     "ttt_linear_dual_bwd_workspace_size", "ttt_linear_dual_bwd",
@@ -81,6 +82,11 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         getattr(lib, name).restype = c_int
         getattr(lib, name).argtypes = [vp, vp, vp, fp, c_float, fp, vp, fp, vp, vp, vp, fp, fp,
                                        c_int, c_int, c_int, c_int, c_int, c_int, vp, c_size, vp]
+    lib.ttt_linear_dual_seg_workspace_size.restype = c_size
+    lib.ttt_linear_dual_seg_workspace_size.argtypes = [c_int] * 7
+    lib.ttt_linear_dual_seg_fwd.restype = c_int
+    lib.ttt_linear_dual_seg_fwd.argtypes = [vp, vp, vp, fp, c_float, fp, vp, fp, c_int, c_int,
+                                            c_int, c_int, c_int, c_int, c_int, vp, c_size, vp]
     lib.ttt_assoc_momentum_fwd.restype = c_int
     lib.ttt_assoc_momentum_fwd.argtypes = [vp, vp, vp, fp, c_float, c_float, fp, fp, vp, fp, fp,
                                            c_int, c_int, c_int, c_int, c_int, c_int, vp, c_size,
@@ -182,6 +188,41 @@ def ttt_linear_dual_fwd(Q, K, V, eta=None, W0=None, *, C: int, eta_scalar: float
     """TTT-Linear mini-batch dual form. Returns (O, W_out); see include/ttt.h."""
     return _state_call("ttt_linear_dual_fwd", "ttt_linear_dual_workspace_size", Q, K, V, eta,
                        eta_scalar, W0, C, O, W_out, workspace, stream)
+
+
+def ttt_linear_dual_seg_fwd(Q, K, V, eta=None, W0=None, *, C: int, segments: int = 0,
+                            eta_scalar: float = 0.0, O=None, W_out=None, workspace=None,
+                            stream=None) -> Tuple:
+    """The dual form evaluated sequence-parallel (segment-affine scan); same results as
+    ttt_linear_dual_fwd. segments = 0 picks the count. Returns (O, W_out); see include/ttt.h."""
+    import torch
+
+    lib = load_library()
+    _require(Q.dim() == 4, "Q, K, V must be [B, H, T, d]")
+    B, H, T, d = Q.shape
+    for t in (Q, K, V):
+        _require(t.is_cuda and t.is_contiguous() and t.shape == Q.shape and t.dtype == Q.dtype,
+                 "Q, K, V must be contiguous CUDA tensors of one shape and dtype")
+    dt = _dtype_code(Q)
+    if eta is not None:
+        _require(eta.is_cuda and eta.dtype == torch.float32 and eta.is_contiguous() and
+                 tuple(eta.shape) == (B, H, T), "eta must be a contiguous fp32 [B, H, T] tensor")
+    if W0 is not None:
+        _require(W0.is_cuda and W0.dtype == torch.float32 and W0.is_contiguous() and
+                 tuple(W0.shape) == (B, H, d, d), "initial state must be fp32 [B, H, d, d]")
+    O = torch.empty_like(Q) if O is None else O
+    if W_out is None:
+        W_out = torch.empty((B, H, d, d), device=Q.device, dtype=torch.float32)
+    ws_bytes = lib.ttt_linear_dual_seg_workspace_size(B, H, T, d, C, dt, segments)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, device=Q.device, dtype=torch.uint8)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.ttt_linear_dual_seg_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta),
+                                     ctypes.c_float(eta_scalar), _ptr(W0), _ptr(O), _ptr(W_out),
+                                     B, H, T, d, C, dt, segments, _ptr(workspace), wsz,
+                                     _stream_ptr(stream))
+    _check("ttt_linear_dual_seg_fwd", st)
+    return O, W_out
 
 
 def ttt_assoc_scan_fwd(Q, K, V, eta=None, S0=None, *, C: int, eta_scalar: float = 0.0,

@@ -104,6 +104,11 @@ struct AssocBwdArgs {
   size_t ws_bytes;
 };
 int launch_assoc_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx);
+// Sequence-parallel dual form (segment-affine scan over the dual-form kernels). segments: the
+// caller's count (must divide T / C) or 0 for the automatic choice; returns -1 if invalid.
+int dual_seg_choose_segments(int B, int H, int T, int C, int requested);
+size_t dual_seg_workspace_bytes(int B, int H, int d, int S);
+int launch_dual_seg(const StateArgs& a, int S, const LaunchCtx& ctx);
 // Dual-form backward (one kernel; S0 / dS_out / dS0 of the arguments are W0 / dW_out / dW0; the
 // workspace holds one bf16 d x d checkpoint per chunk).
 bool dual_bwd_supported(int d, int C, int dt);

@@ -197,6 +197,46 @@ int ttt_linear_dual_fwd(const void* Q, const void* K, const void* V, const float
   return finish(st, msg);
 }
 
+size_t ttt_linear_dual_seg_workspace_size(int B, int H, int T, int d, int C, int dt,
+                                          int segments) {
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0 || segments < 0) return 0;
+  (void)dt;
+  const int S = dual_seg_choose_segments(B, H, T, C, segments);
+  return S < 1 ? 0 : dual_seg_workspace_bytes(B, H, d, S);
+}
+
+int ttt_linear_dual_seg_fwd(const void* Q, const void* K, const void* V, const float* eta,
+                            float eta_scalar, const float* W0, void* O, float* W_out, int B,
+                            int H, int T, int d, int C, int dt, int segments, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream) {
+  const char* fn = "ttt_linear_dual_seg_fwd";
+  StateArgs a{Q, K, V, eta, eta_scalar, W0, O, W_out, B, H, T, d, C, dt, workspace,
+              workspace_bytes};
+  int st = check_state_args(fn, a, 0);
+  if (st != TTT_OK) return st;
+  if (!(d == 32 || d == 64 || d == 128) || C > 64)
+    return fail(TTT_ERR_UNSUPPORTED, std::string(fn) + ": supported d in {32, 64, 128} and "
+                                                       "1 <= C <= 64");
+  if (segments < 0) return fail(TTT_ERR_INVALID_ARG, std::string(fn) + ": segments must be >= 0");
+  const int S = dual_seg_choose_segments(B, H, T, C, segments);
+  if (S < 1)
+    return fail(TTT_ERR_INVALID_ARG,
+                std::string(fn) + ": segments must divide the number of chunks T / C");
+  const size_t need = dual_seg_workspace_bytes(B, H, d, S);
+  st = check_state_args(fn, a, need);
+  if (st != TTT_OK) return st;
+  if (need && overlap(workspace, workspace_bytes, O, (size_t)B * H * T * d * (dt ? 2 : 4)))
+    return fail(TTT_ERR_INVALID_ARG, std::string(fn) + ": workspace overlaps O");
+  if (need && (overlap(workspace, workspace_bytes, W_out, (size_t)B * H * d * d * 4) ||
+               overlap(workspace, workspace_bytes, W0, (size_t)B * H * d * d * 4)))
+    return fail(TTT_ERR_INVALID_ARG, std::string(fn) + ": workspace overlaps a state");
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  return finish(launch_dual_seg(a, S, ctx), msg);
+}
+
 size_t ttt_assoc_scan_workspace_size(int B, int H, int T, int d, int C, int dt) {
   if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || !assoc_supported(d, C, dt)) return 0;
   return assoc_workspace_bytes(B, H, T, d, C);

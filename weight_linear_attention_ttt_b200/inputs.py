@@ -80,6 +80,12 @@ WORKLOADS = {
     "inplace_lm_bf16_T32768_Dff9728_D2560_Dm2560_C1024": Workload(
         "inplace_lm_bf16_T32768_Dff9728_D2560_Dm2560_C1024", "inplace_lm", 1008, T=32768,
         C=1024, Dff=9728, D=2560, Dm=2560, k=4, eta="const", eta_const=1e-3),
+    "dual_bf16_B1H4T262144_d64C16": Workload(
+        "dual_bf16_B1H4T262144_d64C16", "dual", 1010, B=1, H=4, T=262144, d=64, C=16,
+        normalise=("K", "V")),
+    "dual_seg_bf16_B1H4T262144_d64C16": Workload(
+        "dual_seg_bf16_B1H4T262144_d64C16", "dual_seg", 1010, B=1, H=4, T=262144, d=64, C=16,
+        normalise=("K", "V")),
     "dual_bwd_bf16_B8H12T2048_d64C16": Workload(
         "dual_bwd_bf16_B8H12T2048_d64C16", "dual_bwd", 1006, B=8, H=12, T=2048, d=64, C=16,
         normalise=("K", "V")),
@@ -207,7 +213,7 @@ def make_inputs(w: Workload, device="cpu", *, seed: Optional[int] = None, **over
     if overrides:
         w = dataclasses.replace(w, **overrides)
     s = w.seed if seed is None else seed
-    if w.kind in ("dual", "assoc", "assoc_momentum"):
+    if w.kind in ("dual", "dual_seg", "assoc", "assoc_momentum"):
         return dual_or_assoc_inputs(w.B, w.H, w.T, w.d, seed=s, device=device, dtype=w.dtype,
                                     qkv=w.qkv, normalise=w.normalise, eta=w.eta,
                                     eta_const=w.eta_const, w0=w.w0)

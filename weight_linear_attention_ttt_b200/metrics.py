@@ -30,6 +30,9 @@ def algorithmic(w: Workload) -> dict:
         a = algorithmic(dataclasses.replace(w, kind="assoc"))
         return {"flops": 2 * a["flops"], "bytes": a["bytes"] + w.B * w.H * 2 * w.d * w.d * 4,
                 "tokens": a["tokens"]}
+    if w.kind == "dual_seg":
+        # the same operation as the dual form; the two extra passes are overhead
+        return algorithmic(dataclasses.replace(w, kind="dual"))
     if w.kind in ("dual", "assoc"):
         e = 4 if w.dtype == "f32" else 2
         th = w.B * w.H * w.T
