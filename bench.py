@@ -44,6 +44,7 @@ DOMINANT_KERNEL = {"dual": ("dual_mma_kernel", "dual_mma.cu"),
                    "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu"),
                    "assoc_bwd": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "dual_bwd": ("dual_bwd_kernel", "dual_bwd.cu"),
+                   "dual_seg_bwd": ("dual_bwd_kernel", "dual_bwd.cu"),
                    "assoc_momentum": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "inplace_lm": ("inplace_chunk_kernel", "inplace_ttt.cu")}
 
@@ -196,6 +197,19 @@ def make_call(w, x, stream_outputs=None):
         return lambda: ttt.ttt_assoc_scan_bwd(x["Q"], x["K"], x["V"], x["eta"], None, x["dO"],
                                               x["dS_out"], C=w.C, eta_scalar=x["eta_scalar"],
                                               workspace=ws, **outs)
+    if w.kind == "dual_seg_bwd":
+        dev = x["Q"].device
+        outs = dict(dQ=torch.empty_like(x["Q"]), dK=torch.empty_like(x["Q"]),
+                    dV=torch.empty_like(x["Q"]),
+                    deta=torch.empty((w.B, w.H, w.T), device=dev, dtype=torch.float32),
+                    dW0=torch.empty((w.B, w.H, w.d, w.d), device=dev, dtype=torch.float32))
+        lib = ttt.load_library()
+        nbytes = lib.ttt_linear_dual_seg_bwd_workspace_size(w.B, w.H, w.T, w.d, w.C, 1, 0)
+        ws = torch.empty(max(nbytes, 16), device=dev, dtype=torch.uint8)
+        return lambda: ttt.ttt_linear_dual_seg_bwd(x["Q"], x["K"], x["V"], x["eta"], x["W0"],
+                                                   x["dO"], x["dW_out"], C=w.C, segments=0,
+                                                   eta_scalar=x["eta_scalar"], workspace=ws,
+                                                   **outs)
     if w.kind == "dual_bwd":
         dev = x["Q"].device
         outs = dict(dQ=torch.empty_like(x["Q"]), dK=torch.empty_like(x["Q"]),
@@ -242,7 +256,7 @@ def e2e_measure(w, x, steps: int, warmup: int):
     elif w.kind == "assoc_momentum":
         out_shapes = [((w.B, w.H, w.T, w.d), x["Q"].dtype), ((w.B, w.H, w.d, w.d), torch.float32),
                       ((w.B, w.H, w.d, w.d), torch.float32)]
-    elif w.kind in ("assoc_bwd", "dual_bwd"):
+    elif w.kind in ("assoc_bwd", "dual_bwd", "dual_seg_bwd"):
         out_shapes = [((w.B, w.H, w.T, w.d), x["Q"].dtype)] * 3 + [
             ((w.B, w.H, w.T), torch.float32), ((w.B, w.H, w.d, w.d), torch.float32)]
     else:
@@ -287,18 +301,19 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
 
     threads = os.cpu_count() or 1
     t0 = time.perf_counter()
-    if w.kind in ("dual", "dual_seg", "assoc", "assoc_bwd", "assoc_momentum", "dual_bwd"):
+    if w.kind in ("dual", "dual_seg", "assoc", "assoc_bwd", "assoc_momentum", "dual_bwd",
+                  "dual_seg_bwd"):
         streams = [(b, h) for b in range(w.B) for h in range(w.H)]
         Q, K, V = (x[k].float().cpu().numpy() for k in ("Q", "K", "V"))
         eta = None if x["eta"] is None else x["eta"].cpu().numpy()
         W0 = x["W0"].cpu().numpy()
-        if w.kind in ("assoc_bwd", "dual_bwd"):
+        if w.kind in ("assoc_bwd", "dual_bwd", "dual_seg_bwd"):
             dO = x["dO"].float().cpu().numpy()
             G = x["dS_out" if w.kind == "assoc_bwd" else "dW_out"].cpu().numpy()
         # probe the cost of one chunk-run of one stream to size the sample
         tok = 0
         n_streams = 0
-        ncol = w.T if w.kind in ("dual", "dual_seg", "dual_bwd") else min(w.T, 4096)
+        ncol = w.T if w.kind in ("dual", "dual_seg", "dual_bwd", "dual_seg_bwd") else min(w.T, 4096)
         while True:
             b, h = streams[cursor[0] % len(streams)]
             cursor[0] += 1
@@ -309,7 +324,7 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
             elif w.kind == "assoc_momentum":
                 orc.assoc_momentum_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
                                           inp.MOMENTUM_BETA, None, None)
-            elif w.kind == "dual_bwd":
+            elif w.kind in ("dual_bwd", "dual_seg_bwd"):
                 orc.dual_backward_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
                                          W0[b, h], dO[b, h, :ncol], G[b, h], w.C)
             elif w.kind == "assoc_bwd":
@@ -323,7 +338,7 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
             if time.perf_counter() - t0 >= budget_s or n_streams >= len(streams):
                 break
         desc = (f"{n_streams} (b,h) stream(s) x {ncol} tokens of the workload, "
-                f"{ {'dual': 'dual-form per-chunk loop', 'dual_seg': 'dual-form per-chunk loop', 'assoc': 'sequential recurrence', 'assoc_momentum': 'momentum recurrence', 'dual_bwd': 'dual-form chunk adjoint sweeps'}.get(w.kind, 'adjoint sweeps of the recurrence')}"
+                f"{ {'dual': 'dual-form per-chunk loop', 'dual_seg': 'dual-form per-chunk loop', 'assoc': 'sequential recurrence', 'assoc_momentum': 'momentum recurrence', 'dual_bwd': 'dual-form chunk adjoint sweeps', 'dual_seg_bwd': 'dual-form chunk adjoint sweeps'}.get(w.kind, 'adjoint sweeps of the recurrence')}"
                 f", numpy fp64, 1 thread")
         return tok / w.H, time.perf_counter() - t0, 1, desc
     # In-Place: every 80th output column over all chunks (columns are independent)

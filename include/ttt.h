@@ -217,6 +217,27 @@ int ttt_linear_dual_bwd(const void* Q, const void* K, const void* V, const float
                         cudaStream_t stream);
 
 /* --------------------------------------------------------------------------------------------
+ * Backward of the sequence-parallel dual form: the gradients of ttt_linear_dual_bwd (same
+ * arguments, layouts, results up to rounding, support and errors) evaluated over `segments`
+ * segments per stream. The state gradient X follows its own affine recurrence, in reverse and
+ * free of W: X_before = (I - K^T diag(eta) K) X_after + Q^T dO - K^T A^T dO per chunk, so a
+ * segment maps X_before = A_s^T X_after + N_s with the forward's A_s. The library computes the
+ * forward maps and segment start states (as ttt_linear_dual_seg_fwd), the offsets N_s (a
+ * backward pass over the segments from X_after = 0), every segment's X_after (a reverse fold),
+ * and then the gradients (a second backward pass over the segments).
+ *  segments: 0 picks the count as ttt_linear_dual_seg_fwd does (1 = ttt_linear_dual_bwd);
+ *  otherwise it must divide T / C (else TTT_ERR_INVALID_ARG).
+ *  Workspace: ttt_linear_dual_seg_bwd_workspace_size() bytes.
+ * ------------------------------------------------------------------------------------------ */
+size_t ttt_linear_dual_seg_bwd_workspace_size(int B, int H, int T, int d, int C, int dt,
+                                              int segments);
+int ttt_linear_dual_seg_bwd(const void* Q, const void* K, const void* V, const float* eta,
+                            float eta_scalar, const float* W0, const void* dO,
+                            const float* dW_out, void* dQ, void* dK, void* dV, float* deta,
+                            float* dW0, int B, int H, int T, int d, int C, int dt, int segments,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------------------------
  * State increment of a sequence slice in the associative mode (the first pass of the prefix
  * scan over states, "KV 바인딩 기반 테스트 시간 학습은 사실상 선형 어텐션이다", associativity
  * paragraph; per-chunk deltas combined by a prefix sum for context parallelism, "In-Place

@@ -96,3 +96,68 @@ def test_errors(cuda_lib):
     with pytest.raises(ttt.TTTError) as e:
         run(x, 16, 4, workspace=torch.empty(16, device="cuda", dtype=torch.uint8))
     assert e.value.status == 3
+
+
+def _bwd_case(B, H, T, d, seed, eta="sigmoid"):
+    x = inp.dual_or_assoc_inputs(B, H, T, d, seed=seed, device="cuda", normalise=("K", "V"),
+                                 eta=eta, eta_const=0.3)
+    g = torch.Generator("cuda").manual_seed(seed + 1)
+    x["dO"] = torch.randn(B, H, T, d, device="cuda", generator=g).to(torch.bfloat16)
+    x["dW_out"] = torch.randn(B, H, d, d, device="cuda", generator=g) * 0.05
+    return x
+
+
+def check_bwd(x, got, streams=None):
+    eta = x["eta_scalar"] if x["eta"] is None else x["eta"].cpu().numpy()
+    f = lambda t: None if t is None else t.float().cpu().numpy()
+    ref = orc.dual_form_bwd(f(x["Q"]), f(x["K"]), f(x["V"]), eta, f(x["W0"]), f(x["dO"]),
+                            f(x["dW_out"]), 16, threads=os.cpu_count() or 4, streams=streams)
+    errs = []
+    for name, g, r in zip(("dQ", "dK", "dV", "deta", "dW0"), got, ref):
+        if streams is not None:
+            g = torch.stack([g[b, h] for b, h in streams])
+        e = max_rel_l2(g, r, 1 if streams is not None else 2)
+        errs.append(e)
+        assert e <= 1e-2, (name, e)
+    return errs
+
+
+def run_bwd(x, segments, **kw):
+    return ttt.ttt_linear_dual_seg_bwd(x["Q"], x["K"], x["V"], x["eta"], x["W0"], x["dO"],
+                                       x["dW_out"], C=16, segments=segments,
+                                       eta_scalar=x["eta_scalar"], **kw)
+
+
+@pytest.mark.parametrize("B,H,T,d,S", [(1, 1, 1024, 64, 4), (1, 2, 2048, 64, 8),
+                                       (2, 1, 1024, 64, 0), (1, 2, 1024, 32, 16),
+                                       (1, 1, 512, 128, 4)])
+def test_backward_against_the_sequential_oracle(cuda_lib, B, H, T, d, S):
+    x = _bwd_case(B, H, T, d, seed=T + d + S + 3)
+    check_bwd(x, run_bwd(x, S))
+    assert ttt.read_device_error() == 0
+
+
+def test_backward_scalar_rate_and_zero_states(cuda_lib):
+    x = _bwd_case(1, 2, 1024, 64, seed=31, eta="const")
+    x["W0"], x["dW_out"] = None, None
+    check_bwd(x, run_bwd(x, 8))
+
+
+def test_backward_few_streams_long_sequence(cuda_lib):
+    """B=1, H=4, T=262144, d=64: every stream against the sequential oracle backward."""
+    w = inp.WORKLOADS["dual_seg_bwd_bf16_B1H4T262144_d64C16"]
+    x = inp.make_inputs(w, "cuda")
+    errs = check_bwd(x, run_bwd(x, 0))
+    print("segmented dual backward, B1 H4 T262144 (all streams): max rel L2 dQ %.2e dK %.2e "
+          "dV %.2e deta %.2e dW0 %.2e" % tuple(errs))
+    assert ttt.read_device_error() == 0
+
+
+def test_backward_errors(cuda_lib):
+    x = _bwd_case(1, 1, 1024, 64, seed=2)
+    with pytest.raises(ttt.TTTError) as e:     # 3 does not divide the 64 chunks
+        run_bwd(x, 3)
+    assert e.value.status == 1
+    with pytest.raises(ttt.TTTError) as e:
+        run_bwd(x, 4, workspace=torch.empty(16, device="cuda", dtype=torch.uint8))
+    assert e.value.status == 3

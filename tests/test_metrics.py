@@ -15,6 +15,8 @@ from weight_linear_attention_ttt_b200.shard import split_range
     ("dual_bwd_bf16_B8H12T2048_d64C16", 13.287e9, 182.45, "hbm"),
     ("dual_bf16_B1H4T262144_d64C16", 30.065e9, 541.2, "hbm"),
     ("dual_seg_bf16_B1H4T262144_d64C16", 30.065e9, 541.2, "hbm"),
+    ("dual_bwd_bf16_B1H4T262144_d64C16", 70.867e9, 948.1, "hbm"),
+    ("dual_seg_bwd_bf16_B1H4T262144_d64C16", 70.867e9, 948.1, "hbm"),
     ("assoc_momentum_bf16_B4H16T65536_d128C64", 824.6e9, 4328.5, "hbm"),
     ("inplace_lm_bf16_T32768_Dff9728_D2560_Dm2560_C1024", 3.6943e12, 1135.6, "tensor"),
 ])

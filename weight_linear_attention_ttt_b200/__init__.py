@@ -28,6 +28,7 @@ EXPORTED_SYMBOLS = (
     "ttt_assoc_scan_workspace_size", "ttt_assoc_scan_fwd", "ttt_assoc_state_fwd",
     "ttt_assoc_scan_bwd_workspace_size", "ttt_assoc_scan_bwd",
     "ttt_linear_dual_bwd_workspace_size", "ttt_linear_dual_bwd",
+    "ttt_linear_dual_seg_bwd_workspace_size", "ttt_linear_dual_seg_bwd",
     "ttt_assoc_momentum_workspace_size", "ttt_assoc_momentum_fwd",
     "ttt_state_prefix_sum",
     "inplace_ttt_workspace_size", "inplace_ttt_chunk_fwd",
@@ -82,6 +83,12 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         getattr(lib, name).restype = c_int
         getattr(lib, name).argtypes = [vp, vp, vp, fp, c_float, fp, vp, fp, vp, vp, vp, fp, fp,
                                        c_int, c_int, c_int, c_int, c_int, c_int, vp, c_size, vp]
+    lib.ttt_linear_dual_seg_bwd_workspace_size.restype = c_size
+    lib.ttt_linear_dual_seg_bwd_workspace_size.argtypes = [c_int] * 7
+    lib.ttt_linear_dual_seg_bwd.restype = c_int
+    lib.ttt_linear_dual_seg_bwd.argtypes = [vp, vp, vp, fp, c_float, fp, vp, fp, vp, vp, vp, fp,
+                                            fp, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
+                                            vp, c_size, vp]
     lib.ttt_linear_dual_seg_workspace_size.restype = c_size
     lib.ttt_linear_dual_seg_workspace_size.argtypes = [c_int] * 7
     lib.ttt_linear_dual_seg_fwd.restype = c_int
@@ -311,6 +318,47 @@ def ttt_linear_dual_bwd(Q, K, V, eta, W0, dO, dW_out=None, *, C: int, eta_scalar
                                  _ptr(deta), _ptr(dW0), B, H, T, d, C, dt, _ptr(workspace), wsz,
                                  _stream_ptr(stream))
     _check("ttt_linear_dual_bwd", st)
+    return dQ, dK, dV, deta, dW0
+
+
+def ttt_linear_dual_seg_bwd(Q, K, V, eta, W0, dO, dW_out=None, *, C: int, segments: int = 0,
+                            eta_scalar: float = 0.0, dQ=None, dK=None, dV=None, deta=None,
+                            dW0=None, workspace=None, stream=None) -> Tuple:
+    """ttt_linear_dual_bwd evaluated over segments of each stream (segments = 0 picks the
+    count). Returns (dQ, dK, dV, deta, dW0)."""
+    import torch
+
+    lib = load_library()
+    _require(Q.dim() == 4, "Q, K, V, dO must be [B, H, T, d]")
+    B, H, T, d = Q.shape
+    for t in (Q, K, V, dO):
+        _require(t.is_cuda and t.is_contiguous() and t.shape == Q.shape and t.dtype == Q.dtype,
+                 "Q, K, V, dO must be contiguous CUDA tensors of one shape and dtype")
+    dt = _dtype_code(Q)
+    if eta is not None:
+        _require(eta.is_cuda and eta.dtype == torch.float32 and eta.is_contiguous() and
+                 tuple(eta.shape) == (B, H, T), "eta must be a contiguous fp32 [B, H, T] tensor")
+    for t in (W0, dW_out):
+        if t is not None:
+            _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous() and
+                     tuple(t.shape) == (B, H, d, d), "states must be fp32 [B, H, d, d]")
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(Q) if dK is None else dK
+    dV = torch.empty_like(Q) if dV is None else dV
+    if deta is None:
+        deta = torch.empty((B, H, T), device=Q.device, dtype=torch.float32)
+    if dW0 is None:
+        dW0 = torch.empty((B, H, d, d), device=Q.device, dtype=torch.float32)
+    ws_bytes = lib.ttt_linear_dual_seg_bwd_workspace_size(B, H, T, d, C, dt, segments)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, device=Q.device, dtype=torch.uint8)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.ttt_linear_dual_seg_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(eta),
+                                     ctypes.c_float(eta_scalar), _ptr(W0), _ptr(dO),
+                                     _ptr(dW_out), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta),
+                                     _ptr(dW0), B, H, T, d, C, dt, segments, _ptr(workspace),
+                                     wsz, _stream_ptr(stream))
+    _check("ttt_linear_dual_seg_bwd", st)
     return dQ, dK, dV, deta, dW0
 
 

@@ -14,7 +14,10 @@
 //   4. every segment run from W_start(s), writing O; the last segment's end state is W_out.
 // Passes 1 and 2 write O as scratch (pass 4 overwrites it). The work is three dual-form passes
 // instead of one, spread over S times as many chains: it pays when B*H leaves most SMs idle.
+// The backward (launch_dual_seg_bwd) reuses the maps and the start states and folds the state
+// gradient's own affine recurrence in reverse.
 #include <algorithm>
+#include <string>
 
 #include "internal.h"
 
@@ -67,13 +70,53 @@ __global__ void __launch_bounds__(256) fold_segments_kernel(const float* __restr
   }
 }
 
-__global__ void last_segment_state_kernel(const float* __restrict__ Wend, float* W_out, int S,
-                                          int d, size_t bh_count) {
+// Backward of the segment-affine evaluation: the state gradient X obeys
+// X_before = (I - K^T diag(eta) K) X_after + Q^T dO - K^T A^T dO per chunk (no W in it), so a
+// segment maps X_before = A_s^T X_after + N_s (each chunk factor is symmetric, so the segment's
+// factor is the transpose of the forward's A_s). One CTA per stream, in reverse segment order:
+// segment s stores its X_after, then X <- A_s^T X + N_s.
+template <int D>
+__global__ void __launch_bounds__(256) fold_segments_reverse_kernel(
+    const float* __restrict__ dW_out, const float* __restrict__ Bm, const float* __restrict__ ABm,
+    const float* __restrict__ Noff, float* __restrict__ Xafter, int S) {
+  constexpr int E = D * D / 256;
+  extern __shared__ float fsm[];
+  float* X = fsm;                  // [D][D]
+  float* A = fsm + D * D;          // [D][D] = A_s
+  const size_t bh = blockIdx.x;
+  for (int i = threadIdx.x; i < D * D; i += 256) X[i] = dW_out ? dW_out[bh * D * D + i] : 0.f;
+  __syncthreads();
+  for (int s = S - 1; s >= 0; --s) {
+    const size_t seg = (bh * S + s) * D * D;
+    for (int i = threadIdx.x; i < D * D; i += 256) {
+      Xafter[seg + i] = X[i];
+      A[i] = ABm[seg + i] - Bm[seg + i];
+    }
+    __syncthreads();
+    float out[E];
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+      const int idx = threadIdx.x + 256 * q, i = idx / D, j = idx % D;
+      float acc = Noff[seg + idx];
+#pragma unroll 8
+      for (int k = 0; k < D; ++k) acc = fmaf(A[k * D + i], X[k * D + j], acc);   // (A^T X)[i][j]
+      out[q] = acc;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < E; ++q) X[threadIdx.x + 256 * q] = out[q];
+    __syncthreads();
+  }
+}
+
+// dst[bh] = src[bh * S + s_pick] for bh_count d x d fp32 states
+__global__ void pick_segment_state_kernel(const float* __restrict__ src, float* dst, int S,
+                                          int s_pick, int d, size_t bh_count) {
   const size_t per = (size_t)d * d, total = bh_count * per;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (size_t)gridDim.x * blockDim.x) {
     const size_t bh = i / per, e = i % per;
-    W_out[i] = Wend[(bh * S + (S - 1)) * per + e];
+    dst[i] = src[(bh * S + s_pick) * per + e];
   }
 }
 
@@ -104,32 +147,103 @@ size_t dual_seg_workspace_bytes(int B, int H, int d, int S) {
   return 5 * (size_t)B * H * S * d * d * sizeof(float);
 }
 
+namespace {
+
+int run_dual(const StateArgs& x, const LaunchCtx& ctx) {
+  return dual_mma_supported(x.d, x.C, x.dt) ? launch_dual_mma(x, ctx) : launch_dual_simt(x, ctx);
+}
+
+int check_launch(const LaunchCtx& ctx, const char* what, cudaError_t e = cudaSuccess) {
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e == cudaSuccess) return kOk;
+  *ctx.msg = std::string("dual seg ") + what + ": " + cudaGetErrorString(e);
+  return kCuda;
+}
+
+// Per-stream fold over the segments, forward (start states) or reverse (state gradients).
+int launch_fold(bool reverse, int d, int bh, const float* init, const float* Bm,
+                const float* ABm, const float* Noff, float* dst, int S, const LaunchCtx& ctx) {
+  const size_t smem = 2 * (size_t)d * d * sizeof(float);
+  cudaError_t e = cudaSuccess;
+  switch (d) {
+    case 32:
+      if (reverse)
+        fold_segments_reverse_kernel<32><<<bh, 256, smem, ctx.stream>>>(init, Bm, ABm, Noff, dst, S);
+      else
+        fold_segments_kernel<32><<<bh, 256, smem, ctx.stream>>>(init, Bm, ABm, dst, S);
+      break;
+    case 64:
+      if (reverse)
+        fold_segments_reverse_kernel<64><<<bh, 256, smem, ctx.stream>>>(init, Bm, ABm, Noff, dst, S);
+      else
+        fold_segments_kernel<64><<<bh, 256, smem, ctx.stream>>>(init, Bm, ABm, dst, S);
+      break;
+    case 128:
+      if (reverse) {
+        e = cudaFuncSetAttribute(fold_segments_reverse_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess)
+          fold_segments_reverse_kernel<128><<<bh, 256, smem, ctx.stream>>>(init, Bm, ABm, Noff,
+                                                                           dst, S);
+      } else {
+        e = cudaFuncSetAttribute(fold_segments_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess)
+          fold_segments_kernel<128><<<bh, 256, smem, ctx.stream>>>(init, Bm, ABm, dst, S);
+      }
+      break;
+    default:
+      *ctx.msg = "dual seg: unsupported head dim";
+      return kUnsupported;
+  }
+  count_launch();
+  return check_launch(ctx, "fold launch", e);
+}
+
+// Steps 1-3: the segment maps (B_s from W = 0, A_s + B_s from W = I) and the fold giving every
+// segment's start state Wst. `v` is the segment view; the maps' outputs go to `Ojunk`.
+int maps_and_fold(const StateArgs& v, int S, int bh, const float* W0, void* Ojunk, float* Wid,
+                  float* Bm, float* ABm, float* Wst, const LaunchCtx& ctx) {
+  const size_t n = (size_t)v.B;
+  identity_states_kernel<<<sm_count() * 4, 256, 0, ctx.stream>>>(Wid, n, v.d);
+  count_launch();
+  int st = check_launch(ctx, "identity launch");
+  if (st != kOk) return st;
+  StateArgs pb = v;
+  pb.S0 = nullptr;
+  pb.O = Ojunk;
+  pb.S_out = Bm;
+  if ((st = run_dual(pb, ctx)) != kOk) return st;
+  StateArgs pa = v;
+  pa.S0 = Wid;
+  pa.O = Ojunk;
+  pa.S_out = ABm;
+  if ((st = run_dual(pa, ctx)) != kOk) return st;
+  return launch_fold(false, v.d, bh, W0, Bm, ABm, nullptr, Wst, S, ctx);
+}
+
+int pick(const float* src, float* dst, int S, int s_pick, int d, int bh, const LaunchCtx& ctx) {
+  pick_segment_state_kernel<<<sm_count() * 2, 256, 0, ctx.stream>>>(src, dst, S, s_pick, d,
+                                                                     (size_t)bh);
+  count_launch();
+  return check_launch(ctx, "state launch");
+}
+
+}  // namespace
+
 int launch_dual_seg(const StateArgs& a, int S, const LaunchCtx& ctx) {
-  auto run = [&](const StateArgs& x) {
-    return dual_mma_supported(x.d, x.C, x.dt) ? launch_dual_mma(x, ctx) : launch_dual_simt(x, ctx);
-  };
-  if (S <= 1) return run(a);
+  if (S <= 1) return run_dual(a, ctx);
   const int d = a.d, bh = a.B * a.H;
   const size_t n = (size_t)bh * S, per = (size_t)d * d;
   if (a.ws_bytes < dual_seg_workspace_bytes(a.B, a.H, d, S)) {
     *ctx.msg = "ttt_linear_dual_seg_fwd: workspace smaller than ttt_linear_dual_seg_workspace_size()";
     return kWorkspace;
   }
-  float* ws = static_cast<float*>(a.ws);
-  float* Wid = ws;
+  float* Wid = static_cast<float*>(a.ws);
   float* Bm = Wid + n * per;
   float* ABm = Bm + n * per;
   float* Wst = ABm + n * per;
   float* Wend = Wst + n * per;
-  const int sms = sm_count();
-
-  identity_states_kernel<<<sms * 4, 256, 0, ctx.stream>>>(Wid, n, d);
-  count_launch();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    *ctx.msg = std::string("dual seg identity launch: ") + cudaGetErrorString(e);
-    return kCuda;
-  }
   // segments as independent streams: [B*H*S, 1, T/S, d]
   StateArgs v = a;
   v.B = (int)n;
@@ -137,51 +251,63 @@ int launch_dual_seg(const StateArgs& a, int S, const LaunchCtx& ctx) {
   v.T = a.T / S;
   v.ws = nullptr;
   v.ws_bytes = 0;
-  StateArgs pb = v;   // 1. from W = 0
-  pb.S0 = nullptr;
-  pb.S_out = Bm;
-  int st = run(pb);
+  int st = maps_and_fold(v, S, bh, a.S0, a.O, Wid, Bm, ABm, Wst, ctx);
   if (st != kOk) return st;
-  StateArgs pa = v;   // 2. from W = I
-  pa.S0 = Wid;
-  pa.S_out = ABm;
-  st = run(pa);
-  if (st != kOk) return st;
-  // 3. fold
-  const size_t smem = 2 * per * sizeof(float);
-  if (d == 32) {
-    fold_segments_kernel<32><<<bh, 256, smem, ctx.stream>>>(a.S0, Bm, ABm, Wst, S);
-  } else if (d == 64) {
-    fold_segments_kernel<64><<<bh, 256, smem, ctx.stream>>>(a.S0, Bm, ABm, Wst, S);
-  } else if (d == 128) {
-    e = cudaFuncSetAttribute(fold_segments_kernel<128>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-      fold_segments_kernel<128><<<bh, 256, smem, ctx.stream>>>(a.S0, Bm, ABm, Wst, S);
-  } else {
-    *ctx.msg = "ttt_linear_dual_seg_fwd: unsupported head dim";
-    return kUnsupported;
-  }
-  count_launch();
-  if (e == cudaSuccess) e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    *ctx.msg = std::string("dual seg fold launch: ") + cudaGetErrorString(e);
-    return kCuda;
-  }
-  // 4. outputs from the true segment starts
+  // 4. outputs from the true segment starts; the last segment's end state is W_out
   StateArgs po = v;
   po.S0 = Wst;
   po.S_out = Wend;
-  st = run(po);
-  if (st != kOk) return st;
-  last_segment_state_kernel<<<sms * 2, 256, 0, ctx.stream>>>(Wend, a.S_out, S, d, (size_t)bh);
-  count_launch();
-  e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    *ctx.msg = std::string("dual seg state launch: ") + cudaGetErrorString(e);
-    return kCuda;
+  if ((st = run_dual(po, ctx)) != kOk) return st;
+  return pick(Wend, a.S_out, S, S - 1, d, bh, ctx);
+}
+
+size_t dual_seg_bwd_workspace_bytes(int B, int H, int T, int d, int S) {
+  if (S <= 1) return dual_bwd_workspace_bytes(B, H, T, d);
+  // the backward kernel's checkpoints over the segment view, then seven fp32 states per segment
+  const size_t ck = (dual_bwd_workspace_bytes(B * H * S, 1, T / S, d) + 255) & ~size_t(255);
+  return ck + 7 * (size_t)B * H * S * d * d * sizeof(float);
+}
+
+// Backward: maps and start states as in the forward; a backward pass over the segments from a
+// zero incoming state gradient gives each segment's offset N_s (its dW0 output); the reverse fold
+// gives every segment's incoming state gradient X_after(s); a second backward pass from the
+// true (W_start, X_after) gives the gradients, and segment 0's dW0 is the stream's.
+int launch_dual_seg_bwd(const AssocBwdArgs& a, int S, const LaunchCtx& ctx) {
+  if (S <= 1) return launch_dual_bwd(a, ctx);
+  const int d = a.d, bh = a.B * a.H;
+  const size_t n = (size_t)bh * S, per = (size_t)d * d;
+  if (a.ws_bytes < dual_seg_bwd_workspace_bytes(a.B, a.H, a.T, d, S)) {
+    *ctx.msg = "ttt_linear_dual_seg_bwd: workspace smaller than ttt_linear_dual_seg_bwd_workspace_size()";
+    return kWorkspace;
   }
-  return kOk;
+  const size_t ck = (dual_bwd_workspace_bytes((int)n, 1, a.T / S, d) + 255) & ~size_t(255);
+  float* Wid = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) + ck);
+  float* Bm = Wid + n * per;
+  float* ABm = Bm + n * per;
+  float* Wst = ABm + n * per;
+  float* Noff = Wst + n * per;
+  float* Xaft = Noff + n * per;
+  float* dW0s = Xaft + n * per;
+  StateArgs v{a.Q, a.K, a.V, a.eta, a.eta_scalar, nullptr, nullptr, nullptr, (int)n, 1,
+              a.T / S, d, a.C, 1, nullptr, 0};
+  // the forward maps write their (unused) outputs into dQ, which the last pass overwrites
+  int st = maps_and_fold(v, S, bh, a.S0, a.dQ, Wid, Bm, ABm, Wst, ctx);
+  if (st != kOk) return st;
+  AssocBwdArgs b = a;
+  b.B = (int)n;
+  b.H = 1;
+  b.T = a.T / S;
+  b.S0 = Wst;
+  b.ws = a.ws;
+  b.ws_bytes = ck;
+  b.dS_out = nullptr;   // offsets N_s (the gradients written here are overwritten below)
+  b.dS0 = Noff;
+  if ((st = launch_dual_bwd(b, ctx)) != kOk) return st;
+  if ((st = launch_fold(true, d, bh, a.dS_out, Bm, ABm, Noff, Xaft, S, ctx)) != kOk) return st;
+  b.dS_out = Xaft;
+  b.dS0 = dW0s;
+  if ((st = launch_dual_bwd(b, ctx)) != kOk) return st;
+  return pick(dW0s, a.dS0, S, 0, d, bh, ctx);
 }
 
 }  // namespace ttt

@@ -114,6 +114,9 @@ int launch_dual_seg(const StateArgs& a, int S, const LaunchCtx& ctx);
 bool dual_bwd_supported(int d, int C, int dt);
 size_t dual_bwd_workspace_bytes(int B, int H, int T, int d);
 int launch_dual_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx);
+// Dual-form backward over S segments (S <= 1: launch_dual_bwd).
+size_t dual_seg_bwd_workspace_bytes(int B, int H, int T, int d, int S);
+int launch_dual_seg_bwd(const AssocBwdArgs& a, int S, const LaunchCtx& ctx);
 size_t assoc_momentum_workspace_bytes(int B, int H, int T, int d, int C);
 struct AssocMomentumArgs {
   const void* Q;

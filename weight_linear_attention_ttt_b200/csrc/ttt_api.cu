@@ -374,19 +374,14 @@ int ttt_assoc_scan_bwd(const void* Q, const void* K, const void* V, const float*
   return finish(launch_assoc_bwd(a, ctx), msg);
 }
 
-size_t ttt_linear_dual_bwd_workspace_size(int B, int H, int T, int d, int C, int dt) {
-  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0 ||
-      !dual_bwd_supported(d, C, dt))
-    return 0;
-  return dual_bwd_workspace_bytes(B, H, T, d);
-}
-
-int ttt_linear_dual_bwd(const void* Q, const void* K, const void* V, const float* eta,
-                        float eta_scalar, const float* W0, const void* dO, const float* dW_out,
+namespace {
+// Host-side checks shared by the dual-form backward entry points (before any CUDA call):
+// pointers, sizes, dtype, alignment, support, workspace and overlaps.
+int check_dual_bwd_args(const std::string& f, const void* Q, const void* K, const void* V,
+                        const float* eta, const float* W0, const void* dO, const float* dW_out,
                         void* dQ, void* dK, void* dV, float* deta, float* dW0, int B, int H,
                         int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
-                        cudaStream_t stream) {
-  const std::string f("ttt_linear_dual_bwd");
+                        size_t need) {
   if (!Q || !K || !V || !dO || !dQ || !dK || !dV || !deta || !dW0)
     return fail(TTT_ERR_INVALID_ARG, f + ": Q, K, V, dO and every output must be non-null");
   if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0)
@@ -400,9 +395,9 @@ int ttt_linear_dual_bwd(const void* Q, const void* K, const void* V, const float
       return fail(TTT_ERR_INVALID_ARG, f + ": every device pointer must be 16-byte aligned");
   if (!dual_bwd_supported(d, C, dt))
     return fail(TTT_ERR_UNSUPPORTED, f + ": supported bf16, C == 16, d in {32, 64, 128}");
-  const size_t need = dual_bwd_workspace_bytes(B, H, T, d);
+  if (need == 0) return TTT_OK;   // caller signals an invalid segment count separately
   if (!workspace || workspace_bytes < need)
-    return fail(TTT_ERR_WORKSPACE, f + ": workspace smaller than ttt_linear_dual_bwd_workspace_size()");
+    return fail(TTT_ERR_WORKSPACE, f + ": workspace smaller than the size query returns");
   const size_t nx = (size_t)B * H * T * d * 2, ns = (size_t)B * H * d * d * 4;
   const size_t ne = (size_t)B * H * T * 4;
   struct R { const void* p; size_t n; };
@@ -417,6 +412,28 @@ int ttt_linear_dual_bwd(const void* Q, const void* K, const void* V, const float
       if (overlap(outs[i].p, outs[i].n, outs[j].p, outs[j].n))
         return fail(TTT_ERR_INVALID_ARG, f + ": outputs and workspace must not overlap");
   }
+  return TTT_OK;
+}
+}  // namespace
+
+size_t ttt_linear_dual_bwd_workspace_size(int B, int H, int T, int d, int C, int dt) {
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0 ||
+      !dual_bwd_supported(d, C, dt))
+    return 0;
+  return dual_bwd_workspace_bytes(B, H, T, d);
+}
+
+int ttt_linear_dual_bwd(const void* Q, const void* K, const void* V, const float* eta,
+                        float eta_scalar, const float* W0, const void* dO, const float* dW_out,
+                        void* dQ, void* dK, void* dV, float* deta, float* dW0, int B, int H,
+                        int T, int d, int C, int dt, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
+  const std::string f("ttt_linear_dual_bwd");
+  const size_t need = (B > 0 && H > 0 && T > 0 && d > 0) ? dual_bwd_workspace_bytes(B, H, T, d)
+                                                          : 1;
+  int st = check_dual_bwd_args(f, Q, K, V, eta, W0, dO, dW_out, dQ, dK, dV, deta, dW0, B, H, T,
+                               d, C, dt, workspace, workspace_bytes, need);
+  if (st != TTT_OK) return st;
   AssocBwdArgs a{Q, K, V, eta, eta_scalar, W0, dO, dW_out, dQ, dK, dV, deta, dW0, B, H, T, d, C,
                  workspace, workspace_bytes};
   std::string msg;
@@ -424,6 +441,41 @@ int ttt_linear_dual_bwd(const void* Q, const void* K, const void* V, const float
   if (!err) return fail(TTT_ERR_CUDA, msg);
   LaunchCtx ctx{stream, err, &msg};
   return finish(launch_dual_bwd(a, ctx), msg);
+}
+
+size_t ttt_linear_dual_seg_bwd_workspace_size(int B, int H, int T, int d, int C, int dt,
+                                              int segments) {
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0 || segments < 0 ||
+      !dual_bwd_supported(d, C, dt))
+    return 0;
+  const int S = dual_seg_choose_segments(B, H, T, C, segments);
+  return S < 1 ? 0 : dual_seg_bwd_workspace_bytes(B, H, T, d, S);
+}
+
+int ttt_linear_dual_seg_bwd(const void* Q, const void* K, const void* V, const float* eta,
+                            float eta_scalar, const float* W0, const void* dO,
+                            const float* dW_out, void* dQ, void* dK, void* dV, float* deta,
+                            float* dW0, int B, int H, int T, int d, int C, int dt, int segments,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const std::string f("ttt_linear_dual_seg_bwd");
+  int st = check_dual_bwd_args(f, Q, K, V, eta, W0, dO, dW_out, dQ, dK, dV, deta, dW0, B, H, T,
+                               d, C, dt, workspace, workspace_bytes, 0);
+  if (st != TTT_OK) return st;
+  if (segments < 0) return fail(TTT_ERR_INVALID_ARG, f + ": segments must be >= 0");
+  const int S = dual_seg_choose_segments(B, H, T, C, segments);
+  if (S < 1)
+    return fail(TTT_ERR_INVALID_ARG, f + ": segments must divide the number of chunks T / C");
+  st = check_dual_bwd_args(f, Q, K, V, eta, W0, dO, dW_out, dQ, dK, dV, deta, dW0, B, H, T, d,
+                           C, dt, workspace, workspace_bytes,
+                           dual_seg_bwd_workspace_bytes(B, H, T, d, S));
+  if (st != TTT_OK) return st;
+  AssocBwdArgs a{Q, K, V, eta, eta_scalar, W0, dO, dW_out, dQ, dK, dV, deta, dW0, B, H, T, d, C,
+                 workspace, workspace_bytes};
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  return finish(launch_dual_seg_bwd(a, S, ctx), msg);
 }
 
 int ttt_assoc_state_fwd(const void* K, const void* V, const float* eta, float eta_scalar,

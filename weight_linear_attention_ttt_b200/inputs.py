@@ -86,6 +86,12 @@ WORKLOADS = {
     "dual_seg_bf16_B1H4T262144_d64C16": Workload(
         "dual_seg_bf16_B1H4T262144_d64C16", "dual_seg", 1010, B=1, H=4, T=262144, d=64, C=16,
         normalise=("K", "V")),
+    "dual_bwd_bf16_B1H4T262144_d64C16": Workload(
+        "dual_bwd_bf16_B1H4T262144_d64C16", "dual_bwd", 1011, B=1, H=4, T=262144, d=64, C=16,
+        normalise=("K", "V")),
+    "dual_seg_bwd_bf16_B1H4T262144_d64C16": Workload(
+        "dual_seg_bwd_bf16_B1H4T262144_d64C16", "dual_seg_bwd", 1011, B=1, H=4, T=262144,
+        d=64, C=16, normalise=("K", "V")),
     "dual_bwd_bf16_B8H12T2048_d64C16": Workload(
         "dual_bwd_bf16_B8H12T2048_d64C16", "dual_bwd", 1006, B=8, H=12, T=2048, d=64, C=16,
         normalise=("K", "V")),
@@ -221,7 +227,7 @@ def make_inputs(w: Workload, device="cpu", *, seed: Optional[int] = None, **over
         return assoc_bwd_inputs(w.B, w.H, w.T, w.d, seed=s, device=device, dtype=w.dtype,
                                 qkv=w.qkv, normalise=w.normalise, eta=w.eta,
                                 eta_const=w.eta_const, w0=w.w0)
-    if w.kind == "dual_bwd":
+    if w.kind in ("dual_bwd", "dual_seg_bwd"):
         return dual_bwd_inputs(w.B, w.H, w.T, w.d, seed=s, device=device, dtype=w.dtype,
                                qkv=w.qkv, normalise=w.normalise, eta=w.eta,
                                eta_const=w.eta_const, w0=w.w0)

@@ -50,6 +50,8 @@ def algorithmic(w: Workload) -> dict:
         return {"flops": 3 * th * (4 * w.d * w.d + 4 * w.C * w.d),
                 "bytes": th * (7 * w.d * 2 + 8) + w.B * w.H * 2 * w.d * w.d * 4,
                 "tokens": w.B * w.T}
+    if w.kind == "dual_seg_bwd":
+        return algorithmic(dataclasses.replace(w, kind="dual_bwd"))
     if w.kind == "dual_bwd":
         # the chunk adjoint's products: K W, K X, dO W^T, dG W^T, diag(eta) G X^T, Q^T dO and
         # K^T dG (2 d^2 each) plus the C x C terms Q K^T, dO G^T, A^T dO, dS K, dS^T Q (2 C d
