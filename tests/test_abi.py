@@ -177,3 +177,44 @@ def test_momentum_validation(lib):
     assert mom(0.5, d=64) == 2
     assert mom(0.5, M_out=6 * A + 64) == 1                      # M_out overlaps O
     assert lib.ttt_launch_count() == 0
+
+
+def test_segmented_entry_points_validation(lib):
+    v = ctypes.c_void_p
+
+    def fwd(segments, T=1024, d=64, ws=10 * A, ws_bytes=1 << 30, O=6 * A):
+        return lib.ttt_linear_dual_seg_fwd(v(A), v(2 * A), v(3 * A), v(4 * A),
+                                           ctypes.c_float(0.0), v(5 * A), v(O), v(7 * A), 1, 1,
+                                           T, d, 16, 1, segments, v(ws), ws_bytes, None)
+
+    assert fwd(3) == 1              # 3 does not divide the 64 chunks
+    assert fwd(-1) == 1
+    assert fwd(4, d=48) == 2
+    assert fwd(4, ws_bytes=16) == 3
+    assert fwd(4, ws=0) == 3
+    assert fwd(4, O=A + 64) == 1    # O overlaps Q
+    # sizes: 5 fp32 d x d states per segment (forward); none when one segment is chosen
+    assert lib.ttt_linear_dual_seg_workspace_size(1, 1, 1024, 64, 16, 1, 4) == 5 * 4 * 64 * 64 * 4
+    assert lib.ttt_linear_dual_seg_workspace_size(1, 1, 1024, 64, 16, 1, 3) == 0
+    assert lib.ttt_linear_dual_seg_workspace_size(8, 12, 1024, 64, 16, 1, 0) == 0
+    assert lib.ttt_linear_dual_seg_bwd_workspace_size(1, 1, 1024, 64, 16, 1, 4) > \
+        lib.ttt_linear_dual_bwd_workspace_size(1, 1, 1024, 64, 16, 1)
+    assert lib.ttt_launch_count() == 0
+
+
+def test_segmented_backward_validation(lib):
+    v = ctypes.c_void_p
+
+    def bwd(segments, ws_bytes=1 << 30, dQ=8 * A, d=64):
+        return lib.ttt_linear_dual_seg_bwd(v(A), v(2 * A), v(3 * A), v(4 * A),
+                                           ctypes.c_float(0.0), v(5 * A), v(6 * A), v(7 * A),
+                                           v(dQ), v(9 * A), v(10 * A), v(11 * A), v(12 * A),
+                                           1, 1, 1024, d, 16, 1, segments, v(13 * A), ws_bytes,
+                                           None)
+
+    assert bwd(3) == 1 and bwd(-2) == 1
+    assert bwd(4, d=48) == 2
+    assert bwd(4, ws_bytes=16) == 3
+    assert bwd(4, dQ=2 * A) == 1    # an output on an input
+    assert bwd(4, dQ=0) == 1
+    assert lib.ttt_launch_count() == 0
