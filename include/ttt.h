@@ -238,6 +238,27 @@ int ttt_linear_dual_seg_bwd(const void* Q, const void* K, const void* V, const f
                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* --------------------------------------------------------------------------------------------
+ * Context parallelism of the dual form (the segment-affine maps of ttt_linear_dual_seg_fwd, one
+ * segment per rank; orchestration in weight_linear_attention_ttt_b200/context_parallel.py):
+ *
+ * ttt_linear_dual_slice_maps: for a token slice of every stream (K, V [B,H,T,d], eta [B,H,T]
+ *  or NULL with eta_scalar), the affine map of its chunk updates, W_end = A W_start + B:
+ *  B_out = the end state from W = 0, A_out = the end state from W = I minus B_out
+ *  ([B,H,d,d] fp32 each). Workspace: ttt_linear_dual_slice_maps_workspace_size() bytes. Same
+ *  support as ttt_linear_dual_fwd (d in {32, 64, 128}, C <= 64, fp32 or bf16).
+ * ttt_dual_state_fold: W_out = the state after applying maps 0 .. upto-1 in order to W0 (NULL:
+ *  zeros): W <- A_m W + B_m, with A_maps and B_maps [n_maps][B,H,d,d] fp32 (the all-gathered
+ *  layout). 0 <= upto <= n_maps; W_out may equal W0. fp32 throughout.
+ * ------------------------------------------------------------------------------------------ */
+size_t ttt_linear_dual_slice_maps_workspace_size(int B, int H, int T, int d, int C, int dt);
+int ttt_linear_dual_slice_maps(const void* K, const void* V, const float* eta, float eta_scalar,
+                               float* A_out, float* B_out, int B, int H, int T, int d, int C,
+                               int dt, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+int ttt_dual_state_fold(const float* W0, const float* A_maps, const float* B_maps, int n_maps,
+                        int upto, float* W_out, int B, int H, int d, cudaStream_t stream);
+
+/* --------------------------------------------------------------------------------------------
  * State increment of a sequence slice in the associative mode (the first pass of the prefix
  * scan over states, "KV 바인딩 기반 테스트 시간 학습은 사실상 선형 어텐션이다", associativity
  * paragraph; per-chunk deltas combined by a prefix sum for context parallelism, "In-Place

@@ -218,3 +218,31 @@ def test_segmented_backward_validation(lib):
     assert bwd(4, dQ=2 * A) == 1    # an output on an input
     assert bwd(4, dQ=0) == 1
     assert lib.ttt_launch_count() == 0
+
+
+def test_dual_context_parallel_pieces_validation(lib):
+    v = ctypes.c_void_p
+
+    def maps(**kw):
+        a = dict(K=A, V=2 * A, eta=3 * A, Aout=4 * A, Bout=5 * A, T=256, d=64, C=16, dt=1,
+                 ws=6 * A, ws_bytes=1 << 30)
+        a.update(kw)
+        return lib.ttt_linear_dual_slice_maps(v(a["K"]), v(a["V"]), v(a["eta"]),
+                                              ctypes.c_float(0.0), v(a["Aout"]), v(a["Bout"]),
+                                              1, 1, a["T"], a["d"], a["C"], a["dt"], v(a["ws"]),
+                                              a["ws_bytes"], None)
+
+    assert maps(Bout=0) == 1 and maps(T=250) == 1 and maps(d=48) == 2
+    assert maps(ws_bytes=16) == 3 and maps(Aout=A + 64) == 1 and maps(Bout=4 * A + 256) == 1
+    need = lib.ttt_linear_dual_slice_maps_workspace_size(1, 1, 256, 64, 16, 1)
+    assert need == 256 * 64 * 2 + 64 * 64 * 4
+
+    def fold(**kw):
+        a = dict(W0=A, Am=2 * A, Bm=3 * A, n=4, upto=2, Wout=4 * A, d=64)
+        a.update(kw)
+        return lib.ttt_dual_state_fold(v(a["W0"]), v(a["Am"]), v(a["Bm"]), a["n"], a["upto"],
+                                       v(a["Wout"]), 1, 1, a["d"], None)
+
+    assert fold(upto=5) == 1 and fold(upto=-1) == 1 and fold(n=0) == 1 and fold(Am=0) == 1
+    assert fold(d=48) == 2 and fold(Wout=2 * A + 64) == 1 and fold(Wout=A + 64) == 1
+    assert lib.ttt_launch_count() == 0

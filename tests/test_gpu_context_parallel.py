@@ -1,7 +1,8 @@
-"""GPU checks of the context-parallel associative scan pieces, through the C ABI: the slice
-state increment, the prefix combination of increments, a sequence split into slices evaluated
-slice by slice (the ranks emulated one after another in one process: no kernel waits on
-another), and the orchestrator on a one-rank NCCL group."""
+"""GPU checks of the context-parallel pieces, through the C ABI: for the associative scan the
+slice state increment, the prefix combination of increments, a sequence split into slices
+evaluated slice by slice (the ranks emulated one after another in one process: no kernel waits
+on another), and the orchestrator on a one-rank NCCL group; for the dual form the slice maps,
+their ordered fold and the slices run from the folded starts."""
 import datetime
 import os
 import socket
@@ -95,3 +96,42 @@ def test_orchestrator_on_a_one_rank_nccl_group(cuda_lib):
         dist.destroy_process_group()
     Or, Sr = oracle_full(x, S0)
     assert max_rel_l2(O, Or, 2) <= TOL and max_rel_l2(S, Sr, 2) <= TOL
+
+
+@pytest.mark.parametrize("slices,dtype", [(2, "bf16"), (4, "bf16"), (3, "f32")])
+def test_dual_form_slices_emulated_on_one_gpu(cuda_lib, slices, dtype):
+    """The dual form's context-parallel pieces on one GPU: every slice's affine maps
+    (ttt_linear_dual_slice_maps), the ordered fold of the maps before it
+    (ttt_dual_state_fold) as its start state, and the dual form on the slice from there; the
+    concatenated outputs and the fold of all maps equal the sequential oracle."""
+    import torch
+
+    B, H, T, d, C = 2, 2, 768 if slices == 3 else 1024, 32 if dtype == "f32" else 64, 16
+    x = inp.dual_or_assoc_inputs(B, H, T, d, seed=40 + slices, device="cuda", dtype=dtype,
+                                 normalise=("K", "V"), eta="sigmoid")
+    L = T // slices
+    cut = lambda t, r: t[:, :, r * L:(r + 1) * L].contiguous()
+    maps = [ttt.ttt_linear_dual_slice_maps(cut(x["K"], r), cut(x["V"], r), cut(x["eta"], r),
+                                           C=C) for r in range(slices)]
+    A_all = torch.stack([m[0] for m in maps]).contiguous()
+    B_all = torch.stack([m[1] for m in maps]).contiguous()
+    outs = []
+    for r in range(slices):
+        start = ttt.ttt_dual_state_fold(x["W0"], A_all, B_all, r)
+        O_r, _ = ttt.ttt_linear_dual_fwd(cut(x["Q"], r), cut(x["K"], r), cut(x["V"], r),
+                                         cut(x["eta"], r), start, C=C)
+        outs.append(O_r)
+    W = ttt.ttt_dual_state_fold(x["W0"], A_all, B_all, slices)
+    f = lambda t: t.float().cpu().numpy()
+    Or, Wr = orc.dual_form(f(x["Q"]), f(x["K"]), f(x["V"]), x["eta"].cpu().numpy(),
+                           x["W0"].cpu().numpy(), C)
+    tol = 1e-4 if dtype == "f32" else 1e-2
+    eo = max_rel_l2(torch.cat(outs, dim=2), Or, 2)
+    ew = max_rel_l2(W, Wr, 2)
+    assert eo <= tol and ew <= tol, (eo, ew)
+    # fold of nothing is W0; W_out may be the W0 buffer
+    assert torch.equal(ttt.ttt_dual_state_fold(x["W0"], A_all, B_all, 0), x["W0"])
+    W0c = x["W0"].clone()
+    ttt.ttt_dual_state_fold(W0c, A_all, B_all, slices, W_out=W0c)
+    assert torch.equal(W0c, W)
+    assert ttt.read_device_error() == 0

@@ -159,3 +159,88 @@ def test_context_parallel_assoc_scan_over_gloo_ranks(tmp_path, world):
     for r in range(world):
         np.testing.assert_allclose(np.load(tmp_path / f"cp_S_{r}.npy"), S, rtol=1e-10,
                                    atol=1e-12)
+
+
+def _dual_cp_worker(rank, world, port, outdir):
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from oracle import ttt_oracle as orc
+    from weight_linear_attention_ttt_b200 import inputs as inp
+    from weight_linear_attention_ttt_b200.context_parallel import dual_form_fwd_cp
+    from weight_linear_attention_ttt_b200.shard import split_range
+
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        B, H, T, d, C = 2, 2, 256, 8, 16
+        x = inp.dual_or_assoc_inputs(B, H, T, d, seed=13, device="cpu", normalise=("K", "V"),
+                                     eta="sigmoid", w0="normal_0.02")
+        t0, t1 = split_range(T // C, rank, world)
+        sl = slice(t0 * C, t1 * C)
+        Q, K, V = (x[k][:, :, sl].double() for k in ("Q", "K", "V"))
+        eta = x["eta"][:, :, sl].double()
+        W0 = x["W0"].double()
+
+        def per_stream(fn, *args):
+            return [[fn(*(a[b, h] for a in args)) for h in range(H)] for b in range(B)]
+
+        def maps_fn(K_, V_, e_):
+            res = per_stream(lambda k, v, e: orc.dual_segment_maps_stream(k, v, e, C),
+                             K_.numpy(), V_.numpy(), e_.numpy())
+            A = torch.tensor(np.array([[r[0] for r in row] for row in res]))
+            Bm = torch.tensor(np.array([[r[1] for r in row] for row in res]))
+            return A, Bm
+
+        def scan_fn(Q_, K_, V_, e_, w_):
+            res = per_stream(lambda q, k, v, e, w: orc.dual_form_stream(q, k, v, e, w, C),
+                             Q_.numpy(), K_.numpy(), V_.numpy(), e_.numpy(), w_.numpy())
+            O = torch.tensor(np.array([[r[0] for r in row] for row in res]))
+            W = torch.tensor(np.array([[r[1] for r in row] for row in res]))
+            return O, W
+
+        def fold_fn(w0, A_all, B_all, upto):
+            W = w0.clone()
+            for m in range(upto):
+                W = A_all[m] @ W + B_all[m]
+            return W
+
+        O, W_final = dual_form_fwd_cp(Q, K, V, eta, W0, C=C, maps_fn=maps_fn, scan_fn=scan_fn,
+                                      fold_fn=fold_fn)
+        np.save(os.path.join(outdir, f"dcp_O_{rank}.npy"), O.numpy())
+        np.save(os.path.join(outdir, f"dcp_W_{rank}.npy"), W_final.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_parallel_dual_form_over_gloo_ranks(tmp_path, world):
+    """Each rank owns a slice of the sequence; one all-gather of the slices' affine maps and an
+    ordered fold give every rank its start state; the gathered outputs and the final state equal
+    the sequential dual form."""
+    mp.start_processes(_dual_cp_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    from oracle import ttt_oracle as orc
+    from weight_linear_attention_ttt_b200 import inputs as inp
+
+    x = inp.dual_or_assoc_inputs(2, 2, 256, 8, seed=13, device="cpu", normalise=("K", "V"),
+                                 eta="sigmoid", w0="normal_0.02")
+    O, W = orc.dual_form(x["Q"].double().numpy(), x["K"].double().numpy(),
+                         x["V"].double().numpy(), x["eta"].double().numpy(),
+                         x["W0"].double().numpy(), 16)
+    Og = np.concatenate([np.load(tmp_path / f"dcp_O_{r}.npy") for r in range(world)], axis=2)
+    np.testing.assert_allclose(Og, O, rtol=1e-10, atol=1e-12)
+    for r in range(world):
+        np.testing.assert_allclose(np.load(tmp_path / f"dcp_W_{r}.npy"), W, rtol=1e-10,
+                                   atol=1e-12)

@@ -29,6 +29,8 @@ EXPORTED_SYMBOLS = (
     "ttt_assoc_scan_bwd_workspace_size", "ttt_assoc_scan_bwd",
     "ttt_linear_dual_bwd_workspace_size", "ttt_linear_dual_bwd",
     "ttt_linear_dual_seg_bwd_workspace_size", "ttt_linear_dual_seg_bwd",
+    "ttt_linear_dual_slice_maps_workspace_size", "ttt_linear_dual_slice_maps",
+    "ttt_dual_state_fold",
     "ttt_assoc_momentum_workspace_size", "ttt_assoc_momentum_fwd",
     "ttt_state_prefix_sum",
     "inplace_ttt_workspace_size", "inplace_ttt_chunk_fwd",
@@ -83,6 +85,13 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
         getattr(lib, name).restype = c_int
         getattr(lib, name).argtypes = [vp, vp, vp, fp, c_float, fp, vp, fp, vp, vp, vp, fp, fp,
                                        c_int, c_int, c_int, c_int, c_int, c_int, vp, c_size, vp]
+    lib.ttt_linear_dual_slice_maps_workspace_size.restype = c_size
+    lib.ttt_linear_dual_slice_maps_workspace_size.argtypes = [c_int] * 6
+    lib.ttt_linear_dual_slice_maps.restype = c_int
+    lib.ttt_linear_dual_slice_maps.argtypes = [vp, vp, fp, c_float, fp, fp, c_int, c_int, c_int,
+                                               c_int, c_int, c_int, vp, c_size, vp]
+    lib.ttt_dual_state_fold.restype = c_int
+    lib.ttt_dual_state_fold.argtypes = [fp, fp, fp, c_int, c_int, fp, c_int, c_int, c_int, vp]
     lib.ttt_linear_dual_seg_bwd_workspace_size.restype = c_size
     lib.ttt_linear_dual_seg_bwd_workspace_size.argtypes = [c_int] * 7
     lib.ttt_linear_dual_seg_bwd.restype = c_int
@@ -360,6 +369,59 @@ def ttt_linear_dual_seg_bwd(Q, K, V, eta, W0, dO, dW_out=None, *, C: int, segmen
                                      wsz, _stream_ptr(stream))
     _check("ttt_linear_dual_seg_bwd", st)
     return dQ, dK, dV, deta, dW0
+
+
+def ttt_linear_dual_slice_maps(K, V, eta=None, *, C: int, eta_scalar: float = 0.0,
+                               A_out=None, B_out=None, workspace=None, stream=None) -> Tuple:
+    """The affine map W_end = A W_start + B of a token slice of every stream (dual form).
+    Returns (A [B,H,d,d], B [B,H,d,d]) fp32."""
+    import torch
+
+    lib = load_library()
+    _require(K.dim() == 4, "K, V must be [B, H, T, d]")
+    B, H, T, d = K.shape
+    for t in (K, V):
+        _require(t.is_cuda and t.is_contiguous() and t.shape == K.shape and t.dtype == K.dtype,
+                 "K, V must be contiguous CUDA tensors of one shape and dtype")
+    dt = _dtype_code(K)
+    if eta is not None:
+        _require(eta.is_cuda and eta.dtype == torch.float32 and eta.is_contiguous() and
+                 tuple(eta.shape) == (B, H, T), "eta must be a contiguous fp32 [B, H, T] tensor")
+    if A_out is None:
+        A_out = torch.empty((B, H, d, d), device=K.device, dtype=torch.float32)
+    if B_out is None:
+        B_out = torch.empty((B, H, d, d), device=K.device, dtype=torch.float32)
+    ws_bytes = lib.ttt_linear_dual_slice_maps_workspace_size(B, H, T, d, C, dt)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, device=K.device, dtype=torch.uint8)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.ttt_linear_dual_slice_maps(_ptr(K), _ptr(V), _ptr(eta), ctypes.c_float(eta_scalar),
+                                        _ptr(A_out), _ptr(B_out), B, H, T, d, C, dt,
+                                        _ptr(workspace), wsz, _stream_ptr(stream))
+    _check("ttt_linear_dual_slice_maps", st)
+    return A_out, B_out
+
+
+def ttt_dual_state_fold(W0, A_maps, B_maps, upto: int, *, W_out=None, stream=None):
+    """W_out = maps 0 .. upto-1 of A_maps / B_maps ([n, B, H, d, d] fp32) applied in order to
+    W0 ([B, H, d, d] fp32 or None = zeros)."""
+    import torch
+
+    lib = load_library()
+    _require(A_maps.dim() == 5 and A_maps.shape == B_maps.shape, "maps must be [n, B, H, d, d]")
+    n, B, H, d, _ = A_maps.shape
+    for t in (A_maps, B_maps):
+        _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous(),
+                 "maps must be contiguous fp32 CUDA tensors")
+    if W0 is not None:
+        _require(W0.is_cuda and W0.dtype == torch.float32 and W0.is_contiguous() and
+                 tuple(W0.shape) == (B, H, d, d), "W0 must be fp32 [B, H, d, d]")
+    if W_out is None:
+        W_out = torch.empty((B, H, d, d), device=A_maps.device, dtype=torch.float32)
+    st = lib.ttt_dual_state_fold(_ptr(W0), _ptr(A_maps), _ptr(B_maps), n, upto, _ptr(W_out),
+                                 B, H, d, _stream_ptr(stream))
+    _check("ttt_dual_state_fold", st)
+    return W_out
 
 
 def ttt_assoc_momentum_fwd(Q, K, V, eta, beta: float, S0=None, M0=None, *, C: int,

@@ -120,6 +120,49 @@ __global__ void pick_segment_state_kernel(const float* __restrict__ src, float* 
   }
 }
 
+// a[i] -= b[i] over n elements
+__global__ void sub_states_kernel(float* __restrict__ a, const float* __restrict__ b, size_t n) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    a[i] -= b[i];
+}
+
+// Context parallelism: maps gathered from the ranks, [n_maps][BH][D][D] each (A and B apart).
+// One CTA per stream: W = W0 (or 0), then W <- A_m W + B_m for m < upto; W_out = W.
+template <int D>
+__global__ void __launch_bounds__(256) fold_gathered_kernel(const float* __restrict__ W0,
+                                                            const float* __restrict__ Am,
+                                                            const float* __restrict__ Bm,
+                                                            int upto, size_t bh_count,
+                                                            float* __restrict__ W_out) {
+  constexpr int E = D * D / 256;
+  extern __shared__ float fsm[];
+  float* W = fsm;
+  float* A = fsm + D * D;
+  const size_t bh = blockIdx.x;
+  for (int i = threadIdx.x; i < D * D; i += 256) W[i] = W0 ? W0[bh * D * D + i] : 0.f;
+  __syncthreads();
+  for (int m = 0; m < upto; ++m) {
+    const size_t off = ((size_t)m * bh_count + bh) * D * D;
+    for (int i = threadIdx.x; i < D * D; i += 256) A[i] = Am[off + i];
+    __syncthreads();
+    float out[E];
+#pragma unroll
+    for (int q = 0; q < E; ++q) {
+      const int idx = threadIdx.x + 256 * q, i = idx / D, j = idx % D;
+      float acc = Bm[off + idx];
+#pragma unroll 8
+      for (int k = 0; k < D; ++k) acc = fmaf(A[i * D + k], W[k * D + j], acc);
+      out[q] = acc;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < E; ++q) W[threadIdx.x + 256 * q] = out[q];
+    __syncthreads();
+  }
+  for (int i = threadIdx.x; i < D * D; i += 256) W_out[bh * D * D + i] = W[i];
+}
+
 int sm_count() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -259,6 +302,62 @@ int launch_dual_seg(const StateArgs& a, int S, const LaunchCtx& ctx) {
   po.S_out = Wend;
   if ((st = run_dual(po, ctx)) != kOk) return st;
   return pick(Wend, a.S_out, S, S - 1, d, bh, ctx);
+}
+
+size_t dual_slice_maps_workspace_bytes(int B, int H, int T, int d, int dt) {
+  // scratch outputs of the two passes, then the identity start states
+  const size_t o = ((size_t)B * H * T * d * (dt ? 2 : 4) + 255) & ~size_t(255);
+  return o + (size_t)B * H * d * d * sizeof(float);
+}
+
+// The maps of a token slice of every stream: B from W = 0, A = (end from W = I) - B.
+int launch_dual_slice_maps(const StateArgs& a, float* A_out, float* B_out, const LaunchCtx& ctx) {
+  const size_t bh = (size_t)a.B * a.H, per = (size_t)a.d * a.d;
+  const size_t o = ((size_t)bh * a.T * a.d * (a.dt ? 2 : 4) + 255) & ~size_t(255);
+  float* Wid = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) + o);
+  identity_states_kernel<<<sm_count() * 4, 256, 0, ctx.stream>>>(Wid, bh, a.d);
+  count_launch();
+  int st = check_launch(ctx, "identity launch");
+  if (st != kOk) return st;
+  StateArgs x = a;   // the queries are the keys: the outputs are scratch
+  x.Q = a.K;
+  x.O = a.ws;
+  x.ws = nullptr;
+  x.ws_bytes = 0;
+  x.S0 = nullptr;
+  x.S_out = B_out;
+  if ((st = run_dual(x, ctx)) != kOk) return st;
+  x.S0 = Wid;
+  x.S_out = A_out;
+  if ((st = run_dual(x, ctx)) != kOk) return st;
+  sub_states_kernel<<<sm_count() * 2, 256, 0, ctx.stream>>>(A_out, B_out, bh * per);
+  count_launch();
+  return check_launch(ctx, "subtract launch");
+}
+
+int launch_dual_state_fold(const float* W0, const float* A, const float* B, int upto, int bh,
+                           int d, float* W_out, const LaunchCtx& ctx) {
+  const size_t smem = 2 * (size_t)d * d * sizeof(float);
+  cudaError_t e = cudaSuccess;
+  switch (d) {
+    case 32:
+      fold_gathered_kernel<32><<<bh, 256, smem, ctx.stream>>>(W0, A, B, upto, bh, W_out);
+      break;
+    case 64:
+      fold_gathered_kernel<64><<<bh, 256, smem, ctx.stream>>>(W0, A, B, upto, bh, W_out);
+      break;
+    case 128:
+      e = cudaFuncSetAttribute(fold_gathered_kernel<128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess)
+        fold_gathered_kernel<128><<<bh, 256, smem, ctx.stream>>>(W0, A, B, upto, bh, W_out);
+      break;
+    default:
+      *ctx.msg = "dual state fold: unsupported head dim";
+      return kUnsupported;
+  }
+  count_launch();
+  return check_launch(ctx, "fold launch", e);
 }
 
 size_t dual_seg_bwd_workspace_bytes(int B, int H, int T, int d, int S) {

@@ -114,6 +114,11 @@ int launch_dual_seg(const StateArgs& a, int S, const LaunchCtx& ctx);
 bool dual_bwd_supported(int d, int C, int dt);
 size_t dual_bwd_workspace_bytes(int B, int H, int T, int d);
 int launch_dual_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx);
+// Context parallelism of the dual form: a slice's affine maps, and the fold of gathered maps.
+size_t dual_slice_maps_workspace_bytes(int B, int H, int T, int d, int dt);
+int launch_dual_slice_maps(const StateArgs& a, float* A_out, float* B_out, const LaunchCtx& ctx);
+int launch_dual_state_fold(const float* W0, const float* A, const float* B, int upto, int bh,
+                           int d, float* W_out, const LaunchCtx& ctx);
 // Dual-form backward over S segments (S <= 1: launch_dual_bwd).
 size_t dual_seg_bwd_workspace_bytes(int B, int H, int T, int d, int S);
 int launch_dual_seg_bwd(const AssocBwdArgs& a, int S, const LaunchCtx& ctx);

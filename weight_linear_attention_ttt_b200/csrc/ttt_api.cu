@@ -237,6 +237,79 @@ int ttt_linear_dual_seg_fwd(const void* Q, const void* K, const void* V, const f
   return finish(launch_dual_seg(a, S, ctx), msg);
 }
 
+size_t ttt_linear_dual_slice_maps_workspace_size(int B, int H, int T, int d, int C, int dt) {
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0) return 0;
+  return dual_slice_maps_workspace_bytes(B, H, T, d, dt);
+}
+
+int ttt_linear_dual_slice_maps(const void* K, const void* V, const float* eta, float eta_scalar,
+                               float* A_out, float* B_out, int B, int H, int T, int d, int C,
+                               int dt, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+  const std::string f("ttt_linear_dual_slice_maps");
+  if (!K || !V || !A_out || !B_out)
+    return fail(TTT_ERR_INVALID_ARG, f + ": K, V, A_out and B_out must be non-null");
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0)
+    return fail(TTT_ERR_INVALID_ARG, f + ": B, H, T, d and C must be positive");
+  if (T % C != 0) return fail(TTT_ERR_INVALID_ARG, f + ": T must be a multiple of C");
+  if (dt != TTT_DTYPE_F32 && dt != TTT_DTYPE_BF16)
+    return fail(TTT_ERR_INVALID_ARG, f + ": dtype must be TTT_DTYPE_F32 or TTT_DTYPE_BF16");
+  const void* ptrs[] = {K, V, eta, A_out, B_out, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p))
+      return fail(TTT_ERR_INVALID_ARG, f + ": every device pointer must be 16-byte aligned");
+  if (!(d == 32 || d == 64 || d == 128) || C > 64)
+    return fail(TTT_ERR_UNSUPPORTED, f + ": supported d in {32, 64, 128} and 1 <= C <= 64");
+  const size_t need = dual_slice_maps_workspace_bytes(B, H, T, d, dt);
+  if (!workspace || workspace_bytes < need)
+    return fail(TTT_ERR_WORKSPACE, f + ": workspace smaller than the size query returns");
+  const size_t nx = (size_t)B * H * T * d * (dt ? 2 : 4), ns = (size_t)B * H * d * d * 4;
+  const size_t ne = (size_t)B * H * T * 4;
+  struct R { const void* p; size_t n; };
+  const R ins[] = {{K, nx}, {V, nx}, {eta, ne}};
+  const R outs[] = {{A_out, ns}, {B_out, ns}, {workspace, workspace_bytes}};
+  for (size_t i = 0; i < 3; ++i) {
+    for (const R& in : ins)
+      if (in.p && overlap(outs[i].p, outs[i].n, in.p, in.n))
+        return fail(TTT_ERR_INVALID_ARG, f + ": outputs and workspace must not overlap inputs");
+    for (size_t j = i + 1; j < 3; ++j)
+      if (overlap(outs[i].p, outs[i].n, outs[j].p, outs[j].n))
+        return fail(TTT_ERR_INVALID_ARG, f + ": outputs and workspace must not overlap");
+  }
+  StateArgs a{K, K, V, eta, eta_scalar, nullptr, nullptr, nullptr, B, H, T, d, C, dt, workspace,
+              workspace_bytes};
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  return finish(launch_dual_slice_maps(a, A_out, B_out, ctx), msg);
+}
+
+int ttt_dual_state_fold(const float* W0, const float* A_maps, const float* B_maps, int n_maps,
+                        int upto, float* W_out, int B, int H, int d, cudaStream_t stream) {
+  const std::string f("ttt_dual_state_fold");
+  if (!A_maps || !B_maps || !W_out)
+    return fail(TTT_ERR_INVALID_ARG, f + ": A_maps, B_maps and W_out must be non-null");
+  if (B <= 0 || H <= 0 || d <= 0 || n_maps <= 0 || upto < 0 || upto > n_maps)
+    return fail(TTT_ERR_INVALID_ARG, f + ": B, H, d, n_maps must be positive, 0 <= upto <= n_maps");
+  const void* ptrs[] = {W0, A_maps, B_maps, W_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p))
+      return fail(TTT_ERR_INVALID_ARG, f + ": every device pointer must be 16-byte aligned");
+  if (!(d == 32 || d == 64 || d == 128))
+    return fail(TTT_ERR_UNSUPPORTED, f + ": supported d in {32, 64, 128}");
+  const size_t ns = (size_t)B * H * d * d * 4, nm = ns * n_maps;
+  if (overlap(W_out, ns, A_maps, nm) || overlap(W_out, ns, B_maps, nm))
+    return fail(TTT_ERR_INVALID_ARG, f + ": W_out must not overlap the maps");
+  if (W0 && W0 != W_out && overlap(W0, ns, W_out, ns))
+    return fail(TTT_ERR_INVALID_ARG, f + ": W_out may equal W0 but not partly overlap it");
+  std::string msg;
+  unsigned* err = device_error_word(&msg);
+  if (!err) return fail(TTT_ERR_CUDA, msg);
+  LaunchCtx ctx{stream, err, &msg};
+  return finish(launch_dual_state_fold(W0, A_maps, B_maps, upto, B * H, d, W_out, ctx), msg);
+}
+
 size_t ttt_assoc_scan_workspace_size(int B, int H, int T, int d, int C, int dt) {
   if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || !assoc_supported(d, C, dt)) return 0;
   return assoc_workspace_bytes(B, H, T, d, C);
