@@ -361,6 +361,16 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
 
 
 # ----------------------------------------------------------------------------- arms
+def config_of(w, world: int) -> dict:
+    """The workload description both arms print (the reference arm times the same workload)."""
+    from weight_linear_attention_ttt_b200 import metrics
+
+    return {"workload": w.name, "kind": w.kind, "B": w.B, "H": w.H, "T": w.T, "d": w.d,
+            "C": w.C, "tokens_per_step_per_gpu": metrics.algorithmic(w)["tokens"],
+            "l2": "flushed (256 MiB write) before every timed step",
+            "parallelism": f"dp{world} (independent streams per rank)"}
+
+
 def run_reference(args, w, rank, world):
     """The oracle as the reference arm, on rank 0's host cores."""
     import torch
@@ -385,7 +395,7 @@ def run_reference(args, w, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": w.name, "sample_per_step": desc},
+            "config": config_of(w, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -466,10 +476,7 @@ def run_ours(args, w, rank, world, local_rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": {"workload": w.name, "kind": w.kind, "B": w.B, "H": w.H, "T": w.T,
-                       "d": w.d, "C": w.C, "tokens_per_step_per_gpu": algo["tokens"],
-                       "l2": "flushed (256 MiB write) before every timed step",
-                       "parallelism": f"dp{world} (independent streams per rank)"},
+            "config": config_of(w, world),
             "roofline": roof, "clocks": clk.summary(), "gpu_launches": launches,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}}
