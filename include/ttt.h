@@ -22,6 +22,13 @@
  *                          (gated-MLP paragraph, chunk-update paragraph, associative-scan
  *                          paragraph).
  *
+ * Around them, declared below in this order: the dual form evaluated sequence-parallel
+ * (ttt_linear_dual_seg_fwd), the associative mode with a momentum inner loop, the backwards of
+ * both modes (and of the sequence-parallel dual form), the context-parallel pieces (a slice's
+ * state increment and their prefix for the associative mode; a slice's affine maps and their
+ * ordered fold for the dual form), an allocation-free In-Place entry point, and the LM-aligned
+ * target of the In-Place update.
+ *
  * Conventions shared by every entry point
  *   - Row vectors: q_t, k_t, v_t are 1 x d; the state W (or S) is d x d laid out [d_in][d_out]
  *     (row-major), and a token reads o_t = q_t W.
@@ -58,7 +65,8 @@ typedef enum {
   TTT_ERR_UNSUPPORTED = 2, /* valid but not implemented: head dim, chunk size, dtype combination */
   TTT_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than *_workspace_size() */
   TTT_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed */
-  TTT_ERR_TIMEOUT = 5      /* reserved: a bounded device-side wait gave up (none wait today) */
+  TTT_ERR_TIMEOUT = 5      /* reserved; a bounded device-side wait that gives up is reported
+                              through ttt_read_device_error(), not as a status */
 } ttt_status_t;
 
 typedef enum { TTT_DTYPE_F32 = 0, TTT_DTYPE_BF16 = 1 } ttt_dtype_t;
