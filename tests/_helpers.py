@@ -19,3 +19,34 @@ def max_rel_l2(x, ref, lead: int):
     num = np.linalg.norm(xs - rs, axis=1)
     den = np.linalg.norm(rs, axis=1)
     return float(np.max(np.where(den > 0, num / np.where(den > 0, den, 1), num)))
+
+
+CANARY = 0xA5
+GUARD_BYTES = 4096
+
+
+def guarded(shape, dtype, device):
+    """A contiguous tensor of `shape` inside a larger buffer whose GUARD_BYTES before and after
+    hold the byte CANARY (a stand-in for a memory sanitizer: a kernel writing past its output
+    changes a guard byte). The view starts GUARD_BYTES into the buffer, so it keeps the buffer's
+    alignment. Returns (view, buffer)."""
+    import torch
+
+    elem = torch.empty((), dtype=dtype).element_size()
+    n = 1
+    for s in shape:
+        n *= s
+    pad = GUARD_BYTES // elem
+    buf = torch.empty(n + 2 * pad, dtype=dtype, device=device)
+    buf.view(torch.uint8).fill_(CANARY)
+    return buf[pad:pad + n].view(shape), buf
+
+
+def guards_intact(view, buf) -> bool:
+    """True if no byte outside `view` in `buf` has changed from CANARY."""
+    import torch
+
+    raw = buf.view(torch.uint8)
+    start = (view.data_ptr() - buf.data_ptr())
+    end = start + view.numel() * view.element_size()
+    return bool((raw[:start] == CANARY).all()) and bool((raw[end:] == CANARY).all())
