@@ -98,6 +98,29 @@ def test_orchestrator_on_a_one_rank_nccl_group(cuda_lib):
     assert max_rel_l2(O, Or, 2) <= TOL and max_rel_l2(S, Sr, 2) <= TOL
 
 
+def test_dual_form_orchestrator_on_a_one_rank_nccl_group(cuda_lib):
+    import torch.distributed as dist
+
+    from weight_linear_attention_ttt_b200.context_parallel import dual_form_fwd_cp
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                            world_size=1, timeout=datetime.timedelta(seconds=60))
+    try:
+        x = inp.dual_or_assoc_inputs(1, 2, 512, 64, seed=51, device="cuda",
+                                     normalise=("K", "V"), eta="sigmoid")
+        O, W = dual_form_fwd_cp(x["Q"], x["K"], x["V"], x["eta"], x["W0"], C=16)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    f = lambda t: t.float().cpu().numpy()
+    Or, Wr = orc.dual_form(f(x["Q"]), f(x["K"]), f(x["V"]), x["eta"].cpu().numpy(),
+                           x["W0"].cpu().numpy(), 16)
+    assert max_rel_l2(O, Or, 2) <= TOL and max_rel_l2(W, Wr, 2) <= TOL
+
+
 @pytest.mark.parametrize("slices,dtype", [(2, "bf16"), (4, "bf16"), (3, "f32")])
 def test_dual_form_slices_emulated_on_one_gpu(cuda_lib, slices, dtype):
     """The dual form's context-parallel pieces on one GPU: every slice's affine maps
