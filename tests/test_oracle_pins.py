@@ -466,6 +466,20 @@ def test_dual_segmented_rejects_bad_segment_lengths():
             orc.dual_form_segmented_stream(Q, K, V, 0.1, None, 4, L)
 
 
+def test_dual_segment_maps_compose():
+    """The map of two consecutive segments is the composition of their maps:
+    (A2, B2) o (A1, B1) = (A2 A1, A2 B1 + B2), for any split at a chunk boundary."""
+    T, d, C = 24, 4, 4
+    K, V = _rand(T, d, scale=0.5), _rand(T, d)
+    eta = rng.uniform(0.05, 0.6, T)
+    A, B = orc.dual_segment_maps_stream(K, V, eta, C)
+    for cut in (4, 12, 20):
+        A1, B1 = orc.dual_segment_maps_stream(K[:cut], V[:cut], eta[:cut], C)
+        A2, B2 = orc.dual_segment_maps_stream(K[cut:], V[cut:], eta[cut:], C)
+        np.testing.assert_allclose(A2 @ A1, A, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(A2 @ B1 + B2, B, rtol=1e-12, atol=1e-13)
+
+
 # ----------------------------------------------------------------------------- dual-form backward
 def _dual_loss(Q, K, V, eta, W0, dO, G, C):
     """The scalar whose gradients the dual-form backward returns, from the forward only."""
@@ -600,6 +614,25 @@ def test_dual_backward_pins_catch_planted_mistakes():
     for bad in ((True, False, False), (False, True, False), (False, False, True)):
         dq, dw0 = sweep(*bad)
         assert not (np.allclose(dq, fd_dq, rtol=1e-4) and np.allclose(dw0, fd_w0, rtol=1e-4))
+
+
+def test_backwards_are_linear_in_the_incoming_gradients():
+    """Both backwards are linear maps of (dO, dState): the gradients for a combination of two
+    incoming gradients are the same combination of their gradients (catches a term that squares
+    or drops an incoming gradient)."""
+    T, d, C = 8, 3, 4
+    Q, K, V = _rand(T, d), _rand(T, d, scale=0.5), _rand(T, d)
+    eta = rng.uniform(0.05, 0.5, T)
+    W0 = _rand(d, d, scale=0.3)
+    dO1, dO2 = _rand(T, d), _rand(T, d)
+    G1, G2 = _rand(d, d), _rand(d, d)
+    a, b = 0.7, -1.3
+    for fn in (lambda o, g: orc.dual_backward_stream(Q, K, V, eta, W0, o, g, C),
+               lambda o, g: orc.assoc_backward_stream(Q, K, V, eta, W0, o, g)):
+        g1, g2 = fn(dO1, G1), fn(dO2, G2)
+        gc = fn(a * dO1 + b * dO2, a * G1 + b * G2)
+        for x1, x2, xc in zip(g1, g2, gc):
+            np.testing.assert_allclose(xc, a * x1 + b * x2, rtol=1e-11, atol=1e-12)
 
 
 # ----------------------------------------------------------------------------- momentum
