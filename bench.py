@@ -3,7 +3,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 A step is one call of the operation over one batch of synthetic input (default workload: the
-TTT-Linear dual form at the 125M-layer shape, B=8 H=12 T=2048 d=64 C=16, bf16). Inputs are
+associative linear-attention mode, B=4 H=16 T=65536 d=128 C=64, bf16: of the single-GPU
+workloads it moves the most tokens and bytes per call). Inputs are
 resident in HBM when timing starts; L2 is flushed (a 256 MiB write) before every timed step.
 Each step is bracketed by CUDA events on the launching stream; the sum over K steps, max over
 ranks, is the timed region, itself bracketed by a barrier and a device synchronize.
@@ -36,7 +37,7 @@ METRIC_BWD = "TTT-layer bwd tokens/s on 1 B200; % of bf16 tensor-peak/HBM roofli
 
 def metric_of(w) -> str:
     return METRIC_BWD if w.kind.endswith("_bwd") else METRIC
-DEFAULT_WORKLOAD = "dual_bf16_B8H12T2048_d64C16"
+DEFAULT_WORKLOAD = "assoc_bf16_B4H16T65536_d128C64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DOMINANT_KERNEL = {"dual": ("dual_mma_kernel", "dual_mma.cu"),
                    "dual_seg": ("dual_mma_kernel", "dual_mma.cu"),
@@ -290,58 +291,146 @@ def e2e_measure(w, x, steps: int, warmup: int):
     return ms, h2d, d2h
 
 
+STREAM_KINDS = ("dual", "dual_seg", "assoc", "assoc_bwd", "assoc_momentum", "dual_bwd",
+                "dual_seg_bwd")
+ORACLE_ROUTINE = {"dual": "dual-form per-chunk loop", "dual_seg": "dual-form per-chunk loop",
+                  "assoc": "sequential recurrence", "assoc_momentum": "momentum recurrence",
+                  "dual_bwd": "dual-form chunk adjoint sweeps",
+                  "dual_seg_bwd": "dual-form chunk adjoint sweeps",
+                  "assoc_bwd": "adjoint sweeps of the recurrence"}
+
+
+def host_cores() -> int:
+    """Cores this process may run on (its affinity mask)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _pool_init(root: str):
+    # one BLAS thread per worker: the workers already occupy every core
+    for v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[v] = "1"
+    if root not in sys.path:
+        sys.path.insert(0, root)
+
+
+def _oracle_streams_task(kind: str, C: int, eta_const, beta, arrays: dict) -> int:
+    """Runs the fp64 oracle over a group of whole (b,h) streams in a pool worker; returns the
+    token-head count processed. `arrays` holds [n, tokens, d] slices (and [n, tokens] rates)."""
+    from oracle import ttt_oracle as orc
+
+    Q, K, V = arrays["Q"], arrays["K"], arrays["V"]
+    n, ncol = Q.shape[0], Q.shape[1]
+    for i in range(n):
+        e = eta_const if arrays.get("eta") is None else arrays["eta"][i]
+        if kind in ("dual", "dual_seg"):
+            orc.dual_form_stream(Q[i], K[i], V[i], e, arrays["W0"][i], C)
+        elif kind == "assoc_momentum":
+            orc.assoc_momentum_stream(Q[i], K[i], V[i], e, beta, None, None)
+        elif kind in ("dual_bwd", "dual_seg_bwd"):
+            orc.dual_backward_stream(Q[i], K[i], V[i], e, arrays["W0"][i], arrays["dO"][i],
+                                     arrays["G"][i], C)
+        elif kind == "assoc_bwd":
+            orc.assoc_backward_stream(Q[i], K[i], V[i], e, None, arrays["dO"][i],
+                                      arrays["G"][i])
+        else:
+            orc.assoc_recurrence_stream(Q[i], K[i], V[i], e, None)
+    return n * ncol
+
+
+_POOL = {}
+
+
+def close_oracle_pools():
+    for p in _POOL.values():
+        p.close()
+        p.join()
+    _POOL.clear()
+
+
+def oracle_pool(cores: int):
+    """A process pool for the oracle, started with spawn (a forked child of a process that has
+    used CUDA can hang)."""
+    import multiprocessing as mp
+
+    if cores not in _POOL:
+        _POOL[cores] = mp.get_context("spawn").Pool(cores, initializer=_pool_init,
+                                                    initargs=(ROOT,))
+    return _POOL[cores]
+
+
 def oracle_sample(w, x, budget_s: float, cursor: list):
-    """Runs the fp64 oracle on a bounded sample of the workload; returns (tokens, seconds,
-    threads, description). The sample is whole (b,h) streams (a prefix of chunks when one
-    stream exceeds the budget) or output-column subsets of the In-Place workload."""
+    """Runs the fp64 oracle on a bounded sample of the workload on the host's cores; returns
+    (tokens, seconds, cores, description).
+
+    Stream workloads: whole (b,h) streams (a prefix of chunks when one stream exceeds the
+    budget), in groups spread over a spawn-started process pool with one worker per core,
+    timed by wall clock from the first submission to the last result; waves of groups are
+    submitted until the budget is spent. In-Place: output-column subsets (columns are
+    independent), one process with the BLAS library's own threads."""
     import numpy as np
 
     from oracle import ttt_oracle as orc
     from weight_linear_attention_ttt_b200 import inputs as inp
 
-    threads = os.cpu_count() or 1
-    t0 = time.perf_counter()
-    if w.kind in ("dual", "dual_seg", "assoc", "assoc_bwd", "assoc_momentum", "dual_bwd",
-                  "dual_seg_bwd"):
+    if w.kind in STREAM_KINDS:
+        import torch
+
+        cores = host_cores()
         streams = [(b, h) for b in range(w.B) for h in range(w.H)]
-        Q, K, V = (x[k].float().cpu().numpy() for k in ("Q", "K", "V"))
-        eta = None if x["eta"] is None else x["eta"].cpu().numpy()
-        W0 = x["W0"].cpu().numpy()
-        if w.kind in ("assoc_bwd", "dual_bwd", "dual_seg_bwd"):
-            dO = x["dO"].float().cpu().numpy()
-            G = x["dS_out" if w.kind == "assoc_bwd" else "dW_out"].cpu().numpy()
-        # probe the cost of one chunk-run of one stream to size the sample
-        tok = 0
-        n_streams = 0
         ncol = w.T if w.kind in ("dual", "dual_seg", "dual_bwd", "dual_seg_bwd") else min(w.T, 4096)
+        eta = x.get("eta")
+        grad_key = "dS_out" if w.kind == "assoc_bwd" else "dW_out"
+
+        def group(idx):
+            sel = [streams[i % len(streams)] for i in idx]
+            bi = torch.tensor([s[0] for s in sel])
+            hi = torch.tensor([s[1] for s in sel])
+            arr = {k: x[k][bi, hi, :ncol].double().numpy() for k in ("Q", "K", "V")}
+            arr["eta"] = None if eta is None else eta[bi, hi, :ncol].double().numpy()
+            arr["W0"] = x["W0"][bi, hi].double().numpy()
+            if w.kind in ("assoc_bwd", "dual_bwd", "dual_seg_bwd"):
+                arr["dO"] = x["dO"][bi, hi, :ncol].double().numpy()
+                arr["G"] = x[grad_key][bi, hi].double().numpy()
+            return arr
+
+        pool = oracle_pool(cores)
+        # size a group so that one takes roughly a tenth of the budget: time one stream first
+        t0 = time.perf_counter()
+        _oracle_streams_task(w.kind, w.C, w.eta_const, inp.MOMENTUM_BETA,
+                             group([cursor[0] % len(streams)]))
+        per_stream = max(1e-4, time.perf_counter() - t0)
+        per_group = max(1, min(len(streams), int(0.1 * budget_s / per_stream)))
+        tok, waves = 0, 0
+        t0 = time.perf_counter()
         while True:
-            b, h = streams[cursor[0] % len(streams)]
-            cursor[0] += 1
-            e = w.eta_const if eta is None else eta[b, h, :ncol]
-            if w.kind in ("dual", "dual_seg"):
-                orc.dual_form_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
-                                     W0[b, h], w.C)
-            elif w.kind == "assoc_momentum":
-                orc.assoc_momentum_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
-                                          inp.MOMENTUM_BETA, None, None)
-            elif w.kind in ("dual_bwd", "dual_seg_bwd"):
-                orc.dual_backward_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
-                                         W0[b, h], dO[b, h, :ncol], G[b, h], w.C)
-            elif w.kind == "assoc_bwd":
-                orc.assoc_backward_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
-                                          None, dO[b, h, :ncol], G[b, h])
-            else:
-                orc.assoc_recurrence_stream(Q[b, h, :ncol], K[b, h, :ncol], V[b, h, :ncol], e,
-                                            None)
-            tok += ncol
-            n_streams += 1
-            if time.perf_counter() - t0 >= budget_s or n_streams >= len(streams):
+            jobs = []
+            for _ in range(cores):
+                idx = list(range(cursor[0], cursor[0] + per_group))
+                cursor[0] += per_group
+                jobs.append(pool.apply_async(_oracle_streams_task,
+                                             (w.kind, w.C, w.eta_const, inp.MOMENTUM_BETA,
+                                              group(idx))))
+            tok += sum(j.get() for j in jobs)
+            waves += 1
+            if time.perf_counter() - t0 >= budget_s:
                 break
-        desc = (f"{n_streams} (b,h) stream(s) x {ncol} tokens of the workload, "
-                f"{ {'dual': 'dual-form per-chunk loop', 'dual_seg': 'dual-form per-chunk loop', 'assoc': 'sequential recurrence', 'assoc_momentum': 'momentum recurrence', 'dual_bwd': 'dual-form chunk adjoint sweeps', 'dual_seg_bwd': 'dual-form chunk adjoint sweeps'}.get(w.kind, 'adjoint sweeps of the recurrence')}"
-                f", numpy fp64, 1 thread")
-        return tok / w.H, time.perf_counter() - t0, 1, desc
+        sec = time.perf_counter() - t0
+        n_streams = tok // ncol
+        desc = (f"{n_streams} (b,h) stream-runs x {ncol} tokens of the workload "
+                f"({waves} wave(s) of {cores} groups of {per_group} streams), "
+                f"{ORACLE_ROUTINE[w.kind]}, numpy fp64, {cores} worker processes")
+        return tok / w.H, sec, cores, desc
     # In-Place: every 80th output column over all chunks (columns are independent)
+    try:
+        from threadpoolctl import threadpool_info
+
+        blas = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        threads = max(blas) if blas else 1
+    except Exception:
+        threads = 1
     cols = np.arange(cursor[0] % 80, w.D, 80)
     cursor[0] += 1
     Z = x["Z"].float().cpu().numpy()
@@ -357,7 +446,7 @@ def oracle_sample(w, x, budget_s: float, cursor: list):
     dt = time.perf_counter() - t0
     frac = len(cols) / w.D
     return w.T * frac, dt, threads, (f"{len(cols)} of {w.D} output columns over all "
-                                     f"{w.T // w.C} chunks, numpy fp64 BLAS")
+                                     f"{w.T // w.C} chunks, numpy fp64 BLAS, {threads} threads")
 
 
 # ----------------------------------------------------------------------------- arms
@@ -454,7 +543,10 @@ def run_ours(args, w, rank, world, local_rank):
     pk, pk_kind = peaks()
     kname, ksrc = DOMINANT_KERNEL[w.kind]
     launches_per_step = launches / args.steps
-    if w.kind.startswith("inplace"):
+    # the roofline is the slower of the flops at the tensor peak and the bytes at HBM bandwidth
+    t_flops = algo["flops"] / (pk["bf16_tflops"] * 1e12)
+    t_bytes = algo["bytes"] / (pk["hbm_gbs"] * 1e9)
+    if t_flops > t_bytes:
         achieved = algo["flops"] / (ms_per_step / 1e3) / 1e12
         peak = pk["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -464,6 +556,7 @@ def run_ours(args, w, rank, world, local_rank):
         peak = pk["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak}
+    roof["roofline_us"] = 1e6 * max(t_flops, t_bytes)
     sha = kernel_source_sha(ksrc)
     roof.update({"traffic": measured_traffic(w.name, kname, sha), "kernel": kname,
                  "peak_source": f"{pk_kind} (MEASURED_PEAKS.json)" if pk_kind == "measured"
@@ -515,7 +608,10 @@ def main(argv=None):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
-        return run_reference(args, w, rank, world)
+        try:
+            return run_reference(args, w, rank, world)
+        finally:
+            close_oracle_pools()
     import torch
     import torch.distributed as dist
 
@@ -526,6 +622,7 @@ def main(argv=None):
     try:
         return run_ours(args, w, rank, world, local_rank)
     finally:
+        close_oracle_pools()
         if world > 1:
             dist.destroy_process_group()
 

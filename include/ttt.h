@@ -299,7 +299,7 @@ int ttt_state_prefix_sum(const float* S0, const float* increments, int n_increme
  *  W0    [Dff,D] bf16 initial W_down.
  *  O     [T,D]  bf16 output.
  *  W_out [Dff,D] fp32 final W_down (the running fp32 master).
- *  Supported: T % C == 0; C % 128 == 0; Dff % 128 == 0; D % 256 == 0.
+ *  Supported: T % C == 0; C % 128 == 0; Dff % 128 == 0; D % 64 == 0.
  *  Workspace: inplace_ttt_workspace_size() bytes (bf16 copy of the running W).
  * ------------------------------------------------------------------------------------------ */
 size_t inplace_ttt_workspace_size(int T, int Dff, int D, int C);
@@ -327,7 +327,11 @@ int inplace_ttt_chunk_fwd(const void* Z, const void* Vhat, const void* W0, float
  *    before they are read. Calls whose work overlaps on the GPU (different streams, or threads
  *    racing on one device) race on the array: serialise them.
  *  - The first call on each device looks up the array's device address (a one-time runtime
- *    query for the current device). Make that first call before any stream capture begins.
+ *    query for the current device and its context; it is made again after a device reset,
+ *    which gives the device a new context). Make that first call before any stream capture
+ *    begins.
+ *  - Errors name this function in ttt_last_error_message(); the shape, pointer and alignment
+ *    checks are those of inplace_ttt_chunk_fwd.
  * ------------------------------------------------------------------------------------------ */
 size_t inplace_ttt_noalloc_max_scratch_bytes(void);
 int inplace_ttt_chunk_fwd_noalloc(const void* Z, const void* Vhat, const void* W0, float eta,

@@ -75,15 +75,20 @@ def test_forced_superchunk_counts_agree(cuda_lib, monkeypatch, parts):
 RACE_TRIPWIRE = 6e-3
 
 
-def test_full_associative_workload_sampled_streams(cuda_lib):
+def test_full_associative_workload_every_stream(cuda_lib):
+    """Every stream of the full associative workload against the oracle, one batch item (16
+    streams, both superchunks of each) per oracle call."""
     w = inp.WORKLOADS["assoc_bf16_B4H16T65536_d128C64"]
     x = inp.make_inputs(w, "cuda")
     O, S = run(x)
-    streams = [(0, 0), (1, 7), (3, 15)]
-    eo, es = check(x, O, S, streams=streams)
-    print(f"associative workload (3 sampled streams): max rel L2 O {eo:.2e} S {es:.2e}")
-    assert eo <= RACE_TRIPWIRE and es <= RACE_TRIPWIRE, (eo, es)
-    assert torch.isfinite(O.float()).all() and torch.isfinite(S).all()
+    worst = (0.0, 0.0)
+    for b in range(w.B):
+        sub = {k: (v[b:b + 1] if torch.is_tensor(v) else v) for k, v in x.items()}
+        eo, es = check(sub, O[b:b + 1], S[b:b + 1])
+        worst = (max(worst[0], eo), max(worst[1], es))
+    print(f"associative workload (all {w.B * w.H} streams): max rel L2 O {worst[0]:.2e} "
+          f"S {worst[1]:.2e}")
+    assert worst[0] <= RACE_TRIPWIRE and worst[1] <= RACE_TRIPWIRE, worst
     assert ttt.read_device_error() == 0
 
 

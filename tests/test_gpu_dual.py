@@ -68,13 +68,17 @@ def test_bf16_125m_layer_workload(cuda_lib):
 
 
 def test_bf16_long_context_workload(cuda_lib):
+    """Every stream of the 1.3B-layer long-context shape against the oracle, one batch item at a
+    time (32 streams per oracle call keeps the host memory small)."""
     w, x = workload("dual_bf16_B2H32T32768_d64C16")
     O, W = run(x, w.C)
-    streams = [(0, 0), (0, 17), (1, 5), (1, 31)]
-    eo, ew = check(x, w.C, O, W, TOL["bf16"], streams)
-    print(f"dual long-context workload (4 sampled streams): max rel L2 O {eo:.2e} W {ew:.2e}")
-    # every stream is finite and was written
-    assert torch.isfinite(O.float()).all() and torch.isfinite(W).all()
+    worst = (0.0, 0.0)
+    for b in range(w.B):
+        sub = {k: (v[b:b + 1] if torch.is_tensor(v) else v) for k, v in x.items()}
+        eo, ew = check(sub, w.C, O[b:b + 1], W[b:b + 1], TOL["bf16"])
+        worst = (max(worst[0], eo), max(worst[1], ew))
+    print(f"dual long-context workload (all {w.B * w.H} streams): max rel L2 O {worst[0]:.2e} "
+          f"W {worst[1]:.2e}")
     assert ttt.read_device_error() == 0
 
 

@@ -51,7 +51,7 @@ def test_full_wdown_workload_column_subset(cuda_lib):
     w = inp.WORKLOADS["inplace_bf16_T32768_Dff9728_D2560_C1024"]
     x = inp.make_inputs(w, "cuda")
     O, W = run(x, w.C)
-    cols = np.arange(3, w.D, 80)
+    cols = np.arange(3, w.D, 20)  # every 20th column: each is exact on its own
     eo, ew = check(x, w.C, O, W, cols=cols)
     print(f"in-place W_down workload ({len(cols)} of {w.D} columns): max rel L2 O {eo:.2e} "
           f"W {ew:.2e}")

@@ -8,21 +8,31 @@ import pytest
 import torch
 
 import weight_linear_attention_ttt_b200 as ttt
-from _helpers import max_rel_l2
 from weight_linear_attention_ttt_b200 import inputs as inp
 
 pytestmark = pytest.mark.gpu
-TOL = 1e-2  # the bf16 tolerance of the parity tests
 
 
 def _compare(x, C):
+    """Runs the workspace entry point, then the allocation-free one into NaN-filled outputs;
+    both run the same kernels on the same inputs, so their results must be bit-identical. The
+    allocation-free call must leave the device's free memory and torch's allocation unchanged
+    and launch one kernel per chunk, like the workspace call."""
+    T = x["Z"].shape[0]
     O_ref, W_ref = ttt.inplace_ttt_chunk_fwd(x["Z"], x["Vhat"], x["W0"], x["eta"], C=C)
     O = torch.full_like(O_ref, float("nan"))
     W = torch.full_like(W_ref, float("nan"))
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    n0 = ttt.launch_count()
     ttt.inplace_ttt_chunk_fwd_noalloc(x["Z"], x["Vhat"], x["W0"], x["eta"], C=C, O=O, W_out=W)
     torch.cuda.synchronize()
-    assert max_rel_l2(O.t().contiguous(), O_ref.t().contiguous(), 1) <= TOL
-    assert max_rel_l2(W.t().contiguous(), W_ref.t().contiguous(), 1) <= TOL
+    assert ttt.launch_count() - n0 == T // C
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.equal(O, O_ref)
+    assert torch.equal(W, W_ref)
 
 
 def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row(cuda_lib):
@@ -47,4 +57,11 @@ def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_lib):
                                            512, 4096, 4096, 256, None)
     assert st == 2
     assert b"scratch" in lib.ttt_last_error_message()
+    assert lib.ttt_last_error_message().startswith(b"inplace_ttt_chunk_fwd_noalloc")
+    # a shape error found by the shared validation names the function the caller used
+    st = lib.inplace_ttt_chunk_fwd_noalloc(v(1 << 20), v(2 << 20), v(3 << 20),
+                                           ctypes.c_float(1e-3), v(4 << 20), v(5 << 20),
+                                           256, 128, 96, 128, None)
+    assert st == 2
+    assert lib.ttt_last_error_message().startswith(b"inplace_ttt_chunk_fwd_noalloc")
     assert ttt.launch_count() == n0
