@@ -83,6 +83,25 @@ int ttt_version(void);
 /* Number of kernels this library has launched in this process (all entry points, all devices). */
 uint64_t ttt_launch_count(void);
 
+/* Kernel-variant choices, process-wide, for comparing variants (0 = the library's automatic
+ * choice, the default). Keys:
+ *   "dual_column_split"  CTAs per stream of the dual form: 1, 2 or 4 (4 only for d = 64).
+ *   "dual_kernel"        dual form with bf16 inputs and C = 16: 1 = all products on warp MMAs
+ *                        (one warp per 16 columns), 2 = the same on chain/output warp pairs,
+ *                        3 = chain on warp MMAs with the outputs per 128-token stage on the
+ *                        tcgen05 tensor cores (d = 64 only; what 0 picks for d = 64).
+ *   "dual_warp_cols"     dual_kernel 1 with d = 64: 8 or 16 output columns per warp.
+ *   "dual_stage_chunks"  dual_kernel 1 with d = 64 and 8 columns per warp: 4 or 8 chunks per
+ *                        pipeline stage.
+ *   "assoc_parts"        superchunks per stream of the associative mode (must divide T / C).
+ * Every variant computes the same operation within the same tolerance. ttt_set_tuning returns
+ * TTT_ERR_INVALID_ARG for an unknown key or a negative value; ttt_get_tuning returns -1 for an
+ * unknown key; ttt_reset_tuning restores every key to 0. Not synchronised with calls in flight
+ * on other threads: set choices before the calls they should affect. */
+int ttt_set_tuning(const char* key, int value);
+int ttt_get_tuning(const char* key);
+void ttt_reset_tuning(void);
+
 /* Reads and clears the current device's error word. Bit 0 set means a bounded device-side wait
  * gave up (a kernel stopped early; its outputs are incomplete). SYNCHRONOUS: waits for all work
  * on the device to finish. Returns TTT_OK or TTT_ERR_CUDA. */

@@ -23,3 +23,12 @@ def cuda_lib():
 
     ttt.load_library()
     return ttt
+
+
+@pytest.fixture
+def tuning(cuda_lib):
+    """set(key, value) for the library's kernel-variant choices; every choice goes back to the
+    automatic one when the test ends."""
+    cuda_lib.reset_tuning()
+    yield cuda_lib.set_tuning
+    cuda_lib.reset_tuning()

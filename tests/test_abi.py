@@ -246,3 +246,30 @@ def test_dual_context_parallel_pieces_validation(lib):
     assert fold(upto=5) == 1 and fold(upto=-1) == 1 and fold(n=0) == 1 and fold(Am=0) == 1
     assert fold(d=48) == 2 and fold(Wout=2 * A + 64) == 1 and fold(Wout=A + 64) == 1
     assert lib.ttt_launch_count() == 0
+
+
+def test_tuning_choices_set_get_reset(lib):
+    """Kernel-variant choices are explicit library state (nothing is read from the
+    environment): unknown keys and negative values are refused, reset restores 0."""
+    try:
+        assert lib.ttt_get_tuning(b"dual_kernel") == 0
+        assert lib.ttt_set_tuning(b"dual_kernel", 3) == 0
+        assert lib.ttt_get_tuning(b"dual_kernel") == 3
+        assert lib.ttt_set_tuning(b"assoc_parts", 4) == 0
+        assert lib.ttt_set_tuning(b"no_such_key", 1) == 1
+        assert b"unknown key" in lib.ttt_last_error_message()
+        assert lib.ttt_set_tuning(b"dual_column_split", -1) == 1
+        assert lib.ttt_get_tuning(b"no_such_key") == -1
+        lib.ttt_reset_tuning()
+        for key in (b"dual_column_split", b"dual_kernel", b"dual_warp_cols",
+                    b"dual_stage_chunks", b"assoc_parts"):
+            assert lib.ttt_get_tuning(key) == 0
+    finally:
+        lib.ttt_reset_tuning()
+
+
+def test_library_reads_no_environment():
+    """No kernel variant or tuning choice comes from environment variables."""
+    src = glob.glob(os.path.join(ROOT, "weight_linear_attention_ttt_b200", "csrc", "*"))
+    for f in src:
+        assert "getenv" not in open(f, encoding="utf-8").read(), f

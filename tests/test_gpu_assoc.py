@@ -56,9 +56,9 @@ def test_small_shapes_default_parts(cuda_lib, B, H, T):
 
 
 @pytest.mark.parametrize("parts", ["1", "2", "4", "16"])
-def test_forced_superchunk_counts_agree(cuda_lib, monkeypatch, parts):
+def test_forced_superchunk_counts_agree(cuda_lib, tuning, parts):
     """The two-pass prefix scan over P superchunks gives the oracle's result for every P."""
-    monkeypatch.setenv("TTT_ASSOC_PARTS", parts)
+    tuning("assoc_parts", int(parts))
     x = make(1, 2, 1024, seed=77)
     S0 = torch.randn(1, 2, 128, 128, device="cuda", generator=torch.Generator("cuda").manual_seed(3))
     n0 = ttt.launch_count()

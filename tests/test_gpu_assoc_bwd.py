@@ -76,9 +76,9 @@ def test_zero_and_tiny_rates(cuda_lib):
 
 
 @pytest.mark.parametrize("parts", ["1", "2", "4", "16"])
-def test_forced_superchunk_counts(cuda_lib, monkeypatch, parts):
+def test_forced_superchunk_counts(cuda_lib, tuning, parts):
     """The reverse-order passes split into superchunks give the oracle's gradients for every P."""
-    monkeypatch.setenv("TTT_ASSOC_PARTS", parts)
+    tuning("assoc_parts", int(parts))
     x = make(1, 2, 1024, seed=77)
     check(x, run(x))
 

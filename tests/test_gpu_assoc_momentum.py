@@ -54,10 +54,10 @@ def test_momentum_matches_oracle(cuda_lib, B, H, T, beta):
 
 
 @pytest.mark.parametrize("parts", ["1", "2", "4", "16"])
-def test_forced_superchunk_counts(cuda_lib, monkeypatch, parts):
+def test_forced_superchunk_counts(cuda_lib, tuning, parts):
     """Both passes split into superchunks (the decayed one carrying its state across them with
     the superchunk decay) give the oracle's results for every split."""
-    monkeypatch.setenv("TTT_ASSOC_PARTS", parts)
+    tuning("assoc_parts", int(parts))
     x = make(1, 2, 1024, seed=31)
     check(x, 0.9, run(x, 0.9))
     assert ttt.read_device_error() == 0

@@ -102,9 +102,9 @@ def test_sweep_fp32(cuda_lib, d, C, m):
     check(x, C, O, W, TOL["f32"])
 
 
-@pytest.mark.parametrize("T", [16, 48, 64, 80, 112, 1040])
+@pytest.mark.parametrize("T", [16, 48, 64, 80, 112, 128, 272, 1040])
 def test_ragged_stage_tails(cuda_lib, T):
-    """T that is not a multiple of the kernel's 64-token pipeline stage (partial last stage)."""
+    """T that is not a multiple of the kernels' pipeline stages (partial last stage)."""
     x = inp.dual_or_assoc_inputs(2, 3, T, 64, seed=T, device="cuda", normalise=("K", "V"))
     O, W = run(x, 16)
     check(x, 16, O, W, TOL["bf16"])
@@ -144,19 +144,50 @@ def test_determinism_permutation_and_state_carry(cuda_lib):
     assert torch.equal(torch.cat([Oa, Ob], dim=2), O1) and torch.equal(Wb, W1)
 
 
-def test_column_split_variants_agree_bitwise(cuda_lib, monkeypatch):
-    x = inp.dual_or_assoc_inputs(1, 4, 256, 64, seed=5, device="cuda", normalise=("K", "V"))
-    outs = []
-    for split in ("1", "2"):
-        monkeypatch.setenv("TTT_DUAL_COLUMN_SPLIT", split)
-        outs.append(run(x, 16))
-    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
-    x = inp.dual_or_assoc_inputs(1, 2, 128, 128, seed=6, device="cuda", normalise=("K", "V"))
-    outs = []
-    for split in ("1", "2"):
-        monkeypatch.setenv("TTT_DUAL_COLUMN_SPLIT", split)
-        outs.append(run(x, 16))
-    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+def test_column_split_variants_agree_bitwise(cuda_lib, tuning):
+    """The all-warp-MMA kernels compute every column the same way whether a stream sits on one
+    CTA or is split over two."""
+    tuning("dual_kernel", 1)
+    for d, T in ((64, 256), (128, 128)):
+        x = inp.dual_or_assoc_inputs(1, 4, T, d, seed=d, device="cuda", normalise=("K", "V"))
+        outs = []
+        for split in (1, 2):
+            tuning("dual_column_split", split)
+            outs.append(run(x, 16))
+        assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_tensor_core_form_column_splits(cuda_lib, tuning):
+    """The stage-form kernel (chain on warp MMAs, outputs on tcgen05) with 1, 2 and 4 CTAs per
+    stream: the chain of a column is the same arithmetic in every split (final W bit-identical),
+    and every split meets the oracle on full and partial 128-token stages."""
+    tuning("dual_kernel", 3)
+    for T in (16, 144, 400):
+        x = inp.dual_or_assoc_inputs(2, 3, T, 64, seed=T + 11, device="cuda",
+                                     normalise=("K", "V"))
+        outs = []
+        for split in (1, 2, 4):
+            tuning("dual_column_split", split)
+            O, W = run(x, 16)
+            check(x, 16, O, W, TOL["bf16"])
+            outs.append((O, W))
+        for O, W in outs[1:]:
+            assert torch.equal(W, outs[0][1])
+            assert max_rel_l2(O, outs[0][0], 2) < 1e-3
+        assert ttt.read_device_error() == 0
+
+
+def test_tensor_core_and_warp_forms_agree(cuda_lib, tuning):
+    """The stage form regroups the output sum (the earlier chunks of a stage enter through the
+    masked scores instead of the chunk-start state); the chain is the same, so W agrees bit for
+    bit and O within the bf16 rounding of the regrouped terms."""
+    x = inp.dual_or_assoc_inputs(2, 4, 1024, 64, seed=31, device="cuda", normalise=("K", "V"))
+    tuning("dual_kernel", 1)
+    Ow, Ww = run(x, 16)
+    tuning("dual_kernel", 3)
+    Ot, Wt = run(x, 16)
+    assert torch.equal(Ww, Wt)
+    assert max_rel_l2(Ot, Ow, 2) < 5e-3
 
 
 def test_degenerate_cases(cuda_lib):
@@ -195,31 +226,31 @@ def test_invalid_calls_raise_before_launch(cuda_lib):
     assert ttt.launch_count() == n0
 
 
-@pytest.mark.parametrize("form", ["single", "pair"])
-@pytest.mark.parametrize("warp_cols", ["8", "16"])
-@pytest.mark.parametrize("split", ["1", "2"])
-def test_kernel_variants_match_oracle(cuda_lib, monkeypatch, warp_cols, split, form):
-    """Every tensor-core variant (8 or 16 output columns per warp, one or two CTAs per stream,
+@pytest.mark.parametrize("form", [1, 2])
+@pytest.mark.parametrize("warp_cols", [8, 16])
+@pytest.mark.parametrize("split", [1, 2])
+def test_kernel_variants_match_oracle(cuda_lib, tuning, warp_cols, split, form):
+    """Every all-warp-MMA variant (8 or 16 output columns per warp, one or two CTAs per stream,
     chain and outputs on one warp or on a warp pair) meets the bf16 tolerance on full and partial
     pipeline stages."""
-    if form == "pair" and warp_cols == "8":
+    if form == 2 and warp_cols == 8:
         pytest.skip("the warp-pair form exists for 16-column warps")
-    monkeypatch.setenv("TTT_DUAL_WARP_COLS", warp_cols)
-    monkeypatch.setenv("TTT_DUAL_COLUMN_SPLIT", split)
-    monkeypatch.setenv("TTT_DUAL_KERNEL", form)
+    tuning("dual_warp_cols", warp_cols)
+    tuning("dual_column_split", split)
+    tuning("dual_kernel", form)
     for T in (144, 512):
         x = inp.dual_or_assoc_inputs(2, 3, T, 64, seed=T + 3, device="cuda", normalise=("K", "V"))
         O, W = run(x, 16)
         check(x, 16, O, W, TOL["bf16"])
 
 
-def test_pair_and_single_forms_agree_bitwise(cuda_lib, monkeypatch):
+def test_pair_and_single_forms_agree_bitwise(cuda_lib, tuning):
     """The warp-pair form performs the single-warp form's arithmetic in the same order."""
     x = inp.dual_or_assoc_inputs(2, 3, 400, 64, seed=21, device="cuda", normalise=("K", "V"))
-    for split in ("1", "2"):
-        monkeypatch.setenv("TTT_DUAL_COLUMN_SPLIT", split)
+    for split in (1, 2):
+        tuning("dual_column_split", split)
         outs = []
-        for form in ("single", "pair"):
-            monkeypatch.setenv("TTT_DUAL_KERNEL", form)
+        for form in (1, 2):
+            tuning("dual_kernel", form)
             outs.append(run(x, 16))
         assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])

@@ -22,7 +22,7 @@ STATUS = {0: "TTT_OK", 1: "TTT_ERR_INVALID_ARG", 2: "TTT_ERR_UNSUPPORTED",
 # Every symbol include/ttt.h declares.
 EXPORTED_SYMBOLS = (
     "ttt_status_string", "ttt_last_error_message", "ttt_version", "ttt_launch_count",
-    "ttt_read_device_error",
+    "ttt_read_device_error", "ttt_set_tuning", "ttt_get_tuning", "ttt_reset_tuning",
     "ttt_linear_dual_workspace_size", "ttt_linear_dual_fwd",
     "ttt_linear_dual_seg_workspace_size", "ttt_linear_dual_seg_fwd",
     "ttt_assoc_scan_workspace_size", "ttt_assoc_scan_fwd", "ttt_assoc_state_fwd",
@@ -71,6 +71,12 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.ttt_launch_count.restype = ctypes.c_uint64
     lib.ttt_read_device_error.restype = c_int
     lib.ttt_read_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+    lib.ttt_set_tuning.restype = c_int
+    lib.ttt_set_tuning.argtypes = [ctypes.c_char_p, c_int]
+    lib.ttt_get_tuning.restype = c_int
+    lib.ttt_get_tuning.argtypes = [ctypes.c_char_p]
+    lib.ttt_reset_tuning.restype = None
+    lib.ttt_reset_tuning.argtypes = []
     state_args = [vp, vp, vp, fp, c_float, fp, vp, fp, c_int, c_int, c_int, c_int, c_int, c_int,
                   vp, c_size, vp]
     for name in ("ttt_linear_dual_fwd", "ttt_assoc_scan_fwd"):
@@ -562,6 +568,21 @@ def inplace_ttt_chunk_fwd_noalloc(Z, Vhat, W0, eta: float, *, C: int, O=None, W_
 def launch_count() -> int:
     """Kernels launched by the library so far in this process."""
     return int(load_library().ttt_launch_count())
+
+
+def set_tuning(key: str, value: int) -> None:
+    """Selects a kernel variant process-wide (0 = the library's automatic choice); the keys are
+    listed with ttt_set_tuning in include/ttt.h."""
+    _check("ttt_set_tuning", load_library().ttt_set_tuning(key.encode(), int(value)))
+
+
+def get_tuning(key: str) -> int:
+    return int(load_library().ttt_get_tuning(key.encode()))
+
+
+def reset_tuning() -> None:
+    """Restores every tuning choice to the automatic one."""
+    load_library().ttt_reset_tuning()
 
 
 def read_device_error() -> int:

@@ -587,11 +587,8 @@ __global__ void assoc_scan_kernel(const float* __restrict__ S0, float* inc, int 
 
 int choose_parts(int streams, int T) {
   const int nchunks = T / C;
-  const char* env = getenv("TTT_ASSOC_PARTS");  // tuning override
-  if (env) {
-    const int f = atoi(env);
-    if (f >= 1 && nchunks % f == 0) return f;
-  }
+  const int f = tuning(kTuneAssocParts);
+  if (f >= 1 && nchunks % f == 0) return f;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

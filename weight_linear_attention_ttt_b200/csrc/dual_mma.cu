@@ -29,8 +29,6 @@
 // Precision: W is fp32 throughout; its operand copy, E and the scores are rounded to bf16 once
 // per chunk for the tensor cores (relative error ~2^-9 per operand, fp32 accumulation).
 #include <algorithm>
-#include <cstdlib>
-
 #include <string>
 
 #include "internal.h"
@@ -589,19 +587,6 @@ int launch_cfg(const StateArgs& a, const LaunchCtx& ctx) {
   return kOk;
 }
 
-// CTAs per stream. Each CTA holds one stream's column slice for the whole sequence, and one CTA
-// fits per SM, so a stream is split over two SMs (halving each SM's share of the serial chain's
-// MMA work) only when all CTAs still fit in one wave.
-int column_split(int streams) {
-  const char* env = getenv("TTT_DUAL_COLUMN_SPLIT");  // tuning override: 1 or 2
-  const int forced = env ? atoi(env) : 0;
-  if (forced == 1 || forced == 2) return forced;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return 2 * streams <= sms ? 2 : 1;
-}
-
 }  // namespace
 
 bool dual_mma_supported(int d, int C, int dt) {
@@ -609,29 +594,42 @@ bool dual_mma_supported(int d, int C, int dt) {
 }
 
 int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
-  const int split = column_split(a.B * a.H);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int streams = a.B * a.H;
+  const int forced_split = tuning(kTuneDualColumnSplit);
+  const int kernel = tuning(kTuneDualKernel);
+  // d = 64: the chain on warp MMAs with the outputs per 128-token stage on tcgen05 (dual_tc.cu)
+  // measured fastest on the 125M- and 1.3B-layer shapes; the all-warp-MMA forms below remain
+  // selectable through ttt_set_tuning("dual_kernel", ...).
+  if (a.d == 64 && (kernel == kDualKernelAuto || kernel == kDualKernelTensor)) {
+    const int split = (forced_split == 1 || forced_split == 2 || forced_split == 4)
+                          ? forced_split
+                          : dual_tc_split(streams, sms);
+    return launch_dual_tc(a, split, ctx);
+  }
+  // CTAs per stream for the all-warp-MMA kernels. Each CTA holds one stream's column slice for
+  // the whole sequence, and one CTA fits per SM, so a stream is split over two SMs only when
+  // all CTAs still fit in one wave.
+  const int split =
+      (forced_split == 1 || forced_split == 2) ? forced_split : (2 * streams <= sms ? 2 : 1);
   switch (a.d) {
     case 32:
       return split == 2 ? launch_cfg<32, 2>(a, ctx) : launch_cfg<32, 4>(a, ctx);
     case 64: {
-      // 8 chunks per pipeline stage halve the per-stage costs (score pieces, barriers, first
-      // loads); measured faster on the 125M- and 1.3B-layer shapes. 4 is kept as an override.
-      // 16 columns per warp (W^T form, the warp computes its own causal scores) was measured
-      // faster than 8 columns per warp on the 125M- and 1.3B-layer shapes, with one CTA per
-      // stream and with two. 8 columns and 4-chunk stages remain as tuning overrides.
-      const char* env = getenv("TTT_DUAL_STAGE_CHUNKS");  // tuning override: 4 or 8
-      const char* wenv = getenv("TTT_DUAL_WARP_COLS");    // tuning override: 8 or 16
-      const int wcols = wenv ? atoi(wenv) : 16;
-      // Chain and output products on paired warps (dual_pair.cu) measured faster when a stream
-      // is split over two CTAs (two warp pairs per SM) and slower with one CTA per stream (four
-      // pairs per SM: the hand-off and the output warps' own Q/K loads double the shared-memory
-      // traffic). Either form can be forced.
-      const char* kenv = getenv("TTT_DUAL_KERNEL");      // tuning override: pair or single
-      const bool pair = kenv ? std::string(kenv) == "pair" : split == 2;
+      // 16 columns per warp (W^T form, the warp computes its own causal scores) with 8-chunk
+      // stages measured faster than 8 columns per warp; chain and output products on paired
+      // warps (dual_pair.cu) measured faster when a stream is split over two CTAs. The other
+      // forms are kept as tuning choices.
+      const int wcols = tuning(kTuneDualWarpCols) == 8 ? 8 : 16;
+      const bool pair = kernel == kDualKernelPair ? true
+                        : kernel == kDualKernelWarp ? false
+                                                    : split == 2;
       if (wcols == 16 && pair) return launch_dual_pair(a, ctx, split);
       if (wcols == 16)
         return split == 2 ? launch_cfg<64, 2, 8, 16>(a, ctx) : launch_cfg<64, 4, 8, 16>(a, ctx);
-      if (env && atoi(env) == 4)
+      if (tuning(kTuneDualStageChunks) == 4)
         return split == 2 ? launch_cfg<64, 4>(a, ctx) : launch_cfg<64, 8>(a, ctx);
       return split == 2 ? launch_cfg<64, 4, 8>(a, ctx) : launch_cfg<64, 8, 8>(a, ctx);
     }

@@ -61,6 +61,20 @@ struct LaunchCtx {
 };
 
 void count_launch(uint64_t n = 1);
+
+// Tuning choices set through ttt_set_tuning() (0 = the library's automatic choice). They exist to
+// compare kernel variants; nothing reads the environment.
+enum TuneKey : int {
+  kTuneDualColumnSplit = 0,   // CTAs per stream of the dual form: 1, 2 or 4
+  kTuneDualKernel,            // kDualKernel* below
+  kTuneDualWarpCols,          // all-warp-MMA dual form, d = 64: 8 or 16 columns per warp
+  kTuneDualStageChunks,       // all-warp-MMA dual form, d = 64, 8 columns: 4 or 8 chunks/stage
+  kTuneAssocParts,            // superchunks per stream of the associative mode
+  kTuneCount
+};
+enum DualKernel : int { kDualKernelAuto = 0, kDualKernelWarp = 1, kDualKernelPair = 2,
+                        kDualKernelTensor = 3 };
+int tuning(TuneKey key);
 // Records the detail returned by ttt_last_error_message() on this thread.
 void set_last_error(const std::string& msg);
 
@@ -78,6 +92,10 @@ bool dual_mma_supported(int d, int C, int dt);
 int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx);
 int launch_dual_pair(const StateArgs& a, const LaunchCtx& ctx, int split);
 int launch_dual_simt(const StateArgs& a, const LaunchCtx& ctx);
+// d = 64, C = 16, bf16: chain on warp MMAs, outputs per stage on tcgen05; split = CTAs per
+// stream (1, 2 or 4), dual_tc_split() the automatic choice.
+int dual_tc_split(int streams, int sms);
+int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx);
 
 // Associative mode.
 size_t assoc_workspace_bytes(int B, int H, int T, int d, int C);

@@ -20,6 +20,25 @@ void count_launch(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxe
 // Device error word written by bounded waits in the kernels (one per device context).
 __device__ unsigned g_device_error;
 
+static std::atomic<int> g_tuning[kTuneCount];
+int tuning(TuneKey key) { return g_tuning[key].load(std::memory_order_relaxed); }
+
+struct TuneName {
+  const char* name;
+  TuneKey key;
+};
+static const TuneName kTuneNames[] = {{"dual_column_split", kTuneDualColumnSplit},
+                                      {"dual_kernel", kTuneDualKernel},
+                                      {"dual_warp_cols", kTuneDualWarpCols},
+                                      {"dual_stage_chunks", kTuneDualStageChunks},
+                                      {"assoc_parts", kTuneAssocParts}};
+static int tune_key(const char* name) {
+  if (!name) return -1;
+  for (const auto& t : kTuneNames)
+    if (std::strcmp(t.name, name) == 0) return t.key;
+  return -1;
+}
+
 static thread_local std::string t_last_error;
 void set_last_error(const std::string& msg) { t_last_error = msg; }
 
@@ -164,6 +183,25 @@ const char* ttt_last_error_message(void) { return t_last_error.c_str(); }
 int ttt_version(void) { return 10000; }
 
 uint64_t ttt_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int ttt_set_tuning(const char* key, int value) {
+  const int k = ttt::tune_key(key);
+  if (k < 0)
+    return fail(TTT_ERR_INVALID_ARG,
+                std::string("ttt_set_tuning: unknown key ") + (key ? key : "(null)"));
+  if (value < 0) return fail(TTT_ERR_INVALID_ARG, "ttt_set_tuning: value must be >= 0");
+  ttt::g_tuning[k].store(value, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
+int ttt_get_tuning(const char* key) {
+  const int k = ttt::tune_key(key);
+  return k < 0 ? -1 : ttt::g_tuning[k].load(std::memory_order_relaxed);
+}
+
+void ttt_reset_tuning(void) {
+  for (auto& t : ttt::g_tuning) t.store(0, std::memory_order_relaxed);
+}
 
 int ttt_read_device_error(unsigned* value) {
   if (!value) return fail(TTT_ERR_INVALID_ARG, "ttt_read_device_error: null output");
