@@ -39,8 +39,8 @@ def metric_of(w) -> str:
     return METRIC_BWD if w.kind.endswith("_bwd") else METRIC
 DEFAULT_WORKLOAD = "assoc_bf16_B4H16T65536_d128C64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DOMINANT_KERNEL = {"dual": ("dual_mma_kernel", "dual_mma.cu"),
-                   "dual_seg": ("dual_mma_kernel", "dual_mma.cu"),
+DOMINANT_KERNEL = {"dual": ("dual_tc_kernel", "dual_tc.cu"),
+                   "dual_seg": ("dual_tc_kernel", "dual_tc.cu"),
                    "assoc": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu"),
                    "assoc_bwd": ("assoc_chunk_kernel", "assoc_scan.cu"),
@@ -504,6 +504,9 @@ def run_ours(args, w, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     ttt.load_library()
+    for kv in args.tuning:
+        k, v = kv.split("=")
+        ttt.set_tuning(k, int(v))
     x = inp.make_inputs(w, dev, seed=w.seed + 7919 * rank)
     step = make_call(w, x)
     flush = torch.empty(256 << 20, device=dev, dtype=torch.uint8)
@@ -569,7 +572,7 @@ def run_ours(args, w, rank, world, local_rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-            "config": config_of(w, world),
+            "config": dict(config_of(w, world), **({"tuning": args.tuning} if args.tuning else {})),
             "roofline": roof, "clocks": clk.summary(), "gpu_launches": launches,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}}
@@ -594,6 +597,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tuning", action="append", default=[],
+                    help="kernel-variant choice for comparisons, e.g. dual_kernel=1 (see "
+                         "ttt_set_tuning in include/ttt.h)")
     ap.add_argument("--override", action="append", default=[],
                     help="shape override of the workload for reduced profiling cases, e.g. T=8192")
     args = ap.parse_args(argv)

@@ -94,6 +94,11 @@ uint64_t ttt_launch_count(void);
  *   "dual_stage_chunks"  dual_kernel 1 with d = 64 and 8 columns per warp: 4 or 8 chunks per
  *                        pipeline stage.
  *   "assoc_parts"        superchunks per stream of the associative mode (must divide T / C).
+ *   "wait_limit_ns"      limit, in ns, of every pipeline wait of the dual form's d = 64
+ *                        kernels (dual_kernel 2 and 3; 0 = 4 s). A wait that runs out sets bit 0 of the
+ *                        device error word and the kernel returns early with incomplete outputs
+ *                        (see ttt_read_device_error); waits for copies already in flight keep
+ *                        a fixed one-second limit, so nothing is left running.
  * Every variant computes the same operation within the same tolerance. ttt_set_tuning returns
  * TTT_ERR_INVALID_ARG for an unknown key or a negative value; ttt_get_tuning returns -1 for an
  * unknown key; ttt_reset_tuning restores every key to 0. Not synchronised with calls in flight

@@ -69,6 +69,7 @@ struct PairParams {
   float* Wout;
   int T;
   unsigned* err;
+  uint64_t wait_ns;   // limit of every pipeline wait (copies in flight: a fixed second)
 };
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
@@ -134,7 +135,9 @@ __global__ void __launch_bounds__(PairCfg<D, NP, CPS>::THREADS, 1)
       int issued = 0;
       for (int j = 0; j < nstg; ++j) {
         const int s = j % NSTAGE;
-        if (j >= NSTAGE && !mbar_wait(empty_bar + 8 * s, ((j / NSTAGE) - 1) & 1, p.err)) break;
+        if (j >= NSTAGE &&
+            !mbar_wait(empty_bar + 8 * s, ((j / NSTAGE) - 1) & 1, p.err, p.wait_ns))
+          break;
         const int rows = min(R, T - j * R);
         const uint32_t bytes = 3 * Cfg::TILE_BYTES + (p.eta ? rows * 4 : 0);
         const uint32_t fb = full_bar + 8 * s;
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(PairCfg<D, NP, CPS>::THREADS, 1)
       const int s = j % NSTAGE;
       // After a failed wait the warp keeps the hand-off protocol (with meaningless data) so
       // that its output warp never waits on a barrier that no one will reach.
-      if (ok && !mbar_wait(full_bar + 8 * s, (j / NSTAGE) & 1, p.err)) ok = false;
+      if (ok && !mbar_wait(full_bar + 8 * s, (j / NSTAGE) & 1, p.err, p.wait_ns)) ok = false;
       const uint32_t sQ = sbase + s * Cfg::STAGE_BYTES;
       const uint32_t sK = sQ + Cfg::TILE_BYTES;
       const uint32_t sV = sK + Cfg::TILE_BYTES;
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(PairCfg<D, NP, CPS>::THREADS, 1)
   for (int j = 0; j < nstg; ++j) {
     const int s = j % NSTAGE;
     // as in the chain warp, the hand-off protocol runs for every chunk even after a failure
-    if (ok && !mbar_wait(full_bar + 8 * s, (j / NSTAGE) & 1, p.err)) ok = false;
+    if (ok && !mbar_wait(full_bar + 8 * s, (j / NSTAGE) & 1, p.err, p.wait_ns)) ok = false;
     const uint32_t sQ = sbase + s * Cfg::STAGE_BYTES;
     const uint32_t sK = sQ + Cfg::TILE_BYTES;
     const uint32_t sO = sbase + Cfg::OUT_OFF + (j & 1) * Cfg::OTILE_BYTES;
@@ -441,7 +444,9 @@ int launch_pair(const StateArgs& a, const LaunchCtx& ctx) {
     *ctx.msg = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
     return kCuda;
   }
-  PairParams p{a.eta, a.eta_scalar, a.S0, a.S_out, a.T, ctx.err};
+  const int limit = tuning(kTuneWaitLimitNs);
+  PairParams p{a.eta, a.eta_scalar, a.S0, a.S_out, a.T, ctx.err,
+               limit > 0 ? (uint64_t)limit : 4000000000ull};
   kern<<<BH * Cfg::NG, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(tq, tk, tv, to, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -82,6 +82,7 @@ struct TcParams {
   float* Wout;
   int T;
   unsigned* err;
+  uint64_t wait_ns;   // limit of every pipeline wait; copies in flight get a fixed second
 };
 
 __device__ __forceinline__ void bar_sync_named(int id, int threads) {
@@ -98,20 +99,6 @@ __device__ __forceinline__ bool bar_or_named(int id, int threads, bool pred) {
       : "r"((uint32_t)pred), "r"(id), "r"(threads)
       : "memory");
   return r != 0;
-}
-__device__ __forceinline__ void ld32x16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-      "%11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-template <int N>
-__device__ __forceinline__ void reg_fence_n(uint32_t (&r)[N]) {
-#pragma unroll
-  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 // Byte offset inside a TMA-swizzled tile with RB-byte rows (RB = 32, 64 or 128).
 template <int RB>
@@ -183,7 +170,9 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
       int issued = 0;
       for (int j = 0; j < nst; ++j) {
         const int s = j % NSTAGE;
-        if (j >= NSTAGE && !mbar_wait(empty + 8 * s, ((j / NSTAGE) - 1) & 1, p.err)) break;
+        if (j >= NSTAGE &&
+            !mbar_wait(empty + 8 * s, ((j / NSTAGE) - 1) & 1, p.err, p.wait_ns))
+          break;
         const int rows = min(TR, T - j * TR);
         const uint32_t fb = full + 8 * s;
         const uint32_t st = sbase + s * STAGE_BYTES;
@@ -210,7 +199,7 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
     const uint32_t id_o = umma::idesc_bf16(128, COLS, false, false);  // Q W_s and P (-E)
     auto issue_s = [&](int j) -> bool {
       const int s = j % NSTAGE, b = j & 1;
-      if (!mbar_wait_warp(full + 8 * s, (j / NSTAGE) & 1, p.err)) return false;
+      if (!mbar_wait_warp(full + 8 * s, (j / NSTAGE) & 1, p.err, p.wait_ns)) return false;
       umma::fence_after();
       const uint32_t sQ = sbase + s * STAGE_BYTES, sK = sQ + TILE;
 #pragma unroll
@@ -226,8 +215,8 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
       const uint32_t sQ = sbase + s * STAGE_BYTES;
       const uint32_t dO = tmem + TM_O + COLS * b;
       // O = Q W_s once the chain has stored W_s and the epilogue has read out O(j-2)
-      if (!mbar_wait_warp(wready + 8 * b, (j >> 1) & 1, p.err)) break;
-      if (j >= 2 && !mbar_wait_warp(ofree + 8 * b, ((j >> 1) - 1) & 1, p.err)) break;
+      if (!mbar_wait_warp(wready + 8 * b, (j >> 1) & 1, p.err, p.wait_ns)) break;
+      if (j >= 2 && !mbar_wait_warp(ofree + 8 * b, ((j >> 1) - 1) & 1, p.err, p.wait_ns)) break;
       umma::fence_after();
       const uint32_t sW = sbase + Cfg::W_OFF + Cfg::W_BYTES * b;
 #pragma unroll
@@ -235,8 +224,8 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
         umma::mma_ss_elect(dO, umma::desc_kmajor(sQ + 32 * ks), umma::desc_kmajor(sW + 32 * ks),
                            id_o, ks > 0);
       // O += P (-E) once the scores are masked and the chain has stored the stage's -E
-      if (!mbar_wait_warp(pfull + 8 * b, (j >> 1) & 1, p.err)) break;
-      if (!mbar_wait_warp(eready + 8 * b, (j >> 1) & 1, p.err)) break;
+      if (!mbar_wait_warp(pfull + 8 * b, (j >> 1) & 1, p.err, p.wait_ns)) break;
+      if (!mbar_wait_warp(eready + 8 * b, (j >> 1) & 1, p.err, p.wait_ns)) break;
       umma::fence_after();
       const uint32_t sE = sbase + Cfg::E_OFF + Cfg::E_BYTES * b;
 #pragma unroll
@@ -263,7 +252,7 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
     // Masked scores of stage j: P[t][s] = S[t][s] for s <= t, else 0, as bf16 pairs.
     auto mask = [&](int j) -> bool {
       const int b = j & 1;
-      if (!mbar_wait_warp(sfull + 8 * b, (j >> 1) & 1, p.err)) return false;
+      if (!mbar_wait_warp(sfull + 8 * b, (j >> 1) & 1, p.err, p.wait_ns)) return false;
       umma::fence_after();
 #pragma unroll
       for (int pp = 0; pp < 2; ++pp) {        // key tokens 64 pp .. 64 pp + 63
@@ -298,7 +287,7 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
     // Output of stage j: O accumulator -> bf16 -> shared tile -> TMA store.
     auto drain = [&](int j) -> bool {
       const int b = j & 1;
-      const bool got = mbar_wait_warp(ofull + 8 * b, (j >> 1) & 1, p.err);
+      const bool got = mbar_wait_warp(ofull + 8 * b, (j >> 1) & 1, p.err, p.wait_ns);
       // the previous store has finished reading the shared tile before anyone rewrites it
       if (got && etid == 0) bulk_wait_read<0>();
       if (bar_or_named(1, 128, !got)) return false;
@@ -316,9 +305,9 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
         }
       } else {
         uint32_t r[16];
-        ld32x16(tmem + tl + TM_O + COLS * b, r);
+        umma::ld32x16(tmem + tl + TM_O + COLS * b, r);
         umma::wait_ld();
-        reg_fence_n(r);
+        umma::reg_fence_n(r);
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = r[i];
       }
@@ -393,9 +382,10 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
     for (int j = 0; j < nst; ++j) {
       const int s = j % NSTAGE, b = j & 1;
       // warp-uniform waits: the stmatrix stores below need every lane
-      bool got = mbar_wait_warp(full + 8 * s, (j / NSTAGE) & 1, p.err);
+      bool got = mbar_wait_warp(full + 8 * s, (j / NSTAGE) & 1, p.err, p.wait_ns);
       // E and W_s buffers b were last read by the products of stage j-2
-      if (got && j >= 2) got = mbar_wait_warp(ofull + 8 * b, ((j >> 1) - 1) & 1, p.err);
+      if (got && j >= 2)
+        got = mbar_wait_warp(ofull + 8 * b, ((j >> 1) - 1) & 1, p.err, p.wait_ns);
       if (!got) {
         ok = false;
         break;
@@ -535,7 +525,9 @@ int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
     *ctx.msg = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
     return kCuda;
   }
-  TcParams p{a.eta, a.eta_scalar, a.S0, a.S_out, a.T, ctx.err};
+  const int limit = tuning(kTuneWaitLimitNs);
+  TcParams p{a.eta, a.eta_scalar, a.S0, a.S_out, a.T, ctx.err,
+             limit > 0 ? (uint64_t)limit : 4000000000ull};
   kern<<<BH * Cfg::NG, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(tq, tk, tv, to, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -35,8 +35,11 @@ struct IpCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BK * BN * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int WST_OFF = STAGES * STAGE_BYTES;     // 2 x [128 rows][32 fp32] W tiles
-  static constexpr int BAR_OFF = WST_OFF + 2 * 16384;
+  // epilogue staging, per 16-column piece of a tile: 2 x [128 rows][16 fp32] (the running W,
+  // loaded and stored in place) and 2 x [128 rows][16 bf16] (O or the bf16 copy of W)
+  static constexpr int WST_OFF = STAGES * STAGE_BYTES;
+  static constexpr int HST_OFF = WST_OFF + 2 * 8192;
+  static constexpr int BAR_OFF = HST_OFF + 2 * 4096;
   static constexpr int SMEM = 1024 + BAR_OFF + 256;
   static constexpr int TMEM_COLS = 2 * BN;
 };
@@ -59,13 +62,23 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          tmap),
+      "r"(src), "r"(c0), "r"(c1)
+      : "memory");
+}
+
 template <int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     inplace_chunk_kernel(const __grid_constant__ CUtensorMap tmZk,   // Z, box 64 x 128
                          const __grid_constant__ CUtensorMap tmZm,   // Z, box 64 x 64
                          const __grid_constant__ CUtensorMap tmW,    // bf16 W read source
                          const __grid_constant__ CUtensorMap tmV,    // Vhat, box 64 x 64
-                         const __grid_constant__ CUtensorMap tmWf,   // W_out fp32, box 32 x 128
+                         const __grid_constant__ CUtensorMap tmWf,   // W_out fp32, box 16 x 128
+                         const __grid_constant__ CUtensorMap tmO,    // O bf16, box 16 x 128
+                         const __grid_constant__ CUtensorMap tmWb,   // next bf16 W, box 16 x 128
                          const IpParams p) {
   using Cfg = IpCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -191,9 +204,19 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue warps 2..5
+    // A tile leaves in 16-column pieces through shared staging tiles and TMA stores (a thread
+    // owns one row of the accumulator, so direct global stores would scatter one row segment
+    // per thread). Update tiles read the running fp32 W by TMA into the fp32 staging tile two
+    // pieces ahead, add eta * acc in place and store the tile back, with its bf16 copy; the
+    // first chunk's update reads the bf16 W0 directly.
     const int q = warp & 3;  // TMEM subpartition this warp may read
     const int row = 32 * q + lane;
-    uint32_t wld = 0;        // W staging loads issued so far (selects buffer and phase)
+    const int ctid = threadIdx.x - 64;
+    constexpr int NCC = BN / 16;
+    uint32_t ec = 0;             // pieces processed so far: piece e uses staging buffers e & 1
+    uint32_t nld[2] = {0u, 0u};  // W loads consumed per fp32 staging buffer (their phases)
+    auto fbuf = [&](uint32_t e) { return sbase + Cfg::WST_OFF + 8192 * (e & 1); };
+    auto hbuf = [&](uint32_t e) { return sbase + Cfg::HST_OFF + 4096 * (e & 1); };
     for (int j = 0;; ++j) {
       const int slot = j & 1;
       if (!mbar_wait(sfull + 8 * slot, (j >> 1) & 1, p.err)) break;
@@ -207,98 +230,108 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int b = j & 1;
       if (!mbar_wait(tfull + 8 * b, (j >> 1) & 1, p.err)) break;
       umma::fence_after();
-      // Column chunks of 32. The TMEM load of chunk cc+1 is issued before chunk cc is
-      // processed. Update tiles read the running fp32 W through two shared-memory buffers that
-      // one thread fills by TMA two chunks ahead (a 16 KB tile per load); the first chunk's
-      // update reads the bf16 W0 directly from global memory.
-      constexpr int NCC = BN / 32;
       const bool staged = !rd && !p.first;
-      const int ctid = threadIdx.x - 64;
+      // W of piece cc into its fp32 staging tile (one thread; the tile's previous store has
+      // been read out, see the end of every piece)
       auto issue_w = [&](int cc) {
-        const int wb = (int)((wld + cc) & 1);
-        const uint32_t dst = sbase + Cfg::WST_OFF + 16384 * wb;
-        mbar_arrive_expect_tx(wfull + 8 * wb, 16384);
-        tma_load_2d(dst, &tmWf, wfull + 8 * wb, BN * nt + 32 * cc, BM * mt);
+        const uint32_t e = ec + cc;
+        mbar_arrive_expect_tx(wfull + 8 * (e & 1), 8192);
+        tma_load_2d(fbuf(e), &tmWf, wfull + 8 * (e & 1), BN * nt + 16 * cc, BM * mt);
       };
       if (staged && ctid == 0) {
         issue_w(0);
         if (NCC > 1) issue_w(1);
       }
-      uint32_t r[2][32];
-      float w[32];
+      uint32_t r[2][16];
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + b * BN;
-      umma::ld32x32(tbase, r[0]);
+      umma::ld32x16(tbase, r[0]);
 #pragma unroll
       for (int cc = 0; cc < NCC; ++cc) {
+        const uint32_t e = ec + cc;
         umma::wait_ld();
-        umma::reg_fence(r[cc & 1]);
-        if (cc + 1 < NCC) umma::ld32x32(tbase + 32 * (cc + 1), r[(cc + 1) & 1]);
+        umma::reg_fence_n(r[cc & 1]);
+        if (cc + 1 < NCC) umma::ld32x16(tbase + 16 * (cc + 1), r[(cc + 1) & 1]);
         const uint32_t* rv = r[cc & 1];
-        const int col = BN * nt + 32 * cc;
+        const int col = BN * nt + 16 * cc;
+        const uint32_t hb = hbuf(e), fb = fbuf(e);
         if (rd) {
-          uint4* dst = reinterpret_cast<uint4*>(p.O + (size_t)(p.tok0 + BM * mt + row) * p.D +
-                                                col);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pack_bf16(__uint_as_float(rv[8 * v]), __uint_as_float(rv[8 * v + 1])),
-                                pack_bf16(__uint_as_float(rv[8 * v + 2]), __uint_as_float(rv[8 * v + 3])),
-                                pack_bf16(__uint_as_float(rv[8 * v + 4]), __uint_as_float(rv[8 * v + 5])),
-                                pack_bf16(__uint_as_float(rv[8 * v + 6]), __uint_as_float(rv[8 * v + 7])));
+          sts128(hb + swz<32>(row * 32),
+                 make_uint4(pack_bf16(__uint_as_float(rv[0]), __uint_as_float(rv[1])),
+                            pack_bf16(__uint_as_float(rv[2]), __uint_as_float(rv[3])),
+                            pack_bf16(__uint_as_float(rv[4]), __uint_as_float(rv[5])),
+                            pack_bf16(__uint_as_float(rv[6]), __uint_as_float(rv[7]))));
+          sts128(hb + swz<32>(row * 32 + 16),
+                 make_uint4(pack_bf16(__uint_as_float(rv[8]), __uint_as_float(rv[9])),
+                            pack_bf16(__uint_as_float(rv[10]), __uint_as_float(rv[11])),
+                            pack_bf16(__uint_as_float(rv[12]), __uint_as_float(rv[13])),
+                            pack_bf16(__uint_as_float(rv[14]), __uint_as_float(rv[15]))));
         } else {
-          const size_t off = (size_t)(BM * mt + row) * p.D + col;
+          float w[16];
           if (staged) {
-            const int wb = (int)((wld + cc) & 1);
             // a wait that gives up only raises the error word: every thread must still reach
             // the named barrier below
-            mbar_wait(wfull + 8 * wb, (uint32_t)(((wld + cc) >> 1) & 1), p.err);
-            const uint32_t src = sbase + Cfg::WST_OFF + 16384 * wb;
+            mbar_wait(wfull + 8 * (e & 1), nld[e & 1] & 1, p.err);
+            ++nld[e & 1];
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              const uint4 x = lds128(src + swz<128>(row * 128 + 16 * v));
+            for (int v = 0; v < 4; ++v) {
+              const uint4 x = lds128(fb + swz<64>(row * 64 + 16 * v));
               w[4 * v] = __uint_as_float(x.x);
               w[4 * v + 1] = __uint_as_float(x.y);
               w[4 * v + 2] = __uint_as_float(x.z);
               w[4 * v + 3] = __uint_as_float(x.w);
             }
           } else {
-            const uint4* src = reinterpret_cast<const uint4*>(p.W0 + off);
+            const uint4* src =
+                reinterpret_cast<const uint4*>(p.W0 + (size_t)(BM * mt + row) * p.D + col);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
+            for (int v = 0; v < 2; ++v) {
               const uint4 x = src[v];
               const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                w[8 * v + 2 * e] = bf16_lo(xs[e]);
-                w[8 * v + 2 * e + 1] = bf16_hi(xs[e]);
+              for (int k = 0; k < 4; ++k) {
+                w[8 * v + 2 * k] = bf16_lo(xs[k]);
+                w[8 * v + 2 * k + 1] = bf16_hi(xs[k]);
               }
             }
           }
 #pragma unroll
-          for (int e = 0; e < 32; ++e) w[e] = fmaf(p.eta, __uint_as_float(rv[e]), w[e]);
-          float4* dst = reinterpret_cast<float4*>(p.Wout + off);
+          for (int k = 0; k < 16; ++k) w[k] = fmaf(p.eta, __uint_as_float(rv[k]), w[k]);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          for (int v = 0; v < 4; ++v)
+            sts128(fb + swz<64>(row * 64 + 16 * v),
+                   make_uint4(__float_as_uint(w[4 * v]), __float_as_uint(w[4 * v + 1]),
+                              __float_as_uint(w[4 * v + 2]), __float_as_uint(w[4 * v + 3])));
           if (p.Wbf_next) {
-            uint4* db = reinterpret_cast<uint4*>(p.Wbf_next + off);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              db[v] = make_uint4(pack_bf16(w[8 * v], w[8 * v + 1]), pack_bf16(w[8 * v + 2], w[8 * v + 3]),
-                                 pack_bf16(w[8 * v + 4], w[8 * v + 5]),
-                                 pack_bf16(w[8 * v + 6], w[8 * v + 7]));
-          }
-          if (staged) {
-            // every epilogue thread is done with this buffer: refill it two chunks ahead
-            named_bar_sync(1, 128);
-            if (ctid == 0 && cc + 2 < NCC) issue_w(cc + 2);
+            sts128(hb + swz<32>(row * 32),
+                   make_uint4(pack_bf16(w[0], w[1]), pack_bf16(w[2], w[3]),
+                              pack_bf16(w[4], w[5]), pack_bf16(w[6], w[7])));
+            sts128(hb + swz<32>(row * 32 + 16),
+                   make_uint4(pack_bf16(w[8], w[9]), pack_bf16(w[10], w[11]),
+                              pack_bf16(w[12], w[13]), pack_bf16(w[14], w[15])));
           }
         }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (ctid == 0) {
+          if (rd) {
+            tma_store_2d(&tmO, hb, col, p.tok0 + BM * mt);
+          } else {
+            tma_store_2d(&tmWf, fb, col, BM * mt);
+            if (p.Wbf_next) tma_store_2d(&tmWb, hb, col, BM * mt);
+          }
+          bulk_commit();
+          // this piece's staging tiles are read out before anyone rewrites them (the next
+          // piece with the same parity comes after the next named barrier)
+          bulk_wait_read<0>();
+          if (staged && cc + 2 < NCC) issue_w(cc + 2);
+        }
       }
-      if (staged) wld += NCC;
+      ec += NCC;
       umma::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + 8 * b);
     }
+    if (ctid == 0) bulk_wait<0>();
   }
   umma::fence_before();
   __syncthreads();
@@ -325,24 +358,30 @@ int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
   }
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-  CUtensorMap tzk, tzm, tv, tw0, tw[2], twf;
+  CUtensorMap tzk, tzm, tv, tw0, tw[2], twf, to, twb[2];
   {
     const uint64_t dz[2] = {(uint64_t)a.Dff, (uint64_t)a.T};
     const uint32_t bk[2] = {64, 128}, bm[2] = {64, 64};
     const uint64_t dv[2] = {(uint64_t)a.D, (uint64_t)a.T};
     const uint64_t dw[2] = {(uint64_t)a.D, (uint64_t)a.Dff};
+    const uint32_t bpiece[2] = {16, 128};   // epilogue pieces: 16 columns x 128 rows
     if (!make_tmap_2d(&tzk, a.Z, bf, dz, (uint64_t)a.Dff * 2, bk, sw, ctx.msg) ||
         !make_tmap_2d(&tzm, a.Z, bf, dz, (uint64_t)a.Dff * 2, bm, sw, ctx.msg) ||
         !make_tmap_2d(&tv, a.Vhat, bf, dv, (uint64_t)a.D * 2, bm, sw, ctx.msg) ||
-        !make_tmap_2d(&tw0, a.W0, bf, dw, (uint64_t)a.D * 2, bm, sw, ctx.msg))
+        !make_tmap_2d(&tw0, a.W0, bf, dw, (uint64_t)a.D * 2, bm, sw, ctx.msg) ||
+        !make_tmap_2d(&twf, a.W_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dw, (uint64_t)a.D * 4,
+                      bpiece, CU_TENSOR_MAP_SWIZZLE_64B, ctx.msg) ||
+        !make_tmap_2d(&to, a.O, bf, dv, (uint64_t)a.D * 2, bpiece, CU_TENSOR_MAP_SWIZZLE_32B,
+                      ctx.msg))
       return kCuda;
-    const uint32_t bwf[2] = {32, 128};
-    if (!make_tmap_2d(&twf, a.W_out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dw, (uint64_t)a.D * 4, bwf,
-                      sw, ctx.msg))
-      return kCuda;
-    for (int b = 0; b < 2; ++b)
-      if (wbf[b] && !make_tmap_2d(&tw[b], wbf[b], bf, dw, (uint64_t)a.D * 2, bm, sw, ctx.msg))
+    for (int b = 0; b < 2; ++b) {
+      twb[b] = to;   // a valid map fills the slot when there is no bf16 copy to write
+      if (wbf[b] &&
+          (!make_tmap_2d(&tw[b], wbf[b], bf, dw, (uint64_t)a.D * 2, bm, sw, ctx.msg) ||
+           !make_tmap_2d(&twb[b], wbf[b], bf, dw, (uint64_t)a.D * 2, bpiece,
+                         CU_TENSOR_MAP_SWIZZLE_32B, ctx.msg)))
         return kCuda;
+    }
   }
   auto kern = inplace_chunk_kernel<BN>;
   cudaError_t e =
@@ -375,7 +414,7 @@ int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
     p.counter = counters + i;
     p.err = ctx.err;
     const CUtensorMap& wsrc = i == 0 ? tw0 : tw[(i - 1) & 1];
-    kern<<<grid, THREADS, Cfg::SMEM, ctx.stream>>>(tzk, tzm, wsrc, tv, twf, p);
+    kern<<<grid, THREADS, Cfg::SMEM, ctx.stream>>>(tzk, tzm, wsrc, tv, twf, to, twb[i & 1], p);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
       *ctx.msg = std::string("inplace launch: ") + cudaGetErrorString(e);
@@ -394,17 +433,15 @@ int launch_proj_bn(const void* A, const void* B, void* Out, int M, int K, int N,
   using Cfg = IpCfg<BN>;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-  CUtensorMap tak, tam, tb, tunused;
+  CUtensorMap tak, tam, tb, to;
   const uint64_t da[2] = {(uint64_t)K, (uint64_t)M};
   const uint64_t db[2] = {(uint64_t)N, (uint64_t)K};
-  const uint32_t bk[2] = {64, 128}, bm[2] = {64, 64}, bwf[2] = {32, 128};
+  const uint64_t dout[2] = {(uint64_t)N, (uint64_t)M};
+  const uint32_t bk[2] = {64, 128}, bm[2] = {64, 64}, bpiece[2] = {16, 128};
   if (!make_tmap_2d(&tak, A, bf, da, (uint64_t)K * 2, bk, sw, ctx.msg) ||
       !make_tmap_2d(&tam, A, bf, da, (uint64_t)K * 2, bm, sw, ctx.msg) ||
-      !make_tmap_2d(&tb, B, bf, db, (uint64_t)N * 2, bm, sw, ctx.msg))
-    return kCuda;
-  // the update-tile maps are never used without update tiles; an fp32 view of B fills the slot
-  const uint64_t dw[2] = {(uint64_t)(N / 2), (uint64_t)K};
-  if (!make_tmap_2d(&tunused, B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dw, (uint64_t)N * 2, bwf, sw,
+      !make_tmap_2d(&tb, B, bf, db, (uint64_t)N * 2, bm, sw, ctx.msg) ||
+      !make_tmap_2d(&to, Out, bf, dout, (uint64_t)N * 2, bpiece, CU_TENSOR_MAP_SWIZZLE_32B,
                     ctx.msg))
     return kCuda;
   auto kern = inplace_chunk_kernel<BN>;
@@ -433,8 +470,9 @@ int launch_proj_bn(const void* A, const void* B, void* Out, int M, int K, int N,
   p.n_total = p.n_read;
   p.counter = counter;
   p.err = ctx.err;
-  kern<<<std::min(sms, p.n_read), THREADS, Cfg::SMEM, ctx.stream>>>(tak, tam, tb, tam, tunused,
-                                                                     p);
+  // a read-only tile list: the update-tile maps are never used, valid maps fill their slots
+  kern<<<std::min(sms, p.n_read), THREADS, Cfg::SMEM, ctx.stream>>>(tak, tam, tb, tam, to, to,
+                                                                     to, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *ctx.msg = std::string("projection launch: ") + cudaGetErrorString(e);

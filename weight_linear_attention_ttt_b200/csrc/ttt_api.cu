@@ -31,7 +31,8 @@ static const TuneName kTuneNames[] = {{"dual_column_split", kTuneDualColumnSplit
                                       {"dual_kernel", kTuneDualKernel},
                                       {"dual_warp_cols", kTuneDualWarpCols},
                                       {"dual_stage_chunks", kTuneDualStageChunks},
-                                      {"assoc_parts", kTuneAssocParts}};
+                                      {"assoc_parts", kTuneAssocParts},
+                                      {"wait_limit_ns", kTuneWaitLimitNs}};
 static int tune_key(const char* name) {
   if (!name) return -1;
   for (const auto& t : kTuneNames)
