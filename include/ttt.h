@@ -124,8 +124,10 @@ int ttt_read_device_error(unsigned* value);
  *  W0        [B,H,d,d] fp32 initial state, or NULL for zeros.
  *  O         [B,H,T,d] of dtype `dt` (output).
  *  W_out     [B,H,d,d] fp32 final state (output); may be the same pointer as W0.
- *  Supported: d in {32, 64, 128}; 1 <= C <= 64; T % C == 0. bf16 with C == 16 and d in
- *  {32, 64, 128} runs the tensor-core path; other supported shapes run the CUDA-core path.
+ *  Supported: d in {32, 64, 128}; 1 <= C <= 64; T % C == 0. bf16 runs on tensor cores for
+ *  C == 16 with d in {32, 64, 128} and for C in {32, 64} with d == 64 (d == 64: the chain on
+ *  warp MMAs, the outputs per 128-token stage on tcgen05); other supported shapes run the
+ *  CUDA-core path.
  *  Workspace: none (ttt_linear_dual_workspace_size returns 0; `workspace` may be NULL).
  * ------------------------------------------------------------------------------------------ */
 size_t ttt_linear_dual_workspace_size(int B, int H, int T, int d, int C, int dt);

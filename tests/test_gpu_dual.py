@@ -254,3 +254,16 @@ def test_pair_and_single_forms_agree_bitwise(cuda_lib, tuning):
             tuning("dual_kernel", form)
             outs.append(run(x, 16))
         assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("C,T", [(32, 32), (32, 96), (32, 416), (64, 64), (64, 192), (64, 576)])
+def test_tensor_core_form_larger_chunks(cuda_lib, tuning, C, T):
+    """C = 32 and 64 on the stage kernel (one gradient step per C tokens: the chunk's residuals
+    all at the chunk-start W), with 1, 2 and 4 CTAs per stream, full and partial stages."""
+    x = inp.dual_or_assoc_inputs(2, 3, T, 64, seed=C * 100 + T, device="cuda",
+                                 normalise=("K", "V"))
+    for split in (1, 2, 4):
+        tuning("dual_column_split", split)
+        O, W = run(x, C)
+        check(x, C, O, W, TOL["bf16"])
+    assert ttt.read_device_error() == 0

@@ -8,21 +8,24 @@
 //     W   = W - K_c^T diag(eta_c) G
 //
 // Design. The chunk loop is a serial chain through W, and a 16-token chunk is too little work to
-// hide latency, so the kernel is organised around that chain:
+// hide latency, so the kernel is organised around that chain. It serves d = 32 and d = 128, and
+// d = 64 when a caller selects it with ttt_set_tuning("dual_kernel", 1) (the default for d = 64
+// is the stage-form kernel of dual_tc.cu, which moves the output products to tcgen05).
 //   * The state never leaves registers. Columns of W are independent (the update mixes rows
-//     only), so each compute warp owns 8 output columns and keeps W[:, cols] (d x 8, fp32) as
-//     m16n8 MMA accumulators for the whole sequence. Two compute warps share each SM sub-
-//     partition, so two chains interleave and hide each other's latency.
-//   * Per chunk and warp (E = diag(eta) G, all products on mma.sync m16n8k16, fp32 accumulate):
-//         P    = K_c W[:, cols]            A = K_c (ldmatrix), B = bf16(W) (movmatrix.trans of
-//                                          the accumulators: no shared-memory round trip)
-//         E    = diag(eta) (P - V_c[:, cols])
-//         W[:, cols] -= K_c^T E           A = K_c^T (ldmatrix.trans), B = E (movmatrix.trans)
-//         O_c[:, cols] = Q_c W[:, cols] - mask(Q_c K_c^T) E
+//     only), so each compute warp owns WC output columns and keeps them as m16n8 fp32 MMA
+//     accumulators for the whole sequence. Two forms:
+//       - WC = 8 (d = 32 and d = 128): W[:, cols] (d x 8); per chunk
+//             P    = K_c W[:, cols]            A = K_c (ldmatrix), B = bf16(W) (movmatrix.trans
+//                                              of the accumulators: no shared-memory round trip)
+//             E    = diag(eta) (P - V_c[:, cols])
+//             W[:, cols] -= K_c^T E           A = K_c^T (ldmatrix.trans), B = E (movmatrix.trans)
+//             O_c[:, cols] = Q_c W[:, cols] - mask(Q_c K_c^T) E
+//         with the causal scores formed once per stage (one 16x8 piece per warp) and shared
+//         through shared memory in MMA-fragment order.
+//       - WC = 16 (d = 64): W^T[16 cols, :]; the packed accumulators are directly the A operand
+//         of the next chunk's W^T K_c^T, so the chain needs no register transposes, and each
+//         warp forms the causal scores itself from the Q and K fragments it holds.
 //     Only P -> E -> update sits on the chain; the output products hang off it.
-//   * The causal scores mask(Q_c K_c^T) do not depend on W: the warps compute them once per
-//     pipeline stage (one 16x8 piece each), negate, round to bf16 and share them through shared
-//     memory in MMA-fragment order.
 //   * Q/K/V tiles arrive by TMA (3-D tensor maps over [B*H, T, d], 128-byte swizzle) into a
 //     multi-stage mbarrier ring filled by one producer warp; outputs leave through a
 //     double-buffered shared tile and TMA stores (rows past T are clipped by the tensor map).
@@ -590,7 +593,7 @@ int launch_cfg(const StateArgs& a, const LaunchCtx& ctx) {
 }  // namespace
 
 bool dual_mma_supported(int d, int C, int dt) {
-  return dt == 1 && C == 16 && (d == 32 || d == 64 || d == 128);
+  return (dt == 1 && C == 16 && (d == 32 || d == 64 || d == 128)) || dual_tc_supported(d, C, dt);
 }
 
 int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
@@ -603,7 +606,8 @@ int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
   // d = 64: the chain on warp MMAs with the outputs per 128-token stage on tcgen05 (dual_tc.cu)
   // measured fastest on the 125M- and 1.3B-layer shapes; the all-warp-MMA forms below remain
   // selectable through ttt_set_tuning("dual_kernel", ...).
-  if (a.d == 64 && (kernel == kDualKernelAuto || kernel == kDualKernelTensor)) {
+  // (C = 32 and 64 exist only in that form)
+  if (a.d == 64 && (a.C != 16 || kernel == kDualKernelAuto || kernel == kDualKernelTensor)) {
     const int split = (forced_split == 1 || forced_split == 2 || forced_split == 4)
                           ? forced_split
                           : dual_tc_split(streams, sms);

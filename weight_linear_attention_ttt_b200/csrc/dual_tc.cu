@@ -1,5 +1,5 @@
-// TTT-Linear mini-batch dual form, bf16 inputs, d = 64, chunk C = 16: the serial chain on warp
-// MMAs in registers, the outputs on tcgen05 tensor cores with TMEM accumulators.
+// TTT-Linear mini-batch dual form, bf16 inputs, d = 64, chunk C = 16, 32 or 64: the serial chain
+// on warp MMAs in registers, the outputs on tcgen05 tensor cores with TMEM accumulators.
 //
 // Computes, per (batch, head) stream and chunk c (source: "RNN의 기억을 작은 모델로 바꾼다면:
 // Test-Time Training 읽기", section "gradient를 효율적인 layer로 만드는 작업" for the mini-batch
@@ -8,7 +8,7 @@
 //     O_c = Q_c W - tril(Q_c K_c^T) E
 //     W   = W - K_c^T E
 //
-// Outputs per stage. A pipeline stage holds R = 128 tokens (8 chunks). Inside it the state at
+// Outputs per stage. A pipeline stage holds R = 128 tokens (128 / C chunks). Inside it the state at
 // the start of chunk c is W_c = W_s - sum_{c' < c} K_c'^T E_c' (W_s: the state at the stage's
 // start), so
 //     O_c = Q_c W_s - sum_{c' < c} (Q_c K_c'^T) E_c' - tril(Q_c K_c^T) E_c,
@@ -17,6 +17,9 @@
 //     O_stage = Q W_s - tril(Q K^T) E_stage          (128 x COLS, K = 64 and K = 128)
 // Only E depends on the chain; the 128-row products are what the 5th-generation tensor core is
 // built for, and they run asynchronously to the warps that carry the chain.
+//
+// The mask does not depend on C: only the chain does (a chunk of C = 16 CM tokens takes the CM
+// residuals of its 16-token sub-chunks at the chunk-start W, then applies their CM updates).
 //
 // Roles (NC chain warps, COLS = 16 NC output columns of the stream per CTA):
 //   * chain warps 0 .. NC-1: each keeps W^T[16 columns, 64] as fp32 m16n8 accumulators for the
@@ -44,9 +47,9 @@ namespace ttt {
 namespace {
 
 constexpr int TD = 64;             // head dim
-constexpr int TC = 16;             // chunk
+constexpr int TC = 16;             // sub-chunk (the warp-MMA tile height)
 constexpr int TR = 128;            // tokens per stage
-constexpr int TCPS = TR / TC;      // chunks per stage
+constexpr int TCPS = TR / TC;      // sub-chunks per stage
 constexpr int TKS = TD / 16;       // 16-wide k-steps over d
 constexpr int NSTAGE = 3;
 constexpr int TILE = TR * TD * 2;  // one [128][64] bf16 tile, 128-byte swizzle
@@ -106,7 +109,7 @@ __device__ __forceinline__ uint32_t swz_rows(uint32_t row, uint32_t colbyte) {
   return swz<RB>(row * RB + colbyte);
 }
 
-template <int NC>
+template <int NC, int CM>
 __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
     dual_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -460,20 +463,91 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
         stsm_x4(sE + (c >> 2) * Cfg::ESUB + swz_rows<128>(srow, 2 * (16 * (c & 3) + scol)), n0,
                 n1, n2, n3);
       };
-      if (chunks == TCPS) {
-        Ops ops[2];
-        load(ops[0], 0);
+      if constexpr (CM == 1) {
+        if (chunks == TCPS) {
+          Ops ops[2];
+          load(ops[0], 0);
 #pragma unroll
-        for (int c = 0; c < TCPS; ++c) {
-          if (c + 1 < TCPS) load(ops[(c + 1) & 1], c + 1);
-          chain(ops[c & 1], c);
+          for (int c = 0; c < TCPS; ++c) {
+            if (c + 1 < TCPS) load(ops[(c + 1) & 1], c + 1);
+            chain(ops[c & 1], c);
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < chunks; ++c) {
+            Ops o;
+            load(o, c);
+            chain(o, c);
+          }
         }
       } else {
+        // C = 16 CM: every sub-chunk's residual is taken at the chunk-start W (one gradient
+        // step per chunk), then the CM updates are applied.
+        auto chain_chunk = [&](const int cc) {
+          uint32_t wa[TKS][4];
+#pragma unroll
+          for (int ks = 0; ks < TKS; ++ks) {
+            wa[ks][0] = pack_bf16(wc[2 * ks][0], wc[2 * ks][1]);
+            wa[ks][1] = pack_bf16(wc[2 * ks][2], wc[2 * ks][3]);
+            wa[ks][2] = pack_bf16(wc[2 * ks + 1][0], wc[2 * ks + 1][1]);
+            wa[ks][3] = pack_bf16(wc[2 * ks + 1][2], wc[2 * ks + 1][3]);
+          }
+          uint32_t ne[CM][4];
+#pragma unroll
+          for (int m = 0; m < CM; ++m) {
+            const int c = CM * cc + m;   // 16-token sub-chunk within the stage
+            const uint32_t cb = c * CHUNK_BYTES;
+            uint32_t kb[TKS][4], vt[4];
+#pragma unroll
+            for (int ks = 0; ks < TKS; ++ks) ldsm_x4(sK + cb + o_brow[ks], kb[ks]);
+            ldsm_x4_t(sV + cb + o_vt, vt);
+            const float e0 = ldsf(sEta + 4 * (16 * c + 2 * tq));
+            const float e1 = ldsf(sEta + 4 * (16 * c + 2 * tq + 1));
+            const float e8 = ldsf(sEta + 4 * (16 * c + 8 + 2 * tq));
+            const float e9 = ldsf(sEta + 4 * (16 * c + 9 + 2 * tq));
+            float pa[2][4] = {}, pb[2][4] = {};
+#pragma unroll
+            for (int ks = 0; ks < TKS; ++ks) {
+              float (&acc)[2][4] = (ks & 1) ? pb : pa;
+              mma16816(acc[0], wa[ks][0], wa[ks][1], wa[ks][2], wa[ks][3], kb[ks][0], kb[ks][1]);
+              mma16816(acc[1], wa[ks][0], wa[ks][1], wa[ks][2], wa[ks][3], kb[ks][2], kb[ks][3]);
+            }
+            float E[2][4];
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+              const float ea0 = n ? e8 : e0, ea1 = n ? e9 : e1;
+              E[n][0] = (pa[n][0] + pb[n][0] - bf16_lo(vt[2 * n])) * ea0;
+              E[n][1] = (pa[n][1] + pb[n][1] - bf16_hi(vt[2 * n])) * ea1;
+              E[n][2] = (pa[n][2] + pb[n][2] - bf16_lo(vt[2 * n + 1])) * ea0;
+              E[n][3] = (pa[n][3] + pb[n][3] - bf16_hi(vt[2 * n + 1])) * ea1;
+            }
+            ne[m][0] = pack_bf16(E[0][0], E[0][1]) ^ 0x80008000u;
+            ne[m][1] = pack_bf16(E[0][2], E[0][3]) ^ 0x80008000u;
+            ne[m][2] = pack_bf16(E[1][0], E[1][1]) ^ 0x80008000u;
+            ne[m][3] = pack_bf16(E[1][2], E[1][3]) ^ 0x80008000u;
+            stsm_x4(sE + (c >> 2) * Cfg::ESUB + swz_rows<128>(srow, 2 * (16 * (c & 3) + scol)),
+                    ne[m][0], ne[m][1], ne[m][2], ne[m][3]);
+          }
+#pragma unroll
+          for (int m = 0; m < CM; ++m) {
+            const uint32_t cb = (CM * cc + m) * CHUNK_BYTES;
+            uint32_t kt[TKS][4];
+#pragma unroll
+            for (int ks = 0; ks < TKS; ++ks) ldsm_x4_t(sK + cb + o_btrn[ks], kt[ks]);
+#pragma unroll
+            for (int jp = 0; jp < TKS; ++jp) {
+              mma16816(wc[2 * jp], ne[m][0], ne[m][1], ne[m][2], ne[m][3], kt[jp][0], kt[jp][1]);
+              mma16816(wc[2 * jp + 1], ne[m][0], ne[m][1], ne[m][2], ne[m][3], kt[jp][2],
+                       kt[jp][3]);
+            }
+          }
+        };
+        if (chunks == TCPS) {
+#pragma unroll
+          for (int cc = 0; cc < TCPS / CM; ++cc) chain_chunk(cc);
+        } else {
 #pragma unroll 1
-        for (int c = 0; c < chunks; ++c) {
-          Ops o;
-          load(o, c);
-          chain(o, c);
+          for (int cc = 0; cc < chunks / CM; ++cc) chain_chunk(cc);
         }
       }
       fence_proxy_async_smem();
@@ -500,7 +574,7 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
   if (warp == Cfg::MMA) umma::tmem_dealloc(tmem, Cfg::TM_COLS);
 }
 
-template <int NC>
+template <int NC, int CM>
 int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
   using Cfg = TcCfg<NC>;
   const int BH = a.B * a.H;
@@ -518,7 +592,7 @@ int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
       !make_tmap_3d(&tv, a.V, bf, dims, strides, box_in, CU_TENSOR_MAP_SWIZZLE_128B, ctx.msg) ||
       !make_tmap_3d(&to, a.O, bf, dims, strides, box_out, osw, ctx.msg))
     return kCuda;
-  auto kern = dual_tc_kernel<NC>;
+  auto kern = dual_tc_kernel<NC, CM>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) {
@@ -538,6 +612,17 @@ int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
   return kOk;
 }
 
+template <int CM>
+int launch_split(const StateArgs& a, int split, const LaunchCtx& ctx) {
+  switch (split) {
+    case 1: return launch_tc<4, CM>(a, ctx);
+    case 2: return launch_tc<2, CM>(a, ctx);
+    case 4: return launch_tc<1, CM>(a, ctx);
+  }
+  *ctx.msg = "dual_tc: column split must be 1, 2 or 4";
+  return kUnsupported;
+}
+
 }  // namespace
 
 // CTAs per stream: 1, 2 or 4 (64, 32 or 16 output columns each). A CTA holds one stream's
@@ -549,13 +634,17 @@ int dual_tc_split(int streams, int sms) {
   return 1;
 }
 
+bool dual_tc_supported(int d, int C, int dt) {
+  return dt == 1 && d == TD && (C == 16 || C == 32 || C == 64);
+}
+
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx) {
-  switch (split) {
-    case 1: return launch_tc<4>(a, ctx);
-    case 2: return launch_tc<2>(a, ctx);
-    case 4: return launch_tc<1>(a, ctx);
+  switch (a.C) {
+    case 16: return launch_split<1>(a, split, ctx);
+    case 32: return launch_split<2>(a, split, ctx);
+    case 64: return launch_split<4>(a, split, ctx);
   }
-  *ctx.msg = "dual_tc: column split must be 1, 2 or 4";
+  *ctx.msg = "dual_tc: chunk must be 16, 32 or 64";
   return kUnsupported;
 }
 

@@ -93,8 +93,9 @@ bool dual_mma_supported(int d, int C, int dt);
 int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx);
 int launch_dual_pair(const StateArgs& a, const LaunchCtx& ctx, int split);
 int launch_dual_simt(const StateArgs& a, const LaunchCtx& ctx);
-// d = 64, C = 16, bf16: chain on warp MMAs, outputs per stage on tcgen05; split = CTAs per
-// stream (1, 2 or 4), dual_tc_split() the automatic choice.
+// d = 64, C = 16, 32 or 64, bf16: chain on warp MMAs, outputs per stage on tcgen05; split =
+// CTAs per stream (1, 2 or 4), dual_tc_split() the automatic choice.
+bool dual_tc_supported(int d, int C, int dt);
 int dual_tc_split(int streams, int sms);
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx);
 
