@@ -342,7 +342,8 @@ int inplace_ttt_chunk_fwd(const void* Z, const void* Vhat, const void* W0, float
  *  Same computation, arguments and validation as inplace_ttt_chunk_fwd, minus the workspace:
  *  the scratch (two bf16 copies of W_down and one tile counter per chunk) is a static device
  *  array of inplace_ttt_noalloc_max_scratch_bytes() bytes (32 MiB) inside the library. Every
- *  GPU that loads the library holds that array until the process exits.
+ *  GPU that loads the library holds that array until the process exits (with CUDA's lazy
+ *  module loading, from this entry point's first call on that GPU).
  *  - Calls allocate nothing: no cudaMalloc, no cudaFree, no allocating library routine. The
  *    caller still provides Z, Vhat, W0, O and W_out.
  *  - Shapes whose scratch (inplace_ttt_workspace_size) exceeds the maximum return

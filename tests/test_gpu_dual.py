@@ -131,17 +131,24 @@ def test_determinism_permutation_and_state_carry(cuda_lib):
     Op, Wp = run(xp, 16)
     assert torch.equal(Op.reshape(6, 512, 64), O1.reshape(6, 512, 64)[perm])
     assert torch.equal(Wp.reshape(6, 64, 64), W1.reshape(6, 64, 64)[perm])
-    # state carry: two calls over the halves, chained through W_out -> W0, equal one call
-    h = 208  # a chunk boundary that is not a pipeline-stage boundary
-    xa = {k: (v[:, :, :h] if torch.is_tensor(v) and v.dim() >= 3 and k != "W0" else v)
-          for k, v in x.items()}
-    xb = {k: (v[:, :, h:].contiguous() if torch.is_tensor(v) and v.dim() >= 3 and k != "W0"
-              else v) for k, v in x.items()}
-    xa = {k: (v.contiguous() if torch.is_tensor(v) else v) for k, v in xa.items()}
-    Oa, Wa = run(xa, 16)
-    xb["W0"] = Wa
-    Ob, Wb = run(xb, 16)
-    assert torch.equal(torch.cat([Oa, Ob], dim=2), O1) and torch.equal(Wb, W1)
+    # state carry: two calls over the halves, chained through W_out -> W0, equal one call. The
+    # chain is the same arithmetic wherever the split falls (W bit-identical); the outputs of the
+    # d = 64 kernel are formed per 128-token stage, so they are bit-identical for a split on a
+    # stage boundary and equal within rounding for a split inside a stage.
+    for h, exact_o in ((256, True), (208, False)):
+        xa = {k: (v[:, :, :h].contiguous() if torch.is_tensor(v) and v.dim() >= 3 and k != "W0"
+                  else v) for k, v in x.items()}
+        xb = {k: (v[:, :, h:].contiguous() if torch.is_tensor(v) and v.dim() >= 3 and k != "W0"
+                  else v) for k, v in x.items()}
+        Oa, Wa = run(xa, 16)
+        xb["W0"] = Wa
+        Ob, Wb = run(xb, 16)
+        assert torch.equal(Wb, W1)
+        Ocat = torch.cat([Oa, Ob], dim=2)
+        if exact_o:
+            assert torch.equal(Ocat, O1)
+        else:
+            assert max_rel_l2(Ocat, O1, 2) < 5e-3
 
 
 def test_column_split_variants_agree_bitwise(cuda_lib, tuning):
