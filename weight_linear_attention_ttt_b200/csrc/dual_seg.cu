@@ -33,14 +33,80 @@ __global__ void identity_states_kernel(float* __restrict__ W, size_t n, int d) {
   }
 }
 
+// Register-tiled D x D fp32 product for the folds: thread t of 256 owns the TT x TT block of
+// outputs at rows TT (t / 16), columns TT (t % 16) (TT = D / 16) and adds
+//     acc[r][c] += sum_k op(A)[row r][k] * W[k][column c],   op(A) = A, or A^T if TRANS,
+// with A and W row-major [D][D] in shared memory. Each k-step of 4 loads 4 TT-wide rows of W
+// and the matching 4 x TT piece of op(A) as whole vectors, then does 16 TT^2 independent FMAs.
+template <int N>
+__device__ __forceinline__ void ld_row(const float* p, float (&v)[N]) {
+  if constexpr (N == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x, v[1] = x.y;
+  } else {
+#pragma unroll
+    for (int h = 0; h < N / 4; ++h) {
+      const float4 x = *reinterpret_cast<const float4*>(p + 4 * h);
+      v[4 * h] = x.x, v[4 * h + 1] = x.y, v[4 * h + 2] = x.z, v[4 * h + 3] = x.w;
+    }
+  }
+}
+template <int D, bool TRANS>
+__device__ __forceinline__ void tile_product(const float* A, const float* W,
+                                             float (&acc)[D / 16][D / 16]) {
+  constexpr int TT = D / 16;
+  const int i0 = TT * (threadIdx.x / 16), j0 = TT * (threadIdx.x % 16);
+#pragma unroll 2
+  for (int k = 0; k < D; k += 4) {
+    float a[4][TT];   // a[kk][r] = op(A)[i0 + r][k + kk]
+    if constexpr (TRANS) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) ld_row<TT>(A + (k + kk) * D + i0, a[kk]);
+    } else {
+#pragma unroll
+      for (int r = 0; r < TT; ++r) {
+        float v[4];
+        ld_row<4>(A + (i0 + r) * D + k, v);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) a[kk][r] = v[kk];
+      }
+    }
+    float w[4][TT];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) ld_row<TT>(W + (k + kk) * D + j0, w[kk]);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+      for (int r = 0; r < TT; ++r)
+#pragma unroll
+        for (int c = 0; c < TT; ++c) acc[r][c] = fmaf(a[kk][r], w[kk][c], acc[r][c]);
+  }
+}
+// W <- op(A) W + bias (bias a global D x D matrix), all threads of the CTA.
+template <int D, bool TRANS>
+__device__ __forceinline__ void affine_step(const float* A, float* W,
+                                            const float* __restrict__ bias) {
+  constexpr int TT = D / 16;
+  const int i0 = TT * (threadIdx.x / 16), j0 = TT * (threadIdx.x % 16);
+  float acc[TT][TT];
+#pragma unroll
+  for (int r = 0; r < TT; ++r) ld_row<TT>(bias + (i0 + r) * D + j0, acc[r]);
+  tile_product<D, TRANS>(A, W, acc);
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < TT; ++r)
+#pragma unroll
+    for (int c = 0; c < TT; ++c) W[(i0 + r) * D + j0 + c] = acc[r][c];
+  __syncthreads();
+}
+
 // One CTA per stream: W (fp32, d x d) and A_s = (A_s + B_s) - B_s in shared memory; segment s
-// stores its start state, then W <- A_s W + B_s. Each thread owns d*d/256 outputs.
+// stores its start state, then W <- A_s W + B_s.
 template <int D>
 __global__ void __launch_bounds__(256) fold_segments_kernel(const float* __restrict__ W0,
                                                             const float* __restrict__ Bm,
                                                             const float* __restrict__ ABm,
                                                             float* __restrict__ Wstart, int S) {
-  constexpr int E = D * D / 256;   // outputs per thread
   extern __shared__ float fsm[];
   float* W = fsm;                  // [D][D]
   float* A = fsm + D * D;          // [D][D]
@@ -54,19 +120,7 @@ __global__ void __launch_bounds__(256) fold_segments_kernel(const float* __restr
       A[i] = ABm[seg + i] - Bm[seg + i];
     }
     __syncthreads();
-    float out[E];
-#pragma unroll
-    for (int q = 0; q < E; ++q) {
-      const int idx = threadIdx.x + 256 * q, i = idx / D, j = idx % D;
-      float acc = Bm[seg + idx];
-#pragma unroll 8
-      for (int k = 0; k < D; ++k) acc = fmaf(A[i * D + k], W[k * D + j], acc);
-      out[q] = acc;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < E; ++q) W[threadIdx.x + 256 * q] = out[q];
-    __syncthreads();
+    affine_step<D, false>(A, W, Bm + seg);
   }
 }
 
@@ -79,7 +133,6 @@ template <int D>
 __global__ void __launch_bounds__(256) fold_segments_reverse_kernel(
     const float* __restrict__ dW_out, const float* __restrict__ Bm, const float* __restrict__ ABm,
     const float* __restrict__ Noff, float* __restrict__ Xafter, int S) {
-  constexpr int E = D * D / 256;
   extern __shared__ float fsm[];
   float* X = fsm;                  // [D][D]
   float* A = fsm + D * D;          // [D][D] = A_s
@@ -93,19 +146,7 @@ __global__ void __launch_bounds__(256) fold_segments_reverse_kernel(
       A[i] = ABm[seg + i] - Bm[seg + i];
     }
     __syncthreads();
-    float out[E];
-#pragma unroll
-    for (int q = 0; q < E; ++q) {
-      const int idx = threadIdx.x + 256 * q, i = idx / D, j = idx % D;
-      float acc = Noff[seg + idx];
-#pragma unroll 8
-      for (int k = 0; k < D; ++k) acc = fmaf(A[k * D + i], X[k * D + j], acc);   // (A^T X)[i][j]
-      out[q] = acc;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < E; ++q) X[threadIdx.x + 256 * q] = out[q];
-    __syncthreads();
+    affine_step<D, true>(A, X, Noff + seg);   // X <- A_s^T X + N_s
   }
 }
 
@@ -135,7 +176,6 @@ __global__ void __launch_bounds__(256) fold_gathered_kernel(const float* __restr
                                                             const float* __restrict__ Bm,
                                                             int upto, size_t bh_count,
                                                             float* __restrict__ W_out) {
-  constexpr int E = D * D / 256;
   extern __shared__ float fsm[];
   float* W = fsm;
   float* A = fsm + D * D;
@@ -146,19 +186,7 @@ __global__ void __launch_bounds__(256) fold_gathered_kernel(const float* __restr
     const size_t off = ((size_t)m * bh_count + bh) * D * D;
     for (int i = threadIdx.x; i < D * D; i += 256) A[i] = Am[off + i];
     __syncthreads();
-    float out[E];
-#pragma unroll
-    for (int q = 0; q < E; ++q) {
-      const int idx = threadIdx.x + 256 * q, i = idx / D, j = idx % D;
-      float acc = Bm[off + idx];
-#pragma unroll 8
-      for (int k = 0; k < D; ++k) acc = fmaf(A[i * D + k], W[k * D + j], acc);
-      out[q] = acc;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < E; ++q) W[threadIdx.x + 256 * q] = out[q];
-    __syncthreads();
+    affine_step<D, false>(A, W, Bm + off);
   }
   for (int i = threadIdx.x; i < D * D; i += 256) W_out[bh * D * D + i] = W[i];
 }
