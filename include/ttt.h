@@ -99,6 +99,9 @@ uint64_t ttt_launch_count(void);
  *                        device error word and the kernel returns early with incomplete outputs
  *                        (see ttt_read_device_error); waits for copies already in flight keep
  *                        a fixed one-second limit, so nothing is left running.
+ *   "inplace_chunks_per_launch"  In-Place update: 1 = one chunk per launch; 0 or 2 = two
+ *                        chunks per launch where the shape allows it (D % 256 == 0, C % 256 == 0),
+ *                        chunk i+1's read corrected by eta (Z_(i+1) Z_i^T) Vhat_i.
  * Every variant computes the same operation within the same tolerance. ttt_set_tuning returns
  * TTT_ERR_INVALID_ARG for an unknown key or a negative value; ttt_get_tuning returns -1 for an
  * unknown key; ttt_reset_tuning restores every key to 0. Not synchronised with calls in flight

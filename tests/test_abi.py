@@ -262,7 +262,8 @@ def test_tuning_choices_set_get_reset(lib):
         assert lib.ttt_get_tuning(b"no_such_key") == -1
         lib.ttt_reset_tuning()
         for key in (b"dual_column_split", b"dual_kernel", b"dual_warp_cols",
-                    b"dual_stage_chunks", b"assoc_parts", b"wait_limit_ns"):
+                    b"dual_stage_chunks", b"assoc_parts", b"wait_limit_ns",
+                    b"inplace_chunks_per_launch"):
             assert lib.ttt_get_tuning(key) == 0
     finally:
         lib.ttt_reset_tuning()

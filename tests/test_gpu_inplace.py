@@ -85,3 +85,24 @@ def test_workspace_and_shape_errors(cuda_lib):
     with pytest.raises(ttt.TTTError) as e:
         run(x, 64)  # C not a multiple of 128
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("T,C,Dff,D", [
+    (512, 256, 256, 256),     # one chunk pair
+    (768, 256, 512, 512),     # a pair, then a single chunk
+    (2048, 512, 384, 768),    # two pairs
+])
+def test_chunk_pairs_match_oracle_and_single_chunks(cuda_lib, tuning, T, C, Dff, D):
+    """Two chunks per launch (chunk i+1's read corrected by eta (Z_(i+1) Z_i^T) Vhat_i, one
+    update over both chunks) against the oracle, and against one chunk per launch."""
+    x = inp.inplace_inputs(T, Dff, D, seed=T + C + D, device="cuda", eta=1e-2)
+    n0 = ttt.launch_count()
+    O2, W2 = run(x, C)
+    n_pairs = (T // C) // 2
+    assert ttt.launch_count() - n0 == T // C - n_pairs
+    check(x, C, O2, W2)
+    tuning("inplace_chunks_per_launch", 1)
+    O1, W1 = run(x, C)
+    assert max_rel_l2(O2.t().contiguous(), O1.t().contiguous(), 1) < 1e-2
+    assert max_rel_l2(W2.t().contiguous(), W1.t().contiguous(), 1) < 1e-4
+    assert ttt.read_device_error() == 0

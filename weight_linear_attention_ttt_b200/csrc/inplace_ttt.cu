@@ -47,16 +47,68 @@ struct IpCfg {
 struct IpParams {
   const __nv_bfloat16* W0;   // [Dff, D] bf16 (source of chunk 0's update)
   float* Wout;               // [Dff, D] fp32 running master
-  __nv_bfloat16* Wbf_next;   // [Dff, D] bf16 copy written by this chunk's update (or null)
+  __nv_bfloat16* Wbf_next;   // [Dff, D] bf16 copy written by this launch's update (or null)
   __nv_bfloat16* O;          // [T, D]
   float eta;
-  int first;                 // chunk 0: the update reads W0
-  int tok0;                  // first token of the chunk
+  int first;                 // the launch holds chunk 0: the update reads W0
+  int tok0;                  // first token of the launch's (first) chunk
   int C, Dff, D;
-  int n_read, n_total;       // read tiles come first in the tile list
+  int pair;                  // 1: the launch covers chunks i and i+1 (see the tile list below)
+  int n_p;                   // pair launches: tiles of eta Z_(i+1) Z_i^T
+  int n_read;                // read tiles per chunk
+  int n_total;
   int* counter;
+  int* pdone;                // pair launches: finished eta Z Z^T tiles per 128-row block
   unsigned* err;
 };
+
+// Tile list of a launch, in the order the global counter hands it out:
+//   single chunk:  read tiles of the chunk (K = Dff), update tiles (K = C);
+//   chunk pair:    tiles of Pc = eta Z_(i+1) Z_i^T (C x C, K = Dff, stored bf16 in the
+//                  workspace), read tiles of chunk i+1 (K = Dff from Z_(i+1) and the bf16 W_(i-1),
+//                  then K = C from Pc and Vhat_i: the exact correction for chunk i's update, which
+//                  chunk i+1 must see), read tiles of chunk i, update tiles over both chunks
+//                  (K = 2C: W_(i+1) = W_(i-1) + eta [Z_i; Z_(i+1)]^T [Vhat_i; Vhat_(i+1)]).
+// The fp32 master is then read and written once per pair. A read tile of chunk i+1 waits for
+// its row block of Pc only after its K = Dff part; Pc tiles come first in the list.
+enum TileKind : int { kRead = 0, kUpdate = 1, kPc = 2, kReadNext = 3 };
+struct Tile {
+  int kind, mt, nt, nkb;
+};
+template <int BN>
+__device__ __forceinline__ Tile decode_tile(const IpParams& p, int t) {
+  const int ntn = p.D / BN;
+  Tile x;
+  if (p.pair && t < p.n_p) {
+    const int per = p.C / BN;
+    x.kind = kPc, x.mt = t / per, x.nt = t % per, x.nkb = p.Dff / BK;
+    return x;
+  }
+  int u = t - (p.pair ? p.n_p : 0);
+  if (p.pair && u < p.n_read) {
+    x.kind = kReadNext, x.mt = u / ntn, x.nt = u % ntn, x.nkb = (p.Dff + p.C) / BK;
+    return x;
+  }
+  if (p.pair) u -= p.n_read;
+  if (u < p.n_read) {
+    x.kind = kRead, x.mt = u / ntn, x.nt = u % ntn, x.nkb = p.Dff / BK;
+    return x;
+  }
+  u -= p.n_read;
+  x.kind = kUpdate, x.mt = u / ntn, x.nt = u % ntn, x.nkb = (p.pair ? 2 * p.C : p.C) / BK;
+  return x;
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* ptr) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int* ptr, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -79,6 +131,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                          const __grid_constant__ CUtensorMap tmWf,   // W_out fp32, box 16 x 128
                          const __grid_constant__ CUtensorMap tmO,    // O bf16, box 16 x 128
                          const __grid_constant__ CUtensorMap tmWb,   // next bf16 W, box 16 x 128
+                         const __grid_constant__ CUtensorMap tmPl,   // Pc, box 64 x 128 (loads)
+                         const __grid_constant__ CUtensorMap tmPs,   // Pc, box 16 x 128 (stores)
                          const IpParams p) {
   using Cfg = IpCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -93,7 +147,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t wfull = tslot + 32;                   // W staging buffers loaded (x2)
   volatile int* sched = reinterpret_cast<volatile int*>(smem + Cfg::BAR_OFF + 16 * STAGES + 80);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntn = p.D / BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -131,32 +184,56 @@ __global__ void __launch_bounds__(THREADS, 1)
         sched[slot] = t;
         mbar_arrive(sfull + 8 * slot);
         if (t >= p.n_total) break;
-        const bool rd = t < p.n_read;
-        const int u = rd ? t : t - p.n_read;
-        const int mt = u / ntn, nt = u % ntn;
-        const int nkb = rd ? p.Dff / BK : p.C / BK;
+        const Tile x = decode_tile<BN>(p, t);
+        const int kbz = p.Dff / BK;   // k-blocks over Dff
+        const int rows = x.kind == kReadNext ? p.tok0 + p.C + BM * x.mt : p.tok0 + BM * x.mt;
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb, ++kbt) {
+        for (int kb = 0; kb < x.nkb; ++kb, ++kbt) {
           const int s = kbt % STAGES;
           if (kbt >= STAGES && !mbar_wait(empty + 8 * s, ((kbt / STAGES) - 1) & 1, p.err)) {
             ok = false;
             break;
           }
+          if (x.kind == kReadNext && kb == kbz) {
+            // the correction part needs this row block of Pc, written by other CTAs' TMA stores:
+            // wait (bounded) for its tiles' release, then order the loads after it
+            const uint64_t t0 = global_timer_ns();
+            while (ld_acquire_gpu(p.pdone + x.mt) < p.C / BN) {
+              if (global_timer_ns() - t0 > 4000000000ull) {
+                raise_device_error(p.err, kErrWaitTimeout);
+                break;
+              }
+              __nanosleep(256);
+            }
+            fence_proxy_async_global();
+          }
           const uint32_t fb = full + 8 * s;
           const uint32_t sA = sbase + s * Cfg::STAGE_BYTES, sB = sA + Cfg::A_BYTES;
           mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
-          if (rd) {
-            tma_load_2d(sA, &tmZk, fb, kb * BK, p.tok0 + BM * mt);
+          if (x.kind == kPc) {
+            // A = Z_(i+1) rows, B = Z_i rows (K-major, N = 256 tokens of chunk i)
+            tma_load_2d(sA, &tmZk, fb, kb * BK, p.tok0 + p.C + BM * x.mt);
+            tma_load_2d(sB, &tmZk, fb, kb * BK, p.tok0 + BN * x.nt);
+            tma_load_2d(sB + 16384, &tmZk, fb, kb * BK, p.tok0 + BN * x.nt + 128);
+          } else if (x.kind == kRead || kb < kbz) {
+            tma_load_2d(sA, &tmZk, fb, kb * BK, rows);
 #pragma unroll
             for (int nb = 0; nb < BN / 64; ++nb)
-              tma_load_2d(sB + nb * 8192, &tmW, fb, BN * nt + 64 * nb, kb * BK);
+              tma_load_2d(sB + nb * 8192, &tmW, fb, BN * x.nt + 64 * nb, kb * BK);
+          } else if (x.kind == kReadNext) {
+            // A = Pc rows of chunk i+1, B = Vhat_i (MN-major, like the update's B)
+            const int k2 = kb - kbz;
+            tma_load_2d(sA, &tmPl, fb, k2 * BK, BM * x.mt);
+#pragma unroll
+            for (int nb = 0; nb < BN / 64; ++nb)
+              tma_load_2d(sB + nb * 8192, &tmV, fb, BN * x.nt + 64 * nb, p.tok0 + k2 * BK);
           } else {
 #pragma unroll
             for (int mb = 0; mb < 2; ++mb)
-              tma_load_2d(sA + mb * 8192, &tmZm, fb, BM * mt + 64 * mb, p.tok0 + kb * BK);
+              tma_load_2d(sA + mb * 8192, &tmZm, fb, BM * x.mt + 64 * mb, p.tok0 + kb * BK);
 #pragma unroll
             for (int nb = 0; nb < BN / 64; ++nb)
-              tma_load_2d(sB + nb * 8192, &tmV, fb, BN * nt + 64 * nb, p.tok0 + kb * BK);
+              tma_load_2d(sB + nb * 8192, &tmV, fb, BN * x.nt + 64 * nb, p.tok0 + kb * BK);
           }
         }
         if (!ok) break;
@@ -167,6 +244,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       const uint32_t idesc_rd = umma::idesc_bf16(BM, BN, false, true);
       const uint32_t idesc_up = umma::idesc_bf16(BM, BN, true, true);
+      const uint32_t idesc_pc = umma::idesc_bf16(BM, BN, false, false);
       uint32_t kbt = 0;
       for (int j = 0;; ++j) {
         const int slot = j & 1;
@@ -174,14 +252,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int t = sched[slot];
         mbar_arrive(sempty + 8 * slot);
         if (t >= p.n_total) break;
-        const bool rd = t < p.n_read;
-        const int nkb = rd ? p.Dff / BK : p.C / BK;
+        const Tile x = decode_tile<BN>(p, t);
         const int b = j & 1;
         if (j >= 2 && !mbar_wait(tempty + 8 * b, ((j >> 1) - 1) & 1, p.err)) break;
         umma::fence_after();
         const uint32_t dt = tmem + b * BN;
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb, ++kbt) {
+        for (int kb = 0; kb < x.nkb; ++kb, ++kbt) {
           const int s = kbt % STAGES;
           if (!mbar_wait(full + 8 * s, (kbt / STAGES) & 1, p.err)) {
             ok = false;
@@ -191,10 +268,22 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t sA = sbase + s * Cfg::STAGE_BYTES, sB = sA + Cfg::A_BYTES;
 #pragma unroll
           for (int ks = 0; ks < BK / 16; ++ks) {
-            const uint64_t ad = rd ? umma::desc_kmajor(sA + 32 * ks)
-                                   : umma::desc_mnmajor(sA + 2048 * ks, 8192);
-            const uint64_t bd = umma::desc_mnmajor(sB + 2048 * ks, 8192);
-            umma::mma_ss(dt, ad, bd, rd ? idesc_rd : idesc_up, kb > 0 || ks > 0);
+            uint64_t ad, bd;
+            uint32_t id;
+            if (x.kind == kUpdate) {
+              ad = umma::desc_mnmajor(sA + 2048 * ks, 8192);
+              bd = umma::desc_mnmajor(sB + 2048 * ks, 8192);
+              id = idesc_up;
+            } else if (x.kind == kPc) {
+              ad = umma::desc_kmajor(sA + 32 * ks);
+              bd = umma::desc_kmajor(sB + 32 * ks);
+              id = idesc_pc;
+            } else {
+              ad = umma::desc_kmajor(sA + 32 * ks);
+              bd = umma::desc_mnmajor(sB + 2048 * ks, 8192);
+              id = idesc_rd;
+            }
+            umma::mma_ss(dt, ad, bd, id, kb > 0 || ks > 0);
           }
           umma::commit(empty + 8 * s);
         }
@@ -224,13 +313,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(sempty + 8 * slot);
       if (t >= p.n_total) break;
-      const bool rd = t < p.n_read;
-      const int u = rd ? t : t - p.n_read;
-      const int mt = u / ntn, nt = u % ntn;
+      const Tile x = decode_tile<BN>(p, t);
+      const bool rd = x.kind != kUpdate;   // read and Pc tiles: a bf16 result, no W
+      const int mt = x.mt, nt = x.nt;
       const int b = j & 1;
       if (!mbar_wait(tfull + 8 * b, (j >> 1) & 1, p.err)) break;
       umma::fence_after();
       const bool staged = !rd && !p.first;
+      const float rscale = x.kind == kPc ? p.eta : 1.f;
+      const int orow = x.kind == kReadNext ? p.tok0 + p.C + BM * mt : p.tok0 + BM * mt;
       // W of piece cc into its fp32 staging tile (one thread; the tile's previous store has
       // been read out, see the end of every piece)
       auto issue_w = [&](int cc) {
@@ -255,16 +346,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int col = BN * nt + 16 * cc;
         const uint32_t hb = hbuf(e), fb = fbuf(e);
         if (rd) {
+          float o[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) o[k] = rscale * __uint_as_float(rv[k]);
           sts128(hb + swz<32>(row * 32),
-                 make_uint4(pack_bf16(__uint_as_float(rv[0]), __uint_as_float(rv[1])),
-                            pack_bf16(__uint_as_float(rv[2]), __uint_as_float(rv[3])),
-                            pack_bf16(__uint_as_float(rv[4]), __uint_as_float(rv[5])),
-                            pack_bf16(__uint_as_float(rv[6]), __uint_as_float(rv[7]))));
+                 make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]), pack_bf16(o[4], o[5]),
+                            pack_bf16(o[6], o[7])));
           sts128(hb + swz<32>(row * 32 + 16),
-                 make_uint4(pack_bf16(__uint_as_float(rv[8]), __uint_as_float(rv[9])),
-                            pack_bf16(__uint_as_float(rv[10]), __uint_as_float(rv[11])),
-                            pack_bf16(__uint_as_float(rv[12]), __uint_as_float(rv[13])),
-                            pack_bf16(__uint_as_float(rv[14]), __uint_as_float(rv[15]))));
+                 make_uint4(pack_bf16(o[8], o[9]), pack_bf16(o[10], o[11]),
+                            pack_bf16(o[12], o[13]), pack_bf16(o[14], o[15])));
         } else {
           float w[16];
           if (staged) {
@@ -313,8 +403,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (ctid == 0) {
-          if (rd) {
-            tma_store_2d(&tmO, hb, col, p.tok0 + BM * mt);
+          if (x.kind == kPc) {
+            tma_store_2d(&tmPs, hb, col, BM * mt);
+          } else if (rd) {
+            tma_store_2d(&tmO, hb, col, orow);
           } else {
             tma_store_2d(&tmWf, fb, col, BM * mt);
             if (p.Wbf_next) tma_store_2d(&tmWb, hb, col, BM * mt);
@@ -327,6 +419,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       ec += NCC;
+      if (x.kind == kPc && ctid == 0) {
+        // the tile is in global memory before it is announced to the read tiles of chunk i+1
+        bulk_wait<0>();
+        fence_proxy_async_global();
+        red_release_gpu_add(p.pdone + mt, 1);
+      }
       umma::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + 8 * b);
@@ -342,23 +440,47 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 int pick_bn(int D) { return D % 256 == 0 ? 256 : (D % 128 == 0 ? 128 : 64); }
 
+// Workspace: two bf16 copies of W (n > 1), the tile counter of every launch, the Pc counters of
+// every launch (C / 128 each) and one C x C bf16 Pc buffer (n > 1).
+struct IpWorkspace {
+  size_t wbf, counters, pc, bytes;
+};
+IpWorkspace ip_workspace(int T, int Dff, int D, int C) {
+  const int n = T / C;
+  IpWorkspace w{};
+  const size_t wbf_bytes = n > 1 ? align256((size_t)Dff * D * 2) : 0;
+  w.wbf = 0;
+  w.counters = 2 * wbf_bytes;
+  const size_t nct = (size_t)std::max(n, 1) * (1 + C / BM);
+  w.pc = w.counters + align256(sizeof(int) * nct);
+  w.bytes = w.pc + (n > 1 ? align256((size_t)C * C * 2) : 0);
+  return w;
+}
+
+// Chunks per launch: 2 (the pair form above) where the tiles allow it (256-wide tiles, C a
+// multiple of 256) unless a tuning choice asks for 1.
+bool pairs_enabled(int BN, int C) {
+  const int choice = tuning(kTuneInplaceChunksPerLaunch);
+  return choice != 1 && BN == 256 && C % 256 == 0;
+}
+
 template <int BN>
 int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
   using Cfg = IpCfg<BN>;
   const int n = a.T / a.C;
-  const size_t wbf_bytes = (size_t)a.Dff * a.D * 2;
+  const IpWorkspace wsl = ip_workspace(a.T, a.Dff, a.D, a.C);
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
   __nv_bfloat16* wbf[2] = {nullptr, nullptr};
-  int* counters = nullptr;
   if (n > 1) {
-    wbf[0] = reinterpret_cast<__nv_bfloat16*>(a.ws);
-    wbf[1] = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(a.ws) + align256(wbf_bytes));
-    counters = reinterpret_cast<int*>(static_cast<uint8_t*>(a.ws) + 2 * align256(wbf_bytes));
-  } else {
-    counters = reinterpret_cast<int*>(a.ws);
+    wbf[0] = reinterpret_cast<__nv_bfloat16*>(ws + wsl.wbf);
+    wbf[1] = reinterpret_cast<__nv_bfloat16*>(ws + wsl.wbf + (wsl.counters - wsl.wbf) / 2);
   }
+  int* counters = reinterpret_cast<int*>(ws + wsl.counters);   // one per launch
+  int* pdone = counters + n;                                    // C / 128 per launch
+  void* pc = n > 1 ? static_cast<void*>(ws + wsl.pc) : nullptr;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-  CUtensorMap tzk, tzm, tv, tw0, tw[2], twf, to, twb[2];
+  CUtensorMap tzk, tzm, tv, tw0, tw[2], twf, to, twb[2], tpl, tps;
   {
     const uint64_t dz[2] = {(uint64_t)a.Dff, (uint64_t)a.T};
     const uint32_t bk[2] = {64, 128}, bm[2] = {64, 64};
@@ -382,11 +504,21 @@ int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
                          CU_TENSOR_MAP_SWIZZLE_32B, ctx.msg)))
         return kCuda;
     }
+    tpl = tzk;   // valid maps fill the Pc slots of launches without Pc tiles
+    tps = to;
+    if (pc) {
+      const uint64_t dp[2] = {(uint64_t)a.C, (uint64_t)a.C};
+      if (!make_tmap_2d(&tpl, pc, bf, dp, (uint64_t)a.C * 2, bk, sw, ctx.msg) ||
+          !make_tmap_2d(&tps, pc, bf, dp, (uint64_t)a.C * 2, bpiece, CU_TENSOR_MAP_SWIZZLE_32B,
+                        ctx.msg))
+        return kCuda;
+    }
   }
   auto kern = inplace_chunk_kernel<BN>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-  if (e == cudaSuccess) e = cudaMemsetAsync(counters, 0, sizeof(int) * n, ctx.stream);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(counters, 0, sizeof(int) * (size_t)n * (1 + a.C / BM), ctx.stream);
   if (e != cudaSuccess) {
     *ctx.msg = std::string("inplace setup: ") + cudaGetErrorString(e);
     return kCuda;
@@ -396,12 +528,15 @@ int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int ntn = a.D / BN;
   const int n_read = (a.C / BM) * ntn, n_up = (a.Dff / BM) * ntn;
-  const int grid = std::min(sms, n_read + n_up);
-  for (int i = 0; i < n; ++i) {
+  const bool pairs = n > 1 && pairs_enabled(BN, a.C);
+  int L = 0;   // launch index: selects the bf16 copy this launch writes
+  for (int i = 0; i < n; ++L) {
+    const bool pair = pairs && i + 1 < n;
+    const int span = pair ? 2 : 1;
     IpParams p;
     p.W0 = static_cast<const __nv_bfloat16*>(a.W0);
     p.Wout = a.W_out;
-    p.Wbf_next = (i + 1 < n) ? wbf[i & 1] : nullptr;
+    p.Wbf_next = (i + span < n) ? wbf[L & 1] : nullptr;
     p.O = static_cast<__nv_bfloat16*>(a.O);
     p.eta = a.eta;
     p.first = i == 0;
@@ -409,18 +544,24 @@ int launch_bn(const InplaceArgs& a, const LaunchCtx& ctx) {
     p.C = a.C;
     p.Dff = a.Dff;
     p.D = a.D;
+    p.pair = pair;
+    p.n_p = pair ? (a.C / BM) * (a.C / BN) : 0;
     p.n_read = n_read;
-    p.n_total = n_read + n_up;
-    p.counter = counters + i;
+    p.n_total = p.n_p + (pair ? 2 : 1) * n_read + n_up;
+    p.counter = counters + L;
+    p.pdone = pdone + (size_t)L * (a.C / BM);
     p.err = ctx.err;
-    const CUtensorMap& wsrc = i == 0 ? tw0 : tw[(i - 1) & 1];
-    kern<<<grid, THREADS, Cfg::SMEM, ctx.stream>>>(tzk, tzm, wsrc, tv, twf, to, twb[i & 1], p);
+    const CUtensorMap& wsrc = L == 0 ? tw0 : tw[(L - 1) & 1];
+    const int grid = std::min(sms, p.n_total);
+    kern<<<grid, THREADS, Cfg::SMEM, ctx.stream>>>(tzk, tzm, wsrc, tv, twf, to, twb[L & 1], tpl,
+                                                   tps, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) {
       *ctx.msg = std::string("inplace launch: ") + cudaGetErrorString(e);
       return kCuda;
     }
     count_launch();
+    i += span;
   }
   return kOk;
 }
@@ -466,13 +607,17 @@ int launch_proj_bn(const void* A, const void* B, void* Out, int M, int K, int N,
   p.C = M;
   p.Dff = K;
   p.D = N;
+  p.pair = 0;
+  p.n_p = 0;
   p.n_read = (M / BM) * (N / BN);
   p.n_total = p.n_read;
   p.counter = counter;
+  p.pdone = nullptr;
   p.err = ctx.err;
-  // a read-only tile list: the update-tile maps are never used, valid maps fill their slots
+  // a read-only tile list: the update-tile and Pc maps are never used, valid maps fill their
+  // slots
   kern<<<std::min(sms, p.n_read), THREADS, Cfg::SMEM, ctx.stream>>>(tak, tam, tb, tam, to, to,
-                                                                     to, p);
+                                                                     to, tak, to, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *ctx.msg = std::string("projection launch: ") + cudaGetErrorString(e);
@@ -485,10 +630,7 @@ int launch_proj_bn(const void* A, const void* B, void* Out, int M, int K, int N,
 }  // namespace
 
 size_t inplace_workspace_bytes(int T, int Dff, int D, int C) {
-  const int n = T / C;
-  const size_t counters = align256(sizeof(int) * (size_t)std::max(n, 1));
-  if (n <= 1) return counters;
-  return 2 * align256((size_t)Dff * D * 2) + counters;
+  return ip_workspace(T, Dff, D, C).bytes;
 }
 
 bool inplace_supported(int T, int Dff, int D, int C, std::string* why) {

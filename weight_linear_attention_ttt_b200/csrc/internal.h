@@ -71,6 +71,7 @@ enum TuneKey : int {
   kTuneDualStageChunks,       // all-warp-MMA dual form, d = 64, 8 columns: 4 or 8 chunks/stage
   kTuneAssocParts,            // superchunks per stream of the associative mode
   kTuneWaitLimitNs,           // limit of the d = 64 dual-form pipeline waits, ns (0: 4 s)
+  kTuneInplaceChunksPerLaunch,  // In-Place: 1 = one chunk per launch, 0 / 2 = chunk pairs
   kTuneCount
 };
 enum DualKernel : int { kDualKernelAuto = 0, kDualKernelWarp = 1, kDualKernelPair = 2,

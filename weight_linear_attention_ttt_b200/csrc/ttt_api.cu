@@ -32,7 +32,9 @@ static const TuneName kTuneNames[] = {{"dual_column_split", kTuneDualColumnSplit
                                       {"dual_warp_cols", kTuneDualWarpCols},
                                       {"dual_stage_chunks", kTuneDualStageChunks},
                                       {"assoc_parts", kTuneAssocParts},
-                                      {"wait_limit_ns", kTuneWaitLimitNs}};
+                                      {"wait_limit_ns", kTuneWaitLimitNs},
+                                      {"inplace_chunks_per_launch",
+                                       kTuneInplaceChunksPerLaunch}};
 static int tune_key(const char* name) {
   if (!name) return -1;
   for (const auto& t : kTuneNames)
