@@ -66,17 +66,18 @@ def kernel_source_sha(fname: str) -> str:
 
 
 def measured_traffic(workload: str, kernel: str, sha: str):
-    """DRAM bytes per launch from a committed ncu summary, valid only for the same kernel
-    source (profiles/dram_traffic.txt: `workload kernel source_sha256_16 bytes_per_launch`)."""
+    """(DRAM bytes, scope) from a committed ncu summary, valid only for the same kernel source
+    (profiles/dram_traffic.txt: `workload kernel source_sha256_16 bytes [launch|call]`), else
+    (None, None)."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
-        return None
+        return None, None
     for line in open(p):
         f = line.split()
         if len(f) >= 4 and not line.startswith("#") and f[0] == workload and f[1] == kernel \
                 and f[2] == sha:
-            return float(f[3])
-    return None
+            return float(f[3]), (f[4] if len(f) > 4 else "launch")
+    return None, None
 
 
 # ----------------------------------------------------------------------------- clocks (NVML)
@@ -561,7 +562,8 @@ def run_ours(args, w, rank, world, local_rank):
                 "frac": achieved / peak}
     roof["roofline_us"] = 1e6 * max(t_flops, t_bytes)
     sha = kernel_source_sha(ksrc)
-    roof.update({"traffic": measured_traffic(w.name, kname, sha), "kernel": kname,
+    traffic, traffic_scope = measured_traffic(w.name, kname, sha)
+    roof.update({"traffic": traffic, "traffic_scope": traffic_scope, "kernel": kname,
                  "peak_source": f"{pk_kind} (MEASURED_PEAKS.json)" if pk_kind == "measured"
                  else "fallback", "launches_per_step": launches_per_step,
                  "kernel_source_sha": sha,

@@ -90,7 +90,9 @@ uint64_t ttt_launch_count(void);
  *                        (one warp per 16 columns), 2 = the same on chain/output warp pairs,
  *                        3 = chain on warp MMAs with the outputs per 128-token stage on the
  *                        tcgen05 tensor cores (d = 64 only; what 0 picks for d = 64).
- *   "dual_warp_cols"     dual_kernel 1 with d = 64: 8 or 16 output columns per warp.
+ *   "dual_warp_cols"     d = 64 with C = 16: 8 or 16 output columns per warp, for dual_kernel
+ *                        1 and for the stage kernel (dual_kernel 3; 8-column chains run two
+ *                        per SM sub-partition).
  *   "dual_stage_chunks"  dual_kernel 1 with d = 64 and 8 columns per warp: 4 or 8 chunks per
  *                        pipeline stage.
  *   "assoc_parts"        superchunks per stream of the associative mode (must divide T / C).
@@ -329,7 +331,8 @@ int ttt_state_prefix_sum(const float* S0, const float* increments, int n_increme
  *  O     [T,D]  bf16 output.
  *  W_out [Dff,D] fp32 final W_down (the running fp32 master).
  *  Supported: T % C == 0; C % 128 == 0; Dff % 128 == 0; D % 64 == 0.
- *  Workspace: inplace_ttt_workspace_size() bytes (bf16 copy of the running W).
+ *  Workspace: inplace_ttt_workspace_size() bytes (two bf16 copies of the running W, per-launch
+ *  tile counters and, with two chunks per launch, the C x C bf16 correction eta Z_(i+1) Z_i^T).
  * ------------------------------------------------------------------------------------------ */
 size_t inplace_ttt_workspace_size(int T, int Dff, int D, int C);
 int inplace_ttt_chunk_fwd(const void* Z, const void* Vhat, const void* W0, float eta, void* O,
@@ -351,7 +354,7 @@ int inplace_ttt_chunk_fwd(const void* Z, const void* Vhat, const void* W0, float
  *    caller still provides Z, Vhat, W0, O and W_out.
  *  - Shapes whose scratch (inplace_ttt_workspace_size) exceeds the maximum return
  *    TTT_ERR_UNSUPPORTED before anything is launched, with the reason in
- *    ttt_last_error_message(). With T > C the need is about 4 * Dff * D bytes.
+ *    ttt_last_error_message(). With T > C the need is about 4 * Dff * D + 2 * C * C bytes.
  *  - All calls share the one array and it keeps the previous call's contents; the tile counters
  *    are zeroed on `stream` at the start of every call, and the W copies are always written
  *    before they are read. Calls whose work overlaps on the GPU (different streams, or threads

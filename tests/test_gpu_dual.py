@@ -164,11 +164,14 @@ def test_column_split_variants_agree_bitwise(cuda_lib, tuning):
         assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
-def test_tensor_core_form_column_splits(cuda_lib, tuning):
+@pytest.mark.parametrize("warp_cols", [16, 8])
+def test_tensor_core_form_column_splits(cuda_lib, tuning, warp_cols):
     """The stage-form kernel (chain on warp MMAs, outputs on tcgen05) with 1, 2 and 4 CTAs per
-    stream: the chain of a column is the same arithmetic in every split (final W bit-identical),
-    and every split meets the oracle on full and partial 128-token stages."""
+    stream and 16 or 8 columns per chain warp: the chain of a column is the same arithmetic in
+    every split (final W bit-identical), and every split meets the oracle on full and partial
+    128-token stages."""
     tuning("dual_kernel", 3)
+    tuning("dual_warp_cols", warp_cols)
     for T in (16, 144, 400):
         x = inp.dual_or_assoc_inputs(2, 3, T, 64, seed=T + 11, device="cuda",
                                      normalise=("K", "V"))
@@ -184,11 +187,14 @@ def test_tensor_core_form_column_splits(cuda_lib, tuning):
         assert ttt.read_device_error() == 0
 
 
-def test_tensor_core_and_warp_forms_agree(cuda_lib, tuning):
+@pytest.mark.parametrize("warp_cols", [16, 8])
+def test_tensor_core_and_warp_forms_agree(cuda_lib, tuning, warp_cols):
     """The stage form regroups the output sum (the earlier chunks of a stage enter through the
-    masked scores instead of the chunk-start state); the chain is the same, so W agrees bit for
-    bit and O within the bf16 rounding of the regrouped terms."""
+    masked scores instead of the chunk-start state); the chain is the same as the all-warp-MMA
+    kernel's with as many columns per warp, so W agrees bit for bit and O within the bf16
+    rounding of the regrouped terms."""
     x = inp.dual_or_assoc_inputs(2, 4, 1024, 64, seed=31, device="cuda", normalise=("K", "V"))
+    tuning("dual_warp_cols", warp_cols)
     tuning("dual_kernel", 1)
     Ow, Ww = run(x, 16)
     tuning("dual_kernel", 3)

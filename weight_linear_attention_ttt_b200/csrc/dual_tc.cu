@@ -56,9 +56,9 @@ constexpr int TILE = TR * TD * 2;  // one [128][64] bf16 tile, 128-byte swizzle
 constexpr int STAGE_BYTES = 3 * TILE + 1024;   // Q, K, V, rates (512 B, padded)
 constexpr uint32_t TM_S = 0, TM_P = 256, TM_O = 384;
 
-template <int NC>
+template <int NC, int WC>
 struct TcCfg {
-  static constexpr int COLS = 16 * NC;            // output columns per CTA
+  static constexpr int COLS = WC * NC;            // output columns per CTA
   static constexpr int NG = TD / COLS;            // CTAs per stream
   static constexpr int ORB = COLS * 2;            // bytes per row of the O tile
   static constexpr int ESUB = COLS * 128;         // one [COLS][64 tokens] sub-tile of E
@@ -103,18 +103,29 @@ __device__ __forceinline__ bool bar_or_named(int id, int threads, bool pred) {
       : "memory");
   return r != 0;
 }
+// Transpose of an 8x8 bf16 tile held as one register per lane in MMA-fragment order.
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+__device__ __forceinline__ void stsm_x2(uint32_t addr, uint32_t r0, uint32_t r1) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x2.shared.b16 [%0], {%1, %2};" ::"r"(addr), "r"(r0),
+               "r"(r1)
+               : "memory");
+}
 // Byte offset inside a TMA-swizzled tile with RB-byte rows (RB = 32, 64 or 128).
 template <int RB>
 __device__ __forceinline__ uint32_t swz_rows(uint32_t row, uint32_t colbyte) {
   return swz<RB>(row * RB + colbyte);
 }
 
-template <int NC, int CM>
-__global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
+template <int NC, int CM, int WC>
+__global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
     dual_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                    const TcParams p) {
-  using Cfg = TcCfg<NC>;
+  using Cfg = TcCfg<NC, WC>;
   constexpr int COLS = Cfg::COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -341,8 +352,153 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
       if (j + 1 == nst) drain(j);
     }
     if (etid == 0) bulk_wait<0>();
+  } else if constexpr (WC == 8) {
+    // ------------------------------------------------------------------ chain warps, 8 columns
+    // Each warp keeps W[:, 8 columns] (d x 8) as four m16n8 fp32 accumulators; bf16(W) and E
+    // reach the B operand of the next products through movmatrix transposes. Two such warps
+    // share each SM sub-partition, so two chains interleave.
+    static_assert(CM == 1, "the 8-column chain takes 16-token chunks");
+    const int g = lane >> 2, tq = lane & 3;
+    const int mi = lane >> 3, rr = lane & 7;
+    const int colw = 8 * warp;
+    const int colg = col_cta + colw;
+    auto off = [&](int row, int col) -> uint32_t { return swz_rows<128>(row, 2 * col); };
+    // K rows as the A operand (matrices (r0-7, lo) (r8-15, lo) (r0-7, hi) (r8-15, hi)); K^T as
+    // the A operand of the update via ldmatrix.trans; V in accumulator order
+    uint32_t o_arow[TKS], o_atrn[TKS];
+#pragma unroll
+    for (int ks = 0; ks < TKS; ++ks) {
+      o_arow[ks] = off(8 * (mi & 1) + rr, 16 * ks + 8 * (mi >> 1));
+      o_atrn[ks] = off(8 * (mi >> 1) + rr, 16 * ks + 8 * (mi & 1));
+    }
+    const uint32_t o_v0 = off(g, colg + 2 * tq), o_v1 = off(g + 8, colg + 2 * tq);
+    constexpr uint32_t CHUNK_BYTES = 16 * 128;
+    // stmatrix rows: W column colw + rr of the [COLS][...] tiles
+    const int srow = colw + rr;
+    float wc[TKS][4];   // W[16 mt + g (+8)][colg + 2 tq (+1)]
+    {
+      const float* w0 = p.W0 ? p.W0 + (size_t)stream * TD * TD : nullptr;
+#pragma unroll
+      for (int mt = 0; mt < TKS; ++mt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float2 v = make_float2(0.f, 0.f);
+          if (w0)
+            v = *reinterpret_cast<const float2*>(w0 + (16 * mt + 8 * h + g) * TD + colg + 2 * tq);
+          wc[mt][2 * h] = v.x;
+          wc[mt][2 * h + 1] = v.y;
+        }
+    }
+    struct Ops8 {
+      uint32_t ka[TKS][4], kt[TKS][4], v0, v1;
+      float eg, eg8;
+    };
+    bool ok = true;
+    for (int j = 0; j < nst; ++j) {
+      const int s = j % NSTAGE, b = j & 1;
+      bool got = mbar_wait_warp(full + 8 * s, (j / NSTAGE) & 1, p.err, p.wait_ns);
+      if (got && j >= 2)
+        got = mbar_wait_warp(ofull + 8 * b, ((j >> 1) - 1) & 1, p.err, p.wait_ns);
+      if (!got) {
+        ok = false;
+        break;
+      }
+      const uint32_t sK = sbase + s * STAGE_BYTES + TILE;
+      const uint32_t sV = sK + TILE;
+      const uint32_t sEta = sV + TILE;
+      const uint32_t sE = sbase + Cfg::E_OFF + Cfg::E_BYTES * b;
+      const uint32_t sW = sbase + Cfg::W_OFF + Cfg::W_BYTES * b;
+      const int chunks = min(TR, T - j * TR) / TC;
+      // bf16(W_s)^T rows for the stage's Q W_s product: the B fragments of two k-steps per
+      // stmatrix (matrix m: k = 32 pp + 8 m)
+#pragma unroll
+      for (int pp = 0; pp < TKS / 2; ++pp) {
+        const uint32_t w00 = movm_t(pack_bf16(wc[2 * pp][0], wc[2 * pp][1]));
+        const uint32_t w01 = movm_t(pack_bf16(wc[2 * pp][2], wc[2 * pp][3]));
+        const uint32_t w10 = movm_t(pack_bf16(wc[2 * pp + 1][0], wc[2 * pp + 1][1]));
+        const uint32_t w11 = movm_t(pack_bf16(wc[2 * pp + 1][2], wc[2 * pp + 1][3]));
+        stsm_x4(sW + swz_rows<128>(srow, 2 * (32 * pp + 8 * mi)), w00, w01, w10, w11);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(wready + 8 * b);
+
+      auto load = [&](Ops8& o, const int c) {
+        const uint32_t cb = c * CHUNK_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < TKS; ++ks) {
+          ldsm_x4(sK + cb + o_arow[ks], o.ka[ks]);
+          ldsm_x4_t(sK + cb + o_atrn[ks], o.kt[ks]);
+        }
+        o.v0 = ldsu32(sV + cb + o_v0);
+        o.v1 = ldsu32(sV + cb + o_v1);
+        o.eg = ldsf(sEta + 4 * (16 * c + g));
+        o.eg8 = ldsf(sEta + 4 * (16 * c + g + 8));
+      };
+      // bf16(W) -> P = K W -> E -> W -= K^T E; -E^T is stored for the outputs
+      auto chain = [&](const Ops8& o, const int c) {
+        uint32_t wb[TKS][2];
+#pragma unroll
+        for (int ks = 0; ks < TKS; ++ks) {
+          wb[ks][0] = movm_t(pack_bf16(wc[ks][0], wc[ks][1]));
+          wb[ks][1] = movm_t(pack_bf16(wc[ks][2], wc[ks][3]));
+        }
+        float pa[4] = {}, pb[4] = {};
+#pragma unroll
+        for (int ks = 0; ks < TKS; ++ks) {
+          if (ks & 1)
+            mma16816(pb, o.ka[ks][0], o.ka[ks][1], o.ka[ks][2], o.ka[ks][3], wb[ks][0], wb[ks][1]);
+          else
+            mma16816(pa, o.ka[ks][0], o.ka[ks][1], o.ka[ks][2], o.ka[ks][3], wb[ks][0], wb[ks][1]);
+        }
+        const float e0 = (pa[0] + pb[0] - bf16_lo(o.v0)) * o.eg;
+        const float e1 = (pa[1] + pb[1] - bf16_hi(o.v0)) * o.eg;
+        const float e2 = (pa[2] + pb[2] - bf16_lo(o.v1)) * o.eg8;
+        const float e3 = (pa[3] + pb[3] - bf16_hi(o.v1)) * o.eg8;
+        const uint32_t n0 = movm_t(pack_bf16(e0, e1)) ^ 0x80008000u;   // -E, tokens 0-7
+        const uint32_t n1 = movm_t(pack_bf16(e2, e3)) ^ 0x80008000u;   // -E, tokens 8-15
+#pragma unroll
+        for (int mt = 0; mt < TKS; ++mt)
+          mma16816(wc[mt], o.kt[mt][0], o.kt[mt][1], o.kt[mt][2], o.kt[mt][3], n0, n1);
+        // -E^T of chunk c (lanes 0-7 address matrix 0, tokens 16c..; lanes 8-15 matrix 1)
+        stsm_x2(sE + (c >> 2) * Cfg::ESUB +
+                    swz_rows<128>(srow, 2 * (16 * (c & 3) + 8 * (mi & 1))),
+                n0, n1);
+      };
+      if (chunks == TCPS) {
+        Ops8 ops[2];
+        load(ops[0], 0);
+#pragma unroll
+        for (int c = 0; c < TCPS; ++c) {
+          if (c + 1 < TCPS) load(ops[(c + 1) & 1], c + 1);
+          chain(ops[c & 1], c);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < chunks; ++c) {
+          Ops8 o;
+          load(o, c);
+          chain(o, c);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(eready + 8 * b);
+        mbar_arrive(empty + 8 * s);
+      }
+    }
+    if (ok) {
+      float* wo = p.Wout + (size_t)stream * TD * TD;
+#pragma unroll
+      for (int mt = 0; mt < TKS; ++mt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          *reinterpret_cast<float2*>(wo + (16 * mt + 8 * h + g) * TD + colg + 2 * tq) =
+              make_float2(wc[mt][2 * h], wc[mt][2 * h + 1]);
+    }
   } else {
-    // ------------------------------------------------------------------ chain warps
+    // ------------------------------------------------------------------ chain warps, 16 columns
     const int g = lane >> 2, tq = lane & 3;
     const int mi = lane >> 3, rr = lane & 7;    // ldmatrix / stmatrix: matrix, row
     const int colw = 16 * warp;                 // first column of this warp inside the CTA's
@@ -574,9 +730,9 @@ __global__ void __launch_bounds__(TcCfg<NC>::THREADS, 1)
   if (warp == Cfg::MMA) umma::tmem_dealloc(tmem, Cfg::TM_COLS);
 }
 
-template <int NC, int CM>
+template <int NC, int CM, int WC>
 int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
-  using Cfg = TcCfg<NC>;
+  using Cfg = TcCfg<NC, WC>;
   const int BH = a.B * a.H;
   CUtensorMap tq, tk, tv, to;
   const uint64_t dims[3] = {(uint64_t)TD, (uint64_t)a.T, (uint64_t)BH};
@@ -592,7 +748,7 @@ int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
       !make_tmap_3d(&tv, a.V, bf, dims, strides, box_in, CU_TENSOR_MAP_SWIZZLE_128B, ctx.msg) ||
       !make_tmap_3d(&to, a.O, bf, dims, strides, box_out, osw, ctx.msg))
     return kCuda;
-  auto kern = dual_tc_kernel<NC, CM>;
+  auto kern = dual_tc_kernel<NC, CM, WC>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) {
@@ -612,12 +768,13 @@ int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
   return kOk;
 }
 
-template <int CM>
+template <int CM, int WC>
 int launch_split(const StateArgs& a, int split, const LaunchCtx& ctx) {
+  constexpr int N1 = 64 / WC;   // chain warps with one CTA per stream
   switch (split) {
-    case 1: return launch_tc<4, CM>(a, ctx);
-    case 2: return launch_tc<2, CM>(a, ctx);
-    case 4: return launch_tc<1, CM>(a, ctx);
+    case 1: return launch_tc<N1, CM, WC>(a, ctx);
+    case 2: return launch_tc<N1 / 2, CM, WC>(a, ctx);
+    case 4: return launch_tc<N1 / 4, CM, WC>(a, ctx);
   }
   *ctx.msg = "dual_tc: column split must be 1, 2 or 4";
   return kUnsupported;
@@ -639,10 +796,13 @@ bool dual_tc_supported(int d, int C, int dt) {
 }
 
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx) {
+  // columns per chain warp: 8 (two chains per sub-partition) or 16, for 16-token chunks
+  const bool eight = tuning(kTuneDualWarpCols) == 8;
   switch (a.C) {
-    case 16: return launch_split<1>(a, split, ctx);
-    case 32: return launch_split<2>(a, split, ctx);
-    case 64: return launch_split<4>(a, split, ctx);
+    case 16:
+      return eight ? launch_split<1, 8>(a, split, ctx) : launch_split<1, 16>(a, split, ctx);
+    case 32: return launch_split<2, 16>(a, split, ctx);
+    case 64: return launch_split<4, 16>(a, split, ctx);
   }
   *ctx.msg = "dual_tc: chunk must be 16, 32 or 64";
   return kUnsupported;
