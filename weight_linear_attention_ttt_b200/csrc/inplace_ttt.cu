@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma_load_2d(sA, &tmZk, fb, kb * BK, p.tok0 + p.C + BM * x.mt);
             tma_load_2d(sB, &tmZk, fb, kb * BK, p.tok0 + BN * x.nt);
             tma_load_2d(sB + 16384, &tmZk, fb, kb * BK, p.tok0 + BN * x.nt + 128);
-          } else if (x.kind == kRead || kb < kbz) {
+          } else if (x.kind == kRead || (x.kind == kReadNext && kb < kbz)) {
             tma_load_2d(sA, &tmZk, fb, kb * BK, rows);
 #pragma unroll
             for (int nb = 0; nb < BN / 64; ++nb)
