@@ -154,13 +154,8 @@ def make_call(w, x, stream_outputs=None):
     if w.kind == "dual":
         O = torch.empty_like(x["Q"])
         W = torch.empty((w.B, w.H, w.d, w.d), device=x["Q"].device, dtype=torch.float32)
-        lib = ttt.load_library()
-        nbytes = lib.ttt_linear_dual_workspace_size(w.B, w.H, w.T, w.d, w.C,
-                                                    1 if w.dtype == "bf16" else 0)
-        ws = torch.empty(max(nbytes, 16), device=x["Q"].device, dtype=torch.uint8)
         return lambda: ttt.ttt_linear_dual_fwd(x["Q"], x["K"], x["V"], x["eta"], x["W0"], C=w.C,
-                                               eta_scalar=x["eta_scalar"], O=O, W_out=W,
-                                               workspace=ws)
+                                               eta_scalar=x["eta_scalar"], O=O, W_out=W)
     if w.kind == "dual_seg":
         O = torch.empty_like(x["Q"])
         W = torch.empty((w.B, w.H, w.d, w.d), device=x["Q"].device, dtype=torch.float32)

@@ -263,7 +263,7 @@ def test_tuning_choices_set_get_reset(lib):
         lib.ttt_reset_tuning()
         for key in (b"dual_column_split", b"dual_kernel", b"dual_warp_cols",
                     b"dual_stage_chunks", b"assoc_parts", b"wait_limit_ns",
-                    b"inplace_chunks_per_launch"):
+                    b"inplace_chunks_per_launch", b"dual_cluster_streams"):
             assert lib.ttt_get_tuning(key) == 0
     finally:
         lib.ttt_reset_tuning()

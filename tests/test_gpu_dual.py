@@ -283,19 +283,20 @@ def test_tensor_core_form_larger_chunks(cuda_lib, tuning, C, T):
 
 
 def test_split_form_matches_oracle_and_stage_kernel(cuda_lib, tuning):
-    """Chain CTAs and output CTAs on separate SMs (one cooperative launch, stages handed over
-    through the workspace): every column split meets the oracle on full and partial stages, the
-    final state equals the single-SM stage kernel's bit for bit (the same chain), and without a
-    large enough workspace the call runs that kernel instead."""
-    for T in (16, 144, 1040):
-        x = inp.dual_or_assoc_inputs(2, 3, T, 64, seed=T + 71, device="cuda",
+    """Chain CTAs and output CTAs on separate SMs of one cluster (stages handed over by
+    distributed-shared-memory copies), with one or two streams per cluster (also an odd stream
+    count: the last cluster holds one): every case meets the oracle on full and partial stages
+    and its final state equals the single-SM stage kernel's bit for bit (the same chain)."""
+    for B, H, T in ((2, 3, 16), (2, 3, 144), (1, 5, 1040)):
+        x = inp.dual_or_assoc_inputs(B, H, T, 64, seed=T + 71 + H, device="cuda",
                                      normalise=("K", "V"))
         tuning("dual_kernel", 3)
         tuning("dual_column_split", 1)
         O_tc, W_tc = run(x, 16)
+        tuning("dual_column_split", 0)
         tuning("dual_kernel", 4)
-        for split in (1, 2, 4):
-            tuning("dual_column_split", split)
+        for ks in (1, 2):
+            tuning("dual_cluster_streams", ks)
             n0 = ttt.launch_count()
             O, W = run(x, 16)
             assert ttt.launch_count() - n0 == 1
@@ -303,22 +304,3 @@ def test_split_form_matches_oracle_and_stage_kernel(cuda_lib, tuning):
             assert torch.equal(W, W_tc)
             assert max_rel_l2(O, O_tc, 2) < 1e-3
         assert ttt.read_device_error() == 0
-    # automatic choice without a workspace: the single-SM stage kernel, same bits
-    tuning("dual_kernel", 0)
-    tuning("dual_column_split", 0)
-    O_small, W_small = run(x, 16, workspace=torch.empty(16, device="cuda", dtype=torch.uint8))
-    tuning("dual_kernel", 3)
-    O_ref, W_ref = run(x, 16)
-    assert torch.equal(O_small, O_ref) and torch.equal(W_small, W_ref)
-
-
-def test_split_form_workspace_checks(cuda_lib):
-    lib = ttt.load_library()
-    assert lib.ttt_linear_dual_workspace_size(8, 12, 2048, 64, 16, 1) > 0
-    assert lib.ttt_linear_dual_workspace_size(8, 12, 2048, 64, 16, 0) == 0
-    assert lib.ttt_linear_dual_workspace_size(8, 12, 2048, 128, 16, 1) == 0
-    x = inp.dual_or_assoc_inputs(1, 2, 128, 64, seed=3, device="cuda", normalise=("K", "V"))
-    with pytest.raises(ttt.TTTError) as e:   # a workspace that overlaps an output
-        O = torch.empty_like(x["Q"])
-        run(x, 16, O=O, workspace=O.view(torch.uint8))
-    assert e.value.status == 1

@@ -606,23 +606,20 @@ int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
   // d = 64: the chain on warp MMAs with the outputs per 128-token stage on tcgen05 (dual_tc.cu)
   // measured fastest on the 125M- and 1.3B-layer shapes; the all-warp-MMA forms below remain
   // selectable through ttt_set_tuning("dual_kernel", ...).
-  // d = 64, C = 16 with a workspace: the chain on some SMs, the stage products on others
-  // (dual_xsm.cu), where the streams leave enough SMs free; measured faster than one SM doing
+  // d = 64, C = 16: the chain on some SMs, the stage products on others of the same cluster
+  // (dual_xsm.cu) where the streams leave enough SMs free; measured faster than one SM doing
   // both, since the output work slows the latency-bound chain it shares an SM with.
   if (dual_xsm_applicable(a.d, a.C, a.dt) &&
       (kernel == kDualKernelAuto || kernel == kDualKernelSplit)) {
-    int n_out = 0;
-    int ng = dual_xsm_plan(streams, sms, &n_out);
-    if (ng && (forced_split == 1 || forced_split == 2 || forced_split == 4)) {
-      const int avail = sms - streams * forced_split;
-      ng = avail >= (streams + 1) / 2 && avail >= 1 ? forced_split : 0;
-      n_out = std::min(avail, streams);
+    int n_clusters = 0;
+    const int ks = dual_xsm_plan(streams, sms, &n_clusters);
+    if (ks) {
+      const int r = launch_dual_xsm(a, ks, n_clusters, ctx);
+      if (r != kUnsupported) return r;
     }
-    if (ng && a.ws && a.ws_bytes >= dual_xsm_workspace_bytes(a.B, a.H))
-      return launch_dual_xsm(a, ng, n_out, ctx);
     if (kernel == kDualKernelSplit) {
-      *ctx.msg = "dual form: the split form needs ttt_linear_dual_workspace_size() bytes of "
-                 "workspace and SMs for at least one output CTA per two streams";
+      *ctx.msg = "dual form: the split form needs one more SM per one or two streams, and "
+                 "its clusters resident at once";
       return kUnsupported;
     }
   }

@@ -1,5 +1,5 @@
 // TTT-Linear mini-batch dual form, bf16 inputs, d = 64, chunk C = 16, with the serial chain and
-// the output products on separate SMs.
+// the output products on separate SMs of one thread-block cluster.
 //
 // Computes, per (batch, head) stream and chunk c (source: "RNN의 기억을 작은 모델로 바꾼다면:
 // Test-Time Training 읽기", section "gradient를 효율적인 layer로 만드는 작업" for the mini-batch
@@ -10,19 +10,22 @@
 //
 // Why two kinds of CTA. The chain (bf16 W -> K_c W -> E -> W update) is serial over the sequence
 // and latency-bound; on an SM that also runs the stage products on tcgen05 and their epilogue,
-// the chain measured about 1.5x slower than alone (the output work competes with it for the
-// tensor pipe and the issue slots even when nothing waits on it). Here one launch holds
-//   * chain CTAs, one per (stream, column group): NC chain warps (16 columns of W each, the state
-//     in registers), a TMA producer warp (K, V, rates) and a publisher warp that copies every
-//     stage's -E^T and bf16(W_s)^T from shared memory to a ring of slots in the workspace and
-//     releases a per-stream counter;
-//   * output CTAs, each serving a fixed set of streams stage by stage: a producer warp waits for
-//     the counters of the stream (acquire), loads Q and K by TMA and the slot by a bulk copy into
-//     one pipeline stage, and releases the slot; an MMA warp issues S = Q K^T, O = Q W_s and
-//     O += P (-E) on tcgen05; four epilogue warps mask S into P (TMEM -> TMEM) and store O.
-// The launch is cooperative, so every CTA is resident and the counters always make progress:
-// a chain CTA only waits for a slot its own output CTA releases after loading it, and an output
-// CTA walks stages in order, so no wait can close a cycle. Every wait is bounded.
+// the chain measured about 1.4x slower than alone (the output work competes with it for the
+// tensor pipe and the issue slots even when nothing waits on it). Here a cluster of KS + 1 CTAs
+// (KS = 1 or 2) holds
+//   * KS chain CTAs, one per stream: 4 chain warps (16 columns of W each, the state in
+//     registers), a TMA producer warp (K, V, rates) and a publisher thread that copies every
+//     stage's -E^T and bf16(W_s)^T from its shared memory into the output CTA's pipeline stage
+//     (a distributed-shared-memory bulk copy completing on the output CTA's mbarrier);
+//   * one output CTA serving the cluster's streams stage by stage: a producer warp loads Q and K
+//     by TMA into a pipeline stage, sets the stage's expected bytes (Q, K and the chain's copy)
+//     and grants the stage to the chain CTA (a remote mbarrier arrival); an MMA warp issues
+//     S = Q K^T, O = Q W_s and O += P (-E) on tcgen05 and, once a stage has landed, frees the
+//     chain CTA's buffer (another remote arrival); four epilogue warps mask S into P
+//     (TMEM -> TMEM) and store O.
+// Every hand-off is an mbarrier phase in shared memory: no global memory, no fence, and the
+// cluster's CTAs are co-scheduled. Every wait is bounded; a cluster barrier ends the kernel so
+// that no CTA leaves while another may still reach its shared memory.
 #include <algorithm>
 #include <string>
 
@@ -39,25 +42,25 @@ constexpr int XR = 128;             // tokens per stage
 constexpr int XCPS = XR / XC;       // chunks per stage
 constexpr int XKS = XD / 16;        // 16-wide k-steps over d
 constexpr int XTILE = XR * XD * 2;  // one [128][64] bf16 tile, 128-byte swizzle
-constexpr int RING = 4;             // published stages kept per stream
 constexpr int PART = 64 * 128;      // one [64][64] bf16 sub-tile (8 KB)
 constexpr int SLOT = 3 * PART;      // -E^T tokens 0-63, tokens 64-127, bf16 W_s^T
+constexpr int NGRANT = 4;           // grant barriers per chain CTA (grants run <= 3 stages ahead)
 constexpr uint32_t XTM_S = 0, XTM_P = 256, XTM_O = 384;
 
 template <int NC>
 struct XCfg {
-  static constexpr int COLS = 16 * NC;             // output columns per chain CTA
-  static constexpr int NG = XD / COLS;             // chain CTAs per stream
+  static constexpr int COLS = 16 * NC;             // output columns per chain CTA (all of W)
+  static_assert(COLS == XD, "one chain CTA per stream");
   // chain CTA
   static constexpr int C_NST = 3;
   static constexpr int C_STAGE = 2 * XTILE + 1024;  // K, V, rates (512 B, padded)
-  static constexpr int C_ESUB = COLS * 128;         // this CTA's rows of one -E^T sub-tile
+  static constexpr int C_ESUB = COLS * 128;         // one -E^T sub-tile (= PART)
   static constexpr int C_E_OFF = C_NST * C_STAGE;   // 2 buffers x 2 sub-tiles
   static constexpr int C_W_OFF = C_E_OFF + 4 * C_ESUB;
   static constexpr int C_END = C_W_OFF + 2 * C_ESUB;
   // output CTA
   static constexpr int O_NST = 3;
-  static constexpr int O_STAGE = 2 * XTILE + SLOT;  // Q, K, then the slot image
+  static constexpr int O_STAGE = 2 * XTILE + SLOT;  // Q, K, then the chain CTA's copy
   static constexpr int O_OT_OFF = O_NST * O_STAGE;
   static constexpr int O_END = O_OT_OFF + XTILE;
   static constexpr int BAR_OFF = C_END > O_END ? C_END : O_END;
@@ -65,7 +68,7 @@ struct XCfg {
   static constexpr int WARPS = NC + 2 > 6 ? NC + 2 : 6;
   static constexpr int THREADS = 32 * WARPS;
   static_assert(SMEM <= 227 * 1024, "shared memory");
-  static_assert(C_ESUB % 1024 == 0 && C_STAGE % 1024 == 0 && O_STAGE % 1024 == 0, "alignment");
+  static_assert(C_ESUB == PART && C_STAGE % 1024 == 0 && O_STAGE % 1024 == 0, "layout");
 };
 
 struct XParams {
@@ -74,10 +77,7 @@ struct XParams {
   const float* W0;
   float* Wout;
   int T, BH;
-  int n_chain, n_out;
-  uint8_t* ring;        // [BH][RING][SLOT]
-  int* ready;           // [BH * NG]: stages published by each chain CTA
-  int* consumed;        // [BH]: stages whose slot the output CTA has loaded
+  int ks;               // streams (chain CTAs) per cluster; the output CTA has rank ks
   unsigned* err;
   uint64_t wait_ns;
 };
@@ -95,35 +95,38 @@ __device__ __forceinline__ bool xbar_or(int id, int threads, bool pred) {
       : "memory");
   return r != 0;
 }
-__device__ __forceinline__ int ld_acquire(const int* ptr) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-  return v;
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
 }
-__device__ __forceinline__ void st_release(int* ptr, int v) {
-  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+__device__ __forceinline__ uint32_t cluster_index() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
 }
-__device__ __forceinline__ void fence_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
+// The cluster-window address of a shared-memory location of CTA `rank`.
+__device__ __forceinline__ uint32_t map_rank(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
 }
-__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-               "r"(src), "r"(bytes)
+__device__ __forceinline__ void remote_arrive(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
                : "memory");
 }
-// Bounded wait for a global counter to reach `target` (acquire); false after the limit.
-__device__ __forceinline__ bool wait_counter(const int* ptr, int target, unsigned* err,
-                                             uint64_t limit_ns) {
-  if (ld_acquire(ptr) >= target) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (ld_acquire(ptr) < target) {
-    if (global_timer_ns() - t0 > limit_ns) {
-      raise_device_error(err, kErrWaitTimeout);
-      return false;
-    }
-    __nanosleep(64);
-  }
-  return true;
+// Bulk copy from this CTA's shared memory into another CTA's, completing on its mbarrier.
+__device__ __forceinline__ void dsmem_copy(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                           uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+      "[%3];" ::"r"(dst_cluster),
+      "r"(src), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
 }
 template <int RB>
 __device__ __forceinline__ uint32_t xswz(uint32_t row, uint32_t colbyte) {
@@ -144,33 +147,69 @@ __global__ void __launch_bounds__(XCfg<NC>::THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.T;
   const int nst = (T + XR - 1) / XR;
+  const int rank = (int)cluster_rank();
+  const int cid = (int)cluster_index();
+  const int out_rank = p.ks;
+  // barriers of both CTA kinds sit at the same offsets, so each side can name the other's
+  const uint32_t c_full = bar, c_empty = bar + 24;     // chain: K/V ring (3)
+  const uint32_t c_eready = bar + 48;                  // chain: -E and W_s stored (x2)
+  const uint32_t c_efree = bar + 64;                   // chain: copy landed (x2, remote)
+  const uint32_t c_grant = bar + 80;                   // chain: slot granted (x4, remote)
+  const uint32_t o_full = bar + 112;                   // output: stage landed (3)
+  const uint32_t o_empty = bar + 136;                  // output: stage consumed (3)
+  const uint32_t o_sfull = bar + 160, o_pfull = bar + 176;
+  const uint32_t o_ofull = bar + 192, o_ofree = bar + 208;
+  const uint32_t o_mdone = bar + 224, o_tslot = bar + 232;
+  // streams of this cluster that exist (the last cluster may hold fewer)
+  const int nmine = max(0, min(p.ks, p.BH - cid * p.ks));
 
-  if ((int)blockIdx.x < p.n_chain) {
-    // ================================================================ chain CTA
-    const uint32_t full = bar, empty = bar + 24;      // stage ring (3)
-    const uint32_t eready = bar + 48;                 // -E and W_s of a stage stored (x2)
-    const uint32_t efree = bar + 64;                  // the stage's copy to the slot done (x2)
-    const int stream = blockIdx.x / Cfg::NG, cg = blockIdx.x % Cfg::NG;
-    const int col_cta = cg * Cfg::COLS;
-    if (threadIdx.x == 0) {
+  if (threadIdx.x == 0) {
+    if (rank < out_rank) {
       for (int s = 0; s < Cfg::C_NST; ++s) {
-        mbar_init(full + 8 * s, 1);
-        mbar_init(empty + 8 * s, NC);
+        mbar_init(c_full + 8 * s, 1);
+        mbar_init(c_empty + 8 * s, NC);
       }
       for (int b = 0; b < 2; ++b) {
-        mbar_init(eready + 8 * b, NC);
-        mbar_init(efree + 8 * b, 1);
+        mbar_init(c_eready + 8 * b, NC);
+        mbar_init(c_efree + 8 * b, 1);
       }
-      fence_mbar_init();
+      for (int g = 0; g < NGRANT; ++g) mbar_init(c_grant + 8 * g, 1);
+    } else {
+      for (int s = 0; s < Cfg::O_NST; ++s) {
+        mbar_init(o_full + 8 * s, 1);
+        mbar_init(o_empty + 8 * s, 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(o_sfull + 8 * b, 1);
+        mbar_init(o_pfull + 8 * b, 4);
+        mbar_init(o_ofull + 8 * b, 1);
+        mbar_init(o_ofree + 8 * b, 4);
+      }
+      mbar_init(o_mdone, 1);
     }
+    fence_mbar_init();
+  }
+  if (rank < out_rank) {
     // -E buffers start at zero: a partial last stage leaves the absent chunks' columns as they
     // are, and the masked product multiplies them by zero scores (they must be finite)
     for (int i = threadIdx.x; i < 4 * Cfg::C_ESUB / 16; i += Cfg::THREADS)
       sts128(sbase + Cfg::C_E_OFF + 16 * i, make_uint4(0u, 0u, 0u, 0u));
     fence_proxy_async_smem();
-    __syncthreads();
+  } else if (warp == 1) {
+    umma::tmem_alloc(o_tslot, 512);
+  }
+  umma::fence_before();
+  // every CTA's barriers are initialised before any CTA of the cluster touches them
+  cluster_sync_all();
+  umma::fence_after();
 
-    if (warp == NC) {
+  if (rank < out_rank) {
+    // ================================================================ chain CTA
+    const int stream = cid * p.ks + rank;
+    const bool active = rank < nmine;
+    const int col_cta = 0;
+    const uint32_t full = c_full, empty = c_empty, eready = c_eready, efree = c_efree;
+    if (active && warp == NC) {
       // ---------------------------------------------------------------- TMA producer
       if (lane == 0) {
         prefetch_tmap(&tmK);
@@ -196,31 +235,30 @@ __global__ void __launch_bounds__(XCfg<NC>::THREADS, 1)
         for (int j = max(0, issued - Cfg::C_NST); j < issued; ++j)
           mbar_wait(full + 8 * (j % Cfg::C_NST), (j / Cfg::C_NST) & 1, p.err, 1000000000ull);
       }
-    } else if (warp == NC + 1) {
+    } else if (active && warp == NC + 1) {
       // ---------------------------------------------------------------- publisher
       if (lane == 0) {
-        uint8_t* ring = p.ring + (size_t)stream * RING * SLOT;
+        int done = 0;
         for (int j = 0; j < nst; ++j) {
           const int b = j & 1;
           if (!mbar_wait(eready + 8 * b, (j >> 1) & 1, p.err, p.wait_ns)) break;
-          // the slot is free once the output CTA has loaded stage j - RING from it
-          if (j >= RING && !wait_counter(p.consumed + stream, j - RING + 1, p.err, p.wait_ns))
-            break;
-          uint8_t* slot = ring + (size_t)(j % RING) * SLOT + (size_t)cg * Cfg::C_ESUB;
+          // the output CTA has set up its pipeline stage for this stage of this stream
+          if (!mbar_wait(c_grant + 8 * (j % NGRANT), (j / NGRANT) & 1, p.err, p.wait_ns)) break;
+          const int it = j * nmine + rank;
+          const uint32_t dst = sbase + (it % Cfg::O_NST) * Cfg::O_STAGE + 2 * XTILE;
+          const uint32_t dbar = map_rank(o_full + 8 * (it % Cfg::O_NST), out_rank);
           const uint32_t sE = sbase + Cfg::C_E_OFF + 2 * Cfg::C_ESUB * b;
           const uint32_t sW = sbase + Cfg::C_W_OFF + Cfg::C_ESUB * b;
-          bulk_store(slot, sE, Cfg::C_ESUB);
-          bulk_store(slot + PART, sE + Cfg::C_ESUB, Cfg::C_ESUB);
-          bulk_store(slot + 2 * PART, sW, Cfg::C_ESUB);
-          bulk_commit();
-          bulk_wait<0>();          // written (and read out of shared memory)
-          fence_async_global();
-          st_release(p.ready + blockIdx.x, j + 1);
-          mbar_arrive(efree + 8 * b);
+          dsmem_copy(map_rank(dst, out_rank), sE, PART, dbar);
+          dsmem_copy(map_rank(dst + PART, out_rank), sE + PART, PART, dbar);
+          dsmem_copy(map_rank(dst + 2 * PART, out_rank), sW, PART, dbar);
+          done = j + 1;
         }
-        bulk_wait<0>();
+        // the last copies have been read out of this CTA's shared memory before it may exit
+        for (int j = max(0, done - 2); j < done; ++j)
+          mbar_wait(efree + 8 * (j & 1), (j >> 1) & 1, p.err, 1000000000ull);
       }
-    } else if (warp < NC) {
+    } else if (active && warp < NC) {
       // ---------------------------------------------------------------- chain warps
       const int g = lane >> 2, tq = lane & 3;
       const int mi = lane >> 3, rr = lane & 7;
@@ -366,233 +404,198 @@ __global__ void __launch_bounds__(XCfg<NC>::THREADS, 1)
           }
       }
     }
+    umma::fence_before();
     __syncthreads();
-    return;
-  }
-  // ================================================================== output CTA
-  const uint32_t full = bar, empty = bar + 24;      // stage ring (3)
-  const uint32_t sfull = bar + 48;    // S accumulator written (x2, MMA commit)
-  const uint32_t pfull = bar + 64;    // P written (x2, 4 epilogue warps)
-  const uint32_t ofull = bar + 80;    // O accumulator complete (x2, MMA commit)
-  const uint32_t ofree = bar + 96;    // O accumulator read out (x2, 4 epilogue warps)
-  const uint32_t mdone = bar + 112;   // every MMA issued has completed
-  const uint32_t tslot = bar + 128;
-  const int oid = blockIdx.x - p.n_chain;
-  // this CTA's streams: oid, oid + n_out, ...; items walk stages in order, streams inside
-  const int nmine = oid < p.BH ? (p.BH - oid + p.n_out - 1) / p.n_out : 0;
-  const int nitems = nst * nmine;
-  auto item_stream = [&](int it) { return oid + (it % nmine) * p.n_out; };
-  auto item_stage = [&](int it) { return it / nmine; };
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < Cfg::O_NST; ++s) {
-      mbar_init(full + 8 * s, 1);
-      mbar_init(empty + 8 * s, 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(sfull + 8 * b, 1);
-      mbar_init(pfull + 8 * b, 4);
-      mbar_init(ofull + 8 * b, 1);
-      mbar_init(ofree + 8 * b, 4);
-    }
-    mbar_init(mdone, 1);
-    fence_mbar_init();
-  }
-  if (warp == 1) umma::tmem_alloc(tslot, 512);
-  umma::fence_before();
-  __syncthreads();
-  umma::fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Cfg::BAR_OFF + 128);
-
-  if (warp == 0) {
-    // ------------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      int issued = 0;
-      for (int it = 0; it < nitems; ++it) {
-        const int s = it % Cfg::O_NST;
-        const int stream = item_stream(it), j = item_stage(it);
-        if (it >= Cfg::O_NST &&
-            !mbar_wait(empty + 8 * s, ((it / Cfg::O_NST) - 1) & 1, p.err, p.wait_ns))
+  } else {
+    // ================================================================ output CTA
+    const uint32_t full = o_full, empty = o_empty, sfull = o_sfull, pfull = o_pfull;
+    const uint32_t ofull = o_ofull, ofree = o_ofree, mdone = o_mdone;
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + Cfg::BAR_OFF + 232);
+    // items walk stages in order, the cluster's streams inside
+    const int nitems = nst * nmine;
+    auto item_rank = [&](int it) { return it % nmine; };
+    auto item_stream = [&](int it) { return cid * p.ks + it % nmine; };
+    auto item_stage = [&](int it) { return it / nmine; };
+    if (warp == 0) {
+      // ------------------------------------------------------------------ producer
+      if (lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        int issued = 0;
+        for (int it = 0; it < nitems; ++it) {
+          const int s = it % Cfg::O_NST;
+          const int stream = item_stream(it), j = item_stage(it);
+          if (it >= Cfg::O_NST &&
+              !mbar_wait(empty + 8 * s, ((it / Cfg::O_NST) - 1) & 1, p.err, p.wait_ns))
+            break;
+          const uint32_t fb = full + 8 * s;
+          const uint32_t st = sbase + s * Cfg::O_STAGE;
+          // Q, K of the stage and the chain CTA's copy of -E and W_s all land on this barrier
+          mbar_arrive_expect_tx(fb, 2 * XTILE + SLOT);
+          tma_load_3d(st, &tmQ, fb, 0, j * XR, stream);
+          tma_load_3d(st + XTILE, &tmK, fb, 0, j * XR, stream);
+          remote_arrive(map_rank(c_grant + 8 * (j % NGRANT), item_rank(it)));
+          issued = it + 1;
+        }
+        for (int it = max(0, issued - Cfg::O_NST); it < issued; ++it)
+          mbar_wait(full + 8 * (it % Cfg::O_NST), (it / Cfg::O_NST) & 1, p.err, 1000000000ull);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ tcgen05 issue warp
+      const uint32_t id_s = umma::idesc_bf16(128, 128, false, false);   // Q K^T
+      const uint32_t id_o = umma::idesc_bf16(128, 64, false, false);    // Q W_s and P (-E)
+      auto issue_s = [&](int it) -> bool {
+        const int s = it % Cfg::O_NST, b = it & 1;
+        if (!mbar_wait_warp(full + 8 * s, (it / Cfg::O_NST) & 1, p.err, p.wait_ns)) return false;
+        umma::fence_after();
+        // the copy has landed: the chain CTA's buffer of this stage is free again
+        if (lane == 0)
+          remote_arrive(map_rank(c_efree + 8 * (item_stage(it) & 1), item_rank(it)));
+        const uint32_t sQ = sbase + s * Cfg::O_STAGE, sK = sQ + XTILE;
+#pragma unroll
+        for (int ks = 0; ks < XKS; ++ks)
+          umma::mma_ss_elect(tmem + XTM_S + 128 * b, umma::desc_kmajor(sQ + 32 * ks),
+                             umma::desc_kmajor(sK + 32 * ks), id_s, ks > 0);
+        umma::commit_elect(sfull + 8 * b);
+        return true;
+      };
+      bool ok = nitems > 0 ? issue_s(0) : true;
+      for (int it = 0; ok && it < nitems; ++it) {
+        const int s = it % Cfg::O_NST, b = it & 1;
+        const uint32_t sQ = sbase + s * Cfg::O_STAGE;
+        const uint32_t sE = sQ + 2 * XTILE, sW = sE + 2 * PART;
+        const uint32_t dO = tmem + XTM_O + 64 * b;
+        if (it >= 2 && !mbar_wait_warp(ofree + 8 * b, ((it >> 1) - 1) & 1, p.err, p.wait_ns))
           break;
-        // every chain CTA of the stream has published stage j (acquire), then the slot is read
-        // through the async proxy
-        bool got = true;
-        for (int cg = 0; cg < Cfg::NG && got; ++cg)
-          got = wait_counter(p.ready + stream * Cfg::NG + cg, j + 1, p.err, p.wait_ns);
-        if (!got) break;
-        fence_async_global();
-        const uint32_t fb = full + 8 * s;
-        const uint32_t st = sbase + s * Cfg::O_STAGE;
-        mbar_arrive_expect_tx(fb, 2 * XTILE + SLOT);
-        tma_load_3d(st, &tmQ, fb, 0, j * XR, stream);
-        tma_load_3d(st + XTILE, &tmK, fb, 0, j * XR, stream);
-        bulk_load(st + 2 * XTILE, p.ring + ((size_t)stream * RING + j % RING) * SLOT, SLOT, fb);
-        issued = it + 1;
+        umma::fence_after();
+#pragma unroll
+        for (int ks = 0; ks < XKS; ++ks)
+          umma::mma_ss_elect(dO, umma::desc_kmajor(sQ + 32 * ks),
+                             umma::desc_kmajor(sW + 32 * ks), id_o, ks > 0);
+        if (!mbar_wait_warp(pfull + 8 * b, (it >> 1) & 1, p.err, p.wait_ns)) break;
+        umma::fence_after();
+#pragma unroll
+        for (int ks = 0; ks < XR / 16; ++ks)
+          umma::mma_ts_elect(dO, tmem + XTM_P + 64 * b + 8 * ks,
+                             umma::desc_kmajor(sE + (ks >> 2) * PART + 32 * (ks & 3)), id_o,
+                             true);
+        umma::commit_elect(ofull + 8 * b);
+        umma::commit_elect(empty + 8 * s);
+        if (it + 1 < nitems) ok = issue_s(it + 1);
       }
-      for (int it = max(0, issued - Cfg::O_NST); it < issued; ++it)
-        mbar_wait(full + 8 * (it % Cfg::O_NST), (it / Cfg::O_NST) & 1, p.err, 1000000000ull);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ tcgen05 issue warp
-    const uint32_t id_s = umma::idesc_bf16(128, 128, false, false);   // Q K^T
-    const uint32_t id_o = umma::idesc_bf16(128, 64, false, false);    // Q W_s and P (-E)
-    auto issue_s = [&](int it) -> bool {
-      const int s = it % Cfg::O_NST, b = it & 1;
-      if (!mbar_wait_warp(full + 8 * s, (it / Cfg::O_NST) & 1, p.err, p.wait_ns)) return false;
-      umma::fence_after();
-      // the slot's contents are in shared memory: the chain CTAs may reuse it
-      if (lane == 0) st_release(p.consumed + item_stream(it), item_stage(it) + 1);
-      const uint32_t sQ = sbase + s * Cfg::O_STAGE, sK = sQ + XTILE;
-#pragma unroll
-      for (int ks = 0; ks < XKS; ++ks)
-        umma::mma_ss_elect(tmem + XTM_S + 128 * b, umma::desc_kmajor(sQ + 32 * ks),
-                           umma::desc_kmajor(sK + 32 * ks), id_s, ks > 0);
-      umma::commit_elect(sfull + 8 * b);
-      return true;
-    };
-    bool ok = nitems > 0 ? issue_s(0) : true;
-    for (int it = 0; ok && it < nitems; ++it) {
-      const int s = it % Cfg::O_NST, b = it & 1;
-      const uint32_t sQ = sbase + s * Cfg::O_STAGE;
-      const uint32_t sE = sQ + 2 * XTILE, sW = sE + 2 * PART;
-      const uint32_t dO = tmem + XTM_O + 64 * b;
-      if (it >= 2 && !mbar_wait_warp(ofree + 8 * b, ((it >> 1) - 1) & 1, p.err, p.wait_ns))
-        break;
-      umma::fence_after();
-#pragma unroll
-      for (int ks = 0; ks < XKS; ++ks)
-        umma::mma_ss_elect(dO, umma::desc_kmajor(sQ + 32 * ks), umma::desc_kmajor(sW + 32 * ks),
-                           id_o, ks > 0);
-      if (!mbar_wait_warp(pfull + 8 * b, (it >> 1) & 1, p.err, p.wait_ns)) break;
-      umma::fence_after();
-#pragma unroll
-      for (int ks = 0; ks < XR / 16; ++ks)
-        umma::mma_ts_elect(dO, tmem + XTM_P + 64 * b + 8 * ks,
-                           umma::desc_kmajor(sE + (ks >> 2) * PART + 32 * (ks & 3)), id_o, true);
-      umma::commit_elect(ofull + 8 * b);
-      umma::commit_elect(empty + 8 * s);
-      if (it + 1 < nitems) ok = issue_s(it + 1);
-    }
-    umma::commit_elect(mdone);
-    mbar_wait_warp(mdone, 0, p.err, 1000000000ull);
-  } else if (warp < 6) {
-    // ------------------------------------------------------------------ epilogue warps 2..5
-    const int q = warp & 3;
-    const int t = 32 * q + lane;
-    const uint32_t tl = (uint32_t)(32 * q) << 16;
-    const int etid = threadIdx.x - 64;
-    const uint32_t sO = sbase + Cfg::O_OT_OFF;
-    auto mask = [&](int it) -> bool {
-      const int b = it & 1;
-      if (!mbar_wait_warp(sfull + 8 * b, (it >> 1) & 1, p.err, p.wait_ns)) return false;
-      umma::fence_after();
-#pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-        uint32_t v[32] = {}, v2[32] = {}, w[32];
-        if (2 * pp <= q) {
-          umma::ld32x32(tmem + tl + XTM_S + 128 * b + 64 * pp, v);
+      umma::commit_elect(mdone);
+      mbar_wait_warp(mdone, 0, p.err, 1000000000ull);
+    } else if (warp < 6) {
+      // ------------------------------------------------------------------ epilogue warps 2..5
+      const int q = warp & 3;
+      const int t = 32 * q + lane;
+      const uint32_t tl = (uint32_t)(32 * q) << 16;
+      const int etid = threadIdx.x - 64;
+      const uint32_t sO = sbase + Cfg::O_OT_OFF;
+      auto mask = [&](int it) -> bool {
+        const int b = it & 1;
+        if (!mbar_wait_warp(sfull + 8 * b, (it >> 1) & 1, p.err, p.wait_ns)) return false;
+        umma::fence_after();
+  #pragma unroll
+        for (int pp = 0; pp < 2; ++pp) {
+          uint32_t v[32] = {}, v2[32] = {}, w[32];
+          if (2 * pp <= q) {
+            umma::ld32x32(tmem + tl + XTM_S + 128 * b + 64 * pp, v);
+            umma::wait_ld();
+            umma::reg_fence(v);
+          }
+          if (2 * pp + 1 <= q) {
+            umma::ld32x32(tmem + tl + XTM_S + 128 * b + 64 * pp + 32, v2);
+            umma::wait_ld();
+            umma::reg_fence(v2);
+          }
+  #pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int s0 = 64 * pp + 2 * i, s1 = s0 + 1;
+            const uint32_t x0 = i < 16 ? v[2 * i] : v2[2 * i - 32];
+            const uint32_t x1 = i < 16 ? v[2 * i + 1] : v2[2 * i - 31];
+            w[i] = pack_bf16(s0 <= t ? __uint_as_float(x0) : 0.f,
+                             s1 <= t ? __uint_as_float(x1) : 0.f);
+          }
+          umma::st32x32(tmem + tl + XTM_P + 64 * b + 32 * pp, w);
+        }
+        umma::wait_st();
+        umma::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(pfull + 8 * b);
+        return true;
+      };
+      auto drain = [&](int it) -> bool {
+        const int b = it & 1;
+        const bool got = mbar_wait_warp(ofull + 8 * b, (it >> 1) & 1, p.err, p.wait_ns);
+        if (got && etid == 0) bulk_wait_read<0>();
+        if (xbar_or(1, 128, !got)) return false;
+        umma::fence_after();
+        uint32_t v[64];
+  #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[32];
+          umma::ld32x32(tmem + tl + XTM_O + 64 * b + 32 * h, r);
           umma::wait_ld();
-          umma::reg_fence(v);
+          umma::reg_fence(r);
+  #pragma unroll
+          for (int i = 0; i < 32; ++i) v[32 * h + i] = r[i];
         }
-        if (2 * pp + 1 <= q) {
-          umma::ld32x32(tmem + tl + XTM_S + 128 * b + 64 * pp + 32, v2);
-          umma::wait_ld();
-          umma::reg_fence(v2);
+        umma::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ofree + 8 * b);
+  #pragma unroll
+        for (int k = 0; k < 8; ++k)
+          sts128(sO + xswz<128>(t, 16 * k),
+                 make_uint4(pack_bf16(__uint_as_float(v[8 * k]), __uint_as_float(v[8 * k + 1])),
+                            pack_bf16(__uint_as_float(v[8 * k + 2]), __uint_as_float(v[8 * k + 3])),
+                            pack_bf16(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5])),
+                            pack_bf16(__uint_as_float(v[8 * k + 6]),
+                                      __uint_as_float(v[8 * k + 7]))));
+        fence_proxy_async_smem();
+        xbar_sync(1, 128);
+        if (etid == 0) {
+          tma_store_3d(&tmO, sO, 0, item_stage(it) * XR, item_stream(it));
+          bulk_commit();
         }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int s0 = 64 * pp + 2 * i, s1 = s0 + 1;
-          const uint32_t x0 = i < 16 ? v[2 * i] : v2[2 * i - 32];
-          const uint32_t x1 = i < 16 ? v[2 * i + 1] : v2[2 * i - 31];
-          w[i] = pack_bf16(s0 <= t ? __uint_as_float(x0) : 0.f,
-                           s1 <= t ? __uint_as_float(x1) : 0.f);
-        }
-        umma::st32x32(tmem + tl + XTM_P + 64 * b + 32 * pp, w);
+        return true;
+      };
+      for (int it = 0; it < nitems; ++it) {
+        const bool ok = mask(it);
+        if (xbar_or(1, 128, !ok)) break;
+        if (it >= 1 && !drain(it - 1)) break;
+        if (it + 1 == nitems) drain(it);
       }
-      umma::wait_st();
-      umma::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(pfull + 8 * b);
-      return true;
-    };
-    auto drain = [&](int it) -> bool {
-      const int b = it & 1;
-      const bool got = mbar_wait_warp(ofull + 8 * b, (it >> 1) & 1, p.err, p.wait_ns);
-      if (got && etid == 0) bulk_wait_read<0>();
-      if (xbar_or(1, 128, !got)) return false;
-      umma::fence_after();
-      uint32_t v[64];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t r[32];
-        umma::ld32x32(tmem + tl + XTM_O + 64 * b + 32 * h, r);
-        umma::wait_ld();
-        umma::reg_fence(r);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[32 * h + i] = r[i];
-      }
-      umma::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(ofree + 8 * b);
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        sts128(sO + xswz<128>(t, 16 * k),
-               make_uint4(pack_bf16(__uint_as_float(v[8 * k]), __uint_as_float(v[8 * k + 1])),
-                          pack_bf16(__uint_as_float(v[8 * k + 2]), __uint_as_float(v[8 * k + 3])),
-                          pack_bf16(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5])),
-                          pack_bf16(__uint_as_float(v[8 * k + 6]),
-                                    __uint_as_float(v[8 * k + 7]))));
-      fence_proxy_async_smem();
-      xbar_sync(1, 128);
-      if (etid == 0) {
-        tma_store_3d(&tmO, sO, 0, item_stage(it) * XR, item_stream(it));
-        bulk_commit();
-      }
-      return true;
-    };
-    for (int it = 0; it < nitems; ++it) {
-      const bool ok = mask(it);
-      if (xbar_or(1, 128, !ok)) break;
-      if (it >= 1 && !drain(it - 1)) break;
-      if (it + 1 == nitems) drain(it);
+      if (etid == 0) bulk_wait<0>();
     }
-    if (etid == 0) bulk_wait<0>();
+    umma::fence_before();
+    __syncthreads();
+    if (warp == 1) umma::tmem_dealloc(tmem, 512);
   }
-  umma::fence_before();
-  __syncthreads();
-  if (warp == 1) umma::tmem_dealloc(tmem, 512);
+  // no CTA leaves while another of the cluster may still reach its shared memory
+  cluster_sync_all();
 }
 
 }  // namespace
 
-// Chain CTAs per stream (1, 2 or 4) and output CTAs for the split form, or 0 if the streams
-// leave too few SMs: every CTA must be resident (one per SM) and an output CTA serves at most
-// two streams.
-int dual_xsm_plan(int streams, int sms, int* n_out) {
-  for (int ng : {4, 2, 1}) {
-    const int chain = streams * ng;
-    const int avail = sms - chain;
-    if (avail >= (streams + 1) / 2 && avail >= 1) {
-      *n_out = std::min(avail, streams);
-      return ng;
+// Streams per cluster (1 or 2; the cluster adds one output CTA) for the split form, or 0 if the
+// streams leave too few SMs: every cluster must be resident at once, one CTA per SM.
+int dual_xsm_plan(int streams, int sms, int* n_clusters) {
+  const int forced = tuning(kTuneDualClusterStreams);
+  for (int ks : {1, 2}) {
+    if (forced && ks != forced) continue;
+    const int clusters = (streams + ks - 1) / ks;
+    if (clusters * (ks + 1) <= sms) {
+      *n_clusters = clusters;
+      return ks;
     }
   }
   return 0;
 }
 
-size_t dual_xsm_workspace_bytes(int B, int H) {
-  const size_t bh = (size_t)B * H;
-  return bh * RING * SLOT + 256 * ((bh * 5 * sizeof(int) + 255) / 256);
-}
-
-int launch_dual_xsm(const StateArgs& a, int ng, int n_out, const LaunchCtx& ctx) {
+int launch_dual_xsm(const StateArgs& a, int ks, int n_clusters, const LaunchCtx& ctx) {
+  using Cfg = XCfg<4>;
   const int BH = a.B * a.H;
-  const size_t ring_bytes = (size_t)BH * RING * SLOT;
-  if (!a.ws || a.ws_bytes < dual_xsm_workspace_bytes(a.B, a.H)) return kWorkspace;
-  uint8_t* ws = static_cast<uint8_t*>(a.ws);
-  int* ready = reinterpret_cast<int*>(ws + ring_bytes);      // [BH * 4] (NG <= 4)
-  int* consumed = ready + (size_t)BH * 4;                    // [BH]
   CUtensorMap tq, tk, tv, to;
   const uint64_t dims[3] = {(uint64_t)XD, (uint64_t)a.T, (uint64_t)BH};
   const uint64_t strides[2] = {(uint64_t)XD * 2, (uint64_t)a.T * XD * 2};
@@ -604,40 +607,36 @@ int launch_dual_xsm(const StateArgs& a, int ng, int n_out, const LaunchCtx& ctx)
       !make_tmap_3d(&tv, a.V, bf, dims, strides, box, sw, ctx.msg) ||
       !make_tmap_3d(&to, a.O, bf, dims, strides, box, sw, ctx.msg))
     return kCuda;
-  cudaError_t e = cudaMemsetAsync(ready, 0, sizeof(int) * (size_t)BH * 5, ctx.stream);
-  if (e != cudaSuccess) {
-    *ctx.msg = std::string("dual_xsm setup: ") + cudaGetErrorString(e);
-    return kCuda;
-  }
-  const int limit = tuning(kTuneWaitLimitNs);
-  XParams p{a.eta, a.eta_scalar, a.S0, a.S_out, a.T, BH, BH * ng, n_out, ws, ready, consumed,
-            ctx.err, limit > 0 ? (uint64_t)limit : 4000000000ull};
-  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, XParams) = nullptr;
-  int threads = 0, smem = 0;
-  switch (ng) {
-    case 1: kern = dual_xsm_kernel<4>; threads = XCfg<4>::THREADS; smem = XCfg<4>::SMEM; break;
-    case 2: kern = dual_xsm_kernel<2>; threads = XCfg<2>::THREADS; smem = XCfg<2>::SMEM; break;
-    case 4: kern = dual_xsm_kernel<1>; threads = XCfg<1>::THREADS; smem = XCfg<1>::SMEM; break;
-    default:
-      *ctx.msg = "dual_xsm: chain CTAs per stream must be 1, 2 or 4";
-      return kUnsupported;
-  }
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto kern = dual_xsm_kernel<4>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) {
     *ctx.msg = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
     return kCuda;
   }
-  // cooperative: every CTA resident at once (the chain and output CTAs wait on each other)
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(BH * ng + n_out);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = smem;
+  cfg.gridDim = dim3(n_clusters * (ks + 1));
+  cfg.blockDim = dim3(Cfg::THREADS);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
   cfg.stream = ctx.stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks + 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // one wave: clusters that could not all be resident would still be correct (they never wait
+  // on each other) but slower; the caller falls back to the single-SM form then
+  int max_clusters = 0;
+  e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+  if (e != cudaSuccess || max_clusters < n_clusters) {
+    cudaGetLastError();
+    return kUnsupported;
+  }
+  const int limit = tuning(kTuneWaitLimitNs);
+  XParams p{a.eta, a.eta_scalar, a.S0, a.S_out, a.T, BH, ks, ctx.err,
+            limit > 0 ? (uint64_t)limit : 4000000000ull};
   e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, to, p);
   if (e != cudaSuccess) {
     *ctx.msg = std::string("dual_xsm launch: ") + cudaGetErrorString(e);

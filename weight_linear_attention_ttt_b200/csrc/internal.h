@@ -72,6 +72,7 @@ enum TuneKey : int {
   kTuneAssocParts,            // superchunks per stream of the associative mode
   kTuneWaitLimitNs,           // limit of the d = 64 dual-form pipeline waits, ns (0: 4 s)
   kTuneInplaceChunksPerLaunch,  // In-Place: 1 = one chunk per launch, 0 / 2 = chunk pairs
+  kTuneDualClusterStreams,    // dual form split across SMs: streams per cluster, 1 or 2
   kTuneCount
 };
 enum DualKernel : int { kDualKernelAuto = 0, kDualKernelWarp = 1, kDualKernelPair = 2,
@@ -97,12 +98,12 @@ int launch_dual_simt(const StateArgs& a, const LaunchCtx& ctx);
 // d = 64, C = 16, 32 or 64, bf16: chain on warp MMAs, outputs per stage on tcgen05; split =
 // CTAs per stream (1, 2 or 4), dual_tc_split() the automatic choice.
 bool dual_tc_supported(int d, int C, int dt);
-// d = 64, C = 16, bf16: the chain and the output products on separate SMs (one cooperative
-// launch; dual_xsm.cu). dual_xsm_plan returns the chain CTAs per stream (0: not possible).
+// d = 64, C = 16, bf16: the chain and the output products on separate SMs of one cluster
+// (dual_xsm.cu). dual_xsm_plan returns the streams per cluster (0: not possible) and the
+// cluster count; launch_dual_xsm returns kUnsupported when the clusters cannot all be resident.
 inline bool dual_xsm_applicable(int d, int C, int dt) { return dt == 1 && d == 64 && C == 16; }
-int dual_xsm_plan(int streams, int sms, int* n_out);
-size_t dual_xsm_workspace_bytes(int B, int H);
-int launch_dual_xsm(const StateArgs& a, int ng, int n_out, const LaunchCtx& ctx);
+int dual_xsm_plan(int streams, int sms, int* n_clusters);
+int launch_dual_xsm(const StateArgs& a, int ks, int n_clusters, const LaunchCtx& ctx);
 int dual_tc_split(int streams, int sms);
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx);
 

@@ -34,7 +34,8 @@ static const TuneName kTuneNames[] = {{"dual_column_split", kTuneDualColumnSplit
                                       {"assoc_parts", kTuneAssocParts},
                                       {"wait_limit_ns", kTuneWaitLimitNs},
                                       {"inplace_chunks_per_launch",
-                                       kTuneInplaceChunksPerLaunch}};
+                                       kTuneInplaceChunksPerLaunch},
+                                      {"dual_cluster_streams", kTuneDualClusterStreams}};
 static int tune_key(const char* name) {
   if (!name) return -1;
   for (const auto& t : kTuneNames)
@@ -217,10 +218,7 @@ int ttt_read_device_error(unsigned* value) {
   return TTT_OK;
 }
 
-size_t ttt_linear_dual_workspace_size(int B, int H, int T, int d, int C, int dt) {
-  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0) return 0;
-  return dual_xsm_applicable(d, C, dt) ? dual_xsm_workspace_bytes(B, H) : 0;
-}
+size_t ttt_linear_dual_workspace_size(int, int, int, int, int, int) { return 0; }
 
 int ttt_linear_dual_fwd(const void* Q, const void* K, const void* V, const float* eta,
                         float eta_scalar, const float* W0, void* O, float* W_out, int B, int H,
@@ -230,19 +228,6 @@ int ttt_linear_dual_fwd(const void* Q, const void* K, const void* V, const float
               workspace_bytes};
   int st = check_state_args("ttt_linear_dual_fwd", a, 0);
   if (st != TTT_OK) return st;
-  if (workspace && workspace_bytes) {   // optional: used by the split form when large enough
-    if (!aligned16(workspace))
-      return fail(TTT_ERR_INVALID_ARG, "ttt_linear_dual_fwd: workspace must be 16-byte aligned");
-    const size_t esz = dt == TTT_DTYPE_F32 ? 4 : 2;
-    const size_t nx = (size_t)B * H * T * d * esz, ns = (size_t)B * H * d * d * 4;
-    const size_t ne = (size_t)B * H * T * 4;
-    if (overlap(workspace, workspace_bytes, Q, nx) || overlap(workspace, workspace_bytes, K, nx) ||
-        overlap(workspace, workspace_bytes, V, nx) || overlap(workspace, workspace_bytes, O, nx) ||
-        overlap(workspace, workspace_bytes, W_out, ns) ||
-        overlap(workspace, workspace_bytes, W0, ns) || overlap(workspace, workspace_bytes, eta, ne))
-      return fail(TTT_ERR_INVALID_ARG,
-                  "ttt_linear_dual_fwd: the workspace must not overlap an input or an output");
-  }
   if (!(d == 32 || d == 64 || d == 128) || C > 64)
     return fail(TTT_ERR_UNSUPPORTED,
                 "ttt_linear_dual_fwd: supported d in {32, 64, 128} and 1 <= C <= 64");
