@@ -89,15 +89,15 @@ uint64_t ttt_launch_count(void);
  *   "dual_kernel"        dual form with bf16 inputs and C = 16: 1 = all products on warp MMAs
  *                        (one warp per 16 columns), 2 = the same on chain/output warp pairs,
  *                        3 = chain on warp MMAs with the outputs per 128-token stage on the
- *                        tcgen05 tensor cores (d = 64 only; what 0 picks for d = 64 without
- *                        cluster room), 4 = the same with the chain and the outputs on
- *                        separate SMs of a cluster (d = 64, C = 16; what 0 picks when the
- *                        streams leave room).
+ *                        tcgen05 tensor cores (d = 64 only; what 0 picks for d = 64),
+ *                        4 = the same with the chain and the outputs on separate SMs of a
+ *                        thread-block cluster (d = 64, C = 16, where the streams leave one
+ *                        more SM per one or two streams; measured slower than 3).
  *   "dual_cluster_streams"  dual_kernel 4: streams per cluster, 1 or 2 (each cluster adds one
  *                        output CTA).
  *   "dual_warp_cols"     d = 64 with C = 16: 8 or 16 output columns per warp, for dual_kernel
- *                        1 and for the stage kernel (dual_kernel 3; 8-column chains run two
- *                        per SM sub-partition).
+ *                        1 and for the stage kernel (dual_kernel 3; by default 16 with one CTA
+ *                        per stream, 8 when a stream is split over several CTAs).
  *   "dual_stage_chunks"  dual_kernel 1 with d = 64 and 8 columns per warp: 4 or 8 chunks per
  *                        pipeline stage.
  *   "assoc_parts"        superchunks per stream of the associative mode (must divide T / C).
@@ -139,10 +139,6 @@ int ttt_read_device_error(unsigned* value);
  *  warp MMAs, the outputs per 128-token stage on tcgen05); other supported shapes run the
  *  CUDA-core path.
  *  Workspace: none (ttt_linear_dual_workspace_size returns 0; `workspace` may be NULL).
- *  bf16, d == 64, C == 16: where the streams leave one more SM per one or two streams, the
- *  chain of each stream and its output products run on separate SMs of one thread-block
- *  cluster; otherwise each stream's work stays on its own SMs. Both forms compute the same
- *  result (outputs equal within bf16 rounding, the final state bit for bit).
  * ------------------------------------------------------------------------------------------ */
 size_t ttt_linear_dual_workspace_size(int B, int H, int T, int d, int C, int dt);
 int ttt_linear_dual_fwd(const void* Q, const void* K, const void* V, const float* eta,

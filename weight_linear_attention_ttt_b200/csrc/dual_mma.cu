@@ -606,26 +606,21 @@ int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
   // d = 64: the chain on warp MMAs with the outputs per 128-token stage on tcgen05 (dual_tc.cu)
   // measured fastest on the 125M- and 1.3B-layer shapes; the all-warp-MMA forms below remain
   // selectable through ttt_set_tuning("dual_kernel", ...).
-  // d = 64, C = 16: the chain on some SMs, the stage products on others of the same cluster
-  // (dual_xsm.cu) where the streams leave enough SMs free; measured faster than one SM doing
-  // both, since the output work slows the latency-bound chain it shares an SM with.
-  if (dual_xsm_applicable(a.d, a.C, a.dt) &&
-      (kernel == kDualKernelAuto || kernel == kDualKernelSplit)) {
+  // d = 64, C = 16, on request: the chain on some SMs, the stage products on others of the same
+  // cluster (dual_xsm.cu). Correct, but measured slower than one SM doing both (the hand-off
+  // moves the bound to the output CTA's epilogue and to the chain's wait for its slot), so the
+  // automatic choice is the single-SM stage kernel below.
+  if (dual_xsm_applicable(a.d, a.C, a.dt) && kernel == kDualKernelSplit) {
     int n_clusters = 0;
     const int ks = dual_xsm_plan(streams, sms, &n_clusters);
-    if (ks) {
-      const int r = launch_dual_xsm(a, ks, n_clusters, ctx);
-      if (r != kUnsupported) return r;
-    }
-    if (kernel == kDualKernelSplit) {
-      *ctx.msg = "dual form: the split form needs one more SM per one or two streams, and "
-                 "its clusters resident at once";
-      return kUnsupported;
-    }
+    const int r = ks ? launch_dual_xsm(a, ks, n_clusters, ctx) : kUnsupported;
+    if (r == kUnsupported)
+      *ctx.msg = "dual form: the split form needs one more SM per one or two streams, and its "
+                 "clusters resident at once";
+    return r;
   }
   // (C = 32 and 64 exist only in that form)
-  if (a.d == 64 && (a.C != 16 || kernel == kDualKernelAuto || kernel == kDualKernelTensor ||
-                    kernel == kDualKernelSplit)) {
+  if (a.d == 64 && (a.C != 16 || kernel == kDualKernelAuto || kernel == kDualKernelTensor)) {
     const int split = (forced_split == 1 || forced_split == 2 || forced_split == 4)
                           ? forced_split
                           : dual_tc_split(streams, sms);

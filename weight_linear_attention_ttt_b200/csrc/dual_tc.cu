@@ -796,8 +796,12 @@ bool dual_tc_supported(int d, int C, int dt) {
 }
 
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx) {
-  // columns per chain warp: 8 (two chains per sub-partition) or 16, for 16-token chunks
-  const bool eight = tuning(kTuneDualWarpCols) == 8;
+  // Columns per chain warp for 16-token chunks: 16 with one CTA per stream (4 chain warps, one
+  // per SM sub-partition; 42.6 against 52.7 us with 8 columns on the 125M-layer shape), 8 when
+  // a stream is split over CTAs (444 against 477 us on the 1.3B-layer shape, 3.20 against
+  // 3.56 ms on 4 streams of 262144 tokens). The tuning choice overrides.
+  const int wcols = tuning(kTuneDualWarpCols);
+  const bool eight = wcols ? wcols == 8 : split >= 2;
   switch (a.C) {
     case 16:
       return eight ? launch_split<1, 8>(a, split, ctx) : launch_split<1, 16>(a, split, ctx);
