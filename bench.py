@@ -39,7 +39,7 @@ def metric_of(w) -> str:
     return METRIC_BWD if w.kind.endswith("_bwd") else METRIC
 DEFAULT_WORKLOAD = "assoc_bf16_B4H16T65536_d128C64"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DOMINANT_KERNEL = {"dual": ("dual_xsm_kernel", "dual_xsm.cu"),
+DOMINANT_KERNEL = {"dual": ("dual_tc_kernel", "dual_tc.cu"),
                    "dual_seg": ("dual_tc_kernel", "dual_tc.cu"),
                    "assoc": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu"),
