@@ -92,7 +92,10 @@ uint64_t ttt_launch_count(void);
  *                        tcgen05 tensor cores (d = 64 only; what 0 picks for d = 64),
  *                        4 = the same with the chain and the outputs on separate SMs of a
  *                        thread-block cluster (d = 64, C = 16, where the streams leave one
- *                        more SM per one or two streams; measured slower than 3).
+ *                        more SM per one or two streams; measured slower than 3),
+ *                        5 = the state resident in TMEM, updated once per 128-token stage on
+ *                        tcgen05, with the chain reduced to 16 x 16 key-Gram-block updates
+ *                        (d = 64, C = 16, 32 or 64).
  *   "dual_cluster_streams"  dual_kernel 4: streams per cluster, 1 or 2 (each cluster adds one
  *                        output CTA).
  *   "dual_warp_cols"     d = 64 with C = 16: 8 or 16 output columns per warp, for dual_kernel

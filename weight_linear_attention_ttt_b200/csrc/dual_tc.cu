@@ -88,21 +88,6 @@ struct TcParams {
   uint64_t wait_ns;   // limit of every pipeline wait; copies in flight get a fixed second
 };
 
-__device__ __forceinline__ void bar_sync_named(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-// Named barrier that also ORs a predicate over its threads: a failed (timed-out) wait in any
-// epilogue warp makes all four leave their loop together.
-__device__ __forceinline__ bool bar_or_named(int id, int threads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n"
-      " selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(threads)
-      : "memory");
-  return r != 0;
-}
 // Transpose of an 8x8 bf16 tile held as one register per lane in MMA-fragment order.
 __device__ __forceinline__ uint32_t movm_t(uint32_t x) {
   uint32_t y;

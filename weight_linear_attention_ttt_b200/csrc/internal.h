@@ -76,7 +76,7 @@ enum TuneKey : int {
   kTuneCount
 };
 enum DualKernel : int { kDualKernelAuto = 0, kDualKernelWarp = 1, kDualKernelPair = 2,
-                        kDualKernelTensor = 3, kDualKernelSplit = 4 };
+                        kDualKernelTensor = 3, kDualKernelSplit = 4, kDualKernelGram = 5 };
 int tuning(TuneKey key);
 // Records the detail returned by ttt_last_error_message() on this thread.
 void set_last_error(const std::string& msg);
@@ -105,6 +105,10 @@ inline bool dual_xsm_applicable(int d, int C, int dt) { return dt == 1 && d == 6
 int dual_xsm_plan(int streams, int sms, int* n_clusters);
 int launch_dual_xsm(const StateArgs& a, int ks, int n_clusters, const LaunchCtx& ctx);
 int dual_tc_split(int streams, int sms);
+// d = 64, C = 16, 32 or 64, bf16: the state in TMEM, updated once per 128-token stage on
+// tcgen05; the chain is a blocked substitution over the stage's key Gram blocks (dual_gram.cu).
+bool dual_gram_supported(int d, int C, int dt);
+int launch_dual_gram(const StateArgs& a, const LaunchCtx& ctx);
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx);
 
 // Associative mode.

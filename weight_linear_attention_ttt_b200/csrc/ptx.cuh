@@ -47,6 +47,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the phase with the given parity (no suspension).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Slow path of a bounded wait: spins until the phase with the given parity completes or
 // `limit_ns` of global time passes, then raises the error word and returns false. Kept out of
 // line so that the inline fast path of mbar_wait is one try_wait and a branch.
@@ -75,6 +86,22 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, un
   return __all_sync(0xffffffffu, mbar_wait_slow(bar, parity, err, limit_ns));
 }
 
+// ------------------------------------------------------------------------------ named barriers
+__device__ __forceinline__ void bar_sync_named(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+// Named barrier that also ORs a predicate over its threads: a failed (timed-out) wait in any
+// participating warp makes all of them leave their loop together.
+__device__ __forceinline__ bool bar_or_named(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
 // ------------------------------------------------------------------------------ TMA
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
