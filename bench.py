@@ -548,6 +548,8 @@ def run_ours(args, w, rank, world, local_rank):
 
     pk, pk_kind = peaks()
     kname, ksrc = DOMINANT_KERNEL[w.kind]
+    if w.kind == "dual" and ttt.get_tuning("dual_kernel") == 5:   # the TMEM-state kernel
+        kname, ksrc = "dual_gram_kernel", "dual_gram.cu"
     launches_per_step = launches / args.steps
     # the roofline is the slower of the flops at the tensor peak and the bytes at HBM bandwidth
     t_flops = algo["flops"] / (pk["bf16_tflops"] * 1e12)
