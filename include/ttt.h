@@ -179,7 +179,10 @@ int ttt_linear_dual_seg_fwd(const void* Q, const void* K, const void* V, const f
  *
  *  Q, K, V, O [B,H,T,d]; eta [B,H,T] fp32 or NULL (eta_scalar); S0 [B,H,d,d] fp32 or NULL
  *  (zeros); S_out [B,H,d,d] fp32, may equal S0.
- *  Supported: bf16, d == 128, C == 64, T % C == 0 (tensor-core path).
+ *  Supported: bf16, d == 64 or 128, C == 16, 32 or 64, T % 64 == 0 (tensor-core path). The
+ *  result does not depend on C (the recurrence is per token; C only sets the evaluation
+ *  granularity): every C is evaluated in 64-token tiles, and d = 64 runs zero-padded to 128
+ *  inside the kernel, at the cost of d = 128 arithmetic for half the bytes.
  *  Workspace: ttt_assoc_scan_workspace_size() bytes (superchunk states, fp32).
  * ------------------------------------------------------------------------------------------ */
 size_t ttt_assoc_scan_workspace_size(int B, int H, int T, int d, int C, int dt);
@@ -197,8 +200,8 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
  *  Q, K, V, O [B,H,T,d] bf16; eta [B,H,T] fp32 or NULL (eta_scalar); S0, M0 [B,H,d,d] fp32 or
  *  NULL (zeros); S_out, M_out [B,H,d,d] fp32 (S_out may equal S0, M_out may equal M0).
  *  beta in [0.25, 0.9] (beta = 0 is ttt_assoc_scan_fwd; the two-pass evaluation subtracts
- *  outputs of size ~1/(1 - beta), which bounds beta for bf16 outputs). Supported: bf16,
- *  d == 128, C == 64.
+ *  outputs of size ~1/(1 - beta), which bounds beta for bf16 outputs). Supported: as
+ *  ttt_assoc_scan_fwd (bf16, d == 64 or 128, C == 16, 32 or 64, T % 64 == 0).
  *  Workspace: ttt_assoc_momentum_workspace_size() bytes. Runs as one plain associative pass and
  *  one decayed pass whose output stage combines the two outputs, then an elementwise
  *  combination of the states (see assoc_momentum.cu).
@@ -222,8 +225,8 @@ int ttt_assoc_momentum_fwd(const void* Q, const void* K, const void* V, const fl
  *  dS_out [B,H,d,d] fp32 or NULL (zeros). Outputs: dQ, dK, dV [B,H,T,d] bf16; deta [B,H,T]
  *  fp32 (per token also when eta is NULL: the scalar's gradient is their sum); dS0 [B,H,d,d]
  *  fp32. Outputs must not overlap the inputs or each other.
- *  Supported: bf16, d == 128, C == 64, T % C == 0. C is the evaluation granularity; the
- *  gradients do not depend on it beyond rounding.
+ *  Supported: as ttt_assoc_scan_fwd (bf16, d == 64 or 128, C == 16, 32 or 64, T % 64 == 0).
+ *  C is the evaluation granularity; the gradients do not depend on it beyond rounding.
  *  Workspace: ttt_assoc_scan_bwd_workspace_size() bytes.
  *  Runs as three passes of the forward kernel (dQ in forward order; dV and dK through the
  *  reverse-order recurrence of the state gradient) and one elementwise pass.
@@ -314,7 +317,7 @@ int ttt_dual_state_fold(const float* W0, const float* A_maps, const float* B_map
  *  K, V [B,H,T,d]; eta [B,H,T] fp32 or NULL (eta_scalar); dS [B,H,d,d] fp32 output.
  *  A context-parallel caller gives each device a slice of the sequence, exchanges the slices'
  *  increments, and starts ttt_assoc_scan_fwd on its slice from S0 plus the earlier slices'
- *  increments. Supported: bf16, d == 128, C == 64, T % C == 0. No workspace.
+ *  increments. Supported: as ttt_assoc_scan_fwd. No workspace.
  * ------------------------------------------------------------------------------------------ */
 int ttt_assoc_state_fwd(const void* K, const void* V, const float* eta, float eta_scalar,
                         float* dS, int B, int H, int T, int d, int C, int dt,

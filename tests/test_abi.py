@@ -143,9 +143,12 @@ def test_backward_validation(lib, fn, base, kw, status):
 
 
 def test_backward_chunk_size_rules(lib):
-    # the dual form's backward runs the C = 16 mini-batch only; the associative one C = 64
+    # the dual form's backward runs the C = 16 mini-batch only; the associative one any C of
+    # 16, 32, 64 on 64-token tiles (T % 64 == 0), and no other head dim than 64 or 128
     assert _bwd(lib, "ttt_linear_dual_bwd", d=64, C=32, T=64, ws_bytes=1 << 30) == 2
-    assert _bwd(lib, "ttt_assoc_scan_bwd", d=128, C=16, T=64, ws_bytes=1 << 30) == 2
+    assert _bwd(lib, "ttt_assoc_scan_bwd", d=128, C=16, T=48, ws_bytes=1 << 30) == 2
+    assert _bwd(lib, "ttt_assoc_scan_bwd", d=128, C=8, T=64, ws_bytes=1 << 30) == 2
+    assert _bwd(lib, "ttt_assoc_scan_bwd", d=96, C=64, T=64, ws_bytes=1 << 30) == 2
     assert lib.ttt_launch_count() == 0
 
 
@@ -156,7 +159,9 @@ def test_workspace_size_queries(lib):
     assert lib.ttt_linear_dual_bwd_workspace_size(8, 12, 2040, 64, 16, 1) == 0   # T % C
     assert lib.ttt_linear_dual_bwd_workspace_size(1, 1, 64, 64, 16, 0) == 0      # fp32
     assert lib.ttt_assoc_scan_bwd_workspace_size(4, 16, 65536, 128, 64, 1) > 0
-    assert lib.ttt_assoc_scan_bwd_workspace_size(4, 16, 65536, 64, 64, 1) == 0
+    assert lib.ttt_assoc_scan_bwd_workspace_size(4, 16, 65536, 64, 16, 1) > 0
+    assert lib.ttt_assoc_scan_bwd_workspace_size(4, 16, 65536, 96, 64, 1) == 0
+    assert lib.ttt_assoc_scan_workspace_size(4, 16, 65536 + 32, 128, 32, 1) == 0   # T % 64
     assert lib.ttt_assoc_momentum_workspace_size(4, 16, 65536, 128, 64, 1) > 0
     assert lib.ttt_assoc_momentum_workspace_size(4, 16, 100, 128, 64, 1) == 0
     # the convolved embeddings (bf16, 256-byte aligned) and one 256-byte counter slot
@@ -174,7 +179,7 @@ def test_momentum_validation(lib):
 
     assert mom(0.95) == 2 and mom(0.1) == 2 and mom(1.0) == 2   # outside [0.25, 0.9]
     assert mom(0.5, M_out=0) == 1
-    assert mom(0.5, d=64) == 2
+    assert mom(0.5, d=96) == 2
     assert mom(0.5, M_out=6 * A + 64) == 1                      # M_out overlaps O
     assert lib.ttt_launch_count() == 0
 

@@ -110,10 +110,11 @@ def test_full_associative_workload_sampled_streams(cuda_lib):
 
 
 def test_errors(cuda_lib):
-    x = make(1, 1, 128, seed=1)
+    x96 = make(1, 1, 96, seed=1)   # T = 96: a multiple of C = 32 but not of the 64-token tile
     with pytest.raises(ttt.TTTError) as e:
-        ttt.ttt_assoc_scan_bwd(x["Q"], x["K"], x["V"], x["eta"], None, x["dO"], C=32)
+        ttt.ttt_assoc_scan_bwd(x96["Q"], x96["K"], x96["V"], x96["eta"], None, x96["dO"], C=32)
     assert e.value.status == 2
+    x = make(1, 1, 128, seed=1)
     with pytest.raises(ttt.TTTError) as e:
         run(x, workspace=torch.empty(16, device="cuda", dtype=torch.uint8))
     assert e.value.status == 3

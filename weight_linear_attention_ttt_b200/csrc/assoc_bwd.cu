@@ -48,30 +48,34 @@ __device__ __forceinline__ uint16_t f_to_bf16(float f) {
   return *reinterpret_cast<const uint16_t*>(&b);
 }
 
-// One warp per token row of d = 128 values (four per lane): dV = eta Y in place, deta = Y . V.
+// One warp per token row of DV = 64 or 128 values (DV / 32 per lane): dV = eta Y in place,
+// deta = Y . V.
+template <int DV>
 __global__ void assoc_bwd_finish_kernel(const uint16_t* __restrict__ V, const float* eta,
                                         float eta_scalar, uint16_t* dV,
                                         float* __restrict__ deta, size_t rows) {
+  constexpr int PER = DV / 32;
+  using Vec = typename std::conditional<PER == 4, uint2, uint32_t>::type;
   const int lane = threadIdx.x & 31;
   const size_t warps = (size_t)gridDim.x * (blockDim.x >> 5);
   for (size_t row = (size_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
        row += warps) {
-    const size_t o = row * 128 + 4 * lane;
-    const uint2 y = *reinterpret_cast<const uint2*>(dV + o);
-    const uint2 v = *reinterpret_cast<const uint2*>(V + o);
+    const size_t o = row * DV + PER * lane;
+    const Vec y = *reinterpret_cast<const Vec*>(dV + o);
+    const Vec v = *reinterpret_cast<const Vec*>(V + o);
     const float e = eta ? eta[row] : eta_scalar;
     const uint16_t* yh = reinterpret_cast<const uint16_t*>(&y);
     const uint16_t* vh = reinterpret_cast<const uint16_t*>(&v);
-    uint2 ov;
+    Vec ov;
     uint16_t* ovh = reinterpret_cast<uint16_t*>(&ov);
     float dot = 0.f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < PER; ++i) {
       const float yf = bf16_to_f(yh[i]);
       dot += yf * bf16_to_f(vh[i]);
       ovh[i] = f_to_bf16(e * yf);
     }
-    *reinterpret_cast<uint2*>(dV + o) = ov;
+    *reinterpret_cast<Vec*>(dV + o) = ov;
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, s);
     if (lane == 0) deta[row] = dot;
@@ -134,9 +138,10 @@ int launch_assoc_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  assoc_bwd_finish_kernel<<<sms * 8, 256, 0, ctx.stream>>>(
-      static_cast<const uint16_t*>(a.V), a.eta, a.eta_scalar, static_cast<uint16_t*>(a.dV),
-      a.deta, (size_t)BH * a.T);
+  auto finish = d == 64 ? assoc_bwd_finish_kernel<64> : assoc_bwd_finish_kernel<128>;
+  finish<<<sms * 8, 256, 0, ctx.stream>>>(static_cast<const uint16_t*>(a.V), a.eta, a.eta_scalar,
+                                          static_cast<uint16_t*>(a.dV), a.deta,
+                                          (size_t)BH * a.T);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *ctx.msg = std::string("assoc bwd finish launch: ") + cudaGetErrorString(e);

@@ -77,10 +77,13 @@ constexpr uint32_t TM_COLS = 512;
 struct AssocParams {
   const float* eta;         // [BH, T] or null
   float eta_scalar;
-  const float* S0;          // [BH, D, D] or null (zeros)
+  const float* S0;          // [BH, dim, dim] or null (zeros)
   const float* S_start;     // [BH, P-1, D, D] starting states of parts 1.. (pass 2, P > 1)
-  float* S_dst;             // pass 1: [BH, P-1, D, D] increments; pass 2: S_out [BH, D, D]
+  float* S_dst;             // pass 1: [BH, P-1, D, D] increments, or with dst_user the caller's
+                            // [BH, dim, dim] state (single part); pass 2: S_out [BH, dim, dim]
   int T, P, part_len;
+  int dim;                  // the caller's head dim: 128, or 64 zero-padded to D in the kernel
+  int dst_user;             // pass 1 writes the caller's state (one part) rather than increments
   int reverse;              // chunks last to first, transposed causal mask
   float eta_mul;            // every rate multiplied by this
   // Decay mode (one superchunk): the state follows M_t = beta M_(t-1) + eta_t k_t^T v_t and
@@ -218,17 +221,26 @@ __global__ void __launch_bounds__(THREADS, 1)
   // Starting state S (d_in x d_out, row-major) of this part, columns [64 half, 64 half + 64)
   // of S^T, into TMEM.
   auto load_state = [&](int half, uint32_t tl, int dout) {
+    // part 0 starts from the caller's [dim][dim] state (zero outside it when dim = 64), later
+    // parts from the workspace's [D][D] prefix
     const float* src = nullptr;
-    if (part == 0) src = p.S0 ? p.S0 + (size_t)stream * D * D : nullptr;
-    else src = p.S_start + ((size_t)stream * (p.P - 1) + (part - 1)) * D * D;
+    int ld = D;
+    if (part == 0) {
+      src = p.S0 ? p.S0 + (size_t)stream * p.dim * p.dim : nullptr;
+      ld = p.dim;
+      if (dout >= p.dim) src = nullptr;
+    } else {
+      src = p.S_start + ((size_t)stream * (p.P - 1) + (part - 1)) * D * D;
+    }
     const float sc = DECAY ? powf(p.beta, H_MID + 1.f) : 1.f;
 #pragma unroll 1
     for (int cc = 0; cc < 2; ++cc) {
       uint32_t v[32];
       const int din0 = 64 * half + 32 * cc;
+      const bool in = src && din0 < (part == 0 ? p.dim : D);
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        v[j] = __float_as_uint(src ? sc * src[(din0 + j) * D + dout] : 0.f);
+        v[j] = __float_as_uint(in ? sc * src[(din0 + j) * ld + dout] : 0.f);
       umma::st32x32(tmem + tl + TM_S + din0, v);
     }
     umma::wait_st();
@@ -414,8 +426,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     // ---- final state of the part: increment (pass 1) or S_out (pass 2, last part)
     if (ok && (SO || part == p.P - 1)) {
-      float* dst = SO ? p.S_dst + ((size_t)stream * (p.P - 1) + part) * D * D
-                      : p.S_dst + (size_t)stream * D * D;
+      // the caller's [dim][dim] state (pass 2, or pass 1 over one part), else a [D][D]
+      // workspace increment
+      const bool user = !SO || p.dst_user;
+      const int ld = user ? p.dim : D;
+      float* dst = user ? p.S_dst + (size_t)stream * p.dim * p.dim
+                        : p.S_dst + ((size_t)stream * (p.P - 1) + part) * D * D;
       // pass 2 in decay mode holds beta^(h+1) M and ends with beta^h times the state; pass 1
       // accumulates the weighted increment itself
       const float sc = (DECAY && !SO) ? powf(p.beta, H_MID) : 1.f;
@@ -425,8 +441,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         umma::ld32x32(tmem + tl + TM_S + 32 * cc, v);
         umma::wait_ld();
         umma::reg_fence(v);
+        if (dout < ld && 32 * cc < ld) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(32 * cc + j) * D + dout] = sc * __uint_as_float(v[j]);
+          for (int j = 0; j < 32; ++j) dst[(32 * cc + j) * ld + dout] = sc * __uint_as_float(v[j]);
+        }
       }
     }
   } else if (warp < 14) {
@@ -465,16 +483,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         // decay mode: the words this lane rewrites, read back before the waits below (all
         // loads in flight at once; each word is read once, before this kernel stores that row)
         uint32_t oadd[DECAY ? 32 : 1];
-        if (DECAY && p.Oadd) {
+        if (DECAY && p.Oadd && dout < p.dim) {
           const uint32_t* ob = reinterpret_cast<const uint32_t*>(
-              p.Oadd + ((size_t)stream * p.T + tok(c)) * D + (dout & ~1));
+              p.Oadd + ((size_t)stream * p.T + tok(c)) * p.dim + (dout & ~1));
 #pragma unroll
           for (int t = 0; t < C; ++t) {
             if (t & 4) continue;
             // volatile asm keeps the load here, ahead of the waits, instead of at its use
             asm volatile("ld.global.u32 %0, [%1];"
                          : "=r"(oadd[(t >> 3) * 4 + (t & 3)])
-                         : "l"(ob + (size_t)(odd ? t + 4 : t) * (D / 2)));
+                         : "l"(ob + (size_t)(odd ? t + 4 : t) * (p.dim / 2)));
           }
         }
         // second half of the bf16 state copy for chunk c+1; the go(c+1) arrival also says
@@ -535,7 +553,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (otid == 0) {
           const uint32_t sO = sbase + L::O_OFF + 16384 * b;
           tma_store_3d(&tmO, sO, 0, tok(c), stream);
-          tma_store_3d(&tmO, sO + 8192, 64, tok(c), stream);
+          if (p.dim > 64) tma_store_3d(&tmO, sO + 8192, 64, tok(c), stream);
           bulk_commit();
           bulk_wait_read<1>();  // the other staging buffer is free again
         }
@@ -573,11 +591,14 @@ done:
 
 // Exclusive prefix over the parts' increments, in place: slot p-1 becomes the start of part p.
 // (decay mode: each step first multiplies the running state by decay_L = beta^L.)
-__global__ void assoc_scan_kernel(const float* __restrict__ S0, float* inc, int P, float decay_L) {
+// S0 is the caller's [dim][dim] state (zero outside it in the [D][D] increments when dim = 64).
+__global__ void assoc_scan_kernel(const float* __restrict__ S0, float* inc, int P, float decay_L,
+                                  int dim) {
   const int stream = blockIdx.y;
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;   // element of the d x d state
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;   // element of the D x D state
   if (e >= D * D) return;
-  float run = S0 ? S0[(size_t)stream * D * D + e] : 0.f;
+  const int r = e / D, col = e % D;
+  float run = (S0 && r < dim && col < dim) ? S0[(size_t)stream * dim * dim + r * dim + col] : 0.f;
   float* base = inc + (size_t)stream * (P - 1) * D * D + e;
   for (int pp = 0; pp < P - 1; ++pp) {
     run = decay_L * run + base[(size_t)pp * D * D];
@@ -630,14 +651,17 @@ int launch_chunk(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap
 
 }  // namespace
 
-bool assoc_supported(int d, int C_, int dt) { return dt == 1 && d == D && C_ == C; }
+bool assoc_supported(int d, int C_, int T, int dt) {
+  return dt == 1 && (d == D || d == 64) && (C_ == 16 || C_ == 32 || C_ == C) && T % C == 0;
+}
 
 int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
   // Pass 1 over the whole sequence as a single superchunk: S_out = sum_t eta_t k_t^T v_t.
   const int BH = a.B * a.H;
   CUtensorMap tq, tk, tv, to;
-  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.T, (uint64_t)BH};
-  const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)a.T * D * 2};
+  // d = 64: the tiles' second 64-wide half lies past the tensor and is filled with zeros
+  const uint64_t dims[3] = {(uint64_t)a.d, (uint64_t)a.T, (uint64_t)BH};
+  const uint64_t strides[2] = {(uint64_t)a.d * 2, (uint64_t)a.T * a.d * 2};
   const uint32_t box[3] = {64, (uint32_t)C, 1};
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -652,6 +676,8 @@ int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
   p.S0 = nullptr;
   p.S_start = nullptr;
   p.S_dst = a.S_out;
+  p.dst_user = 1;
+  p.dim = a.d;
   p.T = a.T;
   p.P = 2;             // parts 0 .. P-2 = the single part [0, T)
   p.part_len = a.T;
@@ -668,7 +694,7 @@ int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
 }
 
 size_t assoc_workspace_bytes(int B, int H, int T, int d, int C_) {
-  if (d != D || C_ != C || T % C != 0) return 0;
+  if (!assoc_supported(d, C_, T, 1)) return 0;
   const int P = choose_parts(B * H, T);
   return (size_t)B * H * (P - 1) * D * D * sizeof(float);
 }
@@ -682,8 +708,10 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
     return kWorkspace;
   }
   CUtensorMap tq, tk, tv, to;
-  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)a.T, (uint64_t)BH};
-  const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)a.T * D * 2};
+  // d = 64: the tiles' second 64-wide half lies past the tensor and is filled with zeros, and
+  // only the first half of each output tile is stored
+  const uint64_t dims[3] = {(uint64_t)a.d, (uint64_t)a.T, (uint64_t)BH};
+  const uint64_t strides[2] = {(uint64_t)a.d * 2, (uint64_t)a.T * a.d * 2};
   const uint32_t box[3] = {64, (uint32_t)C, 1};
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -697,6 +725,8 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   p.eta_scalar = a.eta_scalar;
   p.S0 = a.S0;
   p.S_start = static_cast<const float*>(a.ws);
+  p.dim = a.d;
+  p.dst_user = 0;
   p.T = a.T;
   p.P = P;
   p.part_len = a.T / P;
@@ -714,7 +744,8 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
     int st = launch_chunk<true>(tq, tk, tv, to, p, BH * (P - 1), ctx);
     if (st != kOk) return st;
     const float decay_L = a.decay ? powf(a.beta, (float)p.part_len) : 1.f;
-    assoc_scan_kernel<<<dim3(D * D / 256, BH), 256, 0, ctx.stream>>>(a.S0, p.S_dst, P, decay_L);
+    assoc_scan_kernel<<<dim3(D * D / 256, BH), 256, 0, ctx.stream>>>(a.S0, p.S_dst, P, decay_L,
+                                                                     a.d);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
       *ctx.msg = std::string("assoc scan launch: ") + cudaGetErrorString(e);

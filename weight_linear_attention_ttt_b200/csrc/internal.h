@@ -113,7 +113,10 @@ int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx);
 
 // Associative mode.
 size_t assoc_workspace_bytes(int B, int H, int T, int d, int C);
-bool assoc_supported(int d, int C, int dt);
+// bf16, d = 64 or 128, C = 16, 32 or 64 with T % 64 == 0. The associative result does not
+// depend on C (the recurrence is per token), so every C runs on the 64-token tiles; d = 64
+// runs zero-padded to 128 inside the kernel (TMA fills the missing half, no extra traffic).
+bool assoc_supported(int d, int C, int T, int dt);
 int launch_assoc(const StateArgs& a, const LaunchCtx& ctx);
 int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx);
 size_t assoc_bwd_workspace_bytes(int B, int H, int T, int d, int C);

@@ -353,7 +353,8 @@ int ttt_dual_state_fold(const float* W0, const float* A_maps, const float* B_map
 }
 
 size_t ttt_assoc_scan_workspace_size(int B, int H, int T, int d, int C, int dt) {
-  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || !assoc_supported(d, C, dt)) return 0;
+  if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || !assoc_supported(d, C, T, dt))
+    return 0;
   return assoc_workspace_bytes(B, H, T, d, C);
 }
 
@@ -365,8 +366,9 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
               workspace_bytes};
   int st = check_state_args("ttt_assoc_scan_fwd", a, 0);
   if (st != TTT_OK) return st;
-  if (!assoc_supported(d, C, dt))
-    return fail(TTT_ERR_UNSUPPORTED, "ttt_assoc_scan_fwd: supported bf16, d == 128, C == 64");
+  if (!assoc_supported(d, C, T, dt))
+    return fail(TTT_ERR_UNSUPPORTED, "ttt_assoc_scan_fwd: supported bf16, d == 64 or 128, "
+                                     "C == 16, 32 or 64, T % 64 == 0");
   st = check_state_args("ttt_assoc_scan_fwd", a, assoc_workspace_bytes(B, H, T, d, C));
   if (st != TTT_OK) return st;
   if (overlap(workspace, workspace_bytes, O, (size_t)B * H * T * d * 2) ||
@@ -381,7 +383,7 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
 
 size_t ttt_assoc_momentum_workspace_size(int B, int H, int T, int d, int C, int dt) {
   if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0 ||
-      !assoc_supported(d, C, dt))
+      !assoc_supported(d, C, T, dt))
     return 0;
   return assoc_momentum_workspace_bytes(B, H, T, d, C);
 }
@@ -403,8 +405,9 @@ int ttt_assoc_momentum_fwd(const void* Q, const void* K, const void* V, const fl
   if (!(beta >= 0.25f && beta <= 0.9f))
     return fail(TTT_ERR_UNSUPPORTED, f + ": momentum coefficient must lie in [0.25, 0.9] (0 is "
                                          "the plain associative mode)");
-  if (!assoc_supported(d, C, dt))
-    return fail(TTT_ERR_UNSUPPORTED, f + ": supported bf16, d == 128, C == 64");
+  if (!assoc_supported(d, C, T, dt))
+    return fail(TTT_ERR_UNSUPPORTED,
+                f + ": supported bf16, d == 64 or 128, C == 16, 32 or 64, T % 64 == 0");
   st = check_state_args(fn, a, assoc_momentum_workspace_bytes(B, H, T, d, C));
   if (st != TTT_OK) return st;
   const void* extra[] = {M0, M_out};
@@ -439,7 +442,7 @@ int ttt_assoc_momentum_fwd(const void* Q, const void* K, const void* V, const fl
 
 size_t ttt_assoc_scan_bwd_workspace_size(int B, int H, int T, int d, int C, int dt) {
   if (B <= 0 || H <= 0 || T <= 0 || d <= 0 || C <= 0 || T % C != 0 ||
-      !assoc_supported(d, C, dt))
+      !assoc_supported(d, C, T, dt))
     return 0;
   return assoc_bwd_workspace_bytes(B, H, T, d, C);
 }
@@ -461,8 +464,9 @@ int ttt_assoc_scan_bwd(const void* Q, const void* K, const void* V, const float*
   for (const void* p : ptrs)
     if (p && !aligned16(p))
       return fail(TTT_ERR_INVALID_ARG, f + ": every device pointer must be 16-byte aligned");
-  if (!assoc_supported(d, C, dt))
-    return fail(TTT_ERR_UNSUPPORTED, f + ": supported bf16, d == 128, C == 64");
+  if (!assoc_supported(d, C, T, dt))
+    return fail(TTT_ERR_UNSUPPORTED,
+                f + ": supported bf16, d == 64 or 128, C == 16, 32 or 64, T % 64 == 0");
   const size_t need = assoc_bwd_workspace_bytes(B, H, T, d, C);
   if (!workspace || workspace_bytes < need)
     return fail(TTT_ERR_WORKSPACE, f + ": workspace smaller than ttt_assoc_scan_bwd_workspace_size()");
@@ -607,8 +611,9 @@ int ttt_assoc_state_fwd(const void* K, const void* V, const float* eta, float et
   for (const void* p : ptrs)
     if (p && !aligned16(p))
       return fail(TTT_ERR_INVALID_ARG, f + ": every device pointer must be 16-byte aligned");
-  if (!assoc_supported(d, C, dt))
-    return fail(TTT_ERR_UNSUPPORTED, f + ": supported bf16, d == 128, C == 64");
+  if (!assoc_supported(d, C, T, dt))
+    return fail(TTT_ERR_UNSUPPORTED,
+                f + ": supported bf16, d == 64 or 128, C == 16, 32 or 64, T % 64 == 0");
   const size_t nx = (size_t)B * H * T * d * 2, ns = (size_t)B * H * d * d * 4;
   const size_t ne = (size_t)B * H * T * 4;
   if (overlap(dS, ns, K, nx) || overlap(dS, ns, V, nx) || overlap(dS, ns, eta, ne))

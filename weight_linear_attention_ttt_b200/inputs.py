@@ -98,6 +98,10 @@ WORKLOADS = {
     "assoc_bwd_bf16_B4H16T65536_d128C64": Workload(
         "assoc_bwd_bf16_B4H16T65536_d128C64", "assoc_bwd", 1005, B=4, H=16, T=65536, d=128,
         C=64, normalise=("Q", "K"), eta="sigmoid", w0="zero"),
+    # the associative mode at head dim 64 and a 16-token chunk (evaluated on 64-token tiles)
+    "assoc_bf16_B4H16T65536_d64C16": Workload(
+        "assoc_bf16_B4H16T65536_d64C16", "assoc", 1012, B=4, H=16, T=65536, d=64, C=16,
+        normalise=("Q", "K"), eta="sigmoid", w0="zero"),
 }
 WORKLOAD_ORDER = list(WORKLOADS)
 
