@@ -78,10 +78,12 @@ struct AssocParams {
   const float* eta;         // [BH, T] or null
   float eta_scalar;
   const float* S0;          // [BH, dim, dim] or null (zeros)
-  const float* S_start;     // [BH, P-1, D, D] starting states of parts 1.. (pass 2, P > 1)
+  const float* S_start;     // [BH, nslots, D, D] prefix of the pass-1 pieces (pass 2, P > 1):
+                            // part m (m >= 1) starts from slot m * slot_mul - 1
   float* S_dst;             // pass 1: [BH, P-1, D, D] increments, or with dst_user the caller's
                             // [BH, dim, dim] state (single part); pass 2: S_out [BH, dim, dim]
   int T, P, part_len;
+  int nslots, slot_mul;     // pass 2: prefix slots per stream and pass-1 pieces per part
   int dim;                  // the caller's head dim: 128, or 64 zero-padded to D in the kernel
   int dst_user;             // pass 1 writes the caller's state (one part) rather than increments
   int reverse;              // chunks last to first, transposed causal mask
@@ -230,7 +232,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       ld = p.dim;
       if (dout >= p.dim) src = nullptr;
     } else {
-      src = p.S_start + ((size_t)stream * (p.P - 1) + (part - 1)) * D * D;
+      src = p.S_start + ((size_t)stream * p.nslots + part * p.slot_mul - 1) * D * D;
     }
     const float sc = DECAY ? powf(p.beta, H_MID + 1.f) : 1.f;
 #pragma unroll 1
@@ -676,6 +678,8 @@ int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
   p.S0 = nullptr;
   p.S_start = nullptr;
   p.S_dst = a.S_out;
+  p.nslots = 1;
+  p.slot_mul = 1;
   p.dst_user = 1;
   p.dim = a.d;
   p.T = a.T;
@@ -693,16 +697,31 @@ int launch_assoc_state(const StateArgs& a, const LaunchCtx& ctx) {
   return launch_chunk<true>(tq, tk, tv, to, p, BH, ctx);
 }
 
+// Pass-1 pieces per superchunk: pass 1 covers the first P - 1 superchunks, each cut into F
+// pieces so that about every SM takes a piece (F <= 4, pieces of whole chunks).
+int choose_pieces(int streams, int T, int P) {
+  if (P <= 1) return 1;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int F = std::max(1, std::min(4, sms / (streams * (P - 1))));
+  while (F > 1 && (T / P) % (F * C) != 0) --F;
+  return F;
+}
+
 size_t assoc_workspace_bytes(int B, int H, int T, int d, int C_) {
   if (!assoc_supported(d, C_, T, 1)) return 0;
   const int P = choose_parts(B * H, T);
-  return (size_t)B * H * (P - 1) * D * D * sizeof(float);
+  const int F = choose_pieces(B * H, T, P);
+  return (size_t)B * H * (P - 1) * F * D * D * sizeof(float);
 }
 
 int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   const int BH = a.B * a.H;
   const int P = choose_parts(BH, a.T);
-  const size_t need = (size_t)BH * (P - 1) * D * D * sizeof(float);
+  const int F = choose_pieces(BH, a.T, P);
+  const int pieces = (P - 1) * F;   // pass-1 increments per stream
+  const size_t need = (size_t)BH * pieces * D * D * sizeof(float);
   if (a.ws_bytes < need) {
     *ctx.msg = "ttt_assoc_scan_fwd: workspace smaller than ttt_assoc_scan_workspace_size()";
     return kWorkspace;
@@ -739,13 +758,20 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   p.orow = a.orow;
   p.oscale = a.oscale;
   p.err = ctx.err;
+  p.nslots = pieces;
+  p.slot_mul = F;
   if (P > 1) {
-    p.S_dst = static_cast<float*>(a.ws);
-    int st = launch_chunk<true>(tq, tk, tv, to, p, BH * (P - 1), ctx);
+    // pass 1: the increments of the first P - 1 superchunks, F pieces each (a part of
+    // T / (P F) tokens per CTA); the scan turns them into the starting state of every piece
+    AssocParams p1 = p;
+    p1.S_dst = static_cast<float*>(a.ws);
+    p1.P = pieces + 1;
+    p1.part_len = a.T / P / F;
+    int st = launch_chunk<true>(tq, tk, tv, to, p1, BH * pieces, ctx);
     if (st != kOk) return st;
-    const float decay_L = a.decay ? powf(a.beta, (float)p.part_len) : 1.f;
-    assoc_scan_kernel<<<dim3(D * D / 256, BH), 256, 0, ctx.stream>>>(a.S0, p.S_dst, P, decay_L,
-                                                                     a.d);
+    const float decay_L = a.decay ? powf(a.beta, (float)p1.part_len) : 1.f;
+    assoc_scan_kernel<<<dim3(D * D / 256, BH), 256, 0, ctx.stream>>>(a.S0, p1.S_dst, pieces + 1,
+                                                                     decay_L, a.d);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
       *ctx.msg = std::string("assoc scan launch: ") + cudaGetErrorString(e);
