@@ -550,6 +550,8 @@ def run_ours(args, w, rank, world, local_rank):
     kname, ksrc = DOMINANT_KERNEL[w.kind]
     if w.kind == "dual" and ttt.get_tuning("dual_kernel") == 5:   # the TMEM-state kernel
         kname, ksrc = "dual_gram_kernel", "dual_gram.cu"
+    if w.kind == "dual" and ttt.get_tuning("dual_kernel") == 6:   # the register-state Gram kernel
+        kname, ksrc = "dual_rgram_kernel", "dual_rgram.cu"
     launches_per_step = launches / args.steps
     # the roofline is the slower of the flops at the tensor peak and the bytes at HBM bandwidth
     t_flops = algo["flops"] / (pk["bf16_tflops"] * 1e12)

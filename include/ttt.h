@@ -95,7 +95,9 @@ uint64_t ttt_launch_count(void);
  *                        more SM per one or two streams; measured slower than 3),
  *                        5 = the state resident in TMEM, updated once per 128-token stage on
  *                        tcgen05, with the chain reduced to 16 x 16 key-Gram-block updates
- *                        (d = 64, C = 16, 32 or 64).
+ *                        (d = 64, C = 16, 32 or 64), 6 = the same substitution with the state
+ *                        in registers and its products on warp MMAs, the data-only products
+ *                        on tcgen05 (d = 64, C = 16, 32 or 64).
  *   "dual_cluster_streams"  dual_kernel 4: streams per cluster, 1 or 2 (each cluster adds one
  *                        output CTA).
  *   "dual_warp_cols"     d = 64 with C = 16: 8 or 16 output columns per warp, for dual_kernel

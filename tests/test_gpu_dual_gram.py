@@ -1,7 +1,9 @@
-"""GPU parity of the dual form's TMEM-state kernel (the state updated once per 128-token stage on
-tcgen05, the chain reduced to 16 x 16 key-Gram-block updates) against the fp64 oracle, through
-the C ABI. Tolerance: max over (b,h) slices of the relative L2 error of O and of the final W,
-1e-2 for bf16 inputs (the same bar as every bf16 dual-form kernel)."""
+"""GPU parity of the dual form's Gram-block kernels against the fp64 oracle, through the C ABI:
+dual_kernel 5 (the state in TMEM, updated once per 128-token stage on tcgen05) and dual_kernel 6
+(the state in registers, the stage's substitution and update on warp MMAs). Both reduce the
+serial chain to 16 x 16 key-Gram-block updates. Tolerance: max over (b,h) slices of the relative
+L2 error of O and of the final W, 1e-2 for bf16 inputs (the same bar as every bf16 dual-form
+kernel)."""
 import torch
 import pytest
 
@@ -11,14 +13,15 @@ from weight_linear_attention_ttt_b200 import inputs as inp
 from test_gpu_dual import TOL, check, run, workload
 
 pytestmark = pytest.mark.gpu
-GRAM = 5
+GRAM_KERNELS = [5, 6]
 
 
+@pytest.mark.parametrize("kernel", GRAM_KERNELS)
 @pytest.mark.parametrize("C,T", [(16, 16), (16, 144), (16, 400), (32, 32), (32, 96), (32, 416),
                                  (64, 64), (64, 192), (64, 576)])
-def test_gram_kernel_full_and_partial_stages(cuda_lib, tuning, C, T):
+def test_gram_kernel_full_and_partial_stages(cuda_lib, tuning, kernel, C, T):
     """Per-token rates, a given W0, one to four 128-token stages with a ragged last stage."""
-    tuning("dual_kernel", GRAM)
+    tuning("dual_kernel", kernel)
     x = inp.dual_or_assoc_inputs(2, 3, T, 64, seed=C * 1000 + T, device="cuda",
                                  normalise=("K", "V"))
     n0 = ttt.launch_count()
@@ -28,17 +31,19 @@ def test_gram_kernel_full_and_partial_stages(cuda_lib, tuning, C, T):
     assert ttt.read_device_error() == 0
 
 
-def test_gram_kernel_scalar_rate_and_zero_state(cuda_lib, tuning):
-    tuning("dual_kernel", GRAM)
+@pytest.mark.parametrize("kernel", GRAM_KERNELS)
+def test_gram_kernel_scalar_rate_and_zero_state(cuda_lib, tuning, kernel):
+    tuning("dual_kernel", kernel)
     x = inp.dual_or_assoc_inputs(1, 4, 528, 64, seed=5, device="cuda", normalise=("K", "V"))
     x = dict(x, eta=None, eta_scalar=0.02, W0=None)
     O, W = run(x, 16)
     check(x, 16, O, W, TOL["bf16"])
 
 
-def test_gram_kernel_degenerate_cases(cuda_lib, tuning):
-    tuning("dual_kernel", GRAM)
-    # eta = 0: no update (the fp32 state passes through TMEM unchanged); O = Q W0
+@pytest.mark.parametrize("kernel", GRAM_KERNELS)
+def test_gram_kernel_degenerate_cases(cuda_lib, tuning, kernel):
+    tuning("dual_kernel", kernel)
+    # eta = 0: no update (the fp32 state passes through unchanged); O = Q W0
     x = inp.dual_or_assoc_inputs(1, 2, 256, 64, seed=9, device="cuda", normalise=("K", "V"),
                                  eta="const", eta_const=0.0)
     O, W = run(x, 16)
@@ -52,14 +57,15 @@ def test_gram_kernel_degenerate_cases(cuda_lib, tuning):
     check(x, 16, O, W, TOL["bf16"])
 
 
-def test_gram_kernel_agrees_with_stage_kernel(cuda_lib, tuning):
+@pytest.mark.parametrize("kernel", GRAM_KERNELS)
+def test_gram_kernel_agrees_with_stage_kernel(cuda_lib, tuning, kernel):
     """Both kernels compute the same chunk recurrence with bf16 operands rounded at different
     points (per chunk state against per stage state plus Gram corrections): they agree well
     inside the oracle tolerance."""
     x = inp.dual_or_assoc_inputs(2, 4, 1024, 64, seed=31, device="cuda", normalise=("K", "V"))
     tuning("dual_kernel", 3)
     Ot, Wt = run(x, 16)
-    tuning("dual_kernel", GRAM)
+    tuning("dual_kernel", kernel)
     Og, Wg = run(x, 16)
     assert max_rel_l2(Og, Ot, 2) < 5e-3 and max_rel_l2(Wg, Wt, 2) < 5e-3
     # deterministic: a second call gives the same bits
@@ -67,8 +73,9 @@ def test_gram_kernel_agrees_with_stage_kernel(cuda_lib, tuning):
     assert torch.equal(Og, Og2) and torch.equal(Wg, Wg2)
 
 
-def test_gram_kernel_125m_layer_workload(cuda_lib, tuning):
-    tuning("dual_kernel", GRAM)
+@pytest.mark.parametrize("kernel", GRAM_KERNELS)
+def test_gram_kernel_125m_layer_workload(cuda_lib, tuning, kernel):
+    tuning("dual_kernel", kernel)
     w, x = workload("dual_bf16_B8H12T2048_d64C16")
     O, W = run(x, w.C)
     eo, ew = check(x, w.C, O, W, TOL["bf16"])
@@ -76,9 +83,10 @@ def test_gram_kernel_125m_layer_workload(cuda_lib, tuning):
     assert ttt.read_device_error() == 0
 
 
-def test_gram_kernel_long_context_workload(cuda_lib, tuning):
+@pytest.mark.parametrize("kernel", GRAM_KERNELS)
+def test_gram_kernel_long_context_workload(cuda_lib, tuning, kernel):
     """Every stream of the 1.3B-layer long-context shape, one batch item per oracle call."""
-    tuning("dual_kernel", GRAM)
+    tuning("dual_kernel", kernel)
     w, x = workload("dual_bf16_B2H32T32768_d64C16")
     O, W = run(x, w.C)
     worst = (0.0, 0.0)

@@ -621,6 +621,8 @@ int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
   }
   if (kernel == kDualKernelGram && dual_gram_supported(a.d, a.C, a.dt))
     return launch_dual_gram(a, ctx);
+  if (kernel == kDualKernelRegGram && dual_gram_supported(a.d, a.C, a.dt))
+    return launch_dual_rgram(a, ctx);
   // (C = 32 and 64 exist only in that form)
   if (a.d == 64 && (a.C != 16 || kernel == kDualKernelAuto || kernel == kDualKernelTensor)) {
     const int split = (forced_split == 1 || forced_split == 2 || forced_split == 4)

@@ -76,7 +76,8 @@ enum TuneKey : int {
   kTuneCount
 };
 enum DualKernel : int { kDualKernelAuto = 0, kDualKernelWarp = 1, kDualKernelPair = 2,
-                        kDualKernelTensor = 3, kDualKernelSplit = 4, kDualKernelGram = 5 };
+                        kDualKernelTensor = 3, kDualKernelSplit = 4, kDualKernelGram = 5,
+                        kDualKernelRegGram = 6 };
 int tuning(TuneKey key);
 // Records the detail returned by ttt_last_error_message() on this thread.
 void set_last_error(const std::string& msg);
@@ -109,6 +110,9 @@ int dual_tc_split(int streams, int sms);
 // tcgen05; the chain is a blocked substitution over the stage's key Gram blocks (dual_gram.cu).
 bool dual_gram_supported(int d, int C, int dt);
 int launch_dual_gram(const StateArgs& a, const LaunchCtx& ctx);
+// The same shapes: the state in registers and the stage's Gram-block substitution on warp MMAs,
+// the data-only products on tcgen05 (dual_rgram.cu).
+int launch_dual_rgram(const StateArgs& a, const LaunchCtx& ctx);
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx);
 
 // Associative mode.
