@@ -177,7 +177,10 @@ def test_momentum_validation(lib):
                                           ctypes.c_float(beta), None, None, v(6 * A), v(7 * A),
                                           v(M_out), 1, 1, 128, d, 64, 1, v(10 * A), 1 << 30, None)
 
-    assert mom(0.95) == 2 and mom(0.1) == 2 and mom(1.0) == 2   # outside [0.25, 0.9]
+    assert mom(-0.1) == 2 and mom(1.5) == 2 and mom(float("nan")) == 2   # outside [0, 1]
+    assert lib.ttt_set_tuning(b"momentum_form", 1) == 0                 # the two-pass form
+    assert mom(0.95) == 2 and mom(0.1) == 2 and mom(1.0) == 2          # outside [0.25, 0.9]
+    lib.ttt_reset_tuning()
     assert mom(0.5, M_out=0) == 1
     assert mom(0.5, d=96) == 2
     assert mom(0.5, M_out=6 * A + 64) == 1                      # M_out overlaps O

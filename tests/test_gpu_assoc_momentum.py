@@ -1,7 +1,9 @@
 """GPU parity of ttt_assoc_momentum_fwd (associative mode with a momentum inner loop) against
-the fp64 oracle's token-by-token momentum recurrence, through the C ABI. The oracle is pinned on
-the CPU (tests/test_oracle_pins.py: beta = 0, closed weighted-sum form, hand-worked tokens).
-Tolerance: per-(b,h) relative L2 <= 1e-2 for O, S_out and M_out (bf16 inputs and outputs)."""
+the fp64 oracle's token-by-token momentum recurrence, through the C ABI: the one-pass form that
+carries both states (the default; every beta in [0, 1]) and the two-pass plain + decayed form
+(momentum_form 1; beta in [0.25, 0.9]). The oracle is pinned on the CPU (tests/test_oracle_pins.py:
+beta = 0, closed weighted-sum forms including beta = 1, hand-worked tokens). Tolerance: per-(b,h)
+relative L2 <= 1e-2 for O, S_out and M_out (bf16 inputs and outputs)."""
 import os
 
 import pytest
@@ -45,22 +47,50 @@ def check(x, beta, got, streams=None):
     return errs
 
 
-@pytest.mark.parametrize("beta", [0.25, 0.5, 0.75, 0.9])
+BETAS = [0.0, 0.25, 0.5, 0.9, 0.99, 0.999, 1.0]
+
+
+@pytest.mark.parametrize("beta", BETAS)
 @pytest.mark.parametrize("B,H,T", [(1, 1, 64), (1, 2, 512), (2, 3, 640)])
 def test_momentum_matches_oracle(cuda_lib, B, H, T, beta):
-    x = make(B, H, T, seed=T + 7 * H + int(100 * beta))
+    x = make(B, H, T, seed=T + 7 * H + int(1000 * beta))
     check(x, beta, run(x, beta))
     assert ttt.read_device_error() == 0
 
 
+@pytest.mark.parametrize("beta", [0.25, 0.5, 0.75, 0.9])
+def test_two_pass_form_matches_oracle(cuda_lib, tuning, beta):
+    """The plain + decayed evaluation, kept as a comparison variant, within its beta range."""
+    tuning("momentum_form", 1)
+    x = make(2, 3, 640, seed=11 + int(100 * beta))
+    check(x, beta, run(x, beta))
+    assert ttt.read_device_error() == 0
+
+
+@pytest.mark.parametrize("beta", [0.9, 0.999])
 @pytest.mark.parametrize("parts", ["1", "2", "4", "16"])
-def test_forced_superchunk_counts(cuda_lib, tuning, parts):
-    """Both passes split into superchunks (the decayed one carrying its state across them with
-    the superchunk decay) give the oracle's results for every split."""
+def test_forced_superchunk_counts(cuda_lib, tuning, parts, beta):
+    """Split into superchunks (pass 1 maps the pieces, the scan composes them, pass 2 starts
+    every part from its composed state), every split gives the oracle's results."""
     tuning("assoc_parts", int(parts))
     x = make(1, 2, 1024, seed=31)
-    check(x, 0.9, run(x, 0.9))
+    check(x, beta, run(x, beta))
     assert ttt.read_device_error() == 0
+
+
+def test_forms_agree(cuda_lib, tuning):
+    """Both forms evaluate the same recurrence: well inside the oracle tolerance of each other."""
+    x = make(2, 2, 1024, seed=77)
+    got = run(x, 0.8)
+    tuning("momentum_form", 1)
+    ref = run(x, 0.8)
+    for g, r in zip(got, ref):
+        assert max_rel_l2(g, r, 2) < 5e-3
+    # deterministic: the default form gives the same bits again
+    tuning("momentum_form", 0)
+    again = run(x, 0.8)
+    for g, r in zip(got, again):
+        assert torch.equal(g, r)
 
 
 def test_scalar_eta_zero_states_and_state_aliasing(cuda_lib):
@@ -93,22 +123,30 @@ def test_state_carry_across_calls(cuda_lib):
 
 
 def test_full_associative_workload_sampled_streams(cuda_lib):
-    w = inp.WORKLOADS["assoc_bf16_B4H16T65536_d128C64"]
+    w = inp.WORKLOADS["assoc_momentum_bf16_B4H16T65536_d128C64"]
     x = inp.make_inputs(w, "cuda")
     x["S0"], x["M0"] = None, None
-    got = run(x, 0.9)
-    errs = check(x, 0.9, got, streams=[(0, 0), (3, 15)])
-    print("associative momentum (beta 0.9, 2 sampled streams): max rel L2 O %.2e S %.2e "
+    got = run(x, 0.99)
+    streams = [(0, 0), (1, 7), (2, 9), (3, 15)]
+    errs = check(x, 0.99, got, streams=streams)
+    print("associative momentum (beta 0.99, 4 sampled streams): max rel L2 O %.2e S %.2e "
           "M %.2e" % tuple(errs))
+    assert all(torch.isfinite(t).all() for t in got)
     assert ttt.read_device_error() == 0
 
 
-def test_errors(cuda_lib):
+def test_errors(cuda_lib, tuning):
     x = make(1, 1, 128, seed=1)
+    for beta in (-0.1, 1.5, float("nan")):
+        with pytest.raises(ttt.TTTError) as e:
+            run(x, beta)
+        assert e.value.status == 2
+    tuning("momentum_form", 1)
     for beta in (0.0, 0.1, 0.95, 1.0):
         with pytest.raises(ttt.TTTError) as e:
             run(x, beta)
         assert e.value.status == 2
+    tuning("momentum_form", 0)
     with pytest.raises(ttt.TTTError) as e:
         run(x, 0.5, workspace=torch.empty(16, device="cuda", dtype=torch.uint8))
     assert e.value.status == 3

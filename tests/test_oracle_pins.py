@@ -668,6 +668,24 @@ def test_momentum_closed_weighted_sum(beta):
     assert np.allclose(M, Mt, rtol=1e-10, atol=1e-12)
 
 
+def test_momentum_beta_one_closed_form():
+    """beta = 1: the momentum is the running sum of the updates and the state its running sum,
+    so token s's update enters S_t with weight t - s + 1 and M0 with weight t (t counted from 1)."""
+    T, d = 13, 3
+    Q, K, V = _rand(T, d), _rand(T, d), _rand(T, d)
+    eta = rng.uniform(0.1, 0.6, T)
+    S0, M0 = _rand(d, d), _rand(d, d)
+    O, S, M = orc.assoc_momentum_stream(Q, K, V, eta, 1.0, S0, M0)
+    for t in range(T):
+        St = S0 + (t + 1) * M0
+        for s_ in range(t + 1):
+            St = St + (t - s_ + 1) * eta[s_] * np.outer(K[s_], V[s_])
+        assert np.allclose(O[t], Q[t] @ St, rtol=1e-10, atol=1e-12)
+    assert np.allclose(M, M0 + sum(eta[s_] * np.outer(K[s_], V[s_]) for s_ in range(T)),
+                       rtol=1e-10, atol=1e-12)
+    assert np.allclose(S, St, rtol=1e-10, atol=1e-12)
+
+
 def test_momentum_two_tokens_by_hand():
     """d = 1: q = (1, 2), k = (1, 1), v = (3, 5), eta = (0.5, 1), beta = 0.5, S0 = M0 = 0.
     M1 = 1.5, S1 = 1.5, o1 = 1.5; M2 = 0.75 + 5 = 5.75, S2 = 7.25, o2 = 14.5."""

@@ -1,6 +1,8 @@
-// Associative mode with a momentum inner loop.
+// Associative mode with a momentum inner loop: the dispatch between the one-pass form
+// (assoc_mom.cu, the default) and the two-pass form below (tuning key "momentum_form" = 1, kept
+// for comparison; beta in [0.25, 0.9]).
 //
-// Source: "KV 바인딩 기반 테스트 시간 학습은 사실상 선형 어텐션이다", momentum paragraph: with
+// Two-pass form. Source: "KV 바인딩 기반 테스트 시간 학습은 사실상 선형 어텐션이다", momentum paragraph: with
 // momentum SGD the inner loop is still a weighted sum of linear-attention terms. Per stream,
 //     M_t = beta M_(t-1) + eta_t k_t^T v_t,   S_t = S_(t-1) + M_t,   o_t = q_t S_t.
 // Summing the momentum terms, with A_t = sum_{s<=t} eta_s k_s^T v_s (the plain associative
@@ -13,6 +15,7 @@
 // elementwise.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <string>
 
 #include "internal.h"
@@ -32,12 +35,23 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
-size_t assoc_momentum_workspace_bytes(int B, int H, int T, int d, int C) {
+size_t assoc_momentum_split_workspace_bytes(int B, int H, int T, int d, int C) {
   const size_t BH = (size_t)B * H;
   return align256(assoc_workspace_bytes(B, H, T, d, C)) + BH * d * d * sizeof(float);
 }
 
+// Enough for either form, so that a size queried before a form is chosen stays valid.
+size_t assoc_momentum_workspace_bytes(int B, int H, int T, int d, int C) {
+  return std::max(assoc_momentum_split_workspace_bytes(B, H, T, d, C),
+                  assoc_momentum_fused_workspace_bytes(B, H, T, d, C));
+}
+
 int launch_assoc_momentum(const AssocMomentumArgs& a, const LaunchCtx& ctx) {
+  return tuning(kTuneMomentumForm) == 1 ? launch_assoc_momentum_split(a, ctx)
+                                         : launch_assoc_momentum_fused(a, ctx);
+}
+
+int launch_assoc_momentum_split(const AssocMomentumArgs& a, const LaunchCtx& ctx) {
   const size_t BH = (size_t)a.B * a.H, d = a.d;
   const size_t fwd = align256(assoc_workspace_bytes(a.B, a.H, a.T, a.d, a.C));
   if (a.ws_bytes < fwd + BH * d * d * sizeof(float)) {

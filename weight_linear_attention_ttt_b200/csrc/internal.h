@@ -73,6 +73,7 @@ enum TuneKey : int {
   kTuneWaitLimitNs,           // limit of the d = 64 dual-form pipeline waits, ns (0: 4 s)
   kTuneInplaceChunksPerLaunch,  // In-Place: 1 = one chunk per launch, 0 / 2 = chunk pairs
   kTuneDualClusterStreams,    // dual form split across SMs: streams per cluster, 1 or 2
+  kTuneMomentumForm,          // momentum: 0 = one pass carrying (S, M), 1 = plain + decayed
   kTuneCount
 };
 enum DualKernel : int { kDualKernelAuto = 0, kDualKernelWarp = 1, kDualKernelPair = 2,
@@ -179,6 +180,12 @@ struct AssocMomentumArgs {
   size_t ws_bytes;
 };
 int launch_assoc_momentum(const AssocMomentumArgs& a, const LaunchCtx& ctx);
+// The one-pass form (both states carried through the chunks; every beta in [0, 1]).
+size_t assoc_momentum_fused_workspace_bytes(int B, int H, int T, int d, int C);
+int launch_assoc_momentum_fused(const AssocMomentumArgs& a, const LaunchCtx& ctx);
+// The two-pass form (plain + decayed associative passes; beta in [0.25, 0.9]).
+size_t assoc_momentum_split_workspace_bytes(int B, int H, int T, int d, int C);
+int launch_assoc_momentum_split(const AssocMomentumArgs& a, const LaunchCtx& ctx);
 // Out[M, N] = A[M, K] B[K, N], bf16, on the In-Place kernel's read tiles (M % 128 == 0,
 // K % 64 == 0, N % 64 == 0); `counter` is one int of device memory.
 int launch_projection(const void* A, const void* B, void* Out, int M, int K, int N, int* counter,

@@ -35,7 +35,8 @@ static const TuneName kTuneNames[] = {{"dual_column_split", kTuneDualColumnSplit
                                       {"wait_limit_ns", kTuneWaitLimitNs},
                                       {"inplace_chunks_per_launch",
                                        kTuneInplaceChunksPerLaunch},
-                                      {"dual_cluster_streams", kTuneDualClusterStreams}};
+                                      {"dual_cluster_streams", kTuneDualClusterStreams},
+                                      {"momentum_form", kTuneMomentumForm}};
 static int tune_key(const char* name) {
   if (!name) return -1;
   for (const auto& t : kTuneNames)
@@ -400,11 +401,17 @@ int ttt_assoc_momentum_fwd(const void* Q, const void* K, const void* V, const fl
   int st = check_state_args(fn, a, 0);
   if (st != TTT_OK) return st;
   if (!M_out) return fail(TTT_ERR_INVALID_ARG, f + ": M_out must be non-null");
-  // The two-pass form subtracts two bf16 outputs of size ~1/(1 - beta) times the result
-  // early in a sequence; up to beta = 0.9 that stays within the bf16 accuracy bar.
-  if (!(beta >= 0.25f && beta <= 0.9f))
-    return fail(TTT_ERR_UNSUPPORTED, f + ": momentum coefficient must lie in [0.25, 0.9] (0 is "
-                                         "the plain associative mode)");
+  // The one-pass form weights every term by a sum of non-negative powers of beta: any beta in
+  // [0, 1]. The two-pass form (a comparison variant) subtracts two bf16 outputs of size
+  // ~1/(1 - beta) times the result early in a sequence; up to beta = 0.9 that stays within the
+  // bf16 accuracy bar.
+  if (tuning(kTuneMomentumForm) == 1) {
+    if (!(beta >= 0.25f && beta <= 0.9f))
+      return fail(TTT_ERR_UNSUPPORTED, f + ": the two-pass momentum form (momentum_form 1) needs "
+                                           "a coefficient in [0.25, 0.9]");
+  } else if (!(beta >= 0.f && beta <= 1.f)) {
+    return fail(TTT_ERR_UNSUPPORTED, f + ": momentum coefficient must lie in [0, 1]");
+  }
   if (!assoc_supported(d, C, T, dt))
     return fail(TTT_ERR_UNSUPPORTED,
                 f + ": supported bf16, d == 64 or 128, C == 16, 32 or 64, T % 64 == 0");

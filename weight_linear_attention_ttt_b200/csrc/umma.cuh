@@ -162,6 +162,23 @@ __device__ __forceinline__ void st32x32(uint32_t taddr, const uint32_t (&r)[32])
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+// 32 lanes x 8 columns of 32-bit values.
+__device__ __forceinline__ void st32x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+// 32 lanes x 16 columns of 32-bit values.
+__device__ __forceinline__ void st32x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
 // 16 lanes x 256 bits per repetition (x N repetitions along the columns), in the register order
 // of an m16n8 mma.sync accumulator: in repetition i, thread t holds lane (base + t / 4) in
 // registers 4i and 4i + 1 and lane (base + 8 + t / 4) in registers 4i + 2 and 4i + 3, columns
