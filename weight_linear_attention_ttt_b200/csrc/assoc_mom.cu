@@ -66,7 +66,12 @@ struct MomSmem {
   static constexpr int BAR_OFF = O_OFF + (SO ? 0 : TILE);
   static constexpr int TAB_OFF = BAR_OFF + 256;         // five tables of 64 floats
   static constexpr int BYTES = 1024 + TAB_OFF + 5 * 256;
-  static constexpr int THREADS = SO ? 448 : 576;
+  // warps: 0 TMA, 1 MMA, 2 .. REF0-1 operands, REF0 .. OUT0-1 refresh, OUT0 .. OUT0+3 outputs
+  static constexpr int NOP = SO ? 4 : 8;
+  static constexpr int NREF = 4;               // refresh warps: one per TMEM lane quarter
+  static constexpr int REF0 = 2 + NOP;
+  static constexpr int OUT0 = REF0 + NREF;
+  static constexpr int THREADS = 32 * (OUT0 + (SO ? 0 : 4));
   static constexpr uint32_t TM_COLS = SO ? 256 : 512;
   static_assert(STAGE % 1024 == 0 && EVB_OFF % 1024 == 0 && P_OFF % 1024 == 0 &&
                     O_OFF % 1024 == 0, "tile alignment");
@@ -139,10 +144,10 @@ __global__ void __launch_bounds__(MomSmem<SO>::THREADS, 1)
       mbar_init(empty + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(opready + 8 * b, 4);
+      mbar_init(opready + 8 * b, L::NOP);
       mbar_init(cdone + 8 * b, 1);
     }
-    mbar_init(sready, 8);
+    mbar_init(sready, L::NREF);
     mbar_init(ofree, 4);
     mbar_init(mdone, 1);
     fence_mbar_init();
@@ -256,10 +261,11 @@ __global__ void __launch_bounds__(MomSmem<SO>::THREADS, 1)
     // every MMA this warp issued completes before TMEM is released
     umma::commit_elect(mdone);
     mbar_wait_warp(mdone, 0, p.err, 1000000000ull);
-  } else if (warp < 6) {
-    // ---------------------------------------------------------------- operand warps 2..5
-    const int ow = warp - 2;                  // query rows 16 ow .. 16 ow + 15 of the scores
-    const int otid = threadIdx.x - 64;        // 0..127
+  } else if (warp < L::REF0) {
+    // ---------------------------------------------------------------- operand warps
+    constexpr int NT = 32 * L::NOP;           // operand threads
+    const int ow = warp - 2;
+    const int otid = threadIdx.x - 64;
     const int g = lane >> 2, tq = lane & 3;
     for (int c = 0; c < nch; ++c) {
       const int s = c % ST, b = c & 1;
@@ -271,28 +277,26 @@ __global__ void __launch_bounds__(MomSmem<SO>::THREADS, 1)
       {
         // EVw (in place) and EVb: the V tile is 1024 16-byte pieces (a token row, eight
         // columns); piece i is row (i & 511) / 8 of sub-tile i / 512
+        constexpr int PER = 1024 / NT;
         const uint32_t vt = stg + L::V_OFF;
         const uint32_t eb = sbase + L::EVB_OFF + b * TILE;
-        uint4 x[8];
-        float fw[4], fb[4];
+        uint4 x[PER];
+        float fw[PER], fb[PER];
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int i = otid + 128 * it;
-          const int w = i & 511;
-          x[it] = lds128(vt + (i >> 9) * 8192 + swz<128>((w >> 3) * 128 + (w & 7) * 16));
-          if (it < 4) {   // pieces it and it + 4 share a token row
-            const int row = w >> 3;
-            const float e = p.eta ? ldsf(stg + L::ETA_OFF + 4 * row) : p.eta_scalar;
-            fw[it] = e * ldsf(t_evw + 4 * row);
-            fb[it] = e * ldsf(t_evb + 4 * row);
-          }
+        for (int it = 0; it < PER; ++it) {
+          const int i = otid + NT * it;
+          const int w = i & 511, row = w >> 3;
+          x[it] = lds128(vt + (i >> 9) * 8192 + swz<128>(row * 128 + (w & 7) * 16));
+          const float e = p.eta ? ldsf(stg + L::ETA_OFF + 4 * row) : p.eta_scalar;
+          fw[it] = e * ldsf(t_evw + 4 * row);
+          fb[it] = e * ldsf(t_evb + 4 * row);
         }
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int i = otid + 128 * it;
+        for (int it = 0; it < PER; ++it) {
+          const int i = otid + NT * it;
           const int w = i & 511;
           const uint32_t off = (i >> 9) * 8192 + swz<128>((w >> 3) * 128 + (w & 7) * 16);
-          const float f1 = fw[it & 3], f2 = fb[it & 3];
+          const float f1 = fw[it], f2 = fb[it];
           const uint4 v = x[it];
           sts128(vt + off, make_uint4(pack_bf16(bf16_lo(v.x) * f1, bf16_hi(v.x) * f1),
                                       pack_bf16(bf16_lo(v.y) * f1, bf16_hi(v.y) * f1),
@@ -305,48 +309,50 @@ __global__ void __launch_bounds__(MomSmem<SO>::THREADS, 1)
         }
       }
       if (!SO) {
-        // scores of query rows 16 ow .. +15 against the keys 0 .. 16 ow + 15 that the causal
-        // weights keep, on warp MMAs from the swizzled Q and K tiles
+        // P' block of query rows 16 r .. +15 and keys 32 kh .. +31 (two 16-key blocks): the
+        // blocks with keys past the rows are zero; the others take their scores on warp MMAs
+        // from the swizzled Q and K tiles, then the causal weights
         const uint32_t sQ = stg, sK = stg + L::K_OFF;
-        const int r0 = 16 * ow;
-        const int npairs = ow + 1;            // pairs of 8-key tiles
-        float acc[8][4];
+        const int r = ow >> 1, kh = ow & 1;
+        const int r0 = 16 * r;
+        float acc[4][4];
 #pragma unroll
-        for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+        for (int n = 0; n < 4; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
         const int arow = r0 + (lane & 7) + 8 * ((lane >> 3) & 1);
         const int acol = 8 * (lane >> 4);
         const int brow = (lane & 7) + 8 * (lane >> 4);
         const int bcol = 8 * ((lane >> 3) & 1);
+        if (2 * kh <= r) {
 #pragma unroll
-        for (int ks = 0; ks < MD / 16; ++ks) {
-          const uint32_t sub = (ks >> 2) * 8192;
-          const int k0 = (ks & 3) * 16;
-          uint32_t a[4];
-          ldsm_x4(sQ + sub + swz<128>(arow * 128 + (k0 + acol) * 2), a);
+          for (int ks = 0; ks < MD / 16; ++ks) {
+            const uint32_t sub = (ks >> 2) * 8192;
+            const int k0 = (ks & 3) * 16;
+            uint32_t a[4];
+            ldsm_x4(sQ + sub + swz<128>(arow * 128 + (k0 + acol) * 2), a);
 #pragma unroll
-          for (int np = 0; np < 4; ++np) {
-            if (np < npairs) {
-              uint32_t bb[4];
-              ldsm_x4(sK + sub + swz<128>((16 * np + brow) * 128 + (k0 + bcol) * 2), bb);
-              mma16816(acc[2 * np], a[0], a[1], a[2], a[3], bb[0], bb[1]);
-              mma16816(acc[2 * np + 1], a[0], a[1], a[2], a[3], bb[2], bb[3]);
+            for (int kk = 0; kk < 2; ++kk) {
+              const int kb = 2 * kh + kk;   // 16-key block
+              if (kb <= r) {
+                uint32_t bb[4];
+                ldsm_x4(sK + sub + swz<128>((16 * kb + brow) * 128 + (k0 + bcol) * 2), bb);
+                mma16816(acc[2 * kk], a[0], a[1], a[2], a[3], bb[0], bb[1]);
+                mma16816(acc[2 * kk + 1], a[0], a[1], a[2], a[3], bb[2], bb[3]);
+              }
             }
           }
         }
         // P'[i][j] = [j <= i] w(i - j) / w(63 - j) score, bf16, K-major [t][s] tile
         const uint32_t sP = sbase + L::P_OFF + b * (MC * MC * 2);
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          const int j0 = 8 * n + 2 * tq;
+        for (int n = 0; n < 4; ++n) {
+          const int j0 = 32 * kh + 8 * n + 2 * tq;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int i = r0 + g + 8 * h;
             float v0 = 0.f, v1 = 0.f;
-            if (n < 2 * npairs) {
-              if (j0 <= i) v0 = acc[n][2 * h] * ldsf(t_w + 4 * (i - j0)) * ldsf(t_rw + 4 * j0);
-              if (j0 + 1 <= i)
-                v1 = acc[n][2 * h + 1] * ldsf(t_w + 4 * (i - j0 - 1)) * ldsf(t_rw + 4 * (j0 + 1));
-            }
+            if (j0 <= i) v0 = acc[n][2 * h] * ldsf(t_w + 4 * (i - j0)) * ldsf(t_rw + 4 * j0);
+            if (j0 + 1 <= i)
+              v1 = acc[n][2 * h + 1] * ldsf(t_w + 4 * (i - j0 - 1)) * ldsf(t_rw + 4 * (j0 + 1));
             sts32(sP + swz<128>(i * 128 + j0 * 2), pack_bf16(v0, v1));
           }
         }
@@ -355,9 +361,11 @@ __global__ void __launch_bounds__(MomSmem<SO>::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(opready + 8 * b);
     }
-  } else if (warp < 14) {
+  } else if (warp < L::OUT0) {
     // ---------------------------------------------------------------- refresh warps 6..13
-    const int q = warp & 3, h = (warp - 6) >> 2;   // TMEM lane quarter, half of the d_in columns
+    const int q = warp & 3, h = (warp - L::REF0) >> 2;   // TMEM lane quarter, d_in part
+    constexpr int CW = MD / (L::NREF / 4);              // d_in columns per refresh warp
+    constexpr int NPC = CW / 16;                        // 16-column pieces
     const int dout = 32 * q + lane;
     const uint32_t tl = (uint32_t)(32 * q) << 16;
     float c63, b64;
@@ -400,6 +408,13 @@ __global__ void __launch_bounds__(MomSmem<SO>::THREADS, 1)
         ld = lim = p.dim;
       }
     }
+    // this warp's TMEM stores are complete and ordered before the MMAs that the barrier releases
+    auto signal = [&](uint32_t mb) {
+      umma::wait_st();
+      umma::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(mb);
+    };
     bool ok = true;
     for (int c = 0; c < nch; ++c) {
       if (c > 0) {
@@ -410,38 +425,57 @@ __global__ void __launch_bounds__(MomSmem<SO>::THREADS, 1)
         }
         umma::fence_after();
       }
+      if (c == 0) {
 #pragma unroll 1
-      for (int pc = 0; pc < 4; ++pc) {
-        const int din0 = 64 * h + 16 * pc;
-        uint32_t sv[16], mv[16];
-        if (c == 0) {
+        for (int pc = 0; pc < NPC; ++pc) {
+          const int din0 = CW * h + 16 * pc;
+          uint32_t sv[16], mv[16];
           const bool in = dout < lim && din0 < lim;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             sv[j] = __float_as_uint(s_src && in ? s_src[(size_t)(din0 + j) * ld + dout] : 0.f);
             mv[j] = __float_as_uint(m_src && in ? m_src[(size_t)(din0 + j) * ld + dout] : 0.f);
           }
-        } else {
-          umma::ld32x16(tmem + tl + TM_S + din0, sv);
-          umma::ld32x16(tmem + tl + TM_M + din0, mv);
-          umma::wait_ld();
-          umma::reg_fence_n(sv);
-          umma::reg_fence_n(mv);
+          refresh_piece(din0, sv, mv);
         }
-        refresh_piece(din0, sv, mv);
+      } else {
+        // the loads of the next piece are in flight while a piece is converted and stored
+        uint32_t sa[16], ma[16], sb2[16], mb2[16];
+        umma::ld32x16(tmem + tl + TM_S + CW * h, sa);
+        umma::ld32x16(tmem + tl + TM_M + CW * h, ma);
+        umma::wait_ld();
+        umma::reg_fence_n(sa);
+        umma::reg_fence_n(ma);
+#pragma unroll 1
+        for (int pc = 0; pc < NPC; pc += 2) {
+          const int din0 = CW * h + 16 * pc;
+          umma::ld32x16(tmem + tl + TM_S + din0 + 16, sb2);
+          umma::ld32x16(tmem + tl + TM_M + din0 + 16, mb2);
+          refresh_piece(din0, sa, ma);
+          umma::wait_ld();
+          umma::reg_fence_n(sb2);
+          umma::reg_fence_n(mb2);
+          if (pc + 2 < NPC) {
+            umma::ld32x16(tmem + tl + TM_S + din0 + 32, sa);
+            umma::ld32x16(tmem + tl + TM_M + din0 + 32, ma);
+          }
+          refresh_piece(din0 + 16, sb2, mb2);
+          if (pc + 2 < NPC) {
+            umma::wait_ld();
+            umma::reg_fence_n(sa);
+            umma::reg_fence_n(ma);
+          }
+        }
       }
-      umma::wait_st();
-      umma::fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sready);
+      signal(sready);
     }
     // final states: the piece's (dS, dM) in pass 1; S_out, M_out from the last part in pass 2
     if (ok && nch > 0 && (SO || part == p.P - 1) &&
         mbar_wait_warp(cdone + 8 * ((nch - 1) & 1), ((nch - 1) >> 1) & 1, p.err)) {
       umma::fence_after();
 #pragma unroll 1
-      for (int pc = 0; pc < 2; ++pc) {
-        const int din0 = 64 * h + 32 * pc;
+      for (int pc = 0; pc < CW / 32; ++pc) {
+        const int din0 = CW * h + 32 * pc;
         uint32_t sv[32], mv[32];
         umma::ld32x32(tmem + tl + TM_S + din0, sv);
         umma::ld32x32(tmem + tl + TM_M + din0, mv);
@@ -471,7 +505,7 @@ __global__ void __launch_bounds__(MomSmem<SO>::THREADS, 1)
     const int q = warp & 3;
     const int dout = 32 * q + lane;
     const uint32_t tl = (uint32_t)(32 * q) << 16;
-    const int otid = threadIdx.x - 448;        // 0..127
+    const int otid = threadIdx.x - 32 * L::OUT0;   // 0..127
     const bool odd = lane & 1;
     // Lane pairs (2i, 2i+1) exchange one value per token pair (t, t+4) so that each lane stores
     // a 32-bit word of two adjacent output columns: the even lane row t, the odd lane row t+4.
@@ -486,21 +520,21 @@ __global__ void __launch_bounds__(MomSmem<SO>::THREADS, 1)
       if (otid == 0) bulk_wait_read<0>();
       bar_sync_named(1, 128);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t o[32], m[32];
-        umma::ld32x32(tmem + tl + TM_O + 32 * hf, o);
-        umma::ld32x32(tmem + tl + TM_OM + 32 * hf, m);
+      for (int qt = 0; qt < 4; ++qt) {   // tokens 16 qt .. 16 qt + 15
+        uint32_t o[16], m[16];
+        umma::ld32x16(tmem + tl + TM_O + 16 * qt, o);
+        umma::ld32x16(tmem + tl + TM_OM + 16 * qt, m);
         umma::wait_ld();
-        umma::reg_fence(o);
-        umma::reg_fence(m);
-        if (hf == 1) {   // both accumulators are read out: the next chunk's products may start
+        umma::reg_fence_n(o);
+        umma::reg_fence_n(m);
+        if (qt == 3) {   // both accumulators are read out: the next chunk's products may start
           umma::fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(ofree);
         }
 #pragma unroll
-        for (int t = 0; t < 32; t += 4) {
-          const uint4 cq = lds128(t_cq + 4 * (32 * hf + t));
+        for (int t = 0; t < 16; t += 4) {
+          const uint4 cq = lds128(t_cq + 4 * (16 * qt + t));
           o[t] = __float_as_uint(fmaf(__uint_as_float(cq.x), __uint_as_float(m[t]),
                                       __uint_as_float(o[t])));
           o[t + 1] = __float_as_uint(fmaf(__uint_as_float(cq.y), __uint_as_float(m[t + 1]),
@@ -511,12 +545,12 @@ __global__ void __launch_bounds__(MomSmem<SO>::THREADS, 1)
                                           __uint_as_float(o[t + 3])));
         }
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
+        for (int t = 0; t < 16; ++t) {
           if (t & 4) continue;
           const float a = __uint_as_float(o[t]), a4 = __uint_as_float(o[t + 4]);
           const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
           const float lo = odd ? y : a, hi = odd ? a4 : y;
-          const int row = 32 * hf + (odd ? t + 4 : t);
+          const int row = 16 * qt + (odd ? t + 4 : t);
           sts32(so + swz<128>(row * 128 + cb), pack_bf16(lo, hi));
         }
       }
