@@ -114,6 +114,8 @@ uint64_t ttt_launch_count(void);
  *   "inplace_chunks_per_launch"  In-Place update: 1 = one chunk per launch; 0 or 2 = two
  *                        chunks per launch where the shape allows it (D % 256 == 0, C % 256 == 0),
  *                        chunk i+1's read corrected by eta (Z_(i+1) Z_i^T) Vhat_i.
+ *   "momentum_form"      ttt_assoc_momentum_fwd: 0 = one pass carrying (S, M) (every beta in
+ *                        [0, 1]); 1 = plain + decayed associative passes (beta in [0.25, 0.9]).
  * Every variant computes the same operation within the same tolerance. ttt_set_tuning returns
  * TTT_ERR_INVALID_ARG for an unknown key or a negative value; ttt_get_tuning returns -1 for an
  * unknown key; ttt_reset_tuning restores every key to 0. Not synchronised with calls in flight
@@ -201,12 +203,15 @@ int ttt_assoc_scan_fwd(const void* Q, const void* K, const void* V, const float*
  *  (M_0 = M0, S_0 = S0; the rate scales each token's gradient before it enters the momentum).
  *  Q, K, V, O [B,H,T,d] bf16; eta [B,H,T] fp32 or NULL (eta_scalar); S0, M0 [B,H,d,d] fp32 or
  *  NULL (zeros); S_out, M_out [B,H,d,d] fp32 (S_out may equal S0, M_out may equal M0).
- *  beta in [0.25, 0.9] (beta = 0 is ttt_assoc_scan_fwd; the two-pass evaluation subtracts
- *  outputs of size ~1/(1 - beta), which bounds beta for bf16 outputs). Supported: as
- *  ttt_assoc_scan_fwd (bf16, d == 64 or 128, C == 16, 32 or 64, T % 64 == 0).
- *  Workspace: ttt_assoc_momentum_workspace_size() bytes. Runs as one plain associative pass and
- *  one decayed pass whose output stage combines the two outputs, then an elementwise
- *  combination of the states (see assoc_momentum.cu).
+ *  beta in [0, 1] (beta = 0 is ttt_assoc_scan_fwd; beta = 1 makes M the running sum of the
+ *  updates). Supported: as ttt_assoc_scan_fwd (bf16, d == 64 or 128, C == 16, 32 or 64,
+ *  T % 64 == 0). Workspace: ttt_assoc_momentum_workspace_size() bytes (enough for either form).
+ *  Runs as one pass that carries both states through 64-token chunks: inside a chunk every
+ *  token pair is weighted by w(n) = sum_{r<=n} beta^r, formed directly, so the accuracy does not
+ *  depend on beta; long sequences are cut into superchunks whose (S, M) maps are composed in
+ *  sequence order (see assoc_mom.cu). The tuning key "momentum_form" = 1 selects the two-pass
+ *  comparison form instead (a plain and a decayed associative pass combined in the output
+ *  stage; beta in [0.25, 0.9], since it subtracts outputs of size ~1/(1 - beta)).
  * ------------------------------------------------------------------------------------------ */
 size_t ttt_assoc_momentum_workspace_size(int B, int H, int T, int d, int C, int dt);
 int ttt_assoc_momentum_fwd(const void* Q, const void* K, const void* V, const float* eta,
