@@ -596,6 +596,16 @@ bool dual_mma_supported(int d, int C, int dt) {
   return (dt == 1 && C == 16 && (d == 32 || d == 64 || d == 128)) || dual_tc_supported(d, C, dt);
 }
 
+// Whether launch_dual_mma runs the d = 64 stage kernel for this shape under the current tuning
+// choices, i.e. whether it accepts O = nullptr (the state-only form).
+bool dual_state_only_supported(int d, int C, int dt) {
+  const int kernel = tuning(kTuneDualKernel);
+  if (kernel == kDualKernelSplit || kernel == kDualKernelGram || kernel == kDualKernelRegGram)
+    return false;
+  return dual_tc_supported(d, C, dt) &&
+         (C != 16 || kernel == kDualKernelAuto || kernel == kDualKernelTensor);
+}
+
 int launch_dual_mma(const StateArgs& a, const LaunchCtx& ctx) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)

@@ -385,14 +385,17 @@ int maps_and_fold(const StateArgs& v, int S, int bh, const float* W0, void* Ojun
   count_launch();
   int st = check_launch(ctx, "identity launch");
   if (st != kOk) return st;
+  // the maps need only the final states: the state-only form where it exists, else the
+  // outputs go to scratch
+  void* const maps_O = dual_state_only_supported(v.d, v.C, v.dt) ? nullptr : Ojunk;
   StateArgs pb = v;
   pb.S0 = nullptr;
-  pb.O = Ojunk;
+  pb.O = maps_O;
   pb.S_out = Bm;
   if ((st = run_dual(pb, ctx)) != kOk) return st;
   StateArgs pa = v;
   pa.S0 = Wid;
-  pa.O = Ojunk;
+  pa.O = maps_O;
   pa.S_out = ABm;
   if ((st = run_dual(pa, ctx)) != kOk) return st;
   return launch_fold(false, v.d, bh, W0, Bm, ABm, nullptr, Wst, S, ctx);
@@ -452,9 +455,9 @@ int launch_dual_slice_maps(const StateArgs& a, float* A_out, float* B_out, const
   count_launch();
   int st = check_launch(ctx, "identity launch");
   if (st != kOk) return st;
-  StateArgs x = a;   // the queries are the keys: the outputs are scratch
+  StateArgs x = a;   // final states only: the state-only form, else the outputs are scratch
   x.Q = a.K;
-  x.O = a.ws;
+  x.O = dual_state_only_supported(a.d, a.C, a.dt) ? nullptr : a.ws;
   x.ws = nullptr;
   x.ws_bytes = 0;
   x.S0 = nullptr;

@@ -105,7 +105,9 @@ __device__ __forceinline__ uint32_t swz_rows(uint32_t row, uint32_t colbyte) {
   return swz<RB>(row * RB + colbyte);
 }
 
-template <int NC, int CM, int WC>
+// SO (state only): the chain alone, for callers that need the final state and no outputs (the
+// segment maps of the sequence-parallel form): no Q loads, no tcgen05 products, no O stores.
+template <int NC, int CM, int WC, bool SO>
 __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
     dual_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
       mbar_init(full + 8 * s, 1);
-      mbar_init(empty + 8 * s, NC + 1);
+      mbar_init(empty + 8 * s, SO ? NC : NC + 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(sfull + 8 * b, 1);
@@ -179,8 +181,8 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
         // slot unconditionally (the arrival below releases these stores)
         if (!p.eta)
           for (int i = 0; i < TR; ++i) stsf(st + 3 * TILE + 4 * i, p.eta_scalar);
-        mbar_arrive_expect_tx(fb, 3 * TILE + (p.eta ? rows * 4 : 0));
-        tma_load_3d(st, &tmQ, fb, 0, j * TR, stream);
+        mbar_arrive_expect_tx(fb, (SO ? 2 : 3) * TILE + (p.eta ? rows * 4 : 0));
+        if (!SO) tma_load_3d(st, &tmQ, fb, 0, j * TR, stream);
         tma_load_3d(st + TILE, &tmK, fb, 0, j * TR, stream);
         tma_load_3d(st + 2 * TILE, &tmV, fb, 0, j * TR, stream);
         if (p.eta)
@@ -191,6 +193,8 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
       for (int j = max(0, issued - NSTAGE); j < issued; ++j)
         mbar_wait(full + 8 * (j % NSTAGE), (j / NSTAGE) & 1, p.err, 1000000000ull);
     }
+  } else if (SO && warp >= Cfg::MMA) {
+    // state only: no products and no outputs
   } else if (warp == Cfg::MMA) {
     // ------------------------------------------------------------------ tcgen05 issue warp
     // The whole warp runs the loop (warp-uniform waits); an elected lane issues.
@@ -382,7 +386,7 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
     for (int j = 0; j < nst; ++j) {
       const int s = j % NSTAGE, b = j & 1;
       bool got = mbar_wait_warp(full + 8 * s, (j / NSTAGE) & 1, p.err, p.wait_ns);
-      if (got && j >= 2)
+      if (!SO && got && j >= 2)
         got = mbar_wait_warp(ofull + 8 * b, ((j >> 1) - 1) & 1, p.err, p.wait_ns);
       if (!got) {
         ok = false;
@@ -396,17 +400,19 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
       const int chunks = min(TR, T - j * TR) / TC;
       // bf16(W_s)^T rows for the stage's Q W_s product: the B fragments of two k-steps per
       // stmatrix (matrix m: k = 32 pp + 8 m)
+      if constexpr (!SO) {
 #pragma unroll
-      for (int pp = 0; pp < TKS / 2; ++pp) {
-        const uint32_t w00 = movm_t(pack_bf16(wc[2 * pp][0], wc[2 * pp][1]));
-        const uint32_t w01 = movm_t(pack_bf16(wc[2 * pp][2], wc[2 * pp][3]));
-        const uint32_t w10 = movm_t(pack_bf16(wc[2 * pp + 1][0], wc[2 * pp + 1][1]));
-        const uint32_t w11 = movm_t(pack_bf16(wc[2 * pp + 1][2], wc[2 * pp + 1][3]));
-        stsm_x4(sW + swz_rows<128>(srow, 2 * (32 * pp + 8 * mi)), w00, w01, w10, w11);
+        for (int pp = 0; pp < TKS / 2; ++pp) {
+          const uint32_t w00 = movm_t(pack_bf16(wc[2 * pp][0], wc[2 * pp][1]));
+          const uint32_t w01 = movm_t(pack_bf16(wc[2 * pp][2], wc[2 * pp][3]));
+          const uint32_t w10 = movm_t(pack_bf16(wc[2 * pp + 1][0], wc[2 * pp + 1][1]));
+          const uint32_t w11 = movm_t(pack_bf16(wc[2 * pp + 1][2], wc[2 * pp + 1][3]));
+          stsm_x4(sW + swz_rows<128>(srow, 2 * (32 * pp + 8 * mi)), w00, w01, w10, w11);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(wready + 8 * b);
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(wready + 8 * b);
 
       auto load = [&](Ops8& o, const int c) {
         const uint32_t cb = c * CHUNK_BYTES;
@@ -446,9 +452,10 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
         for (int mt = 0; mt < TKS; ++mt)
           mma16816(wc[mt], o.kt[mt][0], o.kt[mt][1], o.kt[mt][2], o.kt[mt][3], n0, n1);
         // -E^T of chunk c (lanes 0-7 address matrix 0, tokens 16c..; lanes 8-15 matrix 1)
-        stsm_x2(sE + (c >> 2) * Cfg::ESUB +
-                    swz_rows<128>(srow, 2 * (16 * (c & 3) + 8 * (mi & 1))),
-                n0, n1);
+        if constexpr (!SO)
+          stsm_x2(sE + (c >> 2) * Cfg::ESUB +
+                      swz_rows<128>(srow, 2 * (16 * (c & 3) + 8 * (mi & 1))),
+                  n0, n1);
       };
       if (chunks == TCPS) {
         Ops8 ops[2];
@@ -469,7 +476,7 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(eready + 8 * b);
+        if (!SO) mbar_arrive(eready + 8 * b);
         mbar_arrive(empty + 8 * s);
       }
     }
@@ -528,7 +535,7 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
       // warp-uniform waits: the stmatrix stores below need every lane
       bool got = mbar_wait_warp(full + 8 * s, (j / NSTAGE) & 1, p.err, p.wait_ns);
       // E and W_s buffers b were last read by the products of stage j-2
-      if (got && j >= 2)
+      if (!SO && got && j >= 2)
         got = mbar_wait_warp(ofull + 8 * b, ((j >> 1) - 1) & 1, p.err, p.wait_ns);
       if (!got) {
         ok = false;
@@ -542,15 +549,17 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
       const int chunks = min(TR, T - j * TR) / TC;
 
       // bf16(W_s^T) for the stage's Q W_s product
+      if constexpr (!SO) {
 #pragma unroll
-      for (int ks = 0; ks < TKS; ++ks)
-        stsm_x4(sW + swz_rows<128>(srow, 2 * (16 * ks + scol)),
-                pack_bf16(wc[2 * ks][0], wc[2 * ks][1]), pack_bf16(wc[2 * ks][2], wc[2 * ks][3]),
-                pack_bf16(wc[2 * ks + 1][0], wc[2 * ks + 1][1]),
-                pack_bf16(wc[2 * ks + 1][2], wc[2 * ks + 1][3]));
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(wready + 8 * b);
+        for (int ks = 0; ks < TKS; ++ks)
+          stsm_x4(sW + swz_rows<128>(srow, 2 * (16 * ks + scol)),
+                  pack_bf16(wc[2 * ks][0], wc[2 * ks][1]), pack_bf16(wc[2 * ks][2], wc[2 * ks][3]),
+                  pack_bf16(wc[2 * ks + 1][0], wc[2 * ks + 1][1]),
+                  pack_bf16(wc[2 * ks + 1][2], wc[2 * ks + 1][3]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(wready + 8 * b);
+      }
 
       auto load = [&](Ops& o, const int c) {
         const uint32_t cb = c * CHUNK_BYTES;
@@ -601,8 +610,9 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
           mma16816(wc[2 * jp + 1], n0, n1, n2, n3, o.kt[jp][2], o.kt[jp][3]);
         }
         // -E^T of chunk c: tokens 16c .. 16c+15 of the stage's [COLS][128] buffer
-        stsm_x4(sE + (c >> 2) * Cfg::ESUB + swz_rows<128>(srow, 2 * (16 * (c & 3) + scol)), n0,
-                n1, n2, n3);
+        if constexpr (!SO)
+          stsm_x4(sE + (c >> 2) * Cfg::ESUB + swz_rows<128>(srow, 2 * (16 * (c & 3) + scol)),
+                  n0, n1, n2, n3);
       };
       if constexpr (CM == 1) {
         if (chunks == TCPS) {
@@ -666,8 +676,10 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
             ne[m][1] = pack_bf16(E[0][2], E[0][3]) ^ 0x80008000u;
             ne[m][2] = pack_bf16(E[1][0], E[1][1]) ^ 0x80008000u;
             ne[m][3] = pack_bf16(E[1][2], E[1][3]) ^ 0x80008000u;
-            stsm_x4(sE + (c >> 2) * Cfg::ESUB + swz_rows<128>(srow, 2 * (16 * (c & 3) + scol)),
-                    ne[m][0], ne[m][1], ne[m][2], ne[m][3]);
+            if constexpr (!SO)
+              stsm_x4(sE + (c >> 2) * Cfg::ESUB +
+                          swz_rows<128>(srow, 2 * (16 * (c & 3) + scol)),
+                      ne[m][0], ne[m][1], ne[m][2], ne[m][3]);
           }
 #pragma unroll
           for (int m = 0; m < CM; ++m) {
@@ -694,7 +706,7 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(eready + 8 * b);
+        if (!SO) mbar_arrive(eready + 8 * b);
         mbar_arrive(empty + 8 * s);   // K, V and the rates of the stage are consumed
       }
     }
@@ -715,7 +727,7 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
   if (warp == Cfg::MMA) umma::tmem_dealloc(tmem, Cfg::TM_COLS);
 }
 
-template <int NC, int CM, int WC>
+template <int NC, int CM, int WC, bool SO>
 int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
   using Cfg = TcCfg<NC, WC>;
   const int BH = a.B * a.H;
@@ -731,9 +743,9 @@ int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
   if (!make_tmap_3d(&tq, a.Q, bf, dims, strides, box_in, CU_TENSOR_MAP_SWIZZLE_128B, ctx.msg) ||
       !make_tmap_3d(&tk, a.K, bf, dims, strides, box_in, CU_TENSOR_MAP_SWIZZLE_128B, ctx.msg) ||
       !make_tmap_3d(&tv, a.V, bf, dims, strides, box_in, CU_TENSOR_MAP_SWIZZLE_128B, ctx.msg) ||
-      !make_tmap_3d(&to, a.O, bf, dims, strides, box_out, osw, ctx.msg))
+      !make_tmap_3d(&to, SO ? a.K : a.O, bf, dims, strides, box_out, osw, ctx.msg))
     return kCuda;
-  auto kern = dual_tc_kernel<NC, CM, WC>;
+  auto kern = dual_tc_kernel<NC, CM, WC, SO>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) {
@@ -757,9 +769,13 @@ template <int CM, int WC>
 int launch_split(const StateArgs& a, int split, const LaunchCtx& ctx) {
   constexpr int N1 = 64 / WC;   // chain warps with one CTA per stream
   switch (split) {
-    case 1: return launch_tc<N1, CM, WC>(a, ctx);
-    case 2: return launch_tc<N1 / 2, CM, WC>(a, ctx);
-    case 4: return launch_tc<N1 / 4, CM, WC>(a, ctx);
+    case 1: return a.O ? launch_tc<N1, CM, WC, false>(a, ctx) : launch_tc<N1, CM, WC, true>(a, ctx);
+    case 2:
+      return a.O ? launch_tc<N1 / 2, CM, WC, false>(a, ctx)
+                 : launch_tc<N1 / 2, CM, WC, true>(a, ctx);
+    case 4:
+      return a.O ? launch_tc<N1 / 4, CM, WC, false>(a, ctx)
+                 : launch_tc<N1 / 4, CM, WC, true>(a, ctx);
   }
   *ctx.msg = "dual_tc: column split must be 1, 2 or 4";
   return kUnsupported;

@@ -115,6 +115,9 @@ int launch_dual_gram(const StateArgs& a, const LaunchCtx& ctx);
 // the data-only products on tcgen05 (dual_rgram.cu).
 int launch_dual_rgram(const StateArgs& a, const LaunchCtx& ctx);
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx);
+// True when launch_dual_mma takes O = nullptr for this shape (the stage kernel's state-only
+// form: the final state and no outputs).
+bool dual_state_only_supported(int d, int C, int dt);
 
 // Associative mode.
 size_t assoc_workspace_bytes(int B, int H, int T, int d, int C);
