@@ -87,6 +87,7 @@ struct DualBwdParams {
   float* dW0;
   uint16_t* ckpt;       // [streams, T / 16, d, d] bf16
   int T;
+  int have_ckpt;        // the checkpoints are already written (sweep 1 is skipped)
 };
 
 // m16n8k16 operand fragments from padded shared tiles (row stride rs bytes).
@@ -214,10 +215,10 @@ __global__ void __launch_bounds__(THREADS, 1) dual_bwd_kernel(const DualBwdParam
   put_state(sb + L::XB, nullptr);
 #pragma unroll
   for (int s = 0; s < L::NBUF - 1; ++s) {   // one commit group per ring slot, empty past the end
-    if (s < n) load_kv(s);
+    if (s < n && !p.have_ckpt) load_kv(s);
     cp_async_commit();
   }
-  for (int c = 0; c < n; ++c) {
+  for (int c = 0; c < (p.have_ckpt ? 0 : n); ++c) {
     const uint32_t in = sb + (c % L::NBUF) * L::IN_BYTES;
     const uint32_t wb = sb + L::XB + (c & 1) * L::WBYTES;
     const uint32_t wn = sb + L::XB + ((c + 1) & 1) * L::WBYTES;
@@ -550,7 +551,18 @@ int launch_dual_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx) {
   p.dW0 = a.dS0;
   p.ckpt = static_cast<uint16_t*>(a.ws);
   p.T = a.T;
+  p.have_ckpt = 0;
   const int streams = a.B * a.H;
+  // d = 64: the chunk-start checkpoints come from the stage kernel's state-only chain (one SM's
+  // four chain warps per stream, no block barriers), which writes them faster than this
+  // kernel's own forward sweep; "dual_bwd_checkpoints" = 1 keeps the in-kernel sweep
+  if (a.d == 64 && tuning(kTuneDualBwdCheckpoints) != 1) {
+    StateArgs f{a.K, a.K, a.V, a.eta, a.eta_scalar, a.S0, nullptr, nullptr, a.B, a.H, a.T, a.d,
+                BC, 1, nullptr, 0};
+    const int st = launch_dual_tc_checkpoints(f, p.ckpt, ctx);
+    if (st != kOk) return st;
+    p.have_ckpt = 1;
+  }
   switch (a.d) {
     case 32: return launch_d<32>(p, streams, ctx);
     case 64: return launch_d<64>(p, streams, ctx);

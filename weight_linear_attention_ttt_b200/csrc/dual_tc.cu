@@ -107,11 +107,15 @@ __device__ __forceinline__ uint32_t swz_rows(uint32_t row, uint32_t colbyte) {
 
 // SO (state only): the chain alone, for callers that need the final state and no outputs (the
 // segment maps of the sequence-parallel form): no Q loads, no tcgen05 products, no O stores.
-template <int NC, int CM, int WC, bool SO>
+// CK (with SO, 16-column chains, C = 16): every chunk's starting state leaves as a bf16 d x d
+// checkpoint through tmC (the dual-form backward's input): each chain warp stages its 16
+// columns with stmatrix.trans and TMA-stores them.
+template <int NC, int CM, int WC, bool SO, bool CK = false>
 __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
     dual_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                   const TcParams p) {
+                   const __grid_constant__ CUtensorMap tmC, const TcParams p) {
+  static_assert(!CK || (SO && WC == 16 && CM == 1), "checkpoints: state-only 16-column chains");
   using Cfg = TcCfg<NC, WC>;
   constexpr int COLS = Cfg::COLS;
   extern __shared__ uint8_t smem_raw[];
@@ -480,7 +484,7 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
         mbar_arrive(empty + 8 * s);
       }
     }
-    if (ok) {
+    if (ok && p.Wout) {
       float* wo = p.Wout + (size_t)stream * TD * TD;
 #pragma unroll
       for (int mt = 0; mt < TKS; ++mt)
@@ -583,6 +587,25 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
           wa[ks][1] = pack_bf16(wc[2 * ks][2], wc[2 * ks][3]);
           wa[ks][2] = pack_bf16(wc[2 * ks + 1][0], wc[2 * ks + 1][1]);
           wa[ks][3] = pack_bf16(wc[2 * ks + 1][2], wc[2 * ks + 1][3]);
+        }
+        if constexpr (CK) {
+          // checkpoint W_c: wa holds this warp's 16 columns of bf16(W) as W^T fragments;
+          // stmatrix.trans writes them as W rows into a [64 rows][16 columns] tile (32-byte rows,
+          // double-buffered by chunk parity), which one TMA store sends to the checkpoint
+          const int gc = j * TCPS + c;
+          const uint32_t ctile = sbase + Cfg::E_OFF + warp * 4096 + (gc & 1) * 2048;
+          if (lane == 0) bulk_wait_read<1>();   // the store of chunk gc-2 has read this tile
+          __syncwarp();
+#pragma unroll
+          for (int ks = 0; ks < TKS; ++ks)
+            stsm_x4_t(ctile + (16 * ks + (lane & 7) + 8 * (lane >> 4)) * 32 + ((lane >> 3) & 1) * 16,
+                      wa[ks][0], wa[ks][1], wa[ks][2], wa[ks][3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmC, ctile, colg, 0, stream * (T / TC) + gc);
+            bulk_commit();
+          }
         }
         float pa[2][4] = {}, pb[2][4] = {};
 #pragma unroll
@@ -710,7 +733,7 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
         mbar_arrive(empty + 8 * s);   // K, V and the rates of the stage are consumed
       }
     }
-    if (ok) {
+    if (ok && p.Wout) {
       float* wo = p.Wout + (size_t)stream * TD * TD;
 #pragma unroll
       for (int jt = 0; jt < TD / 8; ++jt)
@@ -721,14 +744,17 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
           wo[row * TD + colg + g + 8] = wc[jt][2 + e];
         }
     }
+    if constexpr (CK) {
+      if (lane == 0) bulk_wait<0>();   // the checkpoint stores have completed
+    }
   }
   umma::fence_before();
   __syncthreads();
   if (warp == Cfg::MMA) umma::tmem_dealloc(tmem, Cfg::TM_COLS);
 }
 
-template <int NC, int CM, int WC, bool SO>
-int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
+template <int NC, int CM, int WC, bool SO, bool CK = false>
+int launch_tc(const StateArgs& a, const LaunchCtx& ctx, uint16_t* ckpt = nullptr) {
   using Cfg = TcCfg<NC, WC>;
   const int BH = a.B * a.H;
   CUtensorMap tq, tk, tv, to;
@@ -745,7 +771,16 @@ int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
       !make_tmap_3d(&tv, a.V, bf, dims, strides, box_in, CU_TENSOR_MAP_SWIZZLE_128B, ctx.msg) ||
       !make_tmap_3d(&to, SO ? a.K : a.O, bf, dims, strides, box_out, osw, ctx.msg))
     return kCuda;
-  auto kern = dual_tc_kernel<NC, CM, WC, SO>;
+  CUtensorMap tc = tk;   // checkpoint map (CK only)
+  if (CK) {
+    const int n = a.T / TC;
+    const uint64_t cdims[3] = {(uint64_t)TD, (uint64_t)TD, (uint64_t)BH * n};
+    const uint64_t cstrides[2] = {(uint64_t)TD * 2, (uint64_t)TD * TD * 2};
+    const uint32_t cbox[3] = {16, (uint32_t)TD, 1};
+    if (!make_tmap_3d(&tc, ckpt, bf, cdims, cstrides, cbox, CU_TENSOR_MAP_SWIZZLE_NONE, ctx.msg))
+      return kCuda;
+  }
+  auto kern = dual_tc_kernel<NC, CM, WC, SO, CK>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   if (e != cudaSuccess) {
@@ -755,7 +790,7 @@ int launch_tc(const StateArgs& a, const LaunchCtx& ctx) {
   const int limit = tuning(kTuneWaitLimitNs);
   TcParams p{a.eta, a.eta_scalar, a.S0, a.S_out, a.T, ctx.err,
              limit > 0 ? (uint64_t)limit : 4000000000ull};
-  kern<<<BH * Cfg::NG, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(tq, tk, tv, to, p);
+  kern<<<BH * Cfg::NG, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(tq, tk, tv, to, tc, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *ctx.msg = std::string("dual_tc launch: ") + cudaGetErrorString(e);
@@ -794,6 +829,16 @@ int dual_tc_split(int streams, int sms) {
 
 bool dual_tc_supported(int d, int C, int dt) {
   return dt == 1 && d == TD && (C == 16 || C == 32 || C == 64);
+}
+
+int launch_dual_tc_checkpoints(const StateArgs& a, uint16_t* ckpt, const LaunchCtx& ctx) {
+  if (!(dual_tc_supported(a.d, a.C, a.dt) && a.C == TC)) {
+    *ctx.msg = "dual_tc checkpoints: bf16, d = 64, C = 16 only";
+    return kUnsupported;
+  }
+  StateArgs s = a;
+  s.O = nullptr;
+  return launch_tc<4, 1, 16, true, true>(s, ctx, ckpt);
 }
 
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx) {

@@ -74,6 +74,7 @@ enum TuneKey : int {
   kTuneInplaceChunksPerLaunch,  // In-Place: 1 = one chunk per launch, 0 / 2 = chunk pairs
   kTuneDualClusterStreams,    // dual form split across SMs: streams per cluster, 1 or 2
   kTuneMomentumForm,          // momentum: 0 = one pass carrying (S, M), 1 = plain + decayed
+  kTuneDualBwdCheckpoints,    // dual backward, d = 64: 0 = stage-kernel checkpoints, 1 = own sweep
   kTuneCount
 };
 enum DualKernel : int { kDualKernelAuto = 0, kDualKernelWarp = 1, kDualKernelPair = 2,
@@ -115,6 +116,10 @@ int launch_dual_gram(const StateArgs& a, const LaunchCtx& ctx);
 // the data-only products on tcgen05 (dual_rgram.cu).
 int launch_dual_rgram(const StateArgs& a, const LaunchCtx& ctx);
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx);
+// The chunk-start states of every 16-token chunk as bf16 d x d checkpoints ([streams, T / 16,
+// d, d], the dual-form backward's layout), from the stage kernel's state-only chain (bf16,
+// d = 64, C = 16; S0 = W0, S_out may be null).
+int launch_dual_tc_checkpoints(const StateArgs& a, uint16_t* ckpt, const LaunchCtx& ctx);
 // True when launch_dual_mma takes O = nullptr for this shape (the stage kernel's state-only
 // form: the final state and no outputs).
 bool dual_state_only_supported(int d, int C, int dt);

@@ -242,6 +242,14 @@ __device__ __forceinline__ void stsm_x4(uint32_t addr, uint32_t r0, uint32_t r1,
                "r"(r0), "r"(r1), "r"(r2), "r"(r3)
                : "memory");
 }
+// stmatrix with transpose: register r_i of thread t holds elements (t / 4, 2 (t % 4) .. +1) of
+// 8x8 matrix i; memory row j of matrix i (address from lane 8 i + j) receives its column j.
+__device__ __forceinline__ void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                          uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+               "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
 // D += A * B, m16n8k16, bf16 inputs, fp32 accumulators.
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {

@@ -36,7 +36,8 @@ static const TuneName kTuneNames[] = {{"dual_column_split", kTuneDualColumnSplit
                                       {"inplace_chunks_per_launch",
                                        kTuneInplaceChunksPerLaunch},
                                       {"dual_cluster_streams", kTuneDualClusterStreams},
-                                      {"momentum_form", kTuneMomentumForm}};
+                                      {"momentum_form", kTuneMomentumForm},
+                                      {"dual_bwd_checkpoints", kTuneDualBwdCheckpoints}};
 static int tune_key(const char* name) {
   if (!name) return -1;
   for (const auto& t : kTuneNames)
