@@ -17,7 +17,9 @@
 // where reverse order walks the chunks from the last and keeps, inside a chunk, key tokens at
 // or after the query token. The state the Y pass ends with is dS0. The Z pass scales its output
 // rows by eta in its own epilogue (it writes dK); a last elementwise pass scales Y by eta in
-// place and forms deta = Y . v.
+// place and forms deta = Y . v. Y and Z carry the same state (A and its transpose), so by
+// default they run as one reverse pass (assoc_yz.cu) that reads Q, K, V and dO once; the tuning
+// key "assoc_bwd_form" = 1 runs them as the two separate scans.
 #include <cuda_bf16.h>
 
 #include <string>
@@ -107,7 +109,8 @@ int launch_assoc_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx) {
     transpose_states_kernel<<<tgrid, tblock, 0, ctx.stream>>>(a.S0, s0t, d);
     count_launch();
   }
-  if (a.dS_out) {
+  const bool fused = tuning(kTuneAssocBwdForm) != 1;   // Y and Z in one reverse pass
+  if (a.dS_out && !fused) {
     transpose_states_kernel<<<tgrid, tblock, 0, ctx.stream>>>(a.dS_out, gt, d);
     count_launch();
   }
@@ -121,20 +124,22 @@ int launch_assoc_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx) {
               a.T, d, a.C, 1, a.ws, fwd};
   int r = launch_assoc(q, ctx);
   if (r != kOk) return r;
+  if (fused) {
+    r = launch_assoc_yz(a, a.ws, fwd, ctx);
+    if (r != kOk) return r;
+  }
   // Y (into dV): queries K, keys Q, values dO, reverse order; ends with dS0
   StateArgs y{a.K, a.Q, a.dO, nullptr, 1.0f, a.dS_out, a.dV, a.dS0, a.B, a.H, a.T, d, a.C, 1,
               a.ws, fwd};
   y.reverse = 1;
-  r = launch_assoc(y, ctx);
-  if (r != kOk) return r;
+  if (!fused && (r = launch_assoc(y, ctx)) != kOk) return r;
   // Z (into dK): queries V, keys dO, values Q, reverse order
   StateArgs z{a.V, a.dO, a.Q, nullptr, 1.0f, a.dS_out ? gt : nullptr, a.dK, junk, a.B, a.H, a.T,
               d, a.C, 1, a.ws, fwd};
   z.reverse = 1;
   z.orow = a.eta;                              // dK = eta Z, scaled in the pass's epilogue
   z.oscale = a.eta ? 1.f : a.eta_scalar;
-  r = launch_assoc(z, ctx);
-  if (r != kOk) return r;
+  if (!fused && (r = launch_assoc(z, ctx)) != kOk) return r;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

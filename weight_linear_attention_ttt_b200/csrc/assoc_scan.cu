@@ -716,6 +716,94 @@ size_t assoc_workspace_bytes(int B, int H, int T, int d, int C_) {
   return (size_t)B * H * (P - 1) * F * D * D * sizeof(float);
 }
 
+namespace {
+
+// Tensor maps and the launch parameters shared by both passes of one call.
+int assoc_setup(const StateArgs& a, CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv,
+                CUtensorMap* to, AssocParams* pp, const LaunchCtx& ctx) {
+  const int BH = a.B * a.H;
+  // d = 64: the tiles' second 64-wide half lies past the tensor and is filled with zeros, and
+  // only the first half of each output tile is stored
+  const uint64_t dims[3] = {(uint64_t)a.d, (uint64_t)a.T, (uint64_t)BH};
+  const uint64_t strides[2] = {(uint64_t)a.d * 2, (uint64_t)a.T * a.d * 2};
+  const uint32_t box[3] = {64, (uint32_t)C, 1};
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_tmap_3d(tq, a.Q, bf, dims, strides, box, sw, ctx.msg) ||
+      !make_tmap_3d(tk, a.K, bf, dims, strides, box, sw, ctx.msg) ||
+      !make_tmap_3d(tv, a.V, bf, dims, strides, box, sw, ctx.msg) ||
+      (a.O ? !make_tmap_3d(to, a.O, bf, dims, strides, box, sw, ctx.msg) : (*to = *tk, false)))
+    return kCuda;
+  AssocParams& p = *pp;
+  p.eta = a.eta;
+  p.eta_scalar = a.eta_scalar;
+  p.S0 = a.S0;
+  p.S_start = static_cast<const float*>(a.ws);
+  p.dim = a.d;
+  p.dst_user = 0;
+  p.T = a.T;
+  p.reverse = a.reverse;
+  p.eta_mul = a.eta_mul;
+  p.decay = a.decay;
+  p.beta = a.beta;
+  p.Oadd = static_cast<const uint16_t*>(a.Oadd);
+  p.add_scale = a.add_scale;
+  p.orow = a.orow;
+  p.oscale = a.oscale;
+  p.err = ctx.err;
+  return kOk;
+}
+
+// Pass 1 and the prefix: the increments of the first P - 1 superchunks, F pieces each (a part of
+// T / (P F) tokens per CTA), turned by the scan into the starting state of every piece.
+int run_pass1_prefix(const StateArgs& a, int P, int F, const CUtensorMap& tq,
+                     const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                     const AssocParams& p, const LaunchCtx& ctx) {
+  const int BH = a.B * a.H, pieces = (P - 1) * F;
+  AssocParams p1 = p;
+  p1.S_dst = static_cast<float*>(a.ws);
+  p1.P = pieces + 1;
+  p1.part_len = a.T / P / F;
+  int st = launch_chunk<true>(tq, tk, tv, to, p1, BH * pieces, ctx);
+  if (st != kOk) return st;
+  const float decay_L = a.decay ? powf(a.beta, (float)p1.part_len) : 1.f;
+  assoc_scan_kernel<<<dim3(D * D / 256, BH), 256, 0, ctx.stream>>>(a.S0, p1.S_dst, pieces + 1,
+                                                                   decay_L, a.d);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    *ctx.msg = std::string("assoc scan launch: ") + cudaGetErrorString(e);
+    return kCuda;
+  }
+  count_launch();
+  return kOk;
+}
+
+}  // namespace
+
+int launch_assoc_prefix(const StateArgs& a, AssocPrefix* out, const LaunchCtx& ctx) {
+  const int BH = a.B * a.H;
+  const int P = choose_parts(BH, a.T);
+  const int F = choose_pieces(BH, a.T, P);
+  const int pieces = (P - 1) * F;
+  if (a.ws_bytes < (size_t)BH * pieces * D * D * sizeof(float)) {
+    *ctx.msg = "associative prefix: workspace smaller than the pass-1 increments";
+    return kWorkspace;
+  }
+  out->P = P;
+  out->nslots = pieces;
+  out->slot_mul = F;
+  out->slots = static_cast<const float*>(a.ws);
+  if (P <= 1) return kOk;
+  CUtensorMap tq, tk, tv, to;
+  AssocParams p;
+  StateArgs s = a;
+  s.Q = a.K;   // pass 1 reads no queries
+  s.O = nullptr;
+  int st = assoc_setup(s, &tq, &tk, &tv, &to, &p, ctx);
+  if (st != kOk) return st;
+  return run_pass1_prefix(s, P, F, tq, tk, tv, to, p, ctx);
+}
+
 int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
   const int BH = a.B * a.H;
   const int P = choose_parts(BH, a.T);
@@ -727,58 +815,14 @@ int launch_assoc(const StateArgs& a, const LaunchCtx& ctx) {
     return kWorkspace;
   }
   CUtensorMap tq, tk, tv, to;
-  // d = 64: the tiles' second 64-wide half lies past the tensor and is filled with zeros, and
-  // only the first half of each output tile is stored
-  const uint64_t dims[3] = {(uint64_t)a.d, (uint64_t)a.T, (uint64_t)BH};
-  const uint64_t strides[2] = {(uint64_t)a.d * 2, (uint64_t)a.T * a.d * 2};
-  const uint32_t box[3] = {64, (uint32_t)C, 1};
-  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_tmap_3d(&tq, a.Q, bf, dims, strides, box, sw, ctx.msg) ||
-      !make_tmap_3d(&tk, a.K, bf, dims, strides, box, sw, ctx.msg) ||
-      !make_tmap_3d(&tv, a.V, bf, dims, strides, box, sw, ctx.msg) ||
-      !make_tmap_3d(&to, a.O, bf, dims, strides, box, sw, ctx.msg))
-    return kCuda;
   AssocParams p;
-  p.eta = a.eta;
-  p.eta_scalar = a.eta_scalar;
-  p.S0 = a.S0;
-  p.S_start = static_cast<const float*>(a.ws);
-  p.dim = a.d;
-  p.dst_user = 0;
-  p.T = a.T;
+  int st = assoc_setup(a, &tq, &tk, &tv, &to, &p, ctx);
+  if (st != kOk) return st;
   p.P = P;
   p.part_len = a.T / P;
-  p.reverse = a.reverse;
-  p.eta_mul = a.eta_mul;
-  p.decay = a.decay;
-  p.beta = a.beta;
-  p.Oadd = static_cast<const uint16_t*>(a.Oadd);
-  p.add_scale = a.add_scale;
-  p.orow = a.orow;
-  p.oscale = a.oscale;
-  p.err = ctx.err;
   p.nslots = pieces;
   p.slot_mul = F;
-  if (P > 1) {
-    // pass 1: the increments of the first P - 1 superchunks, F pieces each (a part of
-    // T / (P F) tokens per CTA); the scan turns them into the starting state of every piece
-    AssocParams p1 = p;
-    p1.S_dst = static_cast<float*>(a.ws);
-    p1.P = pieces + 1;
-    p1.part_len = a.T / P / F;
-    int st = launch_chunk<true>(tq, tk, tv, to, p1, BH * pieces, ctx);
-    if (st != kOk) return st;
-    const float decay_L = a.decay ? powf(a.beta, (float)p1.part_len) : 1.f;
-    assoc_scan_kernel<<<dim3(D * D / 256, BH), 256, 0, ctx.stream>>>(a.S0, p1.S_dst, pieces + 1,
-                                                                     decay_L, a.d);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) {
-      *ctx.msg = std::string("assoc scan launch: ") + cudaGetErrorString(e);
-      return kCuda;
-    }
-    count_launch();
-  }
+  if (P > 1 && (st = run_pass1_prefix(a, P, F, tq, tk, tv, to, p, ctx)) != kOk) return st;
   p.S_dst = a.S_out;
   return launch_chunk<false>(tq, tk, tv, to, p, BH * P, ctx);
 }

@@ -75,6 +75,7 @@ enum TuneKey : int {
   kTuneDualClusterStreams,    // dual form split across SMs: streams per cluster, 1 or 2
   kTuneMomentumForm,          // momentum: 0 = one pass carrying (S, M), 1 = plain + decayed
   kTuneDualBwdCheckpoints,    // dual backward, d = 64: 0 = stage-kernel checkpoints, 1 = own sweep
+  kTuneAssocBwdForm,          // associative backward: 0 = fused Y/Z pass, 1 = separate passes
   kTuneCount
 };
 enum DualKernel : int { kDualKernelAuto = 0, kDualKernelWarp = 1, kDualKernelPair = 2,
@@ -152,6 +153,17 @@ struct AssocBwdArgs {
   size_t ws_bytes;
 };
 int launch_assoc_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx);
+// The associative scan's pass 1 and prefix alone (keys a.K, values a.V, the rate and order of
+// `a`): with P > 1 superchunks, part m >= 1 starts from slot m * slot_mul - 1 of `slots`
+// ([B*H, nslots, 128, 128] fp32 in a.ws); with P = 1 nothing is launched.
+struct AssocPrefix {
+  int P, nslots, slot_mul;
+  const float* slots;
+};
+int launch_assoc_prefix(const StateArgs& a, AssocPrefix* out, const LaunchCtx& ctx);
+// Backward of the associative mode, fused reverse pass: dV <- Y (unscaled), dK <- eta Z, dS0,
+// in one pass over Q, K, V and dO (bf16, d = 64 or 128); `ws` holds the prefix slots.
+int launch_assoc_yz(const AssocBwdArgs& a, void* ws, size_t ws_bytes, const LaunchCtx& ctx);
 // Sequence-parallel dual form (segment-affine scan over the dual-form kernels). segments: the
 // caller's count (must divide T / C) or 0 for the automatic choice; returns -1 if invalid.
 int dual_seg_choose_segments(int B, int H, int T, int C, int requested);
