@@ -20,7 +20,8 @@
 // Z^T x2 [256,384), scores P1 [384,448), P2 [448,512) (M = 64).
 //
 // Warps: 0 TMA (2-stage ring of Q/K/V/dO tiles); 1 MMA issue; 2-5 scores -> masked bf16 P1, P2;
-// 6-9 state refresh (A -> bf16 copy); 10-13 outputs (Y -> dV unscaled, eta Z -> dK, TMA stores).
+// 6-9 state refresh (A -> bf16 copy); 10-13 Y -> dV (unscaled); 14-17 eta Z -> dK (each group
+// drains its accumulator through a shared tile to TMA stores).
 // The serial chain per chunk is refresh -> products and update -> refresh.
 #include <algorithm>
 #include <string>
@@ -45,7 +46,7 @@ constexpr int Y_OY = Y_P2 + YC * YC * 2;           // output staging [64 t][128]
 constexpr int Y_OZ = Y_OY + YT;
 constexpr int Y_BAR = Y_OZ + YT;
 constexpr int Y_SMEM = 1024 + Y_BAR + 256;
-constexpr int Y_THREADS = 14 * 32;
+constexpr int Y_THREADS = 18 * 32;
 static_assert(Y_SMEM <= 227 * 1024, "shared memory");
 constexpr uint32_t TY_A = 0, TY_Y = 128, TY_Z = 256, TY_P1 = 384, TY_P2 = 448;
 
@@ -74,7 +75,7 @@ __global__ void __launch_bounds__(Y_THREADS, 1)
   const uint32_t pready = bar + 48;              // P1, P2 tiles written (4 operand warps)
   const uint32_t sready = bar + 56;              // bf16 copy of A refreshed (4 state warps)
   const uint32_t cdone = bar + 64;               // products and update of a chunk done (x2)
-  const uint32_t ofree = bar + 80;               // Y^T, Z^T buffer read out (x2, 4 warps)
+  const uint32_t ofree = bar + 80;               // Y^T, Z^T buffer read out (x2, 8 warps)
   const uint32_t mdone = bar + 96;
   const uint32_t tslot = bar + 104;
   const uint32_t sA = sbase + Y_A;
@@ -97,7 +98,7 @@ __global__ void __launch_bounds__(Y_THREADS, 1)
     mbar_init(sready, 4);
     for (int b = 0; b < 2; ++b) {
       mbar_init(cdone + 8 * b, 1);
-      mbar_init(ofree + 8 * b, 4);
+      mbar_init(ofree + 8 * b, 8);
     }
     mbar_init(mdone, 1);
     fence_mbar_init();
@@ -329,83 +330,80 @@ __global__ void __launch_bounds__(Y_THREADS, 1)
       }
     }
   } else {
-    // ---------------------------------------------------------------- output warps 10..13
+    // ---------------------------------------------------------------- output warps 10..17
+    const bool zg = warp >= 14;                // warps 14..17 drain Z^T, 10..13 Y^T
     const int q = warp & 3;
-    const int row = 32 * q + lane;            // feature: j of Y^T, i of Z^T
+    const int row = 32 * q + lane;             // feature: j of Y^T, i of Z^T
     const uint32_t tl = (uint32_t)(32 * q) << 16;
-    const int otid = threadIdx.x - 320;        // 0..127
+    const int gtid = threadIdx.x - (zg ? 448 : 320);   // 0..127 within the group
+    const int gbar = zg ? 2 : 1;               // the group's named barrier
     const bool odd = lane & 1;
     const uint32_t ocol = (row >> 6) * 8192;
     const uint32_t cb = 2 * ((row & 63) & ~1);
-    // Lane pairs (2i, 2i+1) exchange one value per token pair (t, t+4) so that each lane stores
-    // a 32-bit word of two adjacent output columns: the even lane row t, the odd lane row t+4.
-    auto stage_out = [&](uint32_t tile, const uint32_t (&v)[64]) {
-#pragma unroll
-      for (int t = 0; t < YC; ++t) {
-        if (t & 4) continue;
-        const float a = __uint_as_float(v[t]), a4 = __uint_as_float(v[t + 4]);
-        const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
-        const float lo = odd ? y : a, hi = odd ? a4 : y;
-        sts32(tile + ocol + swz<128>((odd ? t + 4 : t) * 128 + cb), pack_bf16(lo, hi));
-      }
-    };
+    const uint32_t tile = sbase + (zg ? Y_OZ : Y_OY);
+    const uint32_t acc = tmem + tl + (zg ? TY_Z : TY_Y);
     for (int c = 0; c < nch; ++c) {
       const int b = c & 1;
       const bool got = mbar_wait_warp(cdone + 8 * b, (c >> 1) & 1, p.err);
-      if (bar_or_named(1, 128, !got)) break;
+      if (bar_or_named(gbar, 128, !got)) break;
       umma::fence_after();
-      // the previous chunk's stores have read the staging tiles
-      if (otid == 0) bulk_wait_read<0>();
-      bar_sync_named(1, 128);
-      {
-        uint32_t v[64];
-        umma::ld32x32(tmem + tl + TY_Y + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(v));
-        umma::ld32x32(tmem + tl + TY_Y + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      // the previous chunk's store has read the staging tile
+      if (gtid == 0) bulk_wait_read<0>();
+      bar_sync_named(gbar, 128);
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {   // tokens 32 hf .. 32 hf + 31
+        uint32_t v[32];
+        umma::ld32x32(acc + 64 * b + 32 * hf, v);
         umma::wait_ld();
-        umma::reg_fence_n(v);
-        stage_out(sbase + Y_OY, v);
-      }
-      {
-        uint32_t v[64];
-        umma::ld32x32(tmem + tl + TY_Z + 64 * b, *reinterpret_cast<uint32_t(*)[32]>(v));
-        umma::ld32x32(tmem + tl + TY_Z + 64 * b + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-        umma::wait_ld();
-        umma::reg_fence_n(v);
-        umma::fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(ofree + 8 * b);   // both accumulators of buffer b read out
-        // dK = eta Z: token t is column t of Z^T
-        if (p.eta) {
-          const float4* e4 =
-              reinterpret_cast<const float4*>(p.eta + (size_t)stream * p.T + tok(c));
-#pragma unroll
-          for (int t = 0; t < YC; t += 4) {
-            const float4 e = __ldg(e4 + t / 4);
-            v[t] = __float_as_uint(e.x * __uint_as_float(v[t]));
-            v[t + 1] = __float_as_uint(e.y * __uint_as_float(v[t + 1]));
-            v[t + 2] = __float_as_uint(e.z * __uint_as_float(v[t + 2]));
-            v[t + 3] = __float_as_uint(e.w * __uint_as_float(v[t + 3]));
-          }
-        } else {
-#pragma unroll
-          for (int t = 0; t < YC; ++t) v[t] = __float_as_uint(p.eta_scalar * __uint_as_float(v[t]));
+        umma::reg_fence(v);
+        if (hf == 1) {   // this warp's part of buffer b is read out
+          umma::fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(ofree + 8 * b);
         }
-        stage_out(sbase + Y_OZ, v);
+        if (zg) {
+          // dK = eta Z: token t is column t of Z^T
+          if (p.eta) {
+            const float4* e4 = reinterpret_cast<const float4*>(p.eta + (size_t)stream * p.T +
+                                                               tok(c) + 32 * hf);
+#pragma unroll
+            for (int t = 0; t < 32; t += 4) {
+              const float4 e = __ldg(e4 + t / 4);
+              v[t] = __float_as_uint(e.x * __uint_as_float(v[t]));
+              v[t + 1] = __float_as_uint(e.y * __uint_as_float(v[t + 1]));
+              v[t + 2] = __float_as_uint(e.z * __uint_as_float(v[t + 2]));
+              v[t + 3] = __float_as_uint(e.w * __uint_as_float(v[t + 3]));
+            }
+          } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+              v[t] = __float_as_uint(p.eta_scalar * __uint_as_float(v[t]));
+          }
+        }
+        // Lane pairs (2i, 2i+1) exchange one value per token pair (t, t+4) so that each lane
+        // stores a 32-bit word of two adjacent output columns: the even lane row t, the odd
+        // lane row t+4.
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          if (t & 4) continue;
+          const float a = __uint_as_float(v[t]), a4 = __uint_as_float(v[t + 4]);
+          const float y = __shfl_xor_sync(0xffffffffu, odd ? a : a4, 1);
+          const float lo = odd ? y : a, hi = odd ? a4 : y;
+          sts32(tile + ocol + swz<128>((32 * hf + (odd ? t + 4 : t)) * 128 + cb),
+                pack_bf16(lo, hi));
+        }
       }
       fence_proxy_async_smem();
-      bar_sync_named(1, 128);
-      if (otid == 0) {
+      bar_sync_named(gbar, 128);
+      if (gtid == 0) {
         const int t0 = tok(c);
-        tma_store_3d(&tmY, sbase + Y_OY, 0, t0, stream);
-        tma_store_3d(&tmZ, sbase + Y_OZ, 0, t0, stream);
-        if (p.dim > 64) {
-          tma_store_3d(&tmY, sbase + Y_OY + 8192, 64, t0, stream);
-          tma_store_3d(&tmZ, sbase + Y_OZ + 8192, 64, t0, stream);
-        }
+        const CUtensorMap* tm = zg ? &tmZ : &tmY;
+        tma_store_3d(tm, tile, 0, t0, stream);
+        if (p.dim > 64) tma_store_3d(tm, tile + 8192, 64, t0, stream);
         bulk_commit();
       }
     }
-    if (otid == 0) bulk_wait<0>();
+    if (gtid == 0) bulk_wait<0>();
   }
   umma::fence_before();
   __syncthreads();
