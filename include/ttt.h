@@ -116,6 +116,11 @@ uint64_t ttt_launch_count(void);
  *                        chunk i+1's read corrected by eta (Z_(i+1) Z_i^T) Vhat_i.
  *   "momentum_form"      ttt_assoc_momentum_fwd: 0 = one pass carrying (S, M) (every beta in
  *                        [0, 1]); 1 = plain + decayed associative passes (beta in [0.25, 0.9]).
+ *   "assoc_bwd_form"     ttt_assoc_scan_bwd: 0 = dV and dK in one reverse pass; 1 = two
+ *                        separate reverse passes.
+ *   "dual_bwd_checkpoints"  ttt_linear_dual_bwd, d = 64: 0 = the chunk-start checkpoints written
+ *                        by the forward stage kernel's state-only chain; 1 = by the backward
+ *                        kernel's own forward sweep.
  * Every variant computes the same operation within the same tolerance. ttt_set_tuning returns
  * TTT_ERR_INVALID_ARG for an unknown key or a negative value; ttt_get_tuning returns -1 for an
  * unknown key; ttt_reset_tuning restores every key to 0. Not synchronised with calls in flight
@@ -235,8 +240,10 @@ int ttt_assoc_momentum_fwd(const void* Q, const void* K, const void* V, const fl
  *  Supported: as ttt_assoc_scan_fwd (bf16, d == 64 or 128, C == 16, 32 or 64, T % 64 == 0).
  *  C is the evaluation granularity; the gradients do not depend on it beyond rounding.
  *  Workspace: ttt_assoc_scan_bwd_workspace_size() bytes.
- *  Runs as three passes of the forward kernel (dQ in forward order; dV and dK through the
- *  reverse-order recurrence of the state gradient) and one elementwise pass.
+ *  Runs as one pass of the forward kernel for dQ (forward order), one reverse-order pass that
+ *  carries the state gradient and writes dK and the unscaled dV (see assoc_yz.cu), and one
+ *  elementwise pass (dV = eta Y, deta). The tuning key "assoc_bwd_form" = 1 runs dV and dK as
+ *  two separate reverse passes of the forward kernel instead.
  * ------------------------------------------------------------------------------------------ */
 size_t ttt_assoc_scan_bwd_workspace_size(int B, int H, int T, int d, int C, int dt);
 int ttt_assoc_scan_bwd(const void* Q, const void* K, const void* V, const float* eta,
@@ -263,8 +270,9 @@ int ttt_assoc_scan_bwd(const void* Q, const void* K, const void* V, const float*
  *  Supported: bf16, C == 16, d in {32, 64, 128}, T % C == 0 (C changes the result: it is the
  *  mini-batch size of the forward).
  *  Workspace: ttt_linear_dual_bwd_workspace_size() bytes (one bf16 d x d state per chunk:
- *  B*H*(T/16)*d*d*2). One kernel launch: a forward sweep recomputes the chunk-start states,
- *  a reverse sweep forms the gradients (see dual_bwd.cu).
+ *  B*H*(T/16)*d*d*2). A forward sweep recomputes the chunk-start states into the workspace
+ *  (d = 64: the forward stage kernel's state-only chain, a second launch; d = 32 and 128: inside
+ *  the backward kernel), a reverse sweep forms the gradients (see dual_bwd.cu).
  * ------------------------------------------------------------------------------------------ */
 size_t ttt_linear_dual_bwd_workspace_size(int B, int H, int T, int d, int C, int dt);
 int ttt_linear_dual_bwd(const void* Q, const void* K, const void* V, const float* eta,

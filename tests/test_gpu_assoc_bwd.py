@@ -121,3 +121,20 @@ def test_errors(cuda_lib):
     with pytest.raises(ttt.TTTError) as e:    # an output aliasing an input
         run(x, dQ=x["dO"])
     assert e.value.status == 1
+
+
+@pytest.mark.parametrize("parts", [1, 2, 4])
+def test_separate_and_fused_reverse_passes(cuda_lib, tuning, parts):
+    """dV and dK from the two separate reverse passes (assoc_bwd_form 1) and from the fused one
+    that carries the state gradient once (the default) both meet the oracle for every superchunk
+    split, and agree well inside its tolerance."""
+    tuning("assoc_parts", parts)
+    x = make(1, 3, 1024, seed=41 + parts)
+    fused = run(x)
+    check(x, fused)
+    tuning("assoc_bwd_form", 1)
+    separate = run(x)
+    check(x, separate)
+    for g, r in zip(fused, separate):
+        assert max_rel_l2(g, r, 2) < 5e-3
+    assert ttt.read_device_error() == 0
