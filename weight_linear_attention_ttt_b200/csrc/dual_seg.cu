@@ -152,66 +152,58 @@ __global__ void __launch_bounds__(256) fold_segments_reverse_kernel(
 }
 
 // Column-sliced fold, d = 64: one CTA per (stream, 16-column slice of the state); the columns
-// of W <- A W + B (and of the reverse X <- A^T X + N) evolve independently. Per segment, in fold
-// order, the CTA stores the slice of the incoming state, then updates it; the maps of the next
-// segment (A + B and B, 2 x 16 KB) stream in through a double-buffered cp.async ring meanwhile,
-// and the bias of the reverse fold (N_s) is read one segment ahead into registers. Thread t
-// owns rows 4 (t / 16) .. +3 of slice column t % 16.
+// of W <- A W + B (and of the reverse X <- A^T X + N) evolve independently. The segment maps
+// arrive as A itself (the caller subtracts B from the run from W = I beforehand), so a step
+// needs A (16 KB) and the bias's 16 columns (4 KB): both stream in through a double-buffered
+// cp.async ring one segment ahead while the CTA stores the slice of the incoming state and
+// updates it. Thread t owns rows 4 (t / 16) .. +3 of slice column t % 16.
 constexpr int FD = 64, FCW = 16, FCS = FD / FCW, FPITCH = FD + 4;   // padded map rows
-constexpr int FOLD_COLS_SMEM = (FD * FCW + 2 * 2 * FD * FPITCH) * (int)sizeof(float);
+constexpr int FBUF = FD * FPITCH + FD * FCW;                        // A, bias slice (floats)
+constexpr int FOLD_COLS_SMEM = (FD * FCW + 2 * FBUF) * (int)sizeof(float);
 template <bool REV>
 __global__ void __launch_bounds__(256) fold_cols_kernel(const float* __restrict__ init,
-                                                        const float* __restrict__ Bm,
-                                                        const float* __restrict__ ABm,
-                                                        const float* __restrict__ Noff,
+                                                        const float* __restrict__ Am,
+                                                        const float* __restrict__ bias,
                                                         float* __restrict__ out, int S) {
   extern __shared__ __align__(16) float fcm[];
   float* Wsl = fcm;                    // [FD][FCW] state slice
-  float* maps = fcm + FD * FCW;        // 2 buffers x {A + B, B} [FD][FPITCH]
+  float* bufs = fcm + FD * FCW;        // 2 buffers x {A [FD][FPITCH], bias slice [FD][FCW]}
   const size_t bh = blockIdx.x / FCS;
   const int c0 = (blockIdx.x % FCS) * FCW;
   const int c = threadIdx.x % 16, r0 = 4 * (threadIdx.x / 16);
   auto seg_of = [&](int i) { return REV ? S - 1 - i : i; };
   auto prefetch = [&](int i, int b) {
     const size_t seg = (bh * S + seg_of(i)) * FD * FD;
-    float* d = maps + b * 2 * FD * FPITCH;
-    for (int e = threadIdx.x; e < FD * FD / 4; e += 256) {
-      const int r = (4 * e) / FD, k = (4 * e) % FD;
-      cp_async16(smem_u32(d + r * FPITCH + k), ABm + seg + 4 * e);
-      cp_async16(smem_u32(d + FD * FPITCH + r * FPITCH + k), Bm + seg + 4 * e);
-    }
-  };
-  auto noff = [&](int i, float (&n)[4]) {
-    const size_t seg = (bh * S + seg_of(i)) * FD * FD;
+    float* d = bufs + b * FBUF;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) n[r] = Noff[seg + (size_t)(r0 + r) * FD + c0 + c];
+    for (int k = 0; k < FD * FD / 4 / 256; ++k) {   // A: 16-byte pieces, 4 per thread
+      const int e = threadIdx.x + 256 * k;
+      cp_async16(smem_u32(d + (e / 16) * FPITCH + 4 * (e % 16)), Am + seg + 4 * e);
+    }
+    {   // bias columns c0 .. c0 + 15: one 16-byte piece per thread
+      const int row = threadIdx.x / 4, q = threadIdx.x % 4;
+      cp_async16(smem_u32(d + FD * FPITCH + row * FCW + 4 * q),
+                 bias + seg + (size_t)row * FD + c0 + 4 * q);
+    }
   };
   for (int e = threadIdx.x; e < FD * FCW; e += 256)
     Wsl[e] = init ? init[bh * FD * FD + (size_t)(e / FCW) * FD + c0 + e % FCW] : 0.f;
-  float ncur[4] = {0.f, 0.f, 0.f, 0.f}, nnext[4] = {0.f, 0.f, 0.f, 0.f};
-  if (REV && S > 0) noff(0, ncur);
   if (S > 0) prefetch(0, 0);
   cp_async_commit();
   for (int i = 0; i < S; ++i) {
     const int b = i & 1;
     if (i + 1 < S) prefetch(i + 1, b ^ 1);
     cp_async_commit();
-    if (REV && i + 1 < S) noff(i + 1, nnext);
     cp_async_wait<1>();   // segment i's maps have landed (this thread's part) ...
     __syncthreads();      // ... and every thread's; the state slice is complete
     const size_t seg = (bh * S + seg_of(i)) * FD * FD;
     for (int e = threadIdx.x; e < FD * FCW; e += 256)
       out[seg + (size_t)(e / FCW) * FD + c0 + e % FCW] = Wsl[e];
-    float* AB = maps + b * 2 * FD * FPITCH;   // becomes A = (A + B) - B in place
-    const float* Bb = AB + FD * FPITCH;
-    for (int e = threadIdx.x; e < FD * FD; e += 256) {
-      const int r = e / FD, k = e % FD;
-      AB[r * FPITCH + k] -= Bb[r * FPITCH + k];
-    }
+    const float* A = bufs + b * FBUF;
+    const float* bs = A + FD * FPITCH;
     float acc[4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) acc[r] = REV ? ncur[r] : Bb[(r0 + r) * FPITCH + c0 + c];
-    __syncthreads();      // A complete
+    for (int r = 0; r < 4; ++r) acc[r] = bs[(r0 + r) * FCW + c];
 #pragma unroll 4
     for (int k = 0; k < FD; k += 4) {
       float w[4];
@@ -220,7 +212,7 @@ __global__ void __launch_bounds__(256) fold_cols_kernel(const float* __restrict_
       if constexpr (REV) {   // A^T: row k of A, columns r0 .. r0+3
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const float4 a = *reinterpret_cast<const float4*>(AB + (k + kk) * FPITCH + r0);
+          const float4 a = *reinterpret_cast<const float4*>(A + (k + kk) * FPITCH + r0);
           acc[0] = fmaf(a.x, w[kk], acc[0]);
           acc[1] = fmaf(a.y, w[kk], acc[1]);
           acc[2] = fmaf(a.z, w[kk], acc[2]);
@@ -229,7 +221,7 @@ __global__ void __launch_bounds__(256) fold_cols_kernel(const float* __restrict_
       } else {               // A: rows r0 .. r0+3, columns k .. k+3
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const float4 a = *reinterpret_cast<const float4*>(AB + (r0 + r) * FPITCH + k);
+          const float4 a = *reinterpret_cast<const float4*>(A + (r0 + r) * FPITCH + k);
           acc[r] = fmaf(a.x, w[0], fmaf(a.y, w[1], fmaf(a.z, w[2], fmaf(a.w, w[3], acc[r]))));
         }
       }
@@ -237,10 +229,6 @@ __global__ void __launch_bounds__(256) fold_cols_kernel(const float* __restrict_
     __syncthreads();      // every thread has read the slice and the maps of buffer b
 #pragma unroll
     for (int r = 0; r < 4; ++r) Wsl[(r0 + r) * FCW + c] = acc[r];
-    if (REV) {
-#pragma unroll
-      for (int r = 0; r < 4; ++r) ncur[r] = nnext[r];
-    }
   }
   cp_async_wait_all();
 }
@@ -339,19 +327,20 @@ int launch_fold(bool reverse, int d, int bh, const float* init, const float* Bm,
         fold_segments_kernel<32><<<bh, 256, smem, ctx.stream>>>(init, Bm, ABm, dst, S);
       break;
     case 64:
-      // column-sliced, with the maps streamed one segment ahead (fold_cols_kernel)
+      // column-sliced, with the maps streamed one segment ahead (fold_cols_kernel); the maps
+      // buffer holds A itself here (maps_and_fold subtracted B)
       if (reverse) {
         e = cudaFuncSetAttribute(fold_cols_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, FOLD_COLS_SMEM);
         if (e == cudaSuccess)
-          fold_cols_kernel<true><<<bh * FCS, 256, FOLD_COLS_SMEM, ctx.stream>>>(init, Bm, ABm,
-                                                                              Noff, dst, S);
+          fold_cols_kernel<true><<<bh * FCS, 256, FOLD_COLS_SMEM, ctx.stream>>>(init, ABm, Noff,
+                                                                              dst, S);
       } else {
         e = cudaFuncSetAttribute(fold_cols_kernel<false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, FOLD_COLS_SMEM);
         if (e == cudaSuccess)
-          fold_cols_kernel<false><<<bh * FCS, 256, FOLD_COLS_SMEM, ctx.stream>>>(init, Bm, ABm,
-                                                                               nullptr, dst, S);
+          fold_cols_kernel<false><<<bh * FCS, 256, FOLD_COLS_SMEM, ctx.stream>>>(init, ABm, Bm,
+                                                                               dst, S);
       }
       break;
     case 128:
@@ -398,6 +387,11 @@ int maps_and_fold(const StateArgs& v, int S, int bh, const float* W0, void* Ojun
   pa.O = maps_O;
   pa.S_out = ABm;
   if ((st = run_dual(pa, ctx)) != kOk) return st;
+  if (v.d == 64) {   // the column-sliced fold takes A itself: A + B -> A in place
+    sub_states_kernel<<<sm_count() * 2, 256, 0, ctx.stream>>>(ABm, Bm, n * v.d * v.d);
+    count_launch();
+    if ((st = check_launch(ctx, "map difference launch")) != kOk) return st;
+  }
   return launch_fold(false, v.d, bh, W0, Bm, ABm, nullptr, Wst, S, ctx);
 }
 
