@@ -43,7 +43,7 @@ DOMINANT_KERNEL = {"dual": ("dual_tc_kernel", "dual_tc.cu"),
                    "dual_seg": ("dual_tc_kernel", "dual_tc.cu"),
                    "assoc": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu"),
-                   "assoc_bwd": ("assoc_chunk_kernel", "assoc_scan.cu"),
+                   "assoc_bwd": ("assoc_yz_kernel", "assoc_yz.cu"),
                    "dual_bwd": ("dual_bwd_kernel", "dual_bwd.cu"),
                    "dual_seg_bwd": ("dual_bwd_kernel", "dual_bwd.cu"),
                    "assoc_momentum": ("mom_chunk_kernel", "assoc_mom.cu"),
@@ -553,6 +553,8 @@ def run_ours(args, w, rank, world, local_rank):
     if w.kind == "dual" and ttt.get_tuning("dual_kernel") == 6:   # the register-state Gram kernel
         kname, ksrc = "dual_rgram_kernel", "dual_rgram.cu"
     if w.kind == "assoc_momentum" and ttt.get_tuning("momentum_form") == 1:   # two-pass form
+        kname, ksrc = "assoc_chunk_kernel", "assoc_scan.cu"
+    if w.kind == "assoc_bwd" and ttt.get_tuning("assoc_bwd_form") == 1:   # separate passes
         kname, ksrc = "assoc_chunk_kernel", "assoc_scan.cu"
     launches_per_step = launches / args.steps
     # the roofline is the slower of the flops at the tensor peak and the bytes at HBM bandwidth
