@@ -26,7 +26,8 @@ def algorithmic(w: Workload) -> dict:
     """{'flops': F, 'bytes': B, 'tokens': N} for one call of the workload."""
     if w.kind == "assoc_momentum":
         # the momentum recurrence reads and writes what the plain one does, plus the momentum
-        # state (in and out); flops: the plain and the decayed chunk steps
+        # state (in and out); flops: the chunk steps of both states, about twice the plain
+        # recurrence's
         a = algorithmic(dataclasses.replace(w, kind="assoc"))
         return {"flops": 2 * a["flops"], "bytes": a["bytes"] + w.B * w.H * 2 * w.d * w.d * 4,
                 "tokens": a["tokens"]}
