@@ -45,7 +45,7 @@ constexpr int Y_P2 = Y_P1 + YC * YC * 2;
 constexpr int Y_OY = Y_P2 + YC * YC * 2;           // output staging [64 t][128] bf16
 constexpr int Y_OZ = Y_OY + YT;
 constexpr int Y_BAR = Y_OZ + YT;
-constexpr int Y_SMEM = 1024 + Y_BAR + 256;
+constexpr int Y_SMEM = 1024 + Y_BAR + 512;   // barriers, then the Z group's rate table
 constexpr int Y_THREADS = 18 * 32;
 static_assert(Y_SMEM <= 227 * 1024, "shared memory");
 constexpr uint32_t TY_A = 0, TY_Y = 128, TY_Z = 256, TY_P1 = 384, TY_P2 = 448;
@@ -344,10 +344,18 @@ __global__ void __launch_bounds__(Y_THREADS, 1)
     const uint32_t acc = tmem + tl + (zg ? TY_Z : TY_Y);
     for (int c = 0; c < nch; ++c) {
       const int b = c & 1;
+      // Z group: the chunk's 64 rates, loaded before the wait so that their latency hides there
+      float4 e4 = make_float4(p.eta_scalar, p.eta_scalar, p.eta_scalar, p.eta_scalar);
+      if (zg && p.eta && gtid < 16)
+        e4 = __ldg(reinterpret_cast<const float4*>(p.eta + (size_t)stream * p.T + tok(c)) + gtid);
       const bool got = mbar_wait_warp(cdone + 8 * b, (c >> 1) & 1, p.err);
       if (bar_or_named(gbar, 128, !got)) break;
       umma::fence_after();
-      // the previous chunk's store has read the staging tile
+      const uint32_t etab = sbase + Y_BAR + 256;   // the Z group's rates of the chunk
+      if (zg && gtid < 16)
+        sts128(etab + 16 * gtid, make_uint4(__float_as_uint(e4.x), __float_as_uint(e4.y),
+                                            __float_as_uint(e4.z), __float_as_uint(e4.w)));
+      // the previous chunk's store has read the staging tile (and the rates are in place)
       if (gtid == 0) bulk_wait_read<0>();
       bar_sync_named(gbar, 128);
 #pragma unroll 1
@@ -363,21 +371,13 @@ __global__ void __launch_bounds__(Y_THREADS, 1)
         }
         if (zg) {
           // dK = eta Z: token t is column t of Z^T
-          if (p.eta) {
-            const float4* e4 = reinterpret_cast<const float4*>(p.eta + (size_t)stream * p.T +
-                                                               tok(c) + 32 * hf);
 #pragma unroll
-            for (int t = 0; t < 32; t += 4) {
-              const float4 e = __ldg(e4 + t / 4);
-              v[t] = __float_as_uint(e.x * __uint_as_float(v[t]));
-              v[t + 1] = __float_as_uint(e.y * __uint_as_float(v[t + 1]));
-              v[t + 2] = __float_as_uint(e.z * __uint_as_float(v[t + 2]));
-              v[t + 3] = __float_as_uint(e.w * __uint_as_float(v[t + 3]));
-            }
-          } else {
-#pragma unroll
-            for (int t = 0; t < 32; ++t)
-              v[t] = __float_as_uint(p.eta_scalar * __uint_as_float(v[t]));
+          for (int t = 0; t < 32; t += 4) {
+            const uint4 e = lds128(etab + 4 * (32 * hf + t));
+            v[t] = __float_as_uint(__uint_as_float(e.x) * __uint_as_float(v[t]));
+            v[t + 1] = __float_as_uint(__uint_as_float(e.y) * __uint_as_float(v[t + 1]));
+            v[t + 2] = __float_as_uint(__uint_as_float(e.z) * __uint_as_float(v[t + 2]));
+            v[t + 3] = __float_as_uint(__uint_as_float(e.w) * __uint_as_float(v[t + 3]));
           }
         }
         // Lane pairs (2i, 2i+1) exchange one value per token pair (t, t+4) so that each lane
