@@ -577,8 +577,8 @@ def run_ours(args, w, rank, world, local_rank):
                  "peak_source": f"{pk_kind} (MEASURED_PEAKS.json)" if pk_kind == "measured"
                  else "fallback", "launches_per_step": launches_per_step,
                  "kernel_source_sha": sha,
-                 "duration_us": 1e3 * ms_per_step / max(1.0, launches_per_step)
-                 if w.kind in ("dual", "dual_bwd") else None})
+                 "duration_us": 1e3 * ms_per_step
+                 if w.kind in ("dual", "dual_bwd") and launches_per_step <= 1.0 else None})
 
     line = {"metric": metric_of(w), "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
