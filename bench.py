@@ -44,8 +44,8 @@ DOMINANT_KERNEL = {"dual": ("dual_tc_kernel", "dual_tc.cu"),
                    "assoc": ("assoc_chunk_kernel", "assoc_scan.cu"),
                    "inplace": ("inplace_chunk_kernel", "inplace_ttt.cu"),
                    "assoc_bwd": ("assoc_yz_kernel", "assoc_yz.cu"),
-                   "dual_bwd": ("dual_bwd_kernel", "dual_bwd.cu"),
-                   "dual_seg_bwd": ("dual_bwd_kernel", "dual_bwd.cu"),
+                   "dual_bwd": ("dual_bwd_tc_kernel", "dual_bwd_tc.cu"),
+                   "dual_seg_bwd": ("dual_bwd_tc_kernel", "dual_bwd_tc.cu"),
                    "assoc_momentum": ("mom_chunk_kernel", "assoc_mom.cu"),
                    "inplace_lm": ("inplace_chunk_kernel", "inplace_ttt.cu")}
 
@@ -556,6 +556,8 @@ def run_ours(args, w, rank, world, local_rank):
         kname, ksrc = "assoc_chunk_kernel", "assoc_scan.cu"
     if w.kind == "assoc_bwd" and ttt.get_tuning("assoc_bwd_form") == 1:   # separate passes
         kname, ksrc = "assoc_chunk_kernel", "assoc_scan.cu"
+    if w.kind in ("dual_bwd", "dual_seg_bwd") and ttt.get_tuning("dual_bwd_form") in (1, 2):
+        kname, ksrc = "dual_bwd_kernel", "dual_bwd.cu"   # the warp-MMA reverse sweep
     launches_per_step = launches / args.steps
     # the roofline is the slower of the flops at the tensor peak and the bytes at HBM bandwidth
     t_flops = algo["flops"] / (pk["bf16_tflops"] * 1e12)

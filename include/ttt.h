@@ -118,9 +118,13 @@ uint64_t ttt_launch_count(void);
  *                        [0, 1]); 1 = plain + decayed associative passes (beta in [0.25, 0.9]).
  *   "assoc_bwd_form"     ttt_assoc_scan_bwd: 0 = dV and dK in one reverse pass; 1 = two
  *                        separate reverse passes.
- *   "dual_bwd_checkpoints"  ttt_linear_dual_bwd, d = 64: 0 = the chunk-start checkpoints written
- *                        by the forward stage kernel's state-only chain; 1 = by the backward
- *                        kernel's own forward sweep.
+ *   "dual_bwd_form"      ttt_linear_dual_bwd, d = 64: 0 = stage form (the forward's residuals
+ *                        and stage-start states from the stage kernel's state-only chain, then
+ *                        the state gradient's chain on warp MMAs and every product that needs
+ *                        the forward states on tcgen05, per 128-token stage); 1 = one kernel
+ *                        that recomputes every chunk-start state in a forward sweep, then runs
+ *                        the reverse sweep on warp MMAs; 2 = the chunk-start states from the
+ *                        stage kernel's chain, then that reverse sweep.
  * Every variant computes the same operation within the same tolerance. ttt_set_tuning returns
  * TTT_ERR_INVALID_ARG for an unknown key or a negative value; ttt_get_tuning returns -1 for an
  * unknown key; ttt_reset_tuning restores every key to 0. Not synchronised with calls in flight

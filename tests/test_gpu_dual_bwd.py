@@ -121,16 +121,17 @@ def test_errors(cuda_lib):
 
 
 @pytest.mark.parametrize("T", [16, 272, 1024])
-def test_checkpoint_sources_agree(cuda_lib, tuning, T):
-    """d = 64: the chunk-start checkpoints from the forward stage kernel's state-only chain (the
-    default) and from the backward kernel's own forward sweep (dual_bwd_checkpoints 1) both give
+def test_backward_forms_agree(cuda_lib, tuning, T):
+    """d = 64: the stage form (the default), the one-kernel form with its own forward sweep
+    (dual_bwd_form 1) and the reverse sweep on the stage kernel's chunk checkpoints (2) all give
     the oracle's gradients, full and partial 128-token stages included."""
     x = make(2, 2, T, 64, seed=T + 5)
     a = run(x)
     check(x, a)
-    tuning("dual_bwd_checkpoints", 1)
-    b = run(x)
-    check(x, b)
-    for g, r in zip(a, b):
-        assert max_rel_l2(g, r, 2) < 5e-3
+    for form in (1, 2):
+        tuning("dual_bwd_form", form)
+        b = run(x)
+        check(x, b)
+        for g, r in zip(a, b):
+            assert max_rel_l2(g, r, 2) < 5e-3
     assert ttt.read_device_error() == 0

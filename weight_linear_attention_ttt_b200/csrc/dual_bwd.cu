@@ -28,6 +28,8 @@
 // bf16 once per chunk for the tensor cores.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include <string>
 #include <type_traits>
 
@@ -531,7 +533,8 @@ bool dual_bwd_supported(int d, int C, int dt) {
 }
 
 size_t dual_bwd_workspace_bytes(int B, int H, int T, int d) {
-  return (size_t)B * H * (T / BC) * d * d * 2;
+  const size_t chunks = (size_t)B * H * (T / BC) * d * d * 2;   // one checkpoint per chunk
+  return d == 64 ? std::max(chunks, dual_bwd_stage_workspace_bytes(B, H, T)) : chunks;
 }
 
 int launch_dual_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx) {
@@ -553,10 +556,12 @@ int launch_dual_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx) {
   p.T = a.T;
   p.have_ckpt = 0;
   const int streams = a.B * a.H;
-  // d = 64: the chunk-start checkpoints come from the stage kernel's state-only chain (one SM's
-  // four chain warps per stream, no block barriers), which writes them faster than this
-  // kernel's own forward sweep; "dual_bwd_checkpoints" = 1 keeps the in-kernel sweep
-  if (a.d == 64 && tuning(kTuneDualBwdCheckpoints) != 1) {
+  // d = 64: the stage form by default ("dual_bwd_form" 0); with 2 the chunk-start checkpoints
+  // come from the stage kernel's state-only chain (one SM's four chain warps per stream, no block
+  // barriers), which writes them faster than this kernel's own forward sweep (1)
+  const int form = a.d == 64 ? tuning(kTuneDualBwdForm) : 1;
+  if (form == 0) return launch_dual_bwd_stage(a, ctx);
+  if (form == 2) {
     StateArgs f{a.K, a.K, a.V, a.eta, a.eta_scalar, a.S0, nullptr, nullptr, a.B, a.H, a.T, a.d,
                 BC, 1, nullptr, 0};
     const int st = launch_dual_tc_checkpoints(f, p.ckpt, ctx);

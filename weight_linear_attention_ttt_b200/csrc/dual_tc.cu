@@ -107,10 +107,13 @@ __device__ __forceinline__ uint32_t swz_rows(uint32_t row, uint32_t colbyte) {
 
 // SO (state only): the chain alone, for callers that need the final state and no outputs (the
 // segment maps of the sequence-parallel form): no Q loads, no tcgen05 products, no O stores.
-// CK (with SO, 16-column chains, C = 16): every chunk's starting state leaves as a bf16 d x d
-// checkpoint through tmC (the dual-form backward's input): each chain warp stages its 16
-// columns with stmatrix.trans and TMA-stores them.
-template <int NC, int CM, int WC, bool SO, bool CK = false>
+// CK (with SO, 16-column chains, C = 16), the dual-form backward's inputs:
+//   1: every chunk's starting state leaves as a bf16 d x d checkpoint through tmC: each chain
+//      warp stages its 16 columns with stmatrix.trans and TMA-stores them;
+//   2: every stage's starting state W_s leaves the same way (one per 128 tokens), and the
+//      residuals G = K W_c - V of every token leave through tmO as bf16 [T][d] rows (each chain
+//      warp collects its 16 columns of the stage in a [128][16] tile, one TMA store per stage).
+template <int NC, int CM, int WC, bool SO, int CK = 0>
 __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
     dual_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -552,6 +555,27 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
       const uint32_t sW = sbase + Cfg::W_OFF + Cfg::W_BYTES * b;
       const int chunks = min(TR, T - j * TR) / TC;
 
+      if constexpr (CK == 2) {
+        // W_s as W rows (stmatrix.trans of the bf16 W^T fragments), one TMA store per stage
+        const uint32_t wtile = sbase + Cfg::W_OFF + warp * 2048;
+        if (lane == 0) bulk_wait_read<1>();   // the previous stage's W_s store has read it
+        __syncwarp();
+#pragma unroll
+        for (int ks = 0; ks < TKS; ++ks)
+          stsm_x4_t(wtile + (16 * ks + (lane & 7) + 8 * (lane >> 4)) * 32 + ((lane >> 3) & 1) * 16,
+                    pack_bf16(wc[2 * ks][0], wc[2 * ks][1]), pack_bf16(wc[2 * ks][2], wc[2 * ks][3]),
+                    pack_bf16(wc[2 * ks + 1][0], wc[2 * ks + 1][1]),
+                    pack_bf16(wc[2 * ks + 1][2], wc[2 * ks + 1][3]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tmC, wtile, colg, 0, stream * nst + j);
+          bulk_commit();
+          // pending: G of stage j-2 (its tile is rewritten below), W_s of j-1, G of j-1, W_s of j
+          bulk_wait_read<3>();
+        }
+        __syncwarp();
+      }
       // bf16(W_s^T) for the stage's Q W_s product
       if constexpr (!SO) {
 #pragma unroll
@@ -588,7 +612,7 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
           wa[ks][2] = pack_bf16(wc[2 * ks + 1][0], wc[2 * ks + 1][1]);
           wa[ks][3] = pack_bf16(wc[2 * ks + 1][2], wc[2 * ks + 1][3]);
         }
-        if constexpr (CK) {
+        if constexpr (CK == 1) {
           // checkpoint W_c: wa holds this warp's 16 columns of bf16(W) as W^T fragments;
           // stmatrix.trans writes them as W rows into a [64 rows][16 columns] tile (32-byte rows,
           // double-buffered by chunk parity), which one TMA store sends to the checkpoint
@@ -617,11 +641,26 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
         float E[2][4];
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
+          E[n][0] = pa[n][0] + pb[n][0] - bf16_lo(o.vt[2 * n]);   // G^T
+          E[n][1] = pa[n][1] + pb[n][1] - bf16_hi(o.vt[2 * n]);
+          E[n][2] = pa[n][2] + pb[n][2] - bf16_lo(o.vt[2 * n + 1]);
+          E[n][3] = pa[n][3] + pb[n][3] - bf16_hi(o.vt[2 * n + 1]);
+        }
+        if constexpr (CK == 2) {
+          // G rows of chunk c: the G^T fragments, transposed by stmatrix.trans, into rows
+          // 16c .. 16c+15 of this warp's [128 tokens][16 columns] tile of the stage
+          stsm_x4_t(sbase + Cfg::E_OFF + warp * 8192 + (j & 1) * 4096 +
+                        (16 * c + (lane & 7) + 8 * (lane >> 4)) * 32 + ((lane >> 3) & 1) * 16,
+                    pack_bf16(E[0][0], E[0][1]), pack_bf16(E[0][2], E[0][3]),
+                    pack_bf16(E[1][0], E[1][1]), pack_bf16(E[1][2], E[1][3]));
+        }
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
           const float ea0 = n ? o.e8 : o.e0, ea1 = n ? o.e9 : o.e1;
-          E[n][0] = (pa[n][0] + pb[n][0] - bf16_lo(o.vt[2 * n])) * ea0;
-          E[n][1] = (pa[n][1] + pb[n][1] - bf16_hi(o.vt[2 * n])) * ea1;
-          E[n][2] = (pa[n][2] + pb[n][2] - bf16_lo(o.vt[2 * n + 1])) * ea0;
-          E[n][3] = (pa[n][3] + pb[n][3] - bf16_hi(o.vt[2 * n + 1])) * ea1;
+          E[n][0] *= ea0;
+          E[n][1] *= ea1;
+          E[n][2] *= ea0;
+          E[n][3] *= ea1;
         }
         const uint32_t n0 = pack_bf16(E[0][0], E[0][1]) ^ 0x80008000u;
         const uint32_t n1 = pack_bf16(E[0][2], E[0][3]) ^ 0x80008000u;
@@ -731,6 +770,11 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
       if (lane == 0) {
         if (!SO) mbar_arrive(eready + 8 * b);
         mbar_arrive(empty + 8 * s);   // K, V and the rates of the stage are consumed
+        if constexpr (CK == 2) {      // the stage's G rows of this warp's 16 columns
+          tma_store_3d(&tmO, sbase + Cfg::E_OFF + warp * 8192 + (j & 1) * 4096, colg, j * TR,
+                       stream);
+          bulk_commit();
+        }
       }
     }
     if (ok && p.Wout) {
@@ -753,8 +797,9 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
   if (warp == Cfg::MMA) umma::tmem_dealloc(tmem, Cfg::TM_COLS);
 }
 
-template <int NC, int CM, int WC, bool SO, bool CK = false>
-int launch_tc(const StateArgs& a, const LaunchCtx& ctx, uint16_t* ckpt = nullptr) {
+template <int NC, int CM, int WC, bool SO, int CK = 0>
+int launch_tc(const StateArgs& a, const LaunchCtx& ctx, uint16_t* ckpt = nullptr,
+              uint16_t* gbuf = nullptr) {
   using Cfg = TcCfg<NC, WC>;
   const int BH = a.B * a.H;
   CUtensorMap tq, tk, tv, to;
@@ -771,9 +816,14 @@ int launch_tc(const StateArgs& a, const LaunchCtx& ctx, uint16_t* ckpt = nullptr
       !make_tmap_3d(&tv, a.V, bf, dims, strides, box_in, CU_TENSOR_MAP_SWIZZLE_128B, ctx.msg) ||
       !make_tmap_3d(&to, SO ? a.K : a.O, bf, dims, strides, box_out, osw, ctx.msg))
     return kCuda;
+  if (CK == 2) {   // the residual rows G, 16-column boxes of a stage (tmO is unused otherwise)
+    const uint32_t gbox[3] = {16, (uint32_t)TR, 1};
+    if (!make_tmap_3d(&to, gbuf, bf, dims, strides, gbox, CU_TENSOR_MAP_SWIZZLE_NONE, ctx.msg))
+      return kCuda;
+  }
   CUtensorMap tc = tk;   // checkpoint map (CK only)
   if (CK) {
-    const int n = a.T / TC;
+    const int n = CK == 1 ? a.T / TC : (a.T + TR - 1) / TR;
     const uint64_t cdims[3] = {(uint64_t)TD, (uint64_t)TD, (uint64_t)BH * n};
     const uint64_t cstrides[2] = {(uint64_t)TD * 2, (uint64_t)TD * TD * 2};
     const uint32_t cbox[3] = {16, (uint32_t)TD, 1};
@@ -838,7 +888,18 @@ int launch_dual_tc_checkpoints(const StateArgs& a, uint16_t* ckpt, const LaunchC
   }
   StateArgs s = a;
   s.O = nullptr;
-  return launch_tc<4, 1, 16, true, true>(s, ctx, ckpt);
+  return launch_tc<4, 1, 16, true, 1>(s, ctx, ckpt);
+}
+
+int launch_dual_tc_stage_checkpoints(const StateArgs& a, uint16_t* Ws, uint16_t* G,
+                                     const LaunchCtx& ctx) {
+  if (!(dual_tc_supported(a.d, a.C, a.dt) && a.C == TC)) {
+    *ctx.msg = "dual_tc stage checkpoints: bf16, d = 64, C = 16 only";
+    return kUnsupported;
+  }
+  StateArgs s = a;
+  s.O = nullptr;
+  return launch_tc<4, 1, 16, true, 2>(s, ctx, Ws, G);
 }
 
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx) {

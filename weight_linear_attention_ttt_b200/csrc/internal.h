@@ -74,7 +74,7 @@ enum TuneKey : int {
   kTuneInplaceChunksPerLaunch,  // In-Place: 1 = one chunk per launch, 0 / 2 = chunk pairs
   kTuneDualClusterStreams,    // dual form split across SMs: streams per cluster, 1 or 2
   kTuneMomentumForm,          // momentum: 0 = one pass carrying (S, M), 1 = plain + decayed
-  kTuneDualBwdCheckpoints,    // dual backward, d = 64: 0 = stage-kernel checkpoints, 1 = own sweep
+  kTuneDualBwdForm,           // dual backward, d = 64: 0 = stage form, 1 = one kernel, 2 = chunk checkpoints
   kTuneAssocBwdForm,          // associative backward: 0 = fused Y/Z pass, 1 = separate passes
   kTuneCount
 };
@@ -121,6 +121,11 @@ int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx);
 // d, d], the dual-form backward's layout), from the stage kernel's state-only chain (bf16,
 // d = 64, C = 16; S0 = W0, S_out may be null).
 int launch_dual_tc_checkpoints(const StateArgs& a, uint16_t* ckpt, const LaunchCtx& ctx);
+// The same chain writing what the stage-form backward reads: the state at the start of every
+// 128-token stage ([streams, ceil(T / 128), d, d] bf16) and every token's residual
+// G = K W_c - V ([streams, T, d] bf16).
+int launch_dual_tc_stage_checkpoints(const StateArgs& a, uint16_t* Ws, uint16_t* G,
+                                     const LaunchCtx& ctx);
 // True when launch_dual_mma takes O = nullptr for this shape (the stage kernel's state-only
 // form: the final state and no outputs).
 bool dual_state_only_supported(int d, int C, int dt);
@@ -174,6 +179,11 @@ int launch_dual_seg(const StateArgs& a, int S, const LaunchCtx& ctx);
 bool dual_bwd_supported(int d, int C, int dt);
 size_t dual_bwd_workspace_bytes(int B, int H, int T, int d);
 int launch_dual_bwd(const AssocBwdArgs& a, const LaunchCtx& ctx);
+// The stage form (d = 64, C = 16, dual_bwd_tc.cu): the forward's residual rows and stage-start
+// states from the stage kernel's state-only chain (in the workspace), then one kernel with the
+// state gradient's chain on warp MMAs and the stage products on tcgen05.
+size_t dual_bwd_stage_workspace_bytes(int B, int H, int T);
+int launch_dual_bwd_stage(const AssocBwdArgs& a, const LaunchCtx& ctx);
 // Context parallelism of the dual form: a slice's affine maps, and the fold of gathered maps.
 size_t dual_slice_maps_workspace_bytes(int B, int H, int T, int d, int dt);
 int launch_dual_slice_maps(const StateArgs& a, float* A_out, float* B_out, const LaunchCtx& ctx);

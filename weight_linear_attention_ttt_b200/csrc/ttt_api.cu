@@ -37,7 +37,7 @@ static const TuneName kTuneNames[] = {{"dual_column_split", kTuneDualColumnSplit
                                        kTuneInplaceChunksPerLaunch},
                                       {"dual_cluster_streams", kTuneDualClusterStreams},
                                       {"momentum_form", kTuneMomentumForm},
-                                      {"dual_bwd_checkpoints", kTuneDualBwdCheckpoints},
+                                      {"dual_bwd_form", kTuneDualBwdForm},
                                       {"assoc_bwd_form", kTuneAssocBwdForm}};
 static int tune_key(const char* name) {
   if (!name) return -1;
