@@ -132,6 +132,9 @@ def test_backward_forms_agree(cuda_lib, tuning, T):
         tuning("dual_bwd_form", form)
         b = run(x)
         check(x, b)
+        # The forms round different operands to bf16 (the stage form: -diag(eta) G, W_s, dG and
+        # the masked stage scores; the others: G and every chunk-start W), each within the
+        # oracle's 1e-2 bar on its own, so they agree to within that bar, not tighter.
         for g, r in zip(a, b):
-            assert max_rel_l2(g, r, 2) < 5e-3
+            assert max_rel_l2(g, r, 2) < 1e-2
     assert ttt.read_device_error() == 0

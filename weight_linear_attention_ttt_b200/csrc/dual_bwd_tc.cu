@@ -25,28 +25,31 @@
 // P2 carries dG W_c^T's corrections below the chunk diagonal and, transposed, E X_c^T's above it).
 // Only R, dG and the state gradient itself are serial; they stay on the warps.
 //
-// Inputs the forward produced: G of every token and the state at every stage start, written by
-// the forward stage kernel's state-only chain (one launch before this one).
+// Inputs the forward produced: G and -E of every token and the state at every stage start,
+// written by the forward stage kernel's state-only chain (one launch before this one). With -E as
+// the tensor operand the scores come out scaled and negated: P1 = mask(dO (-E)^T),
+// P2 = mask(dG (-E)^T), and -diag(eta) G X_e^T = (-E) X_e^T accumulates into dK directly.
 //
 // Roles (320 threads):
-//   * warp 0: TMA producer, a 2-slot ring of one stage each: Q, K, dO, G [128][64] (128-byte
-//     swizzle), W_s [64][64], the rates; the next stage's rows are prefetched into L2.
-//   * warp 1: owns TMEM, issues every tcgen05.mma (elected lane): S1 = dO G^T, dQ, the P1 part of
-//     dK and G X_e^T as soon as the stage's P1 is masked; S2 = dG G^T and the rest of dK once the
-//     chain has finished the stage.
+//   * warp 0: TMA producer, a 2-slot ring of one stage each: Q, K, dO, -E [128][64] (128-byte
+//     swizzle), W_s [64][64], the rates.
+//   * warp 1: owns TMEM, issues every tcgen05.mma (elected lane): S1 = dO (-E)^T, dQ, the P1
+//     and X_e parts of dK as soon as the stage's P1 is masked; S2 = dG (-E)^T and the rest of dK
+//     once the chain has finished the stage.
 //   * warps 2-5 (one TMEM lane quarter each): mask S1 into P1 and S2 into P2 (bf16, shared
-//     memory, read K-major for P K and MN-major for P^T Q / P^T K), drain dQ and
-//     dK - eta G X_e^T through a shared tile to TMA stores, write deta.
+//     memory, read K-major for P K and MN-major for P^T Q / P^T K), drain dQ and dK through a
+//     shared tile to TMA stores, write deta.
 //   * warps 6-9, the chain: each keeps X^T[16 columns, 64] as fp32 m16n8 accumulators (the state
 //     gradient's columns are independent) and per chunk, from the last, forms A'^T = K Q^T,
 //     R^T = dO^T A' + X^T K^T, dG^T, the chunk's deta partial sums, X^T += dG^T K + dO^T Q;
 //     stores dG^T (the MN-major A operand of the stage's products), dV and, at each stage
-//     start, bf16(X_e^T).
-// TMEM columns: S1 [0, 128), S2 [128, 256), dQ [256, 320), dK [320, 384), G X_e^T [384, 448).
+//     start, bf16(X_e^T). The next chunk's fragments are loaded before this chunk's stores.
+// TMEM columns: S1 [0, 128), S2 [128, 256), dQ [256, 320), dK [320, 384).
 // Precision: X and every accumulation fp32; W_s, G, X_e, dG and the masked scores are bf16 tensor
 // operands (relative error ~2^-9 per operand).
 #include <algorithm>
 #include <string>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -62,7 +65,7 @@ constexpr int BKS = BD / 16;           // 16-wide k-steps over d
 constexpr int TILE = BR * BD * 2;      // [128][64] bf16
 constexpr int WTILE = BD * BD * 2;     // [64][64] bf16
 // one ring slot
-constexpr int SL_Q = 0, SL_K = TILE, SL_DO = 2 * TILE, SL_G = 3 * TILE, SL_W = 4 * TILE;
+constexpr int SL_Q = 0, SL_K = TILE, SL_DO = 2 * TILE, SL_NE = 3 * TILE, SL_W = 4 * TILE;
 constexpr int SL_ETA = SL_W + WTILE;   // 128 fp32 rates
 constexpr int SL_DETA = SL_ETA + 512;  // [4 chain warps][128] fp32 deta partial sums
 constexpr int SLOT = (SL_DETA + 4 * 512 + 1023) / 1024 * 1024;
@@ -73,8 +76,9 @@ constexpr int XE_OFF = DG_OFF + 2 * DG_BYTES;   // bf16 X_e^T [64][64]
 constexpr int BAR_OFF = XE_OFF + WTILE;
 constexpr int SMEM = 1024 + BAR_OFF + 256;
 constexpr int THREADS = 320;
+constexpr float kTinyRate = 1e-20f;   // below it deta is formed from G, not from -E / eta
 constexpr int PRODUCER = 0, MMA = 1, EPI0 = 2, CHAIN0 = 6;
-constexpr uint32_t TM_S1 = 0, TM_S2 = 128, TM_DQ = 256, TM_DK = 320, TM_GX = 384, TM_COLS = 512;
+constexpr uint32_t TM_S1 = 0, TM_S2 = 128, TM_DQ = 256, TM_DK = 320, TM_COLS = 512;
 static_assert(SLOT % 1024 == 0 && P_OFF % 1024 == 0 && DG_OFF % 1024 == 0 &&
                   XE_OFF % 1024 == 0, "1024-byte aligned operand tiles");
 static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -83,6 +87,7 @@ struct DbtParams {
   const float* eta;     // [streams, T] or nullptr (eta_scalar)
   float eta_scalar;
   const float* dW_out;  // [streams, 64, 64] or nullptr
+  const uint16_t* G;    // [streams, T, 64] bf16 residual rows of the forward
   float* dW0;
   float* deta;
   uint16_t* dV;
@@ -104,7 +109,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     dual_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmdO,
-                       const __grid_constant__ CUtensorMap tmG,
+                       const __grid_constant__ CUtensorMap tmNE,
                        const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmdQ,
                        const __grid_constant__ CUtensorMap tmdK, const DbtParams p) {
@@ -120,10 +125,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t dqfree = bar + 56;   // dQ read out of TMEM (4 epilogue warps)
   const uint32_t s2full = bar + 64;   // S2 accumulated (MMA commit)
   const uint32_t p2full = bar + 72;   // P2 written, S2 read (4 epilogue warps)
-  const uint32_t dkfull = bar + 80;   // dK and G X_e^T complete (MMA commit)
-  const uint32_t dkfree = bar + 88;   // dK and G X_e^T read out (4 epilogue warps)
+  const uint32_t dkfull = bar + 80;   // dK complete (MMA commit)
+  const uint32_t dkfree = bar + 88;   // dK read out (4 epilogue warps)
   const uint32_t xeready = bar + 96;  // bf16 X_e^T stored (4 chain warps)
-  const uint32_t xefree = bar + 104;  // G X_e^T has read it (MMA commit)
+  const uint32_t xefree = bar + 104;  // (-E) X_e^T has read it (MMA commit)
   const uint32_t cdone = bar + 112;   // the chain finished a stage: dG^T and deta sums (x2)
   const uint32_t dgfree = bar + 128;  // the stage's products have read dG^T buffer b (x2)
   const uint32_t mdone = bar + 144;   // every MMA issued has completed
@@ -175,7 +180,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmdO);
-      prefetch_tmap(&tmG);
+      prefetch_tmap(&tmNE);
       prefetch_tmap(&tmW);
       int issued = 0;
       for (int i = 0; i < nst; ++i) {
@@ -192,7 +197,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_3d(st + SL_Q, &tmQ, fb, 0, j * BR, stream);
         tma_load_3d(st + SL_K, &tmK, fb, 0, j * BR, stream);
         tma_load_3d(st + SL_DO, &tmdO, fb, 0, j * BR, stream);
-        tma_load_3d(st + SL_G, &tmG, fb, 0, j * BR, stream);
+        tma_load_3d(st + SL_NE, &tmNE, fb, 0, j * BR, stream);
         tma_load_3d(st + SL_W, &tmW, fb, 0, 0, stream * nst + j);
         if (p.eta)
           bulk_load(st + SL_ETA, p.eta + (size_t)stream * T + (size_t)j * BR, rows * 4, fb);
@@ -205,24 +210,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == MMA) {
     // ------------------------------------------------------------------ tcgen05 issue warp
     // The whole warp runs the loop (warp-uniform waits); an elected lane issues.
-    const uint32_t id_s1 = umma::idesc_bf16(128, 128, false, false);   // dO G^T
-    const uint32_t id_kk = umma::idesc_bf16(128, 64, false, false);    // dO W_s^T, G X.. (K, K)
-    const uint32_t id_kn = umma::idesc_bf16(128, 64, false, true);     // P K, G X_e^T
+    const uint32_t id_s1 = umma::idesc_bf16(128, 128, false, false);   // dO (-E)^T
+    const uint32_t id_kk = umma::idesc_bf16(128, 64, false, false);    // dO W_s^T
+    const uint32_t id_kn = umma::idesc_bf16(128, 64, false, true);     // P K, (-E) X_e^T
     const uint32_t id_nn = umma::idesc_bf16(128, 64, true, true);      // P^T Q, P^T K
-    const uint32_t id_s2 = umma::idesc_bf16(128, 128, true, false);    // dG G^T
+    const uint32_t id_s2 = umma::idesc_bf16(128, 128, true, false);    // dG (-E)^T
     const uint32_t id_nk = umma::idesc_bf16(128, 64, true, false);     // dG W_s^T
     const uint32_t sP = sbase + P_OFF;
     auto slot = [&](int i) -> uint32_t { return sbase + (i & 1) * SLOT; };
-    // S1 = dO G^T of stage i
+    // S1 = dO (-E)^T of stage i
     auto issue_s1 = [&](int i) {
       const uint32_t st = slot(i);
 #pragma unroll
       for (int ks = 0; ks < BKS; ++ks)
         umma::mma_ss_elect(tmem + TM_S1, umma::desc_kmajor(st + SL_DO + 32 * ks),
-                           umma::desc_kmajor(st + SL_G + 32 * ks), id_s1, ks > 0);
+                           umma::desc_kmajor(st + SL_NE + 32 * ks), id_s1, ks > 0);
       umma::commit_elect(s1full);
     };
-    // dQ = dO W_s^T + P1 K; dK = P1^T Q; G X_e^T
+    // dQ = dO W_s^T + P1 K; dK = P1^T Q + (-E) X_e^T
     auto early = [&](int i) -> bool {
       const uint32_t st = slot(i);
       if (!mbar_wait_warp(p1full, i & 1, p.err, p.wait_ns)) return false;
@@ -247,12 +252,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       umma::fence_after();
 #pragma unroll
       for (int ks = 0; ks < BKS; ++ks)
-        umma::mma_ss_elect(tmem + TM_GX, umma::desc_kmajor(st + SL_G + 32 * ks),
-                           umma::desc_mnmajor(sbase + XE_OFF + 2048 * ks, WTILE), id_kn, ks > 0);
+        umma::mma_ss_elect(tmem + TM_DK, umma::desc_kmajor(st + SL_NE + 32 * ks),
+                           umma::desc_mnmajor(sbase + XE_OFF + 2048 * ks, WTILE), id_kn, true);
       umma::commit_elect(xefree);
       return true;
     };
-    // S2 = dG G^T; dK += dG W_s^T + P2 K + P2^T K
+    // S2 = dG (-E)^T; dK += dG W_s^T + P2 K + P2^T K
     auto late = [&](int i) -> bool {
       const uint32_t st = slot(i);
       const int b = i & 1;
@@ -262,7 +267,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
       for (int ks = 0; ks < BKS; ++ks)
         umma::mma_ss_elect(tmem + TM_S2, umma::desc_mnmajor(sDG + 2048 * ks, DG_BYTES / 2),
-                           umma::desc_kmajor(st + SL_G + 32 * ks), id_s2, ks > 0);
+                           umma::desc_kmajor(st + SL_NE + 32 * ks), id_s2, ks > 0);
       umma::commit_elect(s2full);
 #pragma unroll
       for (int ks = 0; ks < BKS; ++ks)
@@ -283,6 +288,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       umma::commit_elect(dgfree + 8 * b);
       return true;
     };
+    // Order per iteration: S1 of stage i as soon as its tiles land, then the late products of
+    // stage i-1, then the early products of stage i. (Issuing the late products first overlaps
+    // more of the pipeline with the chain and measured slower, 0.133 against 0.128 ms: the
+    // chain's warp MMAs and shared-memory loads share the SM with the products.)
     bool ok = true;
     for (int i = 0; ok && i < nst; ++i) {
       if (!mbar_wait_warp(full + 8 * (i & 1), (i >> 1) & 1, p.err, p.wait_ns)) break;
@@ -304,45 +313,48 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tl = (uint32_t)(32 * q) << 16;
     const int etid = threadIdx.x - 32 * EPI0;  // 0..127
     const uint32_t sP = sbase + P_OFF;
-    // P[r][:] from the fp32 scores in TMEM columns col0 .. col0+127: P = -eta_col S where
-    // keep(col), else 0; bf16 into the two [128][64] blocks of the P tile. Column halves that are
-    // masked out for all 32 rows of the warp are not loaded.
-    auto mask_rows = [&](uint32_t col0, uint32_t sEta, auto keep, auto live) {
+    // Both masks keep a 32-column group [c0, c0+32) for every row of this warp when c0 < 32q,
+    // for none when c0 > 32q, and row by row in the group c0 = 32q (keep(col) decides there):
+    // the query mask s <= t of P1 and the chunk mask chunk(t) < chunk(s) of P2 alike.
+    auto group_mode = [&](int c0) { return c0 < 32 * q ? 1 : (c0 == 32 * q ? 2 : 0); };
+    // P[r][:] = S[r][col] where kept, else 0, from the fp32 scores in TMEM columns
+    // col0 .. col0+127 (already scaled and negated by the -E operand), as bf16 into the two
+    // [128][64] blocks of the P tile. Groups masked for every row are not loaded.
+    auto mask_rows = [&](uint32_t col0, auto keep) {
 #pragma unroll
       for (int kb = 0; kb < 2; ++kb) {
+        const int m0 = group_mode(64 * kb), m1 = group_mode(64 * kb + 32);   // warp-uniform
         uint32_t v[2][32];
+        if (m0 != 0) umma::ld32x32(tmem + tl + col0 + 64 * kb, v[0]);
+        if (m1 != 0) umma::ld32x32(tmem + tl + col0 + 64 * kb + 32, v[1]);
+        if (m0 != 0) {
+          umma::wait_ld();
+          umma::reg_fence(v[0]);
+          umma::reg_fence(v[1]);
+        }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          if (live(64 * kb + 32 * h)) {
-            umma::ld32x32(tmem + tl + col0 + 64 * kb + 32 * h, v[h]);
-          } else {
+          const int m = h ? m1 : m0;
 #pragma unroll
-            for (int x = 0; x < 32; ++x) v[h][x] = 0u;
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int x0 = 32 * h + 8 * k4;   // column within the block
+            uint4 out = make_uint4(0u, 0u, 0u, 0u);
+            if (m != 0) {
+              uint32_t w[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                float a0 = __uint_as_float(v[h][8 * k4 + 2 * u]);
+                float a1 = __uint_as_float(v[h][8 * k4 + 2 * u + 1]);
+                if (m == 2) {
+                  if (!keep(64 * kb + x0 + 2 * u)) a0 = 0.f;
+                  if (!keep(64 * kb + x0 + 2 * u + 1)) a1 = 0.f;
+                }
+                w[u] = pack_bf16(a0, a1);
+              }
+              out = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            sts128(sP + kb * TILE + swz128(r, 16 * (4 * h + k4)), out);
           }
-        }
-        umma::wait_ld();
-        umma::reg_fence(v[0]);
-        umma::reg_fence(v[1]);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int c0 = 64 * kb + 8 * k;   // first column of this 16-byte piece
-          const uint4 ea = lds128(sEta + 4 * c0), eb = lds128(sEta + 4 * c0 + 16);
-          const float e[8] = {__uint_as_float(ea.x), __uint_as_float(ea.y),
-                              __uint_as_float(ea.z), __uint_as_float(ea.w),
-                              __uint_as_float(eb.x), __uint_as_float(eb.y),
-                              __uint_as_float(eb.z), __uint_as_float(eb.w)};
-          uint32_t w[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int x0 = 8 * k + 2 * u;   // index within the 64 columns of block kb
-            const float a0 = keep(c0 + 2 * u) ? -e[2 * u] * __uint_as_float(v[x0 >> 5][x0 & 31])
-                                              : 0.f;
-            const float a1 = keep(c0 + 2 * u + 1)
-                                 ? -e[2 * u + 1] * __uint_as_float(v[(x0 + 1) >> 5][(x0 + 1) & 31])
-                                 : 0.f;
-            w[u] = pack_bf16(a0, a1);
-          }
-          sts128(sP + kb * TILE + swz128(r, 16 * k), make_uint4(w[0], w[1], w[2], w[3]));
         }
       }
       fence_proxy_async_smem();
@@ -378,13 +390,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; i < nst; ++i) {
       const int j = nst - 1 - i, b = i & 1;
       const uint32_t st = sbase + (i & 1) * SLOT;
-      // P1 = -[s <= t] eta_s (dO G^T)[t][s]; the staging tile's last store must have read P
+      // P1 = [s <= t] (dO (-E)^T)[t][s]; the staging tile's last store must have read P
       bool got = mbar_wait_warp(s1full, i & 1, p.err, p.wait_ns);
       if (got && etid == 0) bulk_wait_read<0>();
       if (bar_or_named(1, 128, !got)) break;
       umma::fence_after();
-      mask_rows(TM_S1, st + SL_ETA, [&](int s) { return s <= r; },
-                [&](int c0) { return c0 <= 32 * q + 31; });
+      mask_rows(TM_S1, [&](int s) { return s <= r; });
       if (lane == 0) mbar_arrive(p1full);
       // dQ
       got = mbar_wait_warp(dqfull, i & 1, p.err, p.wait_ns);
@@ -398,38 +409,31 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) mbar_arrive(dqfree);
         stage_out(v, &tmdQ, j);
       }
-      // P2 = -[chunk(t) < chunk(s)] eta_t (dG G^T)[s][t]
+      // P2 = [chunk(t) < chunk(s)] (dG (-E)^T)[s][t]
       got = mbar_wait_warp(s2full, i & 1, p.err, p.wait_ns);
       if (got) got = mbar_wait_warp(cdone + 8 * b, (i >> 1) & 1, p.err, p.wait_ns);
       if (got && etid == 0) bulk_wait_read<0>();
       if (bar_or_named(1, 128, !got)) break;
       umma::fence_after();
-      mask_rows(TM_S2, st + SL_ETA, [&](int t) { return (t >> 4) < (r >> 4); },
-                [&](int c0) { return c0 < 32 * q + 16; });
+      mask_rows(TM_S2, [&](int t) { return (t >> 4) < (r >> 4); });
       if (lane == 0) mbar_arrive(p2full);
-      // deta of the stage (the four chain warps' partial sums, in a fixed order) and this
-      // row's rate
-      const float eta_r = ldsf(st + SL_ETA + 4 * r);
+      // deta of the stage (the four chain warps' partial sums, in a fixed order)
       if (j * BR + r < T)
         p.deta[(size_t)stream * T + (size_t)j * BR + r] =
             ((ldsf(st + SL_DETA + 4 * r) + ldsf(st + SL_DETA + 512 + 4 * r)) +
              ldsf(st + SL_DETA + 1024 + 4 * r)) + ldsf(st + SL_DETA + 1536 + 4 * r);
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + 8 * (i & 1));
-      // dK - eta G X_e^T
+      // dK
       got = mbar_wait_warp(dkfull, i & 1, p.err, p.wait_ns);
       if (bar_or_named(1, 128, !got)) break;
       umma::fence_after();
       {
-        uint32_t v[64], gx[64];
+        uint32_t v[64];
         load64(TM_DK, v);
-        load64(TM_GX, gx);
         umma::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dkfree);
-#pragma unroll
-        for (int x = 0; x < 64; ++x)
-          v[x] = __float_as_uint(__uint_as_float(v[x]) - eta_r * __uint_as_float(gx[x]));
         stage_out(v, &tmdK, j);
       }
     }
@@ -442,8 +446,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int colw = 16 * cw;                  // this warp's 16 columns of X (and of dG, dV)
     // Fragment offsets in the [128][64] tiles (128-byte swizzle), relative to a chunk's rows:
     // rows as the B operand of (.) x^T (K and Q), via ldmatrix.trans as the B operand of the
-    // state update (K and Q), and via ldmatrix.trans this warp's 16 columns as an A operand
-    // (dO^T and G^T).
+    // state update (K and Q), and via ldmatrix.trans this warp's 16 columns as an A operand (dO^T
+    // and (-E)^T). (Transposing the row fragments in registers with movmatrix instead of the
+    // second ldmatrix pass measured slower: 159 against 129 us per call.)
     uint32_t o_brow[BKS], o_btrn[BKS];
 #pragma unroll
     for (int ks = 0; ks < BKS; ++ks) {
@@ -475,7 +480,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; i < nst; ++i) {
       const int j = nst - 1 - i, b = i & 1;
       const uint32_t st = sbase + (i & 1) * SLOT;
-      const uint32_t sQ = st + SL_Q, sK = st + SL_K, sdO = st + SL_DO, sG = st + SL_G;
+      const uint32_t sQ = st + SL_Q, sK = st + SL_K, sdO = st + SL_DO;
       const uint32_t sEta = st + SL_ETA, sDeta = st + SL_DETA;
       const uint32_t sDG = sbase + DG_OFF + b * DG_BYTES;
       bool got = mbar_wait_warp(full + 8 * (i & 1), (i >> 1) & 1, p.err, p.wait_ns);
@@ -501,32 +506,60 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       const int chunks = min(BR, T - j * BR) / BC;
       uint16_t* dv = p.dV + ((size_t)stream * T + (size_t)j * BR) * BD;
-      auto chunk = [&](const int c) {
+      const uint16_t* gst = p.G + ((size_t)stream * T + (size_t)j * BR) * BD + colw + g;
+      const uint32_t sNE = st + SL_NE;
+      struct Ops {
+        uint32_t kb[BKS][4], qb[BKS][4], kt[BKS][4], qt[BKS][4], dot[4], ne[4];
+        float e0, e1, e8, e9;
+      };
+      auto load = [&](Ops& o, const int c) {
         const uint32_t cb = c * CHUNK_BYTES;
-        uint32_t kb[BKS][4], qb[BKS][4], kt[BKS][4], qt[BKS][4], dot[4], gt[4];
 #pragma unroll
         for (int ks = 0; ks < BKS; ++ks) {
-          ldsm_x4(sK + cb + o_brow[ks], kb[ks]);
-          ldsm_x4(sQ + cb + o_brow[ks], qb[ks]);
+          ldsm_x4(sK + cb + o_brow[ks], o.kb[ks]);
+          ldsm_x4(sQ + cb + o_brow[ks], o.qb[ks]);
         }
-        ldsm_x4_t(sdO + cb + o_at, dot);
-        ldsm_x4_t(sG + cb + o_at, gt);
+        ldsm_x4_t(sdO + cb + o_at, o.dot);
+        ldsm_x4_t(sNE + cb + o_at, o.ne);
 #pragma unroll
         for (int ks = 0; ks < BKS; ++ks) {
-          ldsm_x4_t(sK + cb + o_btrn[ks], kt[ks]);
-          ldsm_x4_t(sQ + cb + o_btrn[ks], qt[ks]);
+          ldsm_x4_t(sK + cb + o_btrn[ks], o.kt[ks]);
+          ldsm_x4_t(sQ + cb + o_btrn[ks], o.qt[ks]);
         }
-        const float e0 = ldsf(sEta + 4 * (16 * c + 2 * tq));
-        const float e1 = ldsf(sEta + 4 * (16 * c + 2 * tq + 1));
-        const float e8 = ldsf(sEta + 4 * (16 * c + 8 + 2 * tq));
-        const float e9 = ldsf(sEta + 4 * (16 * c + 9 + 2 * tq));
-        // A'^T = K Q^T (rows: keys s, columns: queries t), kept where s <= t. The K rows loaded as
-        // B fragments are the A fragments of K in another register order.
+        o.e0 = ldsf(sEta + 4 * (16 * c + 2 * tq));
+        o.e1 = ldsf(sEta + 4 * (16 * c + 2 * tq + 1));
+        o.e8 = ldsf(sEta + 4 * (16 * c + 8 + 2 * tq));
+        o.e9 = ldsf(sEta + 4 * (16 * c + 9 + 2 * tq));
+      };
+      // G[s][j] of chunk c at the R^T fragment's positions (j = colw + g (+8), s = 16c + 2tq
+      // (+1) (+8)) as raw bf16 bits, for chunks with a rate too small to divide by
+      auto load_g = [&](uint32_t (&gq)[8], const int c) {
+        const uint16_t* gp = gst + (size_t)(16 * c + 2 * tq) * BD;
+        gq[0] = __ldg(gp);
+        gq[1] = __ldg(gp + BD);
+        gq[2] = __ldg(gp + 8);
+        gq[3] = __ldg(gp + BD + 8);
+        gq[4] = __ldg(gp + 8 * BD);
+        gq[5] = __ldg(gp + 9 * BD);
+        gq[6] = __ldg(gp + 8 * BD + 8);
+        gq[7] = __ldg(gp + 9 * BD + 8);
+      };
+      auto gval = [](uint32_t x) { return __uint_as_float(x << 16); };
+      struct Res {
+        uint32_t n[4];   // bf16 dG^T fragments
+        float d[4];      // deta partial sums of s = 2tq, 2tq+1, 8+2tq, 9+2tq (lanes g = 0)
+      };
+      // slow_c: the stage holds a rate too small to divide by (see deta below)
+      auto compute = [&](const Ops& o, const int c, Res& res, auto slow_c) {
+        // A'^T = K Q^T (rows: keys s, columns: queries t), kept where s <= t. The K rows loaded
+        // as B fragments are the A fragments of K in another register order.
         float at[2][4] = {};
 #pragma unroll
         for (int ks = 0; ks < BKS; ++ks) {
-          mma16816(at[0], kb[ks][0], kb[ks][2], kb[ks][1], kb[ks][3], qb[ks][0], qb[ks][1]);
-          mma16816(at[1], kb[ks][0], kb[ks][2], kb[ks][1], kb[ks][3], qb[ks][2], qb[ks][3]);
+          mma16816(at[0], o.kb[ks][0], o.kb[ks][2], o.kb[ks][1], o.kb[ks][3], o.qb[ks][0],
+                   o.qb[ks][1]);
+          mma16816(at[1], o.kb[ks][0], o.kb[ks][2], o.kb[ks][1], o.kb[ks][3], o.qb[ks][2],
+                   o.qb[ks][3]);
         }
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -541,8 +574,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t ba1[2] = {pack_bf16(at[0][2], at[0][3]), pack_bf16(at[1][2], at[1][3])};
         // R^T = dO^T A' + X^T K^T (two accumulators halve the dependent chain)
         float ra[2][4] = {}, rb[2][4] = {};
-        mma16816(ra[0], dot[0], dot[1], dot[2], dot[3], ba0[0], ba0[1]);
-        mma16816(ra[1], dot[0], dot[1], dot[2], dot[3], ba1[0], ba1[1]);
+        mma16816(ra[0], o.dot[0], o.dot[1], o.dot[2], o.dot[3], ba0[0], ba0[1]);
+        mma16816(ra[1], o.dot[0], o.dot[1], o.dot[2], o.dot[3], ba1[0], ba1[1]);
 #pragma unroll
         for (int ks = 0; ks < BKS; ++ks) {
           const uint32_t a0 = pack_bf16(xc[2 * ks][0], xc[2 * ks][1]);
@@ -550,13 +583,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t a2 = pack_bf16(xc[2 * ks + 1][0], xc[2 * ks + 1][1]);
           const uint32_t a3 = pack_bf16(xc[2 * ks + 1][2], xc[2 * ks + 1][3]);
           float (&acc)[2][4] = (ks & 1) ? rb : ra;
-          mma16816(acc[0], a0, a1, a2, a3, kb[ks][0], kb[ks][1]);
-          mma16816(acc[1], a0, a1, a2, a3, kb[ks][2], kb[ks][3]);
+          mma16816(acc[0], a0, a1, a2, a3, o.kb[ks][0], o.kb[ks][1]);
+          mma16816(acc[1], a0, a1, a2, a3, o.kb[ks][2], o.kb[ks][3]);
         }
         float R[2][4], dg[2][4];
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
-          const float ea0 = n ? e8 : e0, ea1 = n ? e9 : e1;
+          const float ea0 = n ? o.e8 : o.e0, ea1 = n ? o.e9 : o.e1;
 #pragma unroll
           for (int x = 0; x < 4; ++x) R[n][x] = ra[n][x] + rb[n][x];
           dg[n][0] = -ea0 * R[n][0];
@@ -564,53 +597,107 @@ __global__ void __launch_bounds__(THREADS, 1)
           dg[n][2] = -ea0 * R[n][2];
           dg[n][3] = -ea1 * R[n][3];
         }
-        // deta_s = -G_s . R_s over this warp's 16 columns (the epilogue adds the four warps')
-        {
-          float d0 = bf16_lo(gt[0]) * R[0][0] + bf16_lo(gt[1]) * R[0][2];
-          float d1 = bf16_hi(gt[0]) * R[0][1] + bf16_hi(gt[1]) * R[0][3];
-          float d2 = bf16_lo(gt[2]) * R[1][0] + bf16_lo(gt[3]) * R[1][2];
-          float d3 = bf16_hi(gt[2]) * R[1][1] + bf16_hi(gt[3]) * R[1][3];
-#pragma unroll
-          for (int m = 4; m < 32; m <<= 1) {
-            d0 += __shfl_xor_sync(0xffffffffu, d0, m);
-            d1 += __shfl_xor_sync(0xffffffffu, d1, m);
-            d2 += __shfl_xor_sync(0xffffffffu, d2, m);
-            d3 += __shfl_xor_sync(0xffffffffu, d3, m);
-          }
-          if (g == 0) {
-            const uint32_t dd = sDeta + cw * 512 + 4 * 16 * c;
-            stsf(dd + 4 * (2 * tq), -d0);
-            stsf(dd + 4 * (2 * tq + 1), -d1);
-            stsf(dd + 4 * (8 + 2 * tq), -d2);
-            stsf(dd + 4 * (9 + 2 * tq), -d3);
-          }
-        }
-        const uint32_t n0 = pack_bf16(dg[0][0], dg[0][1]), n1 = pack_bf16(dg[0][2], dg[0][3]);
-        const uint32_t n2 = pack_bf16(dg[1][0], dg[1][1]), n3 = pack_bf16(dg[1][2], dg[1][3]);
+        res.n[0] = pack_bf16(dg[0][0], dg[0][1]);
+        res.n[1] = pack_bf16(dg[0][2], dg[0][3]);
+        res.n[2] = pack_bf16(dg[1][0], dg[1][1]);
+        res.n[3] = pack_bf16(dg[1][2], dg[1][3]);
         // X^T += dG^T K + dO^T Q
 #pragma unroll
         for (int jp = 0; jp < BKS; ++jp) {
-          mma16816(xc[2 * jp], n0, n1, n2, n3, kt[jp][0], kt[jp][1]);
-          mma16816(xc[2 * jp + 1], n0, n1, n2, n3, kt[jp][2], kt[jp][3]);
-          mma16816(xc[2 * jp], dot[0], dot[1], dot[2], dot[3], qt[jp][0], qt[jp][1]);
-          mma16816(xc[2 * jp + 1], dot[0], dot[1], dot[2], dot[3], qt[jp][2], qt[jp][3]);
+          mma16816(xc[2 * jp], res.n[0], res.n[1], res.n[2], res.n[3], o.kt[jp][0], o.kt[jp][1]);
+          mma16816(xc[2 * jp + 1], res.n[0], res.n[1], res.n[2], res.n[3], o.kt[jp][2],
+                   o.kt[jp][3]);
+          mma16816(xc[2 * jp], o.dot[0], o.dot[1], o.dot[2], o.dot[3], o.qt[jp][0], o.qt[jp][1]);
+          mma16816(xc[2 * jp + 1], o.dot[0], o.dot[1], o.dot[2], o.dot[3], o.qt[jp][2],
+                   o.qt[jp][3]);
         }
+        // deta_s = -G_s . R_s over this warp's 16 columns (the epilogue adds the four warps'):
+        // with the -E = -diag(eta) G fragments this is (-E_s . R_s) / eta_s. A stage holding a
+        // rate too small to divide by takes G itself from global memory for those tokens.
+        float d0 = bf16_lo(o.ne[0]) * R[0][0] + bf16_lo(o.ne[1]) * R[0][2];
+        float d1 = bf16_hi(o.ne[0]) * R[0][1] + bf16_hi(o.ne[1]) * R[0][3];
+        float d2 = bf16_lo(o.ne[2]) * R[1][0] + bf16_lo(o.ne[3]) * R[1][2];
+        float d3 = bf16_hi(o.ne[2]) * R[1][1] + bf16_hi(o.ne[3]) * R[1][3];
+#pragma unroll
+        for (int m = 4; m < 32; m <<= 1) {
+          d0 += __shfl_xor_sync(0xffffffffu, d0, m);
+          d1 += __shfl_xor_sync(0xffffffffu, d1, m);
+          d2 += __shfl_xor_sync(0xffffffffu, d2, m);
+          d3 += __shfl_xor_sync(0xffffffffu, d3, m);
+        }
+        res.d[0] = __fdividef(d0, o.e0);
+        res.d[1] = __fdividef(d1, o.e1);
+        res.d[2] = __fdividef(d2, o.e8);
+        res.d[3] = __fdividef(d3, o.e9);
+        if constexpr (decltype(slow_c)::value) {
+          uint32_t gq[8];
+          load_g(gq, c);
+          float g0 = gval(gq[0]) * R[0][0] + gval(gq[2]) * R[0][2];
+          float g1 = gval(gq[1]) * R[0][1] + gval(gq[3]) * R[0][3];
+          float g2 = gval(gq[4]) * R[1][0] + gval(gq[6]) * R[1][2];
+          float g3 = gval(gq[5]) * R[1][1] + gval(gq[7]) * R[1][3];
+#pragma unroll
+          for (int m = 4; m < 32; m <<= 1) {
+            g0 += __shfl_xor_sync(0xffffffffu, g0, m);
+            g1 += __shfl_xor_sync(0xffffffffu, g1, m);
+            g2 += __shfl_xor_sync(0xffffffffu, g2, m);
+            g3 += __shfl_xor_sync(0xffffffffu, g3, m);
+          }
+          if (fabsf(o.e0) < kTinyRate) res.d[0] = -g0;
+          if (fabsf(o.e1) < kTinyRate) res.d[1] = -g1;
+          if (fabsf(o.e8) < kTinyRate) res.d[2] = -g2;
+          if (fabsf(o.e9) < kTinyRate) res.d[3] = -g3;
+        }
+      };
+      auto store = [&](const Res& res, const int c) {
         // dG^T of chunk c: tokens 16c .. 16c+15 of the stage's [2][64][64] buffer
-        stsm_x4(sDG + (c >> 2) * (DG_BYTES / 2) + swz128(srow, 2 * (16 * (c & 3) + scol)), n0, n1,
-                n2, n3);
+        stsm_x4(sDG + (c >> 2) * (DG_BYTES / 2) + swz128(srow, 2 * (16 * (c & 3) + scol)),
+                res.n[0], res.n[1], res.n[2], res.n[3]);
+        if (g == 0) {
+          const uint32_t dd = sDeta + cw * 512 + 4 * 16 * c;
+          stsf(dd + 4 * (2 * tq), res.d[0]);
+          stsf(dd + 4 * (2 * tq + 1), res.d[1]);
+          stsf(dd + 4 * (8 + 2 * tq), res.d[2]);
+          stsf(dd + 4 * (9 + 2 * tq), res.d[3]);
+        }
         // dV = -dG: each 8x8 block transposed in registers into dV rows
         uint16_t* d = dv + (size_t)(16 * c + g) * BD + colw + 2 * tq;
-        *reinterpret_cast<uint32_t*>(d) = movm_t(n0) ^ 0x80008000u;
-        *reinterpret_cast<uint32_t*>(d + 8) = movm_t(n1) ^ 0x80008000u;
-        *reinterpret_cast<uint32_t*>(d + 8 * BD) = movm_t(n2) ^ 0x80008000u;
-        *reinterpret_cast<uint32_t*>(d + 8 * BD + 8) = movm_t(n3) ^ 0x80008000u;
+        *reinterpret_cast<uint32_t*>(d) = movm_t(res.n[0]) ^ 0x80008000u;
+        *reinterpret_cast<uint32_t*>(d + 8) = movm_t(res.n[1]) ^ 0x80008000u;
+        *reinterpret_cast<uint32_t*>(d + 8 * BD) = movm_t(res.n[2]) ^ 0x80008000u;
+        *reinterpret_cast<uint32_t*>(d + 8 * BD + 8) = movm_t(res.n[3]) ^ 0x80008000u;
       };
-      if (chunks == BR / BC) {
+      // a rate too small to divide by anywhere in the stage (absent tokens' rates are zero and
+      // are never divided by: their chunks are not processed)
+      bool slow = false;
 #pragma unroll
-        for (int c = BR / BC - 1; c >= 0; --c) chunk(c);
+      for (int x = 0; x < 4; ++x)
+        slow |= 4 * lane + x < chunks * BC && fabsf(ldsf(sEta + 4 * (4 * lane + x))) < kTinyRate;
+      slow = __any_sync(0xffffffffu, slow);
+      if (chunks == BR / BC && !slow) {
+        // software pipeline: chunk c's products, then chunk c-1's fragments, then chunk c's
+        // stores
+        Ops o[2];
+        load(o[1], BR / BC - 1);
+#pragma unroll
+        for (int c = BR / BC - 1; c >= 0; --c) {
+          Res res;
+          compute(o[c & 1], c, res, std::false_type{});
+          if (c >= 1) load(o[(c - 1) & 1], c - 1);
+          store(res, c);
+        }
       } else {
 #pragma unroll 1
-        for (int c = chunks - 1; c >= 0; --c) chunk(c);
+        for (int c = chunks - 1; c >= 0; --c) {
+          Ops o;
+          load(o, c);
+          Res res;
+          if (slow)
+            compute(o, c, res, std::true_type{});
+          else
+            compute(o, c, res, std::false_type{});
+          store(res, c);
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -640,7 +727,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 size_t dual_bwd_stage_workspace_bytes(int B, int H, int T) {
   const size_t bh = (size_t)B * H;
-  return bh * T * BD * 2 + bh * ((T + BR - 1) / BR) * BD * BD * 2;
+  return 2 * bh * T * BD * 2 + bh * ((T + BR - 1) / BR) * BD * BD * 2;   // -E, G, W_s
 }
 
 int launch_dual_bwd_stage(const AssocBwdArgs& a, const LaunchCtx& ctx) {
@@ -653,12 +740,13 @@ int launch_dual_bwd_stage(const AssocBwdArgs& a, const LaunchCtx& ctx) {
     return kWorkspace;
   }
   const int BH = a.B * a.H, T = a.T, nst = (T + BR - 1) / BR;
-  uint16_t* G = static_cast<uint16_t*>(a.ws);
+  uint16_t* NE = static_cast<uint16_t*>(a.ws);
+  uint16_t* G = NE + (size_t)BH * T * BD;
   uint16_t* Ws = G + (size_t)BH * T * BD;
   // the forward's residuals and stage-start states: the stage kernel's state-only chain
   StateArgs f{a.K, a.K, a.V, a.eta, a.eta_scalar, a.S0, nullptr, nullptr, a.B, a.H, a.T, a.d,
               BC, 1, nullptr, 0};
-  int st = launch_dual_tc_stage_checkpoints(f, Ws, G, ctx);
+  int st = launch_dual_tc_stage_checkpoints(f, Ws, G, NE, ctx);
   if (st != kOk) return st;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -668,11 +756,11 @@ int launch_dual_bwd_stage(const AssocBwdArgs& a, const LaunchCtx& ctx) {
   const uint64_t wdims[3] = {(uint64_t)BD, (uint64_t)BD, (uint64_t)BH * nst};
   const uint64_t wstrides[2] = {(uint64_t)BD * 2, (uint64_t)BD * BD * 2};
   const uint32_t wbox[3] = {(uint32_t)BD, (uint32_t)BD, 1};
-  CUtensorMap tq, tk, tdo, tg, tw, tdq, tdk;
+  CUtensorMap tq, tk, tdo, tne, tw, tdq, tdk;
   if (!make_tmap_3d(&tq, a.Q, bf, dims, strides, box, sw, ctx.msg) ||
       !make_tmap_3d(&tk, a.K, bf, dims, strides, box, sw, ctx.msg) ||
       !make_tmap_3d(&tdo, a.dO, bf, dims, strides, box, sw, ctx.msg) ||
-      !make_tmap_3d(&tg, G, bf, dims, strides, box, sw, ctx.msg) ||
+      !make_tmap_3d(&tne, NE, bf, dims, strides, box, sw, ctx.msg) ||
       !make_tmap_3d(&tw, Ws, bf, wdims, wstrides, wbox, sw, ctx.msg) ||
       !make_tmap_3d(&tdq, a.dQ, bf, dims, strides, box, sw, ctx.msg) ||
       !make_tmap_3d(&tdk, a.dK, bf, dims, strides, box, sw, ctx.msg))
@@ -684,9 +772,9 @@ int launch_dual_bwd_stage(const AssocBwdArgs& a, const LaunchCtx& ctx) {
     return kCuda;
   }
   const int limit = tuning(kTuneWaitLimitNs);
-  DbtParams p{a.eta, a.eta_scalar, a.dS_out, a.dS0, a.deta, static_cast<uint16_t*>(a.dV), T,
+  DbtParams p{a.eta, a.eta_scalar, a.dS_out, G, a.dS0, a.deta, static_cast<uint16_t*>(a.dV), T,
               ctx.err, limit > 0 ? (uint64_t)limit : 4000000000ull};
-  dual_bwd_tc_kernel<<<BH, THREADS, SMEM, ctx.stream>>>(tq, tk, tdo, tg, tw, tdq, tdk, p);
+  dual_bwd_tc_kernel<<<BH, THREADS, SMEM, ctx.stream>>>(tq, tk, tdo, tne, tw, tdq, tdk, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     *ctx.msg = std::string("dual bwd (stage form) launch: ") + cudaGetErrorString(e);

@@ -110,9 +110,10 @@ __device__ __forceinline__ uint32_t swz_rows(uint32_t row, uint32_t colbyte) {
 // CK (with SO, 16-column chains, C = 16), the dual-form backward's inputs:
 //   1: every chunk's starting state leaves as a bf16 d x d checkpoint through tmC: each chain
 //      warp stages its 16 columns with stmatrix.trans and TMA-stores them;
-//   2: every stage's starting state W_s leaves the same way (one per 128 tokens), and the
-//      residuals G = K W_c - V of every token leave through tmO as bf16 [T][d] rows (each chain
-//      warp collects its 16 columns of the stage in a [128][16] tile, one TMA store per stage).
+//   2: every stage's starting state W_s leaves the same way (one per 128 tokens), and of every
+//      token the residual G = K W_c - V through tmO and -E = -diag(eta) G through tmQ, as bf16
+//      [T][d] rows (each chain warp collects its 16 columns of the stage in two [128][16] tiles,
+//      stored once per stage; tmQ and the ring's Q tiles are unused by the state-only chain).
 template <int NC, int CM, int WC, bool SO, int CK = 0>
 __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
     dual_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -571,7 +572,8 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
         if (lane == 0) {
           tma_store_3d(&tmC, wtile, colg, 0, stream * nst + j);
           bulk_commit();
-          // pending: G of stage j-2 (its tile is rewritten below), W_s of j-1, G of j-1, W_s of j
+          // pending: G, -E of stage j-2 (their tiles are rewritten below), W_s of j-1, G, -E of
+          // j-1, W_s of j
           bulk_wait_read<3>();
         }
         __syncwarp();
@@ -666,6 +668,11 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
         const uint32_t n1 = pack_bf16(E[0][2], E[0][3]) ^ 0x80008000u;
         const uint32_t n2 = pack_bf16(E[1][0], E[1][1]) ^ 0x80008000u;
         const uint32_t n3 = pack_bf16(E[1][2], E[1][3]) ^ 0x80008000u;
+        if constexpr (CK == 2) {   // -E rows of chunk c, into the stage's second tile
+          stsm_x4_t(sbase + (j & 1) * STAGE_BYTES + warp * 4096 +
+                        (16 * c + (lane & 7) + 8 * (lane >> 4)) * 32 + ((lane >> 3) & 1) * 16,
+                    n0, n1, n2, n3);
+        }
 #pragma unroll
         for (int jp = 0; jp < TKS; ++jp) {
           mma16816(wc[2 * jp], n0, n1, n2, n3, o.kt[jp][0], o.kt[jp][1]);
@@ -770,9 +777,10 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
       if (lane == 0) {
         if (!SO) mbar_arrive(eready + 8 * b);
         mbar_arrive(empty + 8 * s);   // K, V and the rates of the stage are consumed
-        if constexpr (CK == 2) {      // the stage's G rows of this warp's 16 columns
+        if constexpr (CK == 2) {      // the stage's G and -E rows of this warp's 16 columns
           tma_store_3d(&tmO, sbase + Cfg::E_OFF + warp * 8192 + (j & 1) * 4096, colg, j * TR,
                        stream);
+          tma_store_3d(&tmQ, sbase + (j & 1) * STAGE_BYTES + warp * 4096, colg, j * TR, stream);
           bulk_commit();
         }
       }
@@ -799,7 +807,7 @@ __global__ void __launch_bounds__(TcCfg<NC, WC>::THREADS, 1)
 
 template <int NC, int CM, int WC, bool SO, int CK = 0>
 int launch_tc(const StateArgs& a, const LaunchCtx& ctx, uint16_t* ckpt = nullptr,
-              uint16_t* gbuf = nullptr) {
+              uint16_t* gbuf = nullptr, uint16_t* nebuf = nullptr) {
   using Cfg = TcCfg<NC, WC>;
   const int BH = a.B * a.H;
   CUtensorMap tq, tk, tv, to;
@@ -816,9 +824,10 @@ int launch_tc(const StateArgs& a, const LaunchCtx& ctx, uint16_t* ckpt = nullptr
       !make_tmap_3d(&tv, a.V, bf, dims, strides, box_in, CU_TENSOR_MAP_SWIZZLE_128B, ctx.msg) ||
       !make_tmap_3d(&to, SO ? a.K : a.O, bf, dims, strides, box_out, osw, ctx.msg))
     return kCuda;
-  if (CK == 2) {   // the residual rows G, 16-column boxes of a stage (tmO is unused otherwise)
+  if (CK == 2) {   // the rows of G and -E, 16-column boxes of a stage (tmO, tmQ unused)
     const uint32_t gbox[3] = {16, (uint32_t)TR, 1};
-    if (!make_tmap_3d(&to, gbuf, bf, dims, strides, gbox, CU_TENSOR_MAP_SWIZZLE_NONE, ctx.msg))
+    if (!make_tmap_3d(&to, gbuf, bf, dims, strides, gbox, CU_TENSOR_MAP_SWIZZLE_NONE, ctx.msg) ||
+        !make_tmap_3d(&tq, nebuf, bf, dims, strides, gbox, CU_TENSOR_MAP_SWIZZLE_NONE, ctx.msg))
       return kCuda;
   }
   CUtensorMap tc = tk;   // checkpoint map (CK only)
@@ -892,14 +901,14 @@ int launch_dual_tc_checkpoints(const StateArgs& a, uint16_t* ckpt, const LaunchC
 }
 
 int launch_dual_tc_stage_checkpoints(const StateArgs& a, uint16_t* Ws, uint16_t* G,
-                                     const LaunchCtx& ctx) {
+                                     uint16_t* NE, const LaunchCtx& ctx) {
   if (!(dual_tc_supported(a.d, a.C, a.dt) && a.C == TC)) {
     *ctx.msg = "dual_tc stage checkpoints: bf16, d = 64, C = 16 only";
     return kUnsupported;
   }
   StateArgs s = a;
   s.O = nullptr;
-  return launch_tc<4, 1, 16, true, 2>(s, ctx, Ws, G);
+  return launch_tc<4, 1, 16, true, 2>(s, ctx, Ws, G, NE);
 }
 
 int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx) {

@@ -122,9 +122,9 @@ int launch_dual_tc(const StateArgs& a, int split, const LaunchCtx& ctx);
 // d = 64, C = 16; S0 = W0, S_out may be null).
 int launch_dual_tc_checkpoints(const StateArgs& a, uint16_t* ckpt, const LaunchCtx& ctx);
 // The same chain writing what the stage-form backward reads: the state at the start of every
-// 128-token stage ([streams, ceil(T / 128), d, d] bf16) and every token's residual
-// G = K W_c - V ([streams, T, d] bf16).
-int launch_dual_tc_stage_checkpoints(const StateArgs& a, uint16_t* Ws, uint16_t* G,
+// 128-token stage ([streams, ceil(T / 128), d, d] bf16) and of every token the residual
+// G = K W_c - V and -E = -diag(eta) G ([streams, T, d] bf16 each).
+int launch_dual_tc_stage_checkpoints(const StateArgs& a, uint16_t* Ws, uint16_t* G, uint16_t* NE,
                                      const LaunchCtx& ctx);
 // True when launch_dual_mma takes O = nullptr for this shape (the stage kernel's state-only
 // form: the final state and no outputs).
