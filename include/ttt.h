@@ -273,10 +273,15 @@ int ttt_assoc_scan_bwd(const void* Q, const void* K, const void* V, const float*
  *  overlap the inputs or each other.
  *  Supported: bf16, C == 16, d in {32, 64, 128}, T % C == 0 (C changes the result: it is the
  *  mini-batch size of the forward).
- *  Workspace: ttt_linear_dual_bwd_workspace_size() bytes (one bf16 d x d state per chunk:
- *  B*H*(T/16)*d*d*2). A forward sweep recomputes the chunk-start states into the workspace
- *  (d = 64: the forward stage kernel's state-only chain, a second launch; d = 32 and 128: inside
- *  the backward kernel), a reverse sweep forms the gradients (see dual_bwd.cu).
+ *  Workspace: ttt_linear_dual_bwd_workspace_size() bytes (d = 32, 128: one bf16 d x d state per
+ *  chunk, B*H*(T/16)*d*d*2; d = 64: the larger of that and the stage form's G and -diag(eta) G
+ *  rows plus one bf16 d x d state per 128 tokens, B*H*(4*T*d + ceil(T/128)*2*d*d)). A forward
+ *  recompute fills the workspace, then the reverse pass forms the gradients. d = 64 (stage form,
+ *  dual_bwd_tc.cu): the forward stage kernel's state-only chain writes G, -diag(eta) G and the
+ *  stage-start states; the reverse pass keeps the state gradient's chain on warp MMAs and forms
+ *  every product that needs the forward states per 128-token stage on tcgen05. d = 32, 128
+ *  (dual_bwd.cu): one kernel, a forward sweep of chunk-start states then a reverse sweep of the
+ *  chunk adjoint. The tuning key "dual_bwd_form" selects the other d = 64 forms.
  * ------------------------------------------------------------------------------------------ */
 size_t ttt_linear_dual_bwd_workspace_size(int B, int H, int T, int d, int C, int dt);
 int ttt_linear_dual_bwd(const void* Q, const void* K, const void* V, const float* eta,
