@@ -64,6 +64,29 @@ def test_scalar_eta_and_zero_states(cuda_lib):
     check(x, run(x))
 
 
+@pytest.mark.parametrize("T", [272, 1024])
+def test_zero_and_tiny_rates(cuda_lib, T):
+    """Per-token rates of exactly zero and of 1e-25 mixed with ordinary ones, in the same 16-token
+    chunk, in the same 128-token stage and alone in whole stages; then every rate zero (the
+    states never move, dV = 0, deta = -G . (A'^T dO + K X) still nonzero). The stage form takes
+    deta from G itself wherever a rate is too small to divide by."""
+    x = make(1, 2, T, 64, seed=T + 71)
+    eta = x["eta"].clone()
+    eta[0, 0, 3] = 0.0
+    eta[0, 0, 5] = 1e-25
+    eta[0, 0, 140:150] = 0.0
+    eta[0, 1, 128:256] = 0.0
+    eta[0, 1, 17] = 1e-25
+    x["eta"] = eta
+    check(x, run(x))
+    x["eta"] = torch.zeros_like(eta)
+    got = run(x)
+    check(x, got)
+    assert float(got[2].float().abs().max()) == 0.0   # dV = -dG = 0
+    assert float(got[3].abs().max()) > 0.0            # deta does not vanish with the rates
+    assert ttt.read_device_error() == 0
+
+
 def test_deterministic_and_caller_buffers(cuda_lib):
     x = make(1, 2, 256, 64, seed=8)
     a = run(x)
