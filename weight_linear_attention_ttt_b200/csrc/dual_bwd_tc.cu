@@ -45,8 +45,8 @@
 //     stores dG^T (the MN-major A operand of the stage's products), dV and, at each stage
 //     start, bf16(X_e^T). The next chunk's fragments are loaded before this chunk's stores.
 // TMEM columns: S1 [0, 128), S2 [128, 256), dQ [256, 320), dK [320, 384).
-// Precision: X and every accumulation fp32; W_s, G, X_e, dG and the masked scores are bf16 tensor
-// operands (relative error ~2^-9 per operand).
+// Precision: X and every accumulation fp32; W_s, -E, X_e, dG and the masked scores are bf16
+// tensor operands (relative error ~2^-9 per operand); deta uses the bf16 -E (or G) rows.
 #include <algorithm>
 #include <string>
 #include <type_traits>
@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = false;
         break;
       }
-      // bf16(X_e^T): the B operand (MN-major) of the stage's G X_e^T
+      // bf16(X_e^T): the B operand (MN-major) of the stage's (-E) X_e^T
 #pragma unroll
       for (int ks = 0; ks < BKS; ++ks)
         stsm_x4(sbase + XE_OFF + swz128(srow, 2 * (16 * ks + scol)),
